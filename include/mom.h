@@ -1,0 +1,246 @@
+/*
+ * mom.h -- C ABI of the B200 (sm_100a) Mixture-of-Memories layer library.
+ *
+ * One MoM layer forward: a linear router picks each token's top-k memories;
+ * tokens are reordered into contiguous per-memory segments; every memory
+ * (and an always-on shared memory) projects its own keys/values and runs a
+ * Gated DeltaNet recurrence over only the tokens routed to it; the outputs
+ * are summed with the router weights.  A constant-cost recurrent decode
+ * step runs the same layer one token per sequence.
+ *
+ * Sources (page title, section):
+ *   "MoM: Linear Sequence Modeling with Mixture-of-Memories" (paper card),
+ *       Summary -- the layer as a whole;
+ *   "MoM: Mixture-of-Memories Fixes Linear Attention Recall" (explainer),
+ *       "Router mechanics, step by step" and "Solving scatter-gather without
+ *       new kernels";
+ *   the authors' MoM blog post, sections "Mixture-of-Memories" and
+ *       "硬件高效實現" (hardware-efficient implementation), and its
+ *       experiments section, which fixes Gated DeltaNet as the memory rule.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless documented otherwise; every array
+ *     is dense row-major and 16-byte aligned.
+ *   - The caller owns every buffer.  The library never allocates or frees;
+ *     scratch space is the caller's `ws` of at least the size that the
+ *     matching mom_*_workspace_size() returns.  The first MOM_WS_HEADER_BYTES
+ *     of any workspace hold a device-side error record (see mom_get_error);
+ *     zero the workspace once before its first use.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise the host, except mom_get_error.
+ *   - Projection weights use the [out_features, in_features] layout
+ *     (y = x W^T).  Activations are [rows, H, d]; recurrent states are
+ *     [.., H, d_v, d_k] float32 so that o = S q.
+ *   - `dt` selects the element type of activations and weights (MOM_F32 or
+ *     MOM_BF16).  Router gates, logits, beta, log alpha and states are
+ *     always float32.
+ *   - Arguments are validated before any launch; a failed validation
+ *     launches nothing, writes nothing and returns MOM_ERR_ARG or
+ *     MOM_ERR_UNSUPPORTED.  A failed launch returns MOM_ERR_CUDA.
+ *   - Data-dependent violations seen on the device (a memory index >= M, a
+ *     row index out of range, inconsistent segment bounds) are skipped
+ *     without any out-of-bounds access and recorded in the workspace's error
+ *     record; no kernel traps or aborts.
+ */
+#ifndef MOM_H
+#define MOM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int mom_status;
+#define MOM_OK               0
+#define MOM_ERR_ARG          1  /* bad pointer, size or alignment */
+#define MOM_ERR_UNSUPPORTED  2  /* valid but not implemented (e.g. d not in {64,128,256}) */
+#define MOM_ERR_CUDA         3  /* a launch or CUDA runtime call failed */
+#define MOM_ERR_DEVICE       4  /* mom_get_error: a kernel recorded a data violation */
+
+typedef int mom_dtype;
+#define MOM_F32   0
+#define MOM_BF16  1
+
+/* Device error record codes (mom_get_error's *code). */
+#define MOM_DEVERR_NONE       0
+#define MOM_DEVERR_MEM_INDEX  1  /* topk_idx entry outside [0, n_mem) or repeated in a row */
+#define MOM_DEVERR_ROW_INDEX  2  /* a row / token index outside its array */
+#define MOM_DEVERR_SEGMENT    3  /* segment bounds decreasing or beyond n_rows */
+
+#define MOM_WS_HEADER_BYTES 256
+
+/* Largest supported sizes. */
+#define MOM_MAX_MEM   32   /* routed memories M */
+#define MOM_MAX_HEADS 64
+
+/* Human-readable name of a status code (static string). */
+const char* mom_status_string(mom_status s);
+
+/* Reads the device error record of `ws` (synchronises `stream`).  Writes the
+ * first recorded code (MOM_DEVERR_*) and its offending index to *code and
+ * *info (either may be NULL).  Returns MOM_OK when no violation was
+ * recorded, MOM_ERR_DEVICE when one was, MOM_ERR_CUDA on a runtime error. */
+mom_status mom_get_error(const void* ws, int32_t* code, int32_t* info, void* stream);
+
+/* Clears the device error record of `ws` (asynchronous on `stream`). */
+mom_status mom_clear_error(void* ws, void* stream);
+
+/* Diagnostic: the number of kernels this library has launched in this
+ * process (all devices, all streams).  Host-side counter, thread-safe. */
+uint64_t mom_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * mom_router_topk -- the router: one matmul, one softmax, one top-k, one
+ * renormalisation (explainer, "Router mechanics, step by step"; blog post,
+ * "Mixture-of-Memories").
+ *
+ *   logits[t, m] = x[t, :] . w_r[m, :] + b_r[m]        (float32 accumulate)
+ *   topk_idx[t, :] = the top_k memories by logit, in descending order; equal
+ *                    logits go to the lower memory index
+ *   topk_gate[t, j] = softmax(logits[t])[idx_j] / sum_j' softmax(logits[t])[idx_j']
+ *
+ * x [n_tok, d_model] (dt); w_r [n_mem, d_model] (dt); b_r [n_mem] float32 or
+ * NULL (zero bias).  Outputs: topk_idx [n_tok, top_k] int32, topk_gate
+ * [n_tok, top_k] float32, logits [n_tok, n_mem] float32 or NULL.
+ * Requires 1 <= top_k <= n_mem <= MOM_MAX_MEM, d_model % 8 == 0,
+ * n_tok >= 0 (n_tok == 0 launches nothing).
+ * ---------------------------------------------------------------------- */
+mom_status mom_router_topk(const void* x, const void* w_r, const float* b_r, mom_dtype dt,
+                           int64_t n_tok, int d_model, int n_mem, int top_k,
+                           int32_t* topk_idx, float* topk_gate, float* logits, void* stream);
+
+/* ------------------------------------------------------------------------
+ * mom_permute -- reorder the routed (token, slot) pairs into contiguous
+ * per-memory segments (explainer, "Solving scatter-gather without new
+ * kernels"): a stable counting sort by memory.
+ *
+ * Pair r = t*top_k + j routes token t to memory topk_idx[t, j].  Outputs:
+ *   perm_token [n_tok*top_k]  token of each reordered row;
+ *   row_of     [n_tok*top_k]  reordered row of pair t*top_k + j;
+ *   mem_offset [n_mem+1]      first row of each memory (mem_offset[n_mem] =
+ *                             number of valid pairs);
+ *   seg_cu     [n_mem*n_seq+1] segment bounds, one segment per (memory,
+ *                             sequence), memory-major; rows inside a segment
+ *                             keep token order.  Empty segments are allowed.
+ * cu_seqlens [n_seq+1] int32 (device) gives the sequences of the packed
+ * batch (cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seq] = n_tok).
+ * A pair whose memory index is out of range is recorded
+ * (MOM_DEVERR_MEM_INDEX) and dropped.  ws: mom_permute_workspace_size().
+ * ---------------------------------------------------------------------- */
+size_t mom_permute_workspace_size(int64_t n_tok, int top_k, int n_mem, int n_seq);
+mom_status mom_permute(const int32_t* topk_idx, int64_t n_tok, int top_k, int n_mem,
+                       const int32_t* cu_seqlens, int n_seq,
+                       int32_t* perm_token, int32_t* row_of, int32_t* mem_offset, int32_t* seg_cu,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * mom_kv_proj_grouped -- every projection of the layer (paper card,
+ * Summary: a shared query, and key/value projections of each memory's own):
+ *
+ *   q     = l2norm_h(x W_q^T)              k_sh = l2norm_h(x W_k_sh^T)
+ *   v_sh  = x W_v_sh^T                     beta = sigmoid(x W_beta^T)
+ *   log_alpha = -exp(A) * softplus(x W_a^T + b_a)
+ *   for each memory m and reordered row r in [mem_offset[m], mem_offset[m+1]):
+ *     k_p[r] = l2norm_h(x[perm_token[r]] W_k^m^T),  v_p[r] = x[perm_token[r]] W_v^m^T
+ *
+ * l2norm_h(y) = y / sqrt(|y|^2 + 1e-6) per head of d elements.
+ * x [n_tok, d_model]; w_shared [3*H*d, d_model] = rows W_q | W_k_sh | W_v_sh;
+ * w_gate [2*H, d_model] = rows W_beta | W_a; A, b_a [H] float32;
+ * w_kv [n_mem, 2*H*d, d_model] = per memory rows W_k^m | W_v^m.
+ * Outputs q, k_sh, v_sh [n_tok, H, d] (dt); beta, log_alpha [n_tok, H]
+ * float32; k_p, v_p [n_tok*top_k, H, d] (dt).  Rows of k_p / v_p past
+ * mem_offset[n_mem] are not written.  Requires d in {64, 128, 256},
+ * d_model % 64 == 0.  ws: mom_kv_proj_workspace_size().
+ * ---------------------------------------------------------------------- */
+size_t mom_kv_proj_workspace_size(int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k);
+mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
+                               const void* w_shared, const void* w_gate, const float* A, const float* b_a,
+                               const void* w_kv, mom_dtype dt,
+                               int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k,
+                               void* q, void* k_sh, void* v_sh, float* beta, float* log_alpha,
+                               void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * mom_gdn_chunk_fwd -- the Gated DeltaNet recurrence of one memory over
+ * each segment (blog post, experiments section: every memory uses Gated
+ * DeltaNet's gate and update rule; "Mixture-of-Memories": each memory runs
+ * over only the tokens routed to it):
+ *
+ *   S_0 = h0[seg] (or 0);  for each row r of the segment, in order:
+ *     S_r = alpha_r S_{r-1} (I - beta_r k_r k_r^T) + beta_r v_r k_r^T,
+ *     o_r = S_r (scale * q_r),         alpha_r = exp(log_alpha_r)
+ *   h_final[seg] = S_last.
+ *
+ * k, v, o [n_rows, H, d]; q [n_q_rows, H, d]; beta, log_alpha [n_q_rows, H]
+ * float32.  When qidx (int32 [n_rows]) is non-NULL, row r reads q, beta and
+ * log_alpha at row qidx[r] (the routed memories read the shared query of
+ * the token behind each reordered row); otherwise at row r.  seg_cu
+ * [n_seg+1] int32 row bounds (seg_cu[0] = 0, non-decreasing, <= n_rows).
+ * h0, h_final [n_seg, H, d, d] float32 or NULL.  An empty segment writes
+ * h_final = h0 (or zeros).  In MOM_BF16 mode q, k, v, o are bf16 while the
+ * state and every accumulation stay float32; in MOM_F32 mode everything is
+ * float32.  Requires d in {64, 128, 256}.  ws: mom_gdn_workspace_size().
+ * ---------------------------------------------------------------------- */
+size_t mom_gdn_workspace_size(int64_t n_rows, int n_seg, int H, int d, mom_dtype dt);
+mom_status mom_gdn_chunk_fwd(const void* q, const int32_t* qidx, const void* k, const void* v,
+                             const float* beta, const float* log_alpha,
+                             const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                             int H, int d, float scale, mom_dtype dt,
+                             const float* h0, float* h_final, void* o,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * mom_combine_unpermute -- the combine (paper card, Summary: outputs are
+ * combined using the router weights; blog post, "硬件高效實現": summing the
+ * weighted per-memory outputs equals reading out the mixed memory):
+ *
+ *   out[t] = o_sh[t] + sum_j topk_gate[t, j] * o_p[row_of[t*top_k + j]]
+ *
+ * o_sh, out [n_tok, H, d] (dt); o_p [n_tok*top_k, H, d] (dt); row_of
+ * [n_tok*top_k] int32; topk_gate [n_tok, top_k] float32.  float32
+ * arithmetic.  An out-of-range row_of entry is recorded
+ * (MOM_DEVERR_ROW_INDEX) and contributes nothing.
+ * ws: at least MOM_WS_HEADER_BYTES.
+ * ---------------------------------------------------------------------- */
+mom_status mom_combine_unpermute(const void* o_sh, const void* o_p, const int32_t* row_of,
+                                 const float* topk_gate, int64_t n_tok, int top_k, int H, int d,
+                                 mom_dtype dt, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * mom_decode_step -- one recurrent decode step, one new token per
+ * sequence, constant cost per token (blog post, introduction and
+ * "推理效率" (inference efficiency); paper card, Summary: constant-memory
+ * inference).  For every sequence b: route x[b]; project q, beta, alpha,
+ * the shared memory's k/v and the k/v of the top_k chosen memories; update
+ * those top_k + 1 states in place with the rule of mom_gdn_chunk_fwd; and
+ * write out[b] = o_sh + sum_j gate_j o_j.  The other memories' states are
+ * untouched.
+ *
+ * x [B, d_model] (dt); weights as in mom_router_topk / mom_kv_proj_grouped;
+ * state [B, n_mem+1, H, d, d] float32, slot n_mem being the shared memory,
+ * updated in place; out [B, H, d] (dt); topk_idx [B, top_k] int32 or NULL
+ * (receives the routing).  `w` is a HOST pointer to a struct of device
+ * pointers; it is read during the call only.  ws: mom_decode_workspace_size().
+ * ---------------------------------------------------------------------- */
+typedef struct mom_weights {
+    const void*  w_r;       /* [n_mem, d_model] */
+    const float* b_r;       /* [n_mem] or NULL */
+    const void*  w_shared;  /* [3*H*d, d_model] */
+    const void*  w_gate;    /* [2*H, d_model] */
+    const float* A;         /* [H] */
+    const float* b_a;       /* [H] */
+    const void*  w_kv;      /* [n_mem, 2*H*d, d_model] */
+} mom_weights;
+
+size_t mom_decode_workspace_size(int B, int d_model, int H, int d, int n_mem, int top_k);
+mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_model, int H, int d,
+                           int n_mem, int top_k, float scale, mom_dtype dt,
+                           float* state, void* out, int32_t* topk_idx,
+                           void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOM_H */

@@ -1,0 +1,177 @@
+"""Thin ctypes binding of the C ABI in ``include/mom.h``.
+
+Argument marshalling only: every function here passes device pointers and
+sizes through to the CUDA library, which does all the work.  Tensors are
+torch tensors on the current CUDA device; ``stream`` defaults to torch's
+current stream.  If the library is missing this module raises at import --
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int, c_int32, c_int64, c_size_t, c_void_p
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmom_b200.so")
+
+MOM_OK, MOM_ERR_ARG, MOM_ERR_UNSUPPORTED, MOM_ERR_CUDA, MOM_ERR_DEVICE = 0, 1, 2, 3, 4
+MOM_F32, MOM_BF16 = 0, 1
+MOM_DEVERR_NONE, MOM_DEVERR_MEM_INDEX, MOM_DEVERR_ROW_INDEX, MOM_DEVERR_SEGMENT = 0, 1, 2, 3
+MOM_WS_HEADER_BYTES = 256
+
+# every function the header declares, with (restype, argtypes)
+_VP, _I, _I64, _F, _SZ = c_void_p, c_int, c_int64, c_float, c_size_t
+SIGNATURES = {
+    "mom_status_string": (c_char_p, [_I]),
+    "mom_get_error": (_I, [_VP, POINTER(c_int32), POINTER(c_int32), _VP]),
+    "mom_clear_error": (_I, [_VP, _VP]),
+    "mom_launch_count": (ctypes.c_uint64, []),
+    "mom_router_topk": (_I, [_VP, _VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP, _VP, _VP]),
+    "mom_permute_workspace_size": (_SZ, [_I64, _I, _I, _I]),
+    "mom_permute": (_I, [_VP, _I64, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_kv_proj_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I]),
+    "mom_kv_proj_grouped": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
+                                 _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_gdn_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
+    "mom_gdn_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I,
+                               _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_combine_unpermute": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
+    "mom_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "mom_decode_step": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
+}
+
+
+class MomWeights(ctypes.Structure):
+    """Mirror of ``struct mom_weights`` (device pointers)."""
+    _fields_ = [("w_r", c_void_p), ("b_r", c_void_p), ("w_shared", c_void_p), ("w_gate", c_void_p),
+                ("A", c_void_p), ("b_a", c_void_p), ("w_kv", c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("MoM CUDA library not built (%s missing); run "
+                           "`python -m mixture_memories_layer_b200.build`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+class MomError(RuntimeError):
+    pass
+
+
+def _check(status: int, what: str):
+    if status != MOM_OK:
+        raise MomError("%s failed: %s (%d)" % (what, lib.mom_status_string(status).decode(), status))
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return MOM_BF16
+    if t == torch.float32:
+        return MOM_F32
+    raise ValueError("unsupported dtype %s" % t)
+
+
+# ------------------------------------------------------------------ helpers
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zeroed workspace (the error record starts clear)."""
+    return torch.zeros(max(int(nbytes), MOM_WS_HEADER_BYTES), dtype=torch.uint8, device=device or "cuda")
+
+
+def mom_get_error(ws: torch.Tensor, stream=None):
+    code, info = c_int32(0), c_int32(0)
+    st = lib.mom_get_error(_p(ws), ctypes.byref(code), ctypes.byref(info), _s(stream))
+    if st not in (MOM_OK, MOM_ERR_DEVICE):
+        _check(st, "mom_get_error")
+    return code.value, info.value
+
+
+def mom_launch_count() -> int:
+    return int(lib.mom_launch_count())
+
+
+def mom_clear_error(ws: torch.Tensor, stream=None):
+    _check(lib.mom_clear_error(_p(ws), _s(stream)), "mom_clear_error")
+
+
+# ------------------------------------------------------- the six entry points
+
+def mom_router_topk(x, w_r, b_r, top_k, topk_idx, topk_gate, logits=None, stream=None):
+    n_tok, d_model = x.shape
+    _check(lib.mom_router_topk(_p(x), _p(w_r), _p(b_r), dtype_code(x.dtype), n_tok, d_model, w_r.shape[0],
+                               top_k, _p(topk_idx), _p(topk_gate), _p(logits), _s(stream)), "mom_router_topk")
+
+
+def mom_permute_workspace_size(n_tok, top_k, n_mem, n_seq):
+    return lib.mom_permute_workspace_size(n_tok, top_k, n_mem, n_seq)
+
+
+def mom_permute(topk_idx, n_mem, cu_seqlens, perm_token, row_of, mem_offset, seg_cu, ws, stream=None):
+    n_tok, top_k = topk_idx.shape
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib.mom_permute(_p(topk_idx), n_tok, top_k, n_mem, _p(cu_seqlens), n_seq, _p(perm_token), _p(row_of),
+                           _p(mem_offset), _p(seg_cu), _p(ws), ws.numel(), _s(stream)), "mom_permute")
+
+
+def mom_kv_proj_workspace_size(n_tok, d_model, H, d, n_mem, top_k):
+    return lib.mom_kv_proj_workspace_size(n_tok, d_model, H, d, n_mem, top_k)
+
+
+def mom_kv_proj_grouped(x, perm_token, mem_offset, w_shared, w_gate, A, b_a, w_kv, H, d, top_k,
+                        q, k_sh, v_sh, beta, log_alpha, k_p, v_p, ws, stream=None):
+    n_tok, d_model = x.shape
+    _check(lib.mom_kv_proj_grouped(_p(x), _p(perm_token), _p(mem_offset), _p(w_shared), _p(w_gate), _p(A), _p(b_a),
+                                   _p(w_kv), dtype_code(x.dtype), n_tok, d_model, H, d, w_kv.shape[0], top_k,
+                                   _p(q), _p(k_sh), _p(v_sh), _p(beta), _p(log_alpha), _p(k_p), _p(v_p),
+                                   _p(ws), ws.numel(), _s(stream)), "mom_kv_proj_grouped")
+
+
+def mom_gdn_workspace_size(n_rows, n_seg, H, d, dt):
+    return lib.mom_gdn_workspace_size(n_rows, n_seg, H, d, dt)
+
+
+def mom_gdn_chunk_fwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream=None):
+    n_rows, H, d = k.shape
+    _check(lib.mom_gdn_chunk_fwd(_p(q), _p(qidx), _p(k), _p(v), _p(beta), _p(log_alpha), _p(seg_cu),
+                                 seg_cu.numel() - 1, n_rows, q.shape[0], H, d, float(scale),
+                                 dtype_code(k.dtype), _p(h0), _p(h_final), _p(o), _p(ws), ws.numel(),
+                                 _s(stream)), "mom_gdn_chunk_fwd")
+
+
+def mom_combine_unpermute(o_sh, o_p, row_of, topk_gate, out, ws, stream=None):
+    n_tok, H, d = o_sh.shape
+    top_k = topk_gate.shape[1]
+    _check(lib.mom_combine_unpermute(_p(o_sh), _p(o_p), _p(row_of), _p(topk_gate), n_tok, top_k, H, d,
+                                     dtype_code(o_sh.dtype), _p(out), _p(ws), ws.numel(), _s(stream)),
+           "mom_combine_unpermute")
+
+
+def mom_decode_workspace_size(B, d_model, H, d, n_mem, top_k):
+    return lib.mom_decode_workspace_size(B, d_model, H, d, n_mem, top_k)
+
+
+def mom_decode_step(x, weights: MomWeights, H, d, n_mem, top_k, scale, state, out, topk_idx, ws, stream=None):
+    B, d_model = x.shape
+    _check(lib.mom_decode_step(_p(x), ctypes.byref(weights), B, d_model, H, d, n_mem, top_k, float(scale),
+                               dtype_code(x.dtype), _p(state), _p(out), _p(topk_idx), _p(ws), ws.numel(),
+                               _s(stream)), "mom_decode_step")

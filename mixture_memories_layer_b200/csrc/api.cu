@@ -1,0 +1,246 @@
+// The C ABI of mom.h: argument validation, workspace carving and dispatch.
+// Nothing here computes; every step of the layer runs in the kernels.
+#include <string.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace mom;
+
+static std::atomic<uint64_t> g_launches{0};
+void mom::count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+namespace {
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline size_t esize(int dt) { return dt == MOM_BF16 ? 2 : 4; }
+inline bool dt_ok(int dt) { return dt == MOM_F32 || dt == MOM_BF16; }
+inline bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
+inline mom_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOM_OK : MOM_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mom_status_string(mom_status s) {
+    switch (s) {
+        case MOM_OK: return "ok";
+        case MOM_ERR_ARG: return "invalid argument";
+        case MOM_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case MOM_ERR_CUDA: return "CUDA runtime or launch error";
+        case MOM_ERR_DEVICE: return "a kernel recorded a data violation";
+    }
+    return "unknown status";
+}
+
+mom_status mom_get_error(const void* ws, int32_t* code, int32_t* info, void* stream) {
+    if (ws == nullptr) return MOM_ERR_ARG;
+    int32_t rec[2] = {0, 0};
+    if (cudaMemcpyAsync(rec, ws, sizeof(rec), cudaMemcpyDeviceToHost, as_stream(stream)) != cudaSuccess)
+        return MOM_ERR_CUDA;
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MOM_ERR_CUDA;
+    if (code) *code = rec[0];
+    if (info) *info = rec[1];
+    return rec[0] == MOM_DEVERR_NONE ? MOM_OK : MOM_ERR_DEVICE;
+}
+
+uint64_t mom_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+mom_status mom_clear_error(void* ws, void* stream) {
+    if (ws == nullptr) return MOM_ERR_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, 8, as_stream(stream)));
+}
+
+// ------------------------------------------------------------------ router
+mom_status mom_router_topk(const void* x, const void* w_r, const float* b_r, mom_dtype dt,
+                           int64_t n_tok, int d_model, int n_mem, int top_k,
+                           int32_t* topk_idx, float* topk_gate, float* logits, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || d_model <= 0 || d_model % 8 != 0) return MOM_ERR_ARG;
+    if (top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    if (!x || !w_r || !topk_idx || !topk_gate || !al16(x) || !al16(w_r)) return MOM_ERR_ARG;
+    return cuda_status(launch_router(x, w_r, b_r, dt, n_tok, d_model, n_mem, top_k, topk_idx, topk_gate,
+                                     logits, as_stream(stream)));
+}
+
+// ----------------------------------------------------------------- permute
+size_t mom_permute_workspace_size(int64_t n_tok, int top_k, int n_mem, int n_seq) {
+    (void)top_k; (void)n_seq;
+    return MOM_WS_HEADER_BYTES + up256(permute_scratch_bytes(n_tok, n_mem > 0 ? n_mem : 1));
+}
+
+mom_status mom_permute(const int32_t* topk_idx, int64_t n_tok, int top_k, int n_mem,
+                       const int32_t* cu_seqlens, int n_seq,
+                       int32_t* perm_token, int32_t* row_of, int32_t* mem_offset, int32_t* seg_cu,
+                       void* ws, size_t ws_bytes, void* stream) {
+    if (n_tok < 0 || top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM || n_seq < 1) return MOM_ERR_ARG;
+    if (n_tok * top_k >= ((int64_t)1 << 31)) return MOM_ERR_UNSUPPORTED;
+    if (!cu_seqlens && n_seq != 1) return MOM_ERR_ARG;
+    if (!mem_offset || !seg_cu || !ws || ws_bytes < mom_permute_workspace_size(n_tok, top_k, n_mem, n_seq))
+        return MOM_ERR_ARG;
+    if (n_tok > 0 && (!topk_idx || !perm_token || !row_of)) return MOM_ERR_ARG;
+    return cuda_status(launch_permute(topk_idx, n_tok, top_k, n_mem, cu_seqlens, n_seq, perm_token, row_of,
+                                      mem_offset, seg_cu, ws, (char*)ws + MOM_WS_HEADER_BYTES,
+                                      as_stream(stream)));
+}
+
+// ------------------------------------------------------------- projections
+size_t mom_kv_proj_workspace_size(int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k) {
+    (void)n_tok; (void)d_model; (void)H; (void)d; (void)n_mem; (void)top_k;
+    return MOM_WS_HEADER_BYTES;
+}
+
+static mom_status run_projections(const ProjArgs& a, const void* w_gate, const float* A, const float* b_a,
+                                  int dt, float* beta, float* log_alpha, cudaStream_t st) {
+    cudaError_t e = launch_gate_proj(a.x, w_gate, A, b_a, dt, a.n_tok, a.D, a.H, beta, log_alpha, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    if (proj_tc_supported(a, dt)) e = launch_proj_tc(a, st);
+    else e = launch_proj_simt(a, dt, st);
+    return cuda_status(e);
+}
+
+mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
+                               const void* w_shared, const void* w_gate, const float* A, const float* b_a,
+                               const void* w_kv, mom_dtype dt,
+                               int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k,
+                               void* q, void* k_sh, void* v_sh, float* beta, float* log_alpha,
+                               void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || d_model <= 0 || d_model % 64 != 0) return MOM_ERR_ARG;
+    if (H < 1 || H > MOM_MAX_HEADS || top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM) return MOM_ERR_ARG;
+    if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (n_tok * top_k >= ((int64_t)1 << 31)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < mom_kv_proj_workspace_size(n_tok, d_model, H, d, n_mem, top_k)) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {x, perm_token, mem_offset, w_shared, w_gate, A, b_a, w_kv, q, k_sh, v_sh, beta,
+                          log_alpha, k_p, v_p};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    ProjArgs a{x, perm_token, mem_offset, w_shared, w_kv, n_tok, d_model, H, d, n_mem, top_k,
+               q, k_sh, v_sh, k_p, v_p, ws};
+    return run_projections(a, w_gate, A, b_a, dt, beta, log_alpha, as_stream(stream));
+}
+
+// --------------------------------------------------------- chunked GDN
+size_t mom_gdn_workspace_size(int64_t n_rows, int n_seg, int H, int d, mom_dtype dt) {
+    size_t extra = (dt == MOM_BF16 && head_dim_ok(d)) ? gdn_tc_ws_bytes(n_rows, n_seg, H, d) : 0;
+    return MOM_WS_HEADER_BYTES + up256(extra);
+}
+
+mom_status mom_gdn_chunk_fwd(const void* q, const int32_t* qidx, const void* k, const void* v,
+                             const float* beta, const float* log_alpha,
+                             const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                             int H, int d, float scale, mom_dtype dt,
+                             const float* h0, float* h_final, void* o,
+                             void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_seg < 0 || n_rows < 0 || n_q_rows < 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < mom_gdn_workspace_size(n_rows, n_seg, H, d, dt)) return MOM_ERR_ARG;
+    if (n_seg == 0) return MOM_OK;
+    if (!seg_cu) return MOM_ERR_ARG;
+    if ((h0 && !al16(h0)) || (h_final && !al16(h_final))) return MOM_ERR_ARG;
+    if (n_rows > 0) {
+        const void* ptrs[] = {q, k, v, beta, log_alpha, o};
+        for (const void* p : ptrs)
+            if (!p || !al16(p)) return MOM_ERR_ARG;
+    }
+    GdnArgs a{q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale,
+              h0, h_final, o, ws, ws_bytes};
+    cudaStream_t st = as_stream(stream);
+    if (gdn_tc_supported(a, dt)) return cuda_status(launch_gdn_tc(a, st));
+    return cuda_status(launch_gdn_recurrent(a, dt, st));
+}
+
+// ----------------------------------------------------------------- combine
+mom_status mom_combine_unpermute(const void* o_sh, const void* o_p, const int32_t* row_of,
+                                 const float* topk_gate, int64_t n_tok, int top_k, int H, int d,
+                                 mom_dtype dt, void* out, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || top_k < 1 || H < 1 || d < 8 || (H * d) % 8 != 0) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {o_sh, o_p, row_of, topk_gate, out};
+    for (const void* p : ptrs)
+        if (!p) return MOM_ERR_ARG;
+    if (!al16(o_sh) || !al16(o_p) || !al16(out)) return MOM_ERR_ARG;
+    return cuda_status(launch_combine(o_sh, o_p, row_of, topk_gate, n_tok, top_k, H, d, dt, out, ws,
+                                      as_stream(stream)));
+}
+
+// ------------------------------------------------------------------ decode
+namespace {
+struct DecodeLayout {
+    size_t idx, gate, perm, row_of, mem_off, seg_cu, q, k_sh, v_sh, beta, la, k_p, v_p, perm_scratch, total;
+};
+DecodeLayout decode_layout(int B, int H, int d, int M, int K, int dt) {
+    DecodeLayout L;
+    size_t off = MOM_WS_HEADER_BYTES;
+    auto take = [&](size_t bytes) { size_t o = off; off += up256(bytes); return o; };
+    const size_t BK = (size_t)B * K, HD = (size_t)H * d;
+    L.idx = take(BK * 4);
+    L.gate = take(BK * 4);
+    L.perm = take(BK * 4);
+    L.row_of = take(BK * 4);
+    L.mem_off = take((M + 1) * 4);
+    L.seg_cu = take((M + 1) * 4);
+    L.q = take((size_t)B * HD * esize(dt));
+    L.k_sh = take((size_t)B * HD * esize(dt));
+    L.v_sh = take((size_t)B * HD * esize(dt));
+    L.beta = take((size_t)B * H * 4);
+    L.la = take((size_t)B * H * 4);
+    L.k_p = take(BK * HD * esize(dt));
+    L.v_p = take(BK * HD * esize(dt));
+    L.perm_scratch = take(permute_scratch_bytes(B, M));
+    L.total = off;
+    return L;
+}
+}  // namespace
+
+size_t mom_decode_workspace_size(int B, int d_model, int H, int d, int n_mem, int top_k) {
+    (void)d_model;
+    if (B < 0 || H < 1 || d < 1 || n_mem < 1 || top_k < 1) return 0;
+    // sized for the larger element type so one workspace serves both modes
+    return decode_layout(B, H, d, n_mem, top_k, MOM_F32).total;
+}
+
+mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_model, int H, int d,
+                           int n_mem, int top_k, float scale, mom_dtype dt,
+                           float* state, void* out, int32_t* topk_idx,
+                           void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || B < 0 || d_model <= 0 || d_model % 64 != 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM || !w) return MOM_ERR_ARG;
+    if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < mom_decode_workspace_size(B, d_model, H, d, n_mem, top_k)) return MOM_ERR_ARG;
+    if (B == 0) return MOM_OK;
+    const void* ptrs[] = {x, w->w_r, w->w_shared, w->w_gate, w->A, w->b_a, w->w_kv, state, out};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    cudaStream_t st = as_stream(stream);
+    const DecodeLayout L = decode_layout(B, H, d, n_mem, top_k, dt);
+    char* base = reinterpret_cast<char*>(ws);
+    int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(base + L.idx);
+    float* gate = reinterpret_cast<float*>(base + L.gate);
+    int32_t* perm = reinterpret_cast<int32_t*>(base + L.perm);
+    int32_t* row_of = reinterpret_cast<int32_t*>(base + L.row_of);
+    int32_t* mem_off = reinterpret_cast<int32_t*>(base + L.mem_off);
+    int32_t* seg_cu = reinterpret_cast<int32_t*>(base + L.seg_cu);
+    float* beta = reinterpret_cast<float*>(base + L.beta);
+    float* la = reinterpret_cast<float*>(base + L.la);
+
+    cudaError_t e = launch_router(x, w->w_r, w->b_r, dt, B, d_model, n_mem, top_k, idx, gate, nullptr, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    e = launch_permute(idx, B, top_k, n_mem, nullptr, 1, perm, row_of, mem_off, seg_cu, ws,
+                       base + L.perm_scratch, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    ProjArgs pa{x, perm, mem_off, w->w_shared, w->w_kv, B, d_model, H, d, n_mem, top_k,
+                base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, ws};
+    mom_status s = run_projections(pa, w->w_gate, w->A, w->b_a, dt, beta, la, st);
+    if (s != MOM_OK) return s;
+    DecodeArgs da{base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, beta, la, gate,
+                  idx, row_of, B, H, d, n_mem, top_k, scale, state, out, ws};
+    return cuda_status(launch_decode_state(da, dt, st));
+}
+
+}  // extern "C"

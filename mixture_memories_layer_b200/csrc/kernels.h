@@ -1,0 +1,90 @@
+// Internal launchers of the MoM kernels (host side).  The public C ABI in
+// mom.h validates arguments and calls these; they only launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mom {
+
+// Counts every kernel launch (mom_launch_count).
+void count_launches(int n);
+
+// router.cu
+cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int dt, int64_t n_tok, int D,
+                          int M, int K, int32_t* idx, float* gate, float* logits, cudaStream_t st);
+cudaError_t launch_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, int dt,
+                             int64_t n_tok, int D, int H, float* beta, float* log_alpha, cudaStream_t st);
+
+// permute.cu
+// `err` is the workspace whose header receives device error records;
+// `scratch` (permute_scratch_bytes) holds the tile counts.
+size_t permute_scratch_bytes(int64_t n_tok, int M);
+cudaError_t launch_permute(const int32_t* idx, int64_t n_tok, int K, int M, const int32_t* cu_seqlens, int S,
+                           int32_t* perm_token, int32_t* row_of, int32_t* mem_offset, int32_t* seg_cu,
+                           void* err, void* scratch, cudaStream_t st);
+
+// proj_simt.cu: grouped projections on CUDA cores (float32 mode, and any
+// shape the tensor-core path does not take)
+struct ProjArgs {
+    const void* x;
+    const int32_t* perm_token;
+    const int32_t* mem_offset;
+    const void* w_shared;
+    const void* w_kv;
+    int64_t n_tok;
+    int D, H, d, M, K;
+    void *q, *k_sh, *v_sh, *k_p, *v_p;
+    void* ws;
+};
+cudaError_t launch_proj_simt(const ProjArgs& a, int dt, cudaStream_t st);
+
+// proj_tc.cu: grouped projections on the tcgen05 tensor cores (bf16)
+bool proj_tc_supported(const ProjArgs& a, int dt);
+cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st);
+
+// gdn_recurrent.cu: token-serial Gated DeltaNet on CUDA cores
+struct GdnArgs {
+    const void* q;
+    const int32_t* qidx;
+    const void* k;
+    const void* v;
+    const float* beta;
+    const float* log_alpha;
+    const int32_t* seg_cu;
+    int n_seg;
+    int64_t n_rows, n_q_rows;
+    int H, d;
+    float scale;
+    const float* h0;
+    float* h_final;
+    void* o;
+    void* ws;
+    size_t ws_bytes;
+};
+cudaError_t launch_gdn_recurrent(const GdnArgs& a, int dt, cudaStream_t st);
+
+// gdn_chunk_tc.cu: chunked Gated DeltaNet on the tcgen05 tensor cores (bf16)
+bool gdn_tc_supported(const GdnArgs& a, int dt);
+size_t gdn_tc_ws_bytes(int64_t n_rows, int n_seg, int H, int d);
+cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st);
+
+// combine.cu
+cudaError_t launch_combine(const void* o_sh, const void* o_p, const int32_t* row_of, const float* gate,
+                           int64_t n_tok, int K, int H, int d, int dt, void* out, void* ws, cudaStream_t st);
+
+// decode.cu: the state pass of one decode step with the combine fused
+struct DecodeArgs {
+    const void *q, *k_sh, *v_sh, *k_p, *v_p;
+    const float *beta, *log_alpha, *gate;
+    const int32_t *idx, *row_of;
+    int B, H, d, M, K;
+    float scale;
+    float* state;
+    void* out;
+    void* ws;
+};
+cudaError_t launch_decode_state(const DecodeArgs& a, int dt, cudaStream_t st);
+
+}  // namespace mom

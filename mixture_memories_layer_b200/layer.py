@@ -1,0 +1,142 @@
+"""One MoM layer on the GPU: the six C-ABI calls in order, with torch used
+only to hold device memory.
+
+    router -> permute -> projections -> GDN (shared) -> GDN (routed) -> combine
+
+("MoM: Linear Sequence Modeling with Mixture-of-Memories", Summary; "MoM:
+Mixture-of-Memories Fixes Linear Attention Recall", Router mechanics and
+Solving scatter-gather without new kernels.)  Every step runs in the CUDA
+library; this module packs weights, allocates outputs and workspaces once
+per shape, and passes pointers.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+def pack_weights(p: Dict[str, np.ndarray], dtype: torch.dtype, device="cuda") -> Dict[str, torch.Tensor]:
+    """Stack the per-projection weights into the layouts the library reads:
+    w_shared = [W_q; W_k_sh; W_v_sh], w_gate = [W_beta; W_a],
+    w_kv[m] = [W_k^m; W_v^m] (all [out, in])."""
+    t = lambda a, dt=dtype: torch.as_tensor(np.ascontiguousarray(a)).to(device=device, dtype=dt)
+    M = p["w_k"].shape[0]
+    return dict(
+        w_r=t(p["w_r"]),
+        b_r=t(p["b_r"], torch.float32),
+        w_shared=t(np.concatenate([p["w_q"], p["w_k_sh"], p["w_v_sh"]], axis=0)),
+        w_gate=t(np.concatenate([p["w_beta"], p["w_a"]], axis=0)),
+        A=t(p["A"], torch.float32),
+        b_a=t(p["b_a"], torch.float32),
+        w_kv=t(np.stack([np.concatenate([p["w_k"][m], p["w_v"][m]], axis=0) for m in range(M)])),
+    )
+
+
+class MoMLayer:
+    """Holds packed weights and reusable buffers for one layer shape."""
+
+    def __init__(self, weights: Dict[str, torch.Tensor], heads: int, d_head: int, top_k: int,
+                 scale: float = 1.0):
+        self.w = weights
+        self.H, self.d, self.top_k, self.scale = heads, d_head, top_k, scale
+        self.n_mem, self.d_model = weights["w_r"].shape
+        self.dtype = weights["w_r"].dtype
+        self.device = weights["w_r"].device
+        self._bufs = {}
+        self._c_weights = B.MomWeights(*[ctypes_ptr(weights[k]) for k in
+                                         ("w_r", "b_r", "w_shared", "w_gate", "A", "b_a", "w_kv")])
+
+    # -------------------------------------------------------------- buffers
+    def _buf(self, name, shape, dtype):
+        key = (name, tuple(shape), dtype)
+        t = self._bufs.get(key)
+        if t is None:
+            t = torch.empty(shape, dtype=dtype, device=self.device)
+            self._bufs[key] = t
+        return t
+
+    def _ws(self, name, nbytes):
+        key = ("ws", name)
+        t = self._bufs.get(key)
+        if t is None or t.numel() < nbytes:
+            t = B.new_workspace(nbytes, self.device)
+            self._bufs[key] = t
+        return t
+
+    def buffers(self, n_tok: int, n_seq: int):
+        H, d, K, M, dt = self.H, self.d, self.top_k, self.n_mem, self.dtype
+        f32, i32 = torch.float32, torch.int32
+        b = dict(
+            idx=self._buf("idx", (n_tok, K), i32), gate=self._buf("gate", (n_tok, K), f32),
+            perm=self._buf("perm", (n_tok * K,), i32), row_of=self._buf("row_of", (n_tok * K,), i32),
+            mem_offset=self._buf("mem_offset", (M + 1,), i32), seg_cu=self._buf("seg_cu", (M * n_seq + 1,), i32),
+            q=self._buf("q", (n_tok, H, d), dt), k_sh=self._buf("k_sh", (n_tok, H, d), dt),
+            v_sh=self._buf("v_sh", (n_tok, H, d), dt), beta=self._buf("beta", (n_tok, H), f32),
+            log_alpha=self._buf("log_alpha", (n_tok, H), f32),
+            k_p=self._buf("k_p", (n_tok * K, H, d), dt), v_p=self._buf("v_p", (n_tok * K, H, d), dt),
+            o_sh=self._buf("o_sh", (n_tok, H, d), dt), o_p=self._buf("o_p", (n_tok * K, H, d), dt),
+            out=self._buf("out", (n_tok, H, d), dt),
+            h_shared=self._buf("h_shared", (n_seq, H, d, d), f32),
+            h_mem=self._buf("h_mem", (M, n_seq, H, d, d), f32),
+        )
+        dtc = B.dtype_code(dt)
+        b["ws_perm"] = self._ws("perm", B.mom_permute_workspace_size(n_tok, K, M, n_seq))
+        b["ws_proj"] = self._ws("proj", B.mom_kv_proj_workspace_size(n_tok, self.d_model, H, d, M, K))
+        b["ws_gdn_sh"] = self._ws("gdn_sh", B.mom_gdn_workspace_size(n_tok, n_seq, H, d, dtc))
+        b["ws_gdn_p"] = self._ws("gdn_p", B.mom_gdn_workspace_size(n_tok * K, M * n_seq, H, d, dtc))
+        b["ws_comb"] = self._ws("comb", B.MOM_WS_HEADER_BYTES)
+        return b
+
+    # -------------------------------------------------------------- forward
+    def forward(self, x: torch.Tensor, cu_seqlens: torch.Tensor, h0_shared=None, h0_mem=None,
+                want_states: bool = True, stream=None) -> Dict[str, torch.Tensor]:
+        """x [N, d_model] (device), cu_seqlens [S+1] int32 (device).  Returns
+        the buffers dict; ``out`` is the layer output, ``h_shared`` [S,H,d,d]
+        and ``h_mem`` [M,S,H,d,d] the final states."""
+        n_tok = x.shape[0]
+        n_seq = cu_seqlens.numel() - 1
+        w, b = self.w, self.buffers(n_tok, n_seq)
+        B.mom_router_topk(x, w["w_r"], w["b_r"], self.top_k, b["idx"], b["gate"], stream=stream)
+        B.mom_permute(b["idx"], self.n_mem, cu_seqlens, b["perm"], b["row_of"], b["mem_offset"], b["seg_cu"],
+                      b["ws_perm"], stream=stream)
+        B.mom_kv_proj_grouped(x, b["perm"], b["mem_offset"], w["w_shared"], w["w_gate"], w["A"], w["b_a"],
+                              w["w_kv"], self.H, self.d, self.top_k, b["q"], b["k_sh"], b["v_sh"], b["beta"],
+                              b["log_alpha"], b["k_p"], b["v_p"], b["ws_proj"], stream=stream)
+        hs = b["h_shared"] if want_states else None
+        hm = b["h_mem"] if want_states else None
+        B.mom_gdn_chunk_fwd(b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens,
+                            self.scale, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"], stream=stream)
+        B.mom_gdn_chunk_fwd(b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
+                            self.scale, h0_mem, hm, b["o_p"], b["ws_gdn_p"], stream=stream)
+        B.mom_combine_unpermute(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["out"], b["ws_comb"], stream=stream)
+        return b
+
+    def device_errors(self):
+        """(code, info) of every workspace with a recorded violation."""
+        errs = {}
+        for key, t in self._bufs.items():
+            if isinstance(key, tuple) and key[0] == "ws":
+                code, info = B.mom_get_error(t)
+                if code:
+                    errs[key[1]] = (code, info)
+        return errs
+
+    # --------------------------------------------------------------- decode
+    def decode_step(self, x: torch.Tensor, state: torch.Tensor, stream=None):
+        """x [B, d_model]; state [B, M+1, H, d, d] float32, updated in place.
+        Returns (out [B,H,d], topk_idx [B,k])."""
+        Bn = x.shape[0]
+        out = self._buf("dec_out", (Bn, self.H, self.d), self.dtype)
+        idx = self._buf("dec_idx", (Bn, self.top_k), torch.int32)
+        ws = self._ws("decode", B.mom_decode_workspace_size(Bn, self.d_model, self.H, self.d, self.n_mem, self.top_k))
+        B.mom_decode_step(x, self._c_weights, self.H, self.d, self.n_mem, self.top_k, self.scale, state, out, idx, ws,
+                          stream=stream)
+        return out, idx
+
+
+def ctypes_ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()

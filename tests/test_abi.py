@@ -1,0 +1,61 @@
+"""The C-ABI library loads, exports every entry point that include/mom.h
+declares, and rejects bad arguments on the host before any launch (these
+calls never reach the GPU, so they run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "mom.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:mom_status|size_t|uint64_t|const char\*)\s+(mom_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixture_memories_layer_b200 import build
+    build.build(verbose=False)
+    from mixture_memories_layer_b200 import binding
+    return binding
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib.lib, n), n
+    assert set(names) == set(lib.SIGNATURES), "binding signatures out of sync with mom.h"
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    L, B = lib.lib, lib
+    fake = ctypes.c_void_p(0x10000)       # never dereferenced: validation fails first
+    s = L.mom_router_topk(fake, fake, None, B.MOM_BF16, 10, 64, 4, 5, fake, fake, None, None)
+    assert s == B.MOM_ERR_ARG                                   # top_k > n_mem
+    s = L.mom_router_topk(fake, fake, None, B.MOM_BF16, 10, 60, 4, 2, fake, fake, None, None)
+    assert s == B.MOM_ERR_ARG                                   # d_model % 8
+    s = L.mom_router_topk(fake, fake, None, 7, 10, 64, 4, 2, fake, fake, None, None)
+    assert s == B.MOM_ERR_ARG                                   # dtype
+    s = L.mom_kv_proj_grouped(*([fake] * 8), B.MOM_BF16, 10, 256, 2, 96, 4, 2, *([fake] * 8), 4096, None)
+    assert s == B.MOM_ERR_UNSUPPORTED                           # d = 96
+    s = L.mom_gdn_chunk_fwd(*([fake] * 7), 3, 10, 10, 2, 64, 1.0, B.MOM_BF16, None, None, fake, fake, 8, None)
+    assert s == B.MOM_ERR_ARG                                   # workspace too small
+    s = L.mom_permute(fake, 10, 2, 4, None, 2, fake, fake, fake, fake, fake, 1 << 20, None)
+    assert s == B.MOM_ERR_ARG                                   # no cu_seqlens with 2 sequences
+    s = L.mom_get_error(None, None, None, None)
+    assert s == B.MOM_ERR_ARG
+    assert L.mom_status_string(B.MOM_ERR_UNSUPPORTED) == b"unsupported shape or type"
+
+
+def test_workspace_sizes_are_monotone(lib):
+    L = lib.lib
+    a = L.mom_permute_workspace_size(1000, 2, 4, 3)
+    b = L.mom_permute_workspace_size(100000, 2, 4, 3)
+    assert lib.MOM_WS_HEADER_BYTES <= a <= b
+    assert L.mom_decode_workspace_size(256, 1024, 4, 256, 8, 2) > L.mom_decode_workspace_size(16, 1024, 4, 256, 8, 2)

@@ -1,0 +1,151 @@
+"""GPU parity of the whole MoM layer and of each C-ABI entry point against
+the fp64 oracle, on seeded inputs small enough for the oracle to finish in
+seconds while still spanning several 64-row chunks, several GEMM tiles and
+ragged tails.
+
+Acceptance ("MoM: Linear Sequence Modeling with Mixture-of-Memories",
+Summary, for what the layer computes): router indices and the permutation
+bit-exact, with near-tie tokens (k-th vs (k+1)-th logit gap < 1e-4) counted
+and excluded; outputs and final states within max-abs-rel 1e-4 (float32) or
+2e-2 (bf16 inputs, float32 state).  The oracle is re-run with the GPU's
+routing imposed, so that a near-tie choice does not change a whole memory's
+downstream state.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_memories_layer_b200 import synth
+from oracle import mom_oracle as orc
+from tests.gpu_helpers import TOL, max_abs_rel, run_layer, to_np, torch_dtype
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _small(d, dtype="bf16", lens=(300, 77, 1), M=4, k=2, H=2, D=256, seed=0, bias0=0.0):
+    w = synth.Workload("small", 0, 0, D, H, d, M, k, dtype, seed=seed, router_bias0=bias0)
+    rng = np.random.default_rng(seed)
+    p = synth.make_weights(w, rng)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    p["cu_seqlens"] = cu
+    p["x"] = synth.make_tokens(w, rng, int(cu[-1]))
+    return w, p
+
+
+def _check_layer(w, p, res, seqs=None, scale=1.0, tol=None, out_rows=None):
+    tol = tol or TOL[w.dtype]
+    cu = p["cu_seqlens"]
+    S = len(cu) - 1
+    seqs = range(S) if seqs is None else seqs
+    for s in seqs:
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        if out_rows is not None:
+            t1 = min(t1, t0 + out_rows)
+        ref = orc.mom_forward(p["x"][t0:t1], p, np.array([0, t1 - t0]), w.top_k, w.heads, w.d_head,
+                              scale=scale, forced_idx=res["idx"][t0:t1])
+        # routing: bit-exact outside near ties
+        keep = ~ref["near_tie"]
+        nat = orc.router_topk(p["x"][t0:t1], p["w_r"], p["b_r"], w.top_k)[0]
+        assert np.array_equal(res["idx"][t0:t1][keep], nat[keep]), "router indices differ"
+        assert max_abs_rel(res["gate"][t0:t1], ref["gate"]) < 1e-5
+        e_out = max_abs_rel(res["out"][t0:t1], ref["out"])
+        assert e_out < tol, ("out", s, e_out)
+        if out_rows is None or t1 == int(cu[s + 1]):
+            e_hs = max_abs_rel(res["h_shared"][s], ref["h_shared"][0])
+            e_hm = max_abs_rel(res["h_mem"][:, s], ref["h_mem"][:, 0])
+            assert e_hs < tol and e_hm < tol, ("states", s, e_hs, e_hm)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_layer_small_bf16(d):
+    w, p = _small(d)
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _check_layer(w, p, res)
+
+
+def test_layer_tiny_fp32_workload():
+    w = synth.WORKLOADS["tiny_fp32"]
+    p = synth.make_problem(w)
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _check_layer(w, p, res)
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_layer_small_fp32_ragged(d):
+    w, p = _small(d, dtype="f32", lens=(130, 64, 65, 2))
+    lay, res = run_layer(w, p, scale=0.5)
+    _check_layer(w, p, res, scale=0.5)
+
+
+def test_layer_skewed_routing_and_empty_segments():
+    # +6 on memory 0 sends nearly every token there; memories 1-3 see few or none
+    w, p = _small(128, lens=(200, 0, 90), bias0=6.0)
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _check_layer(w, p, res)
+
+
+def test_layer_all_tokens_one_memory_top1_M1():
+    w, p = _small(64, M=1, k=1, lens=(150,))
+    lay, res = run_layer(w, p)
+    assert np.all(res["idx"] == 0) and np.allclose(res["gate"], 1.0)
+    _check_layer(w, p, res)
+
+
+def test_layer_many_memories_top4():
+    w, p = _small(64, M=16, k=4, lens=(257, 31), H=3, D=192)
+    lay, res = run_layer(w, p)
+    _check_layer(w, p, res)
+
+
+def test_layer_h0_hand_off():
+    """Forward over [0, T) equals [0, T/2) then [T/2, T) seeded with the
+    first call's final states."""
+    w, p = _small(128, lens=(160,))
+    _, full = run_layer(w, p)
+    x = p["x"]
+    pa = dict(p, x=x[:70], cu_seqlens=np.array([0, 70], np.int32))
+    pb = dict(p, x=x[70:], cu_seqlens=np.array([0, 90], np.int32))
+    _, ra = run_layer(w, pa)
+    h0s = torch.as_tensor(ra["h_shared"]).cuda()
+    h0m = torch.as_tensor(ra["h_mem"]).cuda()
+    _, rb = run_layer(w, pb, h0_shared=h0s, h0_mem=h0m)
+    tol = TOL[w.dtype]
+    assert max_abs_rel(rb["out"], full["out"][70:]) < tol
+    assert max_abs_rel(rb["h_mem"], full["h_mem"]) < tol
+    assert max_abs_rel(rb["h_shared"], full["h_shared"]) < tol
+
+
+def test_permute_bit_exact():
+    w, p = _small(64, M=8, k=2, lens=(500, 3, 0, 260))
+    lay, res = run_layer(w, p)
+    perm, row_of, offs, seg = orc.permute(res["idx"], w.n_mem, p["cu_seqlens"])
+    n = int(offs[-1])
+    assert np.array_equal(res["perm"][:n], perm)
+    assert np.array_equal(res["row_of"], row_of)
+    assert np.array_equal(res["mem_offset"], offs)
+    assert np.array_equal(res["seg_cu"], seg)
+
+
+def test_projections_match_oracle():
+    w, p = _small(128, lens=(200, 57))
+    lay, res = run_layer(w, p)
+    q, k_sh, v_sh, beta, la = orc.shared_projections(p["x"], p, w.heads, w.d_head)
+    tol = TOL[w.dtype]
+    for name, ref in (("q", q), ("k_sh", k_sh), ("v_sh", v_sh)):
+        assert max_abs_rel(res[name], ref) < tol, name
+    assert max_abs_rel(res["beta"], beta) < 1e-5
+    assert max_abs_rel(res["log_alpha"], la) < 1e-5
+    perm, _, offs, _ = orc.permute(res["idx"], w.n_mem, p["cu_seqlens"])
+    for m in range(w.n_mem):
+        rows = slice(offs[m], offs[m + 1])
+        km, vm = orc.memory_kv(p["x"][perm[rows]], p, m, w.heads, w.d_head)
+        assert max_abs_rel(res["k_p"][rows], km) < tol
+        assert max_abs_rel(res["v_p"][rows], vm) < tol
