@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the MoM layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is one MoM layer forward (router -> permute -> projections -> GDN
+shared -> GDN routed -> combine) over the 380M-shape workload: 8 sequences
+x 2048 tokens, d_model 1024, 4 heads of d_k = d_v = 256, 4 memories top-2
+plus the shared memory, bf16 activations and weights, float32 state.  Inputs
+are seeded synthetic tensors already resident in HBM; L2 is flushed (a
+256 MiB write) before every timed step, outside its events.  The recurrent
+decode step (256 sequences, 8 memories top-2, one new token per sequence,
+float32 states of 2.4 GB, larger than L2) is timed in the same run and
+reported under "decode".
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own batch of
+sequences: the layer shards by sequence with no collective on the data
+path (weak scaling); the step time is the max over ranks.
+
+`--impl reference` times the CPU oracle (fp64 numpy) on bounded samples of
+the same workload instead: rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "MoM layer fwd tokens/s at 1 B200 and % of roofline; decode tokens/s"
+UNIT = "tokens/s"
+FWD = "mom380m"
+DEC = "decode_b256"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def workload_desc(w):
+    return ("MoM layer forward, %s shape: B=%d x T=%d tokens, d_model=%d, H=%d, d_k=d_v=%d, "
+            "M=%d memories top-%d + shared, bf16 activations / fp32 state"
+            % (w.name, w.batch, w.seq_len, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        p["source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["source"] = "fallback"
+    return p
+
+
+# ------------------------------------------------------------ algorithmic work
+def step_work(w):
+    """Algorithmic FLOPs / bytes of each of the six calls for one forward of
+    workload w (minimum the method needs; intermediates not re-counted)."""
+    N, D, H, d, M, K = w.n_tokens, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k
+    e = 2  # bf16
+    return {
+        "router": {"bound": "hbm", "bytes": N * D * e + M * D * e + N * K * 8},
+        "permute": {"bound": "hbm", "bytes": 2 * N * K * 4 + N * K * 8},
+        "proj": {"bound": "tensor", "flops": 2 * N * D * (3 * H * d + 2 * H) + 2 * N * K * D * 2 * H * d},
+        "gdn_shared": {"bound": "tensor", "flops": 6 * N * H * d * d},
+        "gdn_routed": {"bound": "tensor", "flops": 6 * N * K * H * d * d},
+        "combine": {"bound": "hbm", "bytes": e * N * H * d * (2 + K) + N * K * 8},
+    }
+
+
+def layer_roofline(w, peaks):
+    N, D, H, d, M, K = w.n_tokens, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k
+    S = w.batch
+    sw = step_work(w)
+    flops = sw["proj"]["flops"] + sw["gdn_shared"]["flops"] + sw["gdn_routed"]["flops"] \
+        + 2 * N * D * M + 2 * K * N * H * d
+    weights = (M * D + 3 * H * d * D + 2 * H * D + M * 2 * H * d * D) * 2
+    bytes_ = N * D * 2 + weights + N * H * d * 2 + (S + M * S) * H * d * d * 4 + N * K * 8
+    t = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    return flops, bytes_, t
+
+
+def kernel_source_sha(name):
+    path = os.path.join(ROOT, "mixture_memories_layer_b200", "csrc", name)
+    if not os.path.exists(path):
+        return None
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def measured_traffic(call):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's
+    source is unchanged since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        t = json.load(fh).get(call)
+    if not t or kernel_source_sha(t["source"]) != t.get("source_sha"):
+        return None
+    return t["bytes_per_launch"]
+
+
+# -------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML (read-only) every 10 ms in a thread while the timed region
+    runs: SM clock, its maximum, and the active clock-event reasons."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, torch_device, period=0.01):
+        self.dev, self.period = torch_device, period
+        self.samples = []
+        self._stop = None
+        self.error = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pr = torch.cuda.get_device_properties(self.dev)
+        try:   # NVML numbers GPUs differently from CUDA under CUDA_VISIBLE_DEVICES
+            bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+
+    def _run(self):
+        import pynvml
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception as e:          # keep the first failure for the report
+                self.error = self.error or repr(e)
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.h = self._handle()
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:
+            self.sm_max, self.error = None, repr(e)
+            return self
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._stop is not None:
+            self._stop.set()
+            self._t.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": ["unsampled"], "samples": 0,
+                    "error": self.error}
+        sm = [s for s, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.sm_max, "reasons": reasons,
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- the GPU arm
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    from mixture_memories_layer_b200 import binding as B
+    from mixture_memories_layer_b200 import layer as L
+    from mixture_memories_layer_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d (launch N>1 with torchrun)" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    w = synth.WORKLOADS[FWD]
+    # replicated weights; each rank draws its own batch of sequences
+    p = synth.make_problem(w)
+    if rank:
+        p["x"] = synth.make_tokens(w, np.random.default_rng(w.seed * 1000 + rank), w.n_tokens)
+    dt = torch.bfloat16
+    lay = L.MoMLayer(L.pack_weights(p, dt, dev), w.heads, w.d_head, w.top_k)
+    x = torch.as_tensor(p["x"]).to(dev, dt)
+    cu = torch.as_tensor(p["cu_seqlens"]).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    clocks = ClockSampler(dev).__enter__()     # sampled from warm-up to the end of decode
+    for _ in range(args.warmup):
+        lay.forward(x, cu)
+    torch.cuda.synchronize()
+    errs = lay.device_errors()
+    if errs:
+        raise SystemExit("device error records after warm-up: %s" % errs)
+
+    n_calls = len(L.MoMLayer.STEPS)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_calls + 1)] for _ in range(args.steps)]
+    launches0 = B.mom_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.zero_()                          # evict L2 (outside the step's events)
+        lay.forward(x, cu, marks=marks[s])
+    torch.cuda.synchronize()
+    barrier()
+    launches = B.mom_launch_count() - launches0
+    step_ms = [marks[s][0].elapsed_time(marks[s][n_calls]) for s in range(args.steps)]
+    total_ms = max_over_ranks(sum(step_ms))
+    per_call = {name: sum(marks[s][i].elapsed_time(marks[s][i + 1]) for s in range(args.steps)) / args.steps
+                for i, name in enumerate(L.MoMLayer.STEPS)}
+    ms_per_step = total_ms / args.steps
+    tokens_all = w.n_tokens * world * args.steps
+    value = tokens_all / (total_ms / 1e3)
+
+    # ---- roofline of the dominant call
+    work = step_work(w)
+    top = max(per_call, key=per_call.get)
+    wk = work[top]
+    sec = per_call[top] / 1e3
+    if wk["bound"] == "tensor":
+        achieved = wk["flops"] / sec / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    else:
+        achieved = wk["bytes"] / sec / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof.update({"kernel": top, "traffic": measured_traffic(top), "peak_source": peaks["source"],
+                 "ms_per_launch": per_call[top]})
+    lf, lb, lt = layer_roofline(w, peaks)
+    layer_roof = {"flops": lf, "bytes": lb, "roofline_ms": lt * 1e3, "frac": (lt * 1e3) / ms_per_step}
+
+    # ---- end to end through the C ABI with host buffers
+    x_host = torch.empty(x.shape, dtype=dt, pin_memory=True)
+    x_host.copy_(x.cpu())
+    out_host = torch.empty((w.n_tokens, w.heads, w.d_head), dtype=dt, pin_memory=True)
+    e_ms = []
+    for s in range(max(3, args.steps)):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        x.copy_(x_host, non_blocking=True)
+        b = lay.forward(x, cu)
+        out_host.copy_(b["out"], non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e_ms.append(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(sum(e_ms[-args.steps:]) if args.steps else sum(e_ms))
+    n_e2e = min(len(e_ms), args.steps) if args.steps else len(e_ms)
+    e2e = {"value": w.n_tokens * world * n_e2e / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": x.numel() * x.element_size(),
+           "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+
+    # ---- decode
+    decode = decode_bench(args, dev, world, rank, max_over_ranks, barrier)
+    clocks.__exit__(None, None, None)
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline(w) if (world == 1 and not args.no_cpu_baseline) else None
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded X~N(0,1), weights~N(0,1/d_model), A~U(0,2.7), b_a~U(-4,0)",
+            "config": {"workload": workload_desc(w), "tokens_per_gpu": w.n_tokens, "global_tokens": w.n_tokens * world,
+                       "seq_len": w.seq_len, "parallelism": "dp%d (sequences sharded, no collective)" % world,
+                       "l2": "flushed before every timed step (256 MiB write, untimed)"},
+            "roofline": roof, "layer_roofline": layer_roof,
+            "per_call_ms": per_call, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks.summary(), "decode": decode,
+        }
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return result
+
+
+def decode_bench(args, dev, world, rank, max_over_ranks, barrier):
+    import torch
+
+    from mixture_memories_layer_b200 import layer as L
+    from mixture_memories_layer_b200 import synth
+
+    w = synth.WORKLOADS[DEC]
+    steps = w.decode_steps
+    p = synth.make_decode_problem(w, steps=steps + args.warmup)
+    dt = torch.bfloat16
+    lay = L.MoMLayer(L.pack_weights(p, dt, dev), w.heads, w.d_head, w.top_k)
+    b = lay.forward(torch.as_tensor(p["x_prefill"]).to(dev, dt), torch.as_tensor(p["cu_prefill"]).to(dev))
+    state0 = torch.empty((w.batch, w.n_mem + 1, w.heads, w.d_head, w.d_head), dtype=torch.float32, device=dev)
+    state0[:, :w.n_mem] = b["h_mem"].permute(1, 0, 2, 3, 4)
+    state0[:, w.n_mem] = b["h_shared"]
+    xs = torch.as_tensor(p["x_steps"]).to(dev, dt)
+    state = state0.clone()
+    for s in range(args.warmup):
+        lay.decode_step(xs[steps + s], state)
+    state.copy_(state0)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(steps):
+        lay.decode_step(xs[s], state)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    state_bytes = (w.top_k + 1) * w.batch * w.heads * w.d_head * w.d_head * 4 * 2
+    per_step = ms / steps
+    hbm = load_peaks()["hbm_gbs"]
+    return {"workload": "decode: B=%d sequences, d_model=%d, H=%d, d=%d, M=%d top-%d + shared, %d steps after a "
+                        "%d-token prefill" % (w.batch, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k, steps,
+                                              w.prefill_len),
+            "value": w.batch * world * steps / (ms / 1e3), "unit": "tokens/s", "ms_per_step": per_step,
+            "state_bytes_per_step": state_bytes,
+            "state_gbs": state_bytes / (per_step / 1e3) / 1e9,
+            "frac_hbm": state_bytes / (per_step / 1e3) / 1e9 / hbm}
+
+
+# --------------------------------------------------------- CPU oracle timing
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w, n_tokens=2048):
+    from oracle import mom_oracle as orc
+    from mixture_memories_layer_b200 import synth
+    p = synth.make_problem(w)
+    x = p["x"][:n_tokens]
+    t0 = time.perf_counter()
+    orc.mom_forward(x, p, np.array([0, n_tokens]), w.top_k, w.heads, w.d_head)
+    dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": "first %d tokens of sequence 0 (one full sequence) of the same workload; fp64 numpy, "
+                      "BLAS-threaded projections, single-threaded token recurrence; %.1f s" % (n_tokens, dt)}
+
+
+def reference_arm(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return None
+    from oracle import mom_oracle as orc
+    from mixture_memories_layer_b200 import synth
+    w = synth.WORKLOADS[FWD]
+    p = synth.make_problem(w)
+    T = 128                       # tokens per step: one bounded window of one sequence
+    n_win = w.n_tokens // T
+
+    def step(i):
+        t0 = (i % n_win) * T
+        orc.mom_forward(p["x"][t0:t0 + T], p, np.array([0, T]), w.top_k, w.heads, w.d_head)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    sec = time.perf_counter() - t0
+    value = T * args.steps / sec
+    sample = ("each step: the oracle layer forward on a %d-token window (state from zero) of one sequence of "
+              "the same workload" % T)
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3 / max(args.steps, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic: seeded, same generator as the GPU arm",
+           "config": {"workload": workload_desc(w), "tokens_per_step": T},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()
