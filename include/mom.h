@@ -136,6 +136,38 @@ mom_status mom_permute(const int32_t* topk_idx, int64_t n_tok, int top_k, int n_
                        void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * mom_permute_noalloc -- mom_permute without a workspace.  The MoM pages
+ * have no counterpart to this: it exists for callers that cannot allocate
+ * device memory, such as a plug-in inside a host engine that owns every
+ * byte of the device through its own fixed pool and forbids raw
+ * cudaMalloc, or a latency-critical serving loop where cudaMalloc and
+ * cudaFree are not allowed because they can block the host and synchronise
+ * the device.
+ *
+ * Same arguments, outputs and results as mom_permute, minus ws/ws_bytes.
+ * Its scratch space is a fixed array inside the library (about 1 MiB per
+ * GPU that loads the library, held until the process exits), so:
+ *   - n_tok may not exceed MOM_PERMUTE_NOALLOC_MAX_TOKENS (and n_mem may
+ *     not exceed MOM_MAX_MEM); larger problems return MOM_ERR_UNSUPPORTED
+ *     and launch nothing;
+ *   - the first call on a device looks up the array's device address (a
+ *     runtime query, once per device, cached); make that first call before
+ *     any stream capture on that device;
+ *   - every call on a device shares the array: calls whose kernels overlap
+ *     on the GPU (unordered streams, several host threads) race and may
+ *     give wrong results -- order them on one stream;
+ *   - each call clears the array's error record first; status_out (device
+ *     int32[2], or NULL) receives this call's record {code, info}
+ *     (MOM_DEVERR_*), asynchronously on `stream`.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * ---------------------------------------------------------------------- */
+#define MOM_PERMUTE_NOALLOC_MAX_TOKENS (1 << 20)
+mom_status mom_permute_noalloc(const int32_t* topk_idx, int64_t n_tok, int top_k, int n_mem,
+                               const int32_t* cu_seqlens, int n_seq,
+                               int32_t* perm_token, int32_t* row_of, int32_t* mem_offset, int32_t* seg_cu,
+                               int32_t* status_out, void* stream);
+
+/* ------------------------------------------------------------------------
  * mom_kv_proj_grouped -- every projection of the layer (paper card,
  * Summary: a shared query, and key/value projections of each memory's own):
  *

@@ -31,6 +31,7 @@ SIGNATURES = {
     "mom_router_topk": (_I, [_VP, _VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "mom_permute_workspace_size": (_SZ, [_I64, _I, _I, _I]),
     "mom_permute": (_I, [_VP, _I64, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_permute_noalloc": (_I, [_VP, _I64, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
     "mom_kv_proj_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I]),
     "mom_kv_proj_grouped": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
                                  _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -131,6 +132,21 @@ def mom_permute(topk_idx, n_mem, cu_seqlens, perm_token, row_of, mem_offset, seg
     n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
     _check(lib.mom_permute(_p(topk_idx), n_tok, top_k, n_mem, _p(cu_seqlens), n_seq, _p(perm_token), _p(row_of),
                            _p(mem_offset), _p(seg_cu), _p(ws), ws.numel(), _s(stream)), "mom_permute")
+
+
+MOM_PERMUTE_NOALLOC_MAX_TOKENS = 1 << 20
+
+
+def mom_permute_noalloc(topk_idx, n_mem, cu_seqlens, perm_token, row_of, mem_offset, seg_cu, status=None,
+                        stream=None):
+    """mom_permute for callers that cannot allocate device memory: no
+    workspace; scratch is a fixed array inside the library (shared by all
+    calls on the device, so calls must not overlap on the GPU)."""
+    n_tok, top_k = topk_idx.shape
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib.mom_permute_noalloc(_p(topk_idx), n_tok, top_k, n_mem, _p(cu_seqlens), n_seq, _p(perm_token),
+                                   _p(row_of), _p(mem_offset), _p(seg_cu), _p(status), _s(stream)),
+           "mom_permute_noalloc")
 
 
 def mom_kv_proj_workspace_size(n_tok, d_model, H, d, n_mem, top_k):
