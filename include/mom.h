@@ -68,6 +68,7 @@ typedef int mom_dtype;
 #define MOM_DEVERR_MEM_INDEX  1  /* topk_idx entry outside [0, n_mem) or repeated in a row */
 #define MOM_DEVERR_ROW_INDEX  2  /* a row / token index outside its array */
 #define MOM_DEVERR_SEGMENT    3  /* segment bounds decreasing or beyond n_rows */
+#define MOM_DEVERR_TIMEOUT    4  /* a pipeline wait inside a kernel gave up (internal error) */
 
 #define MOM_WS_HEADER_BYTES 256
 

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmom_b200
 
 MOM_OK, MOM_ERR_ARG, MOM_ERR_UNSUPPORTED, MOM_ERR_CUDA, MOM_ERR_DEVICE = 0, 1, 2, 3, 4
 MOM_F32, MOM_BF16 = 0, 1
-MOM_DEVERR_NONE, MOM_DEVERR_MEM_INDEX, MOM_DEVERR_ROW_INDEX, MOM_DEVERR_SEGMENT = 0, 1, 2, 3
+MOM_DEVERR_NONE, MOM_DEVERR_MEM_INDEX, MOM_DEVERR_ROW_INDEX, MOM_DEVERR_SEGMENT, MOM_DEVERR_TIMEOUT = 0, 1, 2, 3, 4
 MOM_WS_HEADER_BYTES = 256
 
 # every function the header declares, with (restype, argtypes)

@@ -1,10 +1,377 @@
-// Grouped projections on the tcgen05 tensor cores (bf16).  Placeholder until
-// the tensor-core GEMM lands: reports every shape as unsupported, so the
-// CUDA-core kernel runs.
+// Grouped projections on the tcgen05 tensor cores (bf16 in, fp32 accumulate).
+//
+// ("MoM: Linear Sequence Modeling with Mixture-of-Memories", Summary: a
+// shared query and each memory's own key/value projections.)  Two groups of
+// problems share one persistent launch:
+//   shared : every token x [W_q | W_k_sh | W_v_sh]^T      -> q, k_sh, v_sh
+//   memory m: reordered rows mem_offset[m] .. mem_offset[m+1] (token
+//             perm_token[r]) x [W_k^m | W_v^m]^T           -> k_p, v_p
+// Output tiles are 128 rows x 256 columns; a tile never straddles two
+// memories or two projections, and holds whole heads, so the per-head L2
+// norm of q and k is applied in the epilogue straight from TMEM.
+//
+// Roles (288 threads, one CTA per SM, persistent over tiles):
+//   warps 0-3  producers: A rows gathered with 16-byte cp.async into the
+//              128-byte-swizzled K-major layout (rows come from perm_token,
+//              so a tile of routed rows is a gather); thread 0 also issues
+//              the TMA load of the weight tile (B, K-major, 128-byte swizzle)
+//   warp 8     MMA issuer: 4 x tcgen05.mma (M=128, N=256, K=16) per 64-wide
+//              K step into one of two TMEM accumulators (2 x 256 columns)
+//   warps 4-7  epilogue: TMEM -> registers -> (L2 norm) -> bf16 -> global,
+//              overlapping the next tile's main loop
+// Every wait is bounded (sm100.cuh); on a timeout the CTA records
+// MOM_DEVERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace mom {
-bool proj_tc_supported(const ProjArgs&, int) { return false; }
-cudaError_t launch_proj_tc(const ProjArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int B_BYTES = BN * BK * 2;   // 32 KB
+constexpr int NPROD = 128, NEPI = 128;
+constexpr int THREADS = NPROD + NEPI + 32;
+constexpr int LAG = STAGES - 1;        // producer arrives for a stage LAG iterations after issuing it
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+
+struct TcParams {
+    const bf16* x;
+    const int32_t* perm;
+    const int32_t* mem_offset;
+    bf16 *q, *k_sh, *v_sh, *k_p, *v_p;
+    int64_t n_tok;
+    int D, H, d, M, K;
+    int sh_ct, rt_ct;       // column tiles per row tile (shared / routed)
+    int64_t sh_tiles;       // shared tiles
+    int64_t n_tiles;        // shared + an upper bound of routed tiles
+    void* ws;
+};
+
+struct Tile {
+    int64_t r0, r1;  // row range [r0, r1)
+    int ct;          // column tile
+    int m;           // memory, -1 for the shared group
+};
+
+// Tile t of the launch (identical answer in every role).  Routed tiles past
+// the real count (the grid is sized by an upper bound) return false.
+__device__ __forceinline__ bool tile_at(const TcParams& p, int64_t t, Tile& T) {
+    if (t < p.sh_tiles) {
+        const int64_t rt = t / p.sh_ct;
+        T.ct = (int)(t % p.sh_ct);
+        T.r0 = rt * BM;
+        T.r1 = T.r0 + BM < p.n_tok ? T.r0 + BM : p.n_tok;
+        T.m = -1;
+        return true;
+    }
+    const int64_t local = t - p.sh_tiles;
+    int64_t rt = local / p.rt_ct;
+    T.ct = (int)(local % p.rt_ct);
+    const int64_t n_rows = p.n_tok * p.K;
+    for (int m = 0; m < p.M; ++m) {
+        const int64_t lo = p.mem_offset[m], hi = p.mem_offset[m + 1];
+        if (lo < 0 || hi < lo || hi > n_rows) return false;
+        const int64_t nt = (hi - lo + BM - 1) / BM;
+        if (rt < nt) {
+            T.m = m;
+            T.r0 = lo + rt * BM;
+            T.r1 = T.r0 + BM < hi ? T.r0 + BM : hi;
+            return true;
+        }
+        rt -= nt;
+    }
+    return false;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant__ CUtensorMap tm_kv, TcParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                           ~static_cast<uintptr_t>(1023));
+    unsigned char* sA = smem;
+    unsigned char* sB = smem + STAGES * A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t full0 = smem_u32(bars);
+    const uint32_t empty0 = smem_u32(bars + STAGES);
+    const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+    const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+    const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full0 + 8 * s, NPROD + 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull0 + 8 * a, 1);
+            mbar_init(tempty0 + 8 * a, NEPI);
+        }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int KB = p.D / BK;
+
+    if (warp < 4) {
+        // ------------------------------------------------------ producers
+        const int tid = threadIdx.x;
+        const int c = tid & 7, rsub = tid >> 3;   // 8 lanes per 128-byte row, 16 rows per pass
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+            Tile T;
+            if (!tile_at(p, t, T)) continue;
+            const bf16* src[8];
+            uint32_t nbytes[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int64_t row = T.r0 + rsub + 16 * i;
+                int64_t tok = -1;
+                if (row < T.r1) {
+                    tok = T.m < 0 ? row : (int64_t)p.perm[row];
+                    if (tok < 0 || tok >= p.n_tok) {
+                        if (c == 0) record_error(p.ws, MOM_DEVERR_ROW_INDEX, row);
+                        tok = -1;
+                    }
+                }
+                src[i] = p.x + (tok >= 0 ? tok : 0) * p.D + c * 8;
+                nbytes[i] = tok >= 0 ? 16u : 0u;   // rows past the tile are zero-filled
+            }
+            const CUtensorMap* tm = T.m < 0 ? &tm_sh : &tm_kv;
+            const int wrow = (T.m < 0 ? 0 : T.m * 2 * p.H * p.d) + T.ct * BN;
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+                const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.ws, 1)) { ok = false; break; }
+                if (tid == 0) {
+                    mbar_arrive_expect_tx(full0 + 8 * s, B_BYTES);
+                    tma_load_2d(smem_u32(sB + s * B_BYTES), tm, full0 + 8 * s, kb * BK, wrow);
+                }
+                const uint32_t dstA = smem_u32(sA + s * A_BYTES);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = rsub + 16 * i;
+                    cp_async_16(dstA + r * 128 + ((c ^ (r & 7)) << 4), src[i] + kb * BK, nbytes[i]);
+                }
+                cp_async_commit();
+                if (it >= LAG) {
+                    cp_async_wait<LAG>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(full0 + 8 * ((it - LAG) % STAGES));
+                }
+            }
+        }
+        // drain: the last LAG stages still owe their arrival
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        for (uint32_t j = it >= LAG ? it - LAG : 0; j < it; ++j) mbar_arrive(full0 + 8 * (j % STAGES));
+        if (!ok && tid == 0) {
+            // weight tiles still in flight must land before the CTA exits
+            for (uint32_t j = it >= STAGES ? it - STAGES : 0; j < it; ++j)
+                mbar_wait_drain(full0 + 8 * (j % STAGES), (j / STAGES) & 1);
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------------- epilogue
+        const int e = warp - 4;                 // TMEM lanes 32e .. 32e+31
+        const int row_local = 32 * e + lane;
+        const int Hd = p.H * p.d;
+        uint32_t tc = 0;
+        for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+            Tile T;
+            if (!tile_at(p, t, T)) continue;
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!mbar_wait(tfull0 + 8 * acc, aph, abort_flag, p.ws, 2)) break;
+            tc_fence_after();
+            const int64_t row = T.r0 + row_local;
+            const bool live = row < T.r1;
+            const int col0 = T.ct * BN;
+            const int part = col0 / Hd, cc0 = col0 % Hd;
+            bf16* base;
+            bool norm;
+            if (T.m < 0) {
+                base = part == 0 ? p.q : part == 1 ? p.k_sh : p.v_sh;
+                norm = part < 2;
+            } else {
+                base = part == 0 ? p.k_p : p.v_p;
+                norm = part == 0;
+            }
+            bf16* orow = base + (live ? row : 0) * (int64_t)Hd + cc0;
+            const uint32_t taddr = tmem_base + ((uint32_t)(32 * e) << 16) + acc * BN;
+            for (int g = 0; g < BN; g += p.d) {
+                float sc = 1.f;
+                uint32_t r[32];
+                if (norm) {
+                    float ss = 0.f;
+                    for (int cc = 0; cc < p.d; cc += 32) {
+                        tmem_ld_x32(taddr + g + cc, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float v = __uint_as_float(r[i]);
+                            ss = fmaf(v, v, ss);
+                        }
+                    }
+                    sc = rsqrtf(ss + 1e-6f);
+                }
+                for (int cc = 0; cc < p.d; cc += 32) {
+                    tmem_ld_x32(taddr + g + cc, r);
+                    tmem_ld_wait();
+                    if (live) {
+                        uint4 out[4];
+                        uint32_t* o32 = reinterpret_cast<uint32_t*>(out);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * sc,
+                                                                      __uint_as_float(r[2 * i + 1]) * sc);
+                            o32[i] = *reinterpret_cast<uint32_t*>(&h2);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(orow + g + cc);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = out[i];
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(tempty0 + 8 * acc);
+            ++tc;
+        }
+    } else if (lane == 0) {
+        // ------------------------------------------------------ MMA issuer
+        uint32_t it = 0, tc = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+            Tile T;
+            if (!tile_at(p, t, T)) continue;
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1, abort_flag, p.ws, 3)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * BN;
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+                const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                if (!mbar_wait(full0 + 8 * s, ph, abort_flag, p.ws, 4)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(sA + s * A_BYTES), b0 = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+                for (int j = 0; j < BK / 16; ++j)
+                    umma_f16(d_tmem, desc_kmajor_sw128(a0 + 32 * j), desc_kmajor_sw128(b0 + 32 * j), IDESC,
+                             (kb | j) != 0);
+                umma_commit(empty0 + 8 * s);
+            }
+            if (!ok) break;
+            umma_commit(tfull0 + 8 * acc);
+            ++tc;
+        }
+        // every MMA this CTA issued has finished before TMEM is released
+        umma_commit(done_bar);
+        mbar_wait_drain(done_bar, 0);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// --------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// [rows, cols] bf16 row-major matrix, tiles of box_rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool device_is_sm100() {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+    return major == 10;
+}
+
+}  // namespace
+
+bool proj_tc_supported(const ProjArgs& a, int dt) {
+    if (dt != MOM_BF16 || a.n_tok <= 0) return false;
+    if ((a.H * a.d) % BN != 0 || a.D % BK != 0) return false;
+    return device_is_sm100() && encode_fn() != nullptr;
+}
+
+cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
+    const int Hd = a.H * a.d;
+    CUtensorMap tm_sh, tm_kv;
+    if (!make_map(&tm_sh, a.w_shared, (uint64_t)3 * Hd, a.D, BN)) return cudaErrorInvalidValue;
+    if (!make_map(&tm_kv, a.w_kv, (uint64_t)a.M * 2 * Hd, a.D, BN)) return cudaErrorInvalidValue;
+    TcParams p;
+    p.x = reinterpret_cast<const bf16*>(a.x);
+    p.perm = a.perm_token;
+    p.mem_offset = a.mem_offset;
+    p.q = reinterpret_cast<bf16*>(a.q);
+    p.k_sh = reinterpret_cast<bf16*>(a.k_sh);
+    p.v_sh = reinterpret_cast<bf16*>(a.v_sh);
+    p.k_p = reinterpret_cast<bf16*>(a.k_p);
+    p.v_p = reinterpret_cast<bf16*>(a.v_p);
+    p.n_tok = a.n_tok;
+    p.D = a.D; p.H = a.H; p.d = a.d; p.M = a.M; p.K = a.K;
+    p.sh_ct = 3 * Hd / BN;
+    p.rt_ct = 2 * Hd / BN;
+    p.sh_tiles = cdiv(a.n_tok, BM) * p.sh_ct;
+    p.n_tiles = p.sh_tiles + (cdiv(a.n_tok * a.K, BM) + a.M) * p.rt_ct;
+    p.ws = a.ws;
+
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t grid = p.n_tiles < sms ? p.n_tiles : sms;
+    proj_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, st>>>(tm_sh, tm_kv, p);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 }  // namespace mom

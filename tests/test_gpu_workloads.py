@@ -1,0 +1,109 @@
+"""Parity at full workload sizes, in the launch configuration the benchmark
+times: the 380M-shape layer (8 x 2048 tokens), its skewed-routing varlen
+variant, and the 1.3B-shape 16-memory layer.
+
+The GPU runs the whole batch.  What the oracle checks:
+* routing and the reordering on every token (cheap on the CPU), bit-exact
+  outside near ties;
+* projections on a seeded sample of tokens and reordered rows;
+* layer outputs and final states on whole sampled sequences (sequences are
+  independent, so the oracle runs one of them alone with the GPU's routing
+  imposed); for the 1.3B shape, the outputs of the first 384 tokens of a
+  sequence (a prefix of a causal recurrence is exact on its own).
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_memories_layer_b200 import synth
+from oracle import mom_oracle as orc
+from tests.gpu_helpers import TOL, max_abs_rel, run_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _routing_and_permute(w, p, res):
+    idx, gate, logits, near = orc.router_topk(p["x"], p["w_r"], p["b_r"], w.top_k)
+    keep = ~near
+    assert np.array_equal(res["idx"][keep], idx[keep])
+    assert max_abs_rel(res["gate"][keep], gate[keep]) < 1e-5
+    perm, row_of, offs, seg = orc.permute(res["idx"], w.n_mem, p["cu_seqlens"])
+    assert np.array_equal(res["perm"][:offs[-1]], perm)
+    assert np.array_equal(res["row_of"], row_of)
+    assert np.array_equal(res["seg_cu"], seg)
+    return int(near.sum())
+
+
+def _projections_sampled(w, p, res, n=256, seed=0):
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(w.n_tokens, n, replace=False))
+    q, k_sh, v_sh, beta, la = orc.shared_projections(p["x"][toks], p, w.heads, w.d_head)
+    tol = TOL[w.dtype]
+    assert max_abs_rel(res["q"][toks], q) < tol
+    assert max_abs_rel(res["k_sh"][toks], k_sh) < tol
+    assert max_abs_rel(res["v_sh"][toks], v_sh) < tol
+    assert max_abs_rel(res["beta"][toks], beta) < 1e-5
+    assert max_abs_rel(res["log_alpha"][toks], la) < 1e-5
+    offs = res["mem_offset"]
+    rows = np.sort(rng.choice(int(offs[-1]), n, replace=False))
+    mem = np.searchsorted(offs, rows, side="right") - 1
+    for m in np.unique(mem):
+        r = rows[mem == m]
+        km, vm = orc.memory_kv(p["x"][res["perm"][r]], p, int(m), w.heads, w.d_head)
+        assert max_abs_rel(res["k_p"][r], km) < tol
+        assert max_abs_rel(res["v_p"][r], vm) < tol
+
+
+def _sequence(w, p, res, s, max_tokens=None):
+    cu = p["cu_seqlens"]
+    t0, t1 = int(cu[s]), int(cu[s + 1])
+    full = max_tokens is None or t1 - t0 <= max_tokens
+    if not full:
+        t1 = t0 + max_tokens
+    ref = orc.mom_forward(p["x"][t0:t1], p, np.array([0, t1 - t0]), w.top_k, w.heads, w.d_head,
+                          forced_idx=res["idx"][t0:t1])
+    tol = TOL[w.dtype]
+    e = max_abs_rel(res["out"][t0:t1], ref["out"])
+    assert e < tol, ("out", s, e)
+    if full:
+        assert max_abs_rel(res["h_shared"][s], ref["h_shared"][0]) < tol
+        assert max_abs_rel(res["h_mem"][:, s], ref["h_mem"][:, 0]) < tol
+
+
+def test_mom380m_full_size():
+    w = synth.WORKLOADS["mom380m"]
+    p = synth.make_problem(w)
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _routing_and_permute(w, p, res)
+    _projections_sampled(w, p, res)
+    _sequence(w, p, res, s=5)
+
+
+def test_mom380m_skewed_varlen_full_size():
+    w = synth.WORKLOADS["mom380m_skew_varlen"]
+    p = synth.make_problem(w)
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _routing_and_permute(w, p, res)
+    # skewed routing: memory 0 carries far more rows than the others
+    counts = np.diff(res["mem_offset"])
+    assert counts[0] > 2 * counts[1:].max()
+    _projections_sampled(w, p, res, seed=1)
+    S = len(p["cu_seqlens"]) - 1
+    _sequence(w, p, res, s=S - 1)      # the last (clipped, shortest) sequence
+
+
+def test_mom1p3b_m16_full_size():
+    w = synth.WORKLOADS["mom1p3b_m16"]
+    p = synth.make_problem(w)
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _routing_and_permute(w, p, res)
+    _projections_sampled(w, p, res, n=128, seed=2)
+    _sequence(w, p, res, s=2, max_tokens=384)
