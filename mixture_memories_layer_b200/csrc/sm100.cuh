@@ -93,6 +93,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Contiguous global -> shared copy of `bytes` (multiple of 16, both
+// addresses 16-byte aligned), completing on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // -------------------------------------------------------------- cp.async --
 // 16-byte copy global -> shared; src_bytes = 0 fills the 16 bytes with zeros.
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -150,6 +158,20 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// The store counterpart: lane i writes row (lane base + i), columns [col, col+32).
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // ----------------------------------------------------------- descriptors --
 // Shared-memory matrix descriptor (sm_100 format): start address, leading
 // and stride byte offsets (all >> 4), version 1, swizzle mode in bits 61..63
@@ -170,6 +192,18 @@ constexpr uint32_t kSwizzle128B = 2;
 // 1024 B stacked at stride 1024 B.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) {
     return smem_desc(addr, 16, 1024, kSwizzle128B);
+}
+// MN-major operand, 128-byte swizzle: 64 MN-contiguous bf16 per 128-byte
+// row, one row per K index; 8-row (K) atoms at stride 1024 B; successive
+// groups of 64 along MN at stride `mn_group_bytes`.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t addr, uint32_t mn_group_bytes) {
+    return smem_desc(addr, mn_group_bytes, 1024, kSwizzle128B);
+}
+
+// Byte offset of element (row, col) of a [rows x 64] bf16 tile stored with
+// the 128-byte swizzle (row pitch 128 B, 16-byte chunk index XOR row % 8).
+__host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
+    return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + (col & 7u) * 2u;
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
