@@ -70,8 +70,7 @@ def step_work(w):
         "router": {"bound": "hbm", "bytes": N * D * e + M * D * e + N * K * 8},
         "permute": {"bound": "hbm", "bytes": 2 * N * K * 4 + N * K * 8},
         "proj": {"bound": "tensor", "flops": 2 * N * D * (3 * H * d + 2 * H) + 2 * N * K * D * 2 * H * d},
-        "gdn_shared": {"bound": "tensor", "flops": 6 * N * H * d * d},
-        "gdn_routed": {"bound": "tensor", "flops": 6 * N * K * H * d * d},
+        "gdn": {"bound": "tensor", "flops": 6 * N * (1 + K) * H * d * d},
         "combine": {"bound": "hbm", "bytes": e * N * H * d * (2 + K) + N * K * 8},
     }
 
@@ -80,7 +79,7 @@ def layer_roofline(w, peaks):
     N, D, H, d, M, K = w.n_tokens, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k
     S = w.batch
     sw = step_work(w)
-    flops = sw["proj"]["flops"] + sw["gdn_shared"]["flops"] + sw["gdn_routed"]["flops"] \
+    flops = sw["proj"]["flops"] + sw["gdn"]["flops"] \
         + 2 * N * D * M + 2 * K * N * H * d
     weights = (M * D + 3 * H * d * D + 2 * H * D + M * 2 * H * d * D) * 2
     bytes_ = N * D * 2 + weights + N * H * d * 2 + (S + M * S) * H * d * d * 4 + N * K * 8
@@ -262,6 +261,16 @@ def gpu_arm(args):
     layer_roof = {"flops": lf, "bytes": lb, "roofline_ms": lt * 1e3, "frac": (lt * 1e3) / ms_per_step}
 
     # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks)
+    decode = None if args.no_decode else decode_bench(args, dev, world, rank, max_over_ranks, barrier)
+    clocks.__exit__(None, None, None)
+    return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode)
+
+
+def e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks):
+    import torch
     x_host = torch.empty(x.shape, dtype=dt, pin_memory=True)
     x_host.copy_(x.cpu())
     out_host = torch.empty((w.n_tokens, w.heads, w.d_head), dtype=dt, pin_memory=True)
@@ -278,14 +287,13 @@ def gpu_arm(args):
         e_ms.append(e0.elapsed_time(e1))
     e2e_ms = max_over_ranks(sum(e_ms[-args.steps:]) if args.steps else sum(e_ms))
     n_e2e = min(len(e_ms), args.steps) if args.steps else len(e_ms)
-    e2e = {"value": w.n_tokens * world * n_e2e / (e2e_ms / 1e3), "unit": UNIT,
-           "h2d_bytes_per_step": x.numel() * x.element_size(),
-           "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+    return {"value": w.n_tokens * world * n_e2e / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": x.numel() * x.element_size(),
+            "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
 
-    # ---- decode
-    decode = decode_bench(args, dev, world, rank, max_over_ranks, barrier)
-    clocks.__exit__(None, None, None)
 
+def finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode):
+    import torch.distributed as dist
     result = None
     if rank == 0:
         cpu = cpu_baseline(w) if (world == 1 and not args.no_cpu_baseline) else None
@@ -413,6 +421,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode timing")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -5,26 +5,27 @@
 // section: Gated DeltaNet's gate and update rule)
 //   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t
 // is evaluated in chunks of C = 64 rows.  With gamma_r the running sum of
-// log alpha inside the chunk and S the state at the chunk start:
-//   T   = (I + L)^-1,  L_rs = beta_r e^(gamma_r - gamma_s) k_r.k_s  (s < r)
-//   Y^T = [beta_s (v_s - e^(gamma_s) S k_s)]_s         (d_v x C)
-//   U^T = Y^T T^T                                      (u_r: the delta-rule corrections)
+// log alpha inside the chunk, S the state at the chunk start, and
+// Tb = (I + L)^-1 diag(beta), L_rs = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r):
+//   U^T = (V^T - Z~) Tb^T,        Z~ = (S K^T) diag(e^gamma)     (d_v x C)
 //   o_r = e^(gamma_r) S q_r + sum_{s<=r} e^(gamma_r-gamma_s) (q_r.k_s) u_s
 //   S'  = e^(gamma_C) S + sum_s e^(gamma_C-gamma_s) u_s k_s^T
-// All products are written so that the d_v rows of S are the MMA's M
+// where u_r = beta_r (v_r - alpha_r S_{r-1} k_r) are the delta-rule
+// corrections.  Every product keeps the d_v rows of S as the MMA's M
 // dimension (128 TMEM lanes): every MMA is M = 128.
 //
-// Three launches:
+// Three launches per call:
 //   schedule: chunk offsets of every segment (device-side, no host sync)
 //   prep    : per (chunk, head), independent of the state: G = [K;Q] K^T on
-//             the tensor cores, then T (forward substitution, fp32) and the
-//             causal decayed P = (Q K^T) o [e^(gamma_r-gamma_s)]_{s<=r}, both
-//             stored as pre-swizzled bf16 64x64 tiles
+//             the tensor cores; Tb by blocked (16 x 16) forward substitution
+//             in fp32; the causal decayed P = (Q K^T) o [e^(gamma_r-gamma_s)];
+//             both stored as pre-swizzled bf16 64 x 64 tiles
 //   state   : per (segment, head, 128-row d_v tile), the serial walk over the
-//             segment's chunks with warp-specialised roles (producers,
-//             one MMA thread, eight math warps), the state in TMEM.
-// Rows past a segment's end are zero-filled on load and masked in every
-// elementwise step, so a ragged tail chunk needs no padding.
+//             segment's chunks.  Roles: one producer warp (TMA loads, chunk
+//             gates), three gather warps (cp.async rows of q when it is read
+//             through an index), one MMA thread, eight math warps.
+// Rows past a segment's end are masked (zero gates, zeroed key/value rows),
+// so a ragged tail chunk needs no padding.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -37,7 +38,7 @@ using namespace sm100;
 constexpr int C = 64;                 // chunk length
 constexpr int DVT = 128;              // d_v rows per state CTA (TMEM lanes)
 constexpr int IMG = C * C * 2;        // one swizzled 64x64 bf16 tile
-constexpr int GB = 2 * C + 4;         // beta[64], gamma[64], n, e^gamma_last, gamma_last, pad
+constexpr int GB = 2 * C + 4;         // floats per chunk-gate record
 
 struct GdnTc {
     const bf16* q;
@@ -101,11 +102,13 @@ gdn_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_seg, int64_t n_row
     }
 }
 
-// Gates of one chunk, computed by one full warp: beta (0 past n), the running
-// sum gamma of log alpha, and e^gamma of the last valid row.  Both the prep
-// and the state kernel call this, so they agree bit for bit.
-__device__ __forceinline__ void chunk_gates(const GdnTc& p, int64_t r0, int n, int h, float* gb, int lane) {
-    float b[2], l[2];
+// Gates of one chunk, by one full warp (lane l holds rows 2l and 2l+1):
+// beta (0 past n) and gamma, the running sum of log alpha from the chunk
+// start.  Returns gamma of the last valid row.  Both the prep and the state
+// kernel derive their factors from this one scan, so they agree bit for bit.
+__device__ __forceinline__ float chunk_scan(const GdnTc& p, int64_t r0, int n, int h, int lane, float (&b)[2],
+                                            float (&g)[2]) {
+    float l[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int s = 2 * lane + e;
@@ -129,45 +132,83 @@ __device__ __forceinline__ void chunk_gates(const GdnTc& p, int64_t r0, int n, i
         const float t = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += t;
     }
-    const float g0 = incl - pair + l[0], g1 = incl;
-    gb[2 * lane] = b[0];
-    gb[2 * lane + 1] = b[1];
-    gb[C + 2 * lane] = g0;
-    gb[C + 2 * lane + 1] = g1;
+    g[0] = incl - pair + l[0];
+    g[1] = incl;
     const int last = n - 1;
-    const float gl = __shfl_sync(0xffffffffu, (last & 1) ? g1 : g0, last >> 1);
-    if (lane == 0) {
-        gb[2 * C] = __int_as_float(n);
-        gb[2 * C + 1] = expf(gl);
-        gb[2 * C + 2] = gl;
-    }
+    return __shfl_sync(0xffffffffu, (last & 1) ? g[1] : g[0], last >> 1);
 }
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
     return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h2);
+}
+
+// Gathers 64 rows x D of a bf16 [rows, H, D] array through an index (rows
+// past n and bad indices are zero-filled) into 128-byte-swizzled 64-column
+// slabs of `slab_stride` bytes; `nthreads` threads starting at `t0`.
+template <int D>
+__device__ __forceinline__ void gather_rows(const GdnTc& p, const bf16* base, int64_t r0, int n, int h,
+                                            uint32_t dst, uint32_t slab_stride, int t, int nthreads) {
+    for (int idx = t; idx < C * 8; idx += nthreads) {
+        const int row = idx >> 3, c8 = idx & 7;
+        int64_t src_row = -1;
+        if (row < n) {
+            const int64_t r = r0 + row;
+            const int64_t qr = p.qidx ? (int64_t)p.qidx[r] : r;
+            src_row = (qr >= 0 && qr < p.n_q_rows) ? qr : -1;
+        }
+        const bf16* src = base + ((src_row >= 0 ? src_row : 0) * p.H + h) * D + c8 * 8;
+        const uint32_t d0 = dst + row * 128 + ((c8 ^ (row & 7)) << 4);
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j) cp_async_16(d0 + j * slab_stride, src + j * 64, src_row >= 0 ? 16u : 0u);
+    }
+}
+
 // ----------------------------------------------------------------- prep --
 template <int D>
-constexpr size_t prep_smem() { return 1024 + (size_t)(D / 64) * 16384 + C * C * 4 + GB * 4 + 64; }
+struct PrepLayout {
+    static constexpr int SLABS = D / 64;
+    static constexpr int KQ = 0;                      // slab j: K rows 0..63 | Q rows 64..127 (16 KB)
+    static constexpr int TM = 0;                      // fp32 [64][64] T, reusing KQ after the MMA
+    static constexpr int LM = SLABS * 16384;          // fp32 [64][64] L
+    static constexpr int MB = LM + C * C * 4;         // fp32 3 x [16][16] block products
+    static constexpr int GBB = MB + 3 * 256 * 4;      // beta[64], gamma[64]
+    static constexpr int BARS = GBB + 2 * C * 4;      // land, mma
+    static constexpr int MISC = BARS + 16;
+    static constexpr size_t BYTES = 1024 + MISC + 16;
+};
 
 template <int D>
 __global__ void __launch_bounds__(128)
-gdn_prep_kernel(GdnTc p) {
+gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, GdnTc p) {
+    using Lay = PrepLayout<D>;
     constexpr int SLABS = D / 64;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* smem = align1024(smem_raw);
-    unsigned char* kq = smem;                              // slab j: K rows 0..63 | Q rows 64..127, 128 B each
-    float* Lm = reinterpret_cast<float*>(smem + SLABS * 16384);
-    float* gb = Lm + C * C;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(gb + GB);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+    unsigned char* sm = align1024(smem_raw);
+    float* Tm = reinterpret_cast<float*>(sm + Lay::TM);
+    float* Lm = reinterpret_cast<float*>(sm + Lay::LM);
+    float* Mb = reinterpret_cast<float*>(sm + Lay::MB);
+    float* gbeta = reinterpret_cast<float*>(sm + Lay::GBB);
+    float* ggam = gbeta + C;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::BARS);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lay::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+    const uint32_t land = smem_u32(bars), mma_bar = smem_u32(bars + 1);
+    const uint32_t kq = smem_u32(sm + Lay::KQ);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x, h = blockIdx.y;
     if (g >= p.chunk_cu[p.n_seg]) return;                 // uniform over the CTA
-    int lo = 0, hi = p.n_seg;                              // segment s with chunk_cu[s] <= g < chunk_cu[s+1]
+    int lo = 0, hi = p.n_seg;                              // segment with chunk_cu[s] <= g < chunk_cu[s+1]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (p.chunk_cu[mid] <= g) lo = mid; else hi = mid;
@@ -178,42 +219,40 @@ gdn_prep_kernel(GdnTc p) {
     const int n = (int)(rem < C ? rem : C);
 
     if (tid == 0) {
-        mbar_init(smem_u32(bar), 1);
+        mbar_init(land, 1);
+        mbar_init(mma_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    // K rows -> slab rows 0..63, Q rows (through qidx) -> 64..127; rows past n are zero
-    {
-        const int c8 = tid & 7;
+    __syncthreads();
+    // K (and contiguous Q) by TMA; rows past n hold other finite data and are masked below
+    if (tid == 0) {
+        mbar_arrive_expect_tx(land, SLABS * 8192 * (p.qidx ? 1 : 2));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int row = (tid >> 3) + 16 * i;
-            const int rr = row & 63;
-            const bool isq = row >= 64;
-            int64_t src_row = -1;
-            if (rr < n) {
-                const int64_t r = r0 + rr;
-                if (!isq) {
-                    src_row = r;
-                } else {
-                    const int64_t qr = p.qidx ? (int64_t)p.qidx[r] : r;
-                    src_row = (qr >= 0 && qr < p.n_q_rows) ? qr : -1;
-                }
-            }
-            const bf16* src = (isq ? p.q : p.k) + ((src_row >= 0 ? src_row : 0) * p.H + h) * D + c8 * 8;
-            const uint32_t dst = smem_u32(kq) + row * 128 + ((c8 ^ (row & 7)) << 4);
-#pragma unroll
-            for (int j = 0; j < SLABS; ++j) cp_async_16(dst + j * 16384, src + j * 64, src_row >= 0 ? 16u : 0u);
+        for (int j = 0; j < SLABS; ++j) {
+            tma_load_2d(kq + j * 16384, &tm_k, land, h * D + 64 * j, (int)r0);
+            if (!p.qidx) tma_load_2d(kq + j * 16384 + 8192, &tm_q, land, h * D + 64 * j, (int)r0);
         }
+    }
+    if (p.qidx) {
+        gather_rows<D>(p, p.q, r0, n, h, kq + 8192, 16384, tid, 128);
         cp_async_commit();
     }
-    if (warp == 0) chunk_gates(p, r0, n, h, gb, lane);
+    if (warp == 0) {
+        float b[2], gg[2];
+        chunk_scan(p, r0, n, h, lane, b, gg);
+        gbeta[2 * lane] = b[0]; gbeta[2 * lane + 1] = b[1];
+        ggam[2 * lane] = gg[0]; ggam[2 * lane + 1] = gg[1];
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(tslot), 64);
         tmem_relinquish();
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
+    if (p.qidx) {
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+    }
+    mbar_wait(land, 0, abort_flag, p.err, 10);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -226,13 +265,13 @@ gdn_prep_kernel(GdnTc p) {
         for (int j = 0; j < SLABS; ++j)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t a = smem_u32(kq + j * 16384) + kk * 32;
+                const uint32_t a = kq + j * 16384 + kk * 32;
                 umma_f16(tmem, desc_kmajor_sw128(a), desc_kmajor_sw128(a), ID, (j | kk) != 0);
             }
-        umma_commit(smem_u32(bar));
+        umma_commit(mma_bar);
     }
     __syncwarp();
-    mbar_wait(smem_u32(bar), 0, abort_flag, p.err, 10);
+    mbar_wait(mma_bar, 0, abort_flag, p.err, 11);
     tc_fence_after();
     uint32_t ga[32], gc[32];
     const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
@@ -242,20 +281,18 @@ gdn_prep_kernel(GdnTc p) {
 
     unsigned char* img = p.img + ((size_t)g * p.H + h) * 2 * IMG;
     const int r = tid & 63;
-    const float gr = gb[C + r], br = gb[r];
+    const float gr = ggam[r];
     if (tid < 64) {
-        // L row r (strictly lower, rows and columns past n are zero)
+        // L row r: strictly lower, zero in rows and columns past n
+        const float br = gbeta[r];
 #pragma unroll
         for (int s = 0; s < C; ++s) {
             float val = 0.f;
-            if (s < r && r < n) {
-                const float G = __uint_as_float(s < 32 ? ga[s] : gc[s - 32]);
-                val = br * expf(gr - gb[C + s]) * G;
-            }
+            if (s < r && r < n) val = br * __expf(gr - ggam[s]) * __uint_as_float(s < 32 ? ga[s] : gc[s - 32]);
             Lm[r * C + s] = val;
         }
     } else {
-        // P row r = causal, decayed q_r . k_s, bf16, swizzled image
+        // P row r: causal, decayed q_r . k_s, bf16 swizzled image
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
             uint32_t w[4];
@@ -266,13 +303,9 @@ gdn_prep_kernel(GdnTc p) {
                 for (int e = 0; e < 2; ++e) {
                     const int s = c8 * 8 + e2 * 2 + e;
                     pv[e] = 0.f;
-                    if (s <= r && r < n) {
-                        const float G = __uint_as_float(s < 32 ? ga[s] : gc[s - 32]);
-                        pv[e] = expf(gr - gb[C + s]) * G;
-                    }
+                    if (s <= r && r < n) pv[e] = __expf(gr - ggam[s]) * __uint_as_float(s < 32 ? ga[s] : gc[s - 32]);
                 }
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(pv[0], pv[1]);
-                w[e2] = *reinterpret_cast<uint32_t*>(&h2);
+                w[e2] = pack_bf16(pv[0], pv[1]);
             }
             *reinterpret_cast<uint4*>(img + IMG + r * 128 + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -283,38 +316,94 @@ gdn_prep_kernel(GdnTc p) {
         tc_fence_after();
         tmem_dealloc(tmem, 64);
     }
-    // T = (I + L)^-1 by forward substitution, one column per thread
+
+    // T = (I + L)^-1 in 16 x 16 blocks.  Diagonal blocks: forward substitution,
+    // one column per thread.
     if (tid < 64) {
-        const int j = tid;
-        float t[C];
+        const int bk = tid >> 4, cc = tid & 15, base = 16 * bk;
+        float t[16];
 #pragma unroll
-        for (int rr = 0; rr < C; ++rr) t[rr] = rr == j ? 1.f : 0.f;
+        for (int rl = 0; rl < 16; ++rl) t[rl] = rl == cc ? 1.f : 0.f;
 #pragma unroll
-        for (int rr = 1; rr < C; ++rr) {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            const float* Lr = Lm + rr * C;
+        for (int rl = 1; rl < 16; ++rl) {
+            float a0 = 0.f, a1 = 0.f;
+            const float* Lr = Lm + (base + rl) * C + base;
 #pragma unroll
-            for (int s = 0; s < rr; ++s) {
-                const float x = Lr[s] * t[s];
-                if ((s & 3) == 0) a0 += x; else if ((s & 3) == 1) a1 += x; else if ((s & 3) == 2) a2 += x; else a3 += x;
+            for (int sl = 0; sl < rl; ++sl) {
+                if (sl & 1) a1 = fmaf(Lr[sl], t[sl], a1); else a0 = fmaf(Lr[sl], t[sl], a0);
             }
-            if (rr > j) t[rr] = -((a0 + a1) + (a2 + a3));
+            if (rl > cc) t[rl] = -(a0 + a1);
         }
 #pragma unroll
-        for (int rr = 0; rr < C; ++rr)
-            *reinterpret_cast<bf16*>(img + sw128_offset(rr, j)) = __float2bfloat16_rn(t[rr]);
+        for (int rl = 0; rl < 16; ++rl) Tm[(base + rl) * C + base + cc] = t[rl];
+    }
+    __syncthreads();
+    // Off-diagonal blocks by distance from the diagonal:
+    //   T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj      (i > j)
+    for (int lev = 1; lev < 4; ++lev) {
+        const int nb = 4 - lev;
+        for (int e = tid; e < nb * 256; e += 128) {
+            const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
+            const int bi = lev + qb, bj = qb;
+            float acc = 0.f;
+            for (int bkk = bj; bkk < bi; ++bkk) {
+                const float* Lr = Lm + (16 * bi + a) * C + 16 * bkk;
+                const float* Tc = Tm + (16 * bkk) * C + 16 * bj + c;
+#pragma unroll
+                for (int s = 0; s < 16; ++s) acc = fmaf(Lr[s], Tc[s * C], acc);
+            }
+            Mb[qb * 256 + a * 16 + c] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nb * 256; e += 128) {
+            const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
+            const int bi = lev + qb, bj = qb;
+            const float* Tr = Tm + (16 * bi + a) * C + 16 * bi;
+            float acc = 0.f;
+#pragma unroll
+            for (int s = 0; s < 16; ++s) acc = fmaf(Tr[s], Mb[qb * 256 + s * 16 + c], acc);
+            Tm[(16 * bi + a) * C + 16 * bj + c] = -acc;
+        }
+        __syncthreads();
+    }
+    // Tb = T diag(beta): lower triangle (s <= r); beta is zero past n
+    {
+        const int half = tid >> 6;
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const int s = 32 * half + e;
+            const float v0 = s <= r ? Tm[r * C + s] * gbeta[s] : 0.f;
+            const float v1 = s + 1 <= r ? Tm[r * C + s + 1] * gbeta[s + 1] : 0.f;
+            w[e / 2] = pack_bf16(v0, v1);
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const int c8 = 4 * half + c4;
+            *reinterpret_cast<uint4*>(img + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+                make_uint4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+        }
     }
 }
 
 // ---------------------------------------------------------------- state --
 enum Bar {
-    GB_FULL = 0, GB_FREE = 2, K_FULL = 4, K_FREE = 6,
-    Q_FULL = 8, Q_FREE, V_FULL, V_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
-    SBF_READY, Z_FULL, X_FULL, Y_FULL, U_FULL, U_READY, S_FULL, O_FULL, XO_FREE, DONE, NBARS
+    GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, K_FREE = 8, X_FREE = 10,
+    V_LAND = 12, V_FULL, V_FREE, Q_FULL, Q_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
+    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, UO_FREE, DONE, NBARS
 };
 
-constexpr int NMATH = 8, NPROD = 4;                  // warps
-constexpr int STATE_THREADS = (NMATH + NPROD + 1) * 32;
+constexpr int NMATH = 8;              // math warps 0..7
+constexpr int W_PROD = 8;             // producer warp (TMA, gates, tail zeroing)
+constexpr int NGATHER = 3;            // gather warps 9..11 (indexed q rows)
+constexpr int W_MMA = 12;             // MMA warp
+constexpr int STATE_THREADS = 13 * 32;
+
+// gate record of one chunk, derived from chunk_scan
+constexpr int G_EG = 0;               // e^gamma_s (0 past n)
+constexpr int G_DEC = C;              // e^(gamma_last - gamma_s) (0 past n)
+constexpr int G_N = 2 * C;            // n (int bits)
+constexpr int G_EGC = 2 * C + 1;      // e^gamma_last
 
 template <int D>
 struct StateLayout {
@@ -323,12 +412,12 @@ struct StateLayout {
     static constexpr int K0 = S_BF + SLABS * 16384;           // 2 x [64 x D] bf16
     static constexpr int KSZ = SLABS * 8192;
     static constexpr int QB = K0 + 2 * KSZ;                   // [64 x D] bf16
-    static constexpr int VB = QB + KSZ;                       // [64 x 128] bf16, plain rows of 256 B
-    static constexpr int TB = VB + C * DVT * 2;               // T image
+    static constexpr int VB = QB + KSZ;                       // [64 x 128] bf16: two 64-column slabs
+    static constexpr int TB = VB + 2 * 8192;                  // Tb image
     static constexpr int PB = TB + IMG;                       // P image
-    static constexpr int YB = PB + IMG;                       // [128 x 64] bf16: Y, then U^T
-    static constexpr int UB = YB + 16384;                     // [128 x 64] bf16: decayed U^T
-    static constexpr int GBB = UB + 16384;                    // 2 x GB floats
+    static constexpr int ZB = PB + IMG;                       // [128 x 64] bf16: Z~, then U^T
+    static constexpr int UB = ZB + 16384;                     // [128 x 64] bf16: decayed U^T
+    static constexpr int GBB = UB + 16384;                    // 2 gate records
     static constexpr int BARS = GBB + 2 * GB * 4;
     static constexpr int MISC = BARS + NBARS * 8;
     static constexpr size_t BYTES = 1024 + MISC + 16;
@@ -336,11 +425,14 @@ struct StateLayout {
 
 template <int D>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
-gdn_state_kernel(GdnTc p) {
+gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_q, GdnTc p) {
     using Lay = StateLayout<D>;
     constexpr int SLABS = D / 64, NDV = D / DVT;
-    constexpr uint32_t T_S = 0, T_ZU = D, T_X = D + 64, T_O = D + 128;
+    // TMEM columns: state, Z, U then O, and two X buffers
+    constexpr uint32_t T_S = 0, T_Z = D, T_UO = D + 64, T_X = D + 128;
     constexpr uint32_t TMEM_COLS = 512;
+    static_assert(T_X + 128 <= TMEM_COLS, "TMEM budget");
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
@@ -349,9 +441,8 @@ gdn_state_kernel(GdnTc p) {
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const uint32_t s_bf = smem_u32(sm + Lay::S_BF), kb0 = smem_u32(sm + Lay::K0), qb = smem_u32(sm + Lay::QB);
-    const uint32_t timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB);
-    const uint32_t yb = smem_u32(sm + Lay::YB), ub = smem_u32(sm + Lay::UB);
-    const bf16* vbuf = reinterpret_cast<const bf16*>(sm + Lay::VB);
+    const uint32_t vb = smem_u32(sm + Lay::VB), timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB);
+    const uint32_t zb = smem_u32(sm + Lay::ZB), ub = smem_u32(sm + Lay::UB);
     float* gbuf = reinterpret_cast<float*>(sm + Lay::GBB);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -365,14 +456,17 @@ gdn_state_kernel(GdnTc p) {
     const int64_t rs1 = nc > 0 ? (int64_t)p.seg_cu[seg + 1] : 0;
 
     if (threadIdx.x == 0) {
-        const int counts[NBARS] = {1, 1, NMATH, NMATH, NPROD, NPROD, 1, 1,
-                                   NPROD, 1, NPROD, NMATH, 1, 1, 1, 1,
-                                   NMATH, 1, 1, NMATH, 1, NMATH, 1, 1, NMATH, 1};
+        int counts[NBARS];
+        for (int i = 0; i < NBARS; ++i) counts[i] = 1;
+        counts[GB_FREE] = counts[GB_FREE + 1] = NMATH;
+        counts[X_FREE] = counts[X_FREE + 1] = NMATH;
+        counts[SBF_READY] = counts[ZT_READY] = counts[U_READY] = counts[UO_FREE] = NMATH;
+        counts[Q_FULL] = p.qidx ? NGATHER : 1;
         for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), counts[i]);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == NMATH + NPROD) {
+    if (warp == W_MMA) {
         tmem_alloc(smem_u32(tslot), TMEM_COLS);
         tmem_relinquish();
     }
@@ -393,7 +487,7 @@ gdn_state_kernel(GdnTc p) {
             float sc = 1.f;
             if (nc > 0) {
                 ok = mbar_wait(bar(GB_FULL), 0, abort_flag, p.err, 20);
-                sc = gbuf[2 * C + 1];
+                sc = gbuf[G_EGC];
             }
             const float* hrow = p.h0 ? p.h0 + (((size_t)seg * p.H + h) * D + dv0 + i) * D : nullptr;
             for (int blk = 0; blk < HALF / 32 && ok; ++blk) {
@@ -421,14 +515,9 @@ gdn_state_kernel(GdnTc p) {
                 for (int c8 = 0; c8 < 4; ++c8) {
                     uint32_t pk[4];
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[c8 * 8 + 2 * e2], v[c8 * 8 + 2 * e2 + 1]);
-                        pk[e2] = *reinterpret_cast<uint32_t*>(&h2);
-                    }
+                    for (int e2 = 0; e2 < 4; ++e2) pk[e2] = pack_bf16(v[c8 * 8 + 2 * e2], v[c8 * 8 + 2 * e2 + 1]);
                     const int cc = (col & 63) / 8 + c8;
-                    const uint32_t dst = s_bf + (col >> 6) * 16384 + i * 128 + ((cc ^ (i & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
-                                 "r"(pk[2]), "r"(pk[3]) : "memory");
+                    st_shared_v4(s_bf + (col >> 6) * 16384 + i * 128 + ((cc ^ (i & 7)) << 4), pk);
                 }
             }
             if (nc > 0) {
@@ -444,78 +533,52 @@ gdn_state_kernel(GdnTc p) {
             const float* gb = gbuf + b * GB;
             const uint32_t ph = c & 1;
             if (!mbar_wait(bar(GB_FULL + b), (c >> 1) & 1, abort_flag, p.err, 21)) break;
-            const int n = __float_as_int(gb[2 * C]);
+            const int n = __float_as_int(gb[G_N]);
             const int64_t r0 = rs0 + (int64_t)c * C;
-            // ---- Y^T = beta_s (v_s - e^gamma_s S k_s)
+            // ---- Z~ = (S K^T) diag(e^gamma) -> bf16 for the U MMA
             if (!mbar_wait(bar(Z_FULL), ph, abort_flag, p.err, 22)) break;
             tc_fence_after();
-            uint32_t z[32];
-            tmem_ld_x32(tmem + lb + T_ZU + hf * 32, z);
-            tmem_ld_wait();
-            if (!mbar_wait(bar(V_FULL), ph, abort_flag, p.err, 23)) break;
             {
+                uint32_t z[32];
+                tmem_ld_x32(tmem + lb + T_Z + hf * 32, z);
+                tmem_ld_wait();
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float y[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int s = hf * 32 + e + u;
-                        y[u] = 0.f;
-                        if (s < n)
-                            y[u] = gb[s] * (__bfloat162float(vbuf[s * DVT + i]) -
-                                            expf(gb[C + s]) * __uint_as_float(z[e + u]));
-                    }
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(y[0], y[1]);
-                    pk[e / 2] = *reinterpret_cast<uint32_t*>(&h2);
-                }
+                for (int e = 0; e < 32; e += 2)
+                    pk[e / 2] = pack_bf16(__uint_as_float(z[e]) * gb[G_EG + hf * 32 + e],
+                                          __uint_as_float(z[e + 1]) * gb[G_EG + hf * 32 + e + 1]);
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
                     const int cc = hf * 4 + c8;
-                    const uint32_t dst = yb + i * 128 + ((cc ^ (i & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(pk[4 * c8]),
-                                 "r"(pk[4 * c8 + 1]), "r"(pk[4 * c8 + 2]), "r"(pk[4 * c8 + 3]) : "memory");
+                    st_shared_v4(zb + i * 128 + ((cc ^ (i & 7)) << 4), pk + 4 * c8);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) { mbar_arrive(bar(Y_FULL)); mbar_arrive(bar(V_FREE)); }
+            if (lane == 0) mbar_arrive(bar(ZT_READY));
             // ---- U^T (for the output) and decayed U^T (for the state)
             if (!mbar_wait(bar(U_FULL), ph, abort_flag, p.err, 24)) break;
             tc_fence_after();
-            uint32_t u[32];
-            tmem_ld_x32(tmem + lb + T_ZU + hf * 32, u);
-            tmem_ld_wait();
             {
-                const float gC = gb[2 * C + 2];
+                uint32_t u[32];
+                tmem_ld_x32(tmem + lb + T_UO + hf * 32, u);
+                tmem_ld_wait();
                 uint32_t pu[16], pd[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    float a[2], dcy[2];
-#pragma unroll
-                    for (int w2 = 0; w2 < 2; ++w2) {
-                        const int s = hf * 32 + e + w2;
-                        a[w2] = 0.f;
-                        dcy[w2] = 0.f;
-                        if (s < n) {
-                            a[w2] = __uint_as_float(u[e + w2]);
-                            dcy[w2] = a[w2] * expf(gC - gb[C + s]);
-                        }
-                    }
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(a[0], a[1]);
-                    pu[e / 2] = *reinterpret_cast<uint32_t*>(&h2);
-                    __nv_bfloat162 d2 = __floats2bfloat162_rn(dcy[0], dcy[1]);
-                    pd[e / 2] = *reinterpret_cast<uint32_t*>(&d2);
+                    const int s = hf * 32 + e;
+                    const float a0 = s < n ? __uint_as_float(u[e]) : 0.f;
+                    const float a1 = s + 1 < n ? __uint_as_float(u[e + 1]) : 0.f;
+                    pu[e / 2] = pack_bf16(a0, a1);
+                    pd[e / 2] = pack_bf16(a0 * gb[G_DEC + s], a1 * gb[G_DEC + s + 1]);
                 }
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
                     const int cc = hf * 4 + c8;
                     const uint32_t off = i * 128 + ((cc ^ (i & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(yb + off), "r"(pu[4 * c8]),
-                                 "r"(pu[4 * c8 + 1]), "r"(pu[4 * c8 + 2]), "r"(pu[4 * c8 + 3]) : "memory");
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(ub + off), "r"(pd[4 * c8]),
-                                 "r"(pd[4 * c8 + 1]), "r"(pd[4 * c8 + 2]), "r"(pd[4 * c8 + 3]) : "memory");
+                    st_shared_v4(zb + off, pu + 4 * c8);
+                    st_shared_v4(ub + off, pd + 4 * c8);
                 }
             }
             fence_proxy_async_smem();
@@ -529,7 +592,7 @@ gdn_state_kernel(GdnTc p) {
             float sc = 1.f;
             if (!last) {
                 if (!mbar_wait(bar(GB_FULL + (b ^ 1)), ((c + 1) >> 1) & 1, abort_flag, p.err, 26)) break;
-                sc = gbuf[(b ^ 1) * GB + 2 * C + 1];
+                sc = gbuf[(b ^ 1) * GB + G_EGC];
             }
             for (int blk = 0; blk < HALF / 32; ++blk) {
                 const int col = hf * HALF + 32 * blk;
@@ -551,15 +614,10 @@ gdn_state_kernel(GdnTc p) {
                 for (int c8 = 0; c8 < 4; ++c8) {
                     uint32_t pk[4];
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(sv[c8 * 8 + 2 * e2]),
-                                                                  __uint_as_float(sv[c8 * 8 + 2 * e2 + 1]));
-                        pk[e2] = *reinterpret_cast<uint32_t*>(&h2);
-                    }
+                    for (int e2 = 0; e2 < 4; ++e2)
+                        pk[e2] = pack_bf16(__uint_as_float(sv[c8 * 8 + 2 * e2]), __uint_as_float(sv[c8 * 8 + 2 * e2 + 1]));
                     const int cc = (col & 63) / 8 + c8;
-                    const uint32_t dst = s_bf + (col >> 6) * 16384 + i * 128 + ((cc ^ (i & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
-                                 "r"(pk[2]), "r"(pk[3]) : "memory");
+                    st_shared_v4(s_bf + (col >> 6) * 16384 + i * 128 + ((cc ^ (i & 7)) << 4), pk);
                 }
 #pragma unroll
                 for (int e = 0; e < 32; ++e) sv[e] = __float_as_uint(__uint_as_float(sv[e]) * sc);
@@ -575,160 +633,200 @@ gdn_state_kernel(GdnTc p) {
             // ---- output o_r = scale (e^gamma_r S q_r + sum_s P_rs u_s)
             if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 27)) break;
             tc_fence_after();
-            uint32_t xr[32], orr[32];
-            tmem_ld_x32(tmem + lb + T_X + hf * 32, xr);
-            tmem_ld_x32(tmem + lb + T_O + hf * 32, orr);
-            tmem_ld_wait();
+            {
+                uint32_t xr[32], orr[32];
+                tmem_ld_x32(tmem + lb + T_X + b * 64 + hf * 32, xr);
+                tmem_ld_x32(tmem + lb + T_UO + hf * 32, orr);
+                tmem_ld_wait();
+                bf16* orow = p.o + (r0 * p.H + h) * D + dv0 + i;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int r = hf * 32 + e;
-                if (r < n) {
-                    const float val = p.scale * fmaf(expf(gb[C + r]), __uint_as_float(xr[e]), __uint_as_float(orr[e]));
-                    p.o[((r0 + r) * p.H + h) * D + dv0 + i] = __float2bfloat16_rn(val);
+                for (int e = 0; e < 32; ++e) {
+                    const int r = hf * 32 + e;
+                    if (r < n)
+                        orow[(int64_t)r * p.H * D] = __float2bfloat16_rn(
+                            p.scale * fmaf(gb[G_EG + r], __uint_as_float(xr[e]), __uint_as_float(orr[e])));
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) { mbar_arrive(bar(XO_FREE)); mbar_arrive(bar(GB_FREE + b)); }
+            if (lane == 0) {
+                mbar_arrive(bar(UO_FREE));
+                mbar_arrive(bar(X_FREE + b));
+                mbar_arrive(bar(GB_FREE + b));
+            }
         }
-    } else if (warp < NMATH + NPROD) {
-        // ------------------------------------------------------ producers
-        const int pw = warp - NMATH;
-        const int pt = threadIdx.x - NMATH * 32;   // 0..127
+    } else if (warp == W_PROD) {
+        // ------------------------------------------ producer: gates + TMA
         bool ok = true;
-        int last_t = -1, last_p = -1;   // chunks whose T / P tiles were last requested
+        int last_k[2] = {-1, -1}, last_v = -1, last_q = -1, last_t = -1, last_p = -1;
         for (int c = 0; c < nc && ok; ++c) {
             const int b = c & 1;
-            const uint32_t ph = c & 1;
+            const uint32_t ph = c & 1, pb = (c >> 1) & 1;
             const int64_t r0 = rs0 + (int64_t)c * C;
             const int64_t rem = rs1 - r0;
             const int n = (int)(rem < C ? rem : C);
-            if (pw == 0) {
-                if (!mbar_wait(bar(GB_FREE + b), ((c >> 1) & 1) ^ 1, abort_flag, p.err, 30)) { ok = false; break; }
-                chunk_gates(p, r0, n, h, gbuf + b * GB, lane);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(GB_FULL + b));
-            }
-            const int c8 = pt & 7;
-            // K rows (zero past n)
-            if (!mbar_wait(bar(K_FREE + b), ((c >> 1) & 1) ^ 1, abort_flag, p.err, 31)) { ok = false; break; }
+            // gates
+            if (!mbar_wait(bar(GB_FREE + b), pb ^ 1, abort_flag, p.err, 30)) { ok = false; break; }
             {
-                const uint32_t kb = kb0 + b * Lay::KSZ;
+                float bt[2], gg[2];
+                const float gl = chunk_scan(p, r0, n, h, lane, bt, gg);
+                float* gb = gbuf + b * GB;
 #pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const int row = (pt >> 3) + 16 * i4;
-                    const bool valid = row < n;
-                    const bf16* src = p.k + ((r0 + (valid ? row : 0)) * p.H + h) * D + c8 * 8;
-                    const uint32_t dst = kb + row * 128 + ((c8 ^ (row & 7)) << 4);
-#pragma unroll
-                    for (int j = 0; j < SLABS; ++j) cp_async_16(dst + j * 8192, src + j * 64, valid ? 16u : 0u);
+                for (int e = 0; e < 2; ++e) {
+                    const int s = 2 * lane + e;
+                    gb[G_EG + s] = s < n ? __expf(gg[e]) : 0.f;
+                    gb[G_DEC + s] = s < n ? __expf(gl - gg[e]) : 0.f;
                 }
-                cp_async_commit();
-            }
-            // Q rows through qidx
-            if (!mbar_wait(bar(Q_FREE), ph ^ 1, abort_flag, p.err, 32)) { ok = false; break; }
-            {
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const int row = (pt >> 3) + 16 * i4;
-                    int64_t qr = -1;
-                    if (row < n) {
-                        const int64_t r = r0 + row;
-                        qr = p.qidx ? (int64_t)p.qidx[r] : r;
-                        if (qr < 0 || qr >= p.n_q_rows) qr = -1;
-                    }
-                    const bf16* src = p.q + ((qr >= 0 ? qr : 0) * p.H + h) * D + c8 * 8;
-                    const uint32_t dst = qb + row * 128 + ((c8 ^ (row & 7)) << 4);
-#pragma unroll
-                    for (int j = 0; j < SLABS; ++j) cp_async_16(dst + j * 8192, src + j * 64, qr >= 0 ? 16u : 0u);
+                if (lane == 0) {
+                    gb[G_N] = __int_as_float(n);
+                    gb[G_EGC] = __expf(gl);
                 }
-                cp_async_commit();
             }
-            // V rows, this CTA's 128 d_v columns, plain layout
-            if (!mbar_wait(bar(V_FREE), ph ^ 1, abort_flag, p.err, 33)) { ok = false; break; }
-            {
-                const int c16 = pt & 15;
-                const uint32_t vb = smem_u32(vbuf);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(GB_FULL + b));
+            // K, V (and contiguous Q) tiles
+            const uint32_t kb = kb0 + b * Lay::KSZ;
+            if (!mbar_wait(bar(K_FREE + b), pb ^ 1, abort_flag, p.err, 31)) { ok = false; break; }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(K_LAND + b), SLABS * 8192);
 #pragma unroll
-                for (int i8 = 0; i8 < 8; ++i8) {
-                    const int row = (pt >> 4) + 8 * i8;
-                    const bool valid = row < n;
-                    const bf16* src = p.v + ((r0 + (valid ? row : 0)) * p.H + h) * D + dv0 + c16 * 8;
-                    cp_async_16(vb + row * (DVT * 2) + c16 * 16, src, valid ? 16u : 0u);
-                }
-                cp_async_commit();
+                for (int j = 0; j < SLABS; ++j) tma_load_2d(kb + j * 8192, &tm_k, bar(K_LAND + b), h * D + 64 * j, (int)r0);
             }
-            cp_async_wait<2>();
-            fence_proxy_async_smem();
+            last_k[b] = c;
+            if (!mbar_wait(bar(V_FREE), ph ^ 1, abort_flag, p.err, 32)) { ok = false; break; }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(V_LAND), 16384);
+                tma_load_2d(vb, &tm_v, bar(V_LAND), h * D + dv0, (int)r0);
+                tma_load_2d(vb + 8192, &tm_v, bar(V_LAND), h * D + dv0 + 64, (int)r0);
+            }
+            last_v = c;
+            if (!p.qidx) {
+                if (!mbar_wait(bar(Q_FREE), ph ^ 1, abort_flag, p.err, 33)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(Q_FULL), SLABS * 8192);
+#pragma unroll
+                    for (int j = 0; j < SLABS; ++j) tma_load_2d(qb + j * 8192, &tm_q, bar(Q_FULL), h * D + 64 * j, (int)r0);
+                }
+                last_q = c;
+            }
+            // zero the key / value rows past n (other segments' data) once they land
+            if (!mbar_wait(bar(K_LAND + b), pb, abort_flag, p.err, 34)) { ok = false; break; }
+            if (n < C) {
+                const uint4 zero = make_uint4(0, 0, 0, 0);
+                for (int idx = lane; idx < (C - n) * 8 * SLABS; idx += 32) {
+                    const int row = n + idx / (8 * SLABS), rest = idx % (8 * SLABS);
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(kb + (rest >> 3) * 8192 + row * 128 + (rest & 7) * 16),
+                                 "r"(zero.x), "r"(zero.y), "r"(zero.z), "r"(zero.w) : "memory");
+                }
+                fence_proxy_async_smem();
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(K_FULL + b));
-            cp_async_wait<1>();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(Q_FULL));
-            cp_async_wait<0>();
+            if (!mbar_wait(bar(V_LAND), ph, abort_flag, p.err, 35)) { ok = false; break; }
+            if (n < C) {
+                for (int idx = lane; idx < (C - n) * 16; idx += 32) {
+                    const int row = n + idx / 16, rest = idx % 16;
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(vb + (rest >> 3) * 8192 + row * 128 + (rest & 7) * 16),
+                                 "r"(0u) : "memory");
+                }
+                fence_proxy_async_smem();
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(V_FULL));
-            if (pt == 0) {
-                const unsigned char* img = p.img + ((size_t)(c_base + c) * p.H + h) * 2 * IMG;
-                if (!mbar_wait(bar(T_FREE), ph ^ 1, abort_flag, p.err, 34)) { ok = false; break; }
+            // Tb and P tiles of this chunk
+            const unsigned char* img = p.img + ((size_t)(c_base + c) * p.H + h) * 2 * IMG;
+            if (!mbar_wait(bar(T_FREE), ph ^ 1, abort_flag, p.err, 36)) { ok = false; break; }
+            if (lane == 0) {
                 mbar_arrive_expect_tx(bar(T_FULL), IMG);
                 bulk_load(timg, img, IMG, bar(T_FULL));
-                last_t = c;
-                if (!mbar_wait(bar(P_FREE), ph ^ 1, abort_flag, p.err, 35)) { ok = false; break; }
+            }
+            last_t = c;
+            if (!mbar_wait(bar(P_FREE), ph ^ 1, abort_flag, p.err, 37)) { ok = false; break; }
+            if (lane == 0) {
                 mbar_arrive_expect_tx(bar(P_FULL), IMG);
                 bulk_load(pimg, img + IMG, IMG, bar(P_FULL));
-                last_p = c;
             }
+            last_p = c;
         }
-        cp_async_wait<0>();
-        if (!ok && pt == 0) {
-            // bulk copies still in flight must land before the CTA exits
+        if (!ok && lane == 0) {
+            // copies still in flight must land before the CTA exits
+            for (int b = 0; b < 2; ++b)
+                if (last_k[b] >= 0) mbar_wait_drain(bar(K_LAND + b), (last_k[b] >> 1) & 1);
+            if (last_v >= 0) mbar_wait_drain(bar(V_LAND), last_v & 1);
+            if (last_q >= 0) mbar_wait_drain(bar(Q_FULL), last_q & 1);
             if (last_t >= 0) mbar_wait_drain(bar(T_FULL), last_t & 1);
             if (last_p >= 0) mbar_wait_drain(bar(P_FULL), last_p & 1);
+        }
+    } else if (warp < W_MMA) {
+        // -------------------------------- gather warps: q rows through qidx
+        if (p.qidx) {
+            const int t = threadIdx.x - (W_PROD + 1) * 32;
+            for (int c = 0; c < nc; ++c) {
+                const int64_t r0 = rs0 + (int64_t)c * C;
+                const int64_t rem = rs1 - r0;
+                const int n = (int)(rem < C ? rem : C);
+                if (!mbar_wait(bar(Q_FREE), (c & 1) ^ 1, abort_flag, p.err, 38)) break;
+                gather_rows<D>(p, p.q, r0, n, h, qb, 8192, t, NGATHER * 32);
+                cp_async_commit();
+                cp_async_wait<0>();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(Q_FULL));
+            }
+            cp_async_wait<0>();
         }
     } else if (lane == 0) {
         // ------------------------------------------------------ MMA issuer
         constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
-        constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);
+        constexpr uint32_t ID64_V = idesc_bf16_f32(128, 64, 1, 0);       // A = V^T (MN-major)
+        constexpr uint32_t ID64_NEG = idesc_bf16_f32(128, 64, 0, 0, 1);  // -A
+        constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);           // B = K (MN-major)
         for (int c = 0; c < nc; ++c) {
             const int b = c & 1;
-            const uint32_t ph = c & 1;
+            const uint32_t ph = c & 1, pb = (c >> 1) & 1;
             const uint32_t kb = kb0 + b * Lay::KSZ;
-            if (!mbar_wait(bar(K_FULL + b), (c >> 1) & 1, abort_flag, p.err, 40)) break;
-            if (!mbar_wait(bar(Q_FULL), ph, abort_flag, p.err, 41)) break;
-            if (!mbar_wait(bar(SBF_READY), ph, abort_flag, p.err, 42)) break;
-            if (!mbar_wait(bar(XO_FREE), ph ^ 1, abort_flag, p.err, 43)) break;
+            // Z = S K^T
+            if (!mbar_wait(bar(K_FULL + b), pb, abort_flag, p.err, 40)) break;
+            if (!mbar_wait(bar(SBF_READY), ph, abort_flag, p.err, 41)) break;
             tc_fence_after();
-            // Z = S K^T and X = S Q^T (K = D)
 #pragma unroll
             for (int j = 0; j < SLABS; ++j)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_ZU, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
+                    umma_f16(tmem + T_Z, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
                              desc_kmajor_sw128(kb + j * 8192 + kk * 32), ID64, (j | kk) != 0);
             umma_commit(bar(Z_FULL));
+            // X = S Q^T into this chunk's X buffer
+            if (!mbar_wait(bar(Q_FULL), ph, abort_flag, p.err, 42)) break;
+            if (!mbar_wait(bar(X_FREE + b), pb ^ 1, abort_flag, p.err, 43)) break;
+            tc_fence_after();
 #pragma unroll
             for (int j = 0; j < SLABS; ++j)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_X, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
+                    umma_f16(tmem + T_X + b * 64, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
                              desc_kmajor_sw128(qb + j * 8192 + kk * 32), ID64, (j | kk) != 0);
-            umma_commit(bar(X_FULL));
             umma_commit(bar(Q_FREE));
-            // U^T = Y^T T^T (K = C)
-            if (!mbar_wait(bar(Y_FULL), ph, abort_flag, p.err, 44)) break;
+            // U^T = V^T Tb^T - Z~ Tb^T
+            if (!mbar_wait(bar(V_FULL), ph, abort_flag, p.err, 44)) break;
             if (!mbar_wait(bar(T_FULL), ph, abort_flag, p.err, 45)) break;
+            if (!mbar_wait(bar(UO_FREE), ph ^ 1, abort_flag, p.err, 46)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_ZU, desc_kmajor_sw128(yb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64,
-                         kk != 0);
+                umma_f16(tmem + T_UO, desc_mnmajor_sw128(vb + kk * 2048, 8192), desc_kmajor_sw128(timg + kk * 32),
+                         ID64_V, kk != 0);
+            umma_commit(bar(V_FREE));
+            if (!mbar_wait(bar(ZT_READY), ph, abort_flag, p.err, 47)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(tmem + T_UO, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64_NEG, 1);
             umma_commit(bar(U_FULL));
             umma_commit(bar(T_FREE));
-            // S += (decayed U^T) K  (B = K tile, MN-major) ; O = U^T P^T
-            if (!mbar_wait(bar(U_READY), ph, abort_flag, p.err, 46)) break;
-            if (!mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 47)) break;
+            // S += (decayed U^T) K ; O = U^T P^T
+            if (!mbar_wait(bar(U_READY), ph, abort_flag, p.err, 48)) break;
+            if (!mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 49)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -738,7 +836,7 @@ gdn_state_kernel(GdnTc p) {
             umma_commit(bar(K_FREE + b));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_O, desc_kmajor_sw128(yb + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64,
+                umma_f16(tmem + T_UO, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64,
                          kk != 0);
             umma_commit(bar(O_FULL));
             umma_commit(bar(P_FREE));
@@ -749,17 +847,10 @@ gdn_state_kernel(GdnTc p) {
 
     tc_fence_before();
     __syncthreads();
-    if (warp == NMATH + NPROD) {
+    if (warp == W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-}
-
-bool device_is_sm100() {
-    int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
-    return major == 10;
 }
 
 int64_t max_chunks(int64_t n_rows, int n_seg) { return n_rows / C + n_seg; }
@@ -769,19 +860,25 @@ cudaError_t launch_d(const GdnTc& t, int64_t mchunks, cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)prep_smem<D>());
+                                             (int)PrepLayout<D>::BYTES);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(gdn_state_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)StateLayout<D>::BYTES);
         if (e != cudaSuccess) return e;
         attr = true;
     }
+    const int HD = t.H * D;
+    CUtensorMap tm_k, tm_v, tm_q;
+    if (!make_tma_2d_bf16(&tm_k, t.k, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
+    if (!make_tma_2d_bf16(&tm_v, t.v, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
+    if (!make_tma_2d_bf16(&tm_q, t.q, (uint64_t)t.n_q_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
     gdn_schedule_kernel<<<1, 1024, 0, st>>>(t.seg_cu, t.n_seg, t.n_rows, t.chunk_cu, t.err);
     if (mchunks > 0) {
         dim3 pg((unsigned)mchunks, t.H);
-        gdn_prep_kernel<D><<<pg, 128, prep_smem<D>(), st>>>(t);
+        gdn_prep_kernel<D><<<pg, 128, PrepLayout<D>::BYTES, st>>>(tm_k, tm_q, t);
     }
-    gdn_state_kernel<D><<<(unsigned)((int64_t)t.n_seg * t.H * (D / DVT)), STATE_THREADS, StateLayout<D>::BYTES, st>>>(t);
+    gdn_state_kernel<D><<<(unsigned)((int64_t)t.n_seg * t.H * (D / DVT)), STATE_THREADS, StateLayout<D>::BYTES, st>>>(
+        tm_k, tm_v, tm_q, t);
     count_launches(mchunks > 0 ? 3 : 2);
     return cudaGetLastError();
 }
@@ -790,8 +887,8 @@ cudaError_t launch_d(const GdnTc& t, int64_t mchunks, cudaStream_t st) {
 
 bool gdn_tc_supported(const GdnArgs& a, int dt) {
     if (dt != MOM_BF16 || (a.d != 128 && a.d != 256)) return false;
-    if (a.n_rows >= ((int64_t)1 << 31) / C) return false;
-    return device_is_sm100();
+    if (a.n_rows <= 0 || a.n_q_rows <= 0 || a.n_rows >= ((int64_t)1 << 31) / C) return false;
+    return device_is_sm100() && tma_available();
 }
 
 size_t gdn_tc_ws_bytes(int64_t n_rows, int n_seg, int H, int d) {

@@ -2,6 +2,7 @@
 // mom.h validates arguments and calls these; they only launch.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -10,6 +11,14 @@ namespace mom {
 
 // Counts every kernel launch (mom_launch_count).
 void count_launches(int n);
+
+// tma_host.cu: tensor maps for bf16 row-major matrices (128-byte swizzle,
+// boxes of box_rows x box_cols with box_cols * 2 == 128 bytes) and the
+// device-generation check of the tcgen05 paths.
+bool tma_available();
+bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t row_pitch_elems,
+                      uint32_t box_cols, uint32_t box_rows);
+bool device_is_sm100();
 
 // router.cu
 cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int dt, int64_t n_tok, int D,

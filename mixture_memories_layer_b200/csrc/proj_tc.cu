@@ -21,8 +21,6 @@
 //              overlapping the next tile's main loop
 // Every wait is bounded (sm100.cuh); on a timeout the CTA records
 // MOM_DEVERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -293,54 +291,19 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
     }
 }
 
-// --------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// [rows, cols] bf16 row-major matrix, tiles of box_rows x 64 columns, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool device_is_sm100() {
-    int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
-    return major == 10;
-}
-
 }  // namespace
 
 bool proj_tc_supported(const ProjArgs& a, int dt) {
     if (dt != MOM_BF16 || a.n_tok <= 0) return false;
     if ((a.H * a.d) % BN != 0 || a.D % BK != 0) return false;
-    return device_is_sm100() && encode_fn() != nullptr;
+    return device_is_sm100() && tma_available();
 }
 
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     const int Hd = a.H * a.d;
     CUtensorMap tm_sh, tm_kv;
-    if (!make_map(&tm_sh, a.w_shared, (uint64_t)3 * Hd, a.D, BN)) return cudaErrorInvalidValue;
-    if (!make_map(&tm_kv, a.w_kv, (uint64_t)a.M * 2 * Hd, a.D, BN)) return cudaErrorInvalidValue;
+    if (!make_tma_2d_bf16(&tm_sh, a.w_shared, (uint64_t)3 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
+    if (!make_tma_2d_bf16(&tm_kv, a.w_kv, (uint64_t)a.M * 2 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
     TcParams p;
     p.x = reinterpret_cast<const bf16*>(a.x);
     p.perm = a.perm_token;

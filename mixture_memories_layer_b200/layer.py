@@ -92,41 +92,55 @@ class MoMLayer:
         return b
 
     # -------------------------------------------------------------- forward
-    STEPS = ("router", "permute", "proj", "gdn_shared", "gdn_routed", "combine")
+    STEPS = ("router", "permute", "proj", "gdn", "combine")
 
     def forward(self, x: torch.Tensor, cu_seqlens: torch.Tensor, h0_shared=None, h0_mem=None,
                 want_states: bool = True, stream=None, marks=None) -> Dict[str, torch.Tensor]:
         """x [N, d_model] (device), cu_seqlens [S+1] int32 (device).  Returns
         the buffers dict; ``out`` is the layer output, ``h_shared`` [S,H,d,d]
         and ``h_mem`` [M,S,H,d,d] the final states.  ``marks``: optional list
-        of 7 CUDA events, recorded before the first call and after each of
-        the six (per-step timing on the launching stream)."""
+        of 6 CUDA events, recorded before the first call and after each step
+        of STEPS (per-step timing on the launching stream).  The shared and
+        the routed recurrences are independent: the shared one runs on a side
+        stream joined back before the combine."""
         n_tok = x.shape[0]
         n_seq = cu_seqlens.numel() - 1
         w, b = self.w, self.buffers(n_tok, n_seq)
         st = stream if stream is not None else torch.cuda.current_stream()
         mark = (lambda i: marks[i].record(st)) if marks is not None else (lambda i: None)
         mark(0)
-        B.mom_router_topk(x, w["w_r"], w["b_r"], self.top_k, b["idx"], b["gate"], stream=stream)
+        B.mom_router_topk(x, w["w_r"], w["b_r"], self.top_k, b["idx"], b["gate"], stream=st)
         mark(1)
         B.mom_permute(b["idx"], self.n_mem, cu_seqlens, b["perm"], b["row_of"], b["mem_offset"], b["seg_cu"],
-                      b["ws_perm"], stream=stream)
+                      b["ws_perm"], stream=st)
         mark(2)
         B.mom_kv_proj_grouped(x, b["perm"], b["mem_offset"], w["w_shared"], w["w_gate"], w["A"], w["b_a"],
                               w["w_kv"], self.H, self.d, self.top_k, b["q"], b["k_sh"], b["v_sh"], b["beta"],
-                              b["log_alpha"], b["k_p"], b["v_p"], b["ws_proj"], stream=stream)
+                              b["log_alpha"], b["k_p"], b["v_p"], b["ws_proj"], stream=st)
         mark(3)
         hs = b["h_shared"] if want_states else None
         hm = b["h_mem"] if want_states else None
+        side = self._side_stream()
+        fork = torch.cuda.Event()
+        fork.record(st)
+        side.wait_event(fork)
         B.mom_gdn_chunk_fwd(b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens,
-                            self.scale, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"], stream=stream)
-        mark(4)
+                            self.scale, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"], stream=side)
         B.mom_gdn_chunk_fwd(b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
-                            self.scale, h0_mem, hm, b["o_p"], b["ws_gdn_p"], stream=stream)
+                            self.scale, h0_mem, hm, b["o_p"], b["ws_gdn_p"], stream=st)
+        join = torch.cuda.Event()
+        join.record(side)
+        st.wait_event(join)
+        mark(4)
+        B.mom_combine_unpermute(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["out"], b["ws_comb"], stream=st)
         mark(5)
-        B.mom_combine_unpermute(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["out"], b["ws_comb"], stream=stream)
-        mark(6)
         return b
+
+    def _side_stream(self):
+        s = getattr(self, "_side", None)
+        if s is None:
+            s = self._side = torch.cuda.Stream(device=self.device)
+        return s
 
     def device_errors(self):
         """(code, info) of every workspace with a recorded violation."""
