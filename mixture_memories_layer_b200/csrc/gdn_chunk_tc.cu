@@ -56,6 +56,7 @@ struct GdnTc {
     float* h_final;
     bf16* o;
     int32_t* chunk_cu;
+    int4* chunk_info;     // per chunk: segment, first row, rows (<= C)
     unsigned char* img;
     void* err;
 };
@@ -63,7 +64,7 @@ struct GdnTc {
 // ------------------------------------------------------------- schedule --
 __global__ void __launch_bounds__(1024)
 gdn_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_seg, int64_t n_rows, int32_t* __restrict__ chunk_cu,
-                    void* err) {
+                    int4* __restrict__ chunk_info, void* err) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     if (threadIdx.x == 0) { carry = 0; chunk_cu[0] = 0; }
@@ -99,6 +100,15 @@ gdn_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_seg, int64_t n_row
         __syncthreads();
         if (threadIdx.x == 0) carry += warp_tot[31];
         __syncthreads();
+    }
+    // every chunk's segment, first row and length (chunk_cu is visible to the CTA after the barrier)
+    for (int s = threadIdx.x; s < n_seg; s += 1024) {
+        const int c0 = chunk_cu[s], c1 = chunk_cu[s + 1];
+        const int a = seg_cu[s], b = seg_cu[s + 1];
+        for (int c = c0; c < c1; ++c) {
+            const int r0 = a + (c - c0) * C;
+            chunk_info[c] = make_int4(s, r0, b - r0 < C ? b - r0 : C, 0);
+        }
     }
 }
 
@@ -147,6 +157,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* v) {
                  : "memory");
 }
 
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, float* v) {
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(addr));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h2);
@@ -176,13 +190,12 @@ __device__ __forceinline__ void gather_rows(const GdnTc& p, const bf16* base, in
 // ----------------------------------------------------------------- prep --
 template <int D>
 struct PrepLayout {
-    static constexpr int SLABS = D / 64;
-    static constexpr int KQ = 0;                      // slab j: K rows 0..63 | Q rows 64..127 (16 KB)
-    static constexpr int TM = 0;                      // fp32 [64][64] T, reusing KQ after the MMA
-    static constexpr int LM = SLABS * 16384;          // fp32 [64][64] L
+    static constexpr int KQ = 0;                      // two slabs: K rows 0..63 | Q rows 64..127 (16 KB each)
+    static constexpr int TM = 0;                      // fp32 [64][64] T, reusing KQ after the MMAs
+    static constexpr int LM = 2 * 16384;              // fp32 [64][64] L
     static constexpr int MB = LM + C * C * 4;         // fp32 3 x [16][16] block products
     static constexpr int GBB = MB + 3 * 256 * 4;      // beta[64], gamma[64]
-    static constexpr int BARS = GBB + 2 * C * 4;      // land, mma
+    static constexpr int BARS = GBB + 2 * C * 4;      // land, mma (one phase per pair of slabs)
     static constexpr int MISC = BARS + 16;
     static constexpr size_t BYTES = 1024 + MISC + 16;
 };
@@ -208,35 +221,15 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x, h = blockIdx.y;
     if (g >= p.chunk_cu[p.n_seg]) return;                 // uniform over the CTA
-    int lo = 0, hi = p.n_seg;                              // segment with chunk_cu[s] <= g < chunk_cu[s+1]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (p.chunk_cu[mid] <= g) lo = mid; else hi = mid;
-    }
-    const int seg = lo;
-    const int64_t r0 = p.seg_cu[seg] + (int64_t)(g - p.chunk_cu[seg]) * C;
-    const int64_t rem = p.seg_cu[seg + 1] - r0;
-    const int n = (int)(rem < C ? rem : C);
+    const int4 info = p.chunk_info[g];
+    const int64_t r0 = info.y;
+    const int n = info.z;
 
     if (tid == 0) {
         mbar_init(land, 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
-    }
-    __syncthreads();
-    // K (and contiguous Q) by TMA; rows past n hold other finite data and are masked below
-    if (tid == 0) {
-        mbar_arrive_expect_tx(land, SLABS * 8192 * (p.qidx ? 1 : 2));
-#pragma unroll
-        for (int j = 0; j < SLABS; ++j) {
-            tma_load_2d(kq + j * 16384, &tm_k, land, h * D + 64 * j, (int)r0);
-            if (!p.qidx) tma_load_2d(kq + j * 16384 + 8192, &tm_q, land, h * D + 64 * j, (int)r0);
-        }
-    }
-    if (p.qidx) {
-        gather_rows<D>(p, p.q, r0, n, h, kq + 8192, 16384, tid, 128);
-        cp_async_commit();
     }
     if (warp == 0) {
         float b[2], gg[2];
@@ -248,31 +241,56 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tmem_alloc(smem_u32(tslot), 64);
         tmem_relinquish();
     }
-    if (p.qidx) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-    }
-    mbar_wait(land, 0, abort_flag, p.err, 10);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    // G = [K; Q] K^T : M = 128, N = 64, K = D
-    if (tid == 0) {
-        constexpr uint32_t ID = idesc_bf16_f32(128, 64);
-#pragma unroll
-        for (int j = 0; j < SLABS; ++j)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t a = kq + j * 16384 + kk * 32;
-                umma_f16(tmem, desc_kmajor_sw128(a), desc_kmajor_sw128(a), ID, (j | kk) != 0);
+    // G = [K; Q] K^T : M = 128, N = 64, K = D, two slabs (128 columns of D) per phase.
+    // K (and contiguous Q) by TMA; rows past n hold other finite data and are masked below.
+    constexpr int NPH = SLABS / 2 > 0 ? SLABS / 2 : 1;
+    for (int ph = 0; ph < NPH; ++ph) {
+        const int j0 = 2 * ph, nj = SLABS - j0 < 2 ? SLABS - j0 : 2;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(land, nj * 8192 * (p.qidx ? 1 : 2));
+            for (int jj = 0; jj < nj; ++jj) {
+                tma_load_2d(kq + jj * 16384, &tm_k, land, h * D + 64 * (j0 + jj), (int)r0);
+                if (!p.qidx) tma_load_2d(kq + jj * 16384 + 8192, &tm_q, land, h * D + 64 * (j0 + jj), (int)r0);
             }
-        umma_commit(mma_bar);
+        }
+        if (p.qidx) {
+            for (int idx = tid; idx < C * 8; idx += 128) {
+                const int row = idx >> 3, c8 = idx & 7;
+                int64_t src_row = -1;
+                if (row < n) {
+                    const int64_t qr = p.qidx[r0 + row];
+                    src_row = (qr >= 0 && qr < p.n_q_rows) ? qr : -1;
+                }
+                const bf16* src = p.q + ((src_row >= 0 ? src_row : 0) * p.H + h) * D + j0 * 64 + c8 * 8;
+                const uint32_t d0 = kq + 8192 + row * 128 + ((c8 ^ (row & 7)) << 4);
+                for (int jj = 0; jj < nj; ++jj) cp_async_16(d0 + jj * 16384, src + jj * 64, src_row >= 0 ? 16u : 0u);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+        }
+        mbar_wait(land, ph & 1, abort_flag, p.err, 10);
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t ID = idesc_bf16_f32(128, 64);
+            for (int jj = 0; jj < nj; ++jj)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t a = kq + jj * 16384 + kk * 32;
+                    umma_f16(tmem, desc_kmajor_sw128(a), desc_kmajor_sw128(a), ID, (ph | jj | kk) != 0);
+                }
+            umma_commit(mma_bar);
+        }
+        __syncwarp();
+        mbar_wait(mma_bar, ph & 1, abort_flag, p.err, 11);   // the buffer is free again
+        tc_fence_after();
     }
-    __syncwarp();
-    mbar_wait(mma_bar, 0, abort_flag, p.err, 11);
-    tc_fence_after();
     uint32_t ga[32], gc[32];
     const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
     tmem_ld_x32(taddr, ga);
@@ -388,9 +406,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 // ---------------------------------------------------------------- state --
 enum Bar {
-    GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, K_FREE = 8, X_FREE = 10,
+    GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, K_FREE = 8, UO_FREE = 10,
     V_LAND = 12, V_FULL, V_FREE, Q_FULL, Q_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
-    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, UO_FREE, DONE, NBARS
+    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, X_FREE, DONE, NBARS
 };
 
 constexpr int NMATH = 8;              // math warps 0..7
@@ -426,13 +444,13 @@ struct StateLayout {
 template <int D>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const __grid_constant__ CUtensorMap tm_q, GdnTc p) {
+                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, GdnTc p) {
     using Lay = StateLayout<D>;
     constexpr int SLABS = D / 64, NDV = D / DVT;
-    // TMEM columns: state, Z, U then O, and two X buffers
-    constexpr uint32_t T_S = 0, T_Z = D, T_UO = D + 64, T_X = D + 128;
+    // TMEM columns: state, Z, X, and two buffers each holding U then O
+    constexpr uint32_t T_S = 0, T_Z = D, T_X = D + 64, T_UO = D + 128;
     constexpr uint32_t TMEM_COLS = 512;
-    static_assert(T_X + 128 <= TMEM_COLS, "TMEM budget");
+    static_assert(T_UO + 128 <= TMEM_COLS, "TMEM budget");
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
@@ -459,8 +477,8 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int counts[NBARS];
         for (int i = 0; i < NBARS; ++i) counts[i] = 1;
         counts[GB_FREE] = counts[GB_FREE + 1] = NMATH;
-        counts[X_FREE] = counts[X_FREE + 1] = NMATH;
-        counts[SBF_READY] = counts[ZT_READY] = counts[U_READY] = counts[UO_FREE] = NMATH;
+        counts[UO_FREE] = counts[UO_FREE + 1] = NMATH;
+        counts[SBF_READY] = counts[ZT_READY] = counts[U_READY] = counts[X_FREE] = NMATH;
         counts[Q_FULL] = p.qidx ? NGATHER : 1;
         for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), counts[i]);
         *abort_flag = 0;
@@ -542,11 +560,13 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 uint32_t z[32];
                 tmem_ld_x32(tmem + lb + T_Z + hf * 32, z);
                 tmem_ld_wait();
+                float eg[32];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_EG + hf * 32 + e), eg + e);
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
-                    pk[e / 2] = pack_bf16(__uint_as_float(z[e]) * gb[G_EG + hf * 32 + e],
-                                          __uint_as_float(z[e + 1]) * gb[G_EG + hf * 32 + e + 1]);
+                    pk[e / 2] = pack_bf16(__uint_as_float(z[e]) * eg[e], __uint_as_float(z[e + 1]) * eg[e + 1]);
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
                     const int cc = hf * 4 + c8;
@@ -559,11 +579,19 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             if (lane == 0) mbar_arrive(bar(ZT_READY));
             // ---- U^T (for the output) and decayed U^T (for the state)
             if (!mbar_wait(bar(U_FULL), ph, abort_flag, p.err, 24)) break;
+            if (c > 0) {
+                // ub still holds the previous chunk's output tile until its TMA store has read it
+                if (warp == 0 && lane == 0) bulk_wait_read0();
+                named_sync(1, NMATH * 32);
+            }
             tc_fence_after();
             {
                 uint32_t u[32];
-                tmem_ld_x32(tmem + lb + T_UO + hf * 32, u);
+                tmem_ld_x32(tmem + lb + T_UO + b * 64 + hf * 32, u);
                 tmem_ld_wait();
+                float dc[32];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_DEC + hf * 32 + e), dc + e);
                 uint32_t pu[16], pd[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -571,7 +599,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     const float a0 = s < n ? __uint_as_float(u[e]) : 0.f;
                     const float a1 = s + 1 < n ? __uint_as_float(u[e + 1]) : 0.f;
                     pu[e / 2] = pack_bf16(a0, a1);
-                    pd[e / 2] = pack_bf16(a0 * gb[G_DEC + s], a1 * gb[G_DEC + s + 1]);
+                    pd[e / 2] = pack_bf16(a0 * dc[e], a1 * dc[e + 1]);
                 }
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
@@ -594,11 +622,15 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 if (!mbar_wait(bar(GB_FULL + (b ^ 1)), ((c + 1) >> 1) & 1, abort_flag, p.err, 26)) break;
                 sc = gbuf[(b ^ 1) * GB + G_EGC];
             }
-            for (int blk = 0; blk < HALF / 32; ++blk) {
-                const int col = hf * HALF + 32 * blk;
-                uint32_t sv[32];
-                tmem_ld_x32(tmem + lb + T_S + col, sv);
-                tmem_ld_wait();
+            for (int blk2 = 0; blk2 < HALF / 32; blk2 += 2) {
+              uint32_t svp[2][32];
+              tmem_ld_x32(tmem + lb + T_S + hf * HALF + 32 * blk2, svp[0]);
+              tmem_ld_x32(tmem + lb + T_S + hf * HALF + 32 * blk2 + 32, svp[1]);
+              tmem_ld_wait();
+#pragma unroll
+              for (int u2 = 0; u2 < 2; ++u2) {
+                const int col = hf * HALF + 32 * (blk2 + u2);
+                uint32_t* sv = svp[u2];
                 if (last) {
                     if (p.h_final) {
                         float* out = p.h_final + (((size_t)seg * p.H + h) * D + dv0 + i) * D + col;
@@ -621,7 +653,8 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
 #pragma unroll
                 for (int e = 0; e < 32; ++e) sv[e] = __float_as_uint(__uint_as_float(sv[e]) * sc);
-                tmem_st_x32(tmem + lb + T_S + col, sv);
+                tmem_st_x32(tmem + lb + T_S + col, svp[u2]);
+              }
             }
             if (!last) {
                 tmem_st_wait();
@@ -635,26 +668,50 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tc_fence_after();
             {
                 uint32_t xr[32], orr[32];
-                tmem_ld_x32(tmem + lb + T_X + b * 64 + hf * 32, xr);
-                tmem_ld_x32(tmem + lb + T_UO + hf * 32, orr);
+                tmem_ld_x32(tmem + lb + T_X + hf * 32, xr);
+                tmem_ld_x32(tmem + lb + T_UO + b * 64 + hf * 32, orr);
                 tmem_ld_wait();
-                bf16* orow = p.o + (r0 * p.H + h) * D + dv0 + i;
+                // stage the [64 rows x 128 d_v] output tile row-major in ub
+                const uint32_t stage = ub + i * 2;
+                float eg[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
+                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_EG + hf * 32 + e), eg + e);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
                     const int r = hf * 32 + e;
-                    if (r < n)
-                        orow[(int64_t)r * p.H * D] = __float2bfloat16_rn(
-                            p.scale * fmaf(gb[G_EG + r], __uint_as_float(xr[e]), __uint_as_float(orr[e])));
+                    const uint32_t pr = pack_bf16(
+                        p.scale * fmaf(eg[e], __uint_as_float(xr[e]), __uint_as_float(orr[e])),
+                        p.scale * fmaf(eg[e + 1], __uint_as_float(xr[e + 1]), __uint_as_float(orr[e + 1])));
+                    asm volatile("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                                 "st.shared.b16 [%0], lo;\n\tst.shared.b16 [%1], hi;\n\t}"
+                                 ::"r"(stage + r * DVT * 2), "r"(stage + (r + 1) * DVT * 2), "r"(pr) : "memory");
                 }
             }
             tc_fence_before();
+            fence_proxy_async_smem();
+            named_sync(1, NMATH * 32);
+            if (n == C) {
+                if (warp == 0 && lane == 0) {
+                    tma_store_2d(&tm_o, ub, h * D + dv0, (int)r0);
+                    bulk_commit();
+                }
+            } else {
+                // ragged last chunk: only rows < n belong to this segment
+                const int tid = threadIdx.x;
+                for (int idx = tid; idx < n * (DVT / 8); idx += NMATH * 32) {
+                    const int row = idx / (DVT / 8), ch = idx % (DVT / 8);
+                    const uint4 v = *reinterpret_cast<const uint4*>(sm + Lay::UB + row * DVT * 2 + ch * 16);
+                    *reinterpret_cast<uint4*>(p.o + ((r0 + row) * p.H + h) * D + dv0 + ch * 8) = v;
+                }
+            }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(bar(UO_FREE));
-                mbar_arrive(bar(X_FREE + b));
+                mbar_arrive(bar(UO_FREE + b));
+                mbar_arrive(bar(X_FREE));
                 mbar_arrive(bar(GB_FREE + b));
             }
         }
+        if (warp == 0 && lane == 0) bulk_wait0();
     } else if (warp == W_PROD) {
         // ------------------------------------------ producer: gates + TMA
         bool ok = true;
@@ -796,34 +853,35 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     umma_f16(tmem + T_Z, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
                              desc_kmajor_sw128(kb + j * 8192 + kk * 32), ID64, (j | kk) != 0);
             umma_commit(bar(Z_FULL));
-            // X = S Q^T into this chunk's X buffer
-            if (!mbar_wait(bar(Q_FULL), ph, abort_flag, p.err, 42)) break;
-            if (!mbar_wait(bar(X_FREE + b), pb ^ 1, abort_flag, p.err, 43)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < SLABS; ++j)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_X + b * 64, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
-                             desc_kmajor_sw128(qb + j * 8192 + kk * 32), ID64, (j | kk) != 0);
-            umma_commit(bar(Q_FREE));
-            // U^T = V^T Tb^T - Z~ Tb^T
+            // U^T = V^T Tb^T - Z~ Tb^T  into this chunk's U/O buffer
+            const uint32_t uo = tmem + T_UO + b * 64;
             if (!mbar_wait(bar(V_FULL), ph, abort_flag, p.err, 44)) break;
             if (!mbar_wait(bar(T_FULL), ph, abort_flag, p.err, 45)) break;
-            if (!mbar_wait(bar(UO_FREE), ph ^ 1, abort_flag, p.err, 46)) break;
+            if (!mbar_wait(bar(UO_FREE + b), pb ^ 1, abort_flag, p.err, 46)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_UO, desc_mnmajor_sw128(vb + kk * 2048, 8192), desc_kmajor_sw128(timg + kk * 32),
-                         ID64_V, kk != 0);
+                umma_f16(uo, desc_mnmajor_sw128(vb + kk * 2048, 8192), desc_kmajor_sw128(timg + kk * 32), ID64_V,
+                         kk != 0);
             umma_commit(bar(V_FREE));
             if (!mbar_wait(bar(ZT_READY), ph, abort_flag, p.err, 47)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_UO, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64_NEG, 1);
+                umma_f16(uo, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64_NEG, 1);
             umma_commit(bar(U_FULL));
             umma_commit(bar(T_FREE));
+            // X = S Q^T (only the output needs it: issued while the math warps write U)
+            if (!mbar_wait(bar(Q_FULL), ph, abort_flag, p.err, 42)) break;
+            if (!mbar_wait(bar(X_FREE), ph ^ 1, abort_flag, p.err, 43)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < SLABS; ++j)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + T_X, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
+                             desc_kmajor_sw128(qb + j * 8192 + kk * 32), ID64, (j | kk) != 0);
+            umma_commit(bar(Q_FREE));
             // S += (decayed U^T) K ; O = U^T P^T
             if (!mbar_wait(bar(U_READY), ph, abort_flag, p.err, 48)) break;
             if (!mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 49)) break;
@@ -836,8 +894,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             umma_commit(bar(K_FREE + b));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_UO, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64,
-                         kk != 0);
+                umma_f16(uo, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64, kk != 0);
             umma_commit(bar(O_FULL));
             umma_commit(bar(P_FREE));
         }
@@ -872,13 +929,15 @@ cudaError_t launch_d(const GdnTc& t, int64_t mchunks, cudaStream_t st) {
     if (!make_tma_2d_bf16(&tm_k, t.k, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
     if (!make_tma_2d_bf16(&tm_v, t.v, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
     if (!make_tma_2d_bf16(&tm_q, t.q, (uint64_t)t.n_q_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
-    gdn_schedule_kernel<<<1, 1024, 0, st>>>(t.seg_cu, t.n_seg, t.n_rows, t.chunk_cu, t.err);
+    CUtensorMap tm_o;
+    if (!make_tma_2d_bf16_plain(&tm_o, t.o, (uint64_t)t.n_rows, HD, HD, DVT, C)) return cudaErrorInvalidValue;
+    gdn_schedule_kernel<<<1, 1024, 0, st>>>(t.seg_cu, t.n_seg, t.n_rows, t.chunk_cu, t.chunk_info, t.err);
     if (mchunks > 0) {
         dim3 pg((unsigned)mchunks, t.H);
         gdn_prep_kernel<D><<<pg, 128, PrepLayout<D>::BYTES, st>>>(tm_k, tm_q, t);
     }
     gdn_state_kernel<D><<<(unsigned)((int64_t)t.n_seg * t.H * (D / DVT)), STATE_THREADS, StateLayout<D>::BYTES, st>>>(
-        tm_k, tm_v, tm_q, t);
+        tm_k, tm_v, tm_q, tm_o, t);
     count_launches(mchunks > 0 ? 3 : 2);
     return cudaGetLastError();
 }
@@ -891,10 +950,12 @@ bool gdn_tc_supported(const GdnArgs& a, int dt) {
     return device_is_sm100() && tma_available();
 }
 
+static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
 size_t gdn_tc_ws_bytes(int64_t n_rows, int n_seg, int H, int d) {
     (void)d;
-    const size_t cu = (((size_t)n_seg + 1) * 4 + 255) & ~(size_t)255;
-    return cu + (size_t)max_chunks(n_rows, n_seg) * H * 2 * IMG;
+    const size_t mc = (size_t)max_chunks(n_rows, n_seg);
+    return up256(((size_t)n_seg + 1) * 4) + up256(mc * sizeof(int4)) + mc * H * 2 * IMG;
 }
 
 cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st) {
@@ -916,10 +977,13 @@ cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st) {
     t.h_final = a.h_final;
     t.o = reinterpret_cast<bf16*>(a.o);
     unsigned char* base = reinterpret_cast<unsigned char*>(a.ws) + MOM_WS_HEADER_BYTES;
-    t.chunk_cu = reinterpret_cast<int32_t*>(base);
-    t.img = base + ((((size_t)a.n_seg + 1) * 4 + 255) & ~(size_t)255);
-    t.err = a.ws;
     const int64_t mc = max_chunks(a.n_rows, a.n_seg);
+    t.chunk_cu = reinterpret_cast<int32_t*>(base);
+    base += up256(((size_t)a.n_seg + 1) * 4);
+    t.chunk_info = reinterpret_cast<int4*>(base);
+    base += up256((size_t)mc * sizeof(int4));
+    t.img = base;
+    t.err = a.ws;
     return a.d == 256 ? launch_d<256>(t, mc, st) : launch_d<128>(t, mc, st);
 }
 

@@ -18,6 +18,9 @@ void count_launches(int n);
 bool tma_available();
 bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t row_pitch_elems,
                       uint32_t box_cols, uint32_t box_rows);
+// Same without swizzle (row-major shared tile, e.g. an output staging tile).
+bool make_tma_2d_bf16_plain(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t row_pitch_elems,
+                            uint32_t box_cols, uint32_t box_rows);
 bool device_is_sm100();
 
 // router.cu
