@@ -39,6 +39,7 @@ constexpr int C = 64;                 // chunk length
 constexpr int DVT = 128;              // d_v rows per state CTA (TMEM lanes)
 constexpr int IMG = C * C * 2;        // one swizzled 64x64 bf16 tile
 constexpr int GB = 2 * C + 4;         // floats per chunk-gate record
+constexpr int LP = C + 1;             // row pitch (floats) of the prep's fp32 tiles: no bank conflicts
 
 struct GdnTc {
     const bf16* q;
@@ -188,12 +189,128 @@ __device__ __forceinline__ void gather_rows(const GdnTc& p, const bf16* base, in
 }
 
 // ----------------------------------------------------------------- prep --
+// Row r of L = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r < n, else 0) from
+// the G row held in registers (ga: columns 0..31, gc: 32..63).  Values are
+// computed before any store so the gamma loads pipeline.
+__device__ __forceinline__ void prep_l_row(int r, int n, const float* __restrict__ gam, const float* __restrict__ bet,
+                                           const uint32_t (&ga)[32], const uint32_t (&gc)[32],
+                                           float* __restrict__ lrow) {
+    const float gr = gam[r], br = bet[r];
+    float v[32];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int s = 32 * half + e;
+            const float G = __uint_as_float(half ? gc[e] : ga[e]);
+            v[e] = (s < r && r < n) ? br * __expf(gr - gam[s]) * G : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) lrow[32 * half + e] = v[e];
+    }
+}
+
+// Row r of P = e^(gamma_r - gamma_s) q_r.k_s (s <= r < n, else 0), bf16,
+// written into the 128-byte-swizzled 64 x 64 image.
+__device__ __forceinline__ void prep_p_row(int r, int n, const float* __restrict__ gam, const uint32_t (&ga)[32],
+                                           const uint32_t (&gc)[32], unsigned char* __restrict__ pimg) {
+    const float gr = gam[r];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            float pv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int s = 32 * half + e + u;
+                const float G = __uint_as_float(half ? gc[e + u] : ga[e + u]);
+                pv[u] = (s <= r && r < n) ? __expf(gr - gam[s]) * G : 0.f;
+            }
+            w[e / 2] = pack_bf16(pv[0], pv[1]);
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const int c8 = 4 * half + c4;
+            *reinterpret_cast<uint4*>(pimg + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+                make_uint4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+        }
+    }
+}
+
+// Row r, columns [32 half, 32 half + 32) of Tb = T diag(beta) (lower triangle), bf16 image.
+__device__ __forceinline__ void prep_tb_row(int r, int half, const float* __restrict__ trow,
+                                            const float* __restrict__ bet, unsigned char* __restrict__ timg) {
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int s = 32 * half + e;
+        v[e] = s <= r ? trow[s] * bet[s] : 0.f;
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) w[e / 2] = pack_bf16(v[e], v[e + 1]);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        const int c8 = 4 * half + c4;
+        *reinterpret_cast<uint4*>(timg + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+            make_uint4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+    }
+}
+
+// One level of the blocked inverse: the 16 x 16 blocks at distance LEV below
+// the diagonal, T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj (i = j + LEV), from the
+// blocks closer to the diagonal.  128 threads; trip counts are compile-time so
+// each thread's independent elements overlap their load latencies.
+template <int LEV>
+__device__ __forceinline__ void offdiag_level(const float* Lm, float* Tm, float* Mb, int tid) {
+    constexpr int NB = 4 - LEV, PER = NB * 256 / 128;
+    float acc[PER];
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        const int e = tid + 128 * q;
+        const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
+        const int bi = LEV + qb, bj = qb;
+        float sacc = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < LEV; ++kb) {
+            const float* Lr = Lm + (16 * bi + a) * LP + 16 * (bj + kb);
+            const float* Tc = Tm + (16 * (bj + kb)) * LP + 16 * bj + c;
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2) sacc = fmaf(Lr[s2], Tc[s2 * LP], sacc);
+        }
+        acc[q] = sacc;
+    }
+#pragma unroll
+    for (int q = 0; q < PER; ++q) Mb[tid + 128 * q] = acc[q];
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        const int e = tid + 128 * q;
+        const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
+        const int bi = LEV + qb;
+        const float* Tr = Tm + (16 * bi + a) * LP + 16 * bi;
+        const float* Mc = Mb + qb * 256 + c;
+        float sacc = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) sacc = fmaf(Tr[s2], Mc[s2 * 16], sacc);
+        acc[q] = -sacc;
+    }
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        const int e = tid + 128 * q;
+        const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
+        Tm[(16 * (LEV + qb) + a) * LP + 16 * qb + c] = acc[q];
+    }
+    __syncthreads();
+}
+
 template <int D>
 struct PrepLayout {
     static constexpr int KQ = 0;                      // two slabs: K rows 0..63 | Q rows 64..127 (16 KB each)
-    static constexpr int TM = 0;                      // fp32 [64][64] T, reusing KQ after the MMAs
-    static constexpr int LM = 2 * 16384;              // fp32 [64][64] L
-    static constexpr int MB = LM + C * C * 4;         // fp32 3 x [16][16] block products
+    static constexpr int TM = 0;                      // fp32 [64][LP] T, reusing KQ after the MMAs
+    static constexpr int LM = 2 * 16384;              // fp32 [64][LP] L
+    static constexpr int MB = LM + C * LP * 4;        // fp32 3 x [16][16] block products
     static constexpr int GBB = MB + 3 * 256 * 4;      // beta[64], gamma[64]
     static constexpr int BARS = GBB + 2 * C * 4;      // land, mma (one phase per pair of slabs)
     static constexpr int MISC = BARS + 16;
@@ -225,11 +342,22 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int64_t r0 = info.y;
     const int n = info.z;
 
+    constexpr int NPH = SLABS / 2 > 0 ? SLABS / 2 : 1;
+    // K (and contiguous Q) of one phase by TMA; rows past n hold other finite data and are masked below
+    auto issue_tma = [&](int ph) {
+        const int j0 = 2 * ph, nj = SLABS - j0 < 2 ? SLABS - j0 : 2;
+        mbar_arrive_expect_tx(land, nj * 8192 * (p.qidx ? 1 : 2));
+        for (int jj = 0; jj < nj; ++jj) {
+            tma_load_2d(kq + jj * 16384, &tm_k, land, h * D + 64 * (j0 + jj), (int)r0);
+            if (!p.qidx) tma_load_2d(kq + jj * 16384 + 8192, &tm_q, land, h * D + 64 * (j0 + jj), (int)r0);
+        }
+    };
     if (tid == 0) {
         mbar_init(land, 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
+        issue_tma(0);
     }
     if (warp == 0) {
         float b[2], gg[2];
@@ -247,17 +375,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t tmem = *tslot;
 
     // G = [K; Q] K^T : M = 128, N = 64, K = D, two slabs (128 columns of D) per phase.
-    // K (and contiguous Q) by TMA; rows past n hold other finite data and are masked below.
-    constexpr int NPH = SLABS / 2 > 0 ? SLABS / 2 : 1;
     for (int ph = 0; ph < NPH; ++ph) {
         const int j0 = 2 * ph, nj = SLABS - j0 < 2 ? SLABS - j0 : 2;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(land, nj * 8192 * (p.qidx ? 1 : 2));
-            for (int jj = 0; jj < nj; ++jj) {
-                tma_load_2d(kq + jj * 16384, &tm_k, land, h * D + 64 * (j0 + jj), (int)r0);
-                if (!p.qidx) tma_load_2d(kq + jj * 16384 + 8192, &tm_q, land, h * D + 64 * (j0 + jj), (int)r0);
-            }
-        }
+        if (ph > 0 && tid == 0) issue_tma(ph);
         if (p.qidx) {
             for (int idx = tid; idx < C * 8; idx += 128) {
                 const int row = idx >> 3, c8 = idx & 7;
@@ -299,35 +419,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     unsigned char* img = p.img + ((size_t)g * p.H + h) * 2 * IMG;
     const int r = tid & 63;
-    const float gr = ggam[r];
-    if (tid < 64) {
-        // L row r: strictly lower, zero in rows and columns past n
-        const float br = gbeta[r];
-#pragma unroll
-        for (int s = 0; s < C; ++s) {
-            float val = 0.f;
-            if (s < r && r < n) val = br * __expf(gr - ggam[s]) * __uint_as_float(s < 32 ? ga[s] : gc[s - 32]);
-            Lm[r * C + s] = val;
-        }
-    } else {
-        // P row r: causal, decayed q_r . k_s, bf16 swizzled image
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-                float pv[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int s = c8 * 8 + e2 * 2 + e;
-                    pv[e] = 0.f;
-                    if (s <= r && r < n) pv[e] = __expf(gr - ggam[s]) * __uint_as_float(s < 32 ? ga[s] : gc[s - 32]);
-                }
-                w[e2] = pack_bf16(pv[0], pv[1]);
-            }
-            *reinterpret_cast<uint4*>(img + IMG + r * 128 + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    }
+    if (tid < 64) prep_l_row(r, n, ggam, gbeta, ga, gc, Lm + r * LP);
+    else prep_p_row(r, n, ggam, ga, gc, img + IMG);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -345,7 +438,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
         for (int rl = 1; rl < 16; ++rl) {
             float a0 = 0.f, a1 = 0.f;
-            const float* Lr = Lm + (base + rl) * C + base;
+            const float* Lr = Lm + (base + rl) * LP + base;
 #pragma unroll
             for (int sl = 0; sl < rl; ++sl) {
                 if (sl & 1) a1 = fmaf(Lr[sl], t[sl], a1); else a0 = fmaf(Lr[sl], t[sl], a0);
@@ -353,55 +446,16 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (rl > cc) t[rl] = -(a0 + a1);
         }
 #pragma unroll
-        for (int rl = 0; rl < 16; ++rl) Tm[(base + rl) * C + base + cc] = t[rl];
+        for (int rl = 0; rl < 16; ++rl) Tm[(base + rl) * LP + base + cc] = t[rl];
     }
     __syncthreads();
     // Off-diagonal blocks by distance from the diagonal:
     //   T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj      (i > j)
-    for (int lev = 1; lev < 4; ++lev) {
-        const int nb = 4 - lev;
-        for (int e = tid; e < nb * 256; e += 128) {
-            const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
-            const int bi = lev + qb, bj = qb;
-            float acc = 0.f;
-            for (int bkk = bj; bkk < bi; ++bkk) {
-                const float* Lr = Lm + (16 * bi + a) * C + 16 * bkk;
-                const float* Tc = Tm + (16 * bkk) * C + 16 * bj + c;
-#pragma unroll
-                for (int s = 0; s < 16; ++s) acc = fmaf(Lr[s], Tc[s * C], acc);
-            }
-            Mb[qb * 256 + a * 16 + c] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nb * 256; e += 128) {
-            const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
-            const int bi = lev + qb, bj = qb;
-            const float* Tr = Tm + (16 * bi + a) * C + 16 * bi;
-            float acc = 0.f;
-#pragma unroll
-            for (int s = 0; s < 16; ++s) acc = fmaf(Tr[s], Mb[qb * 256 + s * 16 + c], acc);
-            Tm[(16 * bi + a) * C + 16 * bj + c] = -acc;
-        }
-        __syncthreads();
-    }
+    offdiag_level<1>(Lm, Tm, Mb, tid);
+    offdiag_level<2>(Lm, Tm, Mb, tid);
+    offdiag_level<3>(Lm, Tm, Mb, tid);
     // Tb = T diag(beta): lower triangle (s <= r); beta is zero past n
-    {
-        const int half = tid >> 6;
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-            const int s = 32 * half + e;
-            const float v0 = s <= r ? Tm[r * C + s] * gbeta[s] : 0.f;
-            const float v1 = s + 1 <= r ? Tm[r * C + s + 1] * gbeta[s + 1] : 0.f;
-            w[e / 2] = pack_bf16(v0, v1);
-        }
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const int c8 = 4 * half + c4;
-            *reinterpret_cast<uint4*>(img + r * 128 + ((c8 ^ (r & 7)) << 4)) =
-                make_uint4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
-        }
-    }
+    prep_tb_row(r, tid >> 6, Tm + r * LP, gbeta, img);
 }
 
 // ---------------------------------------------------------------- state --
