@@ -462,7 +462,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 enum Bar {
     GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, K_FREE = 8, UO_FREE = 10,
     V_LAND = 12, V_FULL, V_FREE, Q_FULL, Q_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
-    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, X_FREE, DONE, NBARS
+    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, X_FREE, DONE,
+    STAGE_IN, STAGE_OUT, NBARS
 };
 
 constexpr int NMATH = 8;              // math warps 0..7
@@ -533,6 +534,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         counts[GB_FREE] = counts[GB_FREE + 1] = NMATH;
         counts[UO_FREE] = counts[UO_FREE + 1] = NMATH;
         counts[SBF_READY] = counts[ZT_READY] = counts[U_READY] = counts[X_FREE] = NMATH;
+        counts[STAGE_IN] = counts[STAGE_OUT] = NMATH;
         counts[Q_FULL] = p.qidx ? NGATHER : 1;
         for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), counts[i]);
         *abort_flag = 0;
@@ -636,7 +638,9 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             if (c > 0) {
                 // ub still holds the previous chunk's output tile until its TMA store has read it
                 if (warp == 0 && lane == 0) bulk_wait_read0();
-                named_sync(1, NMATH * 32);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(STAGE_OUT));
+                if (!mbar_wait(bar(STAGE_OUT), (c - 1) & 1, abort_flag, p.err, 28)) break;
             }
             tc_fence_after();
             {
@@ -743,7 +747,9 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             }
             tc_fence_before();
             fence_proxy_async_smem();
-            named_sync(1, NMATH * 32);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(STAGE_IN));
+            if (!mbar_wait(bar(STAGE_IN), c & 1, abort_flag, p.err, 29)) break;
             if (n == C) {
                 if (warp == 0 && lane == 0) {
                     tma_store_2d(&tm_o, ub, h * D + dv0, (int)r0);

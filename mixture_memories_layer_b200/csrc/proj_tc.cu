@@ -10,14 +10,17 @@
 // memories or two projections, and holds whole heads, so the per-head L2
 // norm of q and k is applied in the epilogue straight from TMEM.
 //
-// Roles (288 threads, one CTA per SM, persistent over tiles):
+// Roles (416 threads, one CTA per SM, persistent over tiles):
 //   warps 0-3  producers: A rows gathered with 16-byte cp.async into the
 //              128-byte-swizzled K-major layout (rows come from perm_token,
-//              so a tile of routed rows is a gather); thread 0 also issues
-//              the TMA load of the weight tile (B, K-major, 128-byte swizzle)
-//   warp 8     MMA issuer: 4 x tcgen05.mma (M=128, N=256, K=16) per 64-wide
+//              so a tile of routed rows is a gather), each thread's arrival
+//              on the stage barrier triggered by the copies' completion;
+//              thread 0 also issues the TMA load of the weight tile (B,
+//              K-major, 128-byte swizzle)
+//   warp 12    MMA issuer: 4 x tcgen05.mma (M=128, N=256, K=16) per 64-wide
 //              K step into one of two TMEM accumulators (2 x 256 columns)
-//   warps 4-7  epilogue: TMEM -> registers -> (L2 norm) -> bf16 -> global,
+//   warps 4-11 epilogue: TMEM -> registers -> (L2 norm) -> bf16 -> global,
+//              two warps per TMEM lane quarter (one per column half),
 //              overlapping the next tile's main loop
 // Every wait is bounded (sm100.cuh); on a timeout the CTA records
 // MOM_DEVERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
@@ -33,11 +36,12 @@ using namespace sm100;
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;   // 32 KB
-constexpr int NPROD = 128, NEPI = 128;
+constexpr int NPROD = 128, NEPI = 256;     // 4 producer warps, 8 epilogue warps
+constexpr int W_MMA = (NPROD + NEPI) / 32;  // MMA warp
 constexpr int THREADS = NPROD + NEPI + 32;
-constexpr int LAG = STAGES - 1;        // producer arrives for a stage LAG iterations after issuing it
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256;
+constexpr int STAGE_PIECE = 32 * 128;               // one warp's 32 rows x 64 columns, bf16, 128-byte swizzle
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + (size_t)(NEPI / 32) * STAGE_PIECE + 256;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
 struct TcParams {
@@ -89,16 +93,23 @@ __device__ __forceinline__ bool tile_at(const TcParams& p, int64_t t, Tile& T) {
     return false;
 }
 
+struct OutMaps {
+    CUtensorMap q, k_sh, v_sh, k_p, v_p;   // [rows, H*d] bf16, boxes of 32 rows x 64 columns
+};
+
 __global__ void __launch_bounds__(THREADS, 1)
-proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant__ CUtensorMap tm_kv, TcParams p) {
+proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant__ CUtensorMap tm_kv,
+               const __grid_constant__ OutMaps om, TcParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                            ~static_cast<uintptr_t>(1023));
     unsigned char* sA = smem;
     unsigned char* sB = smem + STAGES * A_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+    unsigned char* sOut = sB + STAGES * B_BYTES;                       // per epilogue warp staging piece
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + (NEPI / 32) * STAGE_PIECE);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(bars);
@@ -120,7 +131,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 8) {
+    if (warp == W_MMA) {
         tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
         tmem_relinquish();
     }
@@ -136,24 +147,39 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
         const int c = tid & 7, rsub = tid >> 3;   // 8 lanes per 128-byte row, 16 rows per pass
         uint32_t it = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
-            Tile T;
-            if (!tile_at(p, t, T)) continue;
+        // the next valid tile of this CTA at or after t
+        auto next_tile = [&](int64_t t, Tile& T) {
+            while (t < p.n_tiles && !tile_at(p, t, T)) t += gridDim.x;
+            return t;
+        };
+        // token behind each of this thread's 8 rows (-1: zero-fill)
+        auto row_tokens = [&](const Tile& T, int64_t (&tok)[8]) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int64_t row = T.r0 + rsub + 16 * i;
+                tok[i] = row < T.r1 ? (T.m < 0 ? row : (int64_t)p.perm[row]) : -1;
+            }
+        };
+        Tile T;
+        int64_t t = next_tile(blockIdx.x, T);
+        int64_t tok[8];
+        if (t < p.n_tiles) row_tokens(T, tok);
+        while (t < p.n_tiles && ok) {
+            // the next tile and its (gathered) row tokens are fetched half-way
+            // through this tile, so the loads are in flight while it is issued
+            Tile Tn;
+            int64_t tn = p.n_tiles, ntok[8];
             const bf16* src[8];
             uint32_t nbytes[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int64_t row = T.r0 + rsub + 16 * i;
-                int64_t tok = -1;
-                if (row < T.r1) {
-                    tok = T.m < 0 ? row : (int64_t)p.perm[row];
-                    if (tok < 0 || tok >= p.n_tok) {
-                        if (c == 0) record_error(p.ws, MOM_DEVERR_ROW_INDEX, row);
-                        tok = -1;
-                    }
+                int64_t tk = tok[i];
+                if (tk >= p.n_tok || (tk < 0 && T.r0 + rsub + 16 * i < T.r1)) {
+                    if (c == 0) record_error(p.ws, MOM_DEVERR_ROW_INDEX, T.r0 + rsub + 16 * i);
+                    tk = -1;
                 }
-                src[i] = p.x + (tok >= 0 ? tok : 0) * p.D + c * 8;
-                nbytes[i] = tok >= 0 ? 16u : 0u;   // rows past the tile are zero-filled
+                src[i] = p.x + (tk >= 0 ? tk : 0) * p.D + c * 8;
+                nbytes[i] = tk >= 0 ? 16u : 0u;   // rows past the tile are zero-filled
             }
             const CUtensorMap* tm = T.m < 0 ? &tm_sh : &tm_kv;
             const int wrow = (T.m < 0 ? 0 : T.m * 2 * p.H * p.d) + T.ct * BN;
@@ -170,28 +196,31 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
                     const int r = rsub + 16 * i;
                     cp_async_16(dstA + r * 128 + ((c ^ (r & 7)) << 4), src[i] + kb * BK, nbytes[i]);
                 }
-                cp_async_commit();
-                if (it >= LAG) {
-                    cp_async_wait<LAG>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(full0 + 8 * ((it - LAG) % STAGES));
+                // the barrier receives this thread's arrival when its copies land
+                cp_async_arrive_noinc(full0 + 8 * s);
+                if (kb == KB / 2) {
+                    tn = next_tile(t + gridDim.x, Tn);
+                    if (tn < p.n_tiles) row_tokens(Tn, ntok);
                 }
             }
+            t = tn;
+            T = Tn;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tok[i] = ntok[i];
         }
-        // drain: the last LAG stages still owe their arrival
         cp_async_wait<0>();
-        fence_proxy_async_smem();
-        for (uint32_t j = it >= LAG ? it - LAG : 0; j < it; ++j) mbar_arrive(full0 + 8 * (j % STAGES));
         if (!ok && tid == 0) {
             // weight tiles still in flight must land before the CTA exits
             for (uint32_t j = it >= STAGES ? it - STAGES : 0; j < it; ++j)
                 mbar_wait_drain(full0 + 8 * (j % STAGES), (j / STAGES) & 1);
         }
-    } else if (warp < 8) {
+    } else if (warp < W_MMA) {
         // ------------------------------------------------------- epilogue
-        const int e = warp - 4;                 // TMEM lanes 32e .. 32e+31
-        const int row_local = 32 * e + lane;
+        // warp 4 + e: TMEM lanes 32 (e % 4) .. + 31, columns [128 (e / 4), + 128)
+        const int e = warp - 4, qd = e & 3, hf = e >> 2;
+        const int row_local = 32 * qd + lane;
         const int Hd = p.H * p.d;
+        constexpr int HALF = BN / 2;
         uint32_t tc = 0;
         for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
             Tile T;
@@ -202,49 +231,97 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
             const int64_t row = T.r0 + row_local;
             const bool live = row < T.r1;
             const int col0 = T.ct * BN;
-            const int part = col0 / Hd, cc0 = col0 % Hd;
+            const int part_i = col0 / Hd, cc0 = col0 % Hd;
             bf16* base;
             bool norm;
             if (T.m < 0) {
-                base = part == 0 ? p.q : part == 1 ? p.k_sh : p.v_sh;
-                norm = part < 2;
+                base = part_i == 0 ? p.q : part_i == 1 ? p.k_sh : p.v_sh;
+                norm = part_i < 2;
             } else {
-                base = part == 0 ? p.k_p : p.v_p;
-                norm = part == 0;
+                base = part_i == 0 ? p.k_p : p.v_p;
+                norm = part_i == 0;
             }
-            bf16* orow = base + (live ? row : 0) * (int64_t)Hd + cc0;
-            const uint32_t taddr = tmem_base + ((uint32_t)(32 * e) << 16) + acc * BN;
-            for (int g = 0; g < BN; g += p.d) {
-                float sc = 1.f;
+            const CUtensorMap* omap = T.m < 0 ? (part_i == 0 ? &om.q : part_i == 1 ? &om.k_sh : &om.v_sh)
+                                              : (part_i == 0 ? &om.k_p : &om.v_p);
+            // a piece goes out by TMA only when all 32 of its rows belong to this tile
+            const bool full_piece = T.r0 + 32 * qd + 32 <= T.r1;
+            bf16* orow = base + (live ? row : 0) * (int64_t)Hd + cc0 + hf * HALF;
+            const uint32_t taddr = tmem_base + ((uint32_t)(32 * qd) << 16) + acc * BN + hf * HALF;
+            const uint32_t piece = smem_u32(sOut + e * STAGE_PIECE);
+            const int gw = p.d < HALF ? p.d : HALF;          // head-group width inside this half
+            float sc_full = 1.f;
+            if (norm && p.d > HALF) {
+                // a head spans both halves: each thread sums the whole row (TMEM reads are cheap)
+                float ss = 0.f;
                 uint32_t r[32];
-                if (norm) {
+                const uint32_t trow = taddr - hf * HALF;
+                for (int cc = 0; cc < BN; cc += 32) {
+                    tmem_ld_x32(trow + cc, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
+                }
+                sc_full = rsqrtf(ss + 1e-6f);
+            }
+            float scg[HALF / 64 * 2];                        // per 32-column block scale
+#pragma unroll
+            for (int j = 0; j < HALF / 32; ++j) scg[j] = sc_full;
+            if (norm && p.d <= HALF) {
+                for (int g = 0; g < HALF; g += gw) {
                     float ss = 0.f;
-                    for (int cc = 0; cc < p.d; cc += 32) {
+                    uint32_t r[32];
+                    for (int cc = 0; cc < gw; cc += 32) {
                         tmem_ld_x32(taddr + g + cc, r);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float v = __uint_as_float(r[i]);
-                            ss = fmaf(v, v, ss);
-                        }
+                        for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
                     }
-                    sc = rsqrtf(ss + 1e-6f);
+                    const float sc = rsqrtf(ss + 1e-6f);
+#pragma unroll
+                    for (int j = 0; j < HALF / 32; ++j)
+                        if (j * 32 >= g && j * 32 < g + gw) scg[j] = sc;
                 }
-                for (int cc = 0; cc < p.d; cc += 32) {
-                    tmem_ld_x32(taddr + g + cc, r);
+            }
+            // 64-column pieces: registers -> swizzled staging -> TMA store
+#pragma unroll
+            for (int pc = 0; pc < HALF / 64; ++pc) {
+                if (lane == 0) bulk_wait_read0();            // the previous piece has left shared memory
+                __syncwarp();
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int j = pc * 2 + hh;
+                    uint32_t r[32];
+                    tmem_ld_x32(taddr + 32 * j, r);
                     tmem_ld_wait();
-                    if (live) {
-                        uint4 out[4];
-                        uint32_t* o32 = reinterpret_cast<uint32_t*>(out);
+                    const float sc = scg[j];
+                    uint32_t w[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * sc,
-                                                                      __uint_as_float(r[2 * i + 1]) * sc);
-                            o32[i] = *reinterpret_cast<uint32_t*>(&h2);
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * sc,
+                                                                  __uint_as_float(r[2 * i + 1]) * sc);
+                        w[i] = *reinterpret_cast<uint32_t*>(&h2);
+                    }
+                    if (full_piece) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            const int ch = hh * 4 + c4;
+                            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};"
+                                         ::"r"(piece + lane * 128 + ((ch ^ (lane & 7)) << 4)),
+                                           "r"(w[4 * c4]), "r"(w[4 * c4 + 1]), "r"(w[4 * c4 + 2]), "r"(w[4 * c4 + 3])
+                                         : "memory");
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(orow + g + cc);
+                    } else if (live) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * j);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = out[i];
+                        for (int c4 = 0; c4 < 4; ++c4) dst[c4] = make_uint4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+                    }
+                }
+                if (full_piece) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(omap, piece, cc0 + hf * HALF + 64 * pc, (int)(T.r0 + 32 * qd));
+                        bulk_commit();
                     }
                 }
             }
@@ -252,6 +329,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
             mbar_arrive(tempty0 + 8 * acc);
             ++tc;
         }
+        if (lane == 0) bulk_wait0();
     } else if (lane == 0) {
         // ------------------------------------------------------ MMA issuer
         uint32_t it = 0, tc = 0;
@@ -285,7 +363,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
@@ -304,6 +382,12 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     CUtensorMap tm_sh, tm_kv;
     if (!make_tma_2d_bf16(&tm_sh, a.w_shared, (uint64_t)3 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
     if (!make_tma_2d_bf16(&tm_kv, a.w_kv, (uint64_t)a.M * 2 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
+    OutMaps om;
+    const uint64_t nrp = (uint64_t)a.n_tok * a.K;
+    if (!make_tma_2d_bf16(&om.q, a.q, a.n_tok, Hd, Hd, 64, 32) || !make_tma_2d_bf16(&om.k_sh, a.k_sh, a.n_tok, Hd, Hd, 64, 32) ||
+        !make_tma_2d_bf16(&om.v_sh, a.v_sh, a.n_tok, Hd, Hd, 64, 32) || !make_tma_2d_bf16(&om.k_p, a.k_p, nrp, Hd, Hd, 64, 32) ||
+        !make_tma_2d_bf16(&om.v_p, a.v_p, nrp, Hd, Hd, 64, 32))
+        return cudaErrorInvalidValue;
     TcParams p;
     p.x = reinterpret_cast<const bf16*>(a.x);
     p.perm = a.perm_token;
@@ -332,7 +416,7 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t grid = p.n_tiles < sms ? p.n_tiles : sms;
-    proj_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, st>>>(tm_sh, tm_kv, p);
+    proj_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, st>>>(tm_sh, tm_kv, om, p);
     count_launches(1);
     return cudaGetLastError();
 }
