@@ -460,37 +460,43 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 // ---------------------------------------------------------------- state --
 enum Bar {
-    GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, K_FREE = 8, UO_FREE = 10,
-    V_LAND = 12, V_FULL, V_FREE, Q_FULL, Q_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
-    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, X_FREE, DONE,
-    STAGE_IN, STAGE_OUT, NBARS
+    GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, Q_FULL = 8, KQ_FREE = 10,
+    V_LAND = 12, V_FULL, V_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
+    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, XO_FREE, DONE, NBARS
 };
 
 constexpr int NMATH = 8;              // math warps 0..7
 constexpr int W_PROD = 8;             // producer warp (TMA, gates, tail zeroing)
-constexpr int NGATHER = 3;            // gather warps 9..11 (indexed q rows)
+constexpr int NGATHER = 3;            // q~ warps 9..11 (q rows, possibly through the index, scaled in place)
 constexpr int W_MMA = 12;             // MMA warp
 constexpr int STATE_THREADS = 13 * 32;
+constexpr float LOG2E = 1.4426950408889634f;
 
-// gate record of one chunk, derived from chunk_scan
-constexpr int G_EG = 0;               // e^gamma_s (0 past n)
-constexpr int G_DEC = C;              // e^(gamma_last - gamma_s) (0 past n)
+// Gate record of one chunk.  TMEM holds T = rho S with rho = 2^lr a running
+// scalar kept in [2^-1/2, 2^1/2]: the chunk decay a = e^gamma_last is applied
+// as the MMA's power-of-two accumulator scale 2^-e plus a change of rho.
+constexpr int G_EGR = 0;              // e^gamma_s / rho_c                     (0 past n)
+constexpr int G_DEC = C;              // rho_{c+1} e^(gamma_last - gamma_s)    (0 past n)
 constexpr int G_N = 2 * C;            // n (int bits)
-constexpr int G_EGC = 2 * C + 1;      // e^gamma_last
+constexpr int G_SCL = 2 * C + 1;      // e (int bits): T <- 2^-e T + ...; -1: the old T is dropped (a < 2^-15.5)
+constexpr int G_LR = 2 * C + 2;       // lr_{c+1}
 
 template <int D>
 struct StateLayout {
     static constexpr int SLABS = D / 64;
-    static constexpr int S_BF = 0;                            // [128 x D] bf16, SLABS slabs of 16 KB
-    static constexpr int K0 = S_BF + SLABS * 16384;           // 2 x [64 x D] bf16
-    static constexpr int KSZ = SLABS * 8192;
-    static constexpr int QB = K0 + 2 * KSZ;                   // [64 x D] bf16
-    static constexpr int VB = QB + KSZ;                       // [64 x 128] bf16: two 64-column slabs
+    // [K; q~] of a chunk: per 64-column slab, the 64 key rows then the 64
+    // scaled query rows (8 KB each), so that one N = 128 MMA computes
+    // Z = T K^T and X = T q~^T together
+    static constexpr int KQSZ = SLABS * 16384;
+    static constexpr int KQ0 = 0;                             // 2 x [K; q~]
+    static constexpr int VB = KQ0 + 2 * KQSZ;                 // [64 x 128] bf16: two 64-column slabs
     static constexpr int TB = VB + 2 * 8192;                  // Tb image
     static constexpr int PB = TB + IMG;                       // P image
-    static constexpr int ZB = PB + IMG;                       // [128 x 64] bf16: Z~, then U^T
-    static constexpr int UB = ZB + 16384;                     // [128 x 64] bf16: decayed U^T
-    static constexpr int GBB = UB + 16384;                    // 2 gate records
+    static constexpr int YB = PB + IMG;                       // [128 x 64] bf16: V^T - Z~
+    static constexpr int UOB = YB + 16384;                    // [128 x 64] bf16: U^T (output term)
+    static constexpr int USB = UOB + 16384;                   // [128 x 64] bf16: U^T diag(G_DEC) (state term)
+    static constexpr int STG = USB + 16384;                   // 8 x [32 rows x 32 d_v] bf16: per-warp output staging
+    static constexpr int GBB = STG + 16384;                   // 2 gate records
     static constexpr int BARS = GBB + 2 * GB * 4;
     static constexpr int MISC = BARS + NBARS * 8;
     static constexpr size_t BYTES = 1024 + MISC + 16;
@@ -499,13 +505,15 @@ struct StateLayout {
 template <int D>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, GdnTc p) {
+                 const __grid_constant__ CUtensorMap tm_o, GdnTc p) {
     using Lay = StateLayout<D>;
-    constexpr int SLABS = D / 64, NDV = D / DVT;
-    // TMEM columns: state, Z, X, and two buffers each holding U then O
-    constexpr uint32_t T_S = 0, T_Z = D, T_X = D + 64, T_UO = D + 128;
+    constexpr int SLABS = D / 64, NDV = D / DVT, HALF = D / 2;
+    // TMEM columns: T = rho S (fp32), its bf16 copy (the A operand of Z and
+    // X), Z then U, X then X + O (Z and X adjacent: one N = 128 accumulator)
+    constexpr uint32_t T_S = 0, T_SB = D, T_ZU = D + D / 2, T_XO = T_ZU + 64;
     constexpr uint32_t TMEM_COLS = 512;
-    static_assert(T_UO + 128 <= TMEM_COLS, "TMEM budget");
+    static_assert(T_XO + 64 <= TMEM_COLS, "TMEM budget");
+    static_assert(Lay::BYTES <= 232448, "shared memory budget");
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
@@ -513,9 +521,9 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lay::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
     auto bar = [&](int i) { return smem_u32(bars + i); };
-    const uint32_t s_bf = smem_u32(sm + Lay::S_BF), kb0 = smem_u32(sm + Lay::K0), qb = smem_u32(sm + Lay::QB);
-    const uint32_t vb = smem_u32(sm + Lay::VB), timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB);
-    const uint32_t zb = smem_u32(sm + Lay::ZB), ub = smem_u32(sm + Lay::UB);
+    const uint32_t kq0 = smem_u32(sm + Lay::KQ0), vb = smem_u32(sm + Lay::VB);
+    const uint32_t timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB), yb = smem_u32(sm + Lay::YB);
+    const uint32_t uob = smem_u32(sm + Lay::UOB), usb = smem_u32(sm + Lay::USB), stg0 = smem_u32(sm + Lay::STG);
     float* gbuf = reinterpret_cast<float*>(sm + Lay::GBB);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -532,10 +540,8 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int counts[NBARS];
         for (int i = 0; i < NBARS; ++i) counts[i] = 1;
         counts[GB_FREE] = counts[GB_FREE + 1] = NMATH;
-        counts[UO_FREE] = counts[UO_FREE + 1] = NMATH;
-        counts[SBF_READY] = counts[ZT_READY] = counts[U_READY] = counts[X_FREE] = NMATH;
-        counts[STAGE_IN] = counts[STAGE_OUT] = NMATH;
-        counts[Q_FULL] = p.qidx ? NGATHER : 1;
+        counts[V_FREE] = counts[SBF_READY] = counts[ZT_READY] = counts[U_READY] = counts[XO_FREE] = NMATH;
+        counts[Q_FULL] = counts[Q_FULL + 1] = NGATHER;
         for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), counts[i]);
         *abort_flag = 0;
         fence_barrier_init();
@@ -551,57 +557,58 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
     if (warp < NMATH) {
         // ---------------------------------------------------- math warps
+        // warp (qd, hf): TMEM lanes / d_v rows 32 qd .. 32 qd + 31, chunk
+        // positions (and state columns) of half hf
         const int qd = warp & 3, hf = warp >> 2;
         const int i = 32 * qd + lane;                 // d_v row inside the tile
         const uint32_t lb = (uint32_t)(32 * qd) << 16;
-        constexpr int HALF = D / 2;
+        const int sh = 32 * hf;
+        const size_t hoff = (((size_t)seg * p.H + h) * D + dv0 + i) * D;
         bool ok = true;
-        // initial state: h0 (or zeros) -> TMEM (pre-scaled by chunk 0's decay) and bf16 -> s_bf
-        {
-            float sc = 1.f;
-            if (nc > 0) {
-                ok = mbar_wait(bar(GB_FULL), 0, abort_flag, p.err, 20);
-                sc = gbuf[G_EGC];
+        // initial state: rho = 1, T = h0 (or zeros) and its bf16 copy
+        for (int blk = 0; blk < HALF / 64; ++blk) {
+            const int col = hf * HALF + 64 * blk;
+            uint32_t w0[32], w1[32], pk[32];
+#pragma unroll
+            for (int e = 0; e < 64; e += 4) {
+                const float4 f = p.h0 ? *reinterpret_cast<const float4*>(p.h0 + hoff + col + e)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                uint32_t* w = e < 32 ? w0 : w1;
+                const int ee = e & 31;
+                w[ee] = __float_as_uint(f.x); w[ee + 1] = __float_as_uint(f.y);
+                w[ee + 2] = __float_as_uint(f.z); w[ee + 3] = __float_as_uint(f.w);
             }
-            const float* hrow = p.h0 ? p.h0 + (((size_t)seg * p.H + h) * D + dv0 + i) * D : nullptr;
-            for (int blk = 0; blk < HALF / 32 && ok; ++blk) {
-                const int col = hf * HALF + 32 * blk;
-                float v[32];
+            if (nc == 0) {
+                if (p.h_final) {
+                    float* out = p.h_final + hoff + col;
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    float4 f = hrow ? *reinterpret_cast<const float4*>(hrow + col + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[e] = f.x; v[e + 1] = f.y; v[e + 2] = f.z; v[e + 3] = f.w;
-                }
-                if (nc == 0) {
-                    if (p.h_final) {
-                        float* out = p.h_final + (((size_t)seg * p.H + h) * D + dv0 + i) * D + col;
-#pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4*>(out + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    for (int e = 0; e < 32; e += 4) {
+                        *reinterpret_cast<float4*>(out + e) = make_float4(__uint_as_float(w0[e]), __uint_as_float(w0[e + 1]),
+                                                                          __uint_as_float(w0[e + 2]), __uint_as_float(w0[e + 3]));
+                        *reinterpret_cast<float4*>(out + 32 + e) = make_float4(__uint_as_float(w1[e]), __uint_as_float(w1[e + 1]),
+                                                                               __uint_as_float(w1[e + 2]), __uint_as_float(w1[e + 3]));
                     }
-                    continue;
                 }
-                uint32_t w[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(v[e] * sc);
-                tmem_st_x32(tmem + lb + T_S + col, w);
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) pk[e2] = pack_bf16(v[c8 * 8 + 2 * e2], v[c8 * 8 + 2 * e2 + 1]);
-                    const int cc = (col & 63) / 8 + c8;
-                    st_shared_v4(s_bf + (col >> 6) * 16384 + i * 128 + ((cc ^ (i & 7)) << 4), pk);
-                }
+                continue;
             }
-            if (nc > 0) {
-                tmem_st_wait();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(SBF_READY));
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                pk[e] = pack_bf16(__uint_as_float(w0[2 * e]), __uint_as_float(w0[2 * e + 1]));
+                pk[16 + e] = pack_bf16(__uint_as_float(w1[2 * e]), __uint_as_float(w1[2 * e + 1]));
             }
+            tmem_st_x32(tmem + lb + T_S + col, w0);
+            tmem_st_x32(tmem + lb + T_S + col + 32, w1);
+            tmem_st_x32(tmem + lb + T_SB + col / 2, pk);
         }
+        if (nc > 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(SBF_READY));
+        }
+        // this thread's element of V^T: V[s][i] sits in slab i / 64, 16-byte chunk (i % 64) / 8 of row s
+        const uint32_t v_slab = vb + (uint32_t)(i >> 6) * 8192 + (uint32_t)(i & 7) * 2;
+        const uint32_t v_chunk = (uint32_t)((i & 63) >> 3);
         for (int c = 0; c < nc && ok; ++c) {
             const int b = c & 1;
             const float* gb = gbuf + b * GB;
@@ -609,51 +616,59 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             if (!mbar_wait(bar(GB_FULL + b), (c >> 1) & 1, abort_flag, p.err, 21)) break;
             const int n = __float_as_int(gb[G_N]);
             const int64_t r0 = rs0 + (int64_t)c * C;
-            // ---- Z~ = (S K^T) diag(e^gamma) -> bf16 for the U MMA
-            if (!mbar_wait(bar(Z_FULL), ph, abort_flag, p.err, 22)) break;
+            // ---- Y = V^T - Z~,  Z~ = (T K^T) diag(e^gamma / rho)
+            if (!mbar_wait(bar(V_FULL), ph, abort_flag, p.err, 22)) break;
+            uint32_t vv[16];                          // V[s][i] for the 32 positions, bf16 pairs
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+                const int s = sh + e;
+                unsigned short r0s, r1s;
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(r0s) : "r"(v_slab + s * 128 + ((v_chunk ^ (uint32_t)(s & 7)) << 4)));
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(r1s) : "r"(v_slab + (s + 1) * 128 + ((v_chunk ^ (uint32_t)((s + 1) & 7)) << 4)));
+                vv[e / 2] = (uint32_t)r0s | ((uint32_t)r1s << 16);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(V_FREE));
+            if (!mbar_wait(bar(Z_FULL), ph, abort_flag, p.err, 23)) break;
             tc_fence_after();
             {
                 uint32_t z[32];
-                tmem_ld_x32(tmem + lb + T_Z + hf * 32, z);
-                tmem_ld_wait();
+                tmem_ld_x32(tmem + lb + T_ZU + sh, z);
                 float eg[32];
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_EG + hf * 32 + e), eg + e);
+                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_EGR + sh + e), eg + e);
+                tmem_ld_wait();
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
-                    pk[e / 2] = pack_bf16(__uint_as_float(z[e]) * eg[e], __uint_as_float(z[e + 1]) * eg[e + 1]);
+                    pk[e / 2] = pack_bf16(fmaf(-__uint_as_float(z[e]), eg[e], __uint_as_float(vv[e / 2] << 16)),
+                                          fmaf(-__uint_as_float(z[e + 1]), eg[e + 1], __uint_as_float(vv[e / 2] & 0xFFFF0000u)));
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
                     const int cc = hf * 4 + c8;
-                    st_shared_v4(zb + i * 128 + ((cc ^ (i & 7)) << 4), pk + 4 * c8);
+                    st_shared_v4(yb + i * 128 + ((cc ^ (i & 7)) << 4), pk + 4 * c8);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(ZT_READY));
-            // ---- U^T (for the output) and decayed U^T (for the state)
+            // ---- U^T (output term) and U^T diag(G_DEC) (state term)
             if (!mbar_wait(bar(U_FULL), ph, abort_flag, p.err, 24)) break;
-            if (c > 0) {
-                // ub still holds the previous chunk's output tile until its TMA store has read it
-                if (warp == 0 && lane == 0) bulk_wait_read0();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(STAGE_OUT));
-                if (!mbar_wait(bar(STAGE_OUT), (c - 1) & 1, abort_flag, p.err, 28)) break;
-            }
             tc_fence_after();
             {
                 uint32_t u[32];
-                tmem_ld_x32(tmem + lb + T_UO + b * 64 + hf * 32, u);
-                tmem_ld_wait();
+                tmem_ld_x32(tmem + lb + T_ZU + sh, u);
                 float dc[32];
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_DEC + hf * 32 + e), dc + e);
+                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_DEC + sh + e), dc + e);
+                tmem_ld_wait();
                 uint32_t pu[16], pd[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const int s = hf * 32 + e;
+                    const int s = sh + e;
                     const float a0 = s < n ? __uint_as_float(u[e]) : 0.f;
                     const float a1 = s + 1 < n ? __uint_as_float(u[e + 1]) : 0.f;
                     pu[e / 2] = pack_bf16(a0, a1);
@@ -663,119 +678,98 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 for (int c8 = 0; c8 < 4; ++c8) {
                     const int cc = hf * 4 + c8;
                     const uint32_t off = i * 128 + ((cc ^ (i & 7)) << 4);
-                    st_shared_v4(zb + off, pu + 4 * c8);
-                    st_shared_v4(ub + off, pd + 4 * c8);
+                    st_shared_v4(uob + off, pu + 4 * c8);
+                    st_shared_v4(usb + off, pd + 4 * c8);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(U_READY));
-            // ---- state read-back: bf16 copy for the next chunk, pre-scaled fp32 in TMEM
+            // ---- state read-back: the bf16 copy of T for the next chunk (or the final state)
             if (!mbar_wait(bar(S_FULL), ph, abort_flag, p.err, 25)) break;
             tc_fence_after();
-            const bool last = c + 1 == nc;
-            float sc = 1.f;
-            if (!last) {
-                if (!mbar_wait(bar(GB_FULL + (b ^ 1)), ((c + 1) >> 1) & 1, abort_flag, p.err, 26)) break;
-                sc = gbuf[(b ^ 1) * GB + G_EGC];
-            }
-            for (int blk2 = 0; blk2 < HALF / 32; blk2 += 2) {
-              uint32_t svp[2][32];
-              tmem_ld_x32(tmem + lb + T_S + hf * HALF + 32 * blk2, svp[0]);
-              tmem_ld_x32(tmem + lb + T_S + hf * HALF + 32 * blk2 + 32, svp[1]);
-              tmem_ld_wait();
-#pragma unroll
-              for (int u2 = 0; u2 < 2; ++u2) {
-                const int col = hf * HALF + 32 * (blk2 + u2);
-                uint32_t* sv = svp[u2];
-                if (last) {
-                    if (p.h_final) {
-                        float* out = p.h_final + (((size_t)seg * p.H + h) * D + dv0 + i) * D + col;
+            if (c + 1 == nc) {
+                if (p.h_final) {
+                    const float inv = exp2f(-gb[G_LR]);
+                    for (int blk = 0; blk < HALF / 32; ++blk) {
+                        const int col = hf * HALF + 32 * blk;
+                        uint32_t sv[32];
+                        tmem_ld_x32(tmem + lb + T_S + col, sv);
+                        tmem_ld_wait();
+                        float* out = p.h_final + hoff + col;
 #pragma unroll
                         for (int e = 0; e < 32; e += 4)
                             *reinterpret_cast<float4*>(out + e) =
-                                make_float4(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1]),
-                                            __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+                                make_float4(inv * __uint_as_float(sv[e]), inv * __uint_as_float(sv[e + 1]),
+                                            inv * __uint_as_float(sv[e + 2]), inv * __uint_as_float(sv[e + 3]));
                     }
-                    continue;
                 }
+            } else {
+                for (int blk = 0; blk < HALF / 64; ++blk) {
+                    const int col = hf * HALF + 64 * blk;
+                    uint32_t s0[32], s1[32], pk[16];
+                    tmem_ld_x32(tmem + lb + T_S + col, s0);
+                    tmem_ld_x32(tmem + lb + T_S + col + 32, s1);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    uint32_t pk[4];
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(s0[2 * e]), __uint_as_float(s0[2 * e + 1]));
+                    tmem_st_x16(tmem + lb + T_SB + col / 2, pk);
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2)
-                        pk[e2] = pack_bf16(__uint_as_float(sv[c8 * 8 + 2 * e2]), __uint_as_float(sv[c8 * 8 + 2 * e2 + 1]));
-                    const int cc = (col & 63) / 8 + c8;
-                    st_shared_v4(s_bf + (col >> 6) * 16384 + i * 128 + ((cc ^ (i & 7)) << 4), pk);
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(s1[2 * e]), __uint_as_float(s1[2 * e + 1]));
+                    tmem_st_x16(tmem + lb + T_SB + col / 2 + 16, pk);
                 }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) sv[e] = __float_as_uint(__uint_as_float(sv[e]) * sc);
-                tmem_st_x32(tmem + lb + T_S + col, svp[u2]);
-              }
-            }
-            if (!last) {
                 tmem_st_wait();
-                fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(SBF_READY));
             }
-            // ---- output o_r = scale (e^gamma_r S q_r + sum_s P_rs u_s)
-            if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 27)) break;
+            // ---- output o_r = scale (S e^gamma_r q_r + sum_s P_rs u_s), rows r < n
+            if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 26)) break;
             tc_fence_after();
             {
-                uint32_t xr[32], orr[32];
-                tmem_ld_x32(tmem + lb + T_X + hf * 32, xr);
-                tmem_ld_x32(tmem + lb + T_UO + b * 64 + hf * 32, orr);
+                uint32_t xo[32];
+                tmem_ld_x32(tmem + lb + T_XO + sh, xo);
                 tmem_ld_wait();
-                // stage the [64 rows x 128 d_v] output tile row-major in ub
-                const uint32_t stage = ub + i * 2;
-                float eg[32];
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_EG + hf * 32 + e), eg + e);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(XO_FREE));
+                // this warp's [32 rows x 32 d_v] piece, staged row-major, leaves by one TMA store
+                const uint32_t stg = stg0 + warp * 2048 + lane * 2;
+                if (lane == 0) bulk_wait_read0();     // the previous chunk's store has read the piece
+                __syncwarp();
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const int r = hf * 32 + e;
-                    const uint32_t pr = pack_bf16(
-                        p.scale * fmaf(eg[e], __uint_as_float(xr[e]), __uint_as_float(orr[e])),
-                        p.scale * fmaf(eg[e + 1], __uint_as_float(xr[e + 1]), __uint_as_float(orr[e + 1])));
+                    const uint32_t pr = pack_bf16(p.scale * __uint_as_float(xo[e]), p.scale * __uint_as_float(xo[e + 1]));
                     asm volatile("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
                                  "st.shared.b16 [%0], lo;\n\tst.shared.b16 [%1], hi;\n\t}"
-                                 ::"r"(stage + r * DVT * 2), "r"(stage + (r + 1) * DVT * 2), "r"(pr) : "memory");
+                                 ::"r"(stg + e * 64), "r"(stg + (e + 1) * 64), "r"(pr) : "memory");
                 }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(STAGE_IN));
-            if (!mbar_wait(bar(STAGE_IN), c & 1, abort_flag, p.err, 29)) break;
-            if (n == C) {
-                if (warp == 0 && lane == 0) {
-                    tma_store_2d(&tm_o, ub, h * D + dv0, (int)r0);
-                    bulk_commit();
-                }
-            } else {
-                // ragged last chunk: only rows < n belong to this segment
-                const int tid = threadIdx.x;
-                for (int idx = tid; idx < n * (DVT / 8); idx += NMATH * 32) {
-                    const int row = idx / (DVT / 8), ch = idx % (DVT / 8);
-                    const uint4 v = *reinterpret_cast<const uint4*>(sm + Lay::UB + row * DVT * 2 + ch * 16);
-                    *reinterpret_cast<uint4*>(p.o + ((r0 + row) * p.H + h) * D + dv0 + ch * 8) = v;
+                if (sh + 32 <= n) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_o, stg0 + warp * 2048, h * D + dv0 + 32 * qd, (int)(r0 + sh));
+                        bulk_commit();
+                    }
+                } else {
+                    // ragged last chunk: only rows < n belong to this segment
+                    bf16* orow = p.o + (r0 + sh) * (int64_t)p.H * D + (int64_t)h * D + dv0 + i;
+                    const int64_t rstride = (int64_t)p.H * D;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (sh + e < n) orow[e * rstride] = __float2bfloat16_rn(p.scale * __uint_as_float(xo[e]));
                 }
             }
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(UO_FREE + b));
-                mbar_arrive(bar(X_FREE));
-                mbar_arrive(bar(GB_FREE + b));
-            }
+            if (lane == 0) mbar_arrive(bar(GB_FREE + b));
         }
-        if (warp == 0 && lane == 0) bulk_wait0();
+        if (lane == 0) bulk_wait0();
     } else if (warp == W_PROD) {
         // ------------------------------------------ producer: gates + TMA
         bool ok = true;
-        int last_k[2] = {-1, -1}, last_v = -1, last_q = -1, last_t = -1, last_p = -1;
+        int last_k[2] = {-1, -1}, last_v = -1, last_t = -1, last_p = -1;
+        float lr = 0.f;                               // log2 rho at the chunk start
         for (int c = 0; c < nc && ok; ++c) {
             const int b = c & 1;
             const uint32_t ph = c & 1, pb = (c >> 1) & 1;
@@ -787,27 +781,33 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             {
                 float bt[2], gg[2];
                 const float gl = chunk_scan(p, r0, n, h, lane, bt, gg);
+                const float t = lr - gl * LOG2E;      // >= -1/2
+                int e = (int)floorf(t + 0.5f);
+                float lr1 = t - (float)e;
+                if (e > 15) { e = -1; lr1 = 0.f; }
                 float* gb = gbuf + b * GB;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int s = 2 * lane + e;
-                    gb[G_EG + s] = s < n ? __expf(gg[e]) : 0.f;
-                    gb[G_DEC + s] = s < n ? __expf(gl - gg[e]) : 0.f;
+                for (int k = 0; k < 2; ++k) {
+                    const int s = 2 * lane + k;
+                    gb[G_EGR + s] = s < n ? exp2f(gg[k] * LOG2E - lr) : 0.f;
+                    gb[G_DEC + s] = s < n ? exp2f(lr1 + (gl - gg[k]) * LOG2E) : 0.f;
                 }
                 if (lane == 0) {
                     gb[G_N] = __int_as_float(n);
-                    gb[G_EGC] = __expf(gl);
+                    gb[G_SCL] = __int_as_float(e);
+                    gb[G_LR] = lr1;
                 }
+                lr = lr1;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(GB_FULL + b));
-            // K, V (and contiguous Q) tiles
-            const uint32_t kb = kb0 + b * Lay::KSZ;
-            if (!mbar_wait(bar(K_FREE + b), pb ^ 1, abort_flag, p.err, 31)) { ok = false; break; }
+            // K and V tiles
+            const uint32_t kb = kq0 + b * Lay::KQSZ;
+            if (!mbar_wait(bar(KQ_FREE + b), pb ^ 1, abort_flag, p.err, 31)) { ok = false; break; }
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(K_LAND + b), SLABS * 8192);
 #pragma unroll
-                for (int j = 0; j < SLABS; ++j) tma_load_2d(kb + j * 8192, &tm_k, bar(K_LAND + b), h * D + 64 * j, (int)r0);
+                for (int j = 0; j < SLABS; ++j) tma_load_2d(kb + j * 16384, &tm_k, bar(K_LAND + b), h * D + 64 * j, (int)r0);
             }
             last_k[b] = c;
             if (!mbar_wait(bar(V_FREE), ph ^ 1, abort_flag, p.err, 32)) { ok = false; break; }
@@ -817,23 +817,13 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 tma_load_2d(vb + 8192, &tm_v, bar(V_LAND), h * D + dv0 + 64, (int)r0);
             }
             last_v = c;
-            if (!p.qidx) {
-                if (!mbar_wait(bar(Q_FREE), ph ^ 1, abort_flag, p.err, 33)) { ok = false; break; }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bar(Q_FULL), SLABS * 8192);
-#pragma unroll
-                    for (int j = 0; j < SLABS; ++j) tma_load_2d(qb + j * 8192, &tm_q, bar(Q_FULL), h * D + 64 * j, (int)r0);
-                }
-                last_q = c;
-            }
             // zero the key / value rows past n (other segments' data) once they land
             if (!mbar_wait(bar(K_LAND + b), pb, abort_flag, p.err, 34)) { ok = false; break; }
             if (n < C) {
-                const uint4 zero = make_uint4(0, 0, 0, 0);
                 for (int idx = lane; idx < (C - n) * 8 * SLABS; idx += 32) {
                     const int row = n + idx / (8 * SLABS), rest = idx % (8 * SLABS);
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(kb + (rest >> 3) * 8192 + row * 128 + (rest & 7) * 16),
-                                 "r"(zero.x), "r"(zero.y), "r"(zero.z), "r"(zero.w) : "memory");
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(kb + (rest >> 3) * 16384 + row * 128 + (rest & 7) * 16),
+                                 "r"(0u) : "memory");
                 }
                 fence_proxy_async_smem();
             }
@@ -846,7 +836,6 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(vb + (rest >> 3) * 8192 + row * 128 + (rest & 7) * 16),
                                  "r"(0u) : "memory");
                 }
-                fence_proxy_async_smem();
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(V_FULL));
@@ -870,91 +859,96 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             for (int b = 0; b < 2; ++b)
                 if (last_k[b] >= 0) mbar_wait_drain(bar(K_LAND + b), (last_k[b] >> 1) & 1);
             if (last_v >= 0) mbar_wait_drain(bar(V_LAND), last_v & 1);
-            if (last_q >= 0) mbar_wait_drain(bar(Q_FULL), last_q & 1);
             if (last_t >= 0) mbar_wait_drain(bar(T_FULL), last_t & 1);
             if (last_p >= 0) mbar_wait_drain(bar(P_FULL), last_p & 1);
         }
     } else if (warp < W_MMA) {
-        // -------------------------------- gather warps: q rows through qidx
-        if (p.qidx) {
-            const int t = threadIdx.x - (W_PROD + 1) * 32;
-            for (int c = 0; c < nc; ++c) {
-                const int64_t r0 = rs0 + (int64_t)c * C;
-                const int64_t rem = rs1 - r0;
-                const int n = (int)(rem < C ? rem : C);
-                if (!mbar_wait(bar(Q_FREE), (c & 1) ^ 1, abort_flag, p.err, 38)) break;
-                gather_rows<D>(p, p.q, r0, n, h, qb, 8192, t, NGATHER * 32);
-                cp_async_commit();
-                cp_async_wait<0>();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(Q_FULL));
-            }
+        // ------------------- q~ warps: q rows (through the index when given),
+        // then scaled in place by e^gamma_r / rho (the output's state term)
+        const int t = threadIdx.x - (W_PROD + 1) * 32;
+        for (int c = 0; c < nc; ++c) {
+            const int b = c & 1;
+            const uint32_t pb = (c >> 1) & 1;
+            const uint32_t qb = kq0 + b * Lay::KQSZ + 8192;
+            const int64_t r0 = rs0 + (int64_t)c * C;
+            const int64_t rem = rs1 - r0;
+            const int n = (int)(rem < C ? rem : C);
+            if (!mbar_wait(bar(KQ_FREE + b), pb ^ 1, abort_flag, p.err, 38)) break;
+            gather_rows<D>(p, p.q, r0, n, h, qb, 16384, t, NGATHER * 32);
+            cp_async_commit();
+            const bool gates = mbar_wait(bar(GB_FULL + b), pb, abort_flag, p.err, 39);
             cp_async_wait<0>();
+            if (!gates) break;
+            const float* gb = gbuf + b * GB;
+            // the same (row, chunk) assignment as gather_rows: each thread scales what it fetched
+            for (int idx = t; idx < C * 8; idx += NGATHER * 32) {
+                const int row = idx >> 3, c8 = idx & 7;
+                const float f = gb[G_EGR + row];
+                const uint32_t d0 = qb + row * 128 + ((c8 ^ (row & 7)) << 4);
+#pragma unroll
+                for (int j = 0; j < SLABS; ++j) {
+                    uint32_t w[4];
+                    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(d0 + j * 16384));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+                        w[e] = pack_bf16(lo * f, hi * f);
+                    }
+                    st_shared_v4(d0 + j * 16384, w);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(Q_FULL + b));
         }
+        cp_async_wait<0>();
     } else if (lane == 0) {
         // ------------------------------------------------------ MMA issuer
         constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
-        constexpr uint32_t ID64_V = idesc_bf16_f32(128, 64, 1, 0);       // A = V^T (MN-major)
-        constexpr uint32_t ID64_NEG = idesc_bf16_f32(128, 64, 0, 0, 1);  // -A
+        constexpr uint32_t ID128 = idesc_bf16_f32(128, 128);
         constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);           // B = K (MN-major)
         for (int c = 0; c < nc; ++c) {
             const int b = c & 1;
             const uint32_t ph = c & 1, pb = (c >> 1) & 1;
-            const uint32_t kb = kb0 + b * Lay::KSZ;
-            // Z = S K^T
+            const uint32_t kq = kq0 + b * Lay::KQSZ;
+            // [Z | X] = T [K; q~]^T, A = the bf16 copy of T in TMEM
             if (!mbar_wait(bar(K_FULL + b), pb, abort_flag, p.err, 40)) break;
-            if (!mbar_wait(bar(SBF_READY), ph, abort_flag, p.err, 41)) break;
+            if (!mbar_wait(bar(Q_FULL + b), pb, abort_flag, p.err, 41)) break;
+            if (!mbar_wait(bar(SBF_READY), ph, abort_flag, p.err, 42)) break;
+            if (!mbar_wait(bar(XO_FREE), ph ^ 1, abort_flag, p.err, 43)) break;
             tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < SLABS; ++j)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_Z, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
-                             desc_kmajor_sw128(kb + j * 8192 + kk * 32), ID64, (j | kk) != 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+                umma_f16_ts(tmem + T_ZU, tmem + T_SB + 8 * kk, desc_kmajor_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
+                            ID128, kk != 0);
             umma_commit(bar(Z_FULL));
-            // U^T = V^T Tb^T - Z~ Tb^T  into this chunk's U/O buffer
-            const uint32_t uo = tmem + T_UO + b * 64;
-            if (!mbar_wait(bar(V_FULL), ph, abort_flag, p.err, 44)) break;
+            // U^T = Y Tb^T (over Z, which the math warps have read)
+            if (!mbar_wait(bar(ZT_READY), ph, abort_flag, p.err, 44)) break;
             if (!mbar_wait(bar(T_FULL), ph, abort_flag, p.err, 45)) break;
-            if (!mbar_wait(bar(UO_FREE + b), pb ^ 1, abort_flag, p.err, 46)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(uo, desc_mnmajor_sw128(vb + kk * 2048, 8192), desc_kmajor_sw128(timg + kk * 32), ID64_V,
-                         kk != 0);
-            umma_commit(bar(V_FREE));
-            if (!mbar_wait(bar(ZT_READY), ph, abort_flag, p.err, 47)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16(uo, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64_NEG, 1);
+                umma_f16(tmem + T_ZU, desc_kmajor_sw128(yb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64, kk != 0);
             umma_commit(bar(U_FULL));
             umma_commit(bar(T_FREE));
-            // X = S Q^T (only the output needs it: issued while the math warps write U)
-            if (!mbar_wait(bar(Q_FULL), ph, abort_flag, p.err, 42)) break;
-            if (!mbar_wait(bar(X_FREE), ph ^ 1, abort_flag, p.err, 43)) break;
+            // T = 2^-e T + (U^T diag(G_DEC)) K
+            if (!mbar_wait(bar(U_READY), ph, abort_flag, p.err, 46)) break;
             tc_fence_after();
+            const int e = __float_as_int(gbuf[b * GB + G_SCL]);
+            umma_f16_scaled(tmem + T_S, desc_kmajor_sw128(usb), desc_mnmajor_sw128(kq, 16384), IDS, e >= 0 ? 1u : 0u,
+                            e >= 0 ? e : 0);
 #pragma unroll
-            for (int j = 0; j < SLABS; ++j)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_X, desc_kmajor_sw128(s_bf + j * 16384 + kk * 32),
-                             desc_kmajor_sw128(qb + j * 8192 + kk * 32), ID64, (j | kk) != 0);
-            umma_commit(bar(Q_FREE));
-            // S += (decayed U^T) K ; O = U^T P^T
-            if (!mbar_wait(bar(U_READY), ph, abort_flag, p.err, 48)) break;
-            if (!mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 49)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_S, desc_kmajor_sw128(ub + kk * 32), desc_mnmajor_sw128(kb + kk * 2048, 8192), IDS,
-                         1);
+            for (int kk = 1; kk < 4; ++kk)
+                umma_f16(tmem + T_S, desc_kmajor_sw128(usb + kk * 32), desc_mnmajor_sw128(kq + kk * 2048, 16384), IDS, 1);
             umma_commit(bar(S_FULL));
-            umma_commit(bar(K_FREE + b));
+            umma_commit(bar(KQ_FREE + b));
+            // X += U^T P^T
+            if (!mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 47)) break;
+            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(uo, desc_kmajor_sw128(zb + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64, kk != 0);
+                umma_f16(tmem + T_XO, desc_kmajor_sw128(uob + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64, 1);
             umma_commit(bar(O_FULL));
             umma_commit(bar(P_FREE));
         }
@@ -989,15 +983,15 @@ cudaError_t launch_d(const GdnTc& t, int64_t mchunks, cudaStream_t st) {
     if (!make_tma_2d_bf16(&tm_k, t.k, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
     if (!make_tma_2d_bf16(&tm_v, t.v, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
     if (!make_tma_2d_bf16(&tm_q, t.q, (uint64_t)t.n_q_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
-    CUtensorMap tm_o;
-    if (!make_tma_2d_bf16_plain(&tm_o, t.o, (uint64_t)t.n_rows, HD, HD, DVT, C)) return cudaErrorInvalidValue;
     gdn_schedule_kernel<<<1, 1024, 0, st>>>(t.seg_cu, t.n_seg, t.n_rows, t.chunk_cu, t.chunk_info, t.err);
     if (mchunks > 0) {
         dim3 pg((unsigned)mchunks, t.H);
         gdn_prep_kernel<D><<<pg, 128, PrepLayout<D>::BYTES, st>>>(tm_k, tm_q, t);
     }
+    CUtensorMap tm_o;
+    if (!make_tma_2d_bf16_plain(&tm_o, t.o, (uint64_t)t.n_rows, HD, HD, 32, 32)) return cudaErrorInvalidValue;
     gdn_state_kernel<D><<<(unsigned)((int64_t)t.n_seg * t.H * (D / DVT)), STATE_THREADS, StateLayout<D>::BYTES, st>>>(
-        tm_k, tm_v, tm_q, tm_o, t);
+        tm_k, tm_v, tm_o, t);
     count_launches(mchunks > 0 ? 3 : 2);
     return cudaGetLastError();
 }

@@ -29,6 +29,14 @@ cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int 
 cudaError_t launch_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, int dt,
                              int64_t n_tok, int D, int H, float* beta, float* log_alpha, cudaStream_t st);
 
+// skinny.cu: the same two products for bf16 inputs, four threads per token
+// and the weights staged in shared memory (used when skinny_ok holds)
+bool skinny_ok(int dt, int D, int ncol);
+cudaError_t launch_router_skinny(const void* x, const void* w_r, const float* b_r, int64_t n_tok, int D, int M,
+                                 int K, int32_t* idx, float* gate, float* logits, cudaStream_t st);
+cudaError_t launch_gate_skinny(const void* x, const void* w_gate, const float* A, const float* b_a, int64_t n_tok,
+                               int D, int H, float* beta, float* log_alpha, cudaStream_t st);
+
 // permute.cu
 // `err` is the workspace whose header receives device error records;
 // `scratch` (permute_scratch_bytes) holds the tile counts.

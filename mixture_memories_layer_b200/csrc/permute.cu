@@ -11,6 +11,12 @@
 //   bounds : per (memory, sequence), binary search of the memory's rows
 //            (ascending tokens) for the sequence start -> seg_cu
 //
+// When the tile-count table is small (M x tiles <= FUSED_MAX_TABLE) the four
+// steps run as ONE cooperative launch instead: counts, a grid barrier, then
+// every CTA scans the whole table in shared memory (it is a few KB) and
+// scatters its own tiles, and the (memory, sequence) bounds come from the
+// scanned table plus a count over at most one tile -- no binary search.
+//
 // Counts stay on the device: later kernels read mem_offset / seg_cu
 // themselves, so no host synchronisation is needed anywhere in the layer.
 #include "common.cuh"
@@ -150,6 +156,175 @@ __global__ void permute_bounds_kernel(const int32_t* __restrict__ perm_token, co
     seg_cu[i] = lo;
 }
 
+// ----------------------------------------------------------- fused path --
+static constexpr int FUSED_MAX_TABLE = 8192;       // M x tiles entries scanned in shared memory
+static constexpr long long kBarrierCycles = 4000000000LL;
+
+// Grid-wide barrier for a cooperative launch (all CTAs co-resident): one
+// arrival per CTA on a zeroed counter, bounded spin.  False on timeout
+// (recorded as MOM_DEVERR_TIMEOUT).
+__device__ bool grid_barrier(unsigned* counter, unsigned target, void* ws, int* flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(counter, 1u);
+        const long long t0 = clock64();
+        int ok = 1;
+        for (;;) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+            if (v >= target) break;
+            if (clock64() - t0 > kBarrierCycles) { record_error(ws, MOM_DEVERR_TIMEOUT, -1); ok = 0; break; }
+        }
+        *flag = ok;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
+__global__ void __launch_bounds__(TILE)
+permute_fused_kernel(const int32_t* __restrict__ idx, int64_t n_tok, int K, int M, int n_tiles,
+                     const int32_t* __restrict__ cu_seqlens, int S, int32_t* __restrict__ tile_cnt,
+                     unsigned* __restrict__ counter, int32_t* __restrict__ perm_token, int32_t* __restrict__ row_of,
+                     int32_t* __restrict__ mem_offset, int32_t* __restrict__ seg_cu, void* ws) {
+    extern __shared__ int32_t tab[];                   // M x n_tiles, memory-major
+    __shared__ int cnt[MOM_MAX_MEM];
+    __shared__ int32_t warp_cnt[TILE / 32][MOM_MAX_MEM];
+    __shared__ int32_t part[TILE];
+    __shared__ int flag;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // ---- 1. per-tile counts
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        if (tid < MOM_MAX_MEM) cnt[tid] = 0;
+        __syncthreads();
+        const int64_t t = (int64_t)tile * TILE + tid;
+        if (t < n_tok) {
+            uint32_t bits = token_mem_bits(idx, t, K, M, ws);
+            while (bits) {
+                const int m = __ffs(bits) - 1;
+                bits &= bits - 1;
+                atomicAdd(&cnt[m], 1);
+            }
+        }
+        __syncthreads();
+        if (tid < M) tile_cnt[(int64_t)tid * n_tiles + tile] = cnt[tid];
+    }
+    if (!grid_barrier(counter, gridDim.x, ws, &flag)) return;
+    // ---- 2. exclusive scan of the whole table, memory-major (every CTA)
+    const int L = M * n_tiles;
+    const int per = (L + TILE - 1) / TILE;
+    const int b0 = tid * per, b1 = b0 + per < L ? b0 + per : L;
+    int32_t sum = 0;
+    for (int i = b0; i < b1; ++i) {
+        const int32_t v = __ldcg(tile_cnt + i);
+        tab[i] = v;
+        sum += v;
+    }
+    int32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) part[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t w = lane < TILE / 32 ? part[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += u;
+        }
+        if (lane < TILE / 32) part[TILE / 32 + lane] = w;        // inclusive over warps
+    }
+    __syncthreads();
+    int32_t run = (warp ? part[TILE / 32 + warp - 1] : 0) + incl - sum;
+    for (int i = b0; i < b1; ++i) {
+        const int32_t v = tab[i];
+        tab[i] = run;
+        run += v;
+    }
+    const int32_t total = part[TILE / 32 + TILE / 32 - 1];
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        if (tid < M) mem_offset[tid] = tab[tid * n_tiles];
+        if (tid == 0) mem_offset[M] = total;
+    }
+    // ---- 3. scatter this CTA's tiles (stable: token order inside a memory)
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int64_t t = (int64_t)tile * TILE + tid;
+        const bool live = t < n_tok;
+        uint32_t bits = live ? token_mem_bits(idx, t, K, M, nullptr) : 0u;
+        int32_t my_rank[MOM_MAX_MEM];
+#pragma unroll
+        for (int m = 0; m < MOM_MAX_MEM; ++m) {
+            if (m < M) {
+                const uint32_t bl = __ballot_sync(0xffffffffu, (bits >> m) & 1u);
+                my_rank[m] = __popc(bl & lt);
+                if (lane == 0) warp_cnt[warp][m] = __popc(bl);
+            }
+        }
+        __syncthreads();
+        if (live) {
+            for (int j = 0; j < K; ++j) {
+                const int m = idx[t * K + j];
+                if (m < 0 || m >= M || !((bits >> m) & 1u)) { row_of[t * K + j] = -1; continue; }
+                bits &= ~(1u << m);
+                int32_t r = tab[m * n_tiles + tile];
+                for (int w = 0; w < warp; ++w) r += warp_cnt[w][m];
+                int32_t rk = 0;
+#pragma unroll
+                for (int mm = 0; mm < MOM_MAX_MEM; ++mm) if (mm == m) rk = my_rank[mm];
+                perm_token[r + rk] = (int32_t)t;
+                row_of[t * K + j] = r + rk;
+            }
+        }
+        __syncthreads();
+    }
+    // ---- 4. seg_cu[m S + s] = first row of memory m with token >= cu[s]:
+    // the scanned base of cu[s]'s tile plus a count inside that tile
+    for (int pr = blockIdx.x * (TILE / 32) + warp; pr <= M * S; pr += gridDim.x * (TILE / 32)) {
+        if (pr == M * S) {
+            if (lane == 0) seg_cu[pr] = total;
+            continue;
+        }
+        const int m = pr / S, s = pr % S;
+        const int64_t start = cu_seqlens ? cu_seqlens[s] : (s == 0 ? 0 : n_tok);
+        const int tile = (int)(start / TILE);
+        int32_t base;
+        if (tile < n_tiles) base = tab[m * n_tiles + tile];
+        else base = m + 1 < M ? tab[(m + 1) * n_tiles] : total;
+        int c = 0;
+        for (int q = lane; q < TILE; q += 32) {
+            const int64_t t = (int64_t)tile * TILE + q;
+            if (t < start && t < n_tok) c += (token_mem_bits(idx, t, K, M, nullptr) >> m) & 1u;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (lane == 0) seg_cu[pr] = base + c;
+    }
+}
+
+static int fused_grid(int n_tiles, size_t smem) {
+    static int dev_cached = -1, max_blocks = 0, coop = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev != dev_cached) {
+        int sms = 0, per_sm = 0;
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_fused_kernel, TILE,
+                                                          FUSED_MAX_TABLE * sizeof(int32_t)) != cudaSuccess)
+            per_sm = 0;
+        max_blocks = sms * per_sm;
+        dev_cached = dev;
+    }
+    (void)smem;
+    if (!coop || max_blocks <= 0) return 0;
+    return n_tiles < max_blocks ? n_tiles : max_blocks;
+}
+
 size_t permute_scratch_bytes(int64_t n_tok, int M) {
     const int64_t n_tiles = cdiv(n_tok > 0 ? n_tok : 1, TILE);
     return 2 * (size_t)(M * n_tiles) * sizeof(int32_t) + 256;
@@ -161,6 +336,22 @@ cudaError_t launch_permute(const int32_t* idx, int64_t n_tok, int K, int M, cons
     const int n_tiles = (int)cdiv(n_tok > 0 ? n_tok : 1, TILE);
     int32_t* tile_cnt = reinterpret_cast<int32_t*>(scratch);
     int32_t* tile_base = tile_cnt + (size_t)M * n_tiles;
+    if ((int64_t)M * n_tiles <= FUSED_MAX_TABLE) {
+        const size_t smem = (size_t)M * n_tiles * sizeof(int32_t);
+        const int grid = fused_grid(n_tiles, smem);
+        if (grid > 0) {
+            // the barrier counter sits after both tables, in the scratch's slack
+            unsigned* counter = reinterpret_cast<unsigned*>(tile_base + (size_t)M * n_tiles);
+            cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st);
+            if (e != cudaSuccess) return e;
+            void* args[] = {(void*)&idx, (void*)&n_tok, (void*)&K, (void*)&M, (void*)&n_tiles, (void*)&cu_seqlens,
+                            (void*)&S, (void*)&tile_cnt, (void*)&counter, (void*)&perm_token, (void*)&row_of,
+                            (void*)&mem_offset, (void*)&seg_cu, (void*)&ws};
+            e = cudaLaunchCooperativeKernel((const void*)permute_fused_kernel, dim3(grid), dim3(TILE), args, smem, st);
+            count_launches(1);
+            return e;
+        }
+    }
     if (n_tok > 0)
         permute_count_kernel<<<n_tiles, TILE, 0, st>>>(idx, n_tok, K, M, n_tiles, tile_cnt, ws);
     else

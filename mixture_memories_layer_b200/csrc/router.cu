@@ -118,6 +118,7 @@ static int grid_for_tokens(int64_t n_tok, int warps_per_block) {
 cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int dt, int64_t n_tok, int D,
                           int M, int K, int32_t* idx, float* gate, float* logits, cudaStream_t st) {
     if (n_tok == 0) return cudaSuccess;
+    if (skinny_ok(dt, D, M)) return launch_router_skinny(x, w_r, b_r, n_tok, D, M, K, idx, gate, logits, st);
     dim3 grid(grid_for_tokens(n_tok, 8)), block(256);
     if (dt == MOM_BF16) {
         if (M <= 8)
@@ -141,6 +142,7 @@ cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int 
 cudaError_t launch_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, int dt,
                              int64_t n_tok, int D, int H, float* beta, float* log_alpha, cudaStream_t st) {
     if (n_tok == 0) return cudaSuccess;
+    if (skinny_ok(dt, D, 2 * H)) return launch_gate_skinny(x, w_gate, A, b_a, n_tok, D, H, beta, log_alpha, st);
     dim3 grid(grid_for_tokens(n_tok, 8)), block(256);
     if (dt == MOM_BF16)
         gate_proj_kernel<bf16><<<grid, block, 0, st>>>((const bf16*)x, (const bf16*)w_gate, A, b_a, n_tok, D, H, beta, log_alpha);

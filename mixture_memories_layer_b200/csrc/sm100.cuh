@@ -157,6 +157,42 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
           "r"(mask0), "r"(mask1), "r"(mask2), "r"(mask3)
         : "memory");
 }
+// The same with A read from tensor memory: a [128 x K] K-major bf16 matrix,
+// row m in lane m, elements 2j and 2j+1 of a row packed in column j (low
+// half first); one K = 16 step spans 8 columns from `a_tmem`.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D = A B + 2^-S D (S = 0..15, an immediate): the accumulator is scaled by a
+// power of two as it is read (ignored when `accumulate` is 0).
+template <int S>
+__device__ __forceinline__ void umma_f16_scale_imm(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p, %5;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(S)
+        : "memory");
+}
+__device__ __forceinline__ void umma_f16_scaled(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate, int s) {
+    switch (s) {
+#define MOM_SCALED_CASE(S) case S: umma_f16_scale_imm<S>(d_tmem, adesc, bdesc, idesc, accumulate); break;
+        MOM_SCALED_CASE(0) MOM_SCALED_CASE(1) MOM_SCALED_CASE(2) MOM_SCALED_CASE(3)
+        MOM_SCALED_CASE(4) MOM_SCALED_CASE(5) MOM_SCALED_CASE(6) MOM_SCALED_CASE(7)
+        MOM_SCALED_CASE(8) MOM_SCALED_CASE(9) MOM_SCALED_CASE(10) MOM_SCALED_CASE(11)
+        MOM_SCALED_CASE(12) MOM_SCALED_CASE(13) MOM_SCALED_CASE(14)
+#undef MOM_SCALED_CASE
+        default: umma_f16_scale_imm<15>(d_tmem, adesc, bdesc, idesc, accumulate); break;
+    }
+}
 // Arrives once on `bar` when every MMA issued so far by this thread completes.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -188,6 +224,14 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[
           "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
           "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
           "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }

@@ -137,9 +137,15 @@ class MoMLayer:
         return b
 
     def _side_stream(self):
+        """The shared memory's GDN runs here.  Its segments are the whole
+        sequences (twice or more the routed segments' length), so its state
+        walk is the longest serial chain of the layer: a higher-priority
+        stream lets its CTAs take SMs first while the routed work fills the
+        rest."""
         s = getattr(self, "_side", None)
         if s is None:
-            s = self._side = torch.cuda.Stream(device=self.device)
+            lo, hi = torch.cuda.Stream.priority_range()
+            s = self._side = torch.cuda.Stream(device=self.device, priority=hi)
         return s
 
     def device_errors(self):
