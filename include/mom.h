@@ -224,6 +224,34 @@ mom_status mom_gdn_chunk_fwd(const void* q, const int32_t* qidx, const void* k, 
                              const float* h0, float* h_final, void* o,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* The same call in two stream-ordered halves, for callers that schedule
+ * several GDN problems (the layer's shared memory and its routed memories)
+ * against each other:
+ *   mom_gdn_chunk_prep  -- the state-independent work of every chunk (the
+ *                          within-chunk triangular solve and decay masks),
+ *                          left in ws;
+ *   mom_gdn_chunk_state -- the serial walk over each segment's chunks, which
+ *                          reads what the prep left in ws and writes o and
+ *                          h_final.
+ * Both take exactly the arguments of mom_gdn_chunk_fwd; the state call must
+ * follow a prep call with the same arguments and ws (on the same stream, or
+ * ordered after it by an event), and ws must not be reused in between.
+ * prep followed by state is mom_gdn_chunk_fwd.  When the float32 token-serial
+ * path runs (MOM_F32, or a shape the tensor-core path does not take) prep does
+ * nothing and state does everything. */
+mom_status mom_gdn_chunk_prep(const void* q, const int32_t* qidx, const void* k, const void* v,
+                              const float* beta, const float* log_alpha,
+                              const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                              int H, int d, float scale, mom_dtype dt,
+                              const float* h0, float* h_final, void* o,
+                              void* ws, size_t ws_bytes, void* stream);
+mom_status mom_gdn_chunk_state(const void* q, const int32_t* qidx, const void* k, const void* v,
+                               const float* beta, const float* log_alpha,
+                               const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                               int H, int d, float scale, mom_dtype dt,
+                               const float* h0, float* h_final, void* o,
+                               void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * mom_combine_unpermute -- the combine (paper card, Summary: outputs are
  * combined using the router weights; blog post, "硬件高效實現": summing the

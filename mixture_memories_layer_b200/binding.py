@@ -38,6 +38,10 @@ SIGNATURES = {
     "mom_gdn_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
     "mom_gdn_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I,
                                _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_gdn_chunk_prep": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I,
+                               _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_gdn_chunk_state": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I,
+                               _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mom_combine_unpermute": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
     "mom_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "mom_decode_step": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -166,12 +170,24 @@ def mom_gdn_workspace_size(n_rows, n_seg, H, d, dt):
     return lib.mom_gdn_workspace_size(n_rows, n_seg, H, d, dt)
 
 
-def mom_gdn_chunk_fwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream=None):
+def _gdn(name, q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream):
     n_rows, H, d = k.shape
-    _check(lib.mom_gdn_chunk_fwd(_p(q), _p(qidx), _p(k), _p(v), _p(beta), _p(log_alpha), _p(seg_cu),
-                                 seg_cu.numel() - 1, n_rows, q.shape[0], H, d, float(scale),
-                                 dtype_code(k.dtype), _p(h0), _p(h_final), _p(o), _p(ws), ws.numel(),
-                                 _s(stream)), "mom_gdn_chunk_fwd")
+    _check(getattr(lib, name)(_p(q), _p(qidx), _p(k), _p(v), _p(beta), _p(log_alpha), _p(seg_cu),
+                              seg_cu.numel() - 1, n_rows, q.shape[0], H, d, float(scale),
+                              dtype_code(k.dtype), _p(h0), _p(h_final), _p(o), _p(ws), ws.numel(),
+                              _s(stream)), name)
+
+
+def mom_gdn_chunk_fwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream=None):
+    _gdn("mom_gdn_chunk_fwd", q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream)
+
+
+def mom_gdn_chunk_prep(q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream=None):
+    _gdn("mom_gdn_chunk_prep", q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream)
+
+
+def mom_gdn_chunk_state(q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream=None):
+    _gdn("mom_gdn_chunk_state", q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream)
 
 
 def mom_combine_unpermute(o_sh, o_p, row_of, topk_gate, out, ws, stream=None):

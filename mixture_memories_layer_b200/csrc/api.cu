@@ -96,7 +96,7 @@ size_t mom_kv_proj_workspace_size(int64_t n_tok, int d_model, int H, int d, int 
 
 static mom_status run_projections(const ProjArgs& a, const void* w_gate, const float* A, const float* b_a,
                                   int dt, float* beta, float* log_alpha, cudaStream_t st) {
-    cudaError_t e = launch_gate_proj(a.x, w_gate, A, b_a, dt, a.n_tok, a.D, a.H, beta, log_alpha, st);
+    cudaError_t e = launch_gate_proj(a.x, w_gate, A, b_a, dt, a.n_tok, a.D, a.H, beta, log_alpha, a.ws, st);
     if (e != cudaSuccess) return MOM_ERR_CUDA;
     if (proj_tc_supported(a, dt)) e = launch_proj_tc(a, st);
     else e = launch_proj_simt(a, dt, st);
@@ -130,12 +130,10 @@ size_t mom_gdn_workspace_size(int64_t n_rows, int n_seg, int H, int d, mom_dtype
     return MOM_WS_HEADER_BYTES + up256(extra);
 }
 
-mom_status mom_gdn_chunk_fwd(const void* q, const int32_t* qidx, const void* k, const void* v,
-                             const float* beta, const float* log_alpha,
-                             const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
-                             int H, int d, float scale, mom_dtype dt,
-                             const float* h0, float* h_final, void* o,
-                             void* ws, size_t ws_bytes, void* stream) {
+static mom_status gdn_call(const void* q, const int32_t* qidx, const void* k, const void* v, const float* beta,
+                           const float* log_alpha, const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                           int H, int d, float scale, mom_dtype dt, const float* h0, float* h_final, void* o,
+                           void* ws, size_t ws_bytes, void* stream, int phase) {
     if (!dt_ok(dt) || n_seg < 0 || n_rows < 0 || n_q_rows < 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
     if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < mom_gdn_workspace_size(n_rows, n_seg, H, d, dt)) return MOM_ERR_ARG;
@@ -149,9 +147,40 @@ mom_status mom_gdn_chunk_fwd(const void* q, const int32_t* qidx, const void* k, 
     }
     GdnArgs a{q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale,
               h0, h_final, o, ws, ws_bytes};
+    a.phase = phase;
     cudaStream_t st = as_stream(stream);
     if (gdn_tc_supported(a, dt)) return cuda_status(launch_gdn_tc(a, st));
     return cuda_status(launch_gdn_recurrent(a, dt, st));
+}
+
+mom_status mom_gdn_chunk_fwd(const void* q, const int32_t* qidx, const void* k, const void* v,
+                             const float* beta, const float* log_alpha,
+                             const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                             int H, int d, float scale, mom_dtype dt,
+                             const float* h0, float* h_final, void* o,
+                             void* ws, size_t ws_bytes, void* stream) {
+    return gdn_call(q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, dt, h0, h_final, o,
+                    ws, ws_bytes, stream, GDN_PREP | GDN_STATE);
+}
+
+mom_status mom_gdn_chunk_prep(const void* q, const int32_t* qidx, const void* k, const void* v,
+                              const float* beta, const float* log_alpha,
+                              const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                              int H, int d, float scale, mom_dtype dt,
+                              const float* h0, float* h_final, void* o,
+                              void* ws, size_t ws_bytes, void* stream) {
+    return gdn_call(q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, dt, h0, h_final, o,
+                    ws, ws_bytes, stream, GDN_PREP);
+}
+
+mom_status mom_gdn_chunk_state(const void* q, const int32_t* qidx, const void* k, const void* v,
+                               const float* beta, const float* log_alpha,
+                               const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                               int H, int d, float scale, mom_dtype dt,
+                               const float* h0, float* h_final, void* o,
+                               void* ws, size_t ws_bytes, void* stream) {
+    return gdn_call(q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, dt, h0, h_final, o,
+                    ws, ws_bytes, stream, GDN_STATE);
 }
 
 // ----------------------------------------------------------------- combine

@@ -12,69 +12,114 @@
 
 namespace mom {
 
-// One thread per 8 output elements, no loop: the router slots' rows and
-// gates are read first, then the shared output and all K memory rows are
-// in flight together (top_k <= KMAX per pass).
-template <typename T, int KMAX>
-__global__ void __launch_bounds__(256, 4)
+// One warp per token row, persistent: the warp reads the token's K row
+// indices and gates once, then every lane has its CH 16-byte pieces of the
+// shared output and of all K memory rows in flight together before any
+// arithmetic.
+// 8 consecutive elements as loaded (bf16: one 16-byte vector; f32: two),
+// converted to fp32 only at the FMA.
+template <typename T> struct Piece;
+template <> struct Piece<bf16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const bf16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ float at(int e) const {
+        const uint32_t w = e < 2 ? u.x : e < 4 ? u.y : e < 6 ? u.z : u.w;
+        return __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
+    }
+};
+template <> struct Piece<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ float at(int e) const {
+        const float4& f = e < 4 ? a : b;
+        const int k = e & 3;
+        return k == 0 ? f.x : k == 1 ? f.y : k == 2 ? f.z : f.w;
+    }
+};
+
+template <typename T, int KMAX, int CH>
+__global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ o_sh, const T* __restrict__ o_p, const int32_t* __restrict__ row_of,
                const float* __restrict__ gate, int64_t n_tok, int K, int HD, T* __restrict__ out, void* ws) {
-    const int per_tok = HD / 8;
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n_tok * per_tok) return;
+    const int lane = threadIdx.x & 31;
     const int64_t n_rows = n_tok * K;
-    const int64_t t = i / per_tok;
-    const int c = (int)(i % per_tok) * 8;
-    float acc[8];
-    load_vec<8>(o_sh + t * HD + c, acc);
-    for (int j0 = 0; j0 < K; j0 += KMAX) {
-        int64_t r[KMAX];
-        float g[KMAX];
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < n_tok; t += warps) {
+        for (int c0 = 0; c0 < HD; c0 += 8 * 32 * CH) {
+            Piece<T> sh[CH];
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            r[j] = -1;
-            g[j] = 0.f;
-            if (j0 + j < K) {
-                r[j] = __ldg(row_of + t * K + j0 + j);
-                g[j] = __ldg(gate + t * K + j0 + j);
-                if (r[j] < 0 || r[j] >= n_rows) {
-                    record_error(ws, MOM_DEVERR_ROW_INDEX, t);
-                    r[j] = -1;
-                }
+            for (int q = 0; q < CH; ++q) {
+                const int c = c0 + 8 * (lane + 32 * q);
+                if (c < HD) sh[q].load(o_sh + t * HD + c);
             }
-        }
-        float v[KMAX][8];
+            float acc[CH][8];
+            bool first = true;
+            for (int j0 = 0; j0 < K; j0 += KMAX) {       // one pass when K <= KMAX
+                int64_t r[KMAX];
+                float g[KMAX];
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (r[j] >= 0) load_vec<8>(o_p + r[j] * HD + c, v[j]);
-        }
+                for (int j = 0; j < KMAX; ++j) {
+                    r[j] = -1;
+                    g[j] = 0.f;
+                    if (j0 + j < K) {
+                        r[j] = __ldg(row_of + t * K + j0 + j);
+                        g[j] = __ldg(gate + t * K + j0 + j);
+                        if (r[j] < 0 || r[j] >= n_rows) {
+                            if (lane == 0 && c0 == 0) record_error(ws, MOM_DEVERR_ROW_INDEX, t);
+                            r[j] = -1;
+                        }
+                    }
+                }
+                Piece<T> v[KMAX][CH];
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (r[j] >= 0) {
+                for (int q = 0; q < CH; ++q) {
+                    const int c = c0 + 8 * (lane + 32 * q);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = fmaf(g[j], v[j][e], acc[e]);
+                    for (int j = 0; j < KMAX; ++j)
+                        if (r[j] >= 0 && c < HD) v[j][q].load(o_p + r[j] * HD + c);
+                }
+#pragma unroll
+                for (int q = 0; q < CH; ++q) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float a = first ? sh[q].at(e) : acc[q][e];
+#pragma unroll
+                        for (int j = 0; j < KMAX; ++j)
+                            if (r[j] >= 0) a = fmaf(g[j], v[j][q].at(e), a);
+                        acc[q][e] = a;
+                    }
+                }
+                first = false;
+            }
+#pragma unroll
+            for (int q = 0; q < CH; ++q) {
+                const int c = c0 + 8 * (lane + 32 * q);
+                if (c < HD) store_vec<8>(out + t * HD + c, acc[q]);
             }
         }
     }
-    store_vec<8>(out + t * HD + c, acc);
 }
 
 cudaError_t launch_combine(const void* o_sh, const void* o_p, const int32_t* row_of, const float* gate,
                            int64_t n_tok, int K, int H, int d, int dt, void* out, void* ws, cudaStream_t st) {
     if (n_tok == 0) return cudaSuccess;
     const int HD = H * d;
-    const int64_t total = n_tok * (HD / 8);
-    const unsigned g = (unsigned)cdiv(total, 256);
+    int64_t g = cdiv(n_tok, 8);                 // 8 warps (tokens) per CTA
+    if (g > 148 * 8) g = 148 * 8;
+    const dim3 grid((unsigned)g), block(256);
     if (dt == MOM_BF16) {
         if (K <= 2)
-            combine_kernel<bf16, 2><<<g, 256, 0, st>>>((const bf16*)o_sh, (const bf16*)o_p, row_of, gate, n_tok, K, HD, (bf16*)out, ws);
+            combine_kernel<bf16, 2, 4><<<grid, block, 0, st>>>((const bf16*)o_sh, (const bf16*)o_p, row_of, gate, n_tok, K, HD, (bf16*)out, ws);
         else
-            combine_kernel<bf16, 4><<<g, 256, 0, st>>>((const bf16*)o_sh, (const bf16*)o_p, row_of, gate, n_tok, K, HD, (bf16*)out, ws);
+            combine_kernel<bf16, 4, 2><<<grid, block, 0, st>>>((const bf16*)o_sh, (const bf16*)o_p, row_of, gate, n_tok, K, HD, (bf16*)out, ws);
     } else {
         if (K <= 2)
-            combine_kernel<float, 2><<<g, 256, 0, st>>>((const float*)o_sh, (const float*)o_p, row_of, gate, n_tok, K, HD, (float*)out, ws);
+            combine_kernel<float, 2, 2><<<grid, block, 0, st>>>((const float*)o_sh, (const float*)o_p, row_of, gate, n_tok, K, HD, (float*)out, ws);
         else
-            combine_kernel<float, 4><<<g, 256, 0, st>>>((const float*)o_sh, (const float*)o_p, row_of, gate, n_tok, K, HD, (float*)out, ws);
+            combine_kernel<float, 4, 1><<<grid, block, 0, st>>>((const float*)o_sh, (const float*)o_p, row_of, gate, n_tok, K, HD, (float*)out, ws);
     }
     count_launches(1);
     return cudaGetLastError();

@@ -967,7 +967,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 int64_t max_chunks(int64_t n_rows, int n_seg) { return n_rows / C + n_seg; }
 
 template <int D>
-cudaError_t launch_d(const GdnTc& t, int64_t mchunks, cudaStream_t st) {
+cudaError_t launch_d(const GdnTc& t, int64_t mchunks, int phase, cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -983,16 +983,24 @@ cudaError_t launch_d(const GdnTc& t, int64_t mchunks, cudaStream_t st) {
     if (!make_tma_2d_bf16(&tm_k, t.k, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
     if (!make_tma_2d_bf16(&tm_v, t.v, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
     if (!make_tma_2d_bf16(&tm_q, t.q, (uint64_t)t.n_q_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;
-    gdn_schedule_kernel<<<1, 1024, 0, st>>>(t.seg_cu, t.n_seg, t.n_rows, t.chunk_cu, t.chunk_info, t.err);
-    if (mchunks > 0) {
-        dim3 pg((unsigned)mchunks, t.H);
-        gdn_prep_kernel<D><<<pg, 128, PrepLayout<D>::BYTES, st>>>(tm_k, tm_q, t);
+    int launched = 0;
+    if (phase & GDN_PREP) {
+        gdn_schedule_kernel<<<1, 1024, 0, st>>>(t.seg_cu, t.n_seg, t.n_rows, t.chunk_cu, t.chunk_info, t.err);
+        ++launched;
+        if (mchunks > 0) {
+            dim3 pg((unsigned)mchunks, t.H);
+            gdn_prep_kernel<D><<<pg, 128, PrepLayout<D>::BYTES, st>>>(tm_k, tm_q, t);
+            ++launched;
+        }
     }
-    CUtensorMap tm_o;
-    if (!make_tma_2d_bf16_plain(&tm_o, t.o, (uint64_t)t.n_rows, HD, HD, 32, 32)) return cudaErrorInvalidValue;
-    gdn_state_kernel<D><<<(unsigned)((int64_t)t.n_seg * t.H * (D / DVT)), STATE_THREADS, StateLayout<D>::BYTES, st>>>(
-        tm_k, tm_v, tm_o, t);
-    count_launches(mchunks > 0 ? 3 : 2);
+    if (phase & GDN_STATE) {
+        CUtensorMap tm_o;
+        if (!make_tma_2d_bf16_plain(&tm_o, t.o, (uint64_t)t.n_rows, HD, HD, 32, 32)) return cudaErrorInvalidValue;
+        gdn_state_kernel<D><<<(unsigned)((int64_t)t.n_seg * t.H * (D / DVT)), STATE_THREADS, StateLayout<D>::BYTES,
+                              st>>>(tm_k, tm_v, tm_o, t);
+        ++launched;
+    }
+    count_launches(launched);
     return cudaGetLastError();
 }
 
@@ -1038,7 +1046,7 @@ cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st) {
     base += up256((size_t)mc * sizeof(int4));
     t.img = base;
     t.err = a.ws;
-    return a.d == 256 ? launch_d<256>(t, mc, st) : launch_d<128>(t, mc, st);
+    return a.d == 256 ? launch_d<256>(t, mc, a.phase, st) : launch_d<128>(t, mc, a.phase, st);
 }
 
 }  // namespace mom

@@ -105,6 +105,7 @@ static cudaError_t launch_t(const GdnArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_gdn_recurrent(const GdnArgs& a, int dt, cudaStream_t st) {
+    if (!(a.phase & GDN_STATE)) return cudaSuccess;   // token-serial: nothing to prepare
     if (a.n_seg == 0) return cudaSuccess;
     if (dt == MOM_BF16) {
         switch (a.d) {

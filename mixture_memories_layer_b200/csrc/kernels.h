@@ -27,7 +27,7 @@ bool device_is_sm100();
 cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int dt, int64_t n_tok, int D,
                           int M, int K, int32_t* idx, float* gate, float* logits, cudaStream_t st);
 cudaError_t launch_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, int dt,
-                             int64_t n_tok, int D, int H, float* beta, float* log_alpha, cudaStream_t st);
+                             int64_t n_tok, int D, int H, float* beta, float* log_alpha, void* err, cudaStream_t st);
 
 // skinny.cu: the same two products for bf16 inputs, four threads per token
 // and the weights staged in shared memory (used when skinny_ok holds)
@@ -35,7 +35,7 @@ bool skinny_ok(int dt, int D, int ncol);
 cudaError_t launch_router_skinny(const void* x, const void* w_r, const float* b_r, int64_t n_tok, int D, int M,
                                  int K, int32_t* idx, float* gate, float* logits, cudaStream_t st);
 cudaError_t launch_gate_skinny(const void* x, const void* w_gate, const float* A, const float* b_a, int64_t n_tok,
-                               int D, int H, float* beta, float* log_alpha, cudaStream_t st);
+                               int D, int H, float* beta, float* log_alpha, void* err, cudaStream_t st);
 
 // permute.cu
 // `err` is the workspace whose header receives device error records;
@@ -65,6 +65,7 @@ bool proj_tc_supported(const ProjArgs& a, int dt);
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st);
 
 // gdn_recurrent.cu: token-serial Gated DeltaNet on CUDA cores
+enum GdnPhase { GDN_PREP = 1, GDN_STATE = 2 };
 struct GdnArgs {
     const void* q;
     const int32_t* qidx;
@@ -82,6 +83,9 @@ struct GdnArgs {
     void* o;
     void* ws;
     size_t ws_bytes;
+    // GDN_PREP: the state-independent per-chunk work; GDN_STATE: the serial
+    // walk over the chunks (reads what GDN_PREP left in ws); both by default
+    int phase = GDN_PREP | GDN_STATE;
 };
 cudaError_t launch_gdn_recurrent(const GdnArgs& a, int dt, cudaStream_t st);
 

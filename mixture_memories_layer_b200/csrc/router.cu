@@ -140,9 +140,9 @@ cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int 
 }
 
 cudaError_t launch_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, int dt,
-                             int64_t n_tok, int D, int H, float* beta, float* log_alpha, cudaStream_t st) {
+                             int64_t n_tok, int D, int H, float* beta, float* log_alpha, void* err, cudaStream_t st) {
     if (n_tok == 0) return cudaSuccess;
-    if (skinny_ok(dt, D, 2 * H)) return launch_gate_skinny(x, w_gate, A, b_a, n_tok, D, H, beta, log_alpha, st);
+    if (skinny_ok(dt, D, 2 * H)) return launch_gate_skinny(x, w_gate, A, b_a, n_tok, D, H, beta, log_alpha, err, st);
     dim3 grid(grid_for_tokens(n_tok, 8)), block(256);
     if (dt == MOM_BF16)
         gate_proj_kernel<bf16><<<grid, block, 0, st>>>((const bf16*)x, (const bf16*)w_gate, A, b_a, n_tok, D, H, beta, log_alpha);

@@ -1,7 +1,8 @@
 """One MoM layer on the GPU: the six C-ABI calls in order, with torch used
 only to hold device memory.
 
-    router -> permute -> projections -> GDN (shared) -> GDN (routed) -> combine
+    router -> permute -> projections -> GDN prep (shared, routed)
+           -> GDN state walks (shared | routed, two streams) -> combine
 
 ("MoM: Linear Sequence Modeling with Mixture-of-Memories", Summary; "MoM:
 Mixture-of-Memories Fixes Linear Attention Recall", Router mechanics and
@@ -120,14 +121,23 @@ class MoMLayer:
         mark(3)
         hs = b["h_shared"] if want_states else None
         hm = b["h_mem"] if want_states else None
+        gdn_sh = (b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens,
+                  self.scale, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"])
+        gdn_p = (b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
+                 self.scale, h0_mem, hm, b["o_p"], b["ws_gdn_p"])
+        # both problems' state-independent chunk work first, on the whole GPU;
+        # then the two serial state walks side by side.  The shared memory's
+        # walk (whole sequences: the longest serial chain) is launched first,
+        # on the launching stream, so its CTAs hold SMs before the routed
+        # walks (on the side stream) fill the rest.
+        B.mom_gdn_chunk_prep(*gdn_sh, stream=st)
+        B.mom_gdn_chunk_prep(*gdn_p, stream=st)
         side = self._side_stream()
         fork = torch.cuda.Event()
         fork.record(st)
+        B.mom_gdn_chunk_state(*gdn_sh, stream=st)
         side.wait_event(fork)
-        B.mom_gdn_chunk_fwd(b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens,
-                            self.scale, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"], stream=side)
-        B.mom_gdn_chunk_fwd(b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
-                            self.scale, h0_mem, hm, b["o_p"], b["ws_gdn_p"], stream=st)
+        B.mom_gdn_chunk_state(*gdn_p, stream=side)
         join = torch.cuda.Event()
         join.record(side)
         st.wait_event(join)
@@ -137,15 +147,11 @@ class MoMLayer:
         return b
 
     def _side_stream(self):
-        """The shared memory's GDN runs here.  Its segments are the whole
-        sequences (twice or more the routed segments' length), so its state
-        walk is the longest serial chain of the layer: a higher-priority
-        stream lets its CTAs take SMs first while the routed work fills the
-        rest."""
+        """The routed memories' GDN state walks run here, beside the shared
+        memory's on the launching stream."""
         s = getattr(self, "_side", None)
         if s is None:
-            lo, hi = torch.cuda.Stream.priority_range()
-            s = self._side = torch.cuda.Stream(device=self.device, priority=hi)
+            s = self._side = torch.cuda.Stream(device=self.device)
         return s
 
     def device_errors(self):

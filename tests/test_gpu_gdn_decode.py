@@ -70,6 +70,48 @@ def test_gdn_segments_edge_cases(dt, d):
             assert max_abs_rel(o[a:b], ro) < tol, ("o", s, L)
 
 
+@pytest.mark.parametrize("d", [128, 256])
+def test_gdn_prep_then_state_equals_fwd(d):
+    """mom_gdn_chunk_prep followed by mom_gdn_chunk_state (here on two
+    streams ordered by an event, with another problem's prep in between)
+    writes exactly what mom_gdn_chunk_fwd writes."""
+    rng = np.random.default_rng(5 + d)
+    H = 2
+    seg_lens = [130, 0, 64, 200, 3]
+    seg_cu = np.concatenate([[0], np.cumsum(seg_lens)]).astype(np.int32)
+    n_rows = int(seg_cu[-1])
+    q, k, v, beta, la = _gdn_inputs(rng, n_rows, n_rows, H, d)
+    h0 = rng.standard_normal((len(seg_lens), H, d, d)) * 0.1
+    g = lambda a, t=torch.bfloat16: torch.as_tensor(np.ascontiguousarray(a)).to("cuda", t)
+    args = [g(q), None, g(k), g(v), g(beta, torch.float32), g(la, torch.float32), g(seg_cu, torch.int32), 1.0,
+            g(h0, torch.float32)]
+    code = B.dtype_code(torch.bfloat16)
+    outs = []
+    for split in (False, True):
+        o = torch.zeros((n_rows, H, d), dtype=torch.bfloat16, device="cuda")
+        hf = torch.zeros((len(seg_lens), H, d, d), dtype=torch.float32, device="cuda")
+        ws = B.new_workspace(B.mom_gdn_workspace_size(n_rows, len(seg_lens), H, d, code))
+        if split:
+            other_o = torch.zeros_like(o)
+            other_ws = B.new_workspace(B.mom_gdn_workspace_size(n_rows, len(seg_lens), H, d, code))
+            B.mom_gdn_chunk_prep(*args, hf, o, ws)
+            B.mom_gdn_chunk_prep(*args[:8], None, None, other_o, other_ws)
+            side = torch.cuda.Stream()
+            ev = torch.cuda.Event()
+            ev.record(torch.cuda.current_stream())
+            side.wait_event(ev)
+            B.mom_gdn_chunk_state(*args, hf, o, ws, stream=side)
+            B.mom_gdn_chunk_state(*args[:8], None, None, other_o, other_ws)
+            torch.cuda.synchronize()
+        else:
+            B.mom_gdn_chunk_fwd(*args, hf, o, ws)
+            torch.cuda.synchronize()
+        assert B.mom_get_error(ws) == (0, 0)
+        outs.append((to_np(o), to_np(hf)))
+    assert np.array_equal(outs[0][0], outs[1][0])
+    assert np.array_equal(outs[0][1], outs[1][1])
+
+
 def test_device_error_record_on_bad_memory_index():
     """A memory index >= M is recorded and dropped, never read out of bounds."""
     n_tok, K, M = 300, 2, 4
