@@ -307,12 +307,16 @@ __device__ __forceinline__ void offdiag_level(const float* Lm, float* Tm, float*
 
 template <int D>
 struct PrepLayout {
-    static constexpr int KQ = 0;                      // two slabs: K rows 0..63 | Q rows 64..127 (16 KB each)
-    static constexpr int TM = 0;                      // fp32 [64][LP] T, reusing KQ after the MMAs
-    static constexpr int LM = 2 * 16384;              // fp32 [64][LP] L
+    // per 64-column slab: K rows 0..63 | q rows 64..127 (16 KB); after the
+    // MMA has read them, the fp32 work tiles reuse the same bytes
+    static constexpr int KQ = 0;
+    static constexpr int KQ_BYTES = (D / 64) * 16384;
+    static constexpr int TM = 0;                      // fp32 [64][LP] T
+    static constexpr int LM = TM + C * LP * 4;        // fp32 [64][LP] L
     static constexpr int MB = LM + C * LP * 4;        // fp32 3 x [16][16] block products
-    static constexpr int GBB = MB + 3 * 256 * 4;      // beta[64], gamma[64]
-    static constexpr int BARS = GBB + 2 * C * 4;      // land, mma (one phase per pair of slabs)
+    static constexpr int WORK = MB + 3 * 256 * 4;
+    static constexpr int GBB = ((KQ_BYTES > WORK ? KQ_BYTES : WORK) + 15) & ~15;   // beta[64], gamma[64]
+    static constexpr int BARS = GBB + 2 * C * 4;      // land, mma
     static constexpr int MISC = BARS + 16;
     static constexpr size_t BYTES = 1024 + MISC + 16;
 };
@@ -342,74 +346,67 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int64_t r0 = info.y;
     const int n = info.z;
 
-    constexpr int NPH = SLABS / 2 > 0 ? SLABS / 2 : 1;
-    // K (and contiguous Q) of one phase by TMA; rows past n hold other finite data and are masked below
-    auto issue_tma = [&](int ph) {
-        const int j0 = 2 * ph, nj = SLABS - j0 < 2 ? SLABS - j0 : 2;
-        mbar_arrive_expect_tx(land, nj * 8192 * (p.qidx ? 1 : 2));
-        for (int jj = 0; jj < nj; ++jj) {
-            tma_load_2d(kq + jj * 16384, &tm_k, land, h * D + 64 * (j0 + jj), (int)r0);
-            if (!p.qidx) tma_load_2d(kq + jj * 16384 + 8192, &tm_q, land, h * D + 64 * (j0 + jj), (int)r0);
-        }
-    };
+    // Everything the chunk reads is requested at once: K (and contiguous q)
+    // by TMA, indexed q rows by warps 1-3, the gates by warp 0.  Rows past n
+    // hold other finite data and are masked below.
     if (tid == 0) {
         mbar_init(land, 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
-        issue_tma(0);
+        mbar_arrive_expect_tx(land, SLABS * 8192 * (p.qidx ? 1 : 2));
+#pragma unroll
+        for (int j = 0; j < SLABS; ++j) {
+            tma_load_2d(kq + j * 16384, &tm_k, land, h * D + 64 * j, (int)r0);
+            if (!p.qidx) tma_load_2d(kq + j * 16384 + 8192, &tm_q, land, h * D + 64 * j, (int)r0);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tslot), 64);
+        tmem_relinquish();
     }
     if (warp == 0) {
         float b[2], gg[2];
         chunk_scan(p, r0, n, h, lane, b, gg);
         gbeta[2 * lane] = b[0]; gbeta[2 * lane + 1] = b[1];
         ggam[2 * lane] = gg[0]; ggam[2 * lane + 1] = gg[1];
-    }
-    if (warp == 1) {
-        tmem_alloc(smem_u32(tslot), 64);
-        tmem_relinquish();
+    } else if (p.qidx) {
+        gather_rows<D>(p, p.q, r0, n, h, kq + 8192, 16384, tid - 32, 96);
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    // G = [K; Q] K^T : M = 128, N = 64, K = D, two slabs (128 columns of D) per phase.
-    for (int ph = 0; ph < NPH; ++ph) {
-        const int j0 = 2 * ph, nj = SLABS - j0 < 2 ? SLABS - j0 : 2;
-        if (ph > 0 && tid == 0) issue_tma(ph);
-        if (p.qidx) {
-            for (int idx = tid; idx < C * 8; idx += 128) {
-                const int row = idx >> 3, c8 = idx & 7;
-                int64_t src_row = -1;
-                if (row < n) {
-                    const int64_t qr = p.qidx[r0 + row];
-                    src_row = (qr >= 0 && qr < p.n_q_rows) ? qr : -1;
-                }
-                const bf16* src = p.q + ((src_row >= 0 ? src_row : 0) * p.H + h) * D + j0 * 64 + c8 * 8;
-                const uint32_t d0 = kq + 8192 + row * 128 + ((c8 ^ (row & 7)) << 4);
-                for (int jj = 0; jj < nj; ++jj) cp_async_16(d0 + jj * 16384, src + jj * 64, src_row >= 0 ? 16u : 0u);
-            }
-            cp_async_commit();
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-        }
-        mbar_wait(land, ph & 1, abort_flag, p.err, 10);
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t ID = idesc_bf16_f32(128, 64);
-            for (int jj = 0; jj < nj; ++jj)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t a = kq + jj * 16384 + kk * 32;
-                    umma_f16(tmem, desc_kmajor_sw128(a), desc_kmajor_sw128(a), ID, (ph | jj | kk) != 0);
-                }
-            umma_commit(mma_bar);
-        }
-        __syncwarp();
-        mbar_wait(mma_bar, ph & 1, abort_flag, p.err, 11);   // the buffer is free again
+    // G = [K; q] K^T : M = 128, N = 64, K = D
+    mbar_wait(land, 0, abort_flag, p.err, 10);
+    __syncthreads();
+    bool ok = *abort_flag == 0;                           // uniform after the barrier
+    if (!ok) mbar_wait_drain(land, 0);                    // copies in flight land before we leave
+    if (ok && tid == 0) {
         tc_fence_after();
+        constexpr uint32_t ID = idesc_bf16_f32(128, 64);
+#pragma unroll
+        for (int j = 0; j < SLABS; ++j)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t a = kq + j * 16384 + kk * 32;
+                umma_f16(tmem, desc_kmajor_sw128(a), desc_kmajor_sw128(a), ID, (j | kk) != 0);
+            }
+        umma_commit(mma_bar);
+    }
+    if (ok) {
+        if (!mbar_wait(mma_bar, 0, abort_flag, p.err, 11)) mbar_wait_drain(mma_bar, 0);   // K/q bytes free again
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*abort_flag) {
+        if (warp == 1) tmem_dealloc(tmem, 64);
+        return;
     }
     uint32_t ga[32], gc[32];
     const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
@@ -462,7 +459,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 enum Bar {
     GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, Q_FULL = 8, KQ_FREE = 10,
     V_LAND = 12, V_FULL, V_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
-    SBF_READY, Z_FULL, ZT_READY, U_FULL, U_READY, S_FULL, O_FULL, XO_FREE, DONE, NBARS
+    SBF_LO, SBF_HI, Z_FULL, U_FULL, S_FULL, O_FULL, XO_FREE, DONE,
+    DRAIN0, NBARS = DRAIN0 + 8          // one per math warp (NMATH)
 };
 
 constexpr int NMATH = 8;              // math warps 0..7
@@ -470,6 +468,7 @@ constexpr int W_PROD = 8;             // producer warp (TMA, gates, tail zeroing
 constexpr int NGATHER = 3;            // q~ warps 9..11 (q rows, possibly through the index, scaled in place)
 constexpr int W_MMA = 12;             // MMA warp
 constexpr int STATE_THREADS = 13 * 32;
+static_assert(NMATH == 8, "one drain barrier per math warp");
 constexpr float LOG2E = 1.4426950408889634f;
 
 // Gate record of one chunk.  TMEM holds T = rho S with rho = 2^lr a running
@@ -502,6 +501,14 @@ struct StateLayout {
     static constexpr size_t BYTES = 1024 + MISC + 16;
 };
 
+// Arrival on a math-warp hand-off counter (acquire-release, CTA scope);
+// true for the warp that completes the round of NMATH arrivals.
+__device__ __forceinline__ bool last_arrival(uint32_t counter) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(counter) : "memory");
+    return old % NMATH == NMATH - 1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -520,6 +527,9 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::BARS);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lay::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+    // arrival counters of the math warps' hand-offs: the last warp to finish
+    // Y (resp. U) issues the U (resp. state-update and output) MMAs itself
+    const uint32_t cnt_y = smem_u32(tslot + 2), cnt_u = smem_u32(tslot + 3);
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const uint32_t kq0 = smem_u32(sm + Lay::KQ0), vb = smem_u32(sm + Lay::VB);
     const uint32_t timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB), yb = smem_u32(sm + Lay::YB);
@@ -540,10 +550,12 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int counts[NBARS];
         for (int i = 0; i < NBARS; ++i) counts[i] = 1;
         counts[GB_FREE] = counts[GB_FREE + 1] = NMATH;
-        counts[V_FREE] = counts[SBF_READY] = counts[ZT_READY] = counts[U_READY] = counts[XO_FREE] = NMATH;
+        counts[V_FREE] = counts[SBF_LO] = counts[SBF_HI] = counts[XO_FREE] = NMATH;
         counts[Q_FULL] = counts[Q_FULL + 1] = NGATHER;
         for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), counts[i]);
         *abort_flag = 0;
+        tslot[2] = 0;
+        tslot[3] = 0;
         fence_barrier_init();
     }
     if (warp == W_MMA) {
@@ -604,8 +616,12 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(SBF_READY));
+            if (lane == 0) {
+                mbar_arrive(bar(SBF_LO));
+                mbar_arrive(bar(SBF_HI));
+            }
         }
+        bool issued = false;                          // this warp's lane 0 issued MMAs
         // this thread's element of V^T: V[s][i] sits in slab i / 64, 16-byte chunk (i % 64) / 8 of row s
         const uint32_t v_slab = vb + (uint32_t)(i >> 6) * 8192 + (uint32_t)(i & 7) * 2;
         const uint32_t v_chunk = (uint32_t)((i & 63) >> 3);
@@ -654,7 +670,20 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ZT_READY));
+            if (lane == 0 && last_arrival(cnt_y)) {
+                // U^T = Y Tb^T, over Z (which every math warp has read)
+                if (mbar_wait(bar(T_FULL), ph, abort_flag, p.err, 43)) {
+                    tc_fence_after();
+                    constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_ZU, desc_kmajor_sw128(yb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64,
+                                 kk != 0);
+                    umma_commit(bar(U_FULL));
+                    umma_commit(bar(T_FREE));
+                    issued = true;
+                }
+            }
             // ---- U^T (output term) and U^T diag(G_DEC) (state term)
             if (!mbar_wait(bar(U_FULL), ph, abort_flag, p.err, 24)) break;
             tc_fence_after();
@@ -685,7 +714,32 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(U_READY));
+            if (lane == 0 && last_arrival(cnt_u)) {
+                tc_fence_after();
+                // T = 2^-e T + (U^T diag(G_DEC)) K, then X += U^T P^T
+                const uint32_t kq = kq0 + b * Lay::KQSZ;
+                constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
+                constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);   // B = K (MN-major)
+                const int e = __float_as_int(gb[G_SCL]);
+                umma_f16_scaled(tmem + T_S, desc_kmajor_sw128(usb), desc_mnmajor_sw128(kq, 16384), IDS,
+                                e >= 0 ? 1u : 0u, e >= 0 ? e : 0);
+#pragma unroll
+                for (int kk = 1; kk < 4; ++kk)
+                    umma_f16(tmem + T_S, desc_kmajor_sw128(usb + kk * 32), desc_mnmajor_sw128(kq + kk * 2048, 16384),
+                             IDS, 1);
+                umma_commit(bar(S_FULL));
+                umma_commit(bar(KQ_FREE + b));
+                issued = true;
+                if (mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 47)) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_XO, desc_kmajor_sw128(uob + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64,
+                                 1);
+                    umma_commit(bar(O_FULL));
+                    umma_commit(bar(P_FREE));
+                }
+            }
             // ---- state read-back: the bf16 copy of T for the next chunk (or the final state)
             if (!mbar_wait(bar(S_FULL), ph, abort_flag, p.err, 25)) break;
             tc_fence_after();
@@ -706,23 +760,25 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     }
                 }
             } else {
-                for (int blk = 0; blk < HALF / 64; ++blk) {
-                    const int col = hf * HALF + 64 * blk;
-                    uint32_t s0[32], s1[32], pk[16];
-                    tmem_ld_x32(tmem + lb + T_S + col, s0);
-                    tmem_ld_x32(tmem + lb + T_S + col + 32, s1);
-                    tmem_ld_wait();
+                // first d_k half (both warps of the lane quarter share it), then the
+                // second: the Z | X product starts on the first half meanwhile
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(s0[2 * e]), __uint_as_float(s0[2 * e + 1]));
-                    tmem_st_x16(tmem + lb + T_SB + col / 2, pk);
+                for (int part = 0; part < 2; ++part) {
+                    for (int blk = 0; blk < HALF / 64; ++blk) {
+                        const int col = part * HALF + hf * (HALF / 2) + 32 * blk;
+                        uint32_t s0[32], pk[16];
+                        tmem_ld_x32(tmem + lb + T_S + col, s0);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(s1[2 * e]), __uint_as_float(s1[2 * e + 1]));
-                    tmem_st_x16(tmem + lb + T_SB + col / 2 + 16, pk);
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack_bf16(__uint_as_float(s0[2 * e]), __uint_as_float(s0[2 * e + 1]));
+                        tmem_st_x16(tmem + lb + T_SB + col / 2, pk);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(part ? SBF_HI : SBF_LO));
                 }
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(SBF_READY));
             }
             // ---- output o_r = scale (S e^gamma_r q_r + sum_s P_rs u_s), rows r < n
             if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 26)) break;
@@ -764,7 +820,16 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(GB_FREE + b));
         }
-        if (lane == 0) bulk_wait0();
+        if (lane == 0) {
+            bulk_wait0();
+            // MMAs this lane issued complete before TMEM is freed (already so unless
+            // the walk aborted): a commit to this warp's own barrier, whose only
+            // phase completes when they have
+            if (issued) {
+                umma_commit(bar(DRAIN0 + warp));
+                mbar_wait_drain(bar(DRAIN0 + warp), 0);
+            }
+        }
     } else if (warp == W_PROD) {
         // ------------------------------------------ producer: gates + TMA
         bool ok = true;
@@ -905,52 +970,29 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         cp_async_wait<0>();
     } else if (lane == 0) {
         // ------------------------------------------------------ MMA issuer
-        constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
         constexpr uint32_t ID128 = idesc_bf16_f32(128, 128);
-        constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);           // B = K (MN-major)
         for (int c = 0; c < nc; ++c) {
             const int b = c & 1;
             const uint32_t ph = c & 1, pb = (c >> 1) & 1;
             const uint32_t kq = kq0 + b * Lay::KQSZ;
-            // [Z | X] = T [K; q~]^T, A = the bf16 copy of T in TMEM
+            // [Z | X] = T [K; q~]^T, A = the bf16 copy of T in TMEM: the first
+            // d_k half as soon as its copy is ready, then the second
             if (!mbar_wait(bar(K_FULL + b), pb, abort_flag, p.err, 40)) break;
             if (!mbar_wait(bar(Q_FULL + b), pb, abort_flag, p.err, 41)) break;
-            if (!mbar_wait(bar(SBF_READY), ph, abort_flag, p.err, 42)) break;
             if (!mbar_wait(bar(XO_FREE), ph ^ 1, abort_flag, p.err, 43)) break;
+            if (!mbar_wait(bar(SBF_LO), ph, abort_flag, p.err, 42)) break;
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
+            for (int kk = 0; kk < D / 32; ++kk)
                 umma_f16_ts(tmem + T_ZU, tmem + T_SB + 8 * kk, desc_kmajor_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
                             ID128, kk != 0);
+            if (!mbar_wait(bar(SBF_HI), ph, abort_flag, p.err, 44)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = D / 32; kk < D / 16; ++kk)
+                umma_f16_ts(tmem + T_ZU, tmem + T_SB + 8 * kk, desc_kmajor_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
+                            ID128, 1);
             umma_commit(bar(Z_FULL));
-            // U^T = Y Tb^T (over Z, which the math warps have read)
-            if (!mbar_wait(bar(ZT_READY), ph, abort_flag, p.err, 44)) break;
-            if (!mbar_wait(bar(T_FULL), ph, abort_flag, p.err, 45)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_ZU, desc_kmajor_sw128(yb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64, kk != 0);
-            umma_commit(bar(U_FULL));
-            umma_commit(bar(T_FREE));
-            // T = 2^-e T + (U^T diag(G_DEC)) K
-            if (!mbar_wait(bar(U_READY), ph, abort_flag, p.err, 46)) break;
-            tc_fence_after();
-            const int e = __float_as_int(gbuf[b * GB + G_SCL]);
-            umma_f16_scaled(tmem + T_S, desc_kmajor_sw128(usb), desc_mnmajor_sw128(kq, 16384), IDS, e >= 0 ? 1u : 0u,
-                            e >= 0 ? e : 0);
-#pragma unroll
-            for (int kk = 1; kk < 4; ++kk)
-                umma_f16(tmem + T_S, desc_kmajor_sw128(usb + kk * 32), desc_mnmajor_sw128(kq + kk * 2048, 16384), IDS, 1);
-            umma_commit(bar(S_FULL));
-            umma_commit(bar(KQ_FREE + b));
-            // X += U^T P^T
-            if (!mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 47)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_XO, desc_kmajor_sw128(uob + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64, 1);
-            umma_commit(bar(O_FULL));
-            umma_commit(bar(P_FREE));
         }
         umma_commit(bar(DONE));
         mbar_wait_drain(bar(DONE), 0);

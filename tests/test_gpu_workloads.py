@@ -107,3 +107,25 @@ def test_mom1p3b_m16_full_size():
     _routing_and_permute(w, p, res)
     _projections_sampled(w, p, res, n=128, seed=2)
     _sequence(w, p, res, s=2, max_tokens=384)
+
+
+def test_no_wait_runs_to_its_limit():
+    """Every wait inside the kernels is bounded (about two seconds) and a wait
+    that gives up while tearing down leaves no error record: a layer forward
+    far below that bound shows that none of them ran out."""
+    from mixture_memories_layer_b200 import layer as L
+    w = synth.WORKLOADS["mom380m"]
+    p = synth.make_problem(w)
+    lay = L.MoMLayer(L.pack_weights(p, torch.bfloat16), w.heads, w.d_head, w.top_k)
+    x = torch.as_tensor(p["x"]).cuda().bfloat16()
+    cu = torch.as_tensor(p["cu_seqlens"]).cuda()
+    lay.forward(x, cu)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        lay.forward(x, cu)
+    e1.record()
+    torch.cuda.synchronize()
+    assert e0.elapsed_time(e1) < 200.0, e0.elapsed_time(e1)
+    assert lay.device_errors() == {}
