@@ -189,32 +189,46 @@ __device__ __forceinline__ void gather_rows(const GdnTc& p, const bf16* base, in
 }
 
 // ----------------------------------------------------------------- prep --
-// Row r of L = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r < n, else 0) from
-// the G row held in registers (ga: columns 0..31, gc: 32..63).  Values are
-// computed before any store so the gamma loads pipeline.
-__device__ __forceinline__ void prep_l_row(int r, int n, const float* __restrict__ gam, const float* __restrict__ bet,
+// The decay matrix D_rs = e^(gamma_r - gamma_s) = prod_{t=s+1..r} alpha_t
+// (s <= r, else 0) of one chunk into Dm ([64][LP] fp32), by running products
+// instead of one exponential per entry: thread (r, half) walks s downwards
+// over its half of the columns, multiplying by alpha_s; the lower half starts
+// from e^(gamma_r - gamma_31).  Underflow goes to 0 gracefully.
+__device__ __forceinline__ void prep_decay(int tid, const float* __restrict__ gam, const float* __restrict__ alpha,
+                                           float* __restrict__ Dm) {
+    const int r = tid & 63, half = tid >> 6;
+    const int s_hi = 32 * half + 31;
+    float d = (r > s_hi) ? __expf(gam[r] - gam[s_hi]) : 1.f;
+    float* row = Dm + r * LP;
+#pragma unroll
+    for (int j = 31; j >= 0; --j) {
+        const int s = 32 * half + j;
+        row[s] = s <= r ? d : 0.f;
+        if (s <= r) d *= alpha[s];
+    }
+}
+
+// Row r of L = beta_r D_rs k_r.k_s (s < r < n, else 0) from the G row held
+// in registers (ga: columns 0..31, gc: 32..63).
+__device__ __forceinline__ void prep_l_row(int r, int n, const float* __restrict__ drow, const float* __restrict__ bet,
                                            const uint32_t (&ga)[32], const uint32_t (&gc)[32],
                                            float* __restrict__ lrow) {
-    const float gr = gam[r], br = bet[r];
-    float v[32];
+    const float br = r < n ? bet[r] : 0.f;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int s = 32 * half + e;
             const float G = __uint_as_float(half ? gc[e] : ga[e]);
-            v[e] = (s < r && r < n) ? br * __expf(gr - gam[s]) * G : 0.f;
+            lrow[s] = s < r ? br * drow[s] * G : 0.f;
         }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) lrow[32 * half + e] = v[e];
     }
 }
 
-// Row r of P = e^(gamma_r - gamma_s) q_r.k_s (s <= r < n, else 0), bf16,
-// written into the 128-byte-swizzled 64 x 64 image.
-__device__ __forceinline__ void prep_p_row(int r, int n, const float* __restrict__ gam, const uint32_t (&ga)[32],
+// Row r of P = D_rs q_r.k_s (s <= r < n, else 0), bf16, written into the
+// 128-byte-swizzled 64 x 64 image.
+__device__ __forceinline__ void prep_p_row(int r, int n, const float* __restrict__ drow, const uint32_t (&ga)[32],
                                            const uint32_t (&gc)[32], unsigned char* __restrict__ pimg) {
-    const float gr = gam[r];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         uint32_t w[16];
@@ -225,7 +239,7 @@ __device__ __forceinline__ void prep_p_row(int r, int n, const float* __restrict
             for (int u = 0; u < 2; ++u) {
                 const int s = 32 * half + e + u;
                 const float G = __uint_as_float(half ? gc[e + u] : ga[e + u]);
-                pv[u] = (s <= r && r < n) ? __expf(gr - gam[s]) * G : 0.f;
+                pv[u] = (r < n) ? drow[s] * G : 0.f;       // drow is 0 past the diagonal
             }
             w[e / 2] = pack_bf16(pv[0], pv[1]);
         }
@@ -258,49 +272,67 @@ __device__ __forceinline__ void prep_tb_row(int r, int half, const float* __rest
     }
 }
 
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// d (16 x 8, fp32) += A (16 x 8 at a, row pitch LP) * B (8 x 8 at b, row pitch
+// pb): one m16n8k8 tf32 tensor-core product with fp32 accumulation.
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const float* a, const float* b, int pb, int lane) {
+    const int g = lane >> 2, c = lane & 3;
+    const uint32_t a0 = to_tf32(a[g * LP + c]), a1 = to_tf32(a[(g + 8) * LP + c]);
+    const uint32_t a2 = to_tf32(a[g * LP + c + 4]), a3 = to_tf32(a[(g + 8) * LP + c + 4]);
+    const uint32_t b0 = to_tf32(b[c * pb + g]), b1 = to_tf32(b[(c + 4) * pb + g]);
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // One level of the blocked inverse: the 16 x 16 blocks at distance LEV below
 // the diagonal, T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj (i = j + LEV), from the
-// blocks closer to the diagonal.  128 threads; trip counts are compile-time so
-// each thread's independent elements overlap their load latencies.
+// blocks closer to the diagonal.  The 16 x 16 block products run on the
+// tensor cores (tf32 operands, fp32 accumulation; T is rounded to bf16 for
+// its use anyway): a task is one 8-column half of one block, spread over
+// the 4 warps.
 template <int LEV>
 __device__ __forceinline__ void offdiag_level(const float* Lm, float* Tm, float* Mb, int tid) {
-    constexpr int NB = 4 - LEV, PER = NB * 256 / 128;
-    float acc[PER];
+    constexpr int NB = 4 - LEV;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    // M_q = sum_kb L[bi][bj+kb] T[bj+kb][bj]        (bi = LEV + q, bj = q)
+    for (int task = warp; task < 2 * NB; task += 4) {
+        const int q = task >> 1, nh = task & 1;
+        const int bi = LEV + q, bj = q;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int q = 0; q < PER; ++q) {
-        const int e = tid + 128 * q;
-        const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
-        const int bi = LEV + qb, bj = qb;
-        float sacc = 0.f;
+        for (int kb = 0; kb < LEV; ++kb)
 #pragma unroll
-        for (int kb = 0; kb < LEV; ++kb) {
-            const float* Lr = Lm + (16 * bi + a) * LP + 16 * (bj + kb);
-            const float* Tc = Tm + (16 * (bj + kb)) * LP + 16 * bj + c;
-#pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) sacc = fmaf(Lr[s2], Tc[s2 * LP], sacc);
-        }
-        acc[q] = sacc;
+            for (int ks = 0; ks < 2; ++ks)
+                mma_tf32_16x8x8(d, Lm + (16 * bi) * LP + 16 * (bj + kb) + 8 * ks,
+                                Tm + (16 * (bj + kb) + 8 * ks) * LP + 16 * bj + 8 * nh, LP, lane);
+        float* m = Mb + q * 256;
+        m[g * 16 + 8 * nh + 2 * c] = d[0];
+        m[g * 16 + 8 * nh + 2 * c + 1] = d[1];
+        m[(g + 8) * 16 + 8 * nh + 2 * c] = d[2];
+        m[(g + 8) * 16 + 8 * nh + 2 * c + 1] = d[3];
     }
-#pragma unroll
-    for (int q = 0; q < PER; ++q) Mb[tid + 128 * q] = acc[q];
     __syncthreads();
+    // T[bi][bj] = -T[bi][bi] M_q
+    for (int task = warp; task < 2 * NB; task += 4) {
+        const int q = task >> 1, nh = task & 1;
+        const int bi = LEV + q, bj = q;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int q = 0; q < PER; ++q) {
-        const int e = tid + 128 * q;
-        const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
-        const int bi = LEV + qb;
-        const float* Tr = Tm + (16 * bi + a) * LP + 16 * bi;
-        const float* Mc = Mb + qb * 256 + c;
-        float sacc = 0.f;
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) sacc = fmaf(Tr[s2], Mc[s2 * 16], sacc);
-        acc[q] = -sacc;
-    }
-#pragma unroll
-    for (int q = 0; q < PER; ++q) {
-        const int e = tid + 128 * q;
-        const int qb = e >> 8, a = (e >> 4) & 15, c = e & 15;
-        Tm[(16 * (LEV + qb) + a) * LP + 16 * qb + c] = acc[q];
+        for (int ks = 0; ks < 2; ++ks)
+            mma_tf32_16x8x8(d, Tm + (16 * bi) * LP + 16 * bi + 8 * ks, Mb + q * 256 + (8 * ks) * 16 + 8 * nh, 16, lane);
+        float* t = Tm + (16 * bi) * LP + 16 * bj + 8 * nh;
+        t[g * LP + 2 * c] = -d[0];
+        t[g * LP + 2 * c + 1] = -d[1];
+        t[(g + 8) * LP + 2 * c] = -d[2];
+        t[(g + 8) * LP + 2 * c + 1] = -d[3];
     }
     __syncthreads();
 }
@@ -311,12 +343,12 @@ struct PrepLayout {
     // MMA has read them, the fp32 work tiles reuse the same bytes
     static constexpr int KQ = 0;
     static constexpr int KQ_BYTES = (D / 64) * 16384;
-    static constexpr int TM = 0;                      // fp32 [64][LP] T
+    static constexpr int TM = 0;                      // fp32 [64][LP] T (first the decay matrix D)
     static constexpr int LM = TM + C * LP * 4;        // fp32 [64][LP] L
     static constexpr int MB = LM + C * LP * 4;        // fp32 3 x [16][16] block products
     static constexpr int WORK = MB + 3 * 256 * 4;
-    static constexpr int GBB = ((KQ_BYTES > WORK ? KQ_BYTES : WORK) + 15) & ~15;   // beta[64], gamma[64]
-    static constexpr int BARS = GBB + 2 * C * 4;      // land, mma
+    static constexpr int GBB = ((KQ_BYTES > WORK ? KQ_BYTES : WORK) + 15) & ~15;   // beta, gamma, alpha [64]
+    static constexpr int BARS = GBB + 3 * C * 4;      // land, mma
     static constexpr int MISC = BARS + 16;
     static constexpr size_t BYTES = 1024 + MISC + 16;
 };
@@ -333,6 +365,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     float* Mb = reinterpret_cast<float*>(sm + Lay::MB);
     float* gbeta = reinterpret_cast<float*>(sm + Lay::GBB);
     float* ggam = gbeta + C;
+    float* galpha = ggam + C;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::BARS);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lay::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
@@ -370,6 +403,10 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         chunk_scan(p, r0, n, h, lane, b, gg);
         gbeta[2 * lane] = b[0]; gbeta[2 * lane + 1] = b[1];
         ggam[2 * lane] = gg[0]; ggam[2 * lane + 1] = gg[1];
+        // alpha_s = e^(gamma_s - gamma_{s-1}) (rows past n: gamma is flat there, alpha = 1)
+        const float gprev = __shfl_up_sync(0xffffffffu, gg[1], 1);
+        galpha[2 * lane] = lane ? __expf(gg[0] - gprev) : 1.f;
+        galpha[2 * lane + 1] = __expf(gg[1] - gg[0]);
     } else if (p.qidx) {
         gather_rows<D>(p, p.q, r0, n, h, kq + 8192, 16384, tid - 32, 96);
         cp_async_commit();
@@ -416,8 +453,10 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     unsigned char* img = p.img + ((size_t)g * p.H + h) * 2 * IMG;
     const int r = tid & 63;
-    if (tid < 64) prep_l_row(r, n, ggam, gbeta, ga, gc, Lm + r * LP);
-    else prep_p_row(r, n, ggam, ga, gc, img + IMG);
+    prep_decay(tid, ggam, galpha, Tm);                    // D in T's bytes (T comes later)
+    __syncthreads();
+    if (tid < 64) prep_l_row(r, n, Tm + r * LP, gbeta, ga, gc, Lm + r * LP);
+    else prep_p_row(r, n, Tm + r * LP, ga, gc, img + IMG);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
