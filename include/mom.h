@@ -186,6 +186,9 @@ mom_status mom_permute_noalloc(const int32_t* topk_idx, int64_t n_tok, int top_k
  * float32; k_p, v_p [n_tok*top_k, H, d] (dt).  Rows of k_p / v_p past
  * mem_offset[n_mem] are not written.  Requires d in {64, 128, 256},
  * d_model % 64 == 0.  ws: mom_kv_proj_workspace_size().
+ * beta and log_alpha may both be NULL (w_gate, A, b_a then unused): the
+ * gates are left to mom_gate_proj, which needs no routing and can run on
+ * another stream while the router and the reordering run.
  * ---------------------------------------------------------------------- */
 size_t mom_kv_proj_workspace_size(int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k);
 mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
@@ -194,6 +197,18 @@ mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const i
                                int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k,
                                void* q, void* k_sh, void* v_sh, float* beta, float* log_alpha,
                                void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_gate_proj -- the per-token gates of the memories alone (the Gated
+ * DeltaNet gating every memory uses: blog post, experiments section):
+ *   beta = sigmoid(x W_beta^T),  log_alpha = -exp(A) * softplus(x W_a^T + b_a)
+ * x [n_tok, d_model] (dt), w_gate [2*H, d_model] = rows W_beta | W_a, A and
+ * b_a [H] float32; beta, log_alpha [n_tok, H] float32.  The same values
+ * mom_kv_proj_grouped writes when given beta / log_alpha.
+ * ws: mom_gate_proj_workspace_size(). */
+size_t mom_gate_proj_workspace_size(int64_t n_tok, int d_model, int H);
+mom_status mom_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, mom_dtype dt,
+                         int64_t n_tok, int d_model, int H, float* beta, float* log_alpha,
+                         void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * mom_gdn_chunk_fwd -- the Gated DeltaNet recurrence of one memory over

@@ -33,6 +33,8 @@ SIGNATURES = {
     "mom_permute": (_I, [_VP, _I64, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mom_permute_noalloc": (_I, [_VP, _I64, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
     "mom_kv_proj_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I]),
+    "mom_gate_proj_workspace_size": (_SZ, [_I64, _I, _I]),
+    "mom_gate_proj": (_I, [_VP, _VP, _VP, _VP, _I, _I64, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
     "mom_kv_proj_grouped": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
                                  _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mom_gdn_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
@@ -164,6 +166,17 @@ def mom_kv_proj_grouped(x, perm_token, mem_offset, w_shared, w_gate, A, b_a, w_k
                                    _p(w_kv), dtype_code(x.dtype), n_tok, d_model, H, d, w_kv.shape[0], top_k,
                                    _p(q), _p(k_sh), _p(v_sh), _p(beta), _p(log_alpha), _p(k_p), _p(v_p),
                                    _p(ws), ws.numel(), _s(stream)), "mom_kv_proj_grouped")
+
+
+def mom_gate_proj_workspace_size(n_tok, d_model, H):
+    return lib.mom_gate_proj_workspace_size(n_tok, d_model, H)
+
+
+def mom_gate_proj(x, w_gate, A, b_a, beta, log_alpha, ws, stream=None):
+    n_tok, d_model = x.shape
+    H = A.shape[0]
+    _check(lib.mom_gate_proj(_p(x), _p(w_gate), _p(A), _p(b_a), dtype_code(x.dtype), n_tok, d_model, H,
+                             _p(beta), _p(log_alpha), _p(ws), ws.numel(), _s(stream)), "mom_gate_proj")
 
 
 def mom_gdn_workspace_size(n_rows, n_seg, H, d, dt):

@@ -94,14 +94,6 @@ size_t mom_kv_proj_workspace_size(int64_t n_tok, int d_model, int H, int d, int 
     return MOM_WS_HEADER_BYTES;
 }
 
-static mom_status run_projections(const ProjArgs& a, const void* w_gate, const float* A, const float* b_a,
-                                  int dt, float* beta, float* log_alpha, cudaStream_t st) {
-    cudaError_t e = launch_gate_proj(a.x, w_gate, A, b_a, dt, a.n_tok, a.D, a.H, beta, log_alpha, a.ws, st);
-    if (e != cudaSuccess) return MOM_ERR_CUDA;
-    if (proj_tc_supported(a, dt)) e = launch_proj_tc(a, st);
-    else e = launch_proj_simt(a, dt, st);
-    return cuda_status(e);
-}
 
 mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
                                const void* w_shared, const void* w_gate, const float* A, const float* b_a,
@@ -115,13 +107,42 @@ mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const i
     if (n_tok * top_k >= ((int64_t)1 << 31)) return MOM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < mom_kv_proj_workspace_size(n_tok, d_model, H, d, n_mem, top_k)) return MOM_ERR_ARG;
     if (n_tok == 0) return MOM_OK;
-    const void* ptrs[] = {x, perm_token, mem_offset, w_shared, w_gate, A, b_a, w_kv, q, k_sh, v_sh, beta,
-                          log_alpha, k_p, v_p};
+    const void* ptrs[] = {x, perm_token, mem_offset, w_shared, w_kv, q, k_sh, v_sh, k_p, v_p};
     for (const void* p : ptrs)
         if (!p || !al16(p)) return MOM_ERR_ARG;
+    // the gates are optional here (both NULL: the caller runs mom_gate_proj)
+    const bool gates = beta || log_alpha;
+    if (gates) {
+        const void* gp[] = {w_gate, A, b_a, beta, log_alpha};
+        for (const void* p : gp)
+            if (!p || !al16(p)) return MOM_ERR_ARG;
+    }
     ProjArgs a{x, perm_token, mem_offset, w_shared, w_kv, n_tok, d_model, H, d, n_mem, top_k,
                q, k_sh, v_sh, k_p, v_p, ws};
-    return run_projections(a, w_gate, A, b_a, dt, beta, log_alpha, as_stream(stream));
+    cudaStream_t st = as_stream(stream);
+    if (gates) {
+        cudaError_t e = launch_gate_proj(x, w_gate, A, b_a, dt, n_tok, d_model, H, beta, log_alpha, ws, st);
+        if (e != cudaSuccess) return MOM_ERR_CUDA;
+    }
+    return cuda_status(proj_tc_supported(a, dt) ? launch_proj_tc(a, st) : launch_proj_simt(a, dt, st));
+}
+
+size_t mom_gate_proj_workspace_size(int64_t n_tok, int d_model, int H) {
+    (void)n_tok; (void)d_model; (void)H;
+    return MOM_WS_HEADER_BYTES;
+}
+
+mom_status mom_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, mom_dtype dt,
+                         int64_t n_tok, int d_model, int H, float* beta, float* log_alpha,
+                         void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || d_model <= 0 || d_model % 8 != 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < mom_gate_proj_workspace_size(n_tok, d_model, H)) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {x, w_gate, A, b_a, beta, log_alpha};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    return cuda_status(launch_gate_proj(x, w_gate, A, b_a, dt, n_tok, d_model, H, beta, log_alpha, ws,
+                                        as_stream(stream)));
 }
 
 // --------------------------------------------------------- chunked GDN
@@ -265,8 +286,10 @@ mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_mod
     if (e != cudaSuccess) return MOM_ERR_CUDA;
     ProjArgs pa{x, perm, mem_off, w->w_shared, w->w_kv, B, d_model, H, d, n_mem, top_k,
                 base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, ws};
-    mom_status s = run_projections(pa, w->w_gate, w->A, w->b_a, dt, beta, la, st);
-    if (s != MOM_OK) return s;
+    e = launch_gate_proj(x, w->w_gate, w->A, w->b_a, dt, B, d_model, H, beta, la, ws, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    e = proj_tc_supported(pa, dt) ? launch_proj_tc(pa, st) : launch_proj_simt(pa, dt, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
     DecodeArgs da{base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, beta, la, gate,
                   idx, row_of, B, H, d, n_mem, top_k, scale, state, out, ws};
     return cuda_status(launch_decode_state(da, dt, st));

@@ -41,9 +41,19 @@ class MoMLayer:
     """Holds packed weights and reusable buffers for one layer shape."""
 
     def __init__(self, weights: Dict[str, torch.Tensor], heads: int, d_head: int, top_k: int,
-                 scale: float = 1.0):
+                 scale: float = 1.0, gdn_schedule: str = "auto"):
+        """gdn_schedule: "phased" (both problems' GDN prep, then both state
+        walks), "streams" (each problem's prep and walk on its own stream) or
+        "auto": streams for top_k <= 2, where the shared memory's walk is a
+        large share of the work, phased otherwise (measured on B200 with the
+        380M-shape and 1.3B-shape layers)."""
         self.w = weights
         self.H, self.d, self.top_k, self.scale = heads, d_head, top_k, scale
+        if gdn_schedule == "auto":
+            gdn_schedule = "streams" if top_k <= 2 else "phased"
+        if gdn_schedule not in ("phased", "streams"):
+            raise ValueError("gdn_schedule must be 'auto', 'phased' or 'streams'")
+        self.gdn_schedule = gdn_schedule
         self.n_mem, self.d_model = weights["w_r"].shape
         self.dtype = weights["w_r"].dtype
         self.device = weights["w_r"].device
@@ -87,6 +97,7 @@ class MoMLayer:
         dtc = B.dtype_code(dt)
         b["ws_perm"] = self._ws("perm", B.mom_permute_workspace_size(n_tok, K, M, n_seq))
         b["ws_proj"] = self._ws("proj", B.mom_kv_proj_workspace_size(n_tok, self.d_model, H, d, M, K))
+        b["ws_gate"] = self._ws("gate", B.mom_gate_proj_workspace_size(n_tok, self.d_model, H))
         b["ws_gdn_sh"] = self._ws("gdn_sh", B.mom_gdn_workspace_size(n_tok, n_seq, H, d, dtc))
         b["ws_gdn_p"] = self._ws("gdn_p", B.mom_gdn_workspace_size(n_tok * K, M * n_seq, H, d, dtc))
         b["ws_comb"] = self._ws("comb", B.MOM_WS_HEADER_BYTES)
@@ -101,23 +112,32 @@ class MoMLayer:
         the buffers dict; ``out`` is the layer output, ``h_shared`` [S,H,d,d]
         and ``h_mem`` [M,S,H,d,d] the final states.  ``marks``: optional list
         of 6 CUDA events, recorded before the first call and after each step
-        of STEPS (per-step timing on the launching stream).  The shared and
-        the routed recurrences are independent: the shared one runs on a side
-        stream joined back before the combine."""
+        of STEPS (per-step timing on the launching stream).  The gates and
+        the routed recurrences run on a side stream joined back before the
+        steps that read them."""
         n_tok = x.shape[0]
         n_seq = cu_seqlens.numel() - 1
         w, b = self.w, self.buffers(n_tok, n_seq)
         st = stream if stream is not None else torch.cuda.current_stream()
         mark = (lambda i: marks[i].record(st)) if marks is not None else (lambda i: None)
+        side = self._side_stream()
         mark(0)
+        # the gates need no routing: they run beside the router and the reordering
+        start = torch.cuda.Event()
+        start.record(st)
+        side.wait_event(start)
+        B.mom_gate_proj(x, w["w_gate"], w["A"], w["b_a"], b["beta"], b["log_alpha"], b["ws_gate"], stream=side)
+        gates_done = torch.cuda.Event()
+        gates_done.record(side)
         B.mom_router_topk(x, w["w_r"], w["b_r"], self.top_k, b["idx"], b["gate"], stream=st)
         mark(1)
         B.mom_permute(b["idx"], self.n_mem, cu_seqlens, b["perm"], b["row_of"], b["mem_offset"], b["seg_cu"],
                       b["ws_perm"], stream=st)
         mark(2)
-        B.mom_kv_proj_grouped(x, b["perm"], b["mem_offset"], w["w_shared"], w["w_gate"], w["A"], w["b_a"],
-                              w["w_kv"], self.H, self.d, self.top_k, b["q"], b["k_sh"], b["v_sh"], b["beta"],
-                              b["log_alpha"], b["k_p"], b["v_p"], b["ws_proj"], stream=st)
+        B.mom_kv_proj_grouped(x, b["perm"], b["mem_offset"], w["w_shared"], None, None, None,
+                              w["w_kv"], self.H, self.d, self.top_k, b["q"], b["k_sh"], b["v_sh"], None,
+                              None, b["k_p"], b["v_p"], b["ws_proj"], stream=st)
+        st.wait_event(gates_done)
         mark(3)
         hs = b["h_shared"] if want_states else None
         hm = b["h_mem"] if want_states else None
@@ -125,19 +145,28 @@ class MoMLayer:
                   self.scale, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"])
         gdn_p = (b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
                  self.scale, h0_mem, hm, b["o_p"], b["ws_gdn_p"])
-        # both problems' state-independent chunk work first, on the whole GPU;
-        # then the two serial state walks side by side.  The shared memory's
-        # walk (whole sequences: the longest serial chain) is launched first,
-        # on the launching stream, so its CTAs hold SMs before the routed
-        # walks (on the side stream) fill the rest.
-        B.mom_gdn_chunk_prep(*gdn_sh, stream=st)
-        B.mom_gdn_chunk_prep(*gdn_p, stream=st)
-        side = self._side_stream()
         fork = torch.cuda.Event()
-        fork.record(st)
-        B.mom_gdn_chunk_state(*gdn_sh, stream=st)
-        side.wait_event(fork)
-        B.mom_gdn_chunk_state(*gdn_p, stream=side)
+        if self.gdn_schedule == "phased":
+            # both problems' state-independent chunk work first, on the whole
+            # GPU; then the two serial walks side by side, the shared memory's
+            # (whole sequences: the longest chain) launched first so that its
+            # CTAs hold SMs before the routed walks fill the rest
+            B.mom_gdn_chunk_prep(*gdn_sh, stream=st)
+            B.mom_gdn_chunk_prep(*gdn_p, stream=st)
+            fork.record(st)
+            B.mom_gdn_chunk_state(*gdn_sh, stream=st)
+            side.wait_event(fork)
+            B.mom_gdn_chunk_state(*gdn_p, stream=side)
+        else:
+            # each problem's prep then walk on its own stream: the shared walk
+            # starts as soon as its (smaller) prep is done, the routed prep
+            # and walks fill the rest of the GPU around it
+            fork.record(st)
+            side.wait_event(fork)
+            B.mom_gdn_chunk_prep(*gdn_sh, stream=st)
+            B.mom_gdn_chunk_state(*gdn_sh, stream=st)
+            B.mom_gdn_chunk_prep(*gdn_p, stream=side)
+            B.mom_gdn_chunk_state(*gdn_p, stream=side)
         join = torch.cuda.Event()
         join.record(side)
         st.wait_event(join)
@@ -147,8 +176,8 @@ class MoMLayer:
         return b
 
     def _side_stream(self):
-        """The routed memories' GDN state walks run here, beside the shared
-        memory's on the launching stream."""
+        """Side stream: the gate projections beside the router and the
+        reordering, and the routed memories' GDN beside the shared memory's."""
         s = getattr(self, "_side", None)
         if s is None:
             s = self._side = torch.cuda.Stream(device=self.device)

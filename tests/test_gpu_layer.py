@@ -149,3 +149,32 @@ def test_projections_match_oracle():
         km, vm = orc.memory_kv(p["x"][perm[rows]], p, m, w.heads, w.d_head)
         assert max_abs_rel(res["k_p"][rows], km) < tol
         assert max_abs_rel(res["v_p"][rows], vm) < tol
+
+
+def test_projections_with_gates_equal_separate_gate_call():
+    """mom_kv_proj_grouped given beta / log_alpha writes exactly what the
+    layer's separate mom_gate_proj call (beside the router) writes, and the
+    same k / v."""
+    from mixture_memories_layer_b200 import binding as B
+    w, p = _small(128, lens=(200, 57))
+    lay, res = run_layer(w, p)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    wt = lay.w
+    x = torch.as_tensor(p["x"]).to("cuda", dt)
+    g = lambda a, t=torch.int32: torch.as_tensor(a).to("cuda", t)
+    n, H, d, K = x.shape[0], w.heads, w.d_head, w.top_k
+    outs = {k: torch.empty((n, H, d), dtype=dt, device="cuda") for k in ("q", "k_sh", "v_sh")}
+    kp = torch.empty((n * K, H, d), dtype=dt, device="cuda")
+    vp = torch.empty_like(kp)
+    beta = torch.empty((n, H), dtype=torch.float32, device="cuda")
+    la = torch.empty_like(beta)
+    ws = B.new_workspace(B.mom_kv_proj_workspace_size(n, w.d_model, H, d, w.n_mem, K))
+    B.mom_kv_proj_grouped(x, g(res["perm"]), g(res["mem_offset"]), wt["w_shared"], wt["w_gate"], wt["A"], wt["b_a"],
+                          wt["w_kv"], H, d, K, outs["q"], outs["k_sh"], outs["v_sh"], beta, la, kp, vp, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(beta.cpu().numpy(), res["beta"])
+    assert np.array_equal(la.cpu().numpy(), res["log_alpha"])
+    for k in ("q", "k_sh", "v_sh"):
+        assert np.array_equal(outs[k].float().cpu().numpy(), res[k])
+    rows = int(res["mem_offset"][-1])
+    assert np.array_equal(kp[:rows].float().cpu().numpy(), res["k_p"][:rows])
