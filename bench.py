@@ -171,43 +171,83 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------ ranks (N > 1)
+class Ranks:
+    """One process per GPU (torchrun's RANK / WORLD_SIZE / LOCAL_RANK).  The
+    layer shards by sequence: every rank runs its own batch and nothing on
+    the data path crosses ranks; the only collectives are a barrier around
+    the timed region and the max over ranks of its duration.  `backend` is
+    "nccl" for the bench and "gloo" for the CPU tests of this plumbing."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=120):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v):
+        if self.world == 1:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=self.device if self.device is not None else "cpu")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def rank_problem(w, rank):
+    """This rank's share of the job: the replicated weights and its own batch
+    of sequences (rank 0: the workload's own tokens; rank r: tokens drawn
+    from the seed w.seed * 1000 + r), so that per-GPU work is fixed as N
+    grows."""
+    from mixture_memories_layer_b200 import synth
+    p = synth.make_problem(w)
+    if rank:
+        p["x"] = synth.make_tokens(w, np.random.default_rng(w.seed * 1000 + rank), w.n_tokens)
+    return p
+
+
+def aggregate_throughput(tokens_per_rank, world, steps, max_total_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (max_total_ms / 1e3)
+
+
 # ------------------------------------------------------------- the GPU arm
 def gpu_arm(args):
     import torch
-    import torch.distributed as dist
 
     from mixture_memories_layer_b200 import binding as B
     from mixture_memories_layer_b200 import layer as L
     from mixture_memories_layer_b200 import synth
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         raise SystemExit("--gpus %d but WORLD_SIZE=%d (launch N>1 with torchrun)" % (args.gpus, world))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    rank = ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     peaks = load_peaks()
     w = synth.WORKLOADS[FWD]
-    # replicated weights; each rank draws its own batch of sequences
-    p = synth.make_problem(w)
-    if rank:
-        p["x"] = synth.make_tokens(w, np.random.default_rng(w.seed * 1000 + rank), w.n_tokens)
+    p = rank_problem(w, rank)
     dt = torch.bfloat16
     lay = L.MoMLayer(L.pack_weights(p, dt, dev), w.heads, w.d_head, w.top_k)
     x = torch.as_tensor(p["x"]).to(dev, dt)
@@ -239,8 +279,7 @@ def gpu_arm(args):
     per_call = {name: sum(marks[s][i].elapsed_time(marks[s][i + 1]) for s in range(args.steps)) / args.steps
                 for i, name in enumerate(L.MoMLayer.STEPS)}
     ms_per_step = total_ms / args.steps
-    tokens_all = w.n_tokens * world * args.steps
-    value = tokens_all / (total_ms / 1e3)
+    value = aggregate_throughput(w.n_tokens, world, args.steps, total_ms)
 
     # ---- roofline of the dominant call
     work = step_work(w)
