@@ -14,16 +14,24 @@
 // corrections.  Every product keeps the d_v rows of S as the MMA's M
 // dimension (128 TMEM lanes): every MMA is M = 128.
 //
-// Three launches per call:
+// Three launches per call, in two stream-ordered phases (the prep of
+// every chunk does not depend on the state):
 //   schedule: chunk offsets of every segment (device-side, no host sync)
-//   prep    : per (chunk, head), independent of the state: G = [K;Q] K^T on
-//             the tensor cores; Tb by blocked (16 x 16) forward substitution
-//             in fp32; the causal decayed P = (Q K^T) o [e^(gamma_r-gamma_s)];
-//             both stored as pre-swizzled bf16 64 x 64 tiles
+//   prep    : per (chunk, head): G = [K;Q] K^T on the tensor cores; the
+//             decay matrix by running products of alpha; T = (I + L)^-1 by
+//             16 x 16 blocks (diagonal blocks by forward substitution in
+//             fp32, off-diagonal block products on tf32 tensor cores);
+//             Tb = T diag(beta) and the causal decayed P = (Q K^T) o D as
+//             pre-swizzled bf16 64 x 64 images
 //   state   : per (segment, head, 128-row d_v tile), the serial walk over the
-//             segment's chunks.  Roles: one producer warp (TMA loads, chunk
-//             gates), three gather warps (cp.async rows of q when it is read
-//             through an index), one MMA thread, eight math warps.
+//             segment's chunks with the state resident in TMEM (T = rho S,
+//             fp32) and its bf16 copy in TMEM as the A operand of
+//             [Z | X] = T [K; q~]^T; the chunk decay is the MMA's
+//             power-of-two accumulator scale plus a change of the running
+//             scalar rho.  Roles: one producer warp (TMA loads, chunk gates),
+//             three q~ warps (q rows, through the index when given, scaled
+//             in place), one MMA warp ([Z | X] in two d_k halves), eight math
+//             warps (the last to finish a step issues the next MMAs).
 // Rows past a segment's end are masked (zero gates, zeroed key/value rows),
 // so a ragged tail chunk needs no padding.
 #include "common.cuh"
