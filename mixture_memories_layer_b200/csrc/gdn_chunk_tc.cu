@@ -538,10 +538,7 @@ struct StateLayout {
     static constexpr int VB = KQ0 + 2 * KQSZ;                 // [64 x 128] bf16: two 64-column slabs
     static constexpr int TB = VB + 2 * 8192;                  // Tb image
     static constexpr int PB = TB + IMG;                       // P image
-    static constexpr int YB = PB + IMG;                       // [128 x 64] bf16: V^T - Z~
-    static constexpr int UOB = YB + 16384;                    // [128 x 64] bf16: U^T (output term)
-    static constexpr int USB = UOB + 16384;                   // [128 x 64] bf16: U^T diag(G_DEC) (state term)
-    static constexpr int STG = USB + 16384;                   // 8 x [32 rows x 32 d_v] bf16: per-warp output staging
+    static constexpr int STG = PB + IMG;                      // 8 x [32 rows x 32 d_v] bf16: per-warp output staging
     static constexpr int GBB = STG + 16384;                   // 2 gate records
     static constexpr int BARS = GBB + 2 * GB * 4;
     static constexpr int MISC = BARS + NBARS * 8;
@@ -565,8 +562,15 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // TMEM columns: T = rho S (fp32), its bf16 copy (the A operand of Z and
     // X), Z then U, X then X + O (Z and X adjacent: one N = 128 accumulator)
     constexpr uint32_t T_S = 0, T_SB = D, T_ZU = D + D / 2, T_XO = T_ZU + 64;
+    // bf16 A operands of the U, state-update and output products, [128 x 64]
+    // each (32 columns): inside the state copy's columns for d = 256 (free
+    // between the Z | X product and the read-back; the read-back's first
+    // half does not touch them), after X otherwise
+    constexpr uint32_t T_Y = D == 256 ? T_SB : T_XO + 64;
+    constexpr uint32_t T_US = T_Y + 64, T_UO = T_Y + 96;
     constexpr uint32_t TMEM_COLS = 512;
-    static_assert(T_XO + 64 <= TMEM_COLS, "TMEM budget");
+    static_assert(T_XO + 64 <= TMEM_COLS && T_UO + 32 <= TMEM_COLS, "TMEM budget");
+    static_assert(D != 256 || T_US >= T_SB + D / 4, "operands clear of the read-back's first half");
     static_assert(Lay::BYTES <= 232448, "shared memory budget");
 
     extern __shared__ unsigned char smem_raw[];
@@ -579,8 +583,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const uint32_t cnt_y = smem_u32(tslot + 2), cnt_u = smem_u32(tslot + 3);
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const uint32_t kq0 = smem_u32(sm + Lay::KQ0), vb = smem_u32(sm + Lay::VB);
-    const uint32_t timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB), yb = smem_u32(sm + Lay::YB);
-    const uint32_t uob = smem_u32(sm + Lay::UOB), usb = smem_u32(sm + Lay::USB), stg0 = smem_u32(sm + Lay::STG);
+    const uint32_t timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB), stg0 = smem_u32(sm + Lay::STG);
     float* gbuf = reinterpret_cast<float*>(sm + Lay::GBB);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -708,13 +711,9 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 for (int e = 0; e < 32; e += 2)
                     pk[e / 2] = pack_bf16(fmaf(-__uint_as_float(z[e]), eg[e], __uint_as_float(vv[e / 2] << 16)),
                                           fmaf(-__uint_as_float(z[e + 1]), eg[e + 1], __uint_as_float(vv[e / 2] & 0xFFFF0000u)));
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    const int cc = hf * 4 + c8;
-                    st_shared_v4(yb + i * 128 + ((cc ^ (i & 7)) << 4), pk + 4 * c8);
-                }
+                tmem_st_x16(tmem + lb + T_Y + 16 * hf, pk);
             }
-            fence_proxy_async_smem();
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0 && last_arrival(cnt_y)) {
@@ -724,8 +723,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_ZU, desc_kmajor_sw128(yb + kk * 32), desc_kmajor_sw128(timg + kk * 32), ID64,
-                                 kk != 0);
+                        umma_f16_ts(tmem + T_ZU, tmem + T_Y + 8 * kk, desc_kmajor_sw128(timg + kk * 32), ID64, kk != 0);
                     umma_commit(bar(U_FULL));
                     umma_commit(bar(T_FREE));
                     issued = true;
@@ -750,15 +748,10 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     pu[e / 2] = pack_bf16(a0, a1);
                     pd[e / 2] = pack_bf16(a0 * dc[e], a1 * dc[e + 1]);
                 }
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    const int cc = hf * 4 + c8;
-                    const uint32_t off = i * 128 + ((cc ^ (i & 7)) << 4);
-                    st_shared_v4(uob + off, pu + 4 * c8);
-                    st_shared_v4(usb + off, pd + 4 * c8);
-                }
+                tmem_st_x16(tmem + lb + T_UO + 16 * hf, pu);
+                tmem_st_x16(tmem + lb + T_US + 16 * hf, pd);
             }
-            fence_proxy_async_smem();
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0 && last_arrival(cnt_u)) {
@@ -768,12 +761,11 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
                 constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);   // B = K (MN-major)
                 const int e = __float_as_int(gb[G_SCL]);
-                umma_f16_scaled(tmem + T_S, desc_kmajor_sw128(usb), desc_mnmajor_sw128(kq, 16384), IDS,
-                                e >= 0 ? 1u : 0u, e >= 0 ? e : 0);
+                umma_f16_ts_scaled(tmem + T_S, tmem + T_US, desc_mnmajor_sw128(kq, 16384), IDS, e >= 0 ? 1u : 0u,
+                                   e >= 0 ? e : 0);
 #pragma unroll
                 for (int kk = 1; kk < 4; ++kk)
-                    umma_f16(tmem + T_S, desc_kmajor_sw128(usb + kk * 32), desc_mnmajor_sw128(kq + kk * 2048, 16384),
-                             IDS, 1);
+                    umma_f16_ts(tmem + T_S, tmem + T_US + 8 * kk, desc_mnmajor_sw128(kq + kk * 2048, 16384), IDS, 1);
                 umma_commit(bar(S_FULL));
                 umma_commit(bar(KQ_FREE + b));
                 issued = true;
@@ -781,15 +773,52 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_XO, desc_kmajor_sw128(uob + kk * 32), desc_kmajor_sw128(pimg + kk * 32), ID64,
-                                 1);
+                        umma_f16_ts(tmem + T_XO, tmem + T_UO + 8 * kk, desc_kmajor_sw128(pimg + kk * 32), ID64, 1);
                     umma_commit(bar(O_FULL));
                     umma_commit(bar(P_FREE));
                 }
             }
-            // ---- state read-back: the bf16 copy of T for the next chunk (or the final state)
-            if (!mbar_wait(bar(S_FULL), ph, abort_flag, p.err, 25)) break;
+            // ---- output o_r = scale (S e^gamma_r q_r + sum_s P_rs u_s), rows r < n; read out
+            // of TMEM first, so the next chunk's Z | X product (which overwrites X) need
+            // not wait for the state read-back
+            if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 26)) break;
             tc_fence_after();
+            {
+                uint32_t xo[32];
+                tmem_ld_x32(tmem + lb + T_XO + sh, xo);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(XO_FREE));
+                // this warp's [32 rows x 32 d_v] piece, staged row-major, leaves by one TMA store
+                const uint32_t stg = stg0 + warp * 2048 + lane * 2;
+                if (lane == 0) bulk_wait_read0();     // the previous chunk's store has read the piece
+                __syncwarp();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const uint32_t pr = pack_bf16(p.scale * __uint_as_float(xo[e]), p.scale * __uint_as_float(xo[e + 1]));
+                    asm volatile("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                                 "st.shared.b16 [%0], lo;\n\tst.shared.b16 [%1], hi;\n\t}"
+                                 ::"r"(stg + e * 64), "r"(stg + (e + 1) * 64), "r"(pr) : "memory");
+                }
+                if (sh + 32 <= n) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_o, stg0 + warp * 2048, h * D + dv0 + 32 * qd, (int)(r0 + sh));
+                        bulk_commit();
+                    }
+                } else {
+                    // ragged last chunk: only rows < n belong to this segment
+                    bf16* orow = p.o + (r0 + sh) * (int64_t)p.H * D + (int64_t)h * D + dv0 + i;
+                    const int64_t rstride = (int64_t)p.H * D;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (sh + e < n) orow[e * rstride] = __float2bfloat16_rn(p.scale * __uint_as_float(xo[e]));
+                }
+            }
+            // ---- state read-back: the bf16 copy of T for the next chunk (or the final state)
+            // (O_FULL, waited above, implies S_FULL: both were committed by one thread, S first)
             if (c + 1 == nc) {
                 if (p.h_final) {
                     const float inv = exp2f(-gb[G_LR]);
@@ -825,43 +854,6 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(part ? SBF_HI : SBF_LO));
-                }
-            }
-            // ---- output o_r = scale (S e^gamma_r q_r + sum_s P_rs u_s), rows r < n
-            if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 26)) break;
-            tc_fence_after();
-            {
-                uint32_t xo[32];
-                tmem_ld_x32(tmem + lb + T_XO + sh, xo);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(XO_FREE));
-                // this warp's [32 rows x 32 d_v] piece, staged row-major, leaves by one TMA store
-                const uint32_t stg = stg0 + warp * 2048 + lane * 2;
-                if (lane == 0) bulk_wait_read0();     // the previous chunk's store has read the piece
-                __syncwarp();
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const uint32_t pr = pack_bf16(p.scale * __uint_as_float(xo[e]), p.scale * __uint_as_float(xo[e + 1]));
-                    asm volatile("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-                                 "st.shared.b16 [%0], lo;\n\tst.shared.b16 [%1], hi;\n\t}"
-                                 ::"r"(stg + e * 64), "r"(stg + (e + 1) * 64), "r"(pr) : "memory");
-                }
-                if (sh + 32 <= n) {
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tm_o, stg0 + warp * 2048, h * D + dv0 + 32 * qd, (int)(r0 + sh));
-                        bulk_commit();
-                    }
-                } else {
-                    // ragged last chunk: only rows < n belong to this segment
-                    bf16* orow = p.o + (r0 + sh) * (int64_t)p.H * D + (int64_t)h * D + dv0 + i;
-                    const int64_t rstride = (int64_t)p.H * D;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (sh + e < n) orow[e * rstride] = __float2bfloat16_rn(p.scale * __uint_as_float(xo[e]));
                 }
             }
             __syncwarp();

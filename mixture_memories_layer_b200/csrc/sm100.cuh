@@ -177,6 +177,29 @@ __device__ __forceinline__ void umma_f16_scale_imm(uint32_t d_tmem, uint64_t ade
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(S)
         : "memory");
 }
+template <int S>
+__device__ __forceinline__ void umma_f16_ts_scale_imm(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                      uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p, %5;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(S)
+        : "memory");
+}
+// The same with A from tensor memory.
+__device__ __forceinline__ void umma_f16_ts_scaled(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                   uint32_t accumulate, int s) {
+    switch (s) {
+#define MOM_TS_SCALED_CASE(S) case S: umma_f16_ts_scale_imm<S>(d_tmem, a_tmem, bdesc, idesc, accumulate); break;
+        MOM_TS_SCALED_CASE(0) MOM_TS_SCALED_CASE(1) MOM_TS_SCALED_CASE(2) MOM_TS_SCALED_CASE(3)
+        MOM_TS_SCALED_CASE(4) MOM_TS_SCALED_CASE(5) MOM_TS_SCALED_CASE(6) MOM_TS_SCALED_CASE(7)
+        MOM_TS_SCALED_CASE(8) MOM_TS_SCALED_CASE(9) MOM_TS_SCALED_CASE(10) MOM_TS_SCALED_CASE(11)
+        MOM_TS_SCALED_CASE(12) MOM_TS_SCALED_CASE(13) MOM_TS_SCALED_CASE(14)
+#undef MOM_TS_SCALED_CASE
+        default: umma_f16_ts_scale_imm<15>(d_tmem, a_tmem, bdesc, idesc, accumulate); break;
+    }
+}
 __device__ __forceinline__ void umma_f16_scaled(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                 uint32_t accumulate, int s) {
     switch (s) {
