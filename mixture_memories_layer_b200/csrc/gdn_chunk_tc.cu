@@ -756,19 +756,11 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             __syncwarp();
             if (lane == 0 && last_arrival(cnt_u)) {
                 tc_fence_after();
-                // T = 2^-e T + (U^T diag(G_DEC)) K, then X += U^T P^T
+                // X += U^T P^T first (small; frees X early), then T = 2^-e T + (U^T diag(G_DEC)) K.
+                // One thread commits both, the output first: S_FULL implies O_FULL.
                 const uint32_t kq = kq0 + b * Lay::KQSZ;
                 constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
                 constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);   // B = K (MN-major)
-                const int e = __float_as_int(gb[G_SCL]);
-                umma_f16_ts_scaled(tmem + T_S, tmem + T_US, desc_mnmajor_sw128(kq, 16384), IDS, e >= 0 ? 1u : 0u,
-                                   e >= 0 ? e : 0);
-#pragma unroll
-                for (int kk = 1; kk < 4; ++kk)
-                    umma_f16_ts(tmem + T_S, tmem + T_US + 8 * kk, desc_mnmajor_sw128(kq + kk * 2048, 16384), IDS, 1);
-                umma_commit(bar(S_FULL));
-                umma_commit(bar(KQ_FREE + b));
-                issued = true;
                 if (mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 47)) {
                     tc_fence_after();
 #pragma unroll
@@ -776,21 +768,69 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         umma_f16_ts(tmem + T_XO, tmem + T_UO + 8 * kk, desc_kmajor_sw128(pimg + kk * 32), ID64, 1);
                     umma_commit(bar(O_FULL));
                     umma_commit(bar(P_FREE));
+                    const int e = __float_as_int(gb[G_SCL]);
+                    umma_f16_ts_scaled(tmem + T_S, tmem + T_US, desc_mnmajor_sw128(kq, 16384), IDS, e >= 0 ? 1u : 0u,
+                                       e >= 0 ? e : 0);
+#pragma unroll
+                    for (int kk = 1; kk < 4; ++kk)
+                        umma_f16_ts(tmem + T_S, tmem + T_US + 8 * kk, desc_mnmajor_sw128(kq + kk * 2048, 16384), IDS, 1);
+                    umma_commit(bar(S_FULL));
+                    umma_commit(bar(KQ_FREE + b));
+                    issued = true;
                 }
             }
-            // ---- output o_r = scale (S e^gamma_r q_r + sum_s P_rs u_s), rows r < n; read out
-            // of TMEM first, so the next chunk's Z | X product (which overwrites X) need
-            // not wait for the state read-back
-            if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 26)) break;
-            tc_fence_after();
-            {
-                uint32_t xo[32];
-                tmem_ld_x32(tmem + lb + T_XO + sh, xo);
-                tmem_ld_wait();
+            // ---- the output read out of TMEM as soon as its product is done (the next
+            // chunk's Z | X product overwrites X), then after the state update the bf16
+            // copy of the new T in two d_k halves (the next product starts on the first),
+            // then the output stored
+            const bool last = c + 1 == nc;
+            auto readback_half = [&](int part) {
+                for (int blk = 0; blk < HALF / 64; ++blk) {
+                    const int col = part * HALF + hf * (HALF / 2) + 32 * blk;
+                    uint32_t s0[32], pk[16];
+                    tmem_ld_x32(tmem + lb + T_S + col, s0);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(s0[2 * e]), __uint_as_float(s0[2 * e + 1]));
+                    tmem_st_x16(tmem + lb + T_SB + col / 2, pk);
+                }
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(XO_FREE));
-                // this warp's [32 rows x 32 d_v] piece, staged row-major, leaves by one TMA store
+                if (lane == 0) mbar_arrive(bar(part ? SBF_HI : SBF_LO));
+            };
+            if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 26)) break;
+            tc_fence_after();
+            uint32_t xo[32];
+            tmem_ld_x32(tmem + lb + T_XO + sh, xo);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(XO_FREE));
+            if (!mbar_wait(bar(S_FULL), ph, abort_flag, p.err, 25)) break;
+            tc_fence_after();
+            if (!last) {
+                readback_half(0);
+                readback_half(1);
+            } else if (p.h_final) {
+                // the final state S = T / rho
+                const float inv = exp2f(-gb[G_LR]);
+                for (int blk = 0; blk < HALF / 32; ++blk) {
+                    const int col = hf * HALF + 32 * blk;
+                    uint32_t sv[32];
+                    tmem_ld_x32(tmem + lb + T_S + col, sv);
+                    tmem_ld_wait();
+                    float* out = p.h_final + hoff + col;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(out + e) =
+                            make_float4(inv * __uint_as_float(sv[e]), inv * __uint_as_float(sv[e + 1]),
+                                        inv * __uint_as_float(sv[e + 2]), inv * __uint_as_float(sv[e + 3]));
+                }
+            }
+            // ---- output o_r = scale (S e^gamma_r q_r + sum_s P_rs u_s), rows r < n: this
+            // warp's [32 rows x 32 d_v] piece, staged row-major, leaves by one TMA store
+            {
                 const uint32_t stg = stg0 + warp * 2048 + lane * 2;
                 if (lane == 0) bulk_wait_read0();     // the previous chunk's store has read the piece
                 __syncwarp();
@@ -815,45 +855,6 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (sh + e < n) orow[e * rstride] = __float2bfloat16_rn(p.scale * __uint_as_float(xo[e]));
-                }
-            }
-            // ---- state read-back: the bf16 copy of T for the next chunk (or the final state)
-            // (O_FULL, waited above, implies S_FULL: both were committed by one thread, S first)
-            if (c + 1 == nc) {
-                if (p.h_final) {
-                    const float inv = exp2f(-gb[G_LR]);
-                    for (int blk = 0; blk < HALF / 32; ++blk) {
-                        const int col = hf * HALF + 32 * blk;
-                        uint32_t sv[32];
-                        tmem_ld_x32(tmem + lb + T_S + col, sv);
-                        tmem_ld_wait();
-                        float* out = p.h_final + hoff + col;
-#pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4*>(out + e) =
-                                make_float4(inv * __uint_as_float(sv[e]), inv * __uint_as_float(sv[e + 1]),
-                                            inv * __uint_as_float(sv[e + 2]), inv * __uint_as_float(sv[e + 3]));
-                    }
-                }
-            } else {
-                // first d_k half (both warps of the lane quarter share it), then the
-                // second: the Z | X product starts on the first half meanwhile
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    for (int blk = 0; blk < HALF / 64; ++blk) {
-                        const int col = part * HALF + hf * (HALF / 2) + 32 * blk;
-                        uint32_t s0[32], pk[16];
-                        tmem_ld_x32(tmem + lb + T_S + col, s0);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            pk[e] = pack_bf16(__uint_as_float(s0[2 * e]), __uint_as_float(s0[2 * e + 1]));
-                        tmem_st_x16(tmem + lb + T_SB + col / 2, pk);
-                    }
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(part ? SBF_HI : SBF_LO));
                 }
             }
             __syncwarp();
