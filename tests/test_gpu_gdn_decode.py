@@ -174,3 +174,9 @@ def _decode_case(w, steps, check_seqs, prefill_len):
 def test_decode_small(d, dtype):
     w = synth.Workload("dec_small", 16, 0, 256, 2, d, 8, 2, dtype, seed=9, decode_steps=3, prefill_len=40)
     _decode_case(w, steps=3, check_seqs=range(16), prefill_len=40)
+
+
+def test_decode_one_sequence_every_memory():
+    # a batch of one, top-k = M: the step updates all M + 1 states of the sequence
+    w = synth.Workload("dec_one", 1, 0, 256, 2, 64, 4, 4, "f32", seed=11, decode_steps=2, prefill_len=8)
+    _decode_case(w, steps=2, check_seqs=range(1), prefill_len=8)

@@ -105,6 +105,32 @@ def test_layer_many_memories_top4():
     _check_layer(w, p, res)
 
 
+def test_layer_top_k_equals_memories():
+    # every token reaches every memory: the gates are the whole softmax over M
+    w, p = _small(128, M=4, k=4, lens=(130, 3))
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    assert np.all(np.sort(res["idx"], axis=1) == np.arange(4))
+    _check_layer(w, p, res)
+
+
+def test_layer_single_token():
+    w, p = _small(256, lens=(1,))
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _check_layer(w, p, res)
+
+
+def test_layer_many_tiny_sequences():
+    # 48 sequences of 0-5 tokens: nearly every (memory, sequence) segment
+    # holds 0-3 rows, many chunks are both first and last
+    lens = tuple(int(v) for v in np.random.default_rng(5).integers(0, 6, size=48))
+    w, p = _small(64, lens=lens, seed=5)
+    lay, res = run_layer(w, p)
+    assert lay.device_errors() == {}
+    _check_layer(w, p, res)
+
+
 def test_layer_h0_hand_off():
     """Forward over [0, T) equals [0, T/2) then [T/2, T) seeded with the
     first call's final states."""
