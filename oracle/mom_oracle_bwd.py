@@ -1,0 +1,219 @@
+"""CPU oracle for the reverse pass of one Mixture-of-Memories (MoM) layer:
+plain, slow, fp64.
+
+TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.  The same rules as
+``mom_oracle``: only the test suite may import it; it shares no code with the
+CUDA path.
+
+What it computes.  For the forward of ``mom_oracle.mom_forward`` (the Gated
+DeltaNet rule per memory, "MoM: Linear Sequence Modeling with
+Mixture-of-Memories", Summary; the authors' blog post, "Mixture-of-Memories"
+and the experiments section naming Gated DeltaNet's gate and update rule) and
+a scalar loss
+
+    L = <dout, out> + sum_s <dh_shared[s], h_shared[s]>
+                    + sum_{m,s} <dh_mem[m,s], h_mem[m,s]>,
+
+the gradients of L with respect to the tokens x, every weight (router W_r,
+b_r; shared W_q, W_k_sh, W_v_sh, W_beta, W_a, A, b_a; per-memory W_k, W_v)
+and the initial states.  Each forward step is undone in reverse order by its
+adjoint, written out by hand below; no automatic differentiation.
+
+Routing.  Which memories a token visits (the top-k of the logits) is
+piecewise constant in the inputs, so no gradient flows through the choice;
+gradients do flow through the renormalised gates g_j = exp(l_j) / sum_j'
+exp(l_j') over the chosen logits ("MoM: Mixture-of-Memories Fixes Linear
+Attention Recall", Router mechanics: softmax, top-k, renormalisation).
+
+Pinned by central finite differences of the forward oracle in fp64
+(tests/test_oracle_backward.py): every gradient of the recurrence and of the
+whole layer, on tiny inputs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import mom_oracle as fwd
+
+F64 = np.float64
+
+
+def l2norm_bwd(z, dy, eps: float = fwd.NORM_EPS):
+    """Adjoint of y = z / n, n = sqrt(|z|^2 + eps) over the last axis:
+    dz = dy / n - z (z . dy) / n^3."""
+    z = np.asarray(z, F64)
+    dy = np.asarray(dy, F64)
+    n = np.sqrt(np.sum(z * z, axis=-1, keepdims=True) + eps)
+    return dy / n - z * np.sum(z * dy, axis=-1, keepdims=True) / n ** 3
+
+
+def gdn_recurrence_bwd(q, k, v, beta, log_alpha, do, h0=None, dh_final=None, scale: float = 1.0):
+    """Reverse pass of ``mom_oracle.gdn_recurrence`` over one segment.
+
+    Shapes as the forward: q,k [T,H,dk]; v, do [T,H,dv]; beta, log_alpha
+    [T,H]; h0, dh_final [H,dv,dk] or None.  Returns a dict with dq, dk, dv,
+    dbeta, dlog_alpha (the forward's shapes) and dh0 [H,dv,dk].
+
+    With a = exp(log alpha_t), b = beta_t, y = S_{t-1} k_t and
+    S_t = a S_{t-1} - a b y k^T + b v k^T,  o_t = S_t (scale q_t),
+    and G the adjoint of S_t (do_t (scale q_t)^T plus what flows back from
+    step t+1):
+      dq_t = scale S_t^T do_t
+      dv_t = b G k
+      db_t = (v - a y)^T G k
+      da_t = <G, S_{t-1}> - b y^T G k,       dlog_alpha_t = a da_t
+      dk_t = b G^T v - a b (S_{t-1}^T G k + G^T y)
+      adjoint of S_{t-1} = a G - a b (G k) k^T
+    """
+    q = np.asarray(q, F64)
+    k = np.asarray(k, F64)
+    v = np.asarray(v, F64)
+    beta = np.asarray(beta, F64)
+    log_alpha = np.asarray(log_alpha, F64)
+    do = np.asarray(do, F64)
+    T, H, dk = k.shape
+    dv = v.shape[-1]
+    # forward, keeping every state (S[t] = state after token t-1; S[0] = h0)
+    S = np.zeros((T + 1, H, dv, dk), F64)
+    if h0 is not None:
+        S[0] = np.asarray(h0, F64)
+    for t in range(T):
+        _, S[t + 1] = fwd.gdn_step(S[t], q[t], k[t], v[t], beta[t], log_alpha[t], scale)
+    G = np.zeros((H, dv, dk), F64) if dh_final is None else np.array(dh_final, F64, copy=True)
+    out = {name: np.zeros_like(a) for name, a in
+           (("dq", q), ("dk", k), ("dv", v), ("dbeta", beta), ("dlog_alpha", log_alpha))}
+    for t in range(T - 1, -1, -1):
+        sq = scale * q[t]
+        G = G + do[t][:, :, None] * sq[:, None, :]
+        out["dq"][t] = scale * np.einsum("hvk,hv->hk", S[t + 1], do[t])
+        a = np.exp(log_alpha[t])
+        b = beta[t]
+        kt, vt, Sp = k[t], v[t], S[t]
+        y = np.einsum("hvk,hk->hv", Sp, kt)
+        Gk = np.einsum("hvk,hk->hv", G, kt)
+        out["dv"][t] = b[:, None] * Gk
+        out["dbeta"][t] = np.einsum("hv,hv->h", vt - a[:, None] * y, Gk)
+        da = np.einsum("hvk,hvk->h", G, Sp) - b * np.einsum("hv,hv->h", y, Gk)
+        out["dlog_alpha"][t] = a * da
+        GTv = np.einsum("hvk,hv->hk", G, vt)
+        SGk = np.einsum("hvk,hv->hk", Sp, Gk)
+        GTy = np.einsum("hvk,hv->hk", G, y)
+        out["dk"][t] = b[:, None] * GTv - (a * b)[:, None] * (SGk + GTy)
+        G = a[:, None, None] * G - (a * b)[:, None, None] * Gk[:, :, None] * kt[:, None, :]
+    out["dh0"] = G
+    return out
+
+
+def router_gates_bwd(logits, idx, dgate):
+    """Adjoint of the renormalised top-k gates g = softmax(logits[idx]) with
+    respect to all M logits (zero for memories not chosen)."""
+    logits = np.asarray(logits, F64)
+    idx = np.asarray(idx, np.int64)
+    g = fwd.gates_for(logits, idx)
+    dsel = g * (dgate - np.sum(g * dgate, axis=-1, keepdims=True))
+    dl = np.zeros_like(logits)
+    np.put_along_axis(dl, idx, dsel, axis=-1)
+    return dl
+
+
+def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: float = 1.0,
+                 forced_idx=None, h0_shared=None, h0_mem=None, dh_shared=None, dh_mem=None):
+    """Gradients of L (module docstring) for one layer forward over a packed
+    batch; arguments as ``mom_oracle.mom_forward`` plus the adjoints dout
+    [N,H,d], dh_shared [S,H,d,d] and dh_mem [M,S,H,d,d] (None: zero).
+
+    Returns a dict: dx, dw_r, db_r, dw_q, dw_k_sh, dw_v_sh, dw_beta, dw_a,
+    dA, db_a, dw_k [M,..], dw_v [M,..], dh0_shared [S,..], dh0_mem [M,S,..],
+    and the forward's own results under "fwd".
+    """
+    x = np.asarray(x, F64)
+    dout = np.asarray(dout, F64)
+    cu = np.asarray(cu_seqlens, np.int64)
+    N, D = x.shape
+    S = len(cu) - 1
+    M = np.shape(p["w_r"])[0]
+    W = {name: np.asarray(p[name], F64) for name in
+         ("w_r", "w_q", "w_k_sh", "w_v_sh", "w_beta", "w_a", "A", "b_a", "w_k", "w_v")}
+    f = fwd.mom_forward(x, p, cu, top_k, H, d, scale, forced_idx=forced_idx,
+                        h0_shared=h0_shared, h0_mem=h0_mem)
+    idx, gate = f["idx"], f["gate"]
+
+    # combine: out = o_shared + sum_j gate_j o_mem[:, j]
+    dgate = np.einsum("nhd,njhd->nj", dout, f["o_mem"])
+    do_shared = dout
+
+    # recurrences: adjoints of the per-token quantities they consume
+    dq = np.zeros((N, H, d), F64)
+    dk_sh = np.zeros((N, H, d), F64)
+    dv_sh = np.zeros((N, H, d), F64)
+    dbeta = np.zeros((N, H), F64)
+    dlog_alpha = np.zeros((N, H), F64)
+    dx = np.zeros_like(x)
+    dw_k = np.zeros_like(W["w_k"])
+    dw_v = np.zeros_like(W["w_v"])
+    dh0_shared = np.zeros((S, H, d, d), F64)
+    dh0_mem = np.zeros((M, S, H, d, d), F64)
+    for s in range(S):
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        h0 = None if h0_shared is None else h0_shared[s]
+        dhf = None if dh_shared is None else dh_shared[s]
+        if t1 > t0:
+            r = gdn_recurrence_bwd(f["q"][t0:t1], f["k_sh"][t0:t1], f["v_sh"][t0:t1], f["beta"][t0:t1],
+                                   f["log_alpha"][t0:t1], do_shared[t0:t1], h0, dhf, scale)
+            dq[t0:t1] += r["dq"]
+            dk_sh[t0:t1] += r["dk"]
+            dv_sh[t0:t1] += r["dv"]
+            dbeta[t0:t1] += r["dbeta"]
+            dlog_alpha[t0:t1] += r["dlog_alpha"]
+            dh0_shared[s] = r["dh0"]
+        else:
+            dh0_shared[s] = 0.0 if dhf is None else dhf
+        for m in range(M):
+            hit = idx[t0:t1] == m
+            rows = t0 + np.nonzero(hit.any(axis=1))[0]
+            dhf = None if dh_mem is None else dh_mem[m, s]
+            if len(rows) == 0:
+                dh0_mem[m, s] = 0.0 if dhf is None else dhf
+                continue
+            slot = np.argmax(idx[rows] == m, axis=1)
+            g = gate[rows, slot]
+            z_k = (x[rows] @ W["w_k"][m].T).reshape(len(rows), H, d)
+            k_m = fwd.l2norm(z_k)
+            v_m = (x[rows] @ W["w_v"][m].T).reshape(len(rows), H, d)
+            h0 = None if h0_mem is None else h0_mem[m, s]
+            r = gdn_recurrence_bwd(f["q"][rows], k_m, v_m, f["beta"][rows], f["log_alpha"][rows],
+                                   g[:, None, None] * dout[rows], h0, dhf, scale)
+            dq[rows] += r["dq"]
+            dbeta[rows] += r["dbeta"]
+            dlog_alpha[rows] += r["dlog_alpha"]
+            dh0_mem[m, s] = r["dh0"]
+            # memory m's projections of its rows
+            dz_k = l2norm_bwd(z_k, r["dk"]).reshape(len(rows), H * d)
+            dz_v = r["dv"].reshape(len(rows), H * d)
+            dw_k[m] += dz_k.T @ x[rows]
+            dw_v[m] += dz_v.T @ x[rows]
+            dx[rows] += dz_k @ W["w_k"][m] + dz_v @ W["w_v"][m]
+
+    # router: logits = x W_r^T + b_r, gates renormalised over the chosen ones
+    dl = router_gates_bwd(f["logits"], idx, dgate)
+    dw_r = dl.T @ x
+    db_r = dl.sum(axis=0)
+    dx += dl @ W["w_r"]
+
+    # shared projections
+    z_q = (x @ W["w_q"].T).reshape(N, H, d)
+    z_k = (x @ W["w_k_sh"].T).reshape(N, H, d)
+    dz_q = l2norm_bwd(z_q, dq).reshape(N, H * d)
+    dz_k = l2norm_bwd(z_k, dk_sh).reshape(N, H * d)
+    dz_v = dv_sh.reshape(N, H * d)
+    beta = f["beta"]
+    dz_beta = dbeta * beta * (1.0 - beta)
+    z_a = x @ W["w_a"].T + W["b_a"]
+    # log alpha = -exp(A) softplus(z_a): d/dz_a = -exp(A) sigmoid(z_a); d/dA = log alpha
+    dz_a = dlog_alpha * (-np.exp(W["A"])) * fwd.sigmoid(z_a)
+    dA = np.sum(dlog_alpha * f["log_alpha"], axis=0)
+    db_a = dz_a.sum(axis=0)
+    dx += dz_q @ W["w_q"] + dz_k @ W["w_k_sh"] + dz_v @ W["w_v_sh"] + dz_beta @ W["w_beta"] + dz_a @ W["w_a"]
+    return dict(dx=dx, dw_r=dw_r, db_r=db_r, dw_q=dz_q.T @ x, dw_k_sh=dz_k.T @ x, dw_v_sh=dz_v.T @ x,
+                dw_beta=dz_beta.T @ x, dw_a=dz_a.T @ x, dA=dA, db_a=db_a, dw_k=dw_k, dw_v=dw_v,
+                dh0_shared=dh0_shared, dh0_mem=dh0_mem, fwd=f)
