@@ -104,6 +104,112 @@ def gdn_recurrence_bwd(q, k, v, beta, log_alpha, do, h0=None, dh_final=None, sca
     return out
 
 
+def gdn_chunked_bwd(q, k, v, beta, log_alpha, do, h0=None, dh_final=None, scale: float = 1.0,
+                    chunk: int = 64):
+    """The reverse pass in the chunked (UT / WY) form of
+    ``mom_oracle.gdn_chunked``: a self-check of ``gdn_recurrence_bwd`` (the
+    two must agree to rounding), not a separate definition.
+
+    Per chunk, with H the state at its start, gamma the running sum of
+    log alpha from the chunk start, D_rs = exp(gamma_r - gamma_s) (s <= r),
+    Qs = scale Q, the forward is
+      L = strict_lower(diag(beta) D o K K^T),  T = (I + L)^-1
+      R = diag(beta) V - diag(beta e^gamma) K H^T,   U = T R
+      O = diag(e^gamma) Qs H^T + (Qs K^T o D) U
+      H' = e^gamma_C H + U^T diag(e^(gamma_C - gamma)) K
+    and the adjoints are taken in the reverse order of those lines (dH' is the
+    state adjoint carried back from the next chunk); the adjoint of gamma is
+    turned into that of log alpha by a reversed running sum.
+    """
+    q = np.asarray(q, F64)
+    k = np.asarray(k, F64)
+    v = np.asarray(v, F64)
+    beta = np.asarray(beta, F64)
+    log_alpha = np.asarray(log_alpha, F64)
+    do = np.asarray(do, F64)
+    T, Hn, dk = k.shape
+    dv = v.shape[-1]
+    out = {name: np.zeros_like(a) for name, a in
+           (("dq", q), ("dk", k), ("dv", v), ("dbeta", beta), ("dlog_alpha", log_alpha))}
+    out["dh0"] = np.zeros((Hn, dv, dk), F64)
+    starts = list(range(0, T, chunk))
+    for h in range(Hn):
+        # forward: the state at every chunk start
+        Hs = [np.zeros((dv, dk), F64) if h0 is None else np.array(h0[h], F64, copy=True)]
+        parts = []
+        for c0 in starts:
+            c1 = min(c0 + chunk, T)
+            n = c1 - c0
+            Qs, K, V = scale * q[c0:c1, h], k[c0:c1, h], v[c0:c1, h]
+            b = beta[c0:c1, h]
+            g = np.cumsum(log_alpha[c0:c1, h])
+            causal = np.tril(np.ones((n, n), dtype=bool))
+            D = np.where(causal, np.exp(np.where(causal, g[:, None] - g[None, :], 0.0)), 0.0)
+            strict = np.tril(np.ones((n, n), dtype=bool), -1)
+            L = np.where(strict, b[:, None] * D * (K @ K.T), 0.0)
+            Tm = np.linalg.inv(np.eye(n) + L)
+            Kt = (b * np.exp(g))[:, None] * K
+            R = b[:, None] * V - Kt @ Hs[-1].T
+            U = Tm @ R
+            E = np.exp(g[-1] - g)
+            parts.append((c0, c1, Qs, K, V, b, g, D, causal, strict, L, Tm, Kt, R, U, E))
+            Hs.append(np.exp(g[-1]) * Hs[-1] + U.T @ (E[:, None] * K))
+        # reverse
+        dH = np.zeros((dv, dk), F64) if dh_final is None else np.array(dh_final[h], F64, copy=True)
+        for ci in range(len(starts) - 1, -1, -1):
+            c0, c1, Qs, K, V, b, g, D, causal, strict, L, Tm, Kt, R, U, E = parts[ci]
+            Hc = Hs[ci]
+            dO = do[c0:c1, h]
+            eg = np.exp(g)
+            dg = np.zeros_like(g)
+            # H' = e^gC H + U^T diag(E) K
+            dHp = dH
+            dH = np.exp(g[-1]) * dHp
+            dg[-1] += np.exp(g[-1]) * np.sum(dHp * Hc)
+            dU = E[:, None] * (K @ dHp.T)
+            dK = E[:, None] * (U @ dHp)
+            w_s = E * np.einsum("sv,vk,sk->s", U, dHp, K)      # d/dgamma of each E_s term
+            dg[-1] += w_s.sum()
+            dg -= w_s
+            # O = diag(e^g) Qs H^T + (Qs K^T o D) U
+            A = (Qs @ K.T) * D
+            dU += A.T @ dO
+            dA = np.where(causal, dO @ U.T, 0.0)
+            dAD = dA * D
+            dQs = eg[:, None] * (dO @ Hc) + dAD @ K
+            dK += dAD.T @ Qs
+            dH += (eg[:, None] * dO).T @ Qs
+            dg += eg * np.einsum("rv,rv->r", dO, Qs @ Hc.T)
+            wa = dA * A                                          # d/dgamma_r (+) and d/dgamma_s (-) of D
+            dg += wa.sum(axis=1) - wa.sum(axis=0)
+            # U = T R,  R = diag(b) V - Kt H^T,  Kt = diag(b e^g) K
+            dT = dU @ R.T
+            dR = Tm.T @ dU
+            dV = b[:, None] * dR
+            db = np.einsum("rv,rv->r", V, dR)
+            dKt = -dR @ Hc
+            dH += -dR.T @ Kt
+            dK += (b * eg)[:, None] * dKt
+            kd = np.einsum("rk,rk->r", K, dKt)
+            db += eg * kd
+            dg += b * eg * kd
+            # T = (I + L)^-1,  L = strict(diag(b) D o K K^T)
+            dL = np.where(strict, -Tm.T @ dT @ Tm.T, 0.0)
+            KK = K @ K.T
+            db += np.sum(dL * D * KK, axis=1)
+            P = dL * b[:, None] * D
+            dK += P @ K + P.T @ K
+            wl = dL * L
+            dg += wl.sum(axis=1) - wl.sum(axis=0)
+            out["dq"][c0:c1, h] = scale * dQs
+            out["dk"][c0:c1, h] = dK
+            out["dv"][c0:c1, h] = dV
+            out["dbeta"][c0:c1, h] = db
+            out["dlog_alpha"][c0:c1, h] = np.cumsum(dg[::-1])[::-1]
+        out["dh0"][h] = dH
+    return out
+
+
 def router_gates_bwd(logits, idx, dgate):
     """Adjoint of the renormalised top-k gates g = softmax(logits[idx]) with
     respect to all M logits (zero for memories not chosen)."""

@@ -5,7 +5,8 @@ oracle in fp64, which is pinned on its own (test_oracle_*.py): a dropped
 term, a wrong sign or a transposed operand in any adjoint moves some
 derivative well past the difference quotient's error (~1e-9 here).  The
 recurrence is tested with d_v != d_k so that a transpose cannot hide, and
-against the closed form of the beta = 0 case (pure decay).
+against the closed form of the beta = 0 case (pure decay); its chunked form
+(the one a blocked GPU reverse pass takes) must equal the token loop.
 """
 import numpy as np
 import pytest
@@ -77,6 +78,19 @@ def test_gdn_recurrence_bwd_pure_decay_closed_form():
     St = decay[:, :, None, None] * c["h0"][None]
     assert _rel(g["dq"], scale * np.einsum("thvk,thv->thk", St, adj["do"])) < 1e-12
     assert np.all(g["dv"] == 0) and np.all(g["dk"] == 0)
+
+
+@pytest.mark.parametrize("chunk", [1, 3, 4, 64])
+@pytest.mark.parametrize("with_states", [True, False])
+def test_gdn_chunked_bwd_equals_token_loop(chunk, with_states):
+    # T = 11 leaves a ragged last chunk for every chunk size above 1
+    c, adj = _gdn_case(T=11, seed=5)
+    h0, dh = (c["h0"], adj["dh"]) if with_states else (None, None)
+    ref = bwd.gdn_recurrence_bwd(c["q"], c["k"], c["v"], c["beta"], c["log_alpha"], adj["do"], h0, dh, 0.7)
+    got = bwd.gdn_chunked_bwd(c["q"], c["k"], c["v"], c["beta"], c["log_alpha"], adj["do"], h0, dh, 0.7,
+                              chunk=chunk)
+    for key in ref:
+        assert _rel(got[key], ref[key]) < 1e-12, (key, chunk)
 
 
 def _layer_case(lens=(4, 0, 3), D=5, H=2, d=3, M=3, k=2, seed=1):
