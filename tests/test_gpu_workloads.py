@@ -1,6 +1,6 @@
 """Parity at full workload sizes, in the launch configuration the benchmark
 times: the 380M-shape layer (8 x 2048 tokens), its skewed-routing varlen
-variant, and the 1.3B-shape 16-memory layer.
+variant, the 1.3B-shape 16-memory layer, and the 256-sequence decode.
 
 The GPU runs the whole batch.  What the oracle checks:
 * routing and the reordering on every token (cheap on the CPU), bit-exact
@@ -129,3 +129,60 @@ def test_no_wait_runs_to_its_limit():
     torch.cuda.synchronize()
     assert e0.elapsed_time(e1) < 200.0, e0.elapsed_time(e1)
     assert lay.device_errors() == {}
+
+
+def test_decode_b256_full_size():
+    """The decode workload as the benchmark runs it (256 sequences, d_model
+    1024, H=4, d=256, M=8 top-2 + shared, 256-token prefill, 512 steps):
+    the GPU steps the whole batch; the oracle follows 8 sequences over the
+    first 16 steps and 2 sequences over all 512 (outputs and final states),
+    with the GPU's routing imposed, and checks each step's routing outside
+    near ties."""
+    from mixture_memories_layer_b200 import layer as L
+    w = synth.WORKLOADS["decode_b256"]
+    steps, short_steps = w.decode_steps, 16
+    short_seqs, long_seqs = [0, 37, 74, 111, 148, 185, 222, 255], [5, 200]
+    p = synth.make_decode_problem(w, steps=steps)
+    dt = torch.bfloat16
+    lay = L.MoMLayer(L.pack_weights(p, dt), w.heads, w.d_head, w.top_k)
+    b = lay.forward(torch.as_tensor(p["x_prefill"]).to("cuda", dt), torch.as_tensor(p["cu_prefill"]).to("cuda"))
+    state = torch.empty((w.batch, w.n_mem + 1, w.heads, w.d_head, w.d_head), dtype=torch.float32, device="cuda")
+    state[:, :w.n_mem] = b["h_mem"].permute(1, 0, 2, 3, 4)
+    state[:, w.n_mem] = b["h_shared"]
+    pre_idx = b["idx"].cpu().numpy()
+    xs = torch.as_tensor(p["x_steps"]).to("cuda", dt)
+    outs, idxs = [], []
+    for s in range(steps):
+        out, idx = lay.decode_step(xs[s], state)
+        idxs.append(idx.cpu().numpy())
+        if s < short_steps:
+            outs.append(out.float().cpu().numpy())
+        elif s == steps - 1:
+            last_out = out.float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert lay.device_errors() == {}
+    final = state[long_seqs].cpu().numpy()
+    tol = TOL[w.dtype]
+    Lp = w.prefill_len
+    for bsq in short_seqs + long_seqs:
+        n_steps = steps if bsq in long_seqs else short_steps
+        xs_pre = p["x_prefill"][bsq * Lp:(bsq + 1) * Lp]
+        ref = orc.mom_forward(xs_pre, p, np.array([0, Lp]), w.top_k, w.heads, w.d_head,
+                              forced_idx=pre_idx[bsq * Lp:(bsq + 1) * Lp])
+        st = orc.decode_state_from_prefill(ref["h_shared"], ref["h_mem"])
+        for s in range(n_steps):
+            x1 = p["x_steps"][s][bsq:bsq + 1]
+            nat, _, _, near = orc.router_topk(x1, p["w_r"], p["b_r"], w.top_k)
+            if not near[0]:
+                assert np.array_equal(idxs[s][bsq], nat[0]), ("decode routing", bsq, s)
+            o_ref, st, _, _, _ = orc.mom_decode_step(x1, p, st, w.top_k, w.heads, w.d_head,
+                                                     forced_idx=idxs[s][bsq:bsq + 1])
+            if s < short_steps:
+                e = max_abs_rel(outs[s][bsq:bsq + 1], o_ref)
+                assert e < tol, ("decode out", bsq, s, e)
+            elif s == steps - 1:
+                e = max_abs_rel(last_out[bsq:bsq + 1], o_ref)
+                assert e < tol, ("decode out, last step", bsq, e)
+        if bsq in long_seqs:
+            e = max_abs_rel(final[long_seqs.index(bsq)], st[0])
+            assert e < tol, ("decode final state", bsq, e)
