@@ -180,3 +180,16 @@ def test_decode_one_sequence_every_memory():
     # a batch of one, top-k = M: the step updates all M + 1 states of the sequence
     w = synth.Workload("dec_one", 1, 0, 256, 2, 64, 4, 4, "f32", seed=11, decode_steps=2, prefill_len=8)
     _decode_case(w, steps=2, check_seqs=range(1), prefill_len=8)
+
+
+def test_decode_empty_batch():
+    from mixture_memories_layer_b200 import layer as L
+    w = synth.Workload("dec_empty", 4, 0, 256, 2, 64, 4, 2, "bf16", seed=3, decode_steps=1, prefill_len=8)
+    p = synth.make_decode_problem(w, steps=1)
+    lay = L.MoMLayer(L.pack_weights(p, torch.bfloat16), w.heads, w.d_head, w.top_k)
+    x = torch.empty((0, w.d_model), dtype=torch.bfloat16, device="cuda")
+    state = torch.empty((0, w.n_mem + 1, w.heads, w.d_head, w.d_head), dtype=torch.float32, device="cuda")
+    out, idx = lay.decode_step(x, state)
+    torch.cuda.synchronize()
+    assert tuple(out.shape) == (0, w.heads, w.d_head) and tuple(idx.shape) == (0, w.top_k)
+    assert lay.device_errors() == {}

@@ -131,6 +131,28 @@ def test_layer_many_tiny_sequences():
     _check_layer(w, p, res)
 
 
+@pytest.mark.parametrize("with_h0", [False, True])
+def test_layer_no_tokens(with_h0):
+    # two empty sequences: no output rows; every final state is its initial
+    # state (zeros without one)
+    from mixture_memories_layer_b200 import layer as L
+    w, p = _small(256, lens=(0, 0))
+    dt = torch.bfloat16
+    lay = L.MoMLayer(L.pack_weights(p, dt), w.heads, w.d_head, w.top_k)
+    x = torch.empty((0, w.d_model), dtype=dt, device="cuda")
+    cu = torch.zeros(3, dtype=torch.int32, device="cuda")
+    H, d, M = w.heads, w.d_head, w.n_mem
+    h0s = torch.randn((2, H, d, d), device="cuda") if with_h0 else None
+    h0m = torch.randn((M, 2, H, d, d), device="cuda") if with_h0 else None
+    b = lay.forward(x, cu, h0_shared=h0s, h0_mem=h0m)
+    torch.cuda.synchronize()
+    assert lay.device_errors() == {}
+    assert tuple(b["out"].shape) == (0, H, d)
+    assert torch.equal(b["h_shared"], h0s if with_h0 else torch.zeros_like(b["h_shared"]))
+    assert torch.equal(b["h_mem"], h0m if with_h0 else torch.zeros_like(b["h_mem"]))
+    assert tuple(b["seg_cu"].cpu().tolist()) == (0,) * (M * 2 + 1)
+
+
 def test_layer_h0_hand_off():
     """Forward over [0, T) equals [0, T/2) then [T/2, T) seeded with the
     first call's final states."""
