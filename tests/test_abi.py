@@ -59,3 +59,27 @@ def test_workspace_sizes_are_monotone(lib):
     b = L.mom_permute_workspace_size(100000, 2, 4, 3)
     assert lib.MOM_WS_HEADER_BYTES <= a <= b
     assert L.mom_decode_workspace_size(256, 1024, 4, 256, 8, 2) > L.mom_decode_workspace_size(16, 1024, 4, 256, 8, 2)
+
+
+def test_host_validation_at_the_size_limits(lib):
+    """The largest problems the ABI takes: (token, slot) pairs are counted in
+    int32, so n_tok * top_k must stay below 2^31; M and H have fixed caps; the
+    allocation-free reordering holds at most MOM_PERMUTE_NOALLOC_MAX_TOKENS
+    tokens.  Past a limit the call returns an error and launches nothing."""
+    L, B = lib.lib, lib
+    fake = ctypes.c_void_p(0x10000)       # never dereferenced: validation fails first
+    big = 1 << 30
+    s = L.mom_permute(fake, big, 2, 4, fake, 1, fake, fake, fake, fake, fake, 1 << 20, None)
+    assert s == B.MOM_ERR_UNSUPPORTED                           # n_tok * top_k = 2^31
+    s = L.mom_kv_proj_grouped(*([fake] * 8), B.MOM_BF16, big, 256, 2, 64, 4, 2, *([fake] * 8), 4096, None)
+    assert s == B.MOM_ERR_UNSUPPORTED
+    s = L.mom_permute(fake, 10, 2, 33, fake, 1, fake, fake, fake, fake, fake, 1 << 20, None)
+    assert s == B.MOM_ERR_ARG                                   # M = 33 > MOM_MAX_MEM
+    s = L.mom_router_topk(fake, fake, None, B.MOM_BF16, 10, 64, 33, 2, fake, fake, None, None)
+    assert s == B.MOM_ERR_ARG
+    s = L.mom_kv_proj_grouped(*([fake] * 8), B.MOM_BF16, 10, 256, 65, 64, 4, 2, *([fake] * 8), 4096, None)
+    assert s == B.MOM_ERR_ARG                                   # H = 65 > MOM_MAX_HEADS
+    s = L.mom_permute_noalloc(fake, (1 << 20) + 1, 2, 4, fake, 1, fake, fake, fake, fake, fake, None)
+    assert s == B.MOM_ERR_UNSUPPORTED                           # past the static scratch
+    s = L.mom_permute(fake, -1, 2, 4, fake, 1, fake, fake, fake, fake, fake, 1 << 20, None)
+    assert s == B.MOM_ERR_ARG                                   # negative token count
