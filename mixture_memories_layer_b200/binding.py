@@ -81,7 +81,17 @@ def _check(status: int, what: str):
 
 
 def _p(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device pointer of a tensor (None -> NULL).  The C ABI reads dense
+    row-major buffers in device memory: a host tensor or a strided view is
+    refused here instead of being read as if it were one."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("MoM: a tensor on %s was passed; the library takes CUDA tensors" % t.device)
+    if not t.is_contiguous():
+        raise ValueError("MoM: a non-contiguous tensor (shape %s, strides %s) was passed; use .contiguous()"
+                         % (tuple(t.shape), t.stride()))
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _s(stream):

@@ -220,4 +220,7 @@ class MoMLayer:
 
 
 def ctypes_ptr(t: Optional[torch.Tensor]):
-    return None if t is None else t.data_ptr()
+    """Device address of a weight tensor (checked like every pointer the
+    binding passes: a dense CUDA tensor)."""
+    p = B._p(t)
+    return None if p is None else p.value

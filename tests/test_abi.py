@@ -83,3 +83,10 @@ def test_host_validation_at_the_size_limits(lib):
     assert s == B.MOM_ERR_UNSUPPORTED                           # past the static scratch
     s = L.mom_permute(fake, -1, 2, 4, fake, 1, fake, fake, fake, fake, fake, 1 << 20, None)
     assert s == B.MOM_ERR_ARG                                   # negative token count
+
+
+def test_binding_refuses_host_tensors(lib):
+    import torch
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        lib._p(torch.zeros(4))
+    assert lib._p(None) is None

@@ -153,6 +153,14 @@ def test_layer_no_tokens(with_h0):
     assert tuple(b["seg_cu"].cpu().tolist()) == (0,) * (M * 2 + 1)
 
 
+def test_binding_refuses_strided_views():
+    from mixture_memories_layer_b200 import binding as B
+    x = torch.zeros((64, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError, match="non-contiguous"):
+        B._p(x.t())
+    assert B._p(x).value == x.data_ptr()
+
+
 def test_layer_h0_hand_off():
     """Forward over [0, T) equals [0, T/2) then [T/2, T) seeded with the
     first call's final states."""
