@@ -49,10 +49,17 @@ def _worker(rank, world, port, out_dir):
         json.dump(rec, fh)
 
 
-def test_two_ranks_over_gloo(tmp_path):
+def test_two_ranks_over_gloo():
+    from tests.conftest import ROOT
+    out_dir = os.path.join(ROOT, "mixture_memories_layer_b200", "_build", "gloo_ranks")   # git-ignored scratch
+    os.makedirs(out_dir, exist_ok=True)
+    for r in range(2):
+        stale = os.path.join(out_dir, "rank%d.json" % r)
+        if os.path.exists(stale):
+            os.remove(stale)
     port = _free_port()
     ctx = mp.get_context("spawn")
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, str(tmp_path))) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out_dir)) for r in range(2)]
     for pr in procs:
         pr.start()
     for pr in procs:
@@ -61,7 +68,7 @@ def test_two_ranks_over_gloo(tmp_path):
             pr.kill()
             pytest.fail("a rank did not finish")
         assert pr.exitcode == 0
-    recs = [json.load(open(tmp_path / ("rank%d.json" % r))) for r in range(2)]
+    recs = [json.load(open(os.path.join(out_dir, "rank%d.json" % r))) for r in range(2)]
     assert all(r["world"] == 2 for r in recs)
     assert all(r["max"] == 20.0 for r in recs)                  # max over ranks
     assert recs[0]["x_shape"] == recs[1]["x_shape"]            # same per-rank work
