@@ -92,6 +92,18 @@ mom_status mom_clear_error(void* ws, void* stream);
  * process (all devices, all streams).  Host-side counter, thread-safe. */
 uint64_t mom_launch_count(void);
 
+/* Diagnostic self-test of the failure path every pipelined kernel shares:
+ * launches one thread that waits, with the library's bounded barrier wait,
+ * on a barrier that nothing signals.  After `limit_cycles` SM cycles
+ * (1 .. 4e9; about 2e6 is a millisecond) the wait gives up, records
+ * MOM_DEVERR_TIMEOUT with info MOM_SELFTEST_WAIT_SITE in the error record of
+ * `ws` (at least MOM_WS_HEADER_BYTES), and the kernel returns: the context
+ * stays usable and mom_get_error reports the record.  Asynchronous on
+ * `stream`.  MOM_ERR_ARG for a NULL or short workspace or a limit out of
+ * range. */
+#define MOM_SELFTEST_WAIT_SITE 990
+mom_status mom_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t limit_cycles, void* stream);
+
 /* ------------------------------------------------------------------------
  * mom_router_topk -- the router: one matmul, one softmax, one top-k, one
  * renormalisation (explainer, "Router mechanics, step by step"; blog post,

@@ -20,6 +20,7 @@ MOM_OK, MOM_ERR_ARG, MOM_ERR_UNSUPPORTED, MOM_ERR_CUDA, MOM_ERR_DEVICE = 0, 1, 2
 MOM_F32, MOM_BF16 = 0, 1
 MOM_DEVERR_NONE, MOM_DEVERR_MEM_INDEX, MOM_DEVERR_ROW_INDEX, MOM_DEVERR_SEGMENT, MOM_DEVERR_TIMEOUT = 0, 1, 2, 3, 4
 MOM_WS_HEADER_BYTES = 256
+MOM_SELFTEST_WAIT_SITE = 990
 
 # every function the header declares, with (restype, argtypes)
 _VP, _I, _I64, _F, _SZ = c_void_p, c_int, c_int64, c_float, c_size_t
@@ -28,6 +29,7 @@ SIGNATURES = {
     "mom_get_error": (_I, [_VP, POINTER(c_int32), POINTER(c_int32), _VP]),
     "mom_clear_error": (_I, [_VP, _VP]),
     "mom_launch_count": (ctypes.c_uint64, []),
+    "mom_selftest_wait_timeout": (_I, [_VP, _SZ, _I64, _VP]),
     "mom_router_topk": (_I, [_VP, _VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "mom_permute_workspace_size": (_SZ, [_I64, _I, _I, _I]),
     "mom_permute": (_I, [_VP, _I64, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -129,6 +131,11 @@ def mom_launch_count() -> int:
 
 def mom_clear_error(ws: torch.Tensor, stream=None):
     _check(lib.mom_clear_error(_p(ws), _s(stream)), "mom_clear_error")
+
+
+def mom_selftest_wait_timeout(ws: torch.Tensor, limit_cycles: int, stream=None):
+    _check(lib.mom_selftest_wait_timeout(_p(ws), ws.numel(), int(limit_cycles), _s(stream)),
+           "mom_selftest_wait_timeout")
 
 
 # ------------------------------------------------------- the six entry points

@@ -46,15 +46,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // timeout it raises *abort and records MOM_DEVERR_TIMEOUT.  Returns false
 // when the caller must stop.
 constexpr long long kWaitCycles = 4000000000LL;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, void* err,
-                                          int where) {
+// The same with the limit given (the self-test of this failure path uses a
+// short one); mbar_wait is this with kWaitCycles.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, volatile int* abort, void* err,
+                                                int where, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     uint32_t n = 0;
     while (!mbar_try_wait(bar, parity)) {
         if ((++n & 63u) == 0) {
             if (*abort) return false;
-            if (clock64() - t0 > kWaitCycles) {
+            if (clock64() - t0 > limit) {
                 *abort = 1;
                 record_error(err, MOM_DEVERR_TIMEOUT, where);
                 return false;
@@ -62,6 +64,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         }
     }
     return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, void* err,
+                                          int where) {
+    return mbar_wait_limit(bar, parity, abort, err, where, kWaitCycles);
 }
 
 // Bounded wait used while tearing down (ignores the abort flag): waits for
