@@ -75,9 +75,13 @@ def step_work(w):
     }
 
 
-def layer_roofline(w, peaks):
+def layer_roofline(w, peaks, n_seq=None):
+    """(FLOPs, bytes, roofline seconds) of one layer forward: the bytes are
+    x, the weights, the output, every final state (one per sequence for the
+    shared memory and for each routed memory) and the routing; n_seq is the
+    number of sequences (default: the workload's fixed batch)."""
     N, D, H, d, M, K = w.n_tokens, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k
-    S = w.batch
+    S = w.batch if n_seq is None else n_seq
     sw = step_work(w)
     flops = sw["proj"]["flops"] + sw["gdn"]["flops"] \
         + 2 * N * D * M + 2 * K * N * H * d

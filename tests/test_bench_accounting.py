@@ -1,0 +1,58 @@
+"""The arithmetic behind bench.py's line: algorithmic work of each call, the
+layer roofline and whole-job throughput, checked against figures worked out
+independently from the definitions (the FLOP and byte counts of the 380M
+and 1.3B layer shapes), and the DRAM-traffic record's tie to the GDN source
+it was measured on."""
+import numpy as np
+import pytest
+
+import bench
+from mixture_memories_layer_b200 import synth
+
+PEAKS = {"bf16_tflops": 1631.7, "hbm_gbs": 6540.2}
+
+
+def _close(a, b, rel=5e-4):
+    return abs(a - b) <= rel * abs(b)
+
+
+def test_380m_layer_work_and_roofline():
+    w = synth.WORKLOADS["mom380m"]
+    sw = bench.step_work(w)
+    # projections 2 N D (3Hd + 2H) + 2 N k D 2Hd; recurrence 6 N (1+k) H d^2
+    assert _close(sw["proj"]["flops"], 240.8e9, 1e-3)
+    assert _close(sw["gdn"]["flops"], 77.3e9, 1e-3)
+    flops, bytes_, t = bench.layer_roofline(w, PEAKS)
+    assert _close(flops, 318.3e9, 1e-3)
+    assert _close(bytes_, 132.4e6, 1e-3)
+    assert _close(t, 0.1951e-3, 1e-3)                 # tensor-bound: flops / peak
+    assert _close(w.n_tokens / t, 84.0e6, 1e-3)       # roofline tokens/s
+
+
+def test_1p3b_layer_work():
+    w = synth.WORKLOADS["mom1p3b_m16"]
+    flops, bytes_, t = bench.layer_roofline(w, PEAKS)
+    assert _close(flops, 1771.9e9, 1e-3)
+    assert _close(bytes_, 571.1e6, 1e-3)
+    assert _close(t, 1.0859e-3, 1e-3)
+
+
+def test_final_states_are_counted_per_sequence():
+    # varlen workloads have no fixed batch: the number of sequences is passed
+    w = synth.WORKLOADS["mom380m_skew_varlen"]
+    S = len(synth.make_problem(w)["cu_seqlens"]) - 1
+    b0 = bench.layer_roofline(w, PEAKS, n_seq=0)[1]
+    bS = bench.layer_roofline(w, PEAKS, n_seq=S)[1]
+    assert bS - b0 == (1 + w.n_mem) * S * w.heads * w.d_head ** 2 * 4
+
+
+def test_whole_job_throughput_uses_the_slowest_rank():
+    assert bench.aggregate_throughput(16384, 2, 20, 12.4) == pytest.approx(16384 * 2 * 20 / 0.0124)
+
+
+def test_gdn_traffic_record_matches_the_current_source():
+    # profiles/traffic.json holds the ncu DRAM bytes of one GDN call together
+    # with the hash of the source they were measured on; the bench reports
+    # them only while that source is unchanged
+    t = bench.measured_traffic("gdn")
+    assert t == 622_900_000, "gdn_chunk_tc.cu changed since its traffic was captured: re-capture it"
