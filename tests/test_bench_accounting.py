@@ -56,3 +56,15 @@ def test_gdn_traffic_record_matches_the_current_source():
     # them only while that source is unchanged
     t = bench.measured_traffic("gdn")
     assert t == 622_900_000, "gdn_chunk_tc.cu changed since its traffic was captured: re-capture it"
+
+
+def test_clock_summary_names_every_throttle_reason_seen():
+    c = bench.ClockSampler(torch_device=None)
+    c.sm_max = 1965
+    c.samples = [(1965, 0x0), (1950, 0x4), (1800, 0x8 | 0x4), (1965, 0x40)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1957.5 and s["sm_max_mhz"] == 1965 and s["samples"] == 4
+    assert s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
+    empty = bench.ClockSampler(torch_device=None)
+    empty.sm_max = None
+    assert empty.summary()["reasons"] == ["unsampled"]
