@@ -195,3 +195,18 @@ def test_projection_closed_forms():
             for c in range(d):
                 ref = sum(x[n, i] * p["w_v_sh"][h * d + c, i] for i in range(D))
                 assert abs(v_sh[n, h, c] - ref) < 1e-12
+
+
+def test_elementwise_helpers_against_math_module():
+    # the gates' building blocks, checked against Python's math library one
+    # value at a time, including inputs far outside the workloads' range
+    import math
+    for z in (-30.0, -5.0, -0.3, 0.0, 0.7, 5.0, 30.0):
+        assert abs(orc.softplus(np.array(z)) - math.log1p(math.exp(z))) <= 1e-15 * max(1.0, abs(z))
+        assert abs(orc.sigmoid(np.array(z)) - 1.0 / (1.0 + math.exp(-z))) <= 1e-16
+        assert abs(orc.sigmoid(np.array(-z)) - (1.0 - orc.sigmoid(np.array(z)))) <= 1e-15
+    assert orc.softplus(np.array(800.0)) == 800.0 and orc.softplus(np.array(-800.0)) == 0.0
+    y = orc.l2norm(np.array([[3.0, 4.0], [0.0, 0.0]]))
+    assert abs(y[0, 0] - 3.0 / math.sqrt(25.0 + orc.NORM_EPS)) <= 1e-16 and np.all(y[1] == 0.0)
+    p = orc.softmax(np.array([1000.0, 1000.0, 998.0]))     # no overflow
+    assert abs(p[0] - 1.0 / (2.0 + math.exp(-2.0))) <= 1e-15
