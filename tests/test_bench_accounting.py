@@ -1,8 +1,8 @@
 """The arithmetic behind bench.py's line: algorithmic work of each call, the
 layer roofline and whole-job throughput, checked against figures worked out
 independently from the definitions (the FLOP and byte counts of the 380M
-and 1.3B layer shapes), and the DRAM-traffic record's tie to the GDN source
-it was measured on."""
+and 1.3B layer shapes); the DRAM-traffic record's tie to the source it was
+measured on; the clock summary."""
 import numpy as np
 import pytest
 
@@ -50,12 +50,28 @@ def test_whole_job_throughput_uses_the_slowest_rank():
     assert bench.aggregate_throughput(16384, 2, 20, 12.4) == pytest.approx(16384 * 2 * 20 / 0.0124)
 
 
-def test_gdn_traffic_record_matches_the_current_source():
-    # profiles/traffic.json holds the ncu DRAM bytes of one GDN call together
-    # with the hash of the source they were measured on; the bench reports
-    # them only while that source is unchanged
-    t = bench.measured_traffic("gdn")
-    assert t == 622_900_000, "gdn_chunk_tc.cu changed since its traffic was captured: re-capture it"
+def test_traffic_record_is_reported_only_for_the_source_it_was_measured_on(monkeypatch):
+    # profiles/traffic.json holds a kernel's ncu DRAM bytes with the hash of
+    # the source they were measured on; the bench reports them only while that
+    # source is unchanged (a scratch tree stands in for the repository here)
+    import json
+    import os
+    from tests.conftest import ROOT
+    root = os.path.join(ROOT, "mixture_memories_layer_b200", "_build", "traffic_check")
+    os.makedirs(os.path.join(root, "profiles"), exist_ok=True)
+    os.makedirs(os.path.join(root, "mixture_memories_layer_b200", "csrc"), exist_ok=True)
+    src = os.path.join(root, "mixture_memories_layer_b200", "csrc", "k.cu")
+    with open(src, "w") as fh:
+        fh.write("// kernel v1\n")
+    monkeypatch.setattr(bench, "ROOT", root)
+    rec = {"k": {"source": "k.cu", "source_sha": bench.kernel_source_sha("k.cu"), "bytes_per_launch": 123}}
+    with open(os.path.join(root, "profiles", "traffic.json"), "w") as fh:
+        json.dump(rec, fh)
+    assert bench.measured_traffic("k") == 123
+    assert bench.measured_traffic("other") is None
+    with open(src, "w") as fh:
+        fh.write("// kernel v2\n")
+    assert bench.measured_traffic("k") is None
 
 
 def test_clock_summary_names_every_throttle_reason_seen():
