@@ -210,3 +210,59 @@ def test_elementwise_helpers_against_math_module():
     assert abs(y[0, 0] - 3.0 / math.sqrt(25.0 + orc.NORM_EPS)) <= 1e-16 and np.all(y[1] == 0.0)
     p = orc.softmax(np.array([1000.0, 1000.0, 998.0]))     # no overflow
     assert abs(p[0] - 1.0 / (2.0 + math.exp(-2.0))) <= 1e-15
+
+
+def _check_memory_kv(fn):
+    """Memory m's key/value projection against a pure-Python dot product per
+    element (paper card, Summary: every memory has its own key and value
+    projections): k is x . W_k^m row, then L2-normalised per head with the
+    1e-6 epsilon; v is x . W_v^m row unnormalised.  Three memories with
+    different weights, so that reading another memory's weights fails."""
+    rng = np.random.default_rng(11)
+    N, D, H, d, M = 4, 10, 2, 3, 3
+    p = dict(w_k=rng.standard_normal((M, H * d, D)), w_v=rng.standard_normal((M, H * d, D)))
+    x = rng.standard_normal((N, D))
+    for m in range(M):
+        k, v = fn(x, p, m, H, d)
+        assert k.shape == (N, H, d) and v.shape == (N, H, d)
+        for n in range(N):
+            for h in range(H):
+                raw = [sum(x[n, i] * p["w_k"][m][h * d + c][i] for i in range(D)) for c in range(d)]
+                nrm = math.sqrt(sum(r * r for r in raw) + orc.NORM_EPS)
+                for c in range(d):
+                    assert abs(k[n, h, c] - raw[c] / nrm) < 1e-12, ("k", m, n, h, c)
+                    ref_v = sum(x[n, i] * p["w_v"][m][h * d + c][i] for i in range(D))
+                    assert abs(v[n, h, c] - ref_v) < 1e-12, ("v", m, n, h, c)
+                # every head of k has unit norm (up to the epsilon)
+                assert abs(math.sqrt(sum(float(kc) ** 2 for kc in k[n, h])) - 1.0) < 1e-6
+
+
+def test_memory_kv_pure_python():
+    _check_memory_kv(orc.memory_kv)
+
+
+def _kv_swapped(x, p, m, H, d):
+    n = x.shape[0]
+    return (orc.l2norm((x @ p["w_v"][m].T).reshape(n, H, d)), (x @ p["w_k"][m].T).reshape(n, H, d))
+
+
+def _kv_unnormalised(x, p, m, H, d):
+    n = x.shape[0]
+    return (x @ p["w_k"][m].T).reshape(n, H, d), (x @ p["w_v"][m].T).reshape(n, H, d)
+
+
+def _kv_wrong_memory(x, p, m, H, d):
+    return orc.memory_kv(x, p, (m + 1) % len(p["w_k"]), H, d)
+
+
+def _kv_norm_over_all_heads(x, p, m, H, d):
+    n = x.shape[0]
+    k = orc.l2norm(x @ p["w_k"][m].T).reshape(n, H, d)
+    return k, (x @ p["w_v"][m].T).reshape(n, H, d)
+
+
+@pytest.mark.parametrize("planted", [_kv_swapped, _kv_unnormalised, _kv_wrong_memory, _kv_norm_over_all_heads])
+def test_memory_kv_pin_catches_planted_mistakes(planted):
+    # the pin above must fail for each plausible mistake in memory_kv
+    with pytest.raises(AssertionError):
+        _check_memory_kv(planted)
