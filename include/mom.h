@@ -160,12 +160,14 @@ mom_status mom_permute(const int32_t* topk_idx, int64_t n_tok, int top_k, int n_
  * Same arguments, outputs and results as mom_permute, minus ws/ws_bytes.
  * Its scratch space is a fixed array inside the library (about 1 MiB per
  * GPU that loads the library, held until the process exits), so:
- *   - n_tok may not exceed MOM_PERMUTE_NOALLOC_MAX_TOKENS (and n_mem may
- *     not exceed MOM_MAX_MEM); larger problems return MOM_ERR_UNSUPPORTED
- *     and launch nothing;
- *   - the first call on a device looks up the array's device address (a
- *     runtime query, once per device, cached); make that first call before
- *     any stream capture on that device;
+ *   - n_tok may not exceed MOM_PERMUTE_NOALLOC_MAX_TOKENS: a larger n_tok
+ *     returns MOM_ERR_UNSUPPORTED and launches nothing; n_mem above
+ *     MOM_MAX_MEM returns MOM_ERR_ARG, as for mom_permute;
+ *   - the first call in a CUDA context on a device looks up the array's
+ *     device address in that context (a runtime query, then cached while
+ *     that context stays current on the device); make that first call
+ *     before any stream capture on that device, and again after a
+ *     cudaDeviceReset or a switch to another context;
  *   - every call on a device shares the array: calls whose kernels overlap
  *     on the GPU (unordered streams, several host threads) race and may
  *     give wrong results -- order them on one stream;

@@ -16,6 +16,8 @@
 // kernels overlap on the GPU (different streams without ordering, or
 // different host threads) race on it and may produce wrong results; order
 // them on one stream.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -33,20 +35,48 @@ static __device__ __align__(256) unsigned char g_permute_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
+// Per device: the CUDA context the address was looked up in, and the address.
+// A device address belongs to one context; a host engine may run its own
+// (non-primary) context on a device, and a context can be destroyed and
+// replaced (cudaDeviceReset), so the cache is keyed on the context too.
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_permute_scratch on the current device.  In host code
+// The driver's cuCtxGetCurrent, found through the runtime (no link-time
+// libcuda dependency).
+PFN_cuCtxGetCurrent_v4000 ctx_get_current_fn() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+    });
+    return fn;
+}
+
+// Device address of g_permute_scratch in the current context.  In host code
 // the array's name is only a host-side stand-in, so the address must come
-// from the runtime; it is looked up once per device (the first call on that
-// device) and cached.
+// from the runtime; it is looked up on the first call in each context of a
+// device and cached for as long as that context stays current there.
 mom_status scratch_address(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOM_ERR_CUDA;
+    auto get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return MOM_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return MOM_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (ctx == nullptr || g_scratch_addr[dev] == nullptr || g_scratch_ctx[dev] != ctx) {
+        // the lookup also makes the runtime create the device's primary
+        // context when none is current yet
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return MOM_ERR_CUDA;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MOM_ERR_CUDA;
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_addr[dev];
     return MOM_OK;

@@ -62,6 +62,50 @@ def test_noalloc_matches_workspace_permute_two_calls_in_a_row():
         assert status.tolist() == [0, 0]
 
 
+def test_noalloc_four_launch_path_matches_workspace_permute():
+    """A tile-count table above the single cooperative launch's limit
+    (32 memories x 274 tiles of 256 tokens) takes the four-launch path, whose
+    scan also keeps its per-tile bases in the fixed array: bit for bit
+    against mom_permute, twice in a row."""
+    rng = np.random.default_rng(77)
+    n_tok, M, K = 70000, 32, 2
+    lens = [30000, 1, 0, 39999]
+    status = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        idx, cu = _problem(rng, n_tok, M, K, lens)
+        perm, row_of, offs, seg = _outputs(n_tok, M, K, len(lens))
+        B.mom_permute_noalloc(idx, M, cu, perm, row_of, offs, seg, status)
+        ref = _reference(idx, M, cu)
+        torch.cuda.synchronize()
+        for got, want in zip((perm, row_of, offs, seg), ref):
+            assert torch.equal(got, want)
+        assert status.tolist() == [0, 0]
+
+
+def test_noalloc_reports_a_bad_memory_index_in_status_out():
+    """A memory index >= M planted on the host is dropped and reported in
+    status_out as {MOM_DEVERR_MEM_INDEX, token}; the next clean call starts
+    from a cleared record and reports {0, 0}."""
+    rng = np.random.default_rng(5)
+    n_tok, M, K = 300, 4, 2
+    idx, cu = _problem(rng, n_tok, M, K, [n_tok])
+    idx[123, 1] = 9
+    status = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    perm, row_of, offs, seg = _outputs(n_tok, M, K, 1)
+    B.mom_permute_noalloc(idx, M, cu, perm, row_of, offs, seg, status)
+    torch.cuda.synchronize()
+    assert status.tolist() == [B.MOM_DEVERR_MEM_INDEX, 123]
+    assert int(offs[-1]) == n_tok * K - 1            # the bad pair was dropped
+    assert int(row_of[123 * K + 1]) == -1
+    idx[123, 1] = (int(idx[123, 0]) + 1) % M
+    B.mom_permute_noalloc(idx, M, cu, perm, row_of, offs, seg, status)
+    ref = _reference(idx, M, cu)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0, 0]
+    for got, want in zip((perm, row_of, offs, seg), ref):
+        assert torch.equal(got, want)
+
+
 def test_noalloc_refuses_problems_beyond_its_fixed_scratch():
     n_tok = B.MOM_PERMUTE_NOALLOC_MAX_TOKENS + 1
     idx = torch.zeros((n_tok, 1), dtype=torch.int32, device="cuda")
