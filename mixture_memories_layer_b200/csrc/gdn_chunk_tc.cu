@@ -1050,16 +1050,11 @@ int64_t max_chunks(int64_t n_rows, int n_seg) { return n_rows / C + n_seg; }
 
 template <int D>
 cudaError_t launch_d(const GdnTc& t, int64_t mchunks, int phase, cudaStream_t st) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)PrepLayout<D>::BYTES);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(gdn_state_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)StateLayout<D>::BYTES);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static unsigned long long optin_prep = 0, optin_state = 0;
+    cudaError_t e = smem_optin((const void*)gdn_prep_kernel<D>, (int)PrepLayout<D>::BYTES, &optin_prep);
+    if (e != cudaSuccess) return e;
+    e = smem_optin((const void*)gdn_state_kernel<D>, (int)StateLayout<D>::BYTES, &optin_state);
+    if (e != cudaSuccess) return e;
     const int HD = t.H * D;
     CUtensorMap tm_k, tm_v, tm_q;
     if (!make_tma_2d_bf16(&tm_k, t.k, (uint64_t)t.n_rows, HD, HD, 64, C)) return cudaErrorInvalidValue;

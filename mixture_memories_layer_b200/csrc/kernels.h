@@ -12,6 +12,12 @@ namespace mom {
 // Counts every kernel launch (mom_launch_count).
 void count_launches(int n);
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device.  The limit is a per-device setting, so it is set once per
+// (kernel, device): `done` holds one bit per device already set (devices
+// 0..63; others are set on every call).
+cudaError_t smem_optin(const void* func, int bytes, unsigned long long* done);
+
 // tma_host.cu: tensor maps for bf16 row-major matrices (128-byte swizzle,
 // boxes of box_rows x box_cols with box_cols * 2 == 128 bytes) and the
 // device-generation check of the tcgen05 paths.

@@ -405,13 +405,9 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     p.n_tiles = p.sh_tiles + (cdiv(a.n_tok * a.K, BM) + a.M) * p.rt_ct;
     p.ws = a.ws;
 
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static unsigned long long optin_done = 0;
+    cudaError_t e = smem_optin((const void*)proj_tc_kernel, (int)SMEM_BYTES, &optin_done);
+    if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
