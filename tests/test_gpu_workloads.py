@@ -8,8 +8,14 @@ The GPU runs the whole batch.  What the oracle checks:
 * projections on a seeded sample of tokens and reordered rows;
 * layer outputs and final states on whole sampled sequences (sequences are
   independent, so the oracle runs one of them alone with the GPU's routing
-  imposed); for the 1.3B shape, the outputs of the first 384 tokens of a
-  sequence (a prefix of a causal recurrence is exact on its own).
+  imposed): for the skewed varlen batch, the sequence holding memory 0's
+  longest routed segment and the clipped last one; for the 1.3B shape, one
+  whole 4096-token sequence (64 chunks, 16 memories).
+
+Tokens whose k-th and (k+1)-th router logits lie within 1e-4 of each other
+(near ties: rounding may flip their choice) are counted, printed and left
+out of the exact index comparison; the output comparison imposes the GPU's
+routing on the oracle, so they are still covered there.
 """
 import numpy as np
 import pytest
@@ -30,7 +36,9 @@ def _need_cuda():
 def _routing_and_permute(w, p, res):
     idx, gate, logits, near = orc.router_topk(p["x"], p["w_r"], p["b_r"], w.top_k)
     keep = ~near
-    assert np.array_equal(res["idx"][keep], idx[keep])
+    n_near = int(near.sum())
+    print("%s: %d near-tie tokens of %d excluded from the exact index check" % (w.name, n_near, w.n_tokens))
+    assert np.array_equal(res["idx"][keep], idx[keep]), ("routing", w.name, "near ties excluded", n_near)
     assert max_abs_rel(res["gate"][keep], gate[keep]) < 1e-5
     perm, row_of, offs, seg = orc.permute(res["idx"], w.n_mem, p["cu_seqlens"])
     assert np.array_equal(res["perm"][:offs[-1]], perm)
@@ -96,7 +104,15 @@ def test_mom380m_skewed_varlen_full_size():
     assert counts[0] > 2 * counts[1:].max()
     _projections_sampled(w, p, res, seed=1)
     S = len(p["cu_seqlens"]) - 1
-    _sequence(w, p, res, s=S - 1)      # the last (clipped, shortest) sequence
+    # the sequence holding memory 0's longest routed segment (the longest
+    # chain of the routed walks), with its final states, then the last
+    # (clipped, shortest) sequence
+    seg = res["seg_cu"]
+    longest = int(np.argmax(np.diff(seg[:S + 1])))
+    assert seg[longest + 1] - seg[longest] > 1000
+    _sequence(w, p, res, s=longest)
+    if longest != S - 1:
+        _sequence(w, p, res, s=S - 1)
 
 
 def test_mom1p3b_m16_full_size():
@@ -106,7 +122,7 @@ def test_mom1p3b_m16_full_size():
     assert lay.device_errors() == {}
     _routing_and_permute(w, p, res)
     _projections_sampled(w, p, res, n=128, seed=2)
-    _sequence(w, p, res, s=2, max_tokens=384)
+    _sequence(w, p, res, s=2)          # one whole 4096-token sequence with its final states
 
 
 def test_no_wait_runs_to_its_limit():
