@@ -11,7 +11,9 @@ are seeded synthetic tensors already resident in HBM; L2 is flushed (a
 256 MiB write) before every timed step, outside its events.  The recurrent
 decode step (256 sequences, 8 memories top-2, one new token per sequence,
 float32 states of 2.4 GB, larger than L2) is timed in the same run and
-reported under "decode".
+reported under "decode".  The other forward workloads (the tiny float32
+layer, the skewed-routing varlen batch and the 1.3B-shape 16-memory layer)
+are timed the same way and reported under "configs".
 
 With N > 1 (torchrun, one rank per GPU) every rank runs its own batch of
 sequences: the layer shards by sequence with no collective on the data
@@ -39,13 +41,20 @@ METRIC = "MoM layer fwd tokens/s at 1 B200 and % of roofline; decode tokens/s"
 UNIT = "tokens/s"
 FWD = "mom380m"
 DEC = "decode_b256"
+EXTRA = ("tiny_fp32", "mom380m_skew_varlen", "mom1p3b_m16")
+TIE_GAP = 1e-4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 def workload_desc(w):
-    return ("MoM layer forward, %s shape: B=%d x T=%d tokens, d_model=%d, H=%d, d_k=d_v=%d, "
-            "M=%d memories top-%d + shared, bf16 activations / fp32 state"
-            % (w.name, w.batch, w.seq_len, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k))
+    if w.varlen_total:
+        toks = "%d packed tokens, sequence lengths U{%d..%d}" % (w.varlen_total, w.varlen_min, w.varlen_max)
+    else:
+        toks = "B=%d x T=%d tokens" % (w.batch, w.seq_len)
+    bias = ", router bias +%g on memory 0" % w.router_bias0 if w.router_bias0 else ""
+    types = "bf16 activations / fp32 state" if w.dtype == "bf16" else "float32 throughout"
+    return ("MoM layer forward, %s shape: %s, d_model=%d, H=%d, d_k=d_v=%d, M=%d memories top-%d + shared%s, %s"
+            % (w.name, toks, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k, bias, types))
 
 
 def load_peaks():
@@ -99,16 +108,21 @@ def kernel_source_sha(name):
 
 
 def measured_traffic(call):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel's
-    source is unchanged since it was taken."""
+    """(DRAM bytes per launch from a committed ncu capture, status): the
+    bytes only while the kernel's source is unchanged since the capture was
+    taken; status is "current", "stale" (a warning is printed) or "none"."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
-        return None
+        return None, "none"
     with open(path) as fh:
         t = json.load(fh).get(call)
-    if not t or kernel_source_sha(t["source"]) != t.get("source_sha"):
-        return None
-    return t["bytes_per_launch"]
+    if not t:
+        return None, "none"
+    if kernel_source_sha(t["source"]) != t.get("source_sha"):
+        print("warning: profiles/traffic.json predates the current %s; roofline.traffic is null until it is "
+              "re-captured" % t["source"], file=sys.stderr)
+        return None, "stale"
+    return t["bytes_per_launch"], "current"
 
 
 # -------------------------------------------------------------------- clocks
@@ -232,6 +246,72 @@ def aggregate_throughput(tokens_per_rank, world, steps, max_total_ms):
 
 
 # ------------------------------------------------------------- the GPU arm
+def time_forward(lay, x, cu, steps, flush):
+    """`steps` layer forwards, L2 flushed before each outside its events.
+    Returns (per-step ms list, mean ms per call of MoMLayer.STEPS)."""
+    import torch
+    from mixture_memories_layer_b200 import layer as L
+    n_calls = len(L.MoMLayer.STEPS)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_calls + 1)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for s in range(steps):
+        flush.zero_()                          # evict L2 (outside the step's events)
+        lay.forward(x, cu, marks=marks[s])
+    torch.cuda.synchronize()
+    step_ms = [marks[s][0].elapsed_time(marks[s][n_calls]) for s in range(steps)]
+    per_call = {name: sum(marks[s][i].elapsed_time(marks[s][i + 1]) for s in range(steps)) / steps
+                for i, name in enumerate(L.MoMLayer.STEPS)}
+    return step_ms, per_call
+
+
+def near_tie_tokens(x, w_r, b_r, top_k, gap=TIE_GAP):
+    """Tokens whose k-th and (k+1)-th router logits (float32, on the device)
+    lie within `gap`: rounding may flip their choice, so parity tests leave
+    them out of the exact index check.  Reported, not used by the layer."""
+    import torch
+    if top_k >= w_r.shape[0]:
+        return 0
+    logits = x.float() @ w_r.float().t() + b_r.float()
+    top = torch.topk(logits, top_k + 1, dim=-1).values
+    return int(((top[:, top_k - 1] - top[:, top_k]) < gap).sum().item())
+
+
+def config_bench(name, dev, steps, warmup, peaks, flush):
+    """One of the other forward workloads, timed like the headline one."""
+    import torch
+    from mixture_memories_layer_b200 import layer as L
+    from mixture_memories_layer_b200 import synth
+    w = synth.WORKLOADS[name]
+    p = synth.make_problem(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    lay = L.MoMLayer(L.pack_weights(p, dt, dev), w.heads, w.d_head, w.top_k)
+    x = torch.as_tensor(p["x"]).to(dev, dt)
+    cu = torch.as_tensor(p["cu_seqlens"]).to(dev)
+    for _ in range(warmup):
+        lay.forward(x, cu)
+    torch.cuda.synchronize()
+    errs = lay.device_errors()
+    if errs:
+        raise SystemExit("device error records in %s: %s" % (name, errs))
+    step_ms, per_call = time_forward(lay, x, cu, steps, flush)
+    ms = sum(step_ms) / steps
+    S = int(cu.numel()) - 1
+    rows = lay.buffers(w.n_tokens, S)["mem_offset"].cpu().tolist()
+    out = {"workload": workload_desc(w), "dtype": w.dtype, "tokens": w.n_tokens, "sequences": S,
+           "ms_per_step": ms, "value": w.n_tokens / (ms / 1e3), "unit": UNIT, "per_call_ms": per_call,
+           "routed_rows_per_memory": [b - a for a, b in zip(rows[:-1], rows[1:])],
+           "near_tie_tokens": near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)}
+    if w.dtype == "bf16":
+        lf, lb, lt = layer_roofline(w, peaks, n_seq=S)
+        gdn = step_work(w)["gdn"]["flops"] / (per_call["gdn"] / 1e3) / 1e12
+        out["layer_roofline"] = {"flops": lf, "bytes": lb, "roofline_ms": lt * 1e3, "frac": lt * 1e3 / ms}
+        out["gdn_tflops"] = gdn
+        out["gdn_frac"] = gdn / peaks["bf16_tflops"]
+    else:
+        out["layer_roofline"] = {"bound": "latency", "note": "float32 CUDA-core path; latency only"}
+    return out
+
+
 def gpu_arm(args):
     import torch
 
@@ -267,21 +347,12 @@ def gpu_arm(args):
     if errs:
         raise SystemExit("device error records after warm-up: %s" % errs)
 
-    n_calls = len(L.MoMLayer.STEPS)
-    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_calls + 1)] for _ in range(args.steps)]
     launches0 = B.mom_launch_count()
     barrier()
-    torch.cuda.synchronize()
-    for s in range(args.steps):
-        flush.zero_()                          # evict L2 (outside the step's events)
-        lay.forward(x, cu, marks=marks[s])
-    torch.cuda.synchronize()
+    step_ms, per_call = time_forward(lay, x, cu, args.steps, flush)
     barrier()
     launches = B.mom_launch_count() - launches0
-    step_ms = [marks[s][0].elapsed_time(marks[s][n_calls]) for s in range(args.steps)]
     total_ms = max_over_ranks(sum(step_ms))
-    per_call = {name: sum(marks[s][i].elapsed_time(marks[s][i + 1]) for s in range(args.steps)) / args.steps
-                for i, name in enumerate(L.MoMLayer.STEPS)}
     ms_per_step = total_ms / args.steps
     value = aggregate_throughput(w.n_tokens, world, args.steps, total_ms)
 
@@ -298,8 +369,9 @@ def gpu_arm(args):
         achieved = wk["bytes"] / sec / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
-    roof.update({"kernel": top, "traffic": measured_traffic(top), "peak_source": peaks["source"],
-                 "ms_per_launch": per_call[top]})
+    traffic, traffic_status = measured_traffic(top)
+    roof.update({"kernel": top, "traffic": traffic, "traffic_record": traffic_status,
+                 "peak_source": peaks["source"], "ms_per_launch": per_call[top]})
     lf, lb, lt = layer_roofline(w, peaks)
     layer_roof = {"flops": lf, "bytes": lb, "roofline_ms": lt * 1e3, "frac": (lt * 1e3) / ms_per_step}
 
@@ -308,8 +380,13 @@ def gpu_arm(args):
     if not args.no_e2e:
         e2e = e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks)
     decode = None if args.no_decode else decode_bench(args, dev, world, rank, max_over_ranks, barrier)
+    configs = None
+    if not args.no_configs and world == 1:
+        configs = {name: config_bench(name, dev, args.steps, args.warmup, peaks, flush) for name in EXTRA}
     clocks.__exit__(None, None, None)
-    return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode)
+    layer_roof["near_tie_tokens"] = near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)
+    return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,
+                  configs)
 
 
 def e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks):
@@ -363,7 +440,8 @@ def e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks):
                                       "(two buffer sets, three streams); no L2 flush (each step touches ~0.6 GB)"}
 
 
-def finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode):
+def finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,
+           configs=None):
     import torch.distributed as dist
     result = None
     if rank == 0:
@@ -378,7 +456,7 @@ def finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call,
                        "l2": "flushed before every timed step (256 MiB write, untimed)"},
             "roofline": roof, "layer_roofline": layer_roof,
             "per_call_ms": per_call, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clocks.summary(), "decode": decode,
+            "gpu_launches": launches, "clocks": clocks.summary(), "decode": decode, "configs": configs,
         }
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -429,57 +507,94 @@ def decode_bench(args, dev, world, rank, max_over_ranks, barrier):
 
 
 # --------------------------------------------------------- CPU oracle timing
-def _threads():
-    try:
-        from threadpoolctl import threadpool_info
-        info = threadpool_info()
-        return max([i.get("num_threads", 1) for i in info] or [1])
-    except Exception:
-        return 1
+# The oracle is plain single-threaded numpy per sequence; the sequences of a
+# batch are independent, so the timed CPU legs run one sequence (or one
+# window of it) per host process, each process with one BLAS thread.  The
+# pool is started with "spawn" (never forked from a process that has used
+# the GPU).
+_ORACLE = {}
 
 
-def cpu_baseline(w, n_tokens=2048):
-    from oracle import mom_oracle as orc
+def _oracle_init(name):
+    from threadpoolctl import threadpool_limits
     from mixture_memories_layer_b200 import synth
-    p = synth.make_problem(w)
-    x = p["x"][:n_tokens]
-    t0 = time.perf_counter()
-    orc.mom_forward(x, p, np.array([0, n_tokens]), w.top_k, w.heads, w.d_head)
-    dt = time.perf_counter() - t0
-    return {"value": n_tokens / dt, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": "first %d tokens of sequence 0 (one full sequence) of the same workload; fp64 numpy, "
-                      "BLAS-threaded projections, single-threaded token recurrence; %.1f s" % (n_tokens, dt)}
+    _ORACLE["limit"] = threadpool_limits(1)
+    w = synth.WORKLOADS[name]
+    _ORACLE["w"], _ORACLE["p"] = w, synth.make_problem(w)
+
+
+def _oracle_window(job):
+    """Oracle layer forward on tokens [t0, t0 + n) of sequence s (states
+    from zero); returns (tokens, seconds)."""
+    from oracle import mom_oracle as orc
+    s, t0, n = job
+    w, p = _ORACLE["w"], _ORACLE["p"]
+    a = int(p["cu_seqlens"][s]) + t0
+    n = min(n, int(p["cu_seqlens"][s + 1]) - a)
+    t = time.perf_counter()
+    orc.mom_forward(p["x"][a:a + n], p, np.array([0, n]), w.top_k, w.heads, w.d_head)
+    return n, time.perf_counter() - t
+
+
+def _oracle_pool(name, procs):
+    import multiprocessing as mp
+    pool = mp.get_context("spawn").Pool(procs, initializer=_oracle_init, initargs=(name,))
+    pool.map(_oracle_window, [(0, 0, 1)] * procs)      # every worker started and warm
+    return pool
+
+
+def _oracle_procs(w):
+    return max(1, min(w.batch, os.cpu_count() or 1))
+
+
+def cpu_baseline(w):
+    """Whole sequences of the workload through the oracle, one per host
+    process: tokens of all of them over the slowest one's time."""
+    procs = _oracle_procs(w)
+    pool = _oracle_pool(w.name, procs)
+    try:
+        res = pool.map(_oracle_window, [(s, 0, w.seq_len) for s in range(procs)], chunksize=1)
+    finally:
+        pool.close()
+        pool.join()
+    toks, sec = sum(n for n, _ in res), max(t for _, t in res)
+    return {"value": toks / sec, "unit": UNIT, "cores": procs, "kind": "oracle",
+            "sample": "%d whole %d-token sequences of the same workload, one per host process (one BLAS thread "
+                      "each), fp64 numpy; tokens over the slowest process's %.1f s" % (procs, w.seq_len, sec)}
 
 
 def reference_arm(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return None
-    from oracle import mom_oracle as orc
     from mixture_memories_layer_b200 import synth
     w = synth.WORKLOADS[FWD]
-    p = synth.make_problem(w)
-    T = 128                       # tokens per step: one bounded window of one sequence
-    n_win = w.n_tokens // T
+    T = 128                       # tokens per sequence per step: one bounded window
+    n_win = w.seq_len // T
+    procs = _oracle_procs(w)
+    pool = _oracle_pool(w.name, procs)
 
     def step(i):
-        t0 = (i % n_win) * T
-        orc.mom_forward(p["x"][t0:t0 + T], p, np.array([0, T]), w.top_k, w.heads, w.d_head)
+        return pool.map(_oracle_window, [(s, (i % n_win) * T, T) for s in range(procs)], chunksize=1)
 
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(args.warmup + i)
-    sec = time.perf_counter() - t0
-    value = T * args.steps / sec
-    sample = ("each step: the oracle layer forward on a %d-token window (state from zero) of one sequence of "
-              "the same workload" % T)
+    try:
+        for i in range(args.warmup):
+            step(i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            step(args.warmup + i)
+        sec = time.perf_counter() - t0
+    finally:
+        pool.close()
+        pool.join()
+    value = procs * T * args.steps / sec
+    sample = ("each step: the oracle layer forward on a %d-token window (state from zero) of each of %d "
+              "sequences of the same workload, one sequence per host process (one BLAS thread each)" % (T, procs))
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3 / max(args.steps, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic: seeded, same generator as the GPU arm",
-           "config": {"workload": workload_desc(w), "tokens_per_step": T},
-           "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle", "sample": sample},
+           "config": {"workload": workload_desc(w), "tokens_per_step": procs * T},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": procs, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return out
@@ -494,6 +609,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode timing")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other forward workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -67,11 +67,19 @@ def test_traffic_record_is_reported_only_for_the_source_it_was_measured_on(monke
     rec = {"k": {"source": "k.cu", "source_sha": bench.kernel_source_sha("k.cu"), "bytes_per_launch": 123}}
     with open(os.path.join(root, "profiles", "traffic.json"), "w") as fh:
         json.dump(rec, fh)
-    assert bench.measured_traffic("k") == 123
-    assert bench.measured_traffic("other") is None
+    assert bench.measured_traffic("k") == (123, "current")
+    assert bench.measured_traffic("other") == (None, "none")
     with open(src, "w") as fh:
         fh.write("// kernel v2\n")
-    assert bench.measured_traffic("k") is None
+    assert bench.measured_traffic("k") == (None, "stale")
+
+
+def test_committed_traffic_record_status_is_reported():
+    # the repository's own record: either it matches the current GDN source
+    # (its bytes are reported) or the bench says it is stale and reports none
+    traffic, status = bench.measured_traffic("gdn")
+    assert status in ("current", "stale")
+    assert (traffic is not None) == (status == "current")
 
 
 def test_clock_summary_names_every_throttle_reason_seen():
