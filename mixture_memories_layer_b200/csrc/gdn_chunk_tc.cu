@@ -7,12 +7,16 @@
 // is evaluated in chunks of C = 64 rows.  With gamma_r the running sum of
 // log alpha inside the chunk, S the state at the chunk start, and
 // Tb = (I + L)^-1 diag(beta), L_rs = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r):
-//   U^T = (V^T - Z~) Tb^T,        Z~ = (S K^T) diag(e^gamma)     (d_v x C)
+//   U^T = Y Tb^T,   Y = V^T - (S K^T) diag(e^gamma)                 (d_v x C)
 //   o_r = e^(gamma_r) S q_r + sum_{s<=r} e^(gamma_r-gamma_s) (q_r.k_s) u_s
 //   S'  = e^(gamma_C) S + sum_s e^(gamma_C-gamma_s) u_s k_s^T
 // where u_r = beta_r (v_r - alpha_r S_{r-1} k_r) are the delta-rule
-// corrections.  Every product keeps the d_v rows of S as the MMA's M
-// dimension (128 TMEM lanes): every MMA is M = 128.
+// corrections.  U enters both the output and the next state only through
+// products with state-independent matrices, so the serial walk never forms
+// it: with P_rs = e^(gamma_r-gamma_s) q_r.k_s (s <= r),
+//   O = e^gamma S Q^T + Y (P Tb)^T,   S' = e^(gamma_C) S + Y Tb^T diag(e^(gamma_C-gamma)) K.
+// Every product keeps the d_v rows of S as the MMA's M dimension (128 TMEM
+// lanes): every walk MMA is M = 128.
 //
 // Three launches per call, in two stream-ordered phases (the prep of
 // every chunk does not depend on the state):
@@ -20,18 +24,20 @@
 //   prep    : per (chunk, head): G = [K;Q] K^T on the tensor cores; the
 //             decay matrix by running products of alpha; T = (I + L)^-1 by
 //             16 x 16 blocks (diagonal blocks by forward substitution in
-//             fp32, off-diagonal block products on tf32 tensor cores);
-//             Tb = T diag(beta) and the causal decayed P = (Q K^T) o D as
-//             pre-swizzled bf16 64 x 64 images
+//             fp32, off-diagonal block products on tf32 tensor cores); then
+//             on the tensor cores Wk = Tb^T diag(e^(gamma_C-gamma)) K and
+//             Q' = P Tb, stored as one bf16 image per (chunk, head)
 //   state   : per (segment, head, 128-row d_v tile), the serial walk over the
 //             segment's chunks with the state resident in TMEM (T = rho S,
-//             fp32) and its bf16 copy in TMEM as the A operand of
-//             [Z | X] = T [K; q~]^T; the chunk decay is the MMA's
-//             power-of-two accumulator scale plus a change of the running
-//             scalar rho.  Roles: one producer warp (TMA loads, chunk gates),
-//             three q~ warps (q rows, through the index when given, scaled
-//             in place), one MMA warp ([Z | X] in two d_k halves), eight math
-//             warps (the last to finish a step issues the next MMAs).
+//             fp32) and its bf16 copy in TMEM as the A operand of Z = T K^T
+//             and X = T q~^T; per chunk Y = V^T - Z diag(e^gamma / rho), then
+//             X += Y Q'^T and T <- 2^-e T + (rho' Y) Wk.  The chunk decay is
+//             the MMA's power-of-two accumulator scale plus a change of the
+//             running scalar rho.  Roles: one producer warp (TMA and bulk
+//             loads, chunk gates), three q~ warps (q rows, through the index
+//             when given, scaled in place), one MMA warp (Z in two d_k
+//             halves, then X), eight math warps (the last to finish Y issues
+//             the output and state-update MMAs).
 // Rows past a segment's end are masked (zero gates, zeroed key/value rows),
 // so a ragged tail chunk needs no padding.
 #include "common.cuh"
@@ -46,8 +52,7 @@ using namespace sm100;
 constexpr int C = 64;                 // chunk length
 constexpr int DVT = 128;              // d_v rows per state CTA (TMEM lanes)
 constexpr int IMG = C * C * 2;        // one swizzled 64x64 bf16 tile
-constexpr int GB = 2 * C + 4;         // floats per chunk-gate record
-constexpr int LP = C + 1;             // row pitch (floats) of the prep's fp32 tiles: no bank conflicts
+constexpr int GB = C + 4;             // floats per chunk-gate record
 
 struct GdnTc {
     const bf16* q;
@@ -122,12 +127,10 @@ gdn_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_seg, int64_t n_row
 }
 
 // Gates of one chunk, by one full warp (lane l holds rows 2l and 2l+1):
-// beta (0 past n) and gamma, the running sum of log alpha from the chunk
-// start.  Returns gamma of the last valid row.  Both the prep and the state
-// kernel derive their factors from this one scan, so they agree bit for bit.
-__device__ __forceinline__ float chunk_scan(const GdnTc& p, int64_t r0, int n, int h, int lane, float (&b)[2],
-                                            float (&g)[2]) {
-    float l[2];
+// beta (0 past n) and log alpha (0 past n), loaded from global memory
+// (through the row index when given).
+__device__ __forceinline__ void chunk_gates_load(const GdnTc& p, int64_t r0, int n, int h, int lane, float (&b)[2],
+                                                 float (&l)[2]) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int s = 2 * lane + e;
@@ -144,6 +147,12 @@ __device__ __forceinline__ float chunk_scan(const GdnTc& p, int64_t r0, int n, i
             }
         }
     }
+}
+
+// gamma, the running sum of log alpha from the chunk start, of the loaded
+// gates; returns gamma of the last valid row.  Both the prep and the state
+// kernel derive their factors from this one scan, so they agree bit for bit.
+__device__ __forceinline__ float chunk_gates_scan(const float (&l)[2], int n, int lane, float (&g)[2]) {
     const float pair = l[0] + l[1];
     float incl = pair;
 #pragma unroll
@@ -157,8 +166,11 @@ __device__ __forceinline__ float chunk_scan(const GdnTc& p, int64_t r0, int n, i
     return __shfl_sync(0xffffffffu, (last & 1) ? g[1] : g[0], last >> 1);
 }
 
-__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
-    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+__device__ __forceinline__ float chunk_scan(const GdnTc& p, int64_t r0, int n, int h, int lane, float (&b)[2],
+                                            float (&g)[2]) {
+    float l[2];
+    chunk_gates_load(p, r0, n, h, lane, b, l);
+    return chunk_gates_scan(l, n, lane, g);
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* v) {
@@ -197,87 +209,48 @@ __device__ __forceinline__ void gather_rows(const GdnTc& p, const bf16* base, in
 }
 
 // ----------------------------------------------------------------- prep --
-// The decay matrix D_rs = e^(gamma_r - gamma_s) = prod_{t=s+1..r} alpha_t
-// (s <= r, else 0) of one chunk into Dm ([64][LP] fp32), by running products
-// instead of one exponential per entry: thread (r, half) walks s downwards
-// over its half of the columns, multiplying by alpha_s; the lower half starts
-// from e^(gamma_r - gamma_31).  Underflow goes to 0 gracefully.
-__device__ __forceinline__ void prep_decay(int tid, const float* __restrict__ gam, const float* __restrict__ alpha,
-                                           float* __restrict__ Dm) {
-    const int r = tid & 63, half = tid >> 6;
-    const int s_hi = 32 * half + 31;
-    float d = (r > s_hi) ? __expf(gam[r] - gam[s_hi]) : 1.f;
-    float* row = Dm + r * LP;
+// The prep computes, per (chunk, head), everything the serial walk needs
+// that does not depend on the state, in the form the walk's two products
+// take it:
+//   Wk = Tb^T diag(e^(gamma_C - gamma)) K     (C x d_k): the state update is
+//        T <- 2^-e T + (rho' Y) Wk, with Y = V^T - Z~ and rho' the next
+//        running scale (U^T diag(dec) K = Y Tb^T diag(dec) K);
+//   Q' = P Tb                                  (C x C):  the output is
+//        X += Y Q'^T  (U^T P^T = Y Tb^T P^T).
+// Both leave as one contiguous bf16 image per (chunk, head): Wk rows j of
+// the d_k columns (64 chunk positions each, 128-byte swizzled, K-major for
+// the walk's state update), then Q' rows r (the same format).
+
+// fp32 64 x 64 work tile in two 32-row halves of 32 x 64 floats (8 KB each,
+// no padding), the column index XOR-ed with the row: a warp walking one
+// column over 32 rows, or one row over 32 columns, touches 32 banks.
+struct Tile {
+    float* lo;
+    float* hi;
+    __device__ __forceinline__ float& at(int r, int s) const {
+        return (r < 32 ? lo : hi)[(r & 31) * 64 + (s ^ (r & 31))];
+    }
+};
+
+constexpr int PREP_THREADS = 256;      // 8 warps per (chunk, head)
+
+// Writes NCH 16-byte chunks (8 fp32 values each, rounded to bf16) of row r,
+// starting at chunk c8_0, into a 128-byte-swizzled 64-column image.
+template <int NCH>
+__device__ __forceinline__ void image_chunks(unsigned char* __restrict__ img, int r, int c8_0, const float* v) {
 #pragma unroll
-    for (int j = 31; j >= 0; --j) {
-        const int s = 32 * half + j;
-        row[s] = s <= r ? d : 0.f;
-        if (s <= r) d *= alpha[s];
+    for (int k = 0; k < NCH; ++k) {
+        const float* w = v + 8 * k;
+        const int c8 = c8_0 + k;
+        *reinterpret_cast<uint4*>(img + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
     }
 }
 
-// Row r of L = beta_r D_rs k_r.k_s (s < r < n, else 0) from the G row held
-// in registers (ga: columns 0..31, gc: 32..63).
-__device__ __forceinline__ void prep_l_row(int r, int n, const float* __restrict__ drow, const float* __restrict__ bet,
-                                           const uint32_t (&ga)[32], const uint32_t (&gc)[32],
-                                           float* __restrict__ lrow) {
-    const float br = r < n ? bet[r] : 0.f;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int s = 32 * half + e;
-            const float G = __uint_as_float(half ? gc[e] : ga[e]);
-            lrow[s] = s < r ? br * drow[s] * G : 0.f;
-        }
-    }
-}
-
-// Row r of P = D_rs q_r.k_s (s <= r < n, else 0), bf16, written into the
-// 128-byte-swizzled 64 x 64 image.
-__device__ __forceinline__ void prep_p_row(int r, int n, const float* __restrict__ drow, const uint32_t (&ga)[32],
-                                           const uint32_t (&gc)[32], unsigned char* __restrict__ pimg) {
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-            float pv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int s = 32 * half + e + u;
-                const float G = __uint_as_float(half ? gc[e + u] : ga[e + u]);
-                pv[u] = (r < n) ? drow[s] * G : 0.f;       // drow is 0 past the diagonal
-            }
-            w[e / 2] = pack_bf16(pv[0], pv[1]);
-        }
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const int c8 = 4 * half + c4;
-            *reinterpret_cast<uint4*>(pimg + r * 128 + ((c8 ^ (r & 7)) << 4)) =
-                make_uint4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
-        }
-    }
-}
-
-// Row r, columns [32 half, 32 half + 32) of Tb = T diag(beta) (lower triangle), bf16 image.
-__device__ __forceinline__ void prep_tb_row(int r, int half, const float* __restrict__ trow,
-                                            const float* __restrict__ bet, unsigned char* __restrict__ timg) {
-    float v[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const int s = 32 * half + e;
-        v[e] = s <= r ? trow[s] * bet[s] : 0.f;
-    }
-    uint32_t w[16];
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) w[e / 2] = pack_bf16(v[e], v[e + 1]);
-#pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) {
-        const int c8 = 4 * half + c4;
-        *reinterpret_cast<uint4*>(timg + r * 128 + ((c8 ^ (r & 7)) << 4)) =
-            make_uint4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
-    }
+// Writes 64 fp32 values of row r as bf16 into a 128-byte-swizzled 64 x 64
+// shared-memory image.
+__device__ __forceinline__ void image_row(unsigned char* __restrict__ img, int r, const float (&v)[64]) {
+    image_chunks<8>(img, r, 0, v);
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
@@ -286,13 +259,14 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
     return r;
 }
 
-// d (16 x 8, fp32) += A (16 x 8 at a, row pitch LP) * B (8 x 8 at b, row pitch
-// pb): one m16n8k8 tf32 tensor-core product with fp32 accumulation.
-__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const float* a, const float* b, int pb, int lane) {
+// d (16 x 8, fp32) += A (16 x 8) * B (8 x 8): one m16n8k8 tf32 tensor-core
+// product with fp32 accumulation; a(i, k) and b(k, j) fetch the operands.
+template <class FA, class FB>
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], FA a, FB b, int lane) {
     const int g = lane >> 2, c = lane & 3;
-    const uint32_t a0 = to_tf32(a[g * LP + c]), a1 = to_tf32(a[(g + 8) * LP + c]);
-    const uint32_t a2 = to_tf32(a[g * LP + c + 4]), a3 = to_tf32(a[(g + 8) * LP + c + 4]);
-    const uint32_t b0 = to_tf32(b[c * pb + g]), b1 = to_tf32(b[(c + 4) * pb + g]);
+    const uint32_t a0 = to_tf32(a(g, c)), a1 = to_tf32(a(g + 8, c));
+    const uint32_t a2 = to_tf32(a(g, c + 4)), a3 = to_tf32(a(g + 8, c + 4));
+    const uint32_t b0 = to_tf32(b(c, g)), b1 = to_tf32(b(c + 4, g));
     asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
                  "{%0,%1,%2,%3};"
                  : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -304,23 +278,26 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const float* a, c
 // blocks closer to the diagonal.  The 16 x 16 block products run on the
 // tensor cores (tf32 operands, fp32 accumulation; T is rounded to bf16 for
 // its use anyway): a task is one 8-column half of one block, spread over
-// the 4 warps.
+// the warps.
 template <int LEV>
-__device__ __forceinline__ void offdiag_level(const float* Lm, float* Tm, float* Mb, int tid) {
+__device__ __forceinline__ void offdiag_level(const Tile& Lm, const Tile& Tm, float* Mb, int tid) {
     constexpr int NB = 4 - LEV;
+    constexpr int NW = PREP_THREADS / 32;
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
     // M_q = sum_kb L[bi][bj+kb] T[bj+kb][bj]        (bi = LEV + q, bj = q)
-    for (int task = warp; task < 2 * NB; task += 4) {
+    for (int task = warp; task < 2 * NB; task += NW) {
         const int q = task >> 1, nh = task & 1;
         const int bi = LEV + q, bj = q;
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kb = 0; kb < LEV; ++kb)
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-                mma_tf32_16x8x8(d, Lm + (16 * bi) * LP + 16 * (bj + kb) + 8 * ks,
-                                Tm + (16 * (bj + kb) + 8 * ks) * LP + 16 * bj + 8 * nh, LP, lane);
+            for (int ks = 0; ks < 2; ++ks) {
+                const int k0 = 16 * (bj + kb) + 8 * ks;
+                mma_tf32_16x8x8(d, [&](int i, int k) { return Lm.at(16 * bi + i, k0 + k); },
+                                [&](int k, int j) { return Tm.at(k0 + k, 16 * bj + 8 * nh + j); }, lane);
+            }
         float* m = Mb + q * 256;
         m[g * 16 + 8 * nh + 2 * c] = d[0];
         m[g * 16 + 8 * nh + 2 * c + 1] = d[1];
@@ -329,56 +306,72 @@ __device__ __forceinline__ void offdiag_level(const float* Lm, float* Tm, float*
     }
     __syncthreads();
     // T[bi][bj] = -T[bi][bi] M_q
-    for (int task = warp; task < 2 * NB; task += 4) {
+    for (int task = warp; task < 2 * NB; task += NW) {
         const int q = task >> 1, nh = task & 1;
         const int bi = LEV + q, bj = q;
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-            mma_tf32_16x8x8(d, Tm + (16 * bi) * LP + 16 * bi + 8 * ks, Mb + q * 256 + (8 * ks) * 16 + 8 * nh, 16, lane);
-        float* t = Tm + (16 * bi) * LP + 16 * bj + 8 * nh;
-        t[g * LP + 2 * c] = -d[0];
-        t[g * LP + 2 * c + 1] = -d[1];
-        t[(g + 8) * LP + 2 * c] = -d[2];
-        t[(g + 8) * LP + 2 * c + 1] = -d[3];
+        for (int ks = 0; ks < 2; ++ks) {
+            const float* mq = Mb + q * 256 + (8 * ks) * 16 + 8 * nh;
+            mma_tf32_16x8x8(d, [&](int i, int k) { return Tm.at(16 * bi + i, 16 * bi + 8 * ks + k); },
+                            [&](int k, int j) { return mq[k * 16 + j]; }, lane);
+        }
+        const int r0 = 16 * bi, c0 = 16 * bj + 8 * nh;
+        Tm.at(r0 + g, c0 + 2 * c) = -d[0];
+        Tm.at(r0 + g, c0 + 2 * c + 1) = -d[1];
+        Tm.at(r0 + g + 8, c0 + 2 * c) = -d[2];
+        Tm.at(r0 + g + 8, c0 + 2 * c + 1) = -d[3];
     }
     __syncthreads();
 }
 
 template <int D>
 struct PrepLayout {
-    // per 64-column slab: K rows 0..63 | q rows 64..127 (16 KB); after the
-    // MMA has read them, the fp32 work tiles reuse the same bytes
+    static constexpr int SLABS = D / 64;
+    // per 64-column slab: K rows 0..63 | q rows 64..127 (16 KB)
     static constexpr int KQ = 0;
-    static constexpr int KQ_BYTES = (D / 64) * 16384;
-    static constexpr int TM = 0;                      // fp32 [64][LP] T (first the decay matrix D)
-    static constexpr int LM = TM + C * LP * 4;        // fp32 [64][LP] L
-    static constexpr int MB = LM + C * LP * 4;        // fp32 3 x [16][16] block products
-    static constexpr int WORK = MB + 3 * 256 * 4;
-    static constexpr int GBB = ((KQ_BYTES > WORK ? KQ_BYTES : WORK) + 15) & ~15;   // beta, gamma, alpha [64]
-    static constexpr int BARS = GBB + 3 * C * 4;      // land, mma
-    static constexpr int MISC = BARS + 16;
+    static constexpr int KQ_BYTES = SLABS * 16384;
+    // the four 8 KB halves of the fp32 tiles T (first the decay matrix) and
+    // L: in the q halves of the slabs once G has read them (the K halves stay
+    // for the Wk product), the rest after the slabs
+    static constexpr int EXTRA = SLABS >= 4 ? 0 : (4 - SLABS) * 8192;
+    static constexpr int PI = KQ_BYTES + EXTRA;               // P image (A of Q'; the next 8 KB pad it to 128 rows)
+    static constexpr int TDI = PI + IMG;                      // diag(e^(gamma_C - gamma)) Tb image (B of Wk)
+    static constexpr int TBI = TDI + IMG;                     // Tb image (B of Q')
+    static constexpr int MB = TBI + IMG;                      // fp32 3 x [16][16] block products
+    static constexpr int GBB = MB + 3 * 256 * 4;              // beta, gamma log2(e) [64]
+    static constexpr int BARS = GBB + 3 * C * 4;              // land, G done, Wk/Q' done
+    static constexpr int MISC = BARS + 32;
     static constexpr size_t BYTES = 1024 + MISC + 16;
+    static constexpr int OUT = D * 128 + IMG;                 // output image bytes, staged at KQ
+    static constexpr uint32_t TMEM_COLS = D == 256 ? 256 : 128;   // G (then Q') | Wk^T halves
+    static_assert(OUT <= KQ_BYTES + EXTRA, "output staging fits the K/q bytes");
+    static __device__ __forceinline__ int tile_half(int w) {
+        return w < SLABS ? KQ + w * 16384 + 8192 : KQ_BYTES + (w - SLABS) * 8192;
+    }
 };
 
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(PREP_THREADS)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, GdnTc p) {
     using Lay = PrepLayout<D>;
     constexpr int SLABS = D / 64;
+    constexpr float LOG2E_ = 1.4426950408889634f;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = align1024(smem_raw);
-    float* Tm = reinterpret_cast<float*>(sm + Lay::TM);
-    float* Lm = reinterpret_cast<float*>(sm + Lay::LM);
+    unsigned char* sm = align1024_shared(smem_raw);
+    const Tile Tm{reinterpret_cast<float*>(sm + Lay::tile_half(0)), reinterpret_cast<float*>(sm + Lay::tile_half(1))};
+    const Tile Lm{reinterpret_cast<float*>(sm + Lay::tile_half(2)), reinterpret_cast<float*>(sm + Lay::tile_half(3))};
     float* Mb = reinterpret_cast<float*>(sm + Lay::MB);
     float* gbeta = reinterpret_cast<float*>(sm + Lay::GBB);
-    float* ggam = gbeta + C;
-    float* galpha = ggam + C;
+    float* g2 = gbeta + C;                                // gamma * log2(e)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::BARS);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lay::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-    const uint32_t land = smem_u32(bars), mma_bar = smem_u32(bars + 1);
+    const uint32_t land = smem_u32(bars), mma_bar = smem_u32(bars + 1), mma2_bar = smem_u32(bars + 2);
     const uint32_t kq = smem_u32(sm + Lay::KQ);
+    unsigned char* pimg = sm + Lay::PI;
+    unsigned char* tdimg = sm + Lay::TDI;
+    unsigned char* tbimg = sm + Lay::TBI;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x, h = blockIdx.y;
@@ -386,13 +379,19 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int4 info = p.chunk_info[g];
     const int64_t r0 = info.y;
     const int n = info.z;
+    // TMEM lane quarter of this warp and the 32-column half of a 64-column
+    // accumulator it reads (warps w and w + 4 share the lanes)
+    const int quarter = warp & 3, colh = warp >> 2;
+    const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+    const int rho = 32 * quarter + lane;                  // this thread's TMEM lane
 
     // Everything the chunk reads is requested at once: K (and contiguous q)
-    // by TMA, indexed q rows by warps 1-3, the gates by warp 0.  Rows past n
-    // hold other finite data and are masked below.
+    // by TMA, indexed q rows by warps 2-7, the gates by warp 0.  Rows past n
+    // hold other data or zeros and are zeroed below.
     if (tid == 0) {
         mbar_init(land, 1);
         mbar_init(mma_bar, 1);
+        mbar_init(mma2_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
         mbar_arrive_expect_tx(land, SLABS * 8192 * (p.qidx ? 1 : 2));
@@ -403,20 +402,16 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tslot), 64);
+        tmem_alloc(smem_u32(tslot), Lay::TMEM_COLS);
         tmem_relinquish();
     }
     if (warp == 0) {
         float b[2], gg[2];
         chunk_scan(p, r0, n, h, lane, b, gg);
         gbeta[2 * lane] = b[0]; gbeta[2 * lane + 1] = b[1];
-        ggam[2 * lane] = gg[0]; ggam[2 * lane + 1] = gg[1];
-        // alpha_s = e^(gamma_s - gamma_{s-1}) (rows past n: gamma is flat there, alpha = 1)
-        const float gprev = __shfl_up_sync(0xffffffffu, gg[1], 1);
-        galpha[2 * lane] = lane ? __expf(gg[0] - gprev) : 1.f;
-        galpha[2 * lane + 1] = __expf(gg[1] - gg[0]);
-    } else if (p.qidx) {
-        gather_rows<D>(p, p.q, r0, n, h, kq + 8192, 16384, tid - 32, 96);
+        g2[2 * lane] = gg[0] * LOG2E_; g2[2 * lane + 1] = gg[1] * LOG2E_;
+    } else if (p.qidx && warp >= 2) {
+        gather_rows<D>(p, p.q, r0, n, h, kq + 8192, 16384, tid - 64, PREP_THREADS - 64);
         cp_async_commit();
         cp_async_wait<0>();
         fence_proxy_async_smem();
@@ -431,6 +426,17 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     __syncthreads();
     bool ok = *abort_flag == 0;                           // uniform after the barrier
     if (!ok) mbar_wait_drain(land, 0);                    // copies in flight land before we leave
+    if (ok && n < C) {
+        // rows past n belong to other segments (or were never written): zero
+        // them, so that no product below can meet a non-finite value there
+        for (int idx = tid; idx < (C - n) * 8 * SLABS * 2; idx += PREP_THREADS) {
+            const int row = n + idx / (16 * SLABS), rest = idx % (16 * SLABS);
+            const uint32_t dst = kq + (rest >> 4) * 16384 + ((rest >> 3) & 1) * 8192 + row * 128 + (rest & 7) * 16;
+            asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0u) : "memory");
+        }
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
     if (ok && tid == 0) {
         tc_fence_after();
         constexpr uint32_t ID = idesc_bf16_f32(128, 64);
@@ -444,33 +450,44 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         umma_commit(mma_bar);
     }
     if (ok) {
-        if (!mbar_wait(mma_bar, 0, abort_flag, p.err, 11)) mbar_wait_drain(mma_bar, 0);   // K/q bytes free again
+        if (!mbar_wait(mma_bar, 0, abort_flag, p.err, 11)) mbar_wait_drain(mma_bar, 0);   // q bytes free again
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (*abort_flag) {
-        if (warp == 1) tmem_dealloc(tmem, 64);
+        if (warp == 1) tmem_dealloc(tmem, Lay::TMEM_COLS);
         return;
     }
-    uint32_t ga[32], gc[32];
-    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-    tmem_ld_x32(taddr, ga);
-    tmem_ld_x32(taddr + 32, gc);
-    tmem_ld_wait();
-
-    unsigned char* img = p.img + ((size_t)g * p.H + h) * 2 * IMG;
-    const int r = tid & 63;
-    prep_decay(tid, ggam, galpha, Tm);                    // D in T's bytes (T comes later)
-    __syncthreads();
-    if (tid < 64) prep_l_row(r, n, Tm + r * LP, gbeta, ga, gc, Lm + r * LP);
-    else prep_p_row(r, n, Tm + r * LP, ga, gc, img + IMG);
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 64);
+    // L = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r < n) into the L tile, and
+    // P = e^(gamma_r - gamma_s) q_r.k_s (s <= r < n) into the P image: TMEM lane
+    // rho is G row rho (K rows 0..63, then q rows), 32 columns per thread
+    {
+        uint32_t gv[32];
+        tmem_ld_x32(tmem + lane_base + 32 * colh, gv);
+        tmem_ld_wait();
+        const int r = rho & 63;
+        const float g2r = g2[r];
+        float v[32];
+        if (rho < 64) {
+            const float br = gbeta[r];                    // 0 past n
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int s = 32 * colh + e;
+                v[e] = s < r ? br * exp2f(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) Lm.at(r, 32 * colh + e) = v[e];
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int s = 32 * colh + e;
+                v[e] = (s <= r && r < n) ? exp2f(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
+            }
+            image_chunks<4>(pimg, r, 4 * colh, v);
+        }
     }
+    __syncthreads();
 
     // T = (I + L)^-1 in 16 x 16 blocks.  Diagonal blocks: forward substitution,
     // one column per thread.
@@ -482,15 +499,15 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
         for (int rl = 1; rl < 16; ++rl) {
             float a0 = 0.f, a1 = 0.f;
-            const float* Lr = Lm + (base + rl) * LP + base;
 #pragma unroll
             for (int sl = 0; sl < rl; ++sl) {
-                if (sl & 1) a1 = fmaf(Lr[sl], t[sl], a1); else a0 = fmaf(Lr[sl], t[sl], a0);
+                const float l = Lm.at(base + rl, base + sl);
+                if (sl & 1) a1 = fmaf(l, t[sl], a1); else a0 = fmaf(l, t[sl], a0);
             }
             if (rl > cc) t[rl] = -(a0 + a1);
         }
 #pragma unroll
-        for (int rl = 0; rl < 16; ++rl) Tm[(base + rl) * LP + base + cc] = t[rl];
+        for (int rl = 0; rl < 16; ++rl) Tm.at(base + rl, base + cc) = t[rl];
     }
     __syncthreads();
     // Off-diagonal blocks by distance from the diagonal:
@@ -498,15 +515,99 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     offdiag_level<1>(Lm, Tm, Mb, tid);
     offdiag_level<2>(Lm, Tm, Mb, tid);
     offdiag_level<3>(Lm, Tm, Mb, tid);
-    // Tb = T diag(beta): lower triangle (s <= r); beta is zero past n
-    prep_tb_row(r, tid >> 6, Tm + r * LP, gbeta, img);
+    // Tb = T diag(beta) and diag(e^(gamma_C - gamma)) Tb: row r, 16 columns per
+    // thread (rows past n are zero, beta being 0 there)
+    {
+        const int r = tid & 63, q4 = tid >> 6;
+        const float dec = exp2f(g2[n - 1] - g2[r]);
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int s = 16 * q4 + e;
+            v[e] = s <= r ? Tm.at(r, s) * gbeta[s] : 0.f;
+        }
+        image_chunks<2>(tbimg, r, 2 * q4, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] *= dec;
+        image_chunks<2>(tdimg, r, 2 * q4, v);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        tc_fence_after();
+        // Wk^T = K^T TD: A = K^T (MN-major view of the K slabs), B = TD (MN-major),
+        // D[j, t] over s; one M = 128 product per 128 columns of d_k
+        constexpr uint32_t IDW = idesc_bf16_f32(128, 64, 1, 1);
+#pragma unroll
+        for (int half = 0; half < SLABS / 2; ++half)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(tmem + 64 + 64 * half, desc_mnmajor_sw128(kq + 2 * half * 16384 + kk * 2048, 16384),
+                         desc_mnmajor_sw128(smem_u32(tdimg) + kk * 2048, 8192), IDW, kk != 0);
+        // Q' = P Tb: A = P (K-major; rows 64..127 read the next image and are
+        // discarded), B = Tb (MN-major); over G's columns, read out already
+        constexpr uint32_t IDQ = idesc_bf16_f32(128, 64, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            umma_f16(tmem, desc_kmajor_sw128(smem_u32(pimg) + kk * 32),
+                     desc_mnmajor_sw128(smem_u32(tbimg) + kk * 2048, 8192), IDQ, kk != 0);
+        umma_commit(mma2_bar);
+    }
+    if (!mbar_wait(mma2_bar, 0, abort_flag, p.err, 12)) mbar_wait_drain(mma2_bar, 0);
+    tc_fence_after();
+    __syncthreads();
+    if (*abort_flag) {
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem, Lay::TMEM_COLS);
+        }
+        return;
+    }
+    // read out into the output image, staged over the K/q bytes (every
+    // product that read them is done): Wk rows j, then Q' rows r; 32 columns
+    // (4 chunks) of one row per thread and accumulator
+    unsigned char* stage = sm + Lay::KQ;
+#pragma unroll
+    for (int half = 0; half < SLABS / 2; ++half) {
+        uint32_t w[32];
+        tmem_ld_x32(tmem + lane_base + 64 + 64 * half + 32 * colh, w);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(w[e]);
+        image_chunks<4>(stage, 128 * half + rho, 4 * colh, v);
+    }
+    if (quarter < 2) {
+        uint32_t w[32];
+        tmem_ld_x32(tmem + lane_base + 32 * colh, w);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(w[e]);
+        image_chunks<4>(stage + D * 128, rho, 4 * colh, v);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Lay::TMEM_COLS);
+    }
+    if (tid == 0) {
+        unsigned char* img = p.img + ((size_t)g * p.H + h) * (size_t)Lay::OUT;
+        bulk_store(img, smem_u32(stage), Lay::OUT);
+        bulk_commit();
+        bulk_wait_read0();                                // the shared source stays until it is read
+    }
 }
 
 // ---------------------------------------------------------------- state --
 enum Bar {
-    GB_FULL = 0, GB_FREE = 2, K_LAND = 4, K_FULL = 6, Q_FULL = 8, KQ_FREE = 10,
-    V_LAND = 12, V_FULL, V_FREE, T_FULL, T_FREE, P_FULL, P_FREE,
-    SBF_LO, SBF_HI, Z_FULL, U_FULL, S_FULL, O_FULL, XO_FREE, DONE,
+    GB_FULL = 0, GB_FREE = 2, K_FULL = 4, Q_FULL = 6, KQ_FREE = 8,
+    W_FULL = 10, W_FREE, V_FULL, V_FREE, SBF_LO, SBF_HI, Z_FULL, S_FULL, O_FULL, XO_FREE, DONE,
     DRAIN0, NBARS = DRAIN0 + 8          // one per math warp (NMATH)
 };
 
@@ -521,24 +622,22 @@ constexpr float LOG2E = 1.4426950408889634f;
 // Gate record of one chunk.  TMEM holds T = rho S with rho = 2^lr a running
 // scalar kept in [2^-1/2, 2^1/2]: the chunk decay a = e^gamma_last is applied
 // as the MMA's power-of-two accumulator scale 2^-e plus a change of rho.
-constexpr int G_EGR = 0;              // e^gamma_s / rho_c                     (0 past n)
-constexpr int G_DEC = C;              // rho_{c+1} e^(gamma_last - gamma_s)    (0 past n)
-constexpr int G_N = 2 * C;            // n (int bits)
-constexpr int G_SCL = 2 * C + 1;      // e (int bits): T <- 2^-e T + ...; -1: the old T is dropped (a < 2^-15.5)
-constexpr int G_LR = 2 * C + 2;       // lr_{c+1}
+constexpr int G_EGR = 0;              // e^gamma_s / rho_c   (0 past n)
+constexpr int G_N = C;                // n (int bits)
+constexpr int G_SCL = C + 1;          // e (int bits): T <- 2^-e T + ...; -1: the old T is dropped (a < 2^-15.5)
+constexpr int G_LR = C + 2;           // lr_{c+1}
 
 template <int D>
 struct StateLayout {
     static constexpr int SLABS = D / 64;
     // [K; q~] of a chunk: per 64-column slab, the 64 key rows then the 64
-    // scaled query rows (8 KB each), so that one N = 128 MMA computes
-    // Z = T K^T and X = T q~^T together
+    // scaled query rows (8 KB each)
     static constexpr int KQSZ = SLABS * 16384;
     static constexpr int KQ0 = 0;                             // 2 x [K; q~]
     static constexpr int VB = KQ0 + 2 * KQSZ;                 // [64 x 128] bf16: two 64-column slabs
-    static constexpr int TB = VB + 2 * 8192;                  // Tb image
-    static constexpr int PB = TB + IMG;                       // P image
-    static constexpr int STG = PB + IMG;                      // 8 x [32 rows x 32 d_v] bf16: per-warp output staging
+    static constexpr int IMGB = D * 128 + IMG;                // one prep image: Wk (d_k rows x 64), then Q'
+    static constexpr int WB = VB + 2 * 8192;                  // prep image
+    static constexpr int STG = WB + IMGB;                     // 8 x [32 rows x 32 d_v] bf16: per-warp output staging
     static constexpr int GBB = STG + 16384;                   // 2 gate records
     static constexpr int BARS = GBB + 2 * GB * 4;
     static constexpr int MISC = BARS + NBARS * 8;
@@ -553,6 +652,10 @@ __device__ __forceinline__ bool last_arrival(uint32_t counter) {
     return old % NMATH == NMATH - 1;
 }
 
+// TMEM column of K-step kk (16 chunk positions) of Y (off = 0) or rho' Y
+// (off = 16): math warp half hf keeps both inside its own 32 Z columns.
+__device__ __forceinline__ uint32_t y_col(int kk, int off) { return 32 * (kk >> 1) + 8 * (kk & 1) + off; }
+
 template <int D>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -560,30 +663,25 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     using Lay = StateLayout<D>;
     constexpr int SLABS = D / 64, NDV = D / DVT, HALF = D / 2;
     // TMEM columns: T = rho S (fp32), its bf16 copy (the A operand of Z and
-    // X), Z then U, X then X + O (Z and X adjacent: one N = 128 accumulator)
+    // X), Z (then Y and rho' Y, bf16, each math warp over the Z columns it
+    // has read), X (then X + O)
     constexpr uint32_t T_S = 0, T_SB = D, T_ZU = D + D / 2, T_XO = T_ZU + 64;
-    // bf16 A operands of the U, state-update and output products, [128 x 64]
-    // each (32 columns): inside the state copy's columns for d = 256 (free
-    // between the Z | X product and the read-back; the read-back's first
-    // half does not touch them), after X otherwise
-    constexpr uint32_t T_Y = D == 256 ? T_SB : T_XO + 64;
-    constexpr uint32_t T_US = T_Y + 64, T_UO = T_Y + 96;
     constexpr uint32_t TMEM_COLS = 512;
-    static_assert(T_XO + 64 <= TMEM_COLS && T_UO + 32 <= TMEM_COLS, "TMEM budget");
-    static_assert(D != 256 || T_US >= T_SB + D / 4, "operands clear of the read-back's first half");
+    constexpr int IMGB = Lay::IMGB;
+    static_assert(T_XO + 64 <= TMEM_COLS, "TMEM budget");
     static_assert(Lay::BYTES <= 232448, "shared memory budget");
 
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = align1024(smem_raw);
+    unsigned char* sm = align1024_shared(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::BARS);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lay::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-    // arrival counters of the math warps' hand-offs: the last warp to finish
-    // Y (resp. U) issues the U (resp. state-update and output) MMAs itself
-    const uint32_t cnt_y = smem_u32(tslot + 2), cnt_u = smem_u32(tslot + 3);
+    // arrival counter of the math warps' hand-off: the last warp to finish Y
+    // issues the output and state-update MMAs itself
+    const uint32_t cnt_y = smem_u32(tslot + 2);
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const uint32_t kq0 = smem_u32(sm + Lay::KQ0), vb = smem_u32(sm + Lay::VB);
-    const uint32_t timg = smem_u32(sm + Lay::TB), pimg = smem_u32(sm + Lay::PB), stg0 = smem_u32(sm + Lay::STG);
+    const uint32_t wimg = smem_u32(sm + Lay::WB), pimg = wimg + D * 128, stg0 = smem_u32(sm + Lay::STG);
     float* gbuf = reinterpret_cast<float*>(sm + Lay::GBB);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -605,7 +703,6 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), counts[i]);
         *abort_flag = 0;
         tslot[2] = 0;
-        tslot[3] = 0;
         fence_barrier_init();
     }
     if (warp == W_MMA) {
@@ -626,7 +723,6 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const uint32_t lb = (uint32_t)(32 * qd) << 16;
         const int sh = 32 * hf;
         const size_t hoff = (((size_t)seg * p.H + h) * D + dv0 + i) * D;
-        bool ok = true;
         // initial state: rho = 1, T = h0 (or zeros) and its bf16 copy
         for (int blk = 0; blk < HALF / 64; ++blk) {
             const int col = hf * HALF + 64 * blk;
@@ -675,14 +771,14 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         // this thread's element of V^T: V[s][i] sits in slab i / 64, 16-byte chunk (i % 64) / 8 of row s
         const uint32_t v_slab = vb + (uint32_t)(i >> 6) * 8192 + (uint32_t)(i & 7) * 2;
         const uint32_t v_chunk = (uint32_t)((i & 63) >> 3);
-        for (int c = 0; c < nc && ok; ++c) {
+        for (int c = 0; c < nc; ++c) {
             const int b = c & 1;
             const float* gb = gbuf + b * GB;
             const uint32_t ph = c & 1;
             if (!mbar_wait(bar(GB_FULL + b), (c >> 1) & 1, abort_flag, p.err, 21)) break;
             const int n = __float_as_int(gb[G_N]);
             const int64_t r0 = rs0 + (int64_t)c * C;
-            // ---- Y = V^T - Z~,  Z~ = (T K^T) diag(e^gamma / rho)
+            // ---- Y = V^T - Z~,  Z~ = (T K^T) diag(e^gamma / rho), and rho' Y
             if (!mbar_wait(bar(V_FULL), ph, abort_flag, p.err, 22)) break;
             uint32_t vv[16];                          // V[s][i] for the 32 positions, bf16 pairs
 #pragma unroll
@@ -705,84 +801,52 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 float eg[32];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_EGR + sh + e), eg + e);
+                const float rho1 = exp2f(gb[G_LR]);
                 tmem_ld_wait();
-                uint32_t pk[16];
+                uint32_t py[16], pr[16];
+                // positions past n hold other rows' keys and values: Y is 0 there
+                // (a select, so that nothing read there can reach the products)
 #pragma unroll
-                for (int e = 0; e < 32; e += 2)
-                    pk[e / 2] = pack_bf16(fmaf(-__uint_as_float(z[e]), eg[e], __uint_as_float(vv[e / 2] << 16)),
-                                          fmaf(-__uint_as_float(z[e + 1]), eg[e + 1], __uint_as_float(vv[e / 2] & 0xFFFF0000u)));
-                tmem_st_x16(tmem + lb + T_Y + 16 * hf, pk);
+                for (int e = 0; e < 32; e += 2) {
+                    const float y0 = sh + e < n
+                        ? fmaf(-__uint_as_float(z[e]), eg[e], __uint_as_float(vv[e / 2] << 16)) : 0.f;
+                    const float y1 = sh + e + 1 < n
+                        ? fmaf(-__uint_as_float(z[e + 1]), eg[e + 1], __uint_as_float(vv[e / 2] & 0xFFFF0000u)) : 0.f;
+                    py[e / 2] = pack_bf16(y0, y1);
+                    pr[e / 2] = pack_bf16(rho1 * y0, rho1 * y1);
+                }
+                // over this warp's own Z columns, read above
+                tmem_st_x16(tmem + lb + T_ZU + sh, py);
+                tmem_st_x16(tmem + lb + T_ZU + sh + 16, pr);
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0 && last_arrival(cnt_y)) {
-                // U^T = Y Tb^T, over Z (which every math warp has read)
-                if (mbar_wait(bar(T_FULL), ph, abort_flag, p.err, 43)) {
-                    tc_fence_after();
-                    constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tmem + T_ZU, tmem + T_Y + 8 * kk, desc_kmajor_sw128(timg + kk * 32), ID64, kk != 0);
-                    umma_commit(bar(U_FULL));
-                    umma_commit(bar(T_FREE));
-                    issued = true;
-                }
-            }
-            // ---- U^T (output term) and U^T diag(G_DEC) (state term)
-            if (!mbar_wait(bar(U_FULL), ph, abort_flag, p.err, 24)) break;
-            tc_fence_after();
-            {
-                uint32_t u[32];
-                tmem_ld_x32(tmem + lb + T_ZU + sh, u);
-                float dc[32];
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) ld_shared_v4(smem_u32(gb + G_DEC + sh + e), dc + e);
-                tmem_ld_wait();
-                uint32_t pu[16], pd[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int s = sh + e;
-                    const float a0 = s < n ? __uint_as_float(u[e]) : 0.f;
-                    const float a1 = s + 1 < n ? __uint_as_float(u[e + 1]) : 0.f;
-                    pu[e / 2] = pack_bf16(a0, a1);
-                    pd[e / 2] = pack_bf16(a0 * dc[e], a1 * dc[e + 1]);
-                }
-                tmem_st_x16(tmem + lb + T_UO + 16 * hf, pu);
-                tmem_st_x16(tmem + lb + T_US + 16 * hf, pd);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && last_arrival(cnt_u)) {
-                tc_fence_after();
-                // X += U^T P^T first (small; frees X early), then T = 2^-e T + (U^T diag(G_DEC)) K.
-                // One thread commits both, the output first: S_FULL implies O_FULL.
-                const uint32_t kq = kq0 + b * Lay::KQSZ;
+                // T = 2^-e T + (rho' Y) Wk first (the serial chain waits for it), then
+                // X += Y Q'^T; one thread issues and commits both
                 constexpr uint32_t ID64 = idesc_bf16_f32(128, 64);
-                constexpr uint32_t IDS = idesc_bf16_f32(128, D, 0, 1);   // B = K (MN-major)
-                if (mbar_wait(bar(P_FULL), ph, abort_flag, p.err, 47)) {
+                constexpr uint32_t IDS = idesc_bf16_f32(128, D);     // B = Wk, K-major, N = d_k
+                if (mbar_wait(bar(W_FULL), ph, abort_flag, p.err, 48)) {
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tmem + T_XO, tmem + T_UO + 8 * kk, desc_kmajor_sw128(pimg + kk * 32), ID64, 1);
-                    umma_commit(bar(O_FULL));
-                    umma_commit(bar(P_FREE));
                     const int e = __float_as_int(gb[G_SCL]);
-                    umma_f16_ts_scaled(tmem + T_S, tmem + T_US, desc_mnmajor_sw128(kq, 16384), IDS, e >= 0 ? 1u : 0u,
-                                       e >= 0 ? e : 0);
+                    umma_f16_ts_scaled(tmem + T_S, tmem + T_ZU + y_col(0, 16), desc_kmajor_sw128(wimg), IDS,
+                                       e >= 0 ? 1u : 0u, e >= 0 ? e : 0);
 #pragma unroll
                     for (int kk = 1; kk < 4; ++kk)
-                        umma_f16_ts(tmem + T_S, tmem + T_US + 8 * kk, desc_mnmajor_sw128(kq + kk * 2048, 16384), IDS, 1);
+                        umma_f16_ts(tmem + T_S, tmem + T_ZU + y_col(kk, 16), desc_kmajor_sw128(wimg + kk * 32), IDS, 1);
                     umma_commit(bar(S_FULL));
-                    umma_commit(bar(KQ_FREE + b));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ts(tmem + T_XO, tmem + T_ZU + y_col(kk, 0), desc_kmajor_sw128(pimg + kk * 32), ID64, 1);
+                    umma_commit(bar(O_FULL));
+                    umma_commit(bar(W_FREE));
                     issued = true;
                 }
             }
-            // ---- the output read out of TMEM as soon as its product is done (the next
-            // chunk's Z | X product overwrites X), then after the state update the bf16
-            // copy of the new T in two d_k halves (the next product starts on the first),
-            // then the output stored
+            // ---- after the state update the bf16 copy of the new T in two d_k halves
+            // (the next Z | X product starts on the first); between them the output,
+            // read out of TMEM (the next product overwrites X); then the output stored
             const bool last = c + 1 == nc;
             auto readback_half = [&](int part) {
                 for (int blk = 0; blk < HALF / 64; ++blk) {
@@ -799,6 +863,9 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(part ? SBF_HI : SBF_LO));
             };
+            if (!mbar_wait(bar(S_FULL), ph, abort_flag, p.err, 25)) break;
+            tc_fence_after();
+            if (!last) readback_half(0);
             if (!mbar_wait(bar(O_FULL), ph, abort_flag, p.err, 26)) break;
             tc_fence_after();
             uint32_t xo[32];
@@ -807,10 +874,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(XO_FREE));
-            if (!mbar_wait(bar(S_FULL), ph, abort_flag, p.err, 25)) break;
-            tc_fence_after();
             if (!last) {
-                readback_half(0);
                 readback_half(1);
             } else if (p.h_final) {
                 // the final state S = T / rho
@@ -871,21 +935,37 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             }
         }
     } else if (warp == W_PROD) {
-        // ------------------------------------------ producer: gates + TMA
+        // ------------------------------------------ producer: gates + loads
+        // Waits only for buffers to be free, never for a copy to land (the
+        // consumers wait on the copies' transaction barriers): every load is
+        // issued as early as its buffer allows.  The gates of chunk c + 1 are
+        // loaded while chunk c's are scanned.
         bool ok = true;
-        int last_k[2] = {-1, -1}, last_v = -1, last_t = -1, last_p = -1;
+        int last_k[2] = {-1, -1}, last_w = -1, last_v = -1;
         float lr = 0.f;                               // log2 rho at the chunk start
+        float bt[2], la[2];
+        chunk_gates_load(p, rs0, (int)(rs1 - rs0 < C ? rs1 - rs0 : C), h, lane, bt, la);
         for (int c = 0; c < nc && ok; ++c) {
             const int b = c & 1;
             const uint32_t ph = c & 1, pb = (c >> 1) & 1;
             const int64_t r0 = rs0 + (int64_t)c * C;
             const int64_t rem = rs1 - r0;
             const int n = (int)(rem < C ? rem : C);
+            const unsigned char* img = p.img + ((size_t)(c_base + c) * p.H + h) * (size_t)IMGB;
+            // K tile of this chunk
+            const uint32_t kb = kq0 + b * Lay::KQSZ;
+            if (!mbar_wait(bar(KQ_FREE + b), pb ^ 1, abort_flag, p.err, 31)) { ok = false; break; }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(K_FULL + b), SLABS * 8192);
+#pragma unroll
+                for (int j = 0; j < SLABS; ++j) tma_load_2d(kb + j * 16384, &tm_k, bar(K_FULL + b), h * D + 64 * j, (int)r0);
+            }
+            last_k[b] = c;
             // gates
             if (!mbar_wait(bar(GB_FREE + b), pb ^ 1, abort_flag, p.err, 30)) { ok = false; break; }
             {
-                float bt[2], gg[2];
-                const float gl = chunk_scan(p, r0, n, h, lane, bt, gg);
+                float gg[2];
+                const float gl = chunk_gates_scan(la, n, lane, gg);
                 const float t = lr - gl * LOG2E;      // >= -1/2
                 int e = (int)floorf(t + 0.5f);
                 float lr1 = t - (float)e;
@@ -895,7 +975,6 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 for (int k = 0; k < 2; ++k) {
                     const int s = 2 * lane + k;
                     gb[G_EGR + s] = s < n ? exp2f(gg[k] * LOG2E - lr) : 0.f;
-                    gb[G_DEC + s] = s < n ? exp2f(lr1 + (gl - gg[k]) * LOG2E) : 0.f;
                 }
                 if (lane == 0) {
                     gb[G_N] = __int_as_float(n);
@@ -906,66 +985,32 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(GB_FULL + b));
-            // K and V tiles
-            const uint32_t kb = kq0 + b * Lay::KQSZ;
-            if (!mbar_wait(bar(KQ_FREE + b), pb ^ 1, abort_flag, p.err, 31)) { ok = false; break; }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(K_LAND + b), SLABS * 8192);
-#pragma unroll
-                for (int j = 0; j < SLABS; ++j) tma_load_2d(kb + j * 16384, &tm_k, bar(K_LAND + b), h * D + 64 * j, (int)r0);
+            if (c + 1 < nc) {
+                const int64_t rem1 = rs1 - (r0 + C);
+                chunk_gates_load(p, r0 + C, (int)(rem1 < C ? rem1 : C), h, lane, bt, la);
             }
-            last_k[b] = c;
+            // V tile (this CTA's d_v rows)
             if (!mbar_wait(bar(V_FREE), ph ^ 1, abort_flag, p.err, 32)) { ok = false; break; }
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(V_LAND), 16384);
-                tma_load_2d(vb, &tm_v, bar(V_LAND), h * D + dv0, (int)r0);
-                tma_load_2d(vb + 8192, &tm_v, bar(V_LAND), h * D + dv0 + 64, (int)r0);
+                mbar_arrive_expect_tx(bar(V_FULL), 16384);
+                tma_load_2d(vb, &tm_v, bar(V_FULL), h * D + dv0, (int)r0);
+                tma_load_2d(vb + 8192, &tm_v, bar(V_FULL), h * D + dv0 + 64, (int)r0);
             }
             last_v = c;
-            // zero the key / value rows past n (other segments' data) once they land
-            if (!mbar_wait(bar(K_LAND + b), pb, abort_flag, p.err, 34)) { ok = false; break; }
-            if (n < C) {
-                for (int idx = lane; idx < (C - n) * 8 * SLABS; idx += 32) {
-                    const int row = n + idx / (8 * SLABS), rest = idx % (8 * SLABS);
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(kb + (rest >> 3) * 16384 + row * 128 + (rest & 7) * 16),
-                                 "r"(0u) : "memory");
-                }
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(K_FULL + b));
-            if (!mbar_wait(bar(V_LAND), ph, abort_flag, p.err, 35)) { ok = false; break; }
-            if (n < C) {
-                for (int idx = lane; idx < (C - n) * 16; idx += 32) {
-                    const int row = n + idx / 16, rest = idx % 16;
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(vb + (rest >> 3) * 8192 + row * 128 + (rest & 7) * 16),
-                                 "r"(0u) : "memory");
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(V_FULL));
-            // Tb and P tiles of this chunk
-            const unsigned char* img = p.img + ((size_t)(c_base + c) * p.H + h) * 2 * IMG;
-            if (!mbar_wait(bar(T_FREE), ph ^ 1, abort_flag, p.err, 36)) { ok = false; break; }
+            // Wk and Q' images of this chunk
+            if (!mbar_wait(bar(W_FREE), ph ^ 1, abort_flag, p.err, 36)) { ok = false; break; }
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(T_FULL), IMG);
-                bulk_load(timg, img, IMG, bar(T_FULL));
+                mbar_arrive_expect_tx(bar(W_FULL), IMGB);
+                bulk_load(wimg, img, IMGB, bar(W_FULL));
             }
-            last_t = c;
-            if (!mbar_wait(bar(P_FREE), ph ^ 1, abort_flag, p.err, 37)) { ok = false; break; }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(P_FULL), IMG);
-                bulk_load(pimg, img + IMG, IMG, bar(P_FULL));
-            }
-            last_p = c;
+            last_w = c;
         }
         if (!ok && lane == 0) {
             // copies still in flight must land before the CTA exits
             for (int b = 0; b < 2; ++b)
-                if (last_k[b] >= 0) mbar_wait_drain(bar(K_LAND + b), (last_k[b] >> 1) & 1);
-            if (last_v >= 0) mbar_wait_drain(bar(V_LAND), last_v & 1);
-            if (last_t >= 0) mbar_wait_drain(bar(T_FULL), last_t & 1);
-            if (last_p >= 0) mbar_wait_drain(bar(P_FULL), last_p & 1);
+                if (last_k[b] >= 0) mbar_wait_drain(bar(K_FULL + b), (last_k[b] >> 1) & 1);
+            if (last_w >= 0) mbar_wait_drain(bar(W_FULL), last_w & 1);
+            if (last_v >= 0) mbar_wait_drain(bar(V_FULL), last_v & 1);
         }
     } else if (warp < W_MMA) {
         // ------------------- q~ warps: q rows (through the index when given),
@@ -1010,17 +1055,18 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         cp_async_wait<0>();
     } else if (lane == 0) {
         // ------------------------------------------------------ MMA issuer
+        // [Z | X] = T [K; q~]^T, one N = 128 product (per 64-column slab the
+        // key rows then the scaled query rows); A = the bf16 copy of T in TMEM:
+        // the first d_k half as soon as its copy is ready, then the second
         constexpr uint32_t ID128 = idesc_bf16_f32(128, 128);
         for (int c = 0; c < nc; ++c) {
             const int b = c & 1;
             const uint32_t ph = c & 1, pb = (c >> 1) & 1;
             const uint32_t kq = kq0 + b * Lay::KQSZ;
-            // [Z | X] = T [K; q~]^T, A = the bf16 copy of T in TMEM: the first
-            // d_k half as soon as its copy is ready, then the second
             if (!mbar_wait(bar(K_FULL + b), pb, abort_flag, p.err, 40)) break;
             if (!mbar_wait(bar(Q_FULL + b), pb, abort_flag, p.err, 41)) break;
-            if (!mbar_wait(bar(XO_FREE), ph ^ 1, abort_flag, p.err, 43)) break;
             if (!mbar_wait(bar(SBF_LO), ph, abort_flag, p.err, 42)) break;
+            if (!mbar_wait(bar(XO_FREE), ph ^ 1, abort_flag, p.err, 43)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
@@ -1033,6 +1079,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 umma_f16_ts(tmem + T_ZU, tmem + T_SB + 8 * kk, desc_kmajor_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
                             ID128, 1);
             umma_commit(bar(Z_FULL));
+            umma_commit(bar(KQ_FREE + b));
         }
         umma_commit(bar(DONE));
         mbar_wait_drain(bar(DONE), 0);
@@ -1066,7 +1113,7 @@ cudaError_t launch_d(const GdnTc& t, int64_t mchunks, int phase, cudaStream_t st
         ++launched;
         if (mchunks > 0) {
             dim3 pg((unsigned)mchunks, t.H);
-            gdn_prep_kernel<D><<<pg, 128, PrepLayout<D>::BYTES, st>>>(tm_k, tm_q, t);
+            gdn_prep_kernel<D><<<pg, PREP_THREADS, PrepLayout<D>::BYTES, st>>>(tm_k, tm_q, t);
             ++launched;
         }
     }
@@ -1092,9 +1139,8 @@ bool gdn_tc_supported(const GdnArgs& a, int dt) {
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t gdn_tc_ws_bytes(int64_t n_rows, int n_seg, int H, int d) {
-    (void)d;
     const size_t mc = (size_t)max_chunks(n_rows, n_seg);
-    return up256(((size_t)n_seg + 1) * 4) + up256(mc * sizeof(int4)) + mc * H * 2 * IMG;
+    return up256(((size_t)n_seg + 1) * 4) + up256(mc * sizeof(int4)) + mc * H * ((size_t)d * 128 + IMG);
 }
 
 cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st) {

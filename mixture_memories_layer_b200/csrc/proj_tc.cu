@@ -101,8 +101,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant__ CUtensorMap tm_kv,
                const __grid_constant__ OutMaps om, TcParams p) {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~static_cast<uintptr_t>(1023));
+    unsigned char* smem = align1024_shared(smem_raw);
     unsigned char* sA = smem;
     unsigned char* sB = smem + STAGES * A_BYTES;
     unsigned char* sOut = sB + STAGES * B_BYTES;                       // per epilogue warp staging piece

@@ -104,7 +104,7 @@ template <int NT, bool ROUTER>
 __global__ void __launch_bounds__(9 * 32, 1)
 skinny_kernel(const __grid_constant__ CUtensorMap tm_x, SkinnyArgs a, int NS) {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    unsigned char* sm = align1024_shared(smem_raw);
     const size_t stage_bytes = (size_t)TOK * a.D * 2;
     const size_t w_bytes = (size_t)NT * 8 * a.D * 2;
     unsigned char* wsm_p = sm + NS * stage_bytes;                                  // staged W

@@ -16,6 +16,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned address at or after p (the base of dynamic
+// shared memory), by pointer arithmetic on p itself: the result stays a
+// pointer into shared memory for the compiler, so the accesses derived from
+// it compile to shared-memory loads and stores rather than generic ones.
+__device__ __forceinline__ unsigned char* align1024_shared(unsigned char* p) {
+    return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
 // ------------------------------------------------------------- mbarriers --
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
@@ -115,6 +123,13 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Contiguous shared -> global copy of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completing as a bulk group (bulk_commit / bulk_wait*).
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
                  : "memory");
 }
 
