@@ -234,6 +234,15 @@ struct Tile {
 
 constexpr int PREP_THREADS = 256;      // 8 warps per (chunk, head)
 
+// 2^x by the hardware approximation (an error of a few units in the last
+// place of fp32; results below 2^-126 flush to 0): the prep's decay factors,
+// which are rounded to bf16 afterwards.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Writes NCH 16-byte chunks (8 fp32 values each, rounded to bf16) of row r,
 // starting at chunk c8_0, into a 128-byte-swizzled 64-column image.
 template <int NCH>
@@ -331,31 +340,34 @@ struct PrepLayout {
     // per 64-column slab: K rows 0..63 | q rows 64..127 (16 KB)
     static constexpr int KQ = 0;
     static constexpr int KQ_BYTES = SLABS * 16384;
-    // the four 8 KB halves of the fp32 tiles T (first the decay matrix) and
-    // L: in the q halves of the slabs once G has read them (the K halves stay
-    // for the Wk product), the rest after the slabs
+    // the four 8 KB halves of the fp32 tiles T and L: in the q halves of the
+    // slabs once G has read them (the K halves stay for the Wk product), the
+    // rest after the slabs.  After the solve the bf16 images take their
+    // place: Tb over L's first half, TD over L's second, P over T's first.
     static constexpr int EXTRA = SLABS >= 4 ? 0 : (4 - SLABS) * 8192;
-    static constexpr int PI = KQ_BYTES + EXTRA;               // P image (A of Q'; the next 8 KB pad it to 128 rows)
-    static constexpr int TDI = PI + IMG;                      // diag(e^(gamma_C - gamma)) Tb image (B of Wk)
-    static constexpr int TBI = TDI + IMG;                     // Tb image (B of Q')
-    static constexpr int MB = TBI + IMG;                      // fp32 3 x [16][16] block products
+    static constexpr int MB = KQ_BYTES + EXTRA;               // fp32 3 x [16][16] block products
     static constexpr int GBB = MB + 3 * 256 * 4;              // beta, gamma log2(e) [64]
-    static constexpr int BARS = GBB + 3 * C * 4;              // land, G done, Wk/Q' done
+    static constexpr int BARS = GBB + 2 * C * 4;              // land, G done, products done (x2)
     static constexpr int MISC = BARS + 32;
     static constexpr size_t BYTES = 1024 + MISC + 16;
-    static constexpr int OUT = D * 128 + IMG;                 // output image bytes, staged at KQ
-    static constexpr uint32_t TMEM_COLS = D == 256 ? 256 : 128;   // G (then Q') | Wk^T halves
-    static_assert(OUT <= KQ_BYTES + EXTRA, "output staging fits the K/q bytes");
+    static constexpr int OUT = D * 128 + IMG;                 // output image bytes: Wk rows, then Q'
+    // TMEM: G, then one 128-column-of-d_k half of Wk^T and Q' per round
+    static constexpr uint32_t TMEM_COLS = 128;
+    // output staging (every region dead by then): the round-1 Wk half and Q',
+    // then (d = 256) the second round's Wk half
+    static constexpr int ST_W1 = D == 256 ? 24576 : 0;
+    static constexpr int ST_Q = D == 256 ? 40960 : 16384;
+    static_assert(D == 256 || D == 128, "head dimension");
     static __device__ __forceinline__ int tile_half(int w) {
         return w < SLABS ? KQ + w * 16384 + 8192 : KQ_BYTES + (w - SLABS) * 8192;
     }
 };
 
 template <int D>
-__global__ void __launch_bounds__(PREP_THREADS)
+__global__ void __launch_bounds__(PREP_THREADS, 3)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, GdnTc p) {
     using Lay = PrepLayout<D>;
-    constexpr int SLABS = D / 64;
+    constexpr int SLABS = D / 64, HALVES = SLABS / 2;
     constexpr float LOG2E_ = 1.4426950408889634f;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024_shared(smem_raw);
@@ -367,11 +379,12 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::BARS);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lay::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-    const uint32_t land = smem_u32(bars), mma_bar = smem_u32(bars + 1), mma2_bar = smem_u32(bars + 2);
+    const uint32_t land = smem_u32(bars), mma_bar = smem_u32(bars + 1);
+    const uint32_t mma2_bar = smem_u32(bars + 2), mma3_bar = smem_u32(bars + 3);
     const uint32_t kq = smem_u32(sm + Lay::KQ);
-    unsigned char* pimg = sm + Lay::PI;
-    unsigned char* tdimg = sm + Lay::TDI;
-    unsigned char* tbimg = sm + Lay::TBI;
+    unsigned char* pimg = sm + Lay::tile_half(0);
+    unsigned char* tbimg = sm + Lay::tile_half(2);
+    unsigned char* tdimg = sm + Lay::tile_half(3);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.x, h = blockIdx.y;
@@ -392,6 +405,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(land, 1);
         mbar_init(mma_bar, 1);
         mbar_init(mma2_bar, 1);
+        mbar_init(mma3_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
         mbar_arrive_expect_tx(land, SLABS * 8192 * (p.qidx ? 1 : 2));
@@ -459,32 +473,18 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (warp == 1) tmem_dealloc(tmem, Lay::TMEM_COLS);
         return;
     }
-    // L = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r < n) into the L tile, and
-    // P = e^(gamma_r - gamma_s) q_r.k_s (s <= r < n) into the P image: TMEM lane
-    // rho is G row rho (K rows 0..63, then q rows), 32 columns per thread
-    {
+    // L = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r < n) into the L tile:
+    // TMEM lanes 0..63 are the K rows of G, 32 columns per thread
+    if (quarter < 2) {
         uint32_t gv[32];
         tmem_ld_x32(tmem + lane_base + 32 * colh, gv);
         tmem_ld_wait();
-        const int r = rho & 63;
-        const float g2r = g2[r];
-        float v[32];
-        if (rho < 64) {
-            const float br = gbeta[r];                    // 0 past n
+        const int r = rho;
+        const float g2r = g2[r], br = gbeta[r];           // beta is 0 past n
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int s = 32 * colh + e;
-                v[e] = s < r ? br * exp2f(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) Lm.at(r, 32 * colh + e) = v[e];
-        } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int s = 32 * colh + e;
-                v[e] = (s <= r && r < n) ? exp2f(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
-            }
-            image_chunks<4>(pimg, r, 4 * colh, v);
+        for (int e = 0; e < 32; ++e) {
+            const int s = 32 * colh + e;
+            Lm.at(r, s) = s < r ? br * ex2_approx(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
         }
     }
     __syncthreads();
@@ -515,11 +515,11 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     offdiag_level<1>(Lm, Tm, Mb, tid);
     offdiag_level<2>(Lm, Tm, Mb, tid);
     offdiag_level<3>(Lm, Tm, Mb, tid);
-    // Tb = T diag(beta) and diag(e^(gamma_C - gamma)) Tb: row r, 16 columns per
-    // thread (rows past n are zero, beta being 0 there)
+    // Tb = T diag(beta) and diag(e^(gamma_C - gamma)) Tb over L's bytes: row
+    // r, 16 columns per thread (rows past n are zero, beta being 0 there)
     {
         const int r = tid & 63, q4 = tid >> 6;
-        const float dec = exp2f(g2[n - 1] - g2[r]);
+        const float dec = ex2_approx(g2[n - 1] - g2[r]);
         float v[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -531,77 +531,123 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int e = 0; e < 16; ++e) v[e] *= dec;
         image_chunks<2>(tdimg, r, 2 * q4, v);
     }
+    // P = e^(gamma_r - gamma_s) q_r.k_s (s <= r < n) from TMEM lanes 64..127
+    // (the q rows of G), then over T's first half once T is read
+    uint32_t pk[16];
+    if (quarter >= 2) {
+        uint32_t gv[32];
+        tmem_ld_x32(tmem + lane_base + 32 * colh, gv);
+        tmem_ld_wait();
+        const int r = rho - 64;
+        const float g2r = g2[r];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const int s = 32 * colh + e;
+            const float p0 = (s <= r && r < n) ? ex2_approx(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
+            const float p1 = (s + 1 <= r && r < n) ? ex2_approx(g2r - g2[s + 1]) * __uint_as_float(gv[e + 1]) : 0.f;
+            pk[e / 2] = pack_bf16(p0, p1);
+        }
+    }
+    __syncthreads();
+    if (quarter >= 2) {
+        const int r = rho - 64;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int c8 = 4 * colh + k;
+            *reinterpret_cast<uint4*>(pimg + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-        tc_fence_after();
-        // Wk^T = K^T TD: A = K^T (MN-major view of the K slabs), B = TD (MN-major),
-        // D[j, t] over s; one M = 128 product per 128 columns of d_k
-        constexpr uint32_t IDW = idesc_bf16_f32(128, 64, 1, 1);
-#pragma unroll
-        for (int half = 0; half < SLABS / 2; ++half)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + 64 + 64 * half, desc_mnmajor_sw128(kq + 2 * half * 16384 + kk * 2048, 16384),
-                         desc_mnmajor_sw128(smem_u32(tdimg) + kk * 2048, 8192), IDW, kk != 0);
-        // Q' = P Tb: A = P (K-major; rows 64..127 read the next image and are
-        // discarded), B = Tb (MN-major); over G's columns, read out already
-        constexpr uint32_t IDQ = idesc_bf16_f32(128, 64, 0, 1);
+    // Products on the tensor cores, D[j, t] over s:
+    //   Wk^T = K^T TD: A = K^T (MN-major view of two K slabs), B = TD (MN-major)
+    //   Q'  = P Tb:   A = P (K-major; rows 64..127 read the next 8 KB and are
+    //                 discarded), B = Tb (MN-major)
+    constexpr uint32_t IDW = idesc_bf16_f32(128, 64, 1, 1);
+    constexpr uint32_t IDQ = idesc_bf16_f32(128, 64, 0, 1);
+    auto issue_wk = [&](int half) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            umma_f16(tmem, desc_kmajor_sw128(smem_u32(pimg) + kk * 32),
-                     desc_mnmajor_sw128(smem_u32(tbimg) + kk * 2048, 8192), IDQ, kk != 0);
-        umma_commit(mma2_bar);
-    }
-    if (!mbar_wait(mma2_bar, 0, abort_flag, p.err, 12)) mbar_wait_drain(mma2_bar, 0);
-    tc_fence_after();
-    __syncthreads();
-    if (*abort_flag) {
-        tc_fence_before();
-        __syncthreads();
-        if (warp == 1) {
-            tc_fence_after();
-            tmem_dealloc(tmem, Lay::TMEM_COLS);
-        }
-        return;
-    }
-    // read out into the output image, staged over the K/q bytes (every
-    // product that read them is done): Wk rows j, then Q' rows r; 32 columns
-    // (4 chunks) of one row per thread and accumulator
-    unsigned char* stage = sm + Lay::KQ;
-#pragma unroll
-    for (int half = 0; half < SLABS / 2; ++half) {
-        uint32_t w[32];
-        tmem_ld_x32(tmem + lane_base + 64 + 64 * half + 32 * colh, w);
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(w[e]);
-        image_chunks<4>(stage, 128 * half + rho, 4 * colh, v);
-    }
-    if (quarter < 2) {
+            umma_f16(tmem, desc_mnmajor_sw128(kq + 2 * half * 16384 + kk * 2048, 16384),
+                     desc_mnmajor_sw128(smem_u32(tdimg) + kk * 2048, 8192), IDW, kk != 0);
+    };
+    // one Wk^T half (TMEM lanes j, columns 0..63) into rows j of the staged image
+    auto read_wk = [&](int half, unsigned char* st) {
         uint32_t w[32];
         tmem_ld_x32(tmem + lane_base + 32 * colh, w);
         tmem_ld_wait();
         float v[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(w[e]);
-        image_chunks<4>(stage + D * 128, rho, 4 * colh, v);
+        image_chunks<4>(st, rho, 4 * colh, v);
+        (void)half;
+    };
+    // round 1: the last Wk half and Q'
+    if (tid == 0) {
+        tc_fence_after();
+        issue_wk(HALVES - 1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            umma_f16(tmem + 64, desc_kmajor_sw128(smem_u32(pimg) + kk * 32),
+                     desc_mnmajor_sw128(smem_u32(tbimg) + kk * 2048, 8192), IDQ, kk != 0);
+        umma_commit(mma2_bar);
     }
-    fence_proxy_async_smem();
+    if (!mbar_wait(mma2_bar, 0, abort_flag, p.err, 12)) mbar_wait_drain(mma2_bar, 0);
+    tc_fence_after();
+    __syncthreads();
+    bool fail = *abort_flag != 0;
+    unsigned char* img = p.img + ((size_t)g * p.H + h) * (size_t)Lay::OUT;
+    if (!fail) {
+        read_wk(HALVES - 1, sm + Lay::ST_W1);
+        if (quarter < 2) {
+            uint32_t w[32];
+            tmem_ld_x32(tmem + lane_base + 64 + 32 * colh, w);
+            tmem_ld_wait();
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(w[e]);
+            image_chunks<4>(sm + Lay::ST_Q, rho, 4 * colh, v);
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
+    if (!fail && tid == 0) {
+        if (HALVES == 2) {
+            bulk_store(img + 16384, smem_u32(sm + Lay::ST_W1), 16384);
+            bulk_store(img + D * 128, smem_u32(sm + Lay::ST_Q), IMG);
+            // round 2: the first Wk half, over the same TMEM columns (read out above)
+            tc_fence_after();
+            issue_wk(0);
+            umma_commit(mma3_bar);
+        } else {
+            bulk_store(img, smem_u32(sm + Lay::ST_W1), Lay::OUT);
+        }
+        bulk_commit();
+    }
+    if (HALVES == 2 && !fail) {
+        if (!mbar_wait(mma3_bar, 0, abort_flag, p.err, 13)) mbar_wait_drain(mma3_bar, 0);
+        tc_fence_after();
+        __syncthreads();
+        fail = *abort_flag != 0;
+        if (!fail) {
+            read_wk(0, sm + Lay::KQ);                     // K slab 0 and T's first half: both dead now
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (!fail && tid == 0) {
+            bulk_store(img, smem_u32(sm + Lay::KQ), 16384);
+            bulk_commit();
+        }
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, Lay::TMEM_COLS);
     }
-    if (tid == 0) {
-        unsigned char* img = p.img + ((size_t)g * p.H + h) * (size_t)Lay::OUT;
-        bulk_store(img, smem_u32(stage), Lay::OUT);
-        bulk_commit();
-        bulk_wait_read0();                                // the shared source stays until it is read
-    }
+    if (tid == 0) bulk_wait_read0();                      // the shared sources stay until they are read
 }
 
 // ---------------------------------------------------------------- state --
