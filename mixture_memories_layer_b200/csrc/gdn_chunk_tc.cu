@@ -683,8 +683,8 @@ struct StateLayout {
     static constexpr int VB = KQ0 + 2 * KQSZ;                 // [64 x 128] bf16: two 64-column slabs
     static constexpr int IMGB = D * 128 + IMG;                // one prep image: Wk (d_k rows x 64), then Q'
     static constexpr int WB = VB + 2 * 8192;                  // prep image
-    static constexpr int STG = WB + IMGB;                     // 8 x [32 rows x 32 d_v] bf16: per-warp output staging
-    static constexpr int GBB = STG + 16384;                   // 2 gate records
+    static constexpr int STG = WB + IMGB;                     // 2 x 8 x [32 rows x 32 d_v] bf16: per-warp output staging
+    static constexpr int GBB = STG + 2 * 16384;               // 2 gate records
     static constexpr int BARS = GBB + 2 * GB * 4;
     static constexpr int MISC = BARS + NBARS * 8;
     static constexpr size_t BYTES = 1024 + MISC + 16;
@@ -939,10 +939,12 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
             }
             // ---- output o_r = scale (S e^gamma_r q_r + sum_s P_rs u_s), rows r < n: this
-            // warp's [32 rows x 32 d_v] piece, staged row-major, leaves by one TMA store
+            // warp's [32 rows x 32 d_v] piece, staged row-major (two staging buffers,
+            // by chunk parity), leaves by one TMA store
             {
-                const uint32_t stg = stg0 + warp * 2048 + lane * 2;
-                if (lane == 0) bulk_wait_read0();     // the previous chunk's store has read the piece
+                const uint32_t piece = stg0 + b * 16384 + warp * 2048;
+                const uint32_t stg = piece + lane * 2;
+                if (lane == 0) bulk_wait_read1();     // the store from two chunks ago has read this buffer
                 __syncwarp();
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -955,7 +957,7 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tm_o, stg0 + warp * 2048, h * D + dv0 + 32 * qd, (int)(r0 + sh));
+                        tma_store_2d(&tm_o, piece, h * D + dv0 + 32 * qd, (int)(r0 + sh));
                         bulk_commit();
                     }
                 } else {
