@@ -121,18 +121,22 @@ skinny_kernel(const __grid_constant__ CUtensorMap tm_x, SkinnyArgs a, int NS) {
         *abort_flag = 0;
         fence_barrier_init();
     }
-    const uint32_t wsm = smem_u32(wsm_p);
-    for (int i = threadIdx.x; i < NT * 8 * (a.D / 8); i += blockDim.x) {
-        const int row = i / (a.D / 8), f = (i % (a.D / 8)) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < a.ncol) v = __ldg(reinterpret_cast<const uint4*>(a.w + (int64_t)row * a.D + f));
-        const uint32_t chunk = (uint32_t)((f & 63) >> 3);
-        const uint32_t addr = wsm + (uint32_t)(f >> 6) * (NT * 8 * 128) + row * 128 + ((chunk ^ (uint32_t)(row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-    }
     __syncthreads();
+    const uint32_t wsm = smem_u32(wsm_p);
     const uint32_t ring = smem_u32(sm);
     const int nbox = a.D / 64;
+    if (warp < NS) {
+        // the consumers stage W while the producer's first tiles are in flight
+        for (int i = threadIdx.x; i < NT * 8 * (a.D / 8); i += NS * 32) {
+            const int row = i / (a.D / 8), f = (i % (a.D / 8)) * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (row < a.ncol) v = __ldg(reinterpret_cast<const uint4*>(a.w + (int64_t)row * a.D + f));
+            const uint32_t chunk = (uint32_t)((f & 63) >> 3);
+            const uint32_t addr = wsm + (uint32_t)(f >> 6) * (NT * 8 * 128) + row * 128 + ((chunk ^ (uint32_t)(row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(NS * 32) : "memory");
+    }
 
     if (warp == NS) {
         // ---------------------------------------------------- producer
