@@ -36,7 +36,12 @@ the Gated DeltaNet rule those pages name,
     S_t = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
     o_t = S_t (scale * q_t),
 
-with S the d_v x d_k state, read after the write at token t.
+with S the d_v x d_k state, read after the write at token t.  A second rule
+of the family [blog] "Linear Recurrent Memory" lists (linear attention,
+RetNet, Mamba2-style memories: the scalar-gated linear form, without the
+delta correction) is available wherever the rule can be chosen:
+
+    S_t = alpha_t * S_{t-1} + beta_t v_t k_t^T,      o_t = S_t (scale * q_t).
 
 Readings where the pages are silent (each also listed in the design notes):
 q, beta and alpha are shared by all memories (one W_q, W_beta, W_a); every
@@ -209,16 +214,35 @@ def gdn_step(S, q_t, k_t, v_t, beta_t, log_alpha_t, scale: float = 1.0):
     return o, S
 
 
-def gdn_recurrence(q, k, v, beta, log_alpha, h0=None, scale: float = 1.0):
+def gla_step(S, q_t, k_t, v_t, beta_t, log_alpha_t, scale: float = 1.0):
+    """One token of the scalar-gated linear rule (the linear-attention form of
+    the update-rule family in [blog] "Linear Recurrent Memory": linear
+    attention with alpha = beta = 1, RetNet with a fixed alpha per head,
+    Mamba2-style memories with a data-dependent scalar alpha):
+
+        S_t = alpha_t S_{t-1} + beta_t v_t k_t^T,     o_t = S_t (scale q_t)
+
+    Shapes as gdn_step.  Returns (o_t [H,dv], S_t)."""
+    a = np.exp(np.asarray(log_alpha_t, F64))[:, None, None]
+    b = np.asarray(beta_t, F64)[:, None, None]
+    S = a * S + b * np.asarray(v_t, F64)[:, :, None] * np.asarray(k_t, F64)[:, None, :]
+    o = np.einsum("hvk,hk->hv", S, scale * np.asarray(q_t, F64))
+    return o, S
+
+
+RULES = {"gated_delta": gdn_step, "gated_linear": gla_step}
+
+
+def gdn_recurrence(q, k, v, beta, log_alpha, h0=None, scale: float = 1.0, rule: str = "gated_delta"):
     """Token-by-token recurrence over one segment.  q,k [T,H,dk]; v [T,H,dv];
-    beta, log_alpha [T,H]; h0 [H,dv,dk] or None (zeros).  Returns
-    (o [T,H,dv], S_final [H,dv,dk])."""
+    beta, log_alpha [T,H]; h0 [H,dv,dk] or None (zeros); rule one of RULES
+    (default the Gated DeltaNet step).  Returns (o [T,H,dv], S_final [H,dv,dk])."""
     T, H, dk = np.shape(k)
     dv = np.shape(v)[-1]
     S = np.zeros((H, dv, dk), F64) if h0 is None else np.array(h0, F64, copy=True)
     o = np.zeros((T, H, dv), F64)
     for t in range(T):
-        o[t], S = gdn_step(S, q[t], k[t], v[t], beta[t], log_alpha[t], scale)
+        o[t], S = RULES[rule](S, q[t], k[t], v[t], beta[t], log_alpha[t], scale)
     return o, S
 
 
@@ -272,7 +296,7 @@ def gdn_chunked(q, k, v, beta, log_alpha, h0=None, scale: float = 1.0, chunk: in
 # ----------------------------------------------------------------------------
 
 def mom_forward(x, p, cu_seqlens, top_k: int, H: int, d: int, scale: float = 1.0,
-                forced_idx=None, h0_shared=None, h0_mem=None):
+                forced_idx=None, h0_shared=None, h0_mem=None, rule: str = "gated_delta"):
     """One MoM layer forward over a packed batch.
 
     x [N,d_model]; p the weights (see the input generator for names and
@@ -302,7 +326,7 @@ def mom_forward(x, p, cu_seqlens, top_k: int, H: int, d: int, scale: float = 1.0
         t0, t1 = int(cu[s]), int(cu[s + 1])
         h0 = None if h0_shared is None else h0_shared[s]
         o_shared[t0:t1], h_shared[s] = gdn_recurrence(
-            q[t0:t1], k_sh[t0:t1], v_sh[t0:t1], beta[t0:t1], log_alpha[t0:t1], h0, scale)
+            q[t0:t1], k_sh[t0:t1], v_sh[t0:t1], beta[t0:t1], log_alpha[t0:t1], h0, scale, rule)
         for m in range(M):
             # the tokens of sequence s routed to memory m, in token order
             hit = idx[t0:t1] == m
@@ -312,7 +336,7 @@ def mom_forward(x, p, cu_seqlens, top_k: int, H: int, d: int, scale: float = 1.0
                 h_mem[m, s] = 0.0 if h0 is None else h0
                 continue
             k_m, v_m = memory_kv(x[rows], p, m, H, d)
-            o_m, h_mem[m, s] = gdn_recurrence(q[rows], k_m, v_m, beta[rows], log_alpha[rows], h0, scale)
+            o_m, h_mem[m, s] = gdn_recurrence(q[rows], k_m, v_m, beta[rows], log_alpha[rows], h0, scale, rule)
             slot = np.argmax(idx[rows] == m, axis=1)
             o_mem[rows, slot] = o_m
     # combine: shared memory with weight 1 plus the router-weighted memories
@@ -323,7 +347,7 @@ def mom_forward(x, p, cu_seqlens, top_k: int, H: int, d: int, scale: float = 1.0
 
 
 def mom_forward_mixed_state(x, p, cu_seqlens, top_k: int, H: int, d: int, scale: float = 1.0,
-                            forced_idx=None):
+                            forced_idx=None, rule: str = "gated_delta"):
     """The layer in its "mix the memories first, then read out" form
     ([blog] Mixture-of-Memories: the active memories are summed with their
     router weights into one mixed memory, which is then read with q).
@@ -345,11 +369,11 @@ def mom_forward_mixed_state(x, p, cu_seqlens, top_k: int, H: int, d: int, scale:
     for s in range(len(cu) - 1):
         states = np.zeros((M + 1, H, d, d), F64)      # slot M is the shared memory
         for t in range(int(cu[s]), int(cu[s + 1])):
-            _, states[M] = gdn_step(states[M], q[t], k_sh[t], v_sh[t], beta[t], log_alpha[t])
+            _, states[M] = RULES[rule](states[M], q[t], k_sh[t], v_sh[t], beta[t], log_alpha[t])
             for j in range(top_k):
                 m = int(idx[t, j])
                 k_m, v_m = memory_kv(x[t:t + 1], p, m, H, d)
-                _, states[m] = gdn_step(states[m], q[t], k_m[0], v_m[0], beta[t], log_alpha[t])
+                _, states[m] = RULES[rule](states[m], q[t], k_m[0], v_m[0], beta[t], log_alpha[t])
             mixed = states[M] + sum(gate[t, j] * states[int(idx[t, j])] for j in range(top_k))
             out[t] = np.einsum("hvk,hk->hv", mixed, scale * q[t])
     return out
@@ -370,7 +394,8 @@ def decode_state_from_prefill(h_shared, h_mem):
     return st
 
 
-def mom_decode_step(x, p, state, top_k: int, H: int, d: int, scale: float = 1.0, forced_idx=None):
+def mom_decode_step(x, p, state, top_k: int, H: int, d: int, scale: float = 1.0, forced_idx=None,
+                    rule: str = "gated_delta"):
     """One new token per sequence.  x [B,d_model]; state [B,M+1,H,d,d]
     (slot M = shared), not modified.  Each sequence updates only its k routed
     states and the shared one.  Returns (out [B,H,d], new_state, idx, gate,
@@ -386,11 +411,11 @@ def mom_decode_step(x, p, state, top_k: int, H: int, d: int, scale: float = 1.0,
     new = np.array(state, F64, copy=True)
     out = np.zeros((B, H, d), F64)
     for b in range(B):
-        o_sh, new[b, M] = gdn_step(new[b, M], q[b], k_sh[b], v_sh[b], beta[b], log_alpha[b], scale)
+        o_sh, new[b, M] = RULES[rule](new[b, M], q[b], k_sh[b], v_sh[b], beta[b], log_alpha[b], scale)
         out[b] = o_sh
         for j in range(top_k):
             m = int(idx[b, j])
             k_m, v_m = memory_kv(x[b:b + 1], p, m, H, d)
-            o_m, new[b, m] = gdn_step(new[b, m], q[b], k_m[0], v_m[0], beta[b], log_alpha[b], scale)
+            o_m, new[b, m] = RULES[rule](new[b, m], q[b], k_m[0], v_m[0], beta[b], log_alpha[b], scale)
             out[b] += gate[b, j] * o_m
     return out, new, idx, gate, near_tie
