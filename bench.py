@@ -41,7 +41,10 @@ METRIC = "MoM layer fwd tokens/s at 1 B200 and % of roofline; decode tokens/s"
 UNIT = "tokens/s"
 FWD = "mom380m"
 DEC = "decode_b256"
-EXTRA = ("tiny_fp32", "mom380m_skew_varlen", "mom1p3b_m16")
+# (workload, memory rule): the other forward workloads, and the 380M shape with
+# the scalar-gated linear memories
+EXTRA = (("tiny_fp32", "gated_delta"), ("mom380m_skew_varlen", "gated_delta"), ("mom1p3b_m16", "gated_delta"),
+         ("mom380m", "gated_linear"))
 TIE_GAP = 1e-4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -276,7 +279,7 @@ def near_tie_tokens(x, w_r, b_r, top_k, gap=TIE_GAP):
     return int(((top[:, top_k - 1] - top[:, top_k]) < gap).sum().item())
 
 
-def config_bench(name, dev, steps, warmup, peaks, flush):
+def config_bench(name, dev, steps, warmup, peaks, flush, rule="gated_delta"):
     """One of the other forward workloads, timed like the headline one."""
     import torch
     from mixture_memories_layer_b200 import layer as L
@@ -284,7 +287,7 @@ def config_bench(name, dev, steps, warmup, peaks, flush):
     w = synth.WORKLOADS[name]
     p = synth.make_problem(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    lay = L.MoMLayer(L.pack_weights(p, dt, dev), w.heads, w.d_head, w.top_k)
+    lay = L.MoMLayer(L.pack_weights(p, dt, dev), w.heads, w.d_head, w.top_k, rule=rule)
     x = torch.as_tensor(p["x"]).to(dev, dt)
     cu = torch.as_tensor(p["cu_seqlens"]).to(dev)
     for _ in range(warmup):
@@ -292,12 +295,12 @@ def config_bench(name, dev, steps, warmup, peaks, flush):
     torch.cuda.synchronize()
     errs = lay.device_errors()
     if errs:
-        raise SystemExit("device error records in %s: %s" % (name, errs))
+        raise SystemExit("device error records in %s (%s): %s" % (name, rule, errs))
     step_ms, per_call = time_forward(lay, x, cu, steps, flush)
     ms = sum(step_ms) / steps
     S = int(cu.numel()) - 1
     rows = lay.buffers(w.n_tokens, S)["mem_offset"].cpu().tolist()
-    out = {"workload": workload_desc(w), "dtype": w.dtype, "tokens": w.n_tokens, "sequences": S,
+    out = {"workload": workload_desc(w), "memory_rule": rule, "dtype": w.dtype, "tokens": w.n_tokens, "sequences": S,
            "ms_per_step": ms, "value": w.n_tokens / (ms / 1e3), "unit": UNIT, "per_call_ms": per_call,
            "routed_rows_per_memory": [b - a for a, b in zip(rows[:-1], rows[1:])],
            "near_tie_tokens": near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)}
@@ -382,7 +385,8 @@ def gpu_arm(args):
     decode = None if args.no_decode else decode_bench(args, dev, world, rank, max_over_ranks, barrier)
     configs = None
     if not args.no_configs and world == 1:
-        configs = {name: config_bench(name, dev, args.steps, args.warmup, peaks, flush) for name in EXTRA}
+        configs = {(name if rule == "gated_delta" else "%s_%s" % (name, rule)):
+                   config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule) for name, rule in EXTRA}
     clocks.__exit__(None, None, None)
     layer_roof["near_tie_tokens"] = near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)
     return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,

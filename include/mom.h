@@ -63,6 +63,23 @@ typedef int mom_dtype;
 #define MOM_F32   0
 #define MOM_BF16  1
 
+/* Memory update rules.  The authors' MoM blog post ("Linear Recurrent
+ * Memory") lists the family of rules a memory can use -- linear attention,
+ * RetNet, GLA, DeltaNet, Gated DeltaNet, Mamba2, HGRN2 -- in one
+ * linear-attention form (the page's formulas were lost in extraction); its
+ * experiments use Gated DeltaNet.  Both rules here have a scalar gate
+ * alpha_t = exp(log_alpha_t) and a write strength beta_t per token and head:
+ *   MOM_RULE_GATED_DELTA   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *                          (Gated DeltaNet; DeltaNet with alpha = 1)
+ *   MOM_RULE_GATED_LINEAR  S_t = alpha_t S_{t-1} + beta_t v_t k_t^T
+ *                          (linear attention with alpha = beta = 1, RetNet with a
+ *                          fixed alpha per head, Mamba2-style memories)
+ * and the readout o_t = S_t (scale q_t).  Rules with a per-dimension gate
+ * (GLA, HGRN2) are not provided. */
+typedef int mom_rule;
+#define MOM_RULE_GATED_DELTA   0
+#define MOM_RULE_GATED_LINEAR  1
+
 /* Device error record codes (mom_get_error's *code). */
 #define MOM_DEVERR_NONE       0
 #define MOM_DEVERR_MEM_INDEX  1  /* topk_idx entry outside [0, n_mem) or repeated in a row */
@@ -281,6 +298,28 @@ mom_status mom_gdn_chunk_state(const void* q, const int32_t* qidx, const void* k
                                const float* h0, float* h_final, void* o,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* The same three calls for either memory rule (MOM_RULE_*); the mom_gdn_*
+ * calls are these with MOM_RULE_GATED_DELTA.  Same arguments otherwise, same
+ * workspace (mom_gdn_workspace_size); MOM_ERR_ARG for an unknown rule. */
+mom_status mom_memory_chunk_fwd(const void* q, const int32_t* qidx, const void* k, const void* v,
+                                const float* beta, const float* log_alpha,
+                                const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                                int H, int d, float scale, mom_dtype dt, mom_rule rule,
+                                const float* h0, float* h_final, void* o,
+                                void* ws, size_t ws_bytes, void* stream);
+mom_status mom_memory_chunk_prep(const void* q, const int32_t* qidx, const void* k, const void* v,
+                                 const float* beta, const float* log_alpha,
+                                 const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                                 int H, int d, float scale, mom_dtype dt, mom_rule rule,
+                                 const float* h0, float* h_final, void* o,
+                                 void* ws, size_t ws_bytes, void* stream);
+mom_status mom_memory_chunk_state(const void* q, const int32_t* qidx, const void* k, const void* v,
+                                  const float* beta, const float* log_alpha,
+                                  const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                                  int H, int d, float scale, mom_dtype dt, mom_rule rule,
+                                  const float* h0, float* h_final, void* o,
+                                  void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * mom_combine_unpermute -- the combine (paper card, Summary: outputs are
  * combined using the router weights; blog post, "硬件高效實現": summing the
@@ -329,6 +368,12 @@ mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_mod
                            int n_mem, int top_k, float scale, mom_dtype dt,
                            float* state, void* out, int32_t* topk_idx,
                            void* ws, size_t ws_bytes, void* stream);
+/* mom_decode_step for either memory rule (MOM_RULE_*); mom_decode_step is
+ * this with MOM_RULE_GATED_DELTA. */
+mom_status mom_decode_step_rule(const void* x, const mom_weights* w, int B, int d_model, int H, int d,
+                                int n_mem, int top_k, float scale, mom_dtype dt, mom_rule rule,
+                                float* state, void* out, int32_t* topk_idx,
+                                void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -46,9 +46,16 @@ SIGNATURES = {
                                _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mom_gdn_chunk_state": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I,
                                _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_memory_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I,
+                                  _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_memory_chunk_prep": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I,
+                                   _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_memory_chunk_state": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I,
+                                    _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mom_combine_unpermute": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
     "mom_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "mom_decode_step": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_decode_step_rule": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
 }
 
 
@@ -220,6 +227,31 @@ def mom_gdn_chunk_state(q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_fin
     _gdn("mom_gdn_chunk_state", q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_final, o, ws, stream)
 
 
+MOM_RULE_GATED_DELTA, MOM_RULE_GATED_LINEAR = 0, 1
+RULES = {"gated_delta": MOM_RULE_GATED_DELTA, "gated_linear": MOM_RULE_GATED_LINEAR}
+
+
+def _memory(name, q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream):
+    n_rows, H, d = k.shape
+    _check(getattr(lib, name)(_p(q), _p(qidx), _p(k), _p(v), _p(beta), _p(log_alpha), _p(seg_cu),
+                              seg_cu.numel() - 1, n_rows, q.shape[0], H, d, float(scale),
+                              dtype_code(k.dtype), int(rule), _p(h0), _p(h_final), _p(o), _p(ws), ws.numel(),
+                              _s(stream)), name)
+
+
+def mom_memory_chunk_fwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None):
+    _memory("mom_memory_chunk_fwd", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream)
+
+
+def mom_memory_chunk_prep(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None):
+    _memory("mom_memory_chunk_prep", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream)
+
+
+def mom_memory_chunk_state(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None):
+    _memory("mom_memory_chunk_state", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws,
+            stream)
+
+
 def mom_combine_unpermute(o_sh, o_p, row_of, topk_gate, out, ws, stream=None):
     n_tok, H, d = o_sh.shape
     top_k = topk_gate.shape[1]
@@ -237,3 +269,11 @@ def mom_decode_step(x, weights: MomWeights, H, d, n_mem, top_k, scale, state, ou
     _check(lib.mom_decode_step(_p(x), ctypes.byref(weights), B, d_model, H, d, n_mem, top_k, float(scale),
                                dtype_code(x.dtype), _p(state), _p(out), _p(topk_idx), _p(ws), ws.numel(),
                                _s(stream)), "mom_decode_step")
+
+
+def mom_decode_step_rule(x, weights: MomWeights, H, d, n_mem, top_k, scale, rule, state, out, topk_idx, ws,
+                         stream=None):
+    B, d_model = x.shape
+    _check(lib.mom_decode_step_rule(_p(x), ctypes.byref(weights), B, d_model, H, d, n_mem, top_k, float(scale),
+                                    dtype_code(x.dtype), int(rule), _p(state), _p(out), _p(topk_idx), _p(ws),
+                                    ws.numel(), _s(stream)), "mom_decode_step_rule")

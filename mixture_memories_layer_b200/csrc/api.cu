@@ -165,8 +165,9 @@ size_t mom_gdn_workspace_size(int64_t n_rows, int n_seg, int H, int d, mom_dtype
 static mom_status gdn_call(const void* q, const int32_t* qidx, const void* k, const void* v, const float* beta,
                            const float* log_alpha, const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
                            int H, int d, float scale, mom_dtype dt, const float* h0, float* h_final, void* o,
-                           void* ws, size_t ws_bytes, void* stream, int phase) {
+                           void* ws, size_t ws_bytes, void* stream, int phase, int rule = MOM_RULE_GATED_DELTA) {
     if (!dt_ok(dt) || n_seg < 0 || n_rows < 0 || n_q_rows < 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (rule != MOM_RULE_GATED_DELTA && rule != MOM_RULE_GATED_LINEAR) return MOM_ERR_ARG;
     if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < mom_gdn_workspace_size(n_rows, n_seg, H, d, dt)) return MOM_ERR_ARG;
     if (n_seg == 0) return MOM_OK;
@@ -180,6 +181,7 @@ static mom_status gdn_call(const void* q, const int32_t* qidx, const void* k, co
     GdnArgs a{q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale,
               h0, h_final, o, ws, ws_bytes};
     a.phase = phase;
+    a.rule = rule;
     cudaStream_t st = as_stream(stream);
     if (gdn_tc_supported(a, dt)) return cuda_status(launch_gdn_tc(a, st));
     return cuda_status(launch_gdn_recurrent(a, dt, st));
@@ -214,6 +216,19 @@ mom_status mom_gdn_chunk_state(const void* q, const int32_t* qidx, const void* k
     return gdn_call(q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, dt, h0, h_final, o,
                     ws, ws_bytes, stream, GDN_STATE);
 }
+
+#define MOM_MEMORY_CALL(NAME, PHASE)                                                                       \
+    mom_status NAME(const void* q, const int32_t* qidx, const void* k, const void* v, const float* beta,     \
+                    const float* log_alpha, const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows, \
+                    int H, int d, float scale, mom_dtype dt, mom_rule rule, const float* h0, float* h_final,  \
+                    void* o, void* ws, size_t ws_bytes, void* stream) {                                      \
+        return gdn_call(q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, dt, h0,  \
+                        h_final, o, ws, ws_bytes, stream, PHASE, rule);                                      \
+    }
+MOM_MEMORY_CALL(mom_memory_chunk_fwd, GDN_PREP | GDN_STATE)
+MOM_MEMORY_CALL(mom_memory_chunk_prep, GDN_PREP)
+MOM_MEMORY_CALL(mom_memory_chunk_state, GDN_STATE)
+#undef MOM_MEMORY_CALL
 
 // ----------------------------------------------------------------- combine
 mom_status mom_combine_unpermute(const void* o_sh, const void* o_p, const int32_t* row_of,
@@ -270,7 +285,16 @@ mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_mod
                            int n_mem, int top_k, float scale, mom_dtype dt,
                            float* state, void* out, int32_t* topk_idx,
                            void* ws, size_t ws_bytes, void* stream) {
+    return mom_decode_step_rule(x, w, B, d_model, H, d, n_mem, top_k, scale, dt, MOM_RULE_GATED_DELTA, state, out,
+                                topk_idx, ws, ws_bytes, stream);
+}
+
+mom_status mom_decode_step_rule(const void* x, const mom_weights* w, int B, int d_model, int H, int d,
+                                int n_mem, int top_k, float scale, mom_dtype dt, mom_rule rule,
+                                float* state, void* out, int32_t* topk_idx,
+                                void* ws, size_t ws_bytes, void* stream) {
     if (!dt_ok(dt) || B < 0 || d_model <= 0 || d_model % 64 != 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (rule != MOM_RULE_GATED_DELTA && rule != MOM_RULE_GATED_LINEAR) return MOM_ERR_ARG;
     if (top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM || !w) return MOM_ERR_ARG;
     if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < mom_decode_workspace_size(B, d_model, H, d, n_mem, top_k)) return MOM_ERR_ARG;
@@ -303,6 +327,7 @@ mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_mod
     if (e != cudaSuccess) return MOM_ERR_CUDA;
     DecodeArgs da{base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, beta, la, gate,
                   idx, row_of, B, H, d, n_mem, top_k, scale, state, out, ws};
+    da.rule = rule;
     return cuda_status(launch_decode_state(da, dt, st));
 }
 

@@ -8,6 +8,7 @@
 // written once:
 //   y = S k, z = S q (one pass over S), u = beta (v - alpha y),
 //   S' = alpha S + u k^T, o = scale (alpha z + u (k . q)),
+// (with the scalar-gated linear rule u = beta v: no delta correction)
 //   out += w_slot * o   (w = router gate, 1 for the shared memory).
 // The state stream (read + write of (k+1) * d * d floats per sequence and
 // head) is the whole cost, so the kernel is written for HBM bandwidth:
@@ -34,6 +35,7 @@ decode_state_kernel(DecodeArgs a) {
     load_vec<E>(q + ((int64_t)b * H + h) * D + lane * E, qq);
     const float be = a.beta[(int64_t)b * H + h];
     const float al = expf(a.log_alpha[(int64_t)b * H + h]);
+    const float dl = a.rule == MOM_RULE_GATED_DELTA ? al : 0.f;
 
     float out_acc[RPW];
 #pragma unroll
@@ -85,7 +87,7 @@ decode_state_kernel(DecodeArgs a) {
         warp_sum_n<2 * RPW + 1>(red);
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
-            const float u = be * (vv[i] - al * red[2 * i]);
+            const float u = be * (vv[i] - dl * red[2 * i]);
 #pragma unroll
             for (int e = 0; e < E; ++e) S[i][e] = fmaf(al, S[i][e], u * kk[e]);
             out_acc[i] = fmaf(w, a.scale * fmaf(al, red[2 * i + 1], u * red[2 * RPW]), out_acc[i]);

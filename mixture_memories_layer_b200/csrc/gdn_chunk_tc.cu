@@ -38,7 +38,9 @@
 //             when given, scaled in place), one MMA warp (Z in two d_k
 //             halves, then X), eight math warps (the last to finish Y issues
 //             the output and state-update MMAs).
-// Rows past a segment's end are masked (zero gates, zeroed key/value rows),
+// The scalar-gated linear rule S_t = alpha_t S_{t-1} + beta_t v_t k_t^T runs
+// the same kernels with L = 0 (so T = I, U = diag(beta) V) and Y = V^T.
+// Rows past a segment's end are masked (zero gates, zeroed or masked rows),
 // so a ragged tail chunk needs no padding.
 #include "common.cuh"
 #include "kernels.h"
@@ -73,6 +75,7 @@ struct GdnTc {
     int4* chunk_info;     // per chunk: segment, first row, rows (<= C)
     unsigned char* img;
     void* err;
+    int delta;            // 1: the Gated DeltaNet rule; 0: the scalar-gated linear rule (L = 0, Y = V^T)
 };
 
 // ------------------------------------------------------------- schedule --
@@ -480,7 +483,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tmem_ld_x32(tmem + lane_base + 32 * colh, gv);
         tmem_ld_wait();
         const int r = rho;
-        const float g2r = g2[r], br = gbeta[r];           // beta is 0 past n
+        // beta is 0 past n; without the delta correction L = 0 (T = I)
+        const float g2r = g2[r], br = p.delta ? gbeta[r] : 0.f;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int s = 32 * colh + e;
@@ -851,13 +855,15 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 tmem_ld_wait();
                 uint32_t py[16], pr[16];
                 // positions past n hold other rows' keys and values: Y is 0 there
-                // (a select, so that nothing read there can reach the products)
+                // (a select, so that nothing read there can reach the products);
+                // without the delta correction Y = V^T
+                const float zs = p.delta ? -1.f : 0.f;
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const float y0 = sh + e < n
-                        ? fmaf(-__uint_as_float(z[e]), eg[e], __uint_as_float(vv[e / 2] << 16)) : 0.f;
+                        ? fmaf(zs * __uint_as_float(z[e]), eg[e], __uint_as_float(vv[e / 2] << 16)) : 0.f;
                     const float y1 = sh + e + 1 < n
-                        ? fmaf(-__uint_as_float(z[e + 1]), eg[e + 1], __uint_as_float(vv[e / 2] & 0xFFFF0000u)) : 0.f;
+                        ? fmaf(zs * __uint_as_float(z[e + 1]), eg[e + 1], __uint_as_float(vv[e / 2] & 0xFFFF0000u)) : 0.f;
                     py[e / 2] = pack_bf16(y0, y1);
                     pr[e / 2] = pack_bf16(rho1 * y0, rho1 * y1);
                 }
@@ -1217,6 +1223,7 @@ cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st) {
     base += up256((size_t)mc * sizeof(int4));
     t.img = base;
     t.err = a.ws;
+    t.delta = a.rule == MOM_RULE_GATED_DELTA ? 1 : 0;
     return a.d == 256 ? launch_d<256>(t, mc, a.phase, st) : launch_d<128>(t, mc, a.phase, st);
 }
 

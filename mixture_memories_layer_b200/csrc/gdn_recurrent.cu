@@ -2,6 +2,9 @@
 //
 //   S_r = alpha_r S_{r-1} (I - beta_r k_r k_r^T) + beta_r v_r k_r^T,  o_r = S_r (scale q_r)
 //
+// or, with the scalar-gated linear rule, S_r = alpha_r S_{r-1} + beta_r v_r k_r^T
+// (u_i = beta v_i below: the delta correction -alpha y_i drops out).
+//
 // (the authors' MoM blog post, experiments section: every memory uses Gated
 // DeltaNet's gate and update rule).  Each row i of S (one d_v index) evolves
 // on its own given k, beta and alpha:
@@ -80,8 +83,10 @@ gdn_recurrent_kernel(GdnArgs a) {
         const float kq = red[2 * RPW];
         float my_o = 0.f;
 #pragma unroll
+        const float dl = a.rule == MOM_RULE_GATED_DELTA ? al : 0.f;
+#pragma unroll
         for (int i = 0; i < RPW; ++i) {
-            const float u = b * (vv[i] - al * red[2 * i]);
+            const float u = b * (vv[i] - dl * red[2 * i]);
 #pragma unroll
             for (int e = 0; e < E; ++e) S[i][e] = fmaf(al, S[i][e], u * kk[e]);
             const float oi = a.scale * fmaf(al, red[2 * i + 1], u * kq);

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "mom.h"
+
 namespace mom {
 
 // Counts every kernel launch (mom_launch_count).
@@ -92,6 +94,8 @@ struct GdnArgs {
     // GDN_PREP: the state-independent per-chunk work; GDN_STATE: the serial
     // walk over the chunks (reads what GDN_PREP left in ws); both by default
     int phase = GDN_PREP | GDN_STATE;
+    // MOM_RULE_GATED_DELTA or MOM_RULE_GATED_LINEAR
+    int rule = MOM_RULE_GATED_DELTA;
 };
 cudaError_t launch_gdn_recurrent(const GdnArgs& a, int dt, cudaStream_t st);
 
@@ -114,6 +118,7 @@ struct DecodeArgs {
     float* state;
     void* out;
     void* ws;
+    int rule = MOM_RULE_GATED_DELTA;
 };
 cudaError_t launch_decode_state(const DecodeArgs& a, int dt, cudaStream_t st);
 

@@ -41,12 +41,17 @@ class MoMLayer:
     """Holds packed weights and reusable buffers for one layer shape."""
 
     def __init__(self, weights: Dict[str, torch.Tensor], heads: int, d_head: int, top_k: int,
-                 scale: float = 1.0, gdn_schedule: str = "streams"):
+                 scale: float = 1.0, gdn_schedule: str = "streams", rule: str = "gated_delta"):
         """gdn_schedule: "streams" (each problem's GDN prep and walk on its own
         stream, the shared memory's on a high-priority one) or "phased" (both
         problems' prep on the whole GPU, then both walks).  Measured on B200:
-        380M-shape layer 0.336 vs 0.344 ms, 1.3B-shape layer 1.032 vs
-        1.037 ms."""
+        380M-shape layer 0.295 vs 0.308 ms, 1.3B-shape layer 0.904 vs
+        0.963 ms.  rule: the memories' update rule, "gated_delta" (Gated
+        DeltaNet, the default) or "gated_linear" (S_t = alpha_t S_{t-1} +
+        beta_t v_t k_t^T: linear attention, RetNet, Mamba2-style memories)."""
+        if rule not in B.RULES:
+            raise ValueError("rule must be one of %s" % sorted(B.RULES))
+        self.rule = B.RULES[rule]
         self.w = weights
         self.H, self.d, self.top_k, self.scale = heads, d_head, top_k, scale
         if gdn_schedule not in ("phased", "streams"):
@@ -140,21 +145,21 @@ class MoMLayer:
         hs = b["h_shared"] if want_states else None
         hm = b["h_mem"] if want_states else None
         gdn_sh = (b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens,
-                  self.scale, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"])
+                  self.scale, self.rule, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"])
         gdn_p = (b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
-                 self.scale, h0_mem, hm, b["o_p"], b["ws_gdn_p"])
+                 self.scale, self.rule, h0_mem, hm, b["o_p"], b["ws_gdn_p"])
         fork = torch.cuda.Event()
         if self.gdn_schedule == "phased":
             # both problems' state-independent chunk work first, on the whole
             # GPU; then the two serial walks side by side, the shared memory's
             # (whole sequences: the longest chain) launched first so that its
             # CTAs hold SMs before the routed walks fill the rest
-            B.mom_gdn_chunk_prep(*gdn_sh, stream=st)
-            B.mom_gdn_chunk_prep(*gdn_p, stream=st)
+            B.mom_memory_chunk_prep(*gdn_sh, stream=st)
+            B.mom_memory_chunk_prep(*gdn_p, stream=st)
             fork.record(st)
-            B.mom_gdn_chunk_state(*gdn_sh, stream=st)
+            B.mom_memory_chunk_state(*gdn_sh, stream=st)
             side.wait_event(fork)
-            B.mom_gdn_chunk_state(*gdn_p, stream=side)
+            B.mom_memory_chunk_state(*gdn_p, stream=side)
         else:
             # each problem's prep then walk on its own stream: the shared
             # problem on a high-priority stream (its CTAs are dispatched first,
@@ -164,10 +169,10 @@ class MoMLayer:
             fork.record(st)
             hi.wait_event(fork)
             side.wait_event(fork)
-            B.mom_gdn_chunk_prep(*gdn_sh, stream=hi)
-            B.mom_gdn_chunk_state(*gdn_sh, stream=hi)
-            B.mom_gdn_chunk_prep(*gdn_p, stream=side)
-            B.mom_gdn_chunk_state(*gdn_p, stream=side)
+            B.mom_memory_chunk_prep(*gdn_sh, stream=hi)
+            B.mom_memory_chunk_state(*gdn_sh, stream=hi)
+            B.mom_memory_chunk_prep(*gdn_p, stream=side)
+            B.mom_memory_chunk_state(*gdn_p, stream=side)
             hi_done = torch.cuda.Event()
             hi_done.record(hi)
             st.wait_event(hi_done)
@@ -214,8 +219,8 @@ class MoMLayer:
         out = self._buf("dec_out", (Bn, self.H, self.d), self.dtype)
         idx = self._buf("dec_idx", (Bn, self.top_k), torch.int32)
         ws = self._ws("decode", B.mom_decode_workspace_size(Bn, self.d_model, self.H, self.d, self.n_mem, self.top_k))
-        B.mom_decode_step(x, self._c_weights, self.H, self.d, self.n_mem, self.top_k, self.scale, state, out, idx, ws,
-                          stream=stream)
+        B.mom_decode_step_rule(x, self._c_weights, self.H, self.d, self.n_mem, self.top_k, self.scale, self.rule,
+                               state, out, idx, ws, stream=stream)
         return out, idx
 
 

@@ -30,12 +30,12 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
 
 
-def run_layer(w, p, scale=1.0, h0_shared=None, h0_mem=None):
+def run_layer(w, p, scale=1.0, h0_shared=None, h0_mem=None, rule="gated_delta"):
     """Runs the CUDA layer on the problem p; returns (layer, numpy results)."""
     from mixture_memories_layer_b200 import layer as L
     dt = torch_dtype(w)
     weights = L.pack_weights(p, dt)
-    lay = L.MoMLayer(weights, w.heads, w.d_head, w.top_k, scale)
+    lay = L.MoMLayer(weights, w.heads, w.d_head, w.top_k, scale, rule=rule)
     x = torch.as_tensor(p["x"]).to("cuda", dt)
     cu = torch.as_tensor(p["cu_seqlens"]).to("cuda", torch.int32)
     b = lay.forward(x, cu, h0_shared=h0_shared, h0_mem=h0_mem)
