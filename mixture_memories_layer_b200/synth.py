@@ -15,7 +15,9 @@ shared memory, memory-count scaling to 16):
 * X ~ N(0, 1); the router bias is zero, except in the skewed workload where
   memory 0 gets +2;
 * varlen workloads draw sequence lengths U{512..2048} until the packed batch
-  reaches the token budget, the last length clipped to the remainder.
+  reaches the token budget, the last length clipped to the remainder;
+* with per-memory gates, each routed memory's W_beta, W_a ~ N(0, 1/d_model),
+  A ~ U(0, 2.7), b_a ~ U(-4, 0), from a stream of their own.
 
 Storage layout of every projection weight is [out_features, in_features]
 (y = x @ W.T).  In bf16 workloads every array that the kernels read as bf16
@@ -48,6 +50,7 @@ class Workload:
     varlen_max: int = 2048
     decode_steps: int = 0       # >0: recurrent decode workload
     prefill_len: int = 0
+    mem_gates: bool = False     # every routed memory has its own W_beta, W_a, A, b_a
 
     @property
     def n_tokens(self) -> int:
@@ -131,6 +134,14 @@ def make_weights(w: Workload, rng: np.random.Generator,
     p["b_a"] = rng.uniform(-4.0, 0.0, size=w.heads).astype(np.float32)
     p["w_k"] = lin(w.n_mem, Hd, D)
     p["w_v"] = lin(w.n_mem, Hd, D)
+    if w.mem_gates:
+        # drawn from their own stream, so the other weights and the tokens are
+        # those of the same workload without per-memory gates
+        g = np.random.default_rng((w.seed, 1))
+        p["w_beta_mem"] = _act(g.standard_normal((w.n_mem, w.heads, D), dtype=np.float32) * std, w.dtype)
+        p["w_a_mem"] = _act(g.standard_normal((w.n_mem, w.heads, D), dtype=np.float32) * std, w.dtype)
+        p["A_mem"] = g.uniform(0.0, 2.7, size=(w.n_mem, w.heads)).astype(np.float32)
+        p["b_a_mem"] = g.uniform(-4.0, 0.0, size=(w.n_mem, w.heads)).astype(np.float32)
     return p
 
 

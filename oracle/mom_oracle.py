@@ -44,8 +44,10 @@ delta correction) is available wherever the rule can be chosen:
     S_t = alpha_t * S_{t-1} + beta_t v_t k_t^T,      o_t = S_t (scale * q_t).
 
 Readings where the pages are silent (each also listed in the design notes):
-q, beta and alpha are shared by all memories (one W_q, W_beta, W_a); every
-memory, the shared one included, has its own W_k, W_v; a memory's state is
+q, beta and alpha are shared by all memories (one W_q, W_beta, W_a) unless
+the layer has per-memory gates (then each routed memory has its own W_beta,
+W_a, A, b_a: memory_gates); every memory, the shared one included, has its
+own W_k, W_v; a memory's state is
 neither decayed nor updated on tokens not routed to it; the shared memory
 enters the combine with weight 1; top-k is taken on logits with ties going
 to the lower memory index; q and k are L2-normalised per head as
@@ -193,6 +195,23 @@ def memory_kv(x_rows, p, m: int, H: int, d: int):
     return k, v
 
 
+def memory_gates(x_rows, p, m: int):
+    """Memory m's own gates of the rows routed to it, when the layer has
+    per-memory gates (p holds w_beta_mem, w_a_mem [M,H,d_model], A_mem,
+    b_a_mem [M,H]): beta = sigmoid(x W_beta^m), log alpha = -exp(A^m)
+    softplus(x W_a^m + b_a^m).  Without them every memory uses the shared
+    gates of shared_projections."""
+    x_rows = np.asarray(x_rows, F64)
+    beta = sigmoid(x_rows @ np.asarray(p["w_beta_mem"][m], F64).T)
+    a_in = x_rows @ np.asarray(p["w_a_mem"][m], F64).T + np.asarray(p["b_a_mem"][m], F64)
+    log_alpha = -np.exp(np.asarray(p["A_mem"][m], F64)) * softplus(a_in)
+    return beta, log_alpha
+
+
+def has_memory_gates(p) -> bool:
+    return "w_beta_mem" in p
+
+
 # ----------------------------------------------------------------------------
 # Gated DeltaNet recurrence  ([blog] experiments: "Gated DeltaNet gate and
 # update rule" per memory; [sdm] gated delta update as a form check)
@@ -336,7 +355,8 @@ def mom_forward(x, p, cu_seqlens, top_k: int, H: int, d: int, scale: float = 1.0
                 h_mem[m, s] = 0.0 if h0 is None else h0
                 continue
             k_m, v_m = memory_kv(x[rows], p, m, H, d)
-            o_m, h_mem[m, s] = gdn_recurrence(q[rows], k_m, v_m, beta[rows], log_alpha[rows], h0, scale, rule)
+            b_m, la_m = memory_gates(x[rows], p, m) if has_memory_gates(p) else (beta[rows], log_alpha[rows])
+            o_m, h_mem[m, s] = gdn_recurrence(q[rows], k_m, v_m, b_m, la_m, h0, scale, rule)
             slot = np.argmax(idx[rows] == m, axis=1)
             o_mem[rows, slot] = o_m
     # combine: shared memory with weight 1 plus the router-weighted memories
@@ -373,7 +393,8 @@ def mom_forward_mixed_state(x, p, cu_seqlens, top_k: int, H: int, d: int, scale:
             for j in range(top_k):
                 m = int(idx[t, j])
                 k_m, v_m = memory_kv(x[t:t + 1], p, m, H, d)
-                _, states[m] = RULES[rule](states[m], q[t], k_m[0], v_m[0], beta[t], log_alpha[t])
+                b_m, la_m = memory_gates(x[t:t + 1], p, m) if has_memory_gates(p) else (beta[t:t + 1], log_alpha[t:t + 1])
+                _, states[m] = RULES[rule](states[m], q[t], k_m[0], v_m[0], b_m[0], la_m[0])
             mixed = states[M] + sum(gate[t, j] * states[int(idx[t, j])] for j in range(top_k))
             out[t] = np.einsum("hvk,hk->hv", mixed, scale * q[t])
     return out
@@ -416,6 +437,7 @@ def mom_decode_step(x, p, state, top_k: int, H: int, d: int, scale: float = 1.0,
         for j in range(top_k):
             m = int(idx[b, j])
             k_m, v_m = memory_kv(x[b:b + 1], p, m, H, d)
-            o_m, new[b, m] = RULES[rule](new[b, m], q[b], k_m[0], v_m[0], beta[b], log_alpha[b], scale)
+            b_m, la_m = memory_gates(x[b:b + 1], p, m) if has_memory_gates(p) else (beta[b:b + 1], log_alpha[b:b + 1])
+            o_m, new[b, m] = RULES[rule](new[b, m], q[b], k_m[0], v_m[0], b_m[0], la_m[0], scale)
             out[b] += gate[b, j] * o_m
     return out, new, idx, gate, near_tie
