@@ -241,6 +241,27 @@ mom_status mom_gate_proj(const void* x, const void* w_gate, const float* A, cons
                          int64_t n_tok, int d_model, int H, float* beta, float* log_alpha,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* mom_mem_gate_proj -- per-memory gates of the routed rows: memory m keeps
+ * its own W_beta^m, W_a^m, A^m, b_a^m (paper card, Summary: every memory has
+ * its own recurrent update; the blog post's memories are Gated DeltaNet
+ * layers, gates included).  For routed row r of memory m (mem_offset[m] <=
+ * r < mem_offset[m+1]) and token t = perm_token[r]:
+ *   beta_p[r]      = sigmoid(x[t] W_beta^m^T)
+ *   log_alpha_p[r] = -exp(A^m) * softplus(x[t] W_a^m^T + b_a^m)
+ * x [n_tok, d_model] (dt); perm_token, mem_offset as mom_permute writes
+ * them (n_tok*top_k rows in memory order); w_gate_mem [n_mem, 2*H, d_model]
+ * (dt) = rows W_beta^m | W_a^m per memory; A_mem, b_a_mem [n_mem, H]
+ * float32.  Outputs beta_p, log_alpha_p [n_tok*top_k, H] float32, for the
+ * memory calls with MOM_GATES_BY_ROW.  float32 accumulation (bf16 inputs on
+ * the tensor cores).  A row that no memory holds or whose token is out of
+ * range is recorded (MOM_DEVERR_ROW_INDEX) and gets beta = log_alpha = 0.
+ * Requires 1 <= top_k <= n_mem <= MOM_MAX_MEM, d_model % 8 == 0.
+ * ws: at least MOM_WS_HEADER_BYTES. */
+mom_status mom_mem_gate_proj(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
+                             const void* w_gate_mem, const float* A_mem, const float* b_a_mem, mom_dtype dt,
+                             int64_t n_tok, int d_model, int H, int n_mem, int top_k,
+                             float* beta_p, float* log_alpha_p, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * mom_gdn_chunk_fwd -- the Gated DeltaNet recurrence of one memory over
  * each segment (blog post, experiments section: every memory uses Gated
@@ -298,25 +319,32 @@ mom_status mom_gdn_chunk_state(const void* q, const int32_t* qidx, const void* k
                                const float* h0, float* h_final, void* o,
                                void* ws, size_t ws_bytes, void* stream);
 
-/* The same three calls for either memory rule (MOM_RULE_*); the mom_gdn_*
- * calls are these with MOM_RULE_GATED_DELTA.  Same arguments otherwise, same
- * workspace (mom_gdn_workspace_size); MOM_ERR_ARG for an unknown rule. */
+/* The same three calls for either memory rule (MOM_RULE_*) and either gate
+ * layout (MOM_GATES_*); the mom_gdn_* calls are these with
+ * MOM_RULE_GATED_DELTA and MOM_GATES_BY_TOKEN.  Same arguments otherwise,
+ * same workspace (mom_gdn_workspace_size); MOM_ERR_ARG for an unknown rule
+ * or layout.  With MOM_GATES_BY_ROW, beta and log_alpha are [n_rows, H]:
+ * row r's own gates (the per-memory gates mom_mem_gate_proj writes), read at
+ * row r whether or not qidx is given. */
+typedef int mom_gates;
+#define MOM_GATES_BY_TOKEN  0   /* beta, log_alpha [n_q_rows, H], read like q */
+#define MOM_GATES_BY_ROW    1   /* beta, log_alpha [n_rows, H], one per row of k, v */
 mom_status mom_memory_chunk_fwd(const void* q, const int32_t* qidx, const void* k, const void* v,
                                 const float* beta, const float* log_alpha,
                                 const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
-                                int H, int d, float scale, mom_dtype dt, mom_rule rule,
+                                int H, int d, float scale, mom_dtype dt, mom_rule rule, mom_gates gates,
                                 const float* h0, float* h_final, void* o,
                                 void* ws, size_t ws_bytes, void* stream);
 mom_status mom_memory_chunk_prep(const void* q, const int32_t* qidx, const void* k, const void* v,
                                  const float* beta, const float* log_alpha,
                                  const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
-                                 int H, int d, float scale, mom_dtype dt, mom_rule rule,
+                                 int H, int d, float scale, mom_dtype dt, mom_rule rule, mom_gates gates,
                                  const float* h0, float* h_final, void* o,
                                  void* ws, size_t ws_bytes, void* stream);
 mom_status mom_memory_chunk_state(const void* q, const int32_t* qidx, const void* k, const void* v,
                                   const float* beta, const float* log_alpha,
                                   const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
-                                  int H, int d, float scale, mom_dtype dt, mom_rule rule,
+                                  int H, int d, float scale, mom_dtype dt, mom_rule rule, mom_gates gates,
                                   const float* h0, float* h_final, void* o,
                                   void* ws, size_t ws_bytes, void* stream);
 
@@ -368,9 +396,21 @@ mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_mod
                            int n_mem, int top_k, float scale, mom_dtype dt,
                            float* state, void* out, int32_t* topk_idx,
                            void* ws, size_t ws_bytes, void* stream);
-/* mom_decode_step for either memory rule (MOM_RULE_*); mom_decode_step is
- * this with MOM_RULE_GATED_DELTA. */
-mom_status mom_decode_step_rule(const void* x, const mom_weights* w, int B, int d_model, int H, int d,
+/* Per-memory gates for mom_decode_step_rule (device pointers, as in
+ * mom_mem_gate_proj). */
+typedef struct mom_memory_gates {
+    const void*  w_gate_mem;  /* [n_mem, 2*H, d_model]: rows W_beta^m | W_a^m */
+    const float* A_mem;       /* [n_mem, H] */
+    const float* b_a_mem;     /* [n_mem, H] */
+} mom_memory_gates;
+
+/* mom_decode_step for either memory rule (MOM_RULE_*), and with per-memory
+ * gates when `mg` (a HOST pointer, read during the call only) is non-NULL:
+ * each routed slot then takes its memory's own beta and alpha, the shared
+ * slot the layer's.  mom_decode_step is this with MOM_RULE_GATED_DELTA and
+ * mg = NULL.  Same workspace. */
+mom_status mom_decode_step_rule(const void* x, const mom_weights* w, const mom_memory_gates* mg,
+                                int B, int d_model, int H, int d,
                                 int n_mem, int top_k, float scale, mom_dtype dt, mom_rule rule,
                                 float* state, void* out, int32_t* topk_idx,
                                 void* ws, size_t ws_bytes, void* stream);

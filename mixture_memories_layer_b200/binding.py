@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+from typing import Optional
 from ctypes import POINTER, c_char_p, c_float, c_int, c_int32, c_int64, c_size_t, c_void_p
 
 import torch
@@ -46,16 +47,18 @@ SIGNATURES = {
                                _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mom_gdn_chunk_state": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I,
                                _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "mom_memory_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I,
+    "mom_memory_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I, _I,
                                   _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "mom_memory_chunk_prep": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I,
+    "mom_memory_chunk_prep": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I, _I,
                                    _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "mom_memory_chunk_state": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I,
+    "mom_memory_chunk_state": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I, _I,
                                     _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mom_combine_unpermute": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
     "mom_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "mom_decode_step": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "mom_decode_step_rule": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_decode_step_rule": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP, _VP, _SZ,
+                                  _VP]),
+    "mom_mem_gate_proj": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
 }
 
 
@@ -63,6 +66,11 @@ class MomWeights(ctypes.Structure):
     """Mirror of ``struct mom_weights`` (device pointers)."""
     _fields_ = [("w_r", c_void_p), ("b_r", c_void_p), ("w_shared", c_void_p), ("w_gate", c_void_p),
                 ("A", c_void_p), ("b_a", c_void_p), ("w_kv", c_void_p)]
+
+
+class MomMemoryGates(ctypes.Structure):
+    """Mirror of ``struct mom_memory_gates`` (device pointers)."""
+    _fields_ = [("w_gate_mem", c_void_p), ("A_mem", c_void_p), ("b_a_mem", c_void_p)]
 
 
 def _load():
@@ -203,6 +211,16 @@ def mom_gate_proj(x, w_gate, A, b_a, beta, log_alpha, ws, stream=None):
                              _p(beta), _p(log_alpha), _p(ws), ws.numel(), _s(stream)), "mom_gate_proj")
 
 
+def mom_mem_gate_proj(x, perm, mem_offset, w_gate_mem, A_mem, b_a_mem, top_k, beta_p, log_alpha_p, ws,
+                      stream=None):
+    """Per-memory gates of the routed rows: beta_p, log_alpha_p [n_tok*top_k, H]."""
+    n_tok, d_model = x.shape
+    n_mem, H = A_mem.shape
+    _check(lib.mom_mem_gate_proj(_p(x), _p(perm), _p(mem_offset), _p(w_gate_mem), _p(A_mem), _p(b_a_mem),
+                                 dtype_code(x.dtype), n_tok, d_model, H, n_mem, top_k, _p(beta_p),
+                                 _p(log_alpha_p), _p(ws), ws.numel(), _s(stream)), "mom_mem_gate_proj")
+
+
 def mom_gdn_workspace_size(n_rows, n_seg, H, d, dt):
     return lib.mom_gdn_workspace_size(n_rows, n_seg, H, d, dt)
 
@@ -229,27 +247,33 @@ def mom_gdn_chunk_state(q, qidx, k, v, beta, log_alpha, seg_cu, scale, h0, h_fin
 
 MOM_RULE_GATED_DELTA, MOM_RULE_GATED_LINEAR = 0, 1
 RULES = {"gated_delta": MOM_RULE_GATED_DELTA, "gated_linear": MOM_RULE_GATED_LINEAR}
+MOM_GATES_BY_TOKEN, MOM_GATES_BY_ROW = 0, 1
 
 
-def _memory(name, q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream):
+def _memory(name, q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream, gates):
     n_rows, H, d = k.shape
     _check(getattr(lib, name)(_p(q), _p(qidx), _p(k), _p(v), _p(beta), _p(log_alpha), _p(seg_cu),
                               seg_cu.numel() - 1, n_rows, q.shape[0], H, d, float(scale),
-                              dtype_code(k.dtype), int(rule), _p(h0), _p(h_final), _p(o), _p(ws), ws.numel(),
-                              _s(stream)), name)
+                              dtype_code(k.dtype), int(rule), int(gates), _p(h0), _p(h_final), _p(o), _p(ws),
+                              ws.numel(), _s(stream)), name)
 
 
-def mom_memory_chunk_fwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None):
-    _memory("mom_memory_chunk_fwd", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream)
+def mom_memory_chunk_fwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None,
+                         gates=MOM_GATES_BY_TOKEN):
+    _memory("mom_memory_chunk_fwd", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream,
+            gates)
 
 
-def mom_memory_chunk_prep(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None):
-    _memory("mom_memory_chunk_prep", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream)
+def mom_memory_chunk_prep(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None,
+                          gates=MOM_GATES_BY_TOKEN):
+    _memory("mom_memory_chunk_prep", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream,
+            gates)
 
 
-def mom_memory_chunk_state(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None):
-    _memory("mom_memory_chunk_state", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws,
-            stream)
+def mom_memory_chunk_state(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream=None,
+                           gates=MOM_GATES_BY_TOKEN):
+    _memory("mom_memory_chunk_state", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream,
+            gates)
 
 
 def mom_combine_unpermute(o_sh, o_p, row_of, topk_gate, out, ws, stream=None):
@@ -272,8 +296,9 @@ def mom_decode_step(x, weights: MomWeights, H, d, n_mem, top_k, scale, state, ou
 
 
 def mom_decode_step_rule(x, weights: MomWeights, H, d, n_mem, top_k, scale, rule, state, out, topk_idx, ws,
-                         stream=None):
+                         stream=None, mem_gates: Optional[MomMemoryGates] = None):
     B, d_model = x.shape
-    _check(lib.mom_decode_step_rule(_p(x), ctypes.byref(weights), B, d_model, H, d, n_mem, top_k, float(scale),
+    mg = ctypes.byref(mem_gates) if mem_gates is not None else None
+    _check(lib.mom_decode_step_rule(_p(x), ctypes.byref(weights), mg, B, d_model, H, d, n_mem, top_k, float(scale),
                                     dtype_code(x.dtype), int(rule), _p(state), _p(out), _p(topk_idx), _p(ws),
                                     ws.numel(), _s(stream)), "mom_decode_step_rule")

@@ -156,6 +156,23 @@ mom_status mom_gate_proj(const void* x, const void* w_gate, const float* A, cons
                                         as_stream(stream)));
 }
 
+mom_status mom_mem_gate_proj(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
+                             const void* w_gate_mem, const float* A_mem, const float* b_a_mem, mom_dtype dt,
+                             int64_t n_tok, int d_model, int H, int n_mem, int top_k,
+                             float* beta_p, float* log_alpha_p, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || d_model <= 0 || d_model % 8 != 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {x, perm_token, mem_offset, w_gate_mem, A_mem, b_a_mem, beta_p, log_alpha_p};
+    for (const void* p : ptrs)
+        if (!p) return MOM_ERR_ARG;
+    if (!al16(x) || !al16(w_gate_mem)) return MOM_ERR_ARG;
+    return cuda_status(launch_mem_gate_proj(x, perm_token, mem_offset, w_gate_mem, A_mem, b_a_mem, dt, n_tok,
+                                            n_tok * top_k, d_model, H, n_mem, beta_p, log_alpha_p, ws,
+                                            as_stream(stream)));
+}
+
 // --------------------------------------------------------- chunked GDN
 size_t mom_gdn_workspace_size(int64_t n_rows, int n_seg, int H, int d, mom_dtype dt) {
     size_t extra = (dt == MOM_BF16 && head_dim_ok(d)) ? gdn_tc_ws_bytes(n_rows, n_seg, H, d) : 0;
@@ -165,9 +182,11 @@ size_t mom_gdn_workspace_size(int64_t n_rows, int n_seg, int H, int d, mom_dtype
 static mom_status gdn_call(const void* q, const int32_t* qidx, const void* k, const void* v, const float* beta,
                            const float* log_alpha, const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
                            int H, int d, float scale, mom_dtype dt, const float* h0, float* h_final, void* o,
-                           void* ws, size_t ws_bytes, void* stream, int phase, int rule = MOM_RULE_GATED_DELTA) {
+                           void* ws, size_t ws_bytes, void* stream, int phase, int rule = MOM_RULE_GATED_DELTA,
+                           int gates = MOM_GATES_BY_TOKEN) {
     if (!dt_ok(dt) || n_seg < 0 || n_rows < 0 || n_q_rows < 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
     if (rule != MOM_RULE_GATED_DELTA && rule != MOM_RULE_GATED_LINEAR) return MOM_ERR_ARG;
+    if (gates != MOM_GATES_BY_TOKEN && gates != MOM_GATES_BY_ROW) return MOM_ERR_ARG;
     if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < mom_gdn_workspace_size(n_rows, n_seg, H, d, dt)) return MOM_ERR_ARG;
     if (n_seg == 0) return MOM_OK;
@@ -182,6 +201,7 @@ static mom_status gdn_call(const void* q, const int32_t* qidx, const void* k, co
               h0, h_final, o, ws, ws_bytes};
     a.phase = phase;
     a.rule = rule;
+    a.gates_by_row = gates == MOM_GATES_BY_ROW;
     cudaStream_t st = as_stream(stream);
     if (gdn_tc_supported(a, dt)) return cuda_status(launch_gdn_tc(a, st));
     return cuda_status(launch_gdn_recurrent(a, dt, st));
@@ -220,10 +240,10 @@ mom_status mom_gdn_chunk_state(const void* q, const int32_t* qidx, const void* k
 #define MOM_MEMORY_CALL(NAME, PHASE)                                                                       \
     mom_status NAME(const void* q, const int32_t* qidx, const void* k, const void* v, const float* beta,     \
                     const float* log_alpha, const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows, \
-                    int H, int d, float scale, mom_dtype dt, mom_rule rule, const float* h0, float* h_final,  \
-                    void* o, void* ws, size_t ws_bytes, void* stream) {                                      \
+                    int H, int d, float scale, mom_dtype dt, mom_rule rule, mom_gates gates, const float* h0, \
+                    float* h_final, void* o, void* ws, size_t ws_bytes, void* stream) {                      \
         return gdn_call(q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, dt, h0,  \
-                        h_final, o, ws, ws_bytes, stream, PHASE, rule);                                      \
+                        h_final, o, ws, ws_bytes, stream, PHASE, rule, gates);                               \
     }
 MOM_MEMORY_CALL(mom_memory_chunk_fwd, GDN_PREP | GDN_STATE)
 MOM_MEMORY_CALL(mom_memory_chunk_prep, GDN_PREP)
@@ -248,7 +268,8 @@ mom_status mom_combine_unpermute(const void* o_sh, const void* o_p, const int32_
 // ------------------------------------------------------------------ decode
 namespace {
 struct DecodeLayout {
-    size_t idx, gate, perm, row_of, mem_off, seg_cu, q, k_sh, v_sh, beta, la, k_p, v_p, perm_scratch, total;
+    size_t idx, gate, perm, row_of, mem_off, seg_cu, q, k_sh, v_sh, beta, la, beta_p, la_p, k_p, v_p, perm_scratch,
+        total;
 };
 DecodeLayout decode_layout(int B, int H, int d, int M, int K, int dt) {
     DecodeLayout L;
@@ -266,6 +287,8 @@ DecodeLayout decode_layout(int B, int H, int d, int M, int K, int dt) {
     L.v_sh = take((size_t)B * HD * esize(dt));
     L.beta = take((size_t)B * H * 4);
     L.la = take((size_t)B * H * 4);
+    L.beta_p = take(BK * H * 4);
+    L.la_p = take(BK * H * 4);
     L.k_p = take(BK * HD * esize(dt));
     L.v_p = take(BK * HD * esize(dt));
     L.perm_scratch = take(permute_scratch_bytes(B, M));
@@ -285,11 +308,12 @@ mom_status mom_decode_step(const void* x, const mom_weights* w, int B, int d_mod
                            int n_mem, int top_k, float scale, mom_dtype dt,
                            float* state, void* out, int32_t* topk_idx,
                            void* ws, size_t ws_bytes, void* stream) {
-    return mom_decode_step_rule(x, w, B, d_model, H, d, n_mem, top_k, scale, dt, MOM_RULE_GATED_DELTA, state, out,
-                                topk_idx, ws, ws_bytes, stream);
+    return mom_decode_step_rule(x, w, nullptr, B, d_model, H, d, n_mem, top_k, scale, dt, MOM_RULE_GATED_DELTA,
+                                state, out, topk_idx, ws, ws_bytes, stream);
 }
 
-mom_status mom_decode_step_rule(const void* x, const mom_weights* w, int B, int d_model, int H, int d,
+mom_status mom_decode_step_rule(const void* x, const mom_weights* w, const mom_memory_gates* mg,
+                                int B, int d_model, int H, int d,
                                 int n_mem, int top_k, float scale, mom_dtype dt, mom_rule rule,
                                 float* state, void* out, int32_t* topk_idx,
                                 void* ws, size_t ws_bytes, void* stream) {
@@ -302,6 +326,7 @@ mom_status mom_decode_step_rule(const void* x, const mom_weights* w, int B, int 
     const void* ptrs[] = {x, w->w_r, w->w_shared, w->w_gate, w->A, w->b_a, w->w_kv, state, out};
     for (const void* p : ptrs)
         if (!p || !al16(p)) return MOM_ERR_ARG;
+    if (mg && (!mg->w_gate_mem || !al16(mg->w_gate_mem) || !mg->A_mem || !mg->b_a_mem)) return MOM_ERR_ARG;
     cudaStream_t st = as_stream(stream);
     const DecodeLayout L = decode_layout(B, H, d, n_mem, top_k, dt);
     char* base = reinterpret_cast<char*>(ws);
@@ -328,6 +353,15 @@ mom_status mom_decode_step_rule(const void* x, const mom_weights* w, int B, int 
     DecodeArgs da{base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, beta, la, gate,
                   idx, row_of, B, H, d, n_mem, top_k, scale, state, out, ws};
     da.rule = rule;
+    if (mg) {
+        float* beta_p = reinterpret_cast<float*>(base + L.beta_p);
+        float* la_p = reinterpret_cast<float*>(base + L.la_p);
+        e = launch_mem_gate_proj(x, perm, mem_off, mg->w_gate_mem, mg->A_mem, mg->b_a_mem, dt, B, (int64_t)B * top_k,
+                                 d_model, H, n_mem, beta_p, la_p, ws, st);
+        if (e != cudaSuccess) return MOM_ERR_CUDA;
+        da.beta_p = beta_p;
+        da.log_alpha_p = la_p;
+    }
     return cuda_status(launch_decode_state(da, dt, st));
 }
 

@@ -8,7 +8,8 @@
 // written once:
 //   y = S k, z = S q (one pass over S), u = beta (v - alpha y),
 //   S' = alpha S + u k^T, o = scale (alpha z + u (k . q)),
-// (with the scalar-gated linear rule u = beta v: no delta correction)
+// (with the scalar-gated linear rule u = beta v: no delta correction; with
+// per-memory gates a routed slot takes its memory's own beta and alpha)
 //   out += w_slot * o   (w = router gate, 1 for the shared memory).
 // The state stream (read + write of (k+1) * d * d floats per sequence and
 // head) is the whole cost, so the kernel is written for HBM bandwidth:
@@ -33,9 +34,9 @@ decode_state_kernel(DecodeArgs a) {
 
     float qq[E];
     load_vec<E>(q + ((int64_t)b * H + h) * D + lane * E, qq);
-    const float be = a.beta[(int64_t)b * H + h];
-    const float al = expf(a.log_alpha[(int64_t)b * H + h]);
-    const float dl = a.rule == MOM_RULE_GATED_DELTA ? al : 0.f;
+    const float be_tok = a.beta[(int64_t)b * H + h];
+    const float la_tok = a.log_alpha[(int64_t)b * H + h];
+    const bool delta = a.rule == MOM_RULE_GATED_DELTA;
 
     float out_acc[RPW];
 #pragma unroll
@@ -63,6 +64,11 @@ decode_state_kernel(DecodeArgs a) {
             kb = reinterpret_cast<const T*>(a.k_sh);
             vb = reinterpret_cast<const T*>(a.v_sh);
         }
+        // the slot's gates: its memory's own for a routed slot when given
+        const bool own = j < K && a.beta_p;
+        const float be = own ? a.beta_p[r * H + h] : be_tok;
+        const float al = expf(own ? a.log_alpha_p[r * H + h] : la_tok);
+        const float dl = delta ? al : 0.f;
         float* Sp = a.state + ((((int64_t)b * (M + 1) + m) * H + h) * D + row0) * D + lane * E;
         float S[RPW][E];
 #pragma unroll

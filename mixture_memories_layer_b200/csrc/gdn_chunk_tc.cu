@@ -76,6 +76,7 @@ struct GdnTc {
     unsigned char* img;
     void* err;
     int delta;            // 1: the Gated DeltaNet rule; 0: the scalar-gated linear rule (L = 0, Y = V^T)
+    int gates_by_row;     // 1: beta / la [n_rows, H], one per row of k / v (per-memory gates)
 };
 
 // ------------------------------------------------------------- schedule --
@@ -131,7 +132,7 @@ gdn_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_seg, int64_t n_row
 
 // Gates of one chunk, by one full warp (lane l holds rows 2l and 2l+1):
 // beta (0 past n) and log alpha (0 past n), loaded from global memory
-// (through the row index when given).
+// (through the row index when given, unless the gates are per row).
 __device__ __forceinline__ void chunk_gates_load(const GdnTc& p, int64_t r0, int n, int h, int lane, float (&b)[2],
                                                  float (&l)[2]) {
 #pragma unroll
@@ -141,8 +142,8 @@ __device__ __forceinline__ void chunk_gates_load(const GdnTc& p, int64_t r0, int
         l[e] = 0.f;
         if (s < n) {
             const int64_t r = r0 + s;
-            const int64_t qr = p.qidx ? (int64_t)p.qidx[r] : r;
-            if (qr >= 0 && qr < p.n_q_rows) {
+            const int64_t qr = (p.qidx && !p.gates_by_row) ? (int64_t)p.qidx[r] : r;
+            if (qr >= 0 && qr < (p.gates_by_row ? p.n_rows : p.n_q_rows)) {
                 b[e] = p.beta[qr * p.H + h];
                 l[e] = p.la[qr * p.H + h];
             } else {
@@ -1224,6 +1225,7 @@ cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st) {
     t.img = base;
     t.err = a.ws;
     t.delta = a.rule == MOM_RULE_GATED_DELTA ? 1 : 0;
+    t.gates_by_row = a.gates_by_row;
     return a.d == 256 ? launch_d<256>(t, mc, a.phase, st) : launch_d<128>(t, mc, a.phase, st);
 }
 

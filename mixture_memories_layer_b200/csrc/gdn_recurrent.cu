@@ -64,8 +64,9 @@ gdn_recurrent_kernel(GdnArgs a) {
         load_vec<E>(q + (qr * H + h) * D + lane * E, qq);
 #pragma unroll
         for (int i = 0; i < RPW; ++i) vv[i] = to_f(v[(r * H + h) * D + row0 + i]);
-        const float b = a.beta[qr * H + h];
-        const float al = expf(a.log_alpha[qr * H + h]);
+        const int64_t gr = a.gates_by_row ? r : qr;
+        const float b = a.beta[gr * H + h];
+        const float al = expf(a.log_alpha[gr * H + h]);
 
         float red[2 * RPW + 1];
         red[2 * RPW] = 0.f;
@@ -82,7 +83,6 @@ gdn_recurrent_kernel(GdnArgs a) {
         warp_sum_n<2 * RPW + 1>(red);
         const float kq = red[2 * RPW];
         float my_o = 0.f;
-#pragma unroll
         const float dl = a.rule == MOM_RULE_GATED_DELTA ? al : 0.f;
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {

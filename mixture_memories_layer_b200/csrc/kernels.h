@@ -34,6 +34,10 @@ bool device_is_sm100();
 // router.cu
 cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int dt, int64_t n_tok, int D,
                           int M, int K, int32_t* idx, float* gate, float* logits, cudaStream_t st);
+// mem_gates.cu: per-memory gates of the routed rows (beta_p, log_alpha_p [n_rows, H])
+cudaError_t launch_mem_gate_proj(const void* x, const int32_t* perm, const int32_t* mem_offset, const void* w_gate_mem,
+                                 const float* A_mem, const float* b_a_mem, int dt, int64_t n_tok, int64_t n_rows, int D,
+                                 int H, int M, float* beta, float* log_alpha, void* err, cudaStream_t st);
 cudaError_t launch_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, int dt,
                              int64_t n_tok, int D, int H, float* beta, float* log_alpha, void* err, cudaStream_t st);
 
@@ -96,6 +100,9 @@ struct GdnArgs {
     int phase = GDN_PREP | GDN_STATE;
     // MOM_RULE_GATED_DELTA or MOM_RULE_GATED_LINEAR
     int rule = MOM_RULE_GATED_DELTA;
+    // 0: beta / log_alpha [n_q_rows, H], read through qidx like q; 1: one
+    // gate per row of k / v ([n_rows, H], the per-memory gates)
+    int gates_by_row = 0;
 };
 cudaError_t launch_gdn_recurrent(const GdnArgs& a, int dt, cudaStream_t st);
 
@@ -119,6 +126,9 @@ struct DecodeArgs {
     void* out;
     void* ws;
     int rule = MOM_RULE_GATED_DELTA;
+    // per-memory gates of the routed slots, [B*K, H] by reordered row (row_of),
+    // or null: every slot takes the token's beta / log_alpha
+    const float *beta_p = nullptr, *log_alpha_p = nullptr;
 };
 cudaError_t launch_decode_state(const DecodeArgs& a, int dt, cudaStream_t st);
 

@@ -23,10 +23,18 @@ from . import binding as B
 def pack_weights(p: Dict[str, np.ndarray], dtype: torch.dtype, device="cuda") -> Dict[str, torch.Tensor]:
     """Stack the per-projection weights into the layouts the library reads:
     w_shared = [W_q; W_k_sh; W_v_sh], w_gate = [W_beta; W_a],
-    w_kv[m] = [W_k^m; W_v^m] (all [out, in])."""
+    w_kv[m] = [W_k^m; W_v^m] (all [out, in]); with per-memory gates also
+    w_gate_mem[m] = [W_beta^m; W_a^m], A_mem, b_a_mem [M, H]."""
     t = lambda a, dt=dtype: torch.as_tensor(np.ascontiguousarray(a)).to(device=device, dtype=dt)
     M = p["w_k"].shape[0]
-    return dict(
+    mem_gates = {}
+    if "w_beta_mem" in p:
+        mem_gates = dict(
+            w_gate_mem=t(np.stack([np.concatenate([p["w_beta_mem"][m], p["w_a_mem"][m]], axis=0) for m in range(M)])),
+            A_mem=t(p["A_mem"], torch.float32),
+            b_a_mem=t(p["b_a_mem"], torch.float32),
+        )
+    return dict(**mem_gates,
         w_r=t(p["w_r"]),
         b_r=t(p["b_r"], torch.float32),
         w_shared=t(np.concatenate([p["w_q"], p["w_k_sh"], p["w_v_sh"]], axis=0)),
@@ -48,7 +56,9 @@ class MoMLayer:
         380M-shape layer 0.295 vs 0.308 ms, 1.3B-shape layer 0.904 vs
         0.963 ms.  rule: the memories' update rule, "gated_delta" (Gated
         DeltaNet, the default) or "gated_linear" (S_t = alpha_t S_{t-1} +
-        beta_t v_t k_t^T: linear attention, RetNet, Mamba2-style memories)."""
+        beta_t v_t k_t^T: linear attention, RetNet, Mamba2-style memories).
+        Weights that carry w_gate_mem / A_mem / b_a_mem (pack_weights of
+        per-memory gates) give every routed memory its own beta and alpha."""
         if rule not in B.RULES:
             raise ValueError("rule must be one of %s" % sorted(B.RULES))
         self.rule = B.RULES[rule]
@@ -63,6 +73,9 @@ class MoMLayer:
         self._bufs = {}
         self._c_weights = B.MomWeights(*[ctypes_ptr(weights[k]) for k in
                                          ("w_r", "b_r", "w_shared", "w_gate", "A", "b_a", "w_kv")])
+        self.mem_gates = "w_gate_mem" in weights
+        self._c_mem_gates = (B.MomMemoryGates(*[ctypes_ptr(weights[k]) for k in ("w_gate_mem", "A_mem", "b_a_mem")])
+                             if self.mem_gates else None)
 
     # -------------------------------------------------------------- buffers
     def _buf(self, name, shape, dtype):
@@ -97,6 +110,10 @@ class MoMLayer:
             h_shared=self._buf("h_shared", (n_seq, H, d, d), f32),
             h_mem=self._buf("h_mem", (M, n_seq, H, d, d), f32),
         )
+        if self.mem_gates:
+            b["beta_p"] = self._buf("beta_p", (n_tok * K, H), f32)
+            b["log_alpha_p"] = self._buf("log_alpha_p", (n_tok * K, H), f32)
+            b["ws_mem_gate"] = self._ws("mem_gate", B.MOM_WS_HEADER_BYTES)
         dtc = B.dtype_code(dt)
         b["ws_perm"] = self._ws("perm", B.mom_permute_workspace_size(n_tok, K, M, n_seq))
         b["ws_proj"] = self._ws("proj", B.mom_kv_proj_workspace_size(n_tok, self.d_model, H, d, M, K))
@@ -136,6 +153,14 @@ class MoMLayer:
         mark(1)
         B.mom_permute(b["idx"], self.n_mem, cu_seqlens, b["perm"], b["row_of"], b["mem_offset"], b["seg_cu"],
                       b["ws_perm"], stream=st)
+        if self.mem_gates:
+            # the routed rows' own gates, beside the projections
+            permuted = torch.cuda.Event()
+            permuted.record(st)
+            side.wait_event(permuted)
+            B.mom_mem_gate_proj(x, b["perm"], b["mem_offset"], w["w_gate_mem"], w["A_mem"], w["b_a_mem"],
+                                self.top_k, b["beta_p"], b["log_alpha_p"], b["ws_mem_gate"], stream=side)
+            gates_done.record(side)
         mark(2)
         B.mom_kv_proj_grouped(x, b["perm"], b["mem_offset"], w["w_shared"], None, None, None,
                               w["w_kv"], self.H, self.d, self.top_k, b["q"], b["k_sh"], b["v_sh"], None,
@@ -146,8 +171,14 @@ class MoMLayer:
         hm = b["h_mem"] if want_states else None
         gdn_sh = (b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens,
                   self.scale, self.rule, h0_shared, hs, b["o_sh"], b["ws_gdn_sh"])
-        gdn_p = (b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
-                 self.scale, self.rule, h0_mem, hm, b["o_p"], b["ws_gdn_p"])
+        if self.mem_gates:
+            gdn_p = (b["q"], b["perm"], b["k_p"], b["v_p"], b["beta_p"], b["log_alpha_p"], b["seg_cu"],
+                     self.scale, self.rule, h0_mem, hm, b["o_p"], b["ws_gdn_p"])
+            gates_p = B.MOM_GATES_BY_ROW
+        else:
+            gdn_p = (b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
+                     self.scale, self.rule, h0_mem, hm, b["o_p"], b["ws_gdn_p"])
+            gates_p = B.MOM_GATES_BY_TOKEN
         fork = torch.cuda.Event()
         if self.gdn_schedule == "phased":
             # both problems' state-independent chunk work first, on the whole
@@ -155,11 +186,11 @@ class MoMLayer:
             # (whole sequences: the longest chain) launched first so that its
             # CTAs hold SMs before the routed walks fill the rest
             B.mom_memory_chunk_prep(*gdn_sh, stream=st)
-            B.mom_memory_chunk_prep(*gdn_p, stream=st)
+            B.mom_memory_chunk_prep(*gdn_p, stream=st, gates=gates_p)
             fork.record(st)
             B.mom_memory_chunk_state(*gdn_sh, stream=st)
             side.wait_event(fork)
-            B.mom_memory_chunk_state(*gdn_p, stream=side)
+            B.mom_memory_chunk_state(*gdn_p, stream=side, gates=gates_p)
         else:
             # each problem's prep then walk on its own stream: the shared
             # problem on a high-priority stream (its CTAs are dispatched first,
@@ -171,8 +202,8 @@ class MoMLayer:
             side.wait_event(fork)
             B.mom_memory_chunk_prep(*gdn_sh, stream=hi)
             B.mom_memory_chunk_state(*gdn_sh, stream=hi)
-            B.mom_memory_chunk_prep(*gdn_p, stream=side)
-            B.mom_memory_chunk_state(*gdn_p, stream=side)
+            B.mom_memory_chunk_prep(*gdn_p, stream=side, gates=gates_p)
+            B.mom_memory_chunk_state(*gdn_p, stream=side, gates=gates_p)
             hi_done = torch.cuda.Event()
             hi_done.record(hi)
             st.wait_event(hi_done)
@@ -220,7 +251,7 @@ class MoMLayer:
         idx = self._buf("dec_idx", (Bn, self.top_k), torch.int32)
         ws = self._ws("decode", B.mom_decode_workspace_size(Bn, self.d_model, self.H, self.d, self.n_mem, self.top_k))
         B.mom_decode_step_rule(x, self._c_weights, self.H, self.d, self.n_mem, self.top_k, self.scale, self.rule,
-                               state, out, idx, ws, stream=stream)
+                               state, out, idx, ws, stream=stream, mem_gates=self._c_mem_gates)
         return out, idx
 
 
