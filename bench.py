@@ -41,10 +41,14 @@ METRIC = "MoM layer fwd tokens/s at 1 B200 and % of roofline; decode tokens/s"
 UNIT = "tokens/s"
 FWD = "mom380m"
 DEC = "decode_b256"
-# (workload, memory rule): the other forward workloads, and the 380M shape with
-# the scalar-gated linear memories
-EXTRA = (("tiny_fp32", "gated_delta"), ("mom380m_skew_varlen", "gated_delta"), ("mom1p3b_m16", "gated_delta"),
-         ("mom380m", "gated_linear"))
+# (workload, memory rule, per-memory gates): the other forward workloads, the
+# 380M shape with the scalar-gated linear memories, and with per-memory gates
+EXTRA = (("tiny_fp32", "gated_delta", False), ("mom380m_skew_varlen", "gated_delta", False),
+         ("mom1p3b_m16", "gated_delta", False), ("mom380m", "gated_linear", False), ("mom380m", "gated_delta", True))
+
+
+def extra_key(name, rule, mem_gates):
+    return name + ("" if rule == "gated_delta" else "_" + rule) + ("_mem_gates" if mem_gates else "")
 TIE_GAP = 1e-4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -279,12 +283,14 @@ def near_tie_tokens(x, w_r, b_r, top_k, gap=TIE_GAP):
     return int(((top[:, top_k - 1] - top[:, top_k]) < gap).sum().item())
 
 
-def config_bench(name, dev, steps, warmup, peaks, flush, rule="gated_delta"):
+def config_bench(name, dev, steps, warmup, peaks, flush, rule="gated_delta", mem_gates=False):
     """One of the other forward workloads, timed like the headline one."""
+    import dataclasses
+
     import torch
     from mixture_memories_layer_b200 import layer as L
     from mixture_memories_layer_b200 import synth
-    w = synth.WORKLOADS[name]
+    w = dataclasses.replace(synth.WORKLOADS[name], mem_gates=mem_gates)
     p = synth.make_problem(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     lay = L.MoMLayer(L.pack_weights(p, dt, dev), w.heads, w.d_head, w.top_k, rule=rule)
@@ -300,7 +306,7 @@ def config_bench(name, dev, steps, warmup, peaks, flush, rule="gated_delta"):
     ms = sum(step_ms) / steps
     S = int(cu.numel()) - 1
     rows = lay.buffers(w.n_tokens, S)["mem_offset"].cpu().tolist()
-    out = {"workload": workload_desc(w), "memory_rule": rule, "dtype": w.dtype, "tokens": w.n_tokens, "sequences": S,
+    out = {"workload": workload_desc(w), "memory_rule": rule, "per_memory_gates": mem_gates, "dtype": w.dtype, "tokens": w.n_tokens, "sequences": S,
            "ms_per_step": ms, "value": w.n_tokens / (ms / 1e3), "unit": UNIT, "per_call_ms": per_call,
            "routed_rows_per_memory": [b - a for a, b in zip(rows[:-1], rows[1:])],
            "near_tie_tokens": near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)}
@@ -385,8 +391,8 @@ def gpu_arm(args):
     decode = None if args.no_decode else decode_bench(args, dev, world, rank, max_over_ranks, barrier)
     configs = None
     if not args.no_configs and world == 1:
-        configs = {(name if rule == "gated_delta" else "%s_%s" % (name, rule)):
-                   config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule) for name, rule in EXTRA}
+        configs = {extra_key(name, rule, mg): config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule, mg)
+                   for name, rule, mg in EXTRA}
     clocks.__exit__(None, None, None)
     layer_roof["near_tie_tokens"] = near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)
     return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,

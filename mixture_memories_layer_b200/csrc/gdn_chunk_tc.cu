@@ -143,6 +143,9 @@ __device__ __forceinline__ void chunk_gates_load(const GdnTc& p, int64_t r0, int
         if (s < n) {
             const int64_t r = r0 + s;
             const int64_t qr = (p.qidx && !p.gates_by_row) ? (int64_t)p.qidx[r] : r;
+            // per-row gates leave the index unread here: pull its line into L1
+            // for the q-row gather, which looks it up next
+            if (p.gates_by_row && p.qidx) asm volatile("prefetch.global.L1 [%0];" ::"l"(p.qidx + r));
             if (qr >= 0 && qr < (p.gates_by_row ? p.n_rows : p.n_q_rows)) {
                 b[e] = p.beta[qr * p.H + h];
                 l[e] = p.la[qr * p.H + h];
@@ -191,26 +194,47 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h2);
 }
 
-// Gathers 64 rows x D of a bf16 [rows, H, D] array through an index (rows
-// past n and bad indices are zero-filled) into 128-byte-swizzled 64-column
-// slabs of `slab_stride` bytes; `nthreads` threads starting at `t0`.
-template <int D>
-__device__ __forceinline__ void gather_rows(const GdnTc& p, const bf16* base, int64_t r0, int n, int h,
-                                            uint32_t dst, uint32_t slab_stride, int t, int nthreads) {
-    for (int idx = t; idx < C * 8; idx += nthreads) {
-        const int row = idx >> 3, c8 = idx & 7;
-        int64_t src_row = -1;
-        if (row < n) {
-            const int64_t r = r0 + row;
-            const int64_t qr = p.qidx ? (int64_t)p.qidx[r] : r;
-            src_row = (qr >= 0 && qr < p.n_q_rows) ? qr : -1;
-        }
-        const bf16* src = base + ((src_row >= 0 ? src_row : 0) * p.H + h) * D + c8 * 8;
-        const uint32_t d0 = dst + row * 128 + ((c8 ^ (row & 7)) << 4);
+// Gathering 64 rows x D of a bf16 [rows, H, D] array through an index into
+// 128-byte-swizzled 64-column slabs, by NT threads (thread t: items t, t +
+// NT, ...; item = (row, 16-byte column chunk)), in two steps: the source
+// rows of a thread's items (-1 past n or for a bad index: zero-filled), then
+// the copies.  All index loads of a step are in flight together -- between
+// the copies' asm statements they would each wait a full round trip -- and a
+// caller can issue the first step a chunk ahead.
+template <int NT>
+struct GatherRows {
+    static constexpr int ITEMS = (C * 8 + NT - 1) / NT;
+    int32_t src[ITEMS];   // row indices fit: qidx is int32, and n_rows < 2^31 / C
+
+    __device__ __forceinline__ void rows(const GdnTc& p, int64_t r0, int n, int t) {
 #pragma unroll
-        for (int j = 0; j < D / 64; ++j) cp_async_16(d0 + j * slab_stride, src + j * 64, src_row >= 0 ? 16u : 0u);
+        for (int i = 0; i < ITEMS; ++i) {
+            const int idx = t + i * NT, row = idx >> 3;
+            src[i] = -1;
+            if (idx < C * 8 && row < n) {
+                const int64_t r = r0 + row;
+                const int64_t qr = p.qidx ? (int64_t)__ldg(p.qidx + r) : r;
+                src[i] = (qr >= 0 && qr < p.n_q_rows) ? (int32_t)qr : -1;
+            }
+        }
     }
-}
+
+    template <int D>
+    __device__ __forceinline__ void copy(const GdnTc& p, const bf16* base, int h, uint32_t dst, uint32_t slab_stride,
+                                         int t) const {
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            const int idx = t + i * NT;
+            if (idx < C * 8) {
+                const int row = idx >> 3, c8 = idx & 7;
+                const bf16* s = base + ((int64_t)(src[i] >= 0 ? src[i] : 0) * p.H + h) * D + c8 * 8;
+                const uint32_t d0 = dst + row * 128 + ((c8 ^ (row & 7)) << 4);
+#pragma unroll
+                for (int j = 0; j < D / 64; ++j) cp_async_16(d0 + j * slab_stride, s + j * 64, src[i] >= 0 ? 16u : 0u);
+            }
+        }
+    }
+};
 
 // ----------------------------------------------------------------- prep --
 // The prep computes, per (chunk, head), everything the serial walk needs
@@ -429,7 +453,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         gbeta[2 * lane] = b[0]; gbeta[2 * lane + 1] = b[1];
         g2[2 * lane] = gg[0] * LOG2E_; g2[2 * lane + 1] = gg[1] * LOG2E_;
     } else if (p.qidx && warp >= 2) {
-        gather_rows<D>(p, p.q, r0, n, h, kq + 8192, 16384, tid - 64, PREP_THREADS - 64);
+        GatherRows<PREP_THREADS - 64> g;
+        g.rows(p, r0, n, tid - 64);
+        g.copy<D>(p, p.q, h, kq + 8192, 16384, tid - 64);
         cp_async_commit();
         cp_async_wait<0>();
         fence_proxy_async_smem();
@@ -1071,21 +1097,26 @@ gdn_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         // ------------------- q~ warps: q rows (through the index when given),
         // then scaled in place by e^gamma_r / rho (the output's state term)
         const int t = threadIdx.x - (W_PROD + 1) * 32;
+        // the source rows of chunk c + 1 are looked up while chunk c is scaled
+        GatherRows<NGATHER * 32> g;
+        g.rows(p, rs0, (int)(rs1 - rs0 < C ? rs1 - rs0 : C), t);
         for (int c = 0; c < nc; ++c) {
             const int b = c & 1;
             const uint32_t pb = (c >> 1) & 1;
             const uint32_t qb = kq0 + b * Lay::KQSZ + 8192;
             const int64_t r0 = rs0 + (int64_t)c * C;
-            const int64_t rem = rs1 - r0;
-            const int n = (int)(rem < C ? rem : C);
             if (!mbar_wait(bar(KQ_FREE + b), pb ^ 1, abort_flag, p.err, 38)) break;
-            gather_rows<D>(p, p.q, r0, n, h, qb, 16384, t, NGATHER * 32);
+            g.copy<D>(p, p.q, h, qb, 16384, t);
             cp_async_commit();
+            if (c + 1 < nc) {
+                const int64_t rem1 = rs1 - (r0 + C);
+                g.rows(p, r0 + C, (int)(rem1 < C ? rem1 : C), t);
+            }
             const bool gates = mbar_wait(bar(GB_FULL + b), pb, abort_flag, p.err, 39);
             cp_async_wait<0>();
             if (!gates) break;
             const float* gb = gbuf + b * GB;
-            // the same (row, chunk) assignment as gather_rows: each thread scales what it fetched
+            // the same (row, chunk) assignment as the gather: each thread scales what it fetched
             for (int idx = t; idx < C * 8; idx += NGATHER * 32) {
                 const int row = idx >> 3, c8 = idx & 7;
                 const float f = gb[G_EGR + row];

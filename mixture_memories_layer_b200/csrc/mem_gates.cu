@@ -61,6 +61,25 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
     return v;
 }
 
+constexpr int MG_G = 2;        // 64-feature blocks per load group
+
+// x features [fb, fb + 64 * MG_G) of the lane's two rows (blocks past D: not loaded)
+__device__ __forceinline__ void load_group(const bf16* x0, const bf16* x1, int fb, int D, uint4 (&v)[MG_G][2][2]) {
+#pragma unroll
+    for (int j = 0; j < MG_G; ++j) {
+        if (fb + 64 * j < D) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                v[j][h][0] = ld_stream_u4(x0 + fb + 64 * j + 32 * h);
+                v[j][h][1] = ld_stream_u4(x1 + fb + 64 * j + 32 * h);
+            }
+        } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) v[j][h][0] = v[j][h][1] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
 // Memory of routed row r (mem_offset in shared memory), or -1 when no memory
 // holds it.
 __device__ __forceinline__ int memory_of(const int* off, int M, int64_t r) {
@@ -132,21 +151,35 @@ mem_gate_mma_kernel(MemGateArgs a) {
         for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int n = 0; n < NT; ++n) acc[h][n][0] = acc[h][n][1] = acc[h][n][2] = acc[h][n][3] = 0.f;
-#pragma unroll(NT >= 4 ? 1 : 4)
-        for (int fb = 0; fb < D; fb += 64) {
+        // x in groups of MG_G 64-feature blocks, double-buffered: the next
+        // group's loads are issued before this group's products, so each
+        // round trip overlaps the previous group's MMAs (loads and MMAs are
+        // asm statements, kept in source order)
+        uint4 cur[MG_G][2][2], nxt[MG_G][2][2];
+        load_group(x0, x1, 0, D, cur);
+        for (int fb = 0; fb < D; fb += 64 * MG_G) {
+            if (fb + 64 * MG_G < D) load_group(x0, x1, fb + 64 * MG_G, D, nxt);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 xa = ld_stream_u4(x0 + fb + 32 * h);
-                const uint4 xb = ld_stream_u4(x1 + fb + 32 * h);
+            for (int j = 0; j < MG_G; ++j) {
+                if (fb + 64 * j >= D) break;
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const int row = n * 8 + g;
-                    const uint4 wv = row < ncol ? __ldg(reinterpret_cast<const uint4*>(wm + (size_t)row * D + fb + 32 * h))
-                                                : make_uint4(0, 0, 0, 0);
-                    mma_bf16_16816(acc[h][n], xa.x, xb.x, xa.y, xb.y, wv.x, wv.y);
-                    mma_bf16_16816(acc[h][n], xa.z, xb.z, xa.w, xb.w, wv.z, wv.w);
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        const int row = n * 8 + g;
+                        const uint4 wv = row < ncol
+                            ? __ldg(reinterpret_cast<const uint4*>(wm + (size_t)row * D + fb + 64 * j + 32 * h))
+                            : make_uint4(0, 0, 0, 0);
+                        const uint4 xa = cur[j][h][0], xb = cur[j][h][1];
+                        mma_bf16_16816(acc[h][n], xa.x, xb.x, xa.y, xb.y, wv.x, wv.y);
+                        mma_bf16_16816(acc[h][n], xa.z, xb.z, xa.w, xb.w, wv.z, wv.w);
+                    }
                 }
             }
+#pragma unroll
+            for (int j = 0; j < MG_G; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) { cur[j][h][0] = nxt[j][h][0]; cur[j][h][1] = nxt[j][h][1]; }
         }
         // acc[.][n]: (row g: cols n*8 + 2c, +1; row g + 8: the same cols)
 #pragma unroll
