@@ -503,9 +503,13 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (warp == 1) tmem_dealloc(tmem, Lay::TMEM_COLS);
         return;
     }
-    // L = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r < n) into the L tile:
-    // TMEM lanes 0..63 are the K rows of G, 32 columns per thread
-    if (quarter < 2) {
+    // L = beta_r e^(gamma_r - gamma_s) k_r.k_s (s < r < n) into the L tile
+    // from TMEM lanes 0..63 (the K rows of G), 32 columns per thread -- the
+    // quadrant above the diagonal (warp 4) is never read -- while the warps
+    // of lanes 64..127 (the q rows) form P = e^(gamma_r - gamma_s) q_r.k_s
+    // (s <= r < n) in registers, written out once T's bytes are free.
+    uint32_t pk[16];
+    if (quarter < 2 && warp != 4) {
         uint32_t gv[32];
         tmem_ld_x32(tmem + lane_base + 32 * colh, gv);
         tmem_ld_wait();
@@ -517,13 +521,27 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int s = 32 * colh + e;
             Lm.at(r, s) = s < r ? br * ex2_approx(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
         }
+    } else if (quarter >= 2) {
+        uint32_t gv[32];
+        tmem_ld_x32(tmem + lane_base + 32 * colh, gv);
+        tmem_ld_wait();
+        const int r = rho - 64;
+        const float g2r = g2[r];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const int s = 32 * colh + e;
+            const float p0 = (s <= r && r < n) ? ex2_approx(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
+            const float p1 = (s + 1 <= r && r < n) ? ex2_approx(g2r - g2[s + 1]) * __uint_as_float(gv[e + 1]) : 0.f;
+            pk[e / 2] = pack_bf16(p0, p1);
+        }
     }
-    __syncthreads();
-
-    // T = (I + L)^-1 in 16 x 16 blocks.  Diagonal blocks: forward substitution,
-    // one column per thread.
-    if (tid < 64) {
-        const int bk = tid >> 4, cc = tid & 15, base = 16 * bk;
+    // T = (I + L)^-1 in 16 x 16 blocks.  Diagonal blocks: forward
+    // substitution, one column per thread, by the two warps whose L quadrants
+    // hold them (warp 0: blocks 0 and 1, warp 5: blocks 2 and 3), as soon as
+    // their own rows are written.
+    if (warp == 0 || warp == 5) {
+        __syncwarp();
+        const int bk = (warp == 5 ? 2 : 0) + (lane >> 4), cc = lane & 15, base = 16 * bk;
         float t[16];
 #pragma unroll
         for (int rl = 0; rl < 16; ++rl) t[rl] = rl == cc ? 1.f : 0.f;
@@ -562,23 +580,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int e = 0; e < 16; ++e) v[e] *= dec;
         image_chunks<2>(tdimg, r, 2 * q4, v);
     }
-    // P = e^(gamma_r - gamma_s) q_r.k_s (s <= r < n) from TMEM lanes 64..127
-    // (the q rows of G), then over T's first half once T is read
-    uint32_t pk[16];
-    if (quarter >= 2) {
-        uint32_t gv[32];
-        tmem_ld_x32(tmem + lane_base + 32 * colh, gv);
-        tmem_ld_wait();
-        const int r = rho - 64;
-        const float g2r = g2[r];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-            const int s = 32 * colh + e;
-            const float p0 = (s <= r && r < n) ? ex2_approx(g2r - g2[s]) * __uint_as_float(gv[e]) : 0.f;
-            const float p1 = (s + 1 <= r && r < n) ? ex2_approx(g2r - g2[s + 1]) * __uint_as_float(gv[e + 1]) : 0.f;
-            pk[e / 2] = pack_bf16(p0, p1);
-        }
-    }
+    // P over T's first half once T is read
     __syncthreads();
     if (quarter >= 2) {
         const int r = rho - 64;
