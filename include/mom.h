@@ -229,6 +229,42 @@ mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const i
                                void* q, void* k_sh, void* v_sh, float* beta, float* log_alpha,
                                void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream);
 
+/* mom_proj_shared -- the shared projections of mom_kv_proj_grouped alone
+ * (q, k_sh, v_sh), which need no routing: a memory-parallel layer runs them
+ * on the tokens' own rank.  Arguments as in mom_kv_proj_grouped.
+ * ws: mom_kv_proj_workspace_size(n_tok, d_model, H, d, 1, 1). */
+mom_status mom_proj_shared(const void* x, const void* w_shared, mom_dtype dt, int64_t n_tok, int d_model,
+                           int H, int d, void* q, void* k_sh, void* v_sh, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_kv_proj_groups -- the routed key/value projections over an explicit
+ * group table: the rows a memory-parallel layer receives, grouped by
+ * (source rank, memory) (explainer, "Memory count scaling": memories spread
+ * over GPUs).  Group g covers rows group_offset[g] .. group_offset[g+1]-1
+ * (non-decreasing, group_offset[n_groups] <= n_rows) and uses memory
+ * group_mem[g]'s weights (0 <= group_mem[g] < n_mem):
+ *   k_p[r] = l2norm_h(x[perm_token[r]] W_k^m^T),  v_p[r] = x[perm_token[r]] W_v^m^T
+ * with perm_token NULL meaning row r reads x row r.  x [n_x, d_model];
+ * w_kv [n_mem, 2*H*d, d_model]; k_p, v_p [n_rows, H, d] (dt); rows past
+ * group_offset[n_groups] are not written.  A corrupt table or index is
+ * recorded in ws (MOM_DEVERR_*) and the affected tiles are skipped.
+ * ws: at least MOM_WS_HEADER_BYTES. */
+mom_status mom_kv_proj_groups(const void* x, int64_t n_x, const int32_t* perm_token, int64_t n_rows,
+                              const int32_t* group_offset, const int32_t* group_mem, int n_groups,
+                              const void* w_kv, mom_dtype dt, int d_model, int H, int d, int n_mem,
+                              void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_copy_rows -- row copies in 16-byte granules, for packing the routed
+ * rows a memory-parallel layer sends to the owners of their memories and
+ * unpacking what it receives:
+ *   dst[i*dst_stride + dst_off .. + row_bytes) = src[s*src_stride + src_off .. + row_bytes)
+ * for i < n_rows, s = idx[i] (idx NULL: s = i).  Byte strides and offsets
+ * and row_bytes are multiples of 16; src and dst 16-byte aligned.  An index
+ * outside [0, n_src) is recorded (MOM_DEVERR_ROW_INDEX) and its row
+ * zero-filled.  ws: at least MOM_WS_HEADER_BYTES. */
+mom_status mom_copy_rows(const void* src, int64_t n_src, int64_t src_stride, int64_t src_off,
+                         const int32_t* idx, int64_t n_rows, int64_t row_bytes,
+                         void* dst, int64_t dst_stride, int64_t dst_off, void* ws, size_t ws_bytes, void* stream);
+
 /* mom_gate_proj -- the per-token gates of the memories alone (the Gated
  * DeltaNet gating every memory uses: blog post, experiments section):
  *   beta = sigmoid(x W_beta^T),  log_alpha = -exp(A) * softplus(x W_a^T + b_a)

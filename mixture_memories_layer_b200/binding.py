@@ -59,6 +59,10 @@ SIGNATURES = {
     "mom_decode_step_rule": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP, _VP, _SZ,
                                   _VP]),
     "mom_mem_gate_proj": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_proj_shared": (_I, [_VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_kv_proj_groups": (_I, [_VP, _I64, _VP, _I64, _VP, _VP, _I, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ,
+                                _VP]),
+    "mom_copy_rows": (_I, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _VP, _I64, _I64, _VP, _SZ, _VP]),
 }
 
 
@@ -219,6 +223,33 @@ def mom_mem_gate_proj(x, perm, mem_offset, w_gate_mem, A_mem, b_a_mem, top_k, be
     _check(lib.mom_mem_gate_proj(_p(x), _p(perm), _p(mem_offset), _p(w_gate_mem), _p(A_mem), _p(b_a_mem),
                                  dtype_code(x.dtype), n_tok, d_model, H, n_mem, top_k, _p(beta_p),
                                  _p(log_alpha_p), _p(ws), ws.numel(), _s(stream)), "mom_mem_gate_proj")
+
+
+def mom_proj_shared(x, w_shared, H, d, q, k_sh, v_sh, ws, stream=None):
+    n_tok, d_model = x.shape
+    _check(lib.mom_proj_shared(_p(x), _p(w_shared), dtype_code(x.dtype), n_tok, d_model, H, d, _p(q), _p(k_sh),
+                               _p(v_sh), _p(ws), ws.numel(), _s(stream)), "mom_proj_shared")
+
+
+def mom_kv_proj_groups(x, perm, group_offset, group_mem, w_kv, H, d, k_p, v_p, ws, stream=None):
+    """Routed k/v projections over groups: group g = rows group_offset[g] ..
+    group_offset[g+1] with memory group_mem[g]'s weights (perm None: row r
+    reads x row r)."""
+    n_x, d_model = x.shape
+    _check(lib.mom_kv_proj_groups(_p(x), n_x, _p(perm), k_p.shape[0], _p(group_offset), _p(group_mem),
+                                  group_mem.numel(), _p(w_kv), dtype_code(x.dtype), d_model, H, d, w_kv.shape[0],
+                                  _p(k_p), _p(v_p), _p(ws), ws.numel(), _s(stream)), "mom_kv_proj_groups")
+
+
+def mom_copy_rows(src, idx, dst, row_bytes, src_off=0, dst_off=0, ws=None, stream=None, n_rows=None):
+    """dst row i (bytes dst_off ..) = src row idx[i] (or i) (bytes src_off ..);
+    src and dst are 2-D tensors whose rows are byte rows of their stride."""
+    n_src = src.shape[0]
+    n = dst.shape[0] if n_rows is None else n_rows
+    src_stride = src.stride(0) * src.element_size()
+    dst_stride = dst.stride(0) * dst.element_size()
+    _check(lib.mom_copy_rows(_p(src), n_src, src_stride, src_off, _p(idx), n, row_bytes, _p(dst), dst_stride,
+                             dst_off, _p(ws), ws.numel(), _s(stream)), "mom_copy_rows")
 
 
 def mom_gdn_workspace_size(n_rows, n_seg, H, d, dt):

@@ -138,6 +138,63 @@ mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const i
     return cuda_status(proj_tc_supported(a, dt) ? launch_proj_tc(a, st) : launch_proj_simt(a, dt, st));
 }
 
+mom_status mom_proj_shared(const void* x, const void* w_shared, mom_dtype dt, int64_t n_tok, int d_model,
+                           int H, int d, void* q, void* k_sh, void* v_sh, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || d_model <= 0 || d_model % 64 != 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {x, w_shared, q, k_sh, v_sh};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    ProjArgs a{x, nullptr, nullptr, w_shared, nullptr, n_tok, d_model, H, d, 1, 1,
+               q, k_sh, v_sh, nullptr, nullptr, ws};
+    a.parts = PROJ_SHARED;
+    cudaStream_t st = as_stream(stream);
+    return cuda_status(proj_tc_supported(a, dt) ? launch_proj_tc(a, st) : launch_proj_simt(a, dt, st));
+}
+
+mom_status mom_kv_proj_groups(const void* x, int64_t n_x, const int32_t* perm_token, int64_t n_rows,
+                              const int32_t* group_offset, const int32_t* group_mem, int n_groups,
+                              const void* w_kv, mom_dtype dt, int d_model, int H, int d, int n_mem,
+                              void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_x < 0 || n_rows < 0 || d_model <= 0 || d_model % 64 != 0) return MOM_ERR_ARG;
+    if (H < 1 || H > MOM_MAX_HEADS || n_mem < 1 || n_mem > MOM_MAX_MEM || n_groups < 0) return MOM_ERR_ARG;
+    if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (n_rows >= ((int64_t)1 << 31) || n_x >= ((int64_t)1 << 31)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_rows == 0 || n_groups == 0) return MOM_OK;
+    if (n_x == 0) return MOM_ERR_ARG;
+    const void* ptrs[] = {x, w_kv, k_p, v_p};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    if (!group_offset || !group_mem) return MOM_ERR_ARG;
+    ProjArgs a{x, perm_token, group_offset, nullptr, w_kv, n_x, d_model, H, d, n_mem, 1,
+               nullptr, nullptr, nullptr, k_p, v_p, ws};
+    a.parts = PROJ_ROUTED;
+    a.group_mem = group_mem;
+    a.n_groups = n_groups;
+    a.n_routed = n_rows;
+    cudaStream_t st = as_stream(stream);
+    return cuda_status(proj_tc_supported(a, dt) ? launch_proj_tc(a, st) : launch_proj_simt(a, dt, st));
+}
+
+mom_status mom_copy_rows(const void* src, int64_t n_src, int64_t src_stride, int64_t src_off,
+                         const int32_t* idx, int64_t n_rows, int64_t row_bytes,
+                         void* dst, int64_t dst_stride, int64_t dst_off, void* ws, size_t ws_bytes, void* stream) {
+    if (n_src < 0 || n_rows < 0 || row_bytes < 0 || src_stride < 0 || dst_stride < 0 || src_off < 0 || dst_off < 0)
+        return MOM_ERR_ARG;
+    const int64_t al[] = {src_stride, src_off, row_bytes, dst_stride, dst_off};
+    for (int64_t v : al)
+        if (v % 16 != 0) return MOM_ERR_ARG;
+    if (src_off + row_bytes > src_stride || dst_off + row_bytes > dst_stride) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_rows == 0 || row_bytes == 0) return MOM_OK;
+    if (!src || !dst || !al16(src) || !al16(dst) || n_src == 0) return MOM_ERR_ARG;
+    return cuda_status(launch_copy_rows(src, n_src, src_stride, src_off, idx, n_rows, row_bytes, dst, dst_stride,
+                                        dst_off, ws, as_stream(stream)));
+}
+
 size_t mom_gate_proj_workspace_size(int64_t n_tok, int d_model, int H) {
     (void)n_tok; (void)d_model; (void)H;
     return MOM_WS_HEADER_BYTES;

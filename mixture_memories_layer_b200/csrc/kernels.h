@@ -59,16 +59,27 @@ cudaError_t launch_permute(const int32_t* idx, int64_t n_tok, int K, int M, cons
 
 // proj_simt.cu: grouped projections on CUDA cores (float32 mode, and any
 // shape the tensor-core path does not take)
+enum ProjPart { PROJ_SHARED = 1, PROJ_ROUTED = 2 };
 struct ProjArgs {
-    const void* x;
-    const int32_t* perm_token;
-    const int32_t* mem_offset;
+    const void* x;                // [n_tok, D]
+    const int32_t* perm_token;    // routed row -> x row (null: row r reads x row r)
+    const int32_t* mem_offset;    // group g: routed rows mem_offset[g] .. mem_offset[g+1]
     const void* w_shared;
     const void* w_kv;
     int64_t n_tok;
     int D, H, d, M, K;
     void *q, *k_sh, *v_sh, *k_p, *v_p;
     void* ws;
+    // which problems run (PROJ_SHARED | PROJ_ROUTED)
+    int parts = PROJ_SHARED | PROJ_ROUTED;
+    // routed groups: n_groups (0: M, one per memory) with group g using
+    // memory group_mem[g]'s weights (null: memory g); n_routed routed rows
+    // (< 0: n_tok * K)
+    const int32_t* group_mem = nullptr;
+    int n_groups = 0;
+    int64_t n_routed = -1;
+    __host__ __device__ int groups() const { return n_groups > 0 ? n_groups : M; }
+    __host__ __device__ int64_t routed_rows() const { return n_routed >= 0 ? n_routed : n_tok * K; }
 };
 cudaError_t launch_proj_simt(const ProjArgs& a, int dt, cudaStream_t st);
 
@@ -110,6 +121,11 @@ cudaError_t launch_gdn_recurrent(const GdnArgs& a, int dt, cudaStream_t st);
 bool gdn_tc_supported(const GdnArgs& a, int dt);
 size_t gdn_tc_ws_bytes(int64_t n_rows, int n_seg, int H, int d);
 cudaError_t launch_gdn_tc(const GdnArgs& a, cudaStream_t st);
+
+// copy_rows.cu: dst row i = bytes of src row idx[i] (or i), 16-byte granules
+cudaError_t launch_copy_rows(const void* src, int64_t n_src, int64_t src_stride, int64_t src_off, const int32_t* idx,
+                             int64_t n_rows, int64_t row_bytes, void* dst, int64_t dst_stride, int64_t dst_off,
+                             void* err, cudaStream_t st);
 
 // combine.cu
 cudaError_t launch_combine(const void* o_sh, const void* o_p, const int32_t* row_of, const float* gate,

@@ -49,15 +49,16 @@ proj_simt_kernel(ProjArgs a, int64_t sh_tiles) {
         int64_t local = bid - sh_tiles;
         cb = (int)(local % nb);
         int64_t rt = local / nb;
-        const int64_t n_rows = a.n_tok * a.K;
-        for (int mm = 0; mm < a.M; ++mm) {
-            int64_t lo = a.mem_offset[mm], hi = a.mem_offset[mm + 1];
-            if (lo < 0 || hi < lo || hi > n_rows) {          // corrupted offsets: touch nothing
-                if (cb == 0) record_error(a.ws, MOM_DEVERR_SEGMENT, mm);
+        const int64_t n_rows = a.routed_rows();
+        for (int g = 0; g < a.groups(); ++g) {
+            int64_t lo = a.mem_offset[g], hi = a.mem_offset[g + 1];
+            const int gm = a.group_mem ? a.group_mem[g] : g;
+            if (lo < 0 || hi < lo || hi > n_rows || gm < 0 || gm >= a.M) {   // corrupted table: touch nothing
+                if (cb == 0) record_error(a.ws, MOM_DEVERR_SEGMENT, g);
                 return;
             }
             int64_t nt = cdiv(hi - lo, BM);
-            if (rt < nt) { m = mm; r_begin = lo + rt * BM; r_end = (r_begin + BM < hi ? r_begin + BM : hi); break; }
+            if (rt < nt) { m = gm; r_begin = lo + rt * BM; r_end = (r_begin + BM < hi ? r_begin + BM : hi); break; }
             rt -= nt;
         }
         if (m < 0) return;
@@ -74,7 +75,7 @@ proj_simt_kernel(ProjArgs a, int64_t sh_tiles) {
     {
         int64_t r = r_begin + lrow;
         if (r < r_end) {
-            src = (m < 0) ? r : (int64_t)a.perm_token[r];
+            src = (m < 0 || !a.perm_token) ? r : (int64_t)a.perm_token[r];
             if (src < 0 || src >= a.n_tok) { record_error(a.ws, MOM_DEVERR_ROW_INDEX, r); src = -1; }
         }
     }
@@ -138,8 +139,8 @@ proj_simt_kernel(ProjArgs a, int64_t sh_tiles) {
 
 template <typename T, int DH>
 static cudaError_t launch_t(const ProjArgs& a, cudaStream_t st) {
-    const int64_t sh_tiles = cdiv(a.n_tok, BM) * 3 * a.H;
-    const int64_t rt_tiles = (cdiv(a.n_tok * a.K, BM) + a.M) * 2 * a.H;
+    const int64_t sh_tiles = (a.parts & PROJ_SHARED) ? cdiv(a.n_tok, BM) * 3 * a.H : 0;
+    const int64_t rt_tiles = (a.parts & PROJ_ROUTED) ? (cdiv(a.routed_rows(), BM) + a.groups()) * 2 * a.H : 0;
     const int64_t grid = sh_tiles + rt_tiles;
     if (grid == 0) return cudaSuccess;
     proj_simt_kernel<T, DH><<<(unsigned)grid, NT, 0, st>>>(a, sh_tiles);

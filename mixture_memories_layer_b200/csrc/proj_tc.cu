@@ -47,10 +47,11 @@ constexpr uint32_t TMEM_COLS = 2 * BN;
 struct TcParams {
     const bf16* x;
     const int32_t* perm;
-    const int32_t* mem_offset;
+    const int32_t* mem_offset;       // routed group offsets [n_groups + 1]
+    const int32_t* group_mem;        // memory of each group (null: group g = memory g)
     bf16 *q, *k_sh, *v_sh, *k_p, *v_p;
-    int64_t n_tok;
-    int D, H, d, M, K;
+    int64_t n_tok, n_routed;
+    int D, H, d, M, K, n_groups;
     int sh_ct, rt_ct;       // column tiles per row tile (shared / routed)
     int64_t sh_tiles;       // shared tiles
     int64_t n_tiles;        // shared + an upper bound of routed tiles
@@ -77,12 +78,13 @@ __device__ __forceinline__ bool tile_at(const TcParams& p, int64_t t, Tile& T) {
     const int64_t local = t - p.sh_tiles;
     int64_t rt = local / p.rt_ct;
     T.ct = (int)(local % p.rt_ct);
-    const int64_t n_rows = p.n_tok * p.K;
-    for (int m = 0; m < p.M; ++m) {
-        const int64_t lo = p.mem_offset[m], hi = p.mem_offset[m + 1];
-        if (lo < 0 || hi < lo || hi > n_rows) return false;
+    for (int g = 0; g < p.n_groups; ++g) {
+        const int64_t lo = p.mem_offset[g], hi = p.mem_offset[g + 1];
+        if (lo < 0 || hi < lo || hi > p.n_routed) return false;
         const int64_t nt = (hi - lo + BM - 1) / BM;
         if (rt < nt) {
+            const int m = p.group_mem ? p.group_mem[g] : g;
+            if (m < 0 || m >= p.M) return false;
             T.m = m;
             T.r0 = lo + rt * BM;
             T.r1 = T.r0 + BM < hi ? T.r0 + BM : hi;
@@ -156,7 +158,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int64_t row = T.r0 + rsub + 16 * i;
-                tok[i] = row < T.r1 ? (T.m < 0 ? row : (int64_t)p.perm[row]) : -1;
+                tok[i] = row < T.r1 ? ((T.m < 0 || !p.perm) ? row : (int64_t)p.perm[row]) : -1;
             }
         };
         Tile T;
@@ -378,30 +380,42 @@ bool proj_tc_supported(const ProjArgs& a, int dt) {
 
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     const int Hd = a.H * a.d;
+    const bool sh = a.parts & PROJ_SHARED, rt = (a.parts & PROJ_ROUTED) && a.routed_rows() > 0;
+    if (!sh && !rt) return cudaSuccess;
+    // maps of a problem that does not run are copies of one that does (never used)
     CUtensorMap tm_sh, tm_kv;
-    if (!make_tma_2d_bf16(&tm_sh, a.w_shared, (uint64_t)3 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
-    if (!make_tma_2d_bf16(&tm_kv, a.w_kv, (uint64_t)a.M * 2 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
+    if (sh && !make_tma_2d_bf16(&tm_sh, a.w_shared, (uint64_t)3 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
+    if (rt && !make_tma_2d_bf16(&tm_kv, a.w_kv, (uint64_t)a.M * 2 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
+    if (!sh) tm_sh = tm_kv;
+    if (!rt) tm_kv = tm_sh;
     OutMaps om;
-    const uint64_t nrp = (uint64_t)a.n_tok * a.K;
-    if (!make_tma_2d_bf16(&om.q, a.q, a.n_tok, Hd, Hd, 64, 32) || !make_tma_2d_bf16(&om.k_sh, a.k_sh, a.n_tok, Hd, Hd, 64, 32) ||
-        !make_tma_2d_bf16(&om.v_sh, a.v_sh, a.n_tok, Hd, Hd, 64, 32) || !make_tma_2d_bf16(&om.k_p, a.k_p, nrp, Hd, Hd, 64, 32) ||
-        !make_tma_2d_bf16(&om.v_p, a.v_p, nrp, Hd, Hd, 64, 32))
+    const uint64_t nrp = (uint64_t)a.routed_rows();
+    if (sh && (!make_tma_2d_bf16(&om.q, a.q, a.n_tok, Hd, Hd, 64, 32) ||
+               !make_tma_2d_bf16(&om.k_sh, a.k_sh, a.n_tok, Hd, Hd, 64, 32) ||
+               !make_tma_2d_bf16(&om.v_sh, a.v_sh, a.n_tok, Hd, Hd, 64, 32)))
         return cudaErrorInvalidValue;
+    if (rt && (!make_tma_2d_bf16(&om.k_p, a.k_p, nrp, Hd, Hd, 64, 32) || !make_tma_2d_bf16(&om.v_p, a.v_p, nrp, Hd, Hd, 64, 32)))
+        return cudaErrorInvalidValue;
+    if (!sh) om.q = om.k_sh = om.v_sh = om.k_p;
+    if (!rt) om.k_p = om.v_p = om.q;
     TcParams p;
     p.x = reinterpret_cast<const bf16*>(a.x);
     p.perm = a.perm_token;
     p.mem_offset = a.mem_offset;
+    p.group_mem = a.group_mem;
     p.q = reinterpret_cast<bf16*>(a.q);
     p.k_sh = reinterpret_cast<bf16*>(a.k_sh);
     p.v_sh = reinterpret_cast<bf16*>(a.v_sh);
     p.k_p = reinterpret_cast<bf16*>(a.k_p);
     p.v_p = reinterpret_cast<bf16*>(a.v_p);
     p.n_tok = a.n_tok;
+    p.n_routed = nrp;
+    p.n_groups = a.groups();
     p.D = a.D; p.H = a.H; p.d = a.d; p.M = a.M; p.K = a.K;
     p.sh_ct = 3 * Hd / BN;
     p.rt_ct = 2 * Hd / BN;
-    p.sh_tiles = cdiv(a.n_tok, BM) * p.sh_ct;
-    p.n_tiles = p.sh_tiles + (cdiv(a.n_tok * a.K, BM) + a.M) * p.rt_ct;
+    p.sh_tiles = sh ? cdiv(a.n_tok, BM) * p.sh_ct : 0;
+    p.n_tiles = p.sh_tiles + (rt ? (cdiv((int64_t)nrp, BM) + p.n_groups) * p.rt_ct : 0);
     p.ws = a.ws;
 
     static unsigned long long optin_done = 0;
