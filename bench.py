@@ -573,6 +573,89 @@ def cpu_baseline(w):
                       "each), fp64 numpy; tokens over the slowest process's %.1f s" % (procs, w.seq_len, sec)}
 
 
+def memory_parallel_arm(args):
+    """--parallel memory: the routed memories sharded over the ranks (each
+    rank owns a block of memories and its own batch of sequences; routed rows
+    go to their owners and back with NCCL all-to-alls).  The same timing
+    rules as the data-parallel arm: warm-up, barriers, L2 flushed outside the
+    events, max over ranks; the exchange's host reads of split sizes are
+    inside the timed region."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from mixture_memories_layer_b200 import binding as B
+    from mixture_memories_layer_b200 import layer as L
+    from mixture_memories_layer_b200 import synth
+    from mixture_memories_layer_b200.mem_parallel import MemoryParallelMoM, Partition, TorchComm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d (launch N>1 with torchrun)" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world == 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29541")
+        os.environ.setdefault("RANK", "0")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev,
+                            rank=int(os.environ.get("RANK", "0")), world_size=world)
+    try:
+        rank = dist.get_rank()
+        w = synth.WORKLOADS[args.workload]
+        p = rank_problem(w, rank)
+        dt = torch.bfloat16
+        full = L.pack_weights(p, dt, dev)
+        part = Partition(w.n_mem, world)
+        weights = {k: v for k, v in full.items() if k != "w_kv"}
+        weights["w_kv"] = full["w_kv"][part.lo(rank):part.hi(rank)].contiguous()
+        del full
+        meta = dist.new_group(backend="gloo")
+        layer = MemoryParallelMoM(weights, w.heads, w.d_head, w.top_k, w.n_mem, TorchComm(meta_group=meta))
+        x = torch.as_tensor(p["x"]).to(dev, dt)
+        cu = torch.as_tensor(p["cu_seqlens"]).to(dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            layer.forward(x, cu)
+        torch.cuda.synchronize()
+        launches0 = B.mom_launch_count()
+        dist.barrier()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            layer.forward(x, cu)
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        dist.barrier()
+        launches = B.mom_launch_count() - launches0
+        t = torch.tensor([sum(ms)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        if rank == 0:
+            value = aggregate_throughput(w.n_tokens, world, args.steps, total_ms)
+            lf, lb, lt = layer_roofline(w, load_peaks())
+            out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                   "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                   "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                   "data": "synthetic: seeded, same generator as the data-parallel arm",
+                   "config": {"workload": workload_desc(w), "tokens_per_gpu": w.n_tokens,
+                              "global_tokens": w.n_tokens * world,
+                              "parallelism": "mp%d (memories sharded, routed rows to their owners and back by "
+                                             "NCCL all-to-all)" % world,
+                              "l2": "flushed before every timed step (256 MiB write, untimed)"},
+                   "layer_roofline": {"flops": lf, "bytes": lb, "roofline_ms": lt * 1e3,
+                                      "frac": lt * 1e3 / (total_ms / args.steps)},
+                   "gpu_launches": launches}
+            print(json.dumps(out), flush=True)
+    finally:
+        dist.destroy_process_group()
+
+
 def reference_arm(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return None
@@ -620,11 +703,19 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode timing")
     ap.add_argument("--no-configs", action="store_true", help="skip the other forward workloads")
+    ap.add_argument("--parallel", default="data", choices=["data", "memory"],
+                    help="data: every rank runs the whole layer on its own sequences; memory: the routed "
+                         "memories are sharded over the ranks")
+    ap.add_argument("--workload", default=None, help="forward workload of --parallel memory (default: the "
+                    "16-memory 1.3B shape)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         reference_arm(args)
+    elif args.parallel == "memory":
+        args.workload = args.workload or "mom1p3b_m16"
+        memory_parallel_arm(args)
     else:
         gpu_arm(args)
 

@@ -123,20 +123,37 @@ def receive_tables(seg_from: List[np.ndarray], n_seq_of: List[int], part: Partit
 
 # ------------------------------------------------------------ communication
 class TorchComm:
-    """The exchanges of a memory-parallel layer over a torch.distributed
-    process group (NCCL for CUDA buffers)."""
+    """The exchanges of a memory-parallel layer over torch.distributed: the
+    row buffers over `group` (NCCL for CUDA buffers), the few integers of
+    metadata over `meta_group`, a CPU (gloo) group of the same ranks, so that
+    reading them never waits for the GPU's queued work (None: `group`, with
+    host tensors, for a CPU process group)."""
 
-    def __init__(self, group=None):
+    def __init__(self, group=None, meta_group=None):
         import torch.distributed as dist
         self.dist, self.group = dist, group
+        if meta_group is None and dist.get_backend(group) != "gloo":
+            # every rank constructs its TorchComm, so this collective call is matched
+            ranks = dist.get_process_group_ranks(group) if group is not None else None
+            meta_group = dist.new_group(ranks=ranks, backend="gloo")
+        self.meta = meta_group if meta_group is not None else group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
 
-    def all_gather_ints(self, values: List[int], device) -> List[List[int]]:
-        t = torch.tensor(values, dtype=torch.int64, device=device)
+    def gather_ints(self, v: int) -> List[int]:
+        t = torch.tensor([v], dtype=torch.int64)
         out = [torch.empty_like(t) for _ in range(self.world)]
-        self.dist.all_gather(out, t, group=self.group)
-        return [o.cpu().tolist() for o in out]
+        self.dist.all_gather(out, t, group=self.meta)
+        return [int(o.item()) for o in out]
+
+    def exchange_ints(self, per_dest: List[np.ndarray], in_sizes: List[int]) -> List[np.ndarray]:
+        """per_dest[g] to rank g; returns what each rank sent here."""
+        inp = torch.as_tensor(np.concatenate(per_dest).astype(np.int32) if per_dest else np.zeros(0, np.int32))
+        out = torch.empty(sum(in_sizes), dtype=torch.int32)
+        self.dist.all_to_all_single(out, inp, list(in_sizes), [len(a) for a in per_dest], group=self.meta)
+        b = np.concatenate([[0], np.cumsum(in_sizes)]).astype(np.int64)
+        o = out.numpy()
+        return [o[b[r]:b[r + 1]] for r in range(len(in_sizes))]
 
     def all_to_all(self, out: torch.Tensor, inp: torch.Tensor, out_splits: List[int], in_splits: List[int]):
         self.dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
@@ -218,11 +235,36 @@ class MemoryParallelMoM:
         self.k = kernels if kernels is not None else CudaKernels()
         self.part = Partition(n_mem, comm.world)
         self.rank = comm.rank
+        self._ws = {}
+        self._side = None
         own = self.part.hi(self.rank) - self.part.lo(self.rank)
         if weights["w_kv"].shape[0] != own:
             raise ValueError("w_kv holds %d memories; rank %d owns %d" % (weights["w_kv"].shape[0], self.rank, own))
         if any(k.endswith("_mem") for k in weights):
             raise ValueError("per-memory gates are not provided by the memory-parallel layer")
+
+    def _workspace(self, name, nbytes, device):
+        """A workspace kept across calls (zeroed once, grown when needed)."""
+        t = self._ws.get(name)
+        if t is None or t.numel() < nbytes:
+            t = self._ws[name] = self.k.workspace(nbytes, device)
+        return t
+
+    @staticmethod
+    def _to_device(arr: np.ndarray, device) -> torch.Tensor:
+        """A small host table on the device without waiting for the stream's
+        queued work (pinned source, asynchronous copy)."""
+        t = torch.as_tensor(np.ascontiguousarray(arr))
+        if device.type != "cuda":
+            return t
+        return t.pin_memory().to(device, non_blocking=True)
+
+    def _side_stream(self, device):
+        if device.type != "cuda":
+            return None
+        if self._side is None:
+            self._side = torch.cuda.Stream(device=device)
+        return self._side
 
     # -- step 1 and the packing of step 2
     def local_phase(self, x: torch.Tensor, cu: torch.Tensor, stream=None) -> LocalState:
@@ -230,7 +272,7 @@ class MemoryParallelMoM:
         dev, dt = x.device, x.dtype
         n_tok, D = x.shape
         S = cu.numel() - 1
-        ws = k.workspace(256, dev)
+        ws = self._workspace("local", 256, dev)
         idx = torch.empty((n_tok, K), dtype=torch.int32, device=dev)
         gate = torch.empty((n_tok, K), dtype=torch.float32, device=dev)
         k.router(x, w["w_r"], w["b_r"], K, idx, gate, stream)
@@ -238,8 +280,20 @@ class MemoryParallelMoM:
         row_of = torch.empty_like(perm)
         mem_offset = torch.empty(M + 1, dtype=torch.int32, device=dev)
         seg_cu = torch.empty(M * S + 1, dtype=torch.int32, device=dev)
-        ws_perm = k.workspace(k.permute_workspace_size(n_tok, K, M, S), dev)
+        ws_perm = self._workspace("perm", k.permute_workspace_size(n_tok, K, M, S), dev)
         k.permute(idx, M, cu, perm, row_of, mem_offset, seg_cu, ws_perm, stream)
+        # the split sizes go to the host as soon as they exist; the GPU goes on
+        # with the projections, the gates and the packing meanwhile
+        if dev.type == "cuda":
+            counts = torch.empty(M + 1 + M * S + 1, dtype=torch.int32, pin_memory=True)
+            cur = stream if stream is not None else torch.cuda.current_stream(dev)
+            with torch.cuda.stream(cur):
+                counts[:M + 1].copy_(mem_offset, non_blocking=True)
+                counts[M + 1:].copy_(seg_cu, non_blocking=True)
+            counted = torch.cuda.Event()
+            counted.record(cur)
+        else:
+            counts, counted = torch.cat([mem_offset, seg_cu]), None
         q, k_sh, v_sh = (torch.empty((n_tok, H, d), dtype=dt, device=dev) for _ in range(3))
         k.proj_shared(x, w["w_shared"], H, d, q, k_sh, v_sh, ws, stream)
         beta = torch.empty((n_tok, H), dtype=torch.float32, device=dev)
@@ -247,18 +301,33 @@ class MemoryParallelMoM:
         k.gates(x, w["w_gate"], w["A"], w["b_a"], beta, log_alpha, ws, stream)
         o_sh = torch.empty_like(q)
         h_shared = torch.empty((S, H, d, d), dtype=torch.float32, device=dev)
-        ws_gdn = k.workspace(k.gdn_workspace_size(n_tok, S, H, d, dt), dev)
+        ws_gdn = self._workspace("gdn_sh", k.gdn_workspace_size(n_tok, S, H, d, dt), dev)
+        # the shared memory's recurrence beside the exchange and the owners' work
+        side, shared_done = self._side_stream(dev), None
+        if side is not None:
+            ready = torch.cuda.Event()
+            ready.record(stream if stream is not None else torch.cuda.current_stream(dev))
+            side.wait_event(ready)
+            # the allocator must not hand these to the current stream while the side stream reads them
+            for t in (q, k_sh, v_sh, beta, log_alpha, cu, o_sh, h_shared):
+                t.record_stream(side)
         k.recurrence(q, None, k_sh, v_sh, beta, log_alpha, cu, self.scale, k.rule_code(self.rule), None, h_shared,
-                     o_sh, ws_gdn, stream)
+                     o_sh, ws_gdn, side if side is not None else stream)
+        if side is not None:
+            shared_done = torch.cuda.Event()
+            shared_done.record(side)
         # pack [x | q] of every routed row in the reordered order
         xb, qb = D * x.element_size(), H * d * q.element_size()
         send = torch.empty((n_tok * K, xb + qb), dtype=torch.uint8, device=dev)
         k.copy_rows(x.view(n_tok, D), perm, send, xb, 0, 0, ws, stream)
         k.copy_rows(q.view(n_tok, H * d), perm, send, qb, 0, xb, ws, stream)
-        send_rows, _, seg_out = send_plan(mem_offset.cpu().numpy(), seg_cu.cpu().numpy(), S, self.part)
+        if counted is not None:
+            counted.synchronize()
+        c = counts.numpy()
+        send_rows, _, seg_out = send_plan(c[:M + 1], c[M + 1:], S, self.part)
         return LocalState(idx=idx, gate=gate, row_of=row_of, o_sh=o_sh, h_shared=h_shared, send=send,
                           send_rows=send_rows, seg_out=seg_out, n_seq=S,
-                          extras={"ws": ws, "ws_perm": ws_perm, "ws_gdn": ws_gdn})
+                          extras={"ws": ws, "shared_done": shared_done})
 
     # -- step 3
     def owner_phase(self, recv: torch.Tensor, tables: ReceiveTables, dt: torch.dtype, stream=None):
@@ -278,7 +347,7 @@ class MemoryParallelMoM:
             if n_seg:
                 h.zero_()
             return o, h
-        ws = k.workspace(256, dev)
+        ws = self._workspace("owner", 256, dev)
         x_r = torch.empty((n, D), dtype=dt, device=dev)
         q_r = torch.empty((n, H, d), dtype=dt, device=dev)
         k.copy_rows(recv, None, x_r.view(torch.uint8).view(n, xb), xb, 0, 0, ws, stream)
@@ -287,13 +356,13 @@ class MemoryParallelMoM:
         log_alpha = torch.empty_like(beta)
         k.gates(x_r, w["w_gate"], w["A"], w["b_a"], beta, log_alpha, ws, stream)
         lo = self.part.lo(self.rank)
-        go = torch.as_tensor(tables.group_offset).to(dev)
-        gm = torch.as_tensor(tables.group_mem - lo).to(dev)          # index into this rank's w_kv block
+        go = self._to_device(tables.group_offset, dev)
+        gm = self._to_device(tables.group_mem - lo, dev)             # index into this rank's w_kv block
+        seg = self._to_device(tables.seg_cu, dev)
         k_p = torch.empty((n, H, d), dtype=dt, device=dev)
         v_p = torch.empty_like(k_p)
         k.kv_groups(x_r, go, gm, w["w_kv"], H, d, k_p, v_p, ws, stream)
-        seg = torch.as_tensor(tables.seg_cu).to(dev)
-        ws_gdn = k.workspace(k.gdn_workspace_size(n, n_seg, H, d, dt), dev)
+        ws_gdn = self._workspace("gdn_owner", k.gdn_workspace_size(n, n_seg, H, d, dt), dev)
         k.recurrence(q_r, None, k_p, v_p, beta, log_alpha, seg, self.scale, k.rule_code(self.rule), None, h, o,
                      ws_gdn, stream)
         return o, h
@@ -302,6 +371,8 @@ class MemoryParallelMoM:
     def finish_phase(self, st: LocalState, o_back: torch.Tensor, stream=None) -> torch.Tensor:
         n_tok = st.idx.shape[0]
         out = torch.empty((n_tok, self.H, self.d), dtype=st.o_sh.dtype, device=st.o_sh.device)
+        if st.extras.get("shared_done") is not None:
+            (stream if stream is not None else torch.cuda.current_stream(out.device)).wait_event(st.extras["shared_done"])
         self.k.combine(st.o_sh, o_back, st.row_of, st.gate, out, st.extras["ws"], stream)
         return out
 
@@ -311,18 +382,11 @@ class MemoryParallelMoM:
         segments this rank received [n_seg, H, d, d], their ReceiveTables)."""
         st = self.local_phase(x, cu, stream)
         dev, G = x.device, self.comm.world
-        n_seq_of = [row[0] for row in self.comm.all_gather_ints([st.n_seq], dev)]
-        # segment lengths: to rank g, len(owned(g)) * S ints
-        own = [self.part.hi(g) - self.part.lo(g) for g in range(G)]
-        seg_send = torch.as_tensor(np.concatenate(st.seg_out) if st.seg_out else np.zeros(0, np.int32)).to(dev)
-        in_splits = [own[g] * st.n_seq for g in range(G)]
-        out_splits = [own[self.rank] * n_seq_of[r] for r in range(G)]
-        seg_recv = torch.empty(sum(out_splits), dtype=torch.int32, device=dev)
-        self.comm.all_to_all(seg_recv, seg_send.to(torch.int32), out_splits, in_splits)
-        seg_host = seg_recv.cpu().numpy()
-        bounds = np.concatenate([[0], np.cumsum(out_splits)])
-        tables = receive_tables([seg_host[bounds[r]:bounds[r + 1]] for r in range(G)], n_seq_of, self.part,
-                                self.rank)
+        n_seq_of = self.comm.gather_ints(st.n_seq)
+        # segment lengths from each source: len(owned(this rank)) * S_r ints
+        own = self.part.hi(self.rank) - self.part.lo(self.rank)
+        seg_from = self.comm.exchange_ints(st.seg_out, [own * n_seq_of[r] for r in range(G)])
+        tables = receive_tables(seg_from, n_seq_of, self.part, self.rank)
         recv = torch.empty((tables.n_rows, st.send.shape[1]), dtype=torch.uint8, device=dev)
         self.comm.all_to_all(recv, st.send, tables.rows, st.send_rows)
         o_r, h_r = self.owner_phase(recv, tables, x.dtype, stream)

@@ -133,7 +133,8 @@ def test_one_rank_nccl_group_equals_the_layer():
     os.environ["MASTER_PORT"] = str(_free_port())
     dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
     try:
-        mp = MemoryParallelMoM(lay.w, w.heads, w.d_head, w.top_k, w.n_mem, TorchComm())
+        mp = MemoryParallelMoM(lay.w, w.heads, w.d_head, w.top_k, w.n_mem,
+                               TorchComm(meta_group=dist.new_group(backend="gloo")))
         out, h_sh, h_mem, tables = mp.forward(xt, cut)
         torch.cuda.synchronize()
     finally:
