@@ -65,14 +65,27 @@ def workload_desc(w):
 
 
 def load_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
-        with open(path) as fh:
-            p = json.load(fh)
-        p["source"] = "measured"
-        return p
+    """The roofline denominators: MEASURED_PEAKS.json's hbm_gbs, bf16_tflops
+    and bf16_tflops_sustained where it has them (numbers, possibly under a
+    "peaks" key), the fallback figures for any it lacks; "source" says which."""
     p = dict(FALLBACK_PEAKS)
-    p["source"] = "fallback"
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    got = []
+    if os.path.exists(path):
+        try:
+            with open(path) as fh:
+                m = json.load(fh)
+        except (OSError, ValueError):
+            m = {}
+        if isinstance(m, dict) and isinstance(m.get("peaks"), dict):
+            m = m["peaks"]
+        for k in FALLBACK_PEAKS:
+            v = m.get(k) if isinstance(m, dict) else None
+            if isinstance(v, (int, float)) and v > 0:
+                p[k] = float(v)
+                got.append(k)
+    p["source"] = ("measured" if len(got) == len(FALLBACK_PEAKS) else
+                   "measured (%s), fallback otherwise" % ", ".join(got) if got else "fallback")
     return p
 
 

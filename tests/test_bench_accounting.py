@@ -92,3 +92,20 @@ def test_clock_summary_names_every_throttle_reason_seen():
     empty = bench.ClockSampler(torch_device=None)
     empty.sm_max = None
     assert empty.summary()["reasons"] == ["unsampled"]
+
+
+def test_load_peaks_measured_partial_and_fallback(tmp_path, monkeypatch):
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p = bench.load_peaks()
+    assert p["source"] == "fallback" and p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 6540.2, "bf16_tflops": 1631.7, "bf16_tflops_sustained": 1358.8, "clocks": "x"}))
+    p = bench.load_peaks()
+    assert p["source"] == "measured" and p["hbm_gbs"] == 6540.2 and p["bf16_tflops_sustained"] == 1358.8
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"peaks": {"hbm_gbs": 6000.0}}))
+    p = bench.load_peaks()
+    assert p["hbm_gbs"] == 6000.0 and p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    assert p["source"].startswith("measured (hbm_gbs)")
+    (tmp_path / "MEASURED_PEAKS.json").write_text("not json")
+    assert bench.load_peaks()["source"] == "fallback"
