@@ -47,24 +47,29 @@ def l2norm_bwd(z, dy, eps: float = fwd.NORM_EPS):
     return dy / n - z * np.sum(z * dy, axis=-1, keepdims=True) / n ** 3
 
 
-def gdn_recurrence_bwd(q, k, v, beta, log_alpha, do, h0=None, dh_final=None, scale: float = 1.0):
+def gdn_recurrence_bwd(q, k, v, beta, log_alpha, do, h0=None, dh_final=None, scale: float = 1.0,
+                       rule: str = "gated_delta"):
     """Reverse pass of ``mom_oracle.gdn_recurrence`` over one segment.
 
     Shapes as the forward: q,k [T,H,dk]; v, do [T,H,dv]; beta, log_alpha
     [T,H]; h0, dh_final [H,dv,dk] or None.  Returns a dict with dq, dk, dv,
     dbeta, dlog_alpha (the forward's shapes) and dh0 [H,dv,dk].
 
-    With a = exp(log alpha_t), b = beta_t, y = S_{t-1} k_t and
-    S_t = a S_{t-1} - a b y k^T + b v k^T,  o_t = S_t (scale q_t),
+    With a = exp(log alpha_t), b = beta_t, y = S_{t-1} k_t, c = 1 for the
+    Gated DeltaNet rule and 0 for the scalar-gated linear one, and
+    S_t = a S_{t-1} - c a b y k^T + b v k^T,  o_t = S_t (scale q_t),
     and G the adjoint of S_t (do_t (scale q_t)^T plus what flows back from
     step t+1):
       dq_t = scale S_t^T do_t
       dv_t = b G k
-      db_t = (v - a y)^T G k
-      da_t = <G, S_{t-1}> - b y^T G k,       dlog_alpha_t = a da_t
-      dk_t = b G^T v - a b (S_{t-1}^T G k + G^T y)
-      adjoint of S_{t-1} = a G - a b (G k) k^T
+      db_t = (v - c a y)^T G k
+      da_t = <G, S_{t-1}> - c b y^T G k,       dlog_alpha_t = a da_t
+      dk_t = b G^T v - c a b (S_{t-1}^T G k + G^T y)
+      adjoint of S_{t-1} = a G - c a b (G k) k^T
     """
+    if rule not in fwd.RULES:
+        raise ValueError("rule must be one of %s" % sorted(fwd.RULES))
+    c = 1.0 if rule == "gated_delta" else 0.0
     q = np.asarray(q, F64)
     k = np.asarray(k, F64)
     v = np.asarray(v, F64)
@@ -77,8 +82,9 @@ def gdn_recurrence_bwd(q, k, v, beta, log_alpha, do, h0=None, dh_final=None, sca
     S = np.zeros((T + 1, H, dv, dk), F64)
     if h0 is not None:
         S[0] = np.asarray(h0, F64)
+    step = fwd.RULES[rule]
     for t in range(T):
-        _, S[t + 1] = fwd.gdn_step(S[t], q[t], k[t], v[t], beta[t], log_alpha[t], scale)
+        _, S[t + 1] = step(S[t], q[t], k[t], v[t], beta[t], log_alpha[t], scale)
     G = np.zeros((H, dv, dk), F64) if dh_final is None else np.array(dh_final, F64, copy=True)
     out = {name: np.zeros_like(a) for name, a in
            (("dq", q), ("dk", k), ("dv", v), ("dbeta", beta), ("dlog_alpha", log_alpha))}
@@ -92,14 +98,14 @@ def gdn_recurrence_bwd(q, k, v, beta, log_alpha, do, h0=None, dh_final=None, sca
         y = np.einsum("hvk,hk->hv", Sp, kt)
         Gk = np.einsum("hvk,hk->hv", G, kt)
         out["dv"][t] = b[:, None] * Gk
-        out["dbeta"][t] = np.einsum("hv,hv->h", vt - a[:, None] * y, Gk)
-        da = np.einsum("hvk,hvk->h", G, Sp) - b * np.einsum("hv,hv->h", y, Gk)
+        out["dbeta"][t] = np.einsum("hv,hv->h", vt - c * a[:, None] * y, Gk)
+        da = np.einsum("hvk,hvk->h", G, Sp) - c * b * np.einsum("hv,hv->h", y, Gk)
         out["dlog_alpha"][t] = a * da
         GTv = np.einsum("hvk,hv->hk", G, vt)
         SGk = np.einsum("hvk,hv->hk", Sp, Gk)
         GTy = np.einsum("hvk,hv->hk", G, y)
-        out["dk"][t] = b[:, None] * GTv - (a * b)[:, None] * (SGk + GTy)
-        G = a[:, None, None] * G - (a * b)[:, None, None] * Gk[:, :, None] * kt[:, None, :]
+        out["dk"][t] = b[:, None] * GTv - c * (a * b)[:, None] * (SGk + GTy)
+        G = a[:, None, None] * G - c * (a * b)[:, None, None] * Gk[:, :, None] * kt[:, None, :]
     out["dh0"] = G
     return out
 

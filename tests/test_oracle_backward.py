@@ -48,16 +48,17 @@ def _gdn_case(T=6, H=2, dk=3, dv=4, seed=0, beta_zero=False):
     return c, adj
 
 
+@pytest.mark.parametrize("rule", ["gated_delta", "gated_linear"])
 @pytest.mark.parametrize("scale", [1.0, 0.7])
-def test_gdn_recurrence_bwd_matches_finite_differences(scale):
+def test_gdn_recurrence_bwd_matches_finite_differences(scale, rule):
     c, adj = _gdn_case()
 
     def loss():
-        o, S = fwd.gdn_recurrence(c["q"], c["k"], c["v"], c["beta"], c["log_alpha"], c["h0"], scale)
+        o, S = fwd.gdn_recurrence(c["q"], c["k"], c["v"], c["beta"], c["log_alpha"], c["h0"], scale, rule)
         return float(np.sum(adj["do"] * o) + np.sum(adj["dh"] * S))
 
     g = bwd.gdn_recurrence_bwd(c["q"], c["k"], c["v"], c["beta"], c["log_alpha"], adj["do"], c["h0"], adj["dh"],
-                               scale)
+                               scale, rule)
     for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("beta", "dbeta"), ("log_alpha", "dlog_alpha"),
                       ("h0", "dh0")):
         e = _rel(g[key], _fd(loss, c[name]))
@@ -151,3 +152,21 @@ def test_l2norm_bwd_matches_finite_differences():
         return float(np.sum(dy * fwd.l2norm(z)))
 
     assert _rel(bwd.l2norm_bwd(z, dy), _fd(loss, z)) < 1e-8
+
+
+def test_gdn_recurrence_bwd_rules_differ_and_linear_rule_planted_mistake_fails():
+    """The two rules' gradients differ (the delta terms matter), and a
+    planted mistake in the linear rule's adjoint -- the delta term left in --
+    fails its finite differences."""
+    c, adj = _gdn_case(seed=3)
+    args = (c["q"], c["k"], c["v"], c["beta"], c["log_alpha"], adj["do"], c["h0"], adj["dh"], 1.0)
+    gd = bwd.gdn_recurrence_bwd(*args, "gated_delta")
+    gl = bwd.gdn_recurrence_bwd(*args, "gated_linear")
+    assert _rel(gd["dk"], gl["dk"]) > 1e-2 and _rel(gd["dh0"], gl["dh0"]) > 1e-2
+
+    def loss():
+        o, S = fwd.gdn_recurrence(c["q"], c["k"], c["v"], c["beta"], c["log_alpha"], c["h0"], 1.0, "gated_linear")
+        return float(np.sum(adj["do"] * o) + np.sum(adj["dh"] * S))
+
+    # the delta rule's adjoints are the linear rule's with the delta terms kept: they must fail here
+    assert _rel(gd["dk"], _fd(loss, c["k"])) > 1e-3
