@@ -384,6 +384,31 @@ mom_status mom_memory_chunk_state(const void* q, const int32_t* qidx, const void
                                   const float* h0, float* h_final, void* o,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/* mom_memory_chunk_bwd -- the reverse pass of mom_memory_chunk_fwd (either
+ * rule, either gate layout) for the loss <d_o, o> + sum_s <dh_final[s],
+ * h_final[s]> (training is the pages' main workload: paper card, Key points):
+ *   dq, dk, dv [n_rows, H, d] float32, dbeta, dlog_alpha [n_rows, H] float32
+ *   -- one per ROW of the segments (with qidx, row r's dq / dbeta /
+ *   dlog_alpha belong to q row qidx[r]: the caller adds them up per token) --
+ *   and dh0 [n_seg, H, d, d] float32 (NULL: not written).
+ * Inputs as mom_memory_chunk_fwd (q, k, v, the gates, seg_cu, h0 NULL = zero
+ * states), plus d_o [n_rows, H, d] (dt) and dh_final [n_seg, H, d, d]
+ * float32 or NULL (zero).  Rows outside [seg_cu[0], seg_cu[n_seg]) are not
+ * written; a row whose q index is out of range is recorded
+ * (MOM_DEVERR_ROW_INDEX) and contributes nothing.  Token-serial on CUDA
+ * cores in float32 whatever dt is.  Requires d in {64, 128, 256}.
+ * ws: mom_memory_chunk_bwd_workspace_size() (states kept for the reverse
+ * sweep and one partial sum per 64 state rows: about
+ * n_rows * H * d * 8 * d / 64 bytes). */
+size_t mom_memory_chunk_bwd_workspace_size(int64_t n_rows, int n_seg, int H, int d);
+mom_status mom_memory_chunk_bwd(const void* q, const int32_t* qidx, const void* k, const void* v,
+                                const float* beta, const float* log_alpha,
+                                const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                                int H, int d, float scale, mom_dtype dt, mom_rule rule, mom_gates gates,
+                                const float* h0, const void* d_o, const float* dh_final,
+                                float* dq, float* dk, float* dv, float* dbeta, float* dlog_alpha, float* dh0,
+                                void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * mom_combine_unpermute -- the combine (paper card, Summary: outputs are
  * combined using the router weights; blog post, "硬件高效實現": summing the

@@ -63,6 +63,9 @@ SIGNATURES = {
     "mom_kv_proj_groups": (_I, [_VP, _I64, _VP, _I64, _VP, _VP, _I, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ,
                                 _VP]),
     "mom_copy_rows": (_I, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _VP, _I64, _I64, _VP, _SZ, _VP]),
+    "mom_memory_chunk_bwd_workspace_size": (_SZ, [_I64, _I, _I, _I]),
+    "mom_memory_chunk_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I, _I,
+                                  _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
 }
 
 
@@ -305,6 +308,21 @@ def mom_memory_chunk_state(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, 
                            gates=MOM_GATES_BY_TOKEN):
     _memory("mom_memory_chunk_state", q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, h_final, o, ws, stream,
             gates)
+
+
+def mom_memory_chunk_bwd_workspace_size(n_rows, n_seg, H, d):
+    return lib.mom_memory_chunk_bwd_workspace_size(n_rows, n_seg, H, d)
+
+
+def mom_memory_chunk_bwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0, d_o, dh_final,
+                         dq, dk, dv, dbeta, dlog_alpha, dh0, ws, stream=None, gates=MOM_GATES_BY_TOKEN):
+    """Reverse pass of mom_memory_chunk_fwd: float32 gradients per row."""
+    n_rows, H, d = k.shape
+    _check(lib.mom_memory_chunk_bwd(_p(q), _p(qidx), _p(k), _p(v), _p(beta), _p(log_alpha), _p(seg_cu),
+                                    seg_cu.numel() - 1, n_rows, q.shape[0], H, d, float(scale), dtype_code(k.dtype),
+                                    int(rule), int(gates), _p(h0), _p(d_o), _p(dh_final), _p(dq), _p(dk), _p(dv),
+                                    _p(dbeta), _p(dlog_alpha), _p(dh0), _p(ws), ws.numel(), _s(stream)),
+           "mom_memory_chunk_bwd")
 
 
 def mom_combine_unpermute(o_sh, o_p, row_of, topk_gate, out, ws, stream=None):

@@ -307,6 +307,40 @@ MOM_MEMORY_CALL(mom_memory_chunk_prep, GDN_PREP)
 MOM_MEMORY_CALL(mom_memory_chunk_state, GDN_STATE)
 #undef MOM_MEMORY_CALL
 
+// ------------------------------------------------------- reverse pass
+size_t mom_memory_chunk_bwd_workspace_size(int64_t n_rows, int n_seg, int H, int d) {
+    if (n_rows < 0 || n_seg < 0 || H < 1 || !head_dim_ok(d)) return 0;
+    return gdn_bwd_ws_bytes(n_rows, n_seg, H, d);
+}
+
+mom_status mom_memory_chunk_bwd(const void* q, const int32_t* qidx, const void* k, const void* v,
+                                const float* beta, const float* log_alpha,
+                                const int32_t* seg_cu, int n_seg, int64_t n_rows, int64_t n_q_rows,
+                                int H, int d, float scale, mom_dtype dt, mom_rule rule, mom_gates gates,
+                                const float* h0, const void* d_o, const float* dh_final,
+                                float* dq, float* dk, float* dv, float* dbeta, float* dlog_alpha, float* dh0,
+                                void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_seg < 0 || n_rows < 0 || n_q_rows < 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (rule != MOM_RULE_GATED_DELTA && rule != MOM_RULE_GATED_LINEAR) return MOM_ERR_ARG;
+    if (gates != MOM_GATES_BY_TOKEN && gates != MOM_GATES_BY_ROW) return MOM_ERR_ARG;
+    if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (n_rows >= ((int64_t)1 << 31)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < mom_memory_chunk_bwd_workspace_size(n_rows, n_seg, H, d)) return MOM_ERR_ARG;
+    if (n_seg == 0) return MOM_OK;
+    if (!seg_cu) return MOM_ERR_ARG;
+    const void* opt[] = {h0, dh_final, dh0};
+    for (const void* p : opt)
+        if (p && !al16(p)) return MOM_ERR_ARG;
+    if (n_rows > 0) {
+        const void* ptrs[] = {q, k, v, beta, log_alpha, d_o, dq, dk, dv, dbeta, dlog_alpha};
+        for (const void* p : ptrs)
+            if (!p || !al16(p)) return MOM_ERR_ARG;
+    }
+    GdnBwdArgs a{q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, rule,
+                 gates == MOM_GATES_BY_ROW ? 1 : 0, h0, d_o, dh_final, dq, dk, dv, dbeta, dlog_alpha, dh0, ws};
+    return cuda_status(launch_gdn_bwd(a, dt, as_stream(stream)));
+}
+
 // ----------------------------------------------------------------- combine
 mom_status mom_combine_unpermute(const void* o_sh, const void* o_p, const int32_t* row_of,
                                  const float* topk_gate, int64_t n_tok, int top_k, int H, int d,

@@ -1,0 +1,322 @@
+// Reverse pass of a memory's recurrence over each segment, for both update
+// rules (the first GPU path of the layer's backward: training is the pages'
+// main workload, "MoM: Linear Sequence Modeling with Mixture-of-Memories",
+// Key points; the rules: the authors' MoM blog post, experiments section and
+// "Linear Recurrent Memory").  Token-serial, fp32, on CUDA cores.
+//
+// Forward, with a = e^(log alpha_t), b = beta_t, c = 1 (Gated DeltaNet) or 0
+// (scalar-gated linear), row i of the state evolving on its own:
+//   y_i = S_i . k,  u_i = b (v_i - c a y_i),  S_i <- a S_i + u_i k,  o_i = scale S_i . q
+// Reverse, with G_i the adjoint of row i after token t (plus do_i scale q):
+//   dq   += scale S_i(t) do_i            dv_i = b (G_i . k)
+//   dbeta += (v_i - c a y_i)(G_i . k)     dalpha += G_i . S_i(t-1) - c b y_i (G_i . k)
+//   dk   += u_i G_i - c a b (G_i . k) S_i(t-1)
+//   G_i  <- a G_i - c a b (G_i . k) k
+// (sums over the rows i; dlog_alpha = a dalpha).
+//
+// One CTA owns 64 state rows of one (segment, head): 16 warps of 4 rows, a
+// lane holding d/32 columns of each, as in the token-serial forward.  The
+// reverse pass needs S(t-1) at every token: a forward sweep stores the rows
+// every 64 tokens; the chunks are then walked backwards, each recomputed from
+// its stored state with a copy kept every 8 tokens, and the state before a
+// token is rebuilt from the nearest copy (at most 7 steps).  The sums over
+// rows are reduced inside the CTA per token and written as one partial per
+// 64-row tile, which a second kernel adds up (deterministic, no atomics).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mom {
+namespace {
+
+constexpr int BR = 4;               // state rows per warp
+constexpr int BW = 16;              // warps per CTA
+constexpr int ROWS = BR * BW;       // state rows per CTA
+constexpr int CK = 64;              // tokens between stored states
+constexpr int SUB = 8;              // tokens between the copies kept inside a chunk
+constexpr int NSUB = CK / SUB;
+
+struct BwdTables {
+    int32_t* chunk_cu;   // [n_seg + 1] first stored state of each segment
+    float* ckpt;         // [max_chunks][H][tiles][ROWS][D]
+    float* sub;          // [n_seg * tiles * H][NSUB][ROWS][D]
+    float* part;         // [tiles][n_rows][H][2D + 2]: dq | dk | dlog_alpha | dbeta
+};
+
+__global__ void bwd_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_seg, int64_t n_rows,
+                                    int32_t* __restrict__ chunk_cu, void* err) {
+    if (threadIdx.x != 0) return;
+    int64_t acc = 0;
+    for (int s = 0; s < n_seg; ++s) {
+        chunk_cu[s] = (int32_t)acc;
+        const int64_t a = seg_cu[s], b = seg_cu[s + 1];
+        if (a < 0 || b < a || b > n_rows) { record_error(err, MOM_DEVERR_SEGMENT, s); continue; }
+        acc += (b - a + CK - 1) / CK;
+    }
+    chunk_cu[n_seg] = (int32_t)acc;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(BW * 32)
+gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
+    constexpr int E = D / 32;
+    constexpr int TILES = D / ROWS;
+    constexpr int PW = 2 * D + 2;                // partial width
+    __shared__ float red[BW][PW];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int seg = blockIdx.x / TILES, tile = blockIdx.x % TILES, h = blockIdx.y, H = a.H;
+    const int rowt = warp * BR;                  // this warp's first row inside the tile
+    const int row0 = tile * ROWS + rowt;         // ... and inside the head
+    const T* q = reinterpret_cast<const T*>(a.q);
+    const T* k = reinterpret_cast<const T*>(a.k);
+    const T* v = reinterpret_cast<const T*>(a.v);
+    const T* dout = reinterpret_cast<const T*>(a.d_o);
+    const bool delta = a.rule == MOM_RULE_GATED_DELTA;
+
+    int64_t r0 = a.seg_cu[seg], r1 = a.seg_cu[seg + 1];
+    if (r0 < 0 || r1 < r0 || r1 > a.n_rows) r1 = r0;       // recorded by the schedule
+    const int64_t nck = (r1 - r0 + CK - 1) / CK;
+    const size_t ck_stride = (size_t)H * TILES * ROWS * D;
+    float* ck = tb.ckpt + ((size_t)tb.chunk_cu[seg] * H * TILES + (size_t)h * TILES + tile) * ROWS * D +
+                (size_t)rowt * D + lane * E;
+    float* sub = tb.sub + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * NSUB * ROWS * D + (size_t)rowt * D + lane * E;
+
+    // token t's operands; false for a bad row index (recorded, the token is skipped)
+    float kk[E], qq[E], vv[BR], dd[BR], b = 0.f, al = 1.f;
+    auto load_token = [&](int64_t r, bool want_do) -> bool {
+        const int64_t qr = a.qidx ? (int64_t)a.qidx[r] : r;
+        if (qr < 0 || qr >= a.n_q_rows) {
+            if (lane == 0 && warp == 0 && tile == 0) record_error(a.ws, MOM_DEVERR_ROW_INDEX, r);
+            return false;
+        }
+        const int64_t gr = a.gates_by_row ? r : qr;
+        load_vec<E>(k + (r * H + h) * D + lane * E, kk);
+        load_vec<E>(q + (qr * H + h) * D + lane * E, qq);
+#pragma unroll
+        for (int i = 0; i < BR; ++i) {
+            vv[i] = to_f(v[(r * H + h) * D + row0 + i]);
+            dd[i] = want_do ? to_f(dout[(r * H + h) * D + row0 + i]) : 0.f;
+        }
+        b = a.beta[gr * H + h];
+        al = expf(a.log_alpha[gr * H + h]);
+        return true;
+    };
+    // S <- one forward step at row r (S holds the state before r)
+    float S[BR][E];
+    auto step = [&](int64_t r) {
+        if (!load_token(r, false)) return;
+        float y[BR];
+#pragma unroll
+        for (int i = 0; i < BR; ++i) {
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc = fmaf(S[i][e], kk[e], acc);
+            y[i] = acc;
+        }
+        warp_sum_n<BR>(y);
+        const float dl = delta ? al : 0.f;
+#pragma unroll
+        for (int i = 0; i < BR; ++i) {
+            const float u = b * (vv[i] - dl * y[i]);
+#pragma unroll
+            for (int e = 0; e < E; ++e) S[i][e] = fmaf(al, S[i][e], u * kk[e]);
+        }
+    };
+
+    // ---- forward sweep: the rows every CK tokens
+    const size_t hoff = (((size_t)seg * H + h) * D + row0) * D + lane * E;
+#pragma unroll
+    for (int i = 0; i < BR; ++i) {
+        if (a.h0) load_vec<E>(a.h0 + hoff + (size_t)i * D, S[i]);
+        else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) S[i][e] = 0.f;
+        }
+    }
+    for (int64_t r = r0; r < r1; ++r) {
+        if ((r - r0) % CK == 0) {
+#pragma unroll
+            for (int i = 0; i < BR; ++i) store_vec<E>(ck + (size_t)((r - r0) / CK) * ck_stride + (size_t)i * D, S[i]);
+        }
+        step(r);
+    }
+
+    // ---- reverse sweep
+    float G[BR][E];
+#pragma unroll
+    for (int i = 0; i < BR; ++i) {
+        if (a.dh_final) load_vec<E>(a.dh_final + hoff + (size_t)i * D, G[i]);
+        else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) G[i][e] = 0.f;
+        }
+    }
+    for (int64_t j = nck - 1; j >= 0; --j) {
+        const int64_t t0 = r0 + j * CK, t1 = t0 + CK < r1 ? t0 + CK : r1;
+#pragma unroll
+        for (int i = 0; i < BR; ++i) load_vec<E>(ck + (size_t)j * ck_stride + (size_t)i * D, S[i]);
+        for (int64_t r = t0; r < t1; ++r) {
+            if ((r - t0) % SUB == 0) {
+#pragma unroll
+                for (int i = 0; i < BR; ++i) store_vec<E>(sub + (size_t)((r - t0) / SUB) * ROWS * D + (size_t)i * D, S[i]);
+            }
+            step(r);
+        }
+        for (int64_t t = t1 - 1; t >= t0; --t) {
+            // S(t-1): the nearest kept copy, then forward to t
+            const int64_t sb = (t - t0) / SUB, ts = t0 + sb * SUB;
+#pragma unroll
+            for (int i = 0; i < BR; ++i) load_vec<E>(sub + (size_t)sb * ROWS * D + (size_t)i * D, S[i]);
+            for (int64_t r = ts; r < t; ++r) step(r);
+            // the token's own reverse step
+            float* w = red[warp];
+            const bool ok = load_token(t, true);
+            if (ok) {
+                const float dl = delta ? al : 0.f, cab = delta ? al * b : 0.f;
+                float y[BR];
+#pragma unroll
+                for (int i = 0; i < BR; ++i) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) acc = fmaf(S[i][e], kk[e], acc);
+                    y[i] = acc;
+                }
+                warp_sum_n<BR>(y);
+                float u[BR], dq[E], dk[E];
+#pragma unroll
+                for (int e = 0; e < E; ++e) { dq[e] = 0.f; dk[e] = 0.f; }
+                float red2[2 * BR];                      // G.k, G.S(t-1) per row
+#pragma unroll
+                for (int i = 0; i < BR; ++i) {
+                    u[i] = b * (vv[i] - dl * y[i]);
+                    const float sq = dd[i] * a.scale;
+                    float gk = 0.f, gs = 0.f;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        G[i][e] = fmaf(sq, qq[e], G[i][e]);
+                        const float st = fmaf(al, S[i][e], u[i] * kk[e]);     // S(t)
+                        dq[e] = fmaf(sq, st, dq[e]);
+                        gk = fmaf(G[i][e], kk[e], gk);
+                        gs = fmaf(G[i][e], S[i][e], gs);
+                    }
+                    red2[2 * i] = gk;
+                    red2[2 * i + 1] = gs;
+                }
+                warp_sum_n<2 * BR>(red2);
+                float dalpha = 0.f, dbeta = 0.f;
+#pragma unroll
+                for (int i = 0; i < BR; ++i) {
+                    const float gk = red2[2 * i], gs = red2[2 * i + 1];
+                    dbeta += (vv[i] - dl * y[i]) * gk;
+                    dalpha += gs - (delta ? b * y[i] * gk : 0.f);
+                    if (lane == i) a.dv[(t * H + h) * D + row0 + i] = b * gk;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        dk[e] = fmaf(u[i], G[i][e], dk[e]) - cab * gk * S[i][e];
+                        G[i][e] = al * G[i][e] - cab * gk * kk[e];
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) { w[lane * E + e] = dq[e]; w[D + lane * E + e] = dk[e]; }
+                if (lane == 0) { w[2 * D] = al * dalpha; w[2 * D + 1] = dbeta; }
+            } else {
+                for (int c = lane; c < PW; c += 32) w[c] = 0.f;
+            }
+            __syncthreads();
+            float* pout = tb.part + (((size_t)tile * a.n_rows + t) * H + h) * PW;
+            for (int c = threadIdx.x; c < PW; c += BW * 32) {
+                float acc = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < BW; ++ww) acc += red[ww][c];
+                pout[c] = acc;
+            }
+            __syncthreads();
+        }
+    }
+    if (a.dh0) {
+#pragma unroll
+        for (int i = 0; i < BR; ++i) store_vec<E>(a.dh0 + hoff + (size_t)i * D, G[i]);
+    }
+}
+
+// Adds the per-tile partials of every row inside the segments.
+template <int D>
+__global__ void __launch_bounds__(256)
+bwd_reduce_kernel(GdnBwdArgs a, BwdTables tb) {
+    constexpr int TILES = D / ROWS, PW = 2 * D + 2;
+    const int64_t lo = a.seg_cu[0], hi = a.seg_cu[a.n_seg];
+    if (lo < 0 || hi < lo || hi > a.n_rows) return;
+    const int64_t total = (hi - lo) * a.H * PW;
+    const size_t tile_stride = (size_t)a.n_rows * a.H * PW;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rh = i / PW, c = i - rh * PW;
+        const int64_t r = lo + rh / a.H, h = rh % a.H;
+        const size_t off = ((size_t)r * a.H + h) * PW + c;
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < TILES; ++t) acc += tb.part[t * tile_stride + off];
+        if (c < D) a.dq[((size_t)r * a.H + h) * D + c] = acc;
+        else if (c < 2 * D) a.dk[((size_t)r * a.H + h) * D + (c - D)] = acc;
+        else if (c == 2 * D) a.dlog_alpha[(size_t)r * a.H + h] = acc;
+        else a.dbeta[(size_t)r * a.H + h] = acc;
+    }
+}
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct BwdLayout {
+    size_t chunk_cu, ckpt, sub, part, total;
+};
+
+BwdLayout bwd_layout(int64_t n_rows, int n_seg, int H, int d) {
+    BwdLayout L;
+    const int tiles = d / ROWS;
+    const size_t max_chunks = (size_t)(n_rows / CK) + (size_t)n_seg;
+    size_t off = MOM_WS_HEADER_BYTES;
+    auto take = [&](size_t bytes) { size_t o = off; off += up256(bytes); return o; };
+    L.chunk_cu = take(((size_t)n_seg + 1) * 4);
+    L.ckpt = take(max_chunks * H * tiles * ROWS * (size_t)d * 4);
+    L.sub = take((size_t)n_seg * tiles * H * NSUB * ROWS * (size_t)d * 4);
+    L.part = take((size_t)tiles * n_rows * H * (2 * (size_t)d + 2) * 4);
+    L.total = off;
+    return L;
+}
+
+template <typename T, int D>
+cudaError_t launch_bwd_t(const GdnBwdArgs& a, cudaStream_t st) {
+    const BwdLayout L = bwd_layout(a.n_rows, a.n_seg, a.H, a.d);
+    unsigned char* base = reinterpret_cast<unsigned char*>(a.ws);
+    BwdTables tb{reinterpret_cast<int32_t*>(base + L.chunk_cu), reinterpret_cast<float*>(base + L.ckpt),
+                 reinterpret_cast<float*>(base + L.sub), reinterpret_cast<float*>(base + L.part)};
+    bwd_schedule_kernel<<<1, 32, 0, st>>>(a.seg_cu, a.n_seg, a.n_rows, tb.chunk_cu, a.ws);
+    dim3 grid((unsigned)a.n_seg * (D / ROWS), a.H);
+    gdn_bwd_kernel<T, D><<<grid, BW * 32, 0, st>>>(a, tb);
+    const int64_t work = a.n_rows * a.H * (2 * D + 2);
+    const int64_t want = cdiv(work, 256);
+    bwd_reduce_kernel<D><<<(unsigned)(want < 148 * 32 ? (want > 0 ? want : 1) : 148 * 32), 256, 0, st>>>(a, tb);
+    count_launches(3);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gdn_bwd_ws_bytes(int64_t n_rows, int n_seg, int H, int d) { return bwd_layout(n_rows, n_seg, H, d).total; }
+
+cudaError_t launch_gdn_bwd(const GdnBwdArgs& a, int dt, cudaStream_t st) {
+    if (a.n_seg == 0) return cudaSuccess;
+    if (dt == MOM_BF16) {
+        switch (a.d) {
+            case 64: return launch_bwd_t<bf16, 64>(a, st);
+            case 128: return launch_bwd_t<bf16, 128>(a, st);
+            case 256: return launch_bwd_t<bf16, 256>(a, st);
+        }
+    } else {
+        switch (a.d) {
+            case 64: return launch_bwd_t<float, 64>(a, st);
+            case 128: return launch_bwd_t<float, 128>(a, st);
+            case 256: return launch_bwd_t<float, 256>(a, st);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace mom

@@ -117,6 +117,35 @@ struct GdnArgs {
 };
 cudaError_t launch_gdn_recurrent(const GdnArgs& a, int dt, cudaStream_t st);
 
+// gdn_bwd.cu: reverse pass of the recurrence (both rules), token-serial fp32
+struct GdnBwdArgs {
+    const void* q;
+    const int32_t* qidx;
+    const void* k;
+    const void* v;
+    const float* beta;
+    const float* log_alpha;
+    const int32_t* seg_cu;
+    int n_seg;
+    int64_t n_rows, n_q_rows;
+    int H, d;
+    float scale;
+    int rule;
+    int gates_by_row;
+    const float* h0;          // [n_seg, H, d, d] or null
+    const void* d_o;          // [n_rows, H, d] (dt)
+    const float* dh_final;    // [n_seg, H, d, d] or null
+    float* dq;                // [n_rows, H, d], per row
+    float* dk;
+    float* dv;
+    float* dbeta;             // [n_rows, H], per row
+    float* dlog_alpha;
+    float* dh0;               // [n_seg, H, d, d] or null
+    void* ws;
+};
+size_t gdn_bwd_ws_bytes(int64_t n_rows, int n_seg, int H, int d);
+cudaError_t launch_gdn_bwd(const GdnBwdArgs& a, int dt, cudaStream_t st);
+
 // gdn_chunk_tc.cu: chunked Gated DeltaNet on the tcgen05 tensor cores (bf16)
 bool gdn_tc_supported(const GdnArgs& a, int dt);
 size_t gdn_tc_ws_bytes(int64_t n_rows, int n_seg, int H, int d);
