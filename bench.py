@@ -406,6 +406,7 @@ def gpu_arm(args):
     if not args.no_configs and world == 1:
         configs = {extra_key(name, rule, mg): config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule, mg)
                    for name, rule, mg in EXTRA}
+        configs["recurrence_backward"] = backward_bench(lay, w, x, cu, flush)
     clocks.__exit__(None, None, None)
     layer_roof["near_tie_tokens"] = near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)
     return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,
@@ -485,6 +486,54 @@ def finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call,
     if world > 1:
         dist.destroy_process_group()
     return result
+
+
+def backward_bench(lay, w, x, cu, flush, steps=3):
+    """The reverse pass of the layer's two recurrence problems (the shared
+    memory over every token, the routed memories over their segments) on the
+    layer's own q, k, v and gates, with a random output gradient: the first
+    GPU path of the backward (token-serial float32 on CUDA cores)."""
+    import torch
+    from mixture_memories_layer_b200 import binding as B
+    S = cu.numel() - 1
+    b = lay.forward(x, cu)
+    H, d = w.heads, w.d_head
+    probs = {"shared": (b["q"], None, b["k_sh"], b["v_sh"], cu), "routed": (b["q"], b["perm"], b["k_p"], b["v_p"],
+                                                                          b["seg_cu"])}
+    out = {"workload": "reverse pass of the %s layer's recurrences (shared + routed), dout ~ N(0,1)" % w.name,
+           "path": "token-serial float32 on CUDA cores, states kept every 64 tokens and re-walked every 8"}
+    total = 0.0
+    g = torch.Generator(device=x.device).manual_seed(1)
+    for name, (q, qidx, k, v, seg) in probs.items():
+        n = k.shape[0]
+        do = torch.randn((n, H, d), device=x.device, generator=g).to(x.dtype)
+        bufs = [torch.empty((n, H, d), device=x.device) for _ in range(3)] + \
+               [torch.empty((n, H), device=x.device) for _ in range(2)]
+        dh0 = torch.empty((seg.numel() - 1, H, d, d), device=x.device)
+        ws = B.new_workspace(B.mom_memory_chunk_bwd_workspace_size(n, seg.numel() - 1, H, d), x.device)
+        call = lambda: B.mom_memory_chunk_bwd(q, qidx, k, v, b["beta"], b["log_alpha"], seg, lay.scale, lay.rule,
+                                              None, do, None, *bufs, dh0, ws)
+        call()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        code, _ = B.mom_get_error(ws)
+        if code:
+            raise SystemExit("device error record in the recurrence reverse pass (%s): %d" % (name, code))
+        out[name + "_ms"] = sum(ms) / steps
+        total += out[name + "_ms"]
+        del ws, bufs, dh0
+    out["ms"] = total
+    out["value"] = w.n_tokens / (total / 1e3)
+    out["unit"] = UNIT
+    return out
 
 
 def decode_bench(args, dev, world, rank, max_over_ranks, barrier):

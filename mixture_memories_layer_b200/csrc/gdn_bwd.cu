@@ -19,7 +19,10 @@
 // reverse pass needs S(t-1) at every token: a forward sweep stores the rows
 // every 64 tokens; the chunks are then walked backwards, each recomputed from
 // its stored state with a copy kept every 8 tokens, and the state before a
-// token is rebuilt from the nearest copy (at most 7 steps).  The sums over
+// token is rebuilt from the nearest copy (at most 7 steps).  The operands of
+// each 8-token block (k, q, the CTA's v and d_o, the gates) are loaded once
+// by the whole CTA into shared memory, so the replayed steps never wait on
+// L2.  The sums over
 // rows are reduced inside the CTA per token and written as one partial per
 // 64-row tile, which a second kernel adds up (deterministic, no atomics).
 #include "common.cuh"
@@ -55,13 +58,38 @@ __global__ void bwd_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_se
     chunk_cu[n_seg] = (int32_t)acc;
 }
 
+template <int D>
+struct BwdSmem {
+    static constexpr int PW = 2 * D + 2;                      // partial width: dq | dk | dlog_alpha | dbeta
+    static constexpr int RED = 0;                             // [BW][PW] per-warp sums over rows
+    static constexpr int KC = RED + BW * PW;                  // [SUB][D] k of the cached tokens
+    static constexpr int QC = KC + SUB * D;                   // [SUB][D] q
+    static constexpr int VC = QC + SUB * D;                   // [SUB][ROWS] v of this CTA's rows
+    static constexpr int DC = VC + SUB * ROWS;                // [SUB][ROWS] d_o
+    static constexpr int BC = DC + SUB * ROWS;                // [SUB] beta
+    static constexpr int AC = BC + SUB;                       // [SUB] alpha
+    static constexpr int OKC = AC + SUB;                      // [SUB] 1: the token's row index is valid
+    static constexpr int FLOATS = OKC + SUB;
+    static constexpr size_t BYTES = (size_t)FLOATS * 4;
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(BW * 32)
 gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
+    using SM = BwdSmem<D>;
     constexpr int E = D / 32;
     constexpr int TILES = D / ROWS;
-    constexpr int PW = 2 * D + 2;                // partial width
-    __shared__ float red[BW][PW];
+    constexpr int PW = SM::PW;
+    constexpr int NT = BW * 32;
+    extern __shared__ float smf[];
+    float* red = smf + SM::RED;
+    float* kc = smf + SM::KC;
+    float* qc = smf + SM::QC;
+    float* vc = smf + SM::VC;
+    float* dc = smf + SM::DC;
+    float* bc = smf + SM::BC;
+    float* ac = smf + SM::AC;
+    float* okc = smf + SM::OKC;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int seg = blockIdx.x / TILES, tile = blockIdx.x % TILES, h = blockIdx.y, H = a.H;
     const int rowt = warp * BR;                  // this warp's first row inside the tile
@@ -80,30 +108,44 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
                 (size_t)rowt * D + lane * E;
     float* sub = tb.sub + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * NSUB * ROWS * D + (size_t)rowt * D + lane * E;
 
-    // token t's operands; false for a bad row index (recorded, the token is skipped)
-    float kk[E], qq[E], vv[BR], dd[BR], b = 0.f, al = 1.f;
-    auto load_token = [&](int64_t r, bool want_do) -> bool {
-        const int64_t qr = a.qidx ? (int64_t)a.qidx[r] : r;
-        if (qr < 0 || qr >= a.n_q_rows) {
-            if (lane == 0 && warp == 0 && tile == 0) record_error(a.ws, MOM_DEVERR_ROW_INDEX, r);
-            return false;
+    // the operands of tokens ts .. ts+n-1 (n <= SUB) into shared memory, by
+    // the whole CTA (every replay and reverse step then reads them from there)
+    auto fill = [&](int64_t ts, int n, bool want_do) {
+        __syncthreads();                                      // the previous block's readers are done
+        for (int i = threadIdx.x; i < n; i += NT) {
+            const int64_t r = ts + i;
+            const int64_t qr = a.qidx ? (int64_t)a.qidx[r] : r;
+            const bool ok = qr >= 0 && qr < a.n_q_rows;
+            if (!ok && tile == 0) record_error(a.ws, MOM_DEVERR_ROW_INDEX, r);
+            const int64_t gr = a.gates_by_row ? r : qr;
+            okc[i] = ok ? 1.f : 0.f;
+            bc[i] = ok ? a.beta[gr * H + h] : 0.f;
+            ac[i] = ok ? expf(a.log_alpha[gr * H + h]) : 1.f;
         }
-        const int64_t gr = a.gates_by_row ? r : qr;
-        load_vec<E>(k + (r * H + h) * D + lane * E, kk);
-        load_vec<E>(q + (qr * H + h) * D + lane * E, qq);
-#pragma unroll
-        for (int i = 0; i < BR; ++i) {
-            vv[i] = to_f(v[(r * H + h) * D + row0 + i]);
-            dd[i] = want_do ? to_f(dout[(r * H + h) * D + row0 + i]) : 0.f;
+        for (int i = threadIdx.x; i < n * D; i += NT) {
+            const int j = i / D, c = i - j * D;
+            const int64_t r = ts + j;
+            const int64_t qr = a.qidx ? (int64_t)a.qidx[r] : r;
+            const bool ok = qr >= 0 && qr < a.n_q_rows;
+            kc[j * D + c] = to_f(k[(r * H + h) * D + c]);
+            qc[j * D + c] = ok ? to_f(q[(qr * H + h) * D + c]) : 0.f;
         }
-        b = a.beta[gr * H + h];
-        al = expf(a.log_alpha[gr * H + h]);
-        return true;
+        for (int i = threadIdx.x; i < n * ROWS; i += NT) {
+            const int j = i / ROWS, c = i - j * ROWS;
+            const int64_t off = ((ts + j) * H + h) * D + tile * ROWS + c;
+            vc[j * ROWS + c] = to_f(v[off]);
+            dc[j * ROWS + c] = want_do ? to_f(dout[off]) : 0.f;
+        }
+        __syncthreads();
     };
-    // S <- one forward step at row r (S holds the state before r)
+
+    // S <- one forward step at cached token j (S holds the state before it)
     float S[BR][E];
-    auto step = [&](int64_t r) {
-        if (!load_token(r, false)) return;
+    auto step = [&](int j) {
+        if (okc[j] == 0.f) return;
+        float kk[E];
+        load_vec<E>(kc + j * D + lane * E, kk);
+        const float b = bc[j], al = ac[j];
         float y[BR];
 #pragma unroll
         for (int i = 0; i < BR; ++i) {
@@ -116,7 +158,7 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
         const float dl = delta ? al : 0.f;
 #pragma unroll
         for (int i = 0; i < BR; ++i) {
-            const float u = b * (vv[i] - dl * y[i]);
+            const float u = b * (vc[j * ROWS + rowt + i] - dl * y[i]);
 #pragma unroll
             for (int e = 0; e < E; ++e) S[i][e] = fmaf(al, S[i][e], u * kk[e]);
         }
@@ -132,12 +174,14 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
             for (int e = 0; e < E; ++e) S[i][e] = 0.f;
         }
     }
-    for (int64_t r = r0; r < r1; ++r) {
-        if ((r - r0) % CK == 0) {
+    for (int64_t ts = r0; ts < r1; ts += SUB) {
+        const int n = (int)(r1 - ts < SUB ? r1 - ts : SUB);
+        fill(ts, n, false);
+        if ((ts - r0) % CK == 0) {
 #pragma unroll
-            for (int i = 0; i < BR; ++i) store_vec<E>(ck + (size_t)((r - r0) / CK) * ck_stride + (size_t)i * D, S[i]);
+            for (int i = 0; i < BR; ++i) store_vec<E>(ck + (size_t)((ts - r0) / CK) * ck_stride + (size_t)i * D, S[i]);
         }
-        step(r);
+        for (int j = 0; j < n; ++j) step(j);
     }
 
     // ---- reverse sweep
@@ -150,86 +194,96 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
             for (int e = 0; e < E; ++e) G[i][e] = 0.f;
         }
     }
-    for (int64_t j = nck - 1; j >= 0; --j) {
-        const int64_t t0 = r0 + j * CK, t1 = t0 + CK < r1 ? t0 + CK : r1;
+    float* w = red + warp * PW;
+    for (int64_t jc = nck - 1; jc >= 0; --jc) {
+        const int64_t t0 = r0 + jc * CK, t1 = t0 + CK < r1 ? t0 + CK : r1;
 #pragma unroll
-        for (int i = 0; i < BR; ++i) load_vec<E>(ck + (size_t)j * ck_stride + (size_t)i * D, S[i]);
-        for (int64_t r = t0; r < t1; ++r) {
-            if ((r - t0) % SUB == 0) {
+        for (int i = 0; i < BR; ++i) load_vec<E>(ck + (size_t)jc * ck_stride + (size_t)i * D, S[i]);
+        for (int64_t ts = t0; ts < t1; ts += SUB) {
+            const int n = (int)(t1 - ts < SUB ? t1 - ts : SUB);
+            fill(ts, n, false);
 #pragma unroll
-                for (int i = 0; i < BR; ++i) store_vec<E>(sub + (size_t)((r - t0) / SUB) * ROWS * D + (size_t)i * D, S[i]);
-            }
-            step(r);
+            for (int i = 0; i < BR; ++i) store_vec<E>(sub + (size_t)((ts - t0) / SUB) * ROWS * D + (size_t)i * D, S[i]);
+            for (int j = 0; j < n; ++j) step(j);
         }
-        for (int64_t t = t1 - 1; t >= t0; --t) {
-            // S(t-1): the nearest kept copy, then forward to t
-            const int64_t sb = (t - t0) / SUB, ts = t0 + sb * SUB;
+        const int nsb = (int)((t1 - t0 + SUB - 1) / SUB);
+        for (int sb = nsb - 1; sb >= 0; --sb) {
+            const int64_t ts = t0 + (int64_t)sb * SUB;
+            const int n = (int)(t1 - ts < SUB ? t1 - ts : SUB);
+            fill(ts, n, true);
+            for (int jt = n - 1; jt >= 0; --jt) {
+                const int64_t t = ts + jt;
+                // S(t-1): the block's kept copy, then forward to t
 #pragma unroll
-            for (int i = 0; i < BR; ++i) load_vec<E>(sub + (size_t)sb * ROWS * D + (size_t)i * D, S[i]);
-            for (int64_t r = ts; r < t; ++r) step(r);
-            // the token's own reverse step
-            float* w = red[warp];
-            const bool ok = load_token(t, true);
-            if (ok) {
-                const float dl = delta ? al : 0.f, cab = delta ? al * b : 0.f;
-                float y[BR];
+                for (int i = 0; i < BR; ++i) load_vec<E>(sub + (size_t)sb * ROWS * D + (size_t)i * D, S[i]);
+                for (int j = 0; j < jt; ++j) step(j);
+                // the token's own reverse step
+                if (okc[jt] != 0.f) {
+                    float kk[E], qq[E];
+                    load_vec<E>(kc + jt * D + lane * E, kk);
+                    load_vec<E>(qc + jt * D + lane * E, qq);
+                    const float b = bc[jt], al = ac[jt];
+                    const float dl = delta ? al : 0.f, cab = delta ? al * b : 0.f;
+                    float y[BR], vv[BR];
 #pragma unroll
-                for (int i = 0; i < BR; ++i) {
+                    for (int i = 0; i < BR; ++i) {
+                        vv[i] = vc[jt * ROWS + rowt + i];
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < E; ++e) acc = fmaf(S[i][e], kk[e], acc);
+                        y[i] = acc;
+                    }
+                    warp_sum_n<BR>(y);
+                    float u[BR], dq[E], dk[E];
+#pragma unroll
+                    for (int e = 0; e < E; ++e) { dq[e] = 0.f; dk[e] = 0.f; }
+                    float red2[2 * BR];                   // G.k, G.S(t-1) per row
+#pragma unroll
+                    for (int i = 0; i < BR; ++i) {
+                        u[i] = b * (vv[i] - dl * y[i]);
+                        const float sq = dc[jt * ROWS + rowt + i] * a.scale;
+                        float gk = 0.f, gs = 0.f;
+#pragma unroll
+                        for (int e = 0; e < E; ++e) {
+                            G[i][e] = fmaf(sq, qq[e], G[i][e]);
+                            const float st = fmaf(al, S[i][e], u[i] * kk[e]);     // S(t)
+                            dq[e] = fmaf(sq, st, dq[e]);
+                            gk = fmaf(G[i][e], kk[e], gk);
+                            gs = fmaf(G[i][e], S[i][e], gs);
+                        }
+                        red2[2 * i] = gk;
+                        red2[2 * i + 1] = gs;
+                    }
+                    warp_sum_n<2 * BR>(red2);
+                    float dalpha = 0.f, dbeta = 0.f;
+#pragma unroll
+                    for (int i = 0; i < BR; ++i) {
+                        const float gk = red2[2 * i], gs = red2[2 * i + 1];
+                        dbeta += (vv[i] - dl * y[i]) * gk;
+                        dalpha += gs - (delta ? b * y[i] * gk : 0.f);
+                        if (lane == i) a.dv[(t * H + h) * D + row0 + i] = b * gk;
+#pragma unroll
+                        for (int e = 0; e < E; ++e) {
+                            dk[e] = fmaf(u[i], G[i][e], dk[e]) - cab * gk * S[i][e];
+                            G[i][e] = al * G[i][e] - cab * gk * kk[e];
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < E; ++e) { w[lane * E + e] = dq[e]; w[D + lane * E + e] = dk[e]; }
+                    if (lane == 0) { w[2 * D] = al * dalpha; w[2 * D + 1] = dbeta; }
+                } else {
+                    for (int c = lane; c < PW; c += 32) w[c] = 0.f;
+                }
+                __syncthreads();
+                float* pout = tb.part + (((size_t)tile * a.n_rows + t) * H + h) * PW;
+                for (int c = threadIdx.x; c < PW; c += NT) {
                     float acc = 0.f;
 #pragma unroll
-                    for (int e = 0; e < E; ++e) acc = fmaf(S[i][e], kk[e], acc);
-                    y[i] = acc;
+                    for (int ww = 0; ww < BW; ++ww) acc += red[ww * PW + c];
+                    pout[c] = acc;
                 }
-                warp_sum_n<BR>(y);
-                float u[BR], dq[E], dk[E];
-#pragma unroll
-                for (int e = 0; e < E; ++e) { dq[e] = 0.f; dk[e] = 0.f; }
-                float red2[2 * BR];                      // G.k, G.S(t-1) per row
-#pragma unroll
-                for (int i = 0; i < BR; ++i) {
-                    u[i] = b * (vv[i] - dl * y[i]);
-                    const float sq = dd[i] * a.scale;
-                    float gk = 0.f, gs = 0.f;
-#pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        G[i][e] = fmaf(sq, qq[e], G[i][e]);
-                        const float st = fmaf(al, S[i][e], u[i] * kk[e]);     // S(t)
-                        dq[e] = fmaf(sq, st, dq[e]);
-                        gk = fmaf(G[i][e], kk[e], gk);
-                        gs = fmaf(G[i][e], S[i][e], gs);
-                    }
-                    red2[2 * i] = gk;
-                    red2[2 * i + 1] = gs;
-                }
-                warp_sum_n<2 * BR>(red2);
-                float dalpha = 0.f, dbeta = 0.f;
-#pragma unroll
-                for (int i = 0; i < BR; ++i) {
-                    const float gk = red2[2 * i], gs = red2[2 * i + 1];
-                    dbeta += (vv[i] - dl * y[i]) * gk;
-                    dalpha += gs - (delta ? b * y[i] * gk : 0.f);
-                    if (lane == i) a.dv[(t * H + h) * D + row0 + i] = b * gk;
-#pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        dk[e] = fmaf(u[i], G[i][e], dk[e]) - cab * gk * S[i][e];
-                        G[i][e] = al * G[i][e] - cab * gk * kk[e];
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < E; ++e) { w[lane * E + e] = dq[e]; w[D + lane * E + e] = dk[e]; }
-                if (lane == 0) { w[2 * D] = al * dalpha; w[2 * D + 1] = dbeta; }
-            } else {
-                for (int c = lane; c < PW; c += 32) w[c] = 0.f;
+                __syncthreads();
             }
-            __syncthreads();
-            float* pout = tb.part + (((size_t)tile * a.n_rows + t) * H + h) * PW;
-            for (int c = threadIdx.x; c < PW; c += BW * 32) {
-                float acc = 0.f;
-#pragma unroll
-                for (int ww = 0; ww < BW; ++ww) acc += red[ww][c];
-                pout[c] = acc;
-            }
-            __syncthreads();
         }
     }
     if (a.dh0) {
@@ -287,9 +341,12 @@ cudaError_t launch_bwd_t(const GdnBwdArgs& a, cudaStream_t st) {
     unsigned char* base = reinterpret_cast<unsigned char*>(a.ws);
     BwdTables tb{reinterpret_cast<int32_t*>(base + L.chunk_cu), reinterpret_cast<float*>(base + L.ckpt),
                  reinterpret_cast<float*>(base + L.sub), reinterpret_cast<float*>(base + L.part)};
+    static unsigned long long optin_done = 0;
+    cudaError_t e = smem_optin((const void*)gdn_bwd_kernel<T, D>, (int)BwdSmem<D>::BYTES, &optin_done);
+    if (e != cudaSuccess) return e;
     bwd_schedule_kernel<<<1, 32, 0, st>>>(a.seg_cu, a.n_seg, a.n_rows, tb.chunk_cu, a.ws);
     dim3 grid((unsigned)a.n_seg * (D / ROWS), a.H);
-    gdn_bwd_kernel<T, D><<<grid, BW * 32, 0, st>>>(a, tb);
+    gdn_bwd_kernel<T, D><<<grid, BW * 32, BwdSmem<D>::BYTES, st>>>(a, tb);
     const int64_t work = a.n_rows * a.H * (2 * D + 2);
     const int64_t want = cdiv(work, 256);
     bwd_reduce_kernel<D><<<(unsigned)(want < 148 * 32 ? (want > 0 ? want : 1) : 148 * 32), 256, 0, st>>>(a, tb);
