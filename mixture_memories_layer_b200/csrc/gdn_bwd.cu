@@ -18,9 +18,9 @@
 // lane holding d/32 columns of each, as in the token-serial forward.  The
 // reverse pass needs S(t-1) at every token: a forward sweep stores the rows
 // every 64 tokens; the chunks are then walked backwards, each recomputed from
-// its stored state with a copy kept every 8 tokens, and the state before a
-// token is rebuilt from the nearest copy (at most 7 steps).  The operands of
-// each 8-token block (k, q, the CTA's v and d_o, the gates) are loaded once
+// its stored state with a copy kept every 4 tokens, and the state before a
+// token is rebuilt from the nearest copy (at most 3 steps).  The operands of
+// each 16-token block (k, q, the CTA's v and d_o, the gates) are loaded once
 // by the whole CTA into shared memory, so the replayed steps never wait on
 // L2.  The sums over
 // rows are reduced inside the CTA per token and written as one partial per
@@ -35,8 +35,9 @@ constexpr int BR = 4;               // state rows per warp
 constexpr int BW = 16;              // warps per CTA
 constexpr int ROWS = BR * BW;       // state rows per CTA
 constexpr int CK = 64;              // tokens between stored states
-constexpr int SUB = 8;              // tokens between the copies kept inside a chunk
+constexpr int SUB = 4;              // tokens between the copies kept inside a chunk
 constexpr int NSUB = CK / SUB;
+constexpr int CACHE = 16;           // tokens whose operands one fill brings into shared memory
 
 struct BwdTables {
     int32_t* chunk_cu;   // [n_seg + 1] first stored state of each segment
@@ -62,14 +63,14 @@ template <int D>
 struct BwdSmem {
     static constexpr int PW = 2 * D + 2;                      // partial width: dq | dk | dlog_alpha | dbeta
     static constexpr int RED = 0;                             // [BW][PW] per-warp sums over rows
-    static constexpr int KC = RED + BW * PW;                  // [SUB][D] k of the cached tokens
-    static constexpr int QC = KC + SUB * D;                   // [SUB][D] q
-    static constexpr int VC = QC + SUB * D;                   // [SUB][ROWS] v of this CTA's rows
-    static constexpr int DC = VC + SUB * ROWS;                // [SUB][ROWS] d_o
-    static constexpr int BC = DC + SUB * ROWS;                // [SUB] beta
-    static constexpr int AC = BC + SUB;                       // [SUB] alpha
-    static constexpr int OKC = AC + SUB;                      // [SUB] 1: the token's row index is valid
-    static constexpr int FLOATS = OKC + SUB;
+    static constexpr int KC = RED + BW * PW;                  // [CACHE][D] k of the cached tokens
+    static constexpr int QC = KC + CACHE * D;                 // [CACHE][D] q
+    static constexpr int VC = QC + CACHE * D;                 // [CACHE][ROWS] v of this CTA's rows
+    static constexpr int DC = VC + CACHE * ROWS;              // [CACHE][ROWS] d_o
+    static constexpr int BC = DC + CACHE * ROWS;              // [CACHE] beta
+    static constexpr int AC = BC + CACHE;                     // [CACHE] alpha
+    static constexpr int OKC = AC + CACHE;                    // [CACHE] 1: the token's row index is valid
+    static constexpr int FLOATS = OKC + CACHE;
     static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 
@@ -108,7 +109,7 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
                 (size_t)rowt * D + lane * E;
     float* sub = tb.sub + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * NSUB * ROWS * D + (size_t)rowt * D + lane * E;
 
-    // the operands of tokens ts .. ts+n-1 (n <= SUB) into shared memory, by
+    // the operands of tokens ts .. ts+n-1 (n <= CACHE) into shared memory, by
     // the whole CTA (every replay and reverse step then reads them from there)
     auto fill = [&](int64_t ts, int n, bool want_do) {
         __syncthreads();                                      // the previous block's readers are done
@@ -174,8 +175,8 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
             for (int e = 0; e < E; ++e) S[i][e] = 0.f;
         }
     }
-    for (int64_t ts = r0; ts < r1; ts += SUB) {
-        const int n = (int)(r1 - ts < SUB ? r1 - ts : SUB);
+    for (int64_t ts = r0; ts < r1; ts += CACHE) {
+        const int n = (int)(r1 - ts < CACHE ? r1 - ts : CACHE);
         fill(ts, n, false);
         if ((ts - r0) % CK == 0) {
 #pragma unroll
@@ -199,24 +200,31 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
         const int64_t t0 = r0 + jc * CK, t1 = t0 + CK < r1 ? t0 + CK : r1;
 #pragma unroll
         for (int i = 0; i < BR; ++i) load_vec<E>(ck + (size_t)jc * ck_stride + (size_t)i * D, S[i]);
-        for (int64_t ts = t0; ts < t1; ts += SUB) {
-            const int n = (int)(t1 - ts < SUB ? t1 - ts : SUB);
-            fill(ts, n, false);
+        for (int64_t tc = t0; tc < t1; tc += CACHE) {
+            const int n = (int)(t1 - tc < CACHE ? t1 - tc : CACHE);
+            fill(tc, n, false);
+            for (int j = 0; j < n; ++j) {
+                if (j % SUB == 0) {
 #pragma unroll
-            for (int i = 0; i < BR; ++i) store_vec<E>(sub + (size_t)((ts - t0) / SUB) * ROWS * D + (size_t)i * D, S[i]);
-            for (int j = 0; j < n; ++j) step(j);
+                    for (int i = 0; i < BR; ++i)
+                        store_vec<E>(sub + (size_t)((tc + j - t0) / SUB) * ROWS * D + (size_t)i * D, S[i]);
+                }
+                step(j);
+            }
         }
-        const int nsb = (int)((t1 - t0 + SUB - 1) / SUB);
-        for (int sb = nsb - 1; sb >= 0; --sb) {
-            const int64_t ts = t0 + (int64_t)sb * SUB;
-            const int n = (int)(t1 - ts < SUB ? t1 - ts : SUB);
-            fill(ts, n, true);
+        const int ncb = (int)((t1 - t0 + CACHE - 1) / CACHE);
+        for (int cb = ncb - 1; cb >= 0; --cb) {
+            const int64_t tc = t0 + (int64_t)cb * CACHE;
+            const int n = (int)(t1 - tc < CACHE ? t1 - tc : CACHE);
+            fill(tc, n, true);
             for (int jt = n - 1; jt >= 0; --jt) {
-                const int64_t t = ts + jt;
-                // S(t-1): the block's kept copy, then forward to t
+                const int64_t t = tc + jt;
+                // S(t-1): the nearest kept copy, then forward to t
+                const int js = jt - jt % SUB;
 #pragma unroll
-                for (int i = 0; i < BR; ++i) load_vec<E>(sub + (size_t)sb * ROWS * D + (size_t)i * D, S[i]);
-                for (int j = 0; j < jt; ++j) step(j);
+                for (int i = 0; i < BR; ++i)
+                    load_vec<E>(sub + (size_t)((tc + js - t0) / SUB) * ROWS * D + (size_t)i * D, S[i]);
+                for (int j = js; j < jt; ++j) step(j);
                 // the token's own reverse step
                 if (okc[jt] != 0.f) {
                     float kk[E], qq[E];
