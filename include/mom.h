@@ -231,10 +231,13 @@ mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const i
 
 /* mom_proj_shared -- the shared projections of mom_kv_proj_grouped alone
  * (q, k_sh, v_sh), which need no routing: a memory-parallel layer runs them
- * on the tokens' own rank.  Arguments as in mom_kv_proj_grouped.
+ * on the tokens' own rank.  Arguments as in mom_kv_proj_grouped; q_norm and
+ * k_sh_norm [n_tok, H] float32 or NULL receive sqrt(|z|^2 + 1e-6) of every
+ * (token, head) before its L2 norm (what the norm's backward needs).
  * ws: mom_kv_proj_workspace_size(n_tok, d_model, H, d, 1, 1). */
 mom_status mom_proj_shared(const void* x, const void* w_shared, mom_dtype dt, int64_t n_tok, int d_model,
-                           int H, int d, void* q, void* k_sh, void* v_sh, void* ws, size_t ws_bytes, void* stream);
+                           int H, int d, void* q, void* k_sh, void* v_sh, float* q_norm, float* k_sh_norm,
+                           void* ws, size_t ws_bytes, void* stream);
 
 /* mom_kv_proj_groups -- the routed key/value projections over an explicit
  * group table: the rows a memory-parallel layer receives, grouped by
@@ -244,14 +247,15 @@ mom_status mom_proj_shared(const void* x, const void* w_shared, mom_dtype dt, in
  * group_mem[g]'s weights (0 <= group_mem[g] < n_mem):
  *   k_p[r] = l2norm_h(x[perm_token[r]] W_k^m^T),  v_p[r] = x[perm_token[r]] W_v^m^T
  * with perm_token NULL meaning row r reads x row r.  x [n_x, d_model];
- * w_kv [n_mem, 2*H*d, d_model]; k_p, v_p [n_rows, H, d] (dt); rows past
- * group_offset[n_groups] are not written.  A corrupt table or index is
- * recorded in ws (MOM_DEVERR_*) and the affected tiles are skipped.
- * ws: at least MOM_WS_HEADER_BYTES. */
+ * w_kv [n_mem, 2*H*d, d_model]; k_p, v_p [n_rows, H, d] (dt); k_norm
+ * [n_rows, H] float32 or NULL receives sqrt(|z|^2 + 1e-6) of every (row,
+ * head) of k before its norm.  Rows past group_offset[n_groups] are not
+ * written.  A corrupt table or index is recorded in ws (MOM_DEVERR_*) and
+ * the affected tiles are skipped.  ws: at least MOM_WS_HEADER_BYTES. */
 mom_status mom_kv_proj_groups(const void* x, int64_t n_x, const int32_t* perm_token, int64_t n_rows,
                               const int32_t* group_offset, const int32_t* group_mem, int n_groups,
                               const void* w_kv, mom_dtype dt, int d_model, int H, int d, int n_mem,
-                              void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream);
+                              void* k_p, void* v_p, float* k_norm, void* ws, size_t ws_bytes, void* stream);
 
 /* mom_copy_rows -- row copies in 16-byte granules, for packing the routed
  * rows a memory-parallel layer sends to the owners of their memories and
@@ -408,6 +412,73 @@ mom_status mom_memory_chunk_bwd(const void* q, const int32_t* qidx, const void* 
                                 const float* h0, const void* d_o, const float* dh_final,
                                 float* dq, float* dk, float* dv, float* dbeta, float* dlog_alpha, float* dh0,
                                 void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * The layer's backward around the recurrences (training: paper card, Key
+ * points).  MoMLayer.backward strings these with mom_memory_chunk_bwd; the
+ * routing is held fixed (the top-k choice is piecewise constant), gradients
+ * flow through the renormalised gates.  float32 gradients; every call is
+ * asynchronous on `stream`; ws (at least MOM_WS_HEADER_BYTES) takes the
+ * device error record where a call reads indices.
+ *
+ * mom_combine_bwd -- for out_t = o_sh,t + sum_j gate[t,j] o_p[row_of(t,j)]:
+ *   do_p[row_of(t,j)] = gate[t,j] dout[t]          (dt)
+ *   dgate[t,j]        = <dout[t], o_p[row_of(t,j)]>  (float32)
+ * dout [n_tok, H*d], o_p and do_p [n_rows, H*d] (dt); row_of [n_tok*top_k];
+ * gate, dgate [n_tok, top_k].
+ * ---------------------------------------------------------------------- */
+mom_status mom_combine_bwd(const void* dout, const void* o_p, const int32_t* row_of, const float* gate,
+                           int64_t n_tok, int top_k, int64_t n_rows, int H, int d, mom_dtype dt,
+                           void* do_p, float* dgate, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_router_bwd -- the adjoint of the renormalised gates g_j = exp(l_j) /
+ * sum_i exp(l_i) over the chosen memories (explainer, Router mechanics):
+ * dlogits[t, idx[t,j]] = g_j (dgate_j - sum_i g_i dgate_i), zero elsewhere.
+ * topk_idx, gate, dgate [n_tok, top_k]; dlogits [n_tok, n_mem] float32. */
+mom_status mom_router_bwd(const int32_t* topk_idx, const float* gate, const float* dgate, int64_t n_tok,
+                          int top_k, int n_mem, float* dlogits, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_rows_sum -- dst[t] = base[t] (NULL: 0) + sum_j src[row_of[t*top_k+j]]
+ * over float32 rows of width W (a token's gradient from its routed rows).
+ * dst may be base. */
+mom_status mom_rows_sum(const float* src, int64_t n_src, const int32_t* row_of, int top_k, const float* base,
+                        int64_t n_tok, int W, float* dst, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_l2norm_bwd -- for y = z / sqrt(|z|^2 + 1e-6) per (row, head):
+ * dz[r*ldz + col0 + h*d + c] = (dy - y (y . dy)) / norm[r, h]; y [rows, H, d]
+ * (dt), dy [rows, H, d] float32, norm [rows, H] float32 (the projections'
+ * norm outputs). */
+mom_status mom_l2norm_bwd(const void* y, const float* dy, const float* norm, int64_t rows, int H, int d,
+                          mom_dtype dt, float* dz, int64_t ldz, int64_t col0, void* stream);
+
+/* mom_gates_bwd -- beta = sigmoid(z_b), log_alpha = -exp(A) softplus(z_a):
+ * dz[r*ldz + col_b + h] = dbeta beta (1 - beta);
+ * dz[r*ldz + col_a + h] = dlog_alpha (-exp(A_h)) sigmoid(z_a) (sigmoid(z_a)
+ * from log_alpha); dala = dlog_alpha log_alpha.  All [n, H] float32. */
+mom_status mom_gates_bwd(const float* beta, const float* log_alpha, const float* dbeta, const float* dlog_alpha,
+                         const float* A, int64_t n, int H, float* dz, int64_t ldz, int64_t col_b, int64_t col_a,
+                         float* dala, void* stream);
+
+/* mom_col_sums -- out[c] = sum_r a[r*lda + c], c < cols (float32). */
+mom_status mom_col_sums(const float* a, int64_t rows, int64_t lda, int64_t cols, float* out, void* stream);
+
+/* mom_gemm_grouped -- float32 C (+)= op(A) B over groups of rows, for the
+ * projections' input and weight gradients.  A float32, B (dt), C float32,
+ * row-major with leading dimensions lda, ldb, ldc (elements):
+ *   trans_a = 0: group g covers rows group_offset[g]..[g+1]-1 of A [*, K] and
+ *     of C [*, N]; C[r] (+)= A[r] B_g with B_g = B + group_index[g] *
+ *     b_group_stride, [K, N] (the input gradient dZ W);
+ *   trans_a = 1: group g covers reduction rows group_offset[g]..[g+1]-1;
+ *     C_g (+)= sum_r A[r, :M]^T B[b_rows[r] (or r), :N] with C_g = C +
+ *     group_index[g] * c_group_stride, [M, N] (the weight gradient dZ^T X).
+ * group_index NULL: g.  total_rows: group_offset[n_groups] (trans_a = 0).
+ * accumulate: 0 overwrite, 1 add.  A bad row index is recorded in ws and
+ * reads as zero. */
+mom_status mom_gemm_grouped(int trans_a, const float* A, int64_t lda, const void* B, int64_t ldb, mom_dtype dt,
+                            const int32_t* b_rows, int64_t n_b_rows, float* C, int64_t ldc, int64_t M, int64_t N,
+                            int64_t K, int64_t total_rows, const int32_t* group_offset, const int32_t* group_index,
+                            int n_groups, int64_t b_group_stride, int64_t c_group_stride, int accumulate,
+                            void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * mom_combine_unpermute -- the combine (paper card, Summary: outputs are

@@ -59,11 +59,19 @@ SIGNATURES = {
     "mom_decode_step_rule": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP, _VP, _SZ,
                                   _VP]),
     "mom_mem_gate_proj": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
-    "mom_proj_shared": (_I, [_VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "mom_kv_proj_groups": (_I, [_VP, _I64, _VP, _I64, _VP, _VP, _I, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ,
+    "mom_proj_shared": (_I, [_VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_kv_proj_groups": (_I, [_VP, _I64, _VP, _I64, _VP, _VP, _I, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _SZ,
                                 _VP]),
     "mom_copy_rows": (_I, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _VP, _I64, _I64, _VP, _SZ, _VP]),
     "mom_memory_chunk_bwd_workspace_size": (_SZ, [_I64, _I, _I, _I]),
+    "mom_combine_bwd": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I64, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_router_bwd": (_I, [_VP, _VP, _VP, _I64, _I, _I, _VP, _VP, _SZ, _VP]),
+    "mom_rows_sum": (_I, [_VP, _I64, _VP, _I, _VP, _I64, _I, _VP, _VP, _SZ, _VP]),
+    "mom_l2norm_bwd": (_I, [_VP, _VP, _VP, _I64, _I, _I, _I, _VP, _I64, _I64, _VP]),
+    "mom_gates_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _I, _VP, _I64, _I64, _I64, _VP, _VP]),
+    "mom_col_sums": (_I, [_VP, _I64, _I64, _I64, _VP, _VP]),
+    "mom_gemm_grouped": (_I, [_I, _VP, _I64, _VP, _I64, _I, _VP, _I64, _VP, _I64, _I64, _I64, _I64, _I64, _VP, _VP,
+                              _I, _I64, _I64, _I, _VP, _SZ, _VP]),
     "mom_memory_chunk_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I, _I,
                                   _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
 }
@@ -228,20 +236,20 @@ def mom_mem_gate_proj(x, perm, mem_offset, w_gate_mem, A_mem, b_a_mem, top_k, be
                                  _p(log_alpha_p), _p(ws), ws.numel(), _s(stream)), "mom_mem_gate_proj")
 
 
-def mom_proj_shared(x, w_shared, H, d, q, k_sh, v_sh, ws, stream=None):
+def mom_proj_shared(x, w_shared, H, d, q, k_sh, v_sh, ws, stream=None, q_norm=None, k_sh_norm=None):
     n_tok, d_model = x.shape
     _check(lib.mom_proj_shared(_p(x), _p(w_shared), dtype_code(x.dtype), n_tok, d_model, H, d, _p(q), _p(k_sh),
-                               _p(v_sh), _p(ws), ws.numel(), _s(stream)), "mom_proj_shared")
+                               _p(v_sh), _p(q_norm), _p(k_sh_norm), _p(ws), ws.numel(), _s(stream)), "mom_proj_shared")
 
 
-def mom_kv_proj_groups(x, perm, group_offset, group_mem, w_kv, H, d, k_p, v_p, ws, stream=None):
+def mom_kv_proj_groups(x, perm, group_offset, group_mem, w_kv, H, d, k_p, v_p, ws, stream=None, k_norm=None):
     """Routed k/v projections over groups: group g = rows group_offset[g] ..
     group_offset[g+1] with memory group_mem[g]'s weights (perm None: row r
     reads x row r)."""
     n_x, d_model = x.shape
     _check(lib.mom_kv_proj_groups(_p(x), n_x, _p(perm), k_p.shape[0], _p(group_offset), _p(group_mem),
                                   group_mem.numel(), _p(w_kv), dtype_code(x.dtype), d_model, H, d, w_kv.shape[0],
-                                  _p(k_p), _p(v_p), _p(ws), ws.numel(), _s(stream)), "mom_kv_proj_groups")
+                                  _p(k_p), _p(v_p), _p(k_norm), _p(ws), ws.numel(), _s(stream)), "mom_kv_proj_groups")
 
 
 def mom_copy_rows(src, idx, dst, row_bytes, src_off=0, dst_off=0, ws=None, stream=None, n_rows=None):
@@ -323,6 +331,64 @@ def mom_memory_chunk_bwd(q, qidx, k, v, beta, log_alpha, seg_cu, scale, rule, h0
                                     int(rule), int(gates), _p(h0), _p(d_o), _p(dh_final), _p(dq), _p(dk), _p(dv),
                                     _p(dbeta), _p(dlog_alpha), _p(dh0), _p(ws), ws.numel(), _s(stream)),
            "mom_memory_chunk_bwd")
+
+
+def _pa(t, off_elems=0):
+    """Device pointer of a dense CUDA tensor advanced by off_elems elements
+    (a column offset into its rows)."""
+    p = _p(t)
+    return p if p is None or off_elems == 0 else ctypes.c_void_p(p.value + off_elems * t.element_size())
+
+
+def mom_combine_bwd(dout, o_p, row_of, gate, do_p, dgate, ws, stream=None):
+    n_tok, H, d = dout.shape
+    _check(lib.mom_combine_bwd(_p(dout), _p(o_p), _p(row_of), _p(gate), n_tok, gate.shape[1], o_p.shape[0], H, d,
+                               dtype_code(dout.dtype), _p(do_p), _p(dgate), _p(ws), ws.numel(), _s(stream)),
+           "mom_combine_bwd")
+
+
+def mom_router_bwd(topk_idx, gate, dgate, dlogits, ws, stream=None):
+    n_tok, K = topk_idx.shape
+    _check(lib.mom_router_bwd(_p(topk_idx), _p(gate), _p(dgate), n_tok, K, dlogits.shape[1], _p(dlogits), _p(ws),
+                              ws.numel(), _s(stream)), "mom_router_bwd")
+
+
+def mom_rows_sum(src, row_of, top_k, base, dst, ws, stream=None):
+    """dst[t] = base[t] + sum_j src[row_of[t*top_k+j]] (float32 rows)."""
+    n_tok = dst.shape[0]
+    W = dst.numel() // max(n_tok, 1)
+    _check(lib.mom_rows_sum(_p(src), src.shape[0], _p(row_of), top_k, _p(base), n_tok, W, _p(dst), _p(ws), ws.numel(),
+                            _s(stream)), "mom_rows_sum")
+
+
+def mom_l2norm_bwd(y, dy, norm, dz, col0, stream=None):
+    rows, H, d = y.shape
+    _check(lib.mom_l2norm_bwd(_p(y), _p(dy), _p(norm), rows, H, d, dtype_code(y.dtype), _p(dz), dz.shape[1], col0,
+                              _s(stream)), "mom_l2norm_bwd")
+
+
+def mom_gates_bwd(beta, log_alpha, dbeta, dlog_alpha, A, dz, col_b, col_a, dala, stream=None):
+    n, H = beta.shape
+    _check(lib.mom_gates_bwd(_p(beta), _p(log_alpha), _p(dbeta), _p(dlog_alpha), _p(A), n, H, _p(dz), dz.shape[1],
+                             col_b, col_a, _p(dala), _s(stream)), "mom_gates_bwd")
+
+
+def mom_col_sums(a, out, col0=0, stream=None):
+    """out[c] = sum over rows of a[:, col0 + c]."""
+    rows, lda = a.shape
+    _check(lib.mom_col_sums(_pa(a, col0), rows, lda, out.numel(), _p(out), _s(stream)), "mom_col_sums")
+
+
+def mom_gemm_grouped(trans_a, A, B, C, M, N, K, group_offset, group_index, n_groups, ws, a_col=0, b_rows=None,
+                     total_rows=0, b_group_stride=0, c_group_stride=0, accumulate=False, stream=None):
+    """float32 C (+)= op(A) B over groups (see include/mom.h); A, C float32
+    2-D (A read from column a_col), B the weights or tokens (2-D or 3-D,
+    rows of B.shape[-1])."""
+    ldb = B.shape[-1]
+    _check(lib.mom_gemm_grouped(int(trans_a), _pa(A, a_col), A.shape[1], _p(B), ldb, dtype_code(B.dtype), _p(b_rows),
+                                B.numel() // ldb, _p(C), C.shape[-1], M, N, K, total_rows, _p(group_offset),
+                                _p(group_index), n_groups, b_group_stride, c_group_stride, int(accumulate), _p(ws),
+                                ws.numel(), _s(stream)), "mom_gemm_grouped")
 
 
 def mom_combine_unpermute(o_sh, o_p, row_of, topk_gate, out, ws, stream=None):

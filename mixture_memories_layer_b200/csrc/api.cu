@@ -139,7 +139,8 @@ mom_status mom_kv_proj_grouped(const void* x, const int32_t* perm_token, const i
 }
 
 mom_status mom_proj_shared(const void* x, const void* w_shared, mom_dtype dt, int64_t n_tok, int d_model,
-                           int H, int d, void* q, void* k_sh, void* v_sh, void* ws, size_t ws_bytes, void* stream) {
+                           int H, int d, void* q, void* k_sh, void* v_sh, float* q_norm, float* k_sh_norm,
+                           void* ws, size_t ws_bytes, void* stream) {
     if (!dt_ok(dt) || n_tok < 0 || d_model <= 0 || d_model % 64 != 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
     if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
@@ -150,6 +151,8 @@ mom_status mom_proj_shared(const void* x, const void* w_shared, mom_dtype dt, in
     ProjArgs a{x, nullptr, nullptr, w_shared, nullptr, n_tok, d_model, H, d, 1, 1,
                q, k_sh, v_sh, nullptr, nullptr, ws};
     a.parts = PROJ_SHARED;
+    a.q_norm = q_norm;
+    a.k_sh_norm = k_sh_norm;
     cudaStream_t st = as_stream(stream);
     return cuda_status(proj_tc_supported(a, dt) ? launch_proj_tc(a, st) : launch_proj_simt(a, dt, st));
 }
@@ -157,7 +160,7 @@ mom_status mom_proj_shared(const void* x, const void* w_shared, mom_dtype dt, in
 mom_status mom_kv_proj_groups(const void* x, int64_t n_x, const int32_t* perm_token, int64_t n_rows,
                               const int32_t* group_offset, const int32_t* group_mem, int n_groups,
                               const void* w_kv, mom_dtype dt, int d_model, int H, int d, int n_mem,
-                              void* k_p, void* v_p, void* ws, size_t ws_bytes, void* stream) {
+                              void* k_p, void* v_p, float* k_norm, void* ws, size_t ws_bytes, void* stream) {
     if (!dt_ok(dt) || n_x < 0 || n_rows < 0 || d_model <= 0 || d_model % 64 != 0) return MOM_ERR_ARG;
     if (H < 1 || H > MOM_MAX_HEADS || n_mem < 1 || n_mem > MOM_MAX_MEM || n_groups < 0) return MOM_ERR_ARG;
     if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
@@ -175,6 +178,7 @@ mom_status mom_kv_proj_groups(const void* x, int64_t n_x, const int32_t* perm_to
     a.group_mem = group_mem;
     a.n_groups = n_groups;
     a.n_routed = n_rows;
+    a.k_p_norm = k_norm;
     cudaStream_t st = as_stream(stream);
     return cuda_status(proj_tc_supported(a, dt) ? launch_proj_tc(a, st) : launch_proj_simt(a, dt, st));
 }
@@ -339,6 +343,81 @@ mom_status mom_memory_chunk_bwd(const void* q, const int32_t* qidx, const void* 
     GdnBwdArgs a{q, qidx, k, v, beta, log_alpha, seg_cu, n_seg, n_rows, n_q_rows, H, d, scale, rule,
                  gates == MOM_GATES_BY_ROW ? 1 : 0, h0, d_o, dh_final, dq, dk, dv, dbeta, dlog_alpha, dh0, ws};
     return cuda_status(launch_gdn_bwd(a, dt, as_stream(stream)));
+}
+
+// --------------------------------------------------- backward pieces
+mom_status mom_combine_bwd(const void* dout, const void* o_p, const int32_t* row_of, const float* gate,
+                           int64_t n_tok, int top_k, int64_t n_rows, int H, int d, mom_dtype dt,
+                           void* do_p, float* dgate, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || n_rows < 0 || top_k < 1 || H < 1 || d < 1) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {dout, o_p, row_of, gate, do_p, dgate};
+    for (const void* p : ptrs)
+        if (!p) return MOM_ERR_ARG;
+    return cuda_status(launch_combine_bwd(dout, o_p, row_of, gate, n_tok, top_k, H * d, n_rows, dt, do_p, dgate, ws,
+                                          as_stream(stream)));
+}
+
+mom_status mom_router_bwd(const int32_t* topk_idx, const float* gate, const float* dgate, int64_t n_tok,
+                          int top_k, int n_mem, float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+    if (n_tok < 0 || top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    if (!topk_idx || !gate || !dgate || !dlogits) return MOM_ERR_ARG;
+    return cuda_status(launch_router_bwd(topk_idx, gate, dgate, n_tok, top_k, n_mem, dlogits, ws, as_stream(stream)));
+}
+
+mom_status mom_rows_sum(const float* src, int64_t n_src, const int32_t* row_of, int top_k, const float* base,
+                        int64_t n_tok, int W, float* dst, void* ws, size_t ws_bytes, void* stream) {
+    if (n_src < 0 || n_tok < 0 || top_k < 1 || W < 0) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0 || W == 0) return MOM_OK;
+    if (!src || !row_of || !dst) return MOM_ERR_ARG;
+    return cuda_status(launch_rows_sum(src, n_src, row_of, top_k, base, n_tok, W, dst, ws, as_stream(stream)));
+}
+
+mom_status mom_l2norm_bwd(const void* y, const float* dy, const float* norm, int64_t rows, int H, int d,
+                          mom_dtype dt, float* dz, int64_t ldz, int64_t col0, void* stream) {
+    if (!dt_ok(dt) || rows < 0 || H < 1 || d < 1 || col0 < 0 || ldz < col0 + (int64_t)H * d) return MOM_ERR_ARG;
+    if (rows == 0) return MOM_OK;
+    if (!y || !dy || !norm || !dz) return MOM_ERR_ARG;
+    return cuda_status(launch_l2norm_bwd(y, dy, norm, rows, H, d, dt, dz, ldz, col0, as_stream(stream)));
+}
+
+mom_status mom_gates_bwd(const float* beta, const float* log_alpha, const float* dbeta, const float* dlog_alpha,
+                         const float* A, int64_t n, int H, float* dz, int64_t ldz, int64_t col_b, int64_t col_a,
+                         float* dala, void* stream) {
+    if (n < 0 || H < 1 || col_b < 0 || col_a < 0 || ldz < col_b + H || ldz < col_a + H) return MOM_ERR_ARG;
+    if (n == 0) return MOM_OK;
+    const void* ptrs[] = {beta, log_alpha, dbeta, dlog_alpha, A, dz, dala};
+    for (const void* p : ptrs)
+        if (!p) return MOM_ERR_ARG;
+    return cuda_status(launch_gates_bwd(beta, log_alpha, dbeta, dlog_alpha, A, n, H, dz, ldz, col_b, col_a, dala,
+                                        as_stream(stream)));
+}
+
+mom_status mom_col_sums(const float* a, int64_t rows, int64_t lda, int64_t cols, float* out, void* stream) {
+    if (rows < 0 || cols < 0 || lda < cols) return MOM_ERR_ARG;
+    if (cols == 0) return MOM_OK;
+    if (!out || (rows > 0 && !a)) return MOM_ERR_ARG;
+    return cuda_status(launch_col_sums(a, rows, lda, cols, out, as_stream(stream)));
+}
+
+mom_status mom_gemm_grouped(int trans_a, const float* A, int64_t lda, const void* B, int64_t ldb, mom_dtype dt,
+                            const int32_t* b_rows, int64_t n_b_rows, float* C, int64_t ldc, int64_t M, int64_t N,
+                            int64_t K, int64_t total_rows, const int32_t* group_offset, const int32_t* group_index,
+                            int n_groups, int64_t b_group_stride, int64_t c_group_stride, int accumulate,
+                            void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || (trans_a != 0 && trans_a != 1) || n_groups < 0 || N < 0 || M < 0 || K < 0 || total_rows < 0)
+        return MOM_ERR_ARG;
+    if (ldb < N || ldc < N || (trans_a ? lda < M : lda < K)) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_groups == 0 || N == 0 || (trans_a && M == 0)) return MOM_OK;
+    if (!A || !B || !C || !group_offset) return MOM_ERR_ARG;
+    return cuda_status(launch_gemm_grouped(trans_a, A, lda, B, ldb, dt, b_rows, n_b_rows, C, ldc, M, N, K, total_rows,
+                                           group_offset, group_index, n_groups, b_group_stride, c_group_stride,
+                                           accumulate, ws, as_stream(stream)));
 }
 
 // ----------------------------------------------------------------- combine

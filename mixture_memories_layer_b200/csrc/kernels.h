@@ -78,6 +78,12 @@ struct ProjArgs {
     const int32_t* group_mem = nullptr;
     int n_groups = 0;
     int64_t n_routed = -1;
+    // optional: sqrt(|z|^2 + 1e-6) of every normalised (row, head) -- the
+    // lengths the backward of the norm needs: [n_tok, H] for q and k_sh,
+    // [routed rows, H] for k_p
+    float* q_norm = nullptr;
+    float* k_sh_norm = nullptr;
+    float* k_p_norm = nullptr;
     __host__ __device__ int groups() const { return n_groups > 0 ? n_groups : M; }
     __host__ __device__ int64_t routed_rows() const { return n_routed >= 0 ? n_routed : n_tok * K; }
 };
@@ -145,6 +151,26 @@ struct GdnBwdArgs {
 };
 size_t gdn_bwd_ws_bytes(int64_t n_rows, int n_seg, int H, int d);
 cudaError_t launch_gdn_bwd(const GdnBwdArgs& a, int dt, cudaStream_t st);
+
+// layer_bwd.cu: the layer's backward around the recurrences
+cudaError_t launch_combine_bwd(const void* dout, const void* o_p, const int32_t* row_of, const float* gate,
+                               int64_t n_tok, int K, int HD, int64_t n_rows, int dt, void* do_p, float* dgate,
+                               void* err, cudaStream_t st);
+cudaError_t launch_router_bwd(const int32_t* idx, const float* gate, const float* dgate, int64_t n_tok, int K, int M,
+                              float* dlogits, void* err, cudaStream_t st);
+cudaError_t launch_rows_sum(const float* src, int64_t n_src, const int32_t* row_of, int K, const float* base,
+                            int64_t n_tok, int W, float* dst, void* err, cudaStream_t st);
+cudaError_t launch_l2norm_bwd(const void* y, const float* dy, const float* nrm, int64_t rows, int H, int d, int dt,
+                              float* dz, int64_t ldz, int64_t col0, cudaStream_t st);
+cudaError_t launch_gates_bwd(const float* beta, const float* la, const float* dbeta, const float* dla, const float* A,
+                             int64_t n, int H, float* dz, int64_t ldz, int64_t col_b, int64_t col_a, float* dala,
+                             cudaStream_t st);
+cudaError_t launch_col_sums(const float* a, int64_t rows, int64_t lda, int64_t C, float* out, cudaStream_t st);
+cudaError_t launch_gemm_grouped(int trans_a, const float* A, int64_t lda, const void* B, int64_t ldb, int dt,
+                                const int32_t* b_rows, int64_t n_b_rows, float* C, int64_t ldc, int64_t M, int64_t N,
+                                int64_t K, int64_t total_rows, const int32_t* goff, const int32_t* gmem, int n_groups,
+                                int64_t b_group_stride, int64_t c_group_stride, int accumulate, void* err,
+                                cudaStream_t st);
 
 // gdn_chunk_tc.cu: chunked Gated DeltaNet on the tcgen05 tensor cores (bf16)
 bool gdn_tc_supported(const GdnArgs& a, int dt);

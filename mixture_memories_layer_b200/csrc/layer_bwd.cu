@@ -1,0 +1,340 @@
+// The layer's backward around its recurrences (training is the pages' main
+// workload: "MoM: Linear Sequence Modeling with Mixture-of-Memories", Key
+// points): the adjoints of the combine, of the renormalised router gates
+// ("MoM: Mixture-of-Memories Fixes Linear Attention Recall", Router
+// mechanics), of the per-head L2 norms and of the gates, the per-token sums
+// of what the routed rows received, column sums, and one grouped float32
+// GEMM for the input and weight gradients of every projection.  First path:
+// CUDA cores, float32 accumulation.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mom {
+namespace {
+
+// do_p[row_of(t,j)] = g_tj dout_t; dgate_tj = <dout_t, o_p[row_of(t,j)]>.  One warp per token.
+template <typename T>
+__global__ void __launch_bounds__(256)
+combine_bwd_kernel(const T* __restrict__ dout, const T* __restrict__ o_p, const int32_t* __restrict__ row_of,
+                   const float* __restrict__ gate, int64_t n_tok, int K, int HD, int64_t n_rows, T* __restrict__ do_p,
+                   float* __restrict__ dgate, void* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < n_tok; t += warps) {
+        for (int j = 0; j < K; ++j) {
+            const int64_t r = row_of[t * K + j];
+            if (r < 0 || r >= n_rows) {
+                if (lane == 0) { record_error(err, MOM_DEVERR_ROW_INDEX, t * K + j); dgate[t * K + j] = 0.f; }
+                continue;
+            }
+            const float g = gate[t * K + j];
+            float acc = 0.f;
+            for (int c = lane; c < HD; c += 32) {
+                const float dy = to_f(dout[t * HD + c]);
+                do_p[r * HD + c] = from_f<T>(g * dy);
+                acc = fmaf(dy, to_f(o_p[r * HD + c]), acc);
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) dgate[t * K + j] = acc;
+        }
+    }
+}
+
+// dlogits = the adjoint of g_j = exp(l_j) / sum_i exp(l_i) over the chosen
+// memories: dl_j = g_j (dg_j - sum_i g_i dg_i), zero for the others.
+__global__ void __launch_bounds__(256)
+router_bwd_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, const float* __restrict__ dgate,
+                  int64_t n_tok, int K, int M, float* __restrict__ dlogits, void* err) {
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_tok; t += (int64_t)gridDim.x * blockDim.x) {
+        float s = 0.f;
+        for (int j = 0; j < K; ++j) s = fmaf(gate[t * K + j], dgate[t * K + j], s);
+        for (int m = 0; m < M; ++m) dlogits[t * M + m] = 0.f;
+        for (int j = 0; j < K; ++j) {
+            const int m = idx[t * K + j];
+            if (m < 0 || m >= M) { record_error(err, MOM_DEVERR_MEM_INDEX, t); continue; }
+            dlogits[t * M + m] = gate[t * K + j] * (dgate[t * K + j] - s);
+        }
+    }
+}
+
+// dst[t] = base[t] (or 0) + sum_j src[row_of(t, j)], rows of W floats.  One warp per token.
+__global__ void __launch_bounds__(256)
+rows_sum_kernel(const float* __restrict__ src, int64_t n_src, const int32_t* __restrict__ row_of, int K,
+                const float* __restrict__ base, int64_t n_tok, int W, float* __restrict__ dst, void* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < n_tok; t += warps) {
+        if (lane == 0)
+            for (int j = 0; j < K; ++j) {
+                const int64_t r = row_of[t * K + j];
+                if (r < 0 || r >= n_src) record_error(err, MOM_DEVERR_ROW_INDEX, t * K + j);
+            }
+        for (int c = lane; c < W; c += 32) {
+            float acc = base ? base[t * W + c] : 0.f;
+            for (int j = 0; j < K; ++j) {
+                const int64_t r = row_of[t * K + j];
+                if (r >= 0 && r < n_src) acc += src[r * W + c];
+            }
+            dst[t * W + c] = acc;
+        }
+    }
+}
+
+// dz = (dy - y (y . dy)) / n per (row, head); y the normalised value, n its
+// length sqrt(|z|^2 + eps).  One warp per (row, head).
+template <typename T>
+__global__ void __launch_bounds__(256)
+l2norm_bwd_kernel(const T* __restrict__ y, const float* __restrict__ dy, const float* __restrict__ nrm, int64_t rows,
+                  int H, int d, float* __restrict__ dz, int64_t ldz, int64_t col0) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t rh = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); rh < rows * H; rh += warps) {
+        const int64_t r = rh / H;
+        const int h = (int)(rh - r * H);
+        const int64_t o = rh * d;
+        float dot = 0.f;
+        for (int c = lane; c < d; c += 32) dot = fmaf(to_f(y[o + c]), dy[o + c], dot);
+        dot = warp_sum(dot);
+        const float inv = 1.f / nrm[rh];
+        for (int c = lane; c < d; c += 32)
+            dz[r * ldz + col0 + (int64_t)h * d + c] = (dy[o + c] - to_f(y[o + c]) * dot) * inv;
+    }
+}
+
+// beta = sigmoid(z_b): dz_b = dbeta beta (1 - beta).
+// log alpha = -e^A softplus(z_a): dz_a = dla (-e^A) sigmoid(z_a), with
+// sigmoid(z_a) = 1 - e^(-softplus(z_a)) and softplus(z_a) = -log alpha e^-A;
+// dala = dla log alpha (summed over tokens: dA).
+__global__ void __launch_bounds__(256)
+gates_bwd_kernel(const float* __restrict__ beta, const float* __restrict__ la, const float* __restrict__ dbeta,
+                 const float* __restrict__ dla, const float* __restrict__ A, int64_t n, int H, float* __restrict__ dz,
+                 int64_t ldz, int64_t col_b, int64_t col_a, float* __restrict__ dala) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n * H; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / H;
+        const int h = (int)(i - r * H);
+        const float b = beta[i], l = la[i], eA = expf(A[h]);
+        dz[r * ldz + col_b + h] = dbeta[i] * b * (1.f - b);
+        const float sp = -l / eA;
+        const float sg = -expm1f(-sp);                  // 1 - e^-sp
+        dz[r * ldz + col_a + h] = dla[i] * (-eA) * sg;
+        dala[i] = dla[i] * l;
+    }
+}
+
+// out[c] = sum_r a[r * lda + c], c < C: one warp per column, lanes over rows.
+__global__ void __launch_bounds__(256)
+col_sums_kernel(const float* __restrict__ a, int64_t rows, int64_t lda, int64_t C, float* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t c = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); c < C; c += warps) {
+        float acc = 0.f;
+        for (int64_t r = lane; r < rows; r += 32) acc += a[r * lda + c];
+        acc = warp_sum(acc);
+        if (lane == 0) out[c] = acc;
+    }
+}
+
+// ------------------------------------------------------------ grouped GEMM
+constexpr int GBM = 64, GBN = 64, GBK = 16;
+
+struct GemmArgs {
+    int trans_a;
+    const float* A;
+    int64_t lda;
+    const void* B;
+    int64_t ldb;
+    const int32_t* b_rows;     // TRANS: row of B for reduction row r (null: r)
+    float* C;
+    int64_t ldc;
+    int64_t M, N, K;
+    const int32_t* goff;
+    const int32_t* gmem;
+    int n_groups;
+    int64_t b_group_stride, c_group_stride;
+    int accumulate;
+    int64_t n_b_rows;          // rows of B (bounds of b_rows)
+    void* err;
+};
+
+// trans_a = 0: the CTA's 64-row tile of a group (tiles listed over all groups)
+// trans_a = 1: blockIdx.z is the group, the tile of C_g is (blockIdx.y, blockIdx.x)
+template <typename TB>
+__global__ void __launch_bounds__(256)
+gemm_grouped_kernel(GemmArgs g) {
+    __shared__ float As[GBK][GBM + 4];
+    __shared__ float Bs[GBK][GBN + 4];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const TB* B = reinterpret_cast<const TB*>(g.B);
+    const int64_t n0 = (int64_t)blockIdx.x * GBN;
+    int64_t m0, m1, k0, k1;
+    const TB* Bg = B;
+    float* Cg = g.C;
+    if (!g.trans_a) {
+        // find this tile's group: tiles are numbered group by group
+        int64_t t = blockIdx.y;
+        int grp = -1;
+        for (int q = 0; q < g.n_groups; ++q) {
+            const int64_t lo = g.goff[q], hi = g.goff[q + 1];
+            if (lo < 0 || hi < lo) { if (tid == 0 && blockIdx.x == 0) record_error(g.err, MOM_DEVERR_SEGMENT, q); return; }
+            const int64_t nt = (hi - lo + GBM - 1) / GBM;
+            if (t < nt) { grp = q; m0 = lo + t * GBM; m1 = m0 + GBM < hi ? m0 + GBM : hi; break; }
+            t -= nt;
+        }
+        if (grp < 0) return;
+        const int64_t w = g.gmem ? g.gmem[grp] : grp;
+        Bg = B + w * g.b_group_stride;
+        k0 = 0;
+        k1 = g.K;
+    } else {
+        const int grp = blockIdx.z;
+        m0 = (int64_t)blockIdx.y * GBM;
+        m1 = m0 + GBM < g.M ? m0 + GBM : g.M;
+        if (m0 >= g.M) return;
+        k0 = g.goff[grp];
+        k1 = g.goff[grp + 1];
+        if (k0 < 0 || k1 < k0) { if (tid == 0 && blockIdx.x == 0) record_error(g.err, MOM_DEVERR_SEGMENT, grp); return; }
+        const int64_t w = g.gmem ? g.gmem[grp] : grp;
+        Cg = g.C + w * g.c_group_stride;
+    }
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int64_t kb = k0; kb < k1; kb += GBK) {
+        // A tile (GBK x GBM) and B tile (GBK x GBN), zero past the ends
+        for (int e = tid; e < GBK * GBM; e += 256) {
+            int kk, mm;
+            if (!g.trans_a) { mm = e / GBK; kk = e % GBK; } else { kk = e / GBM; mm = e % GBM; }
+            const int64_t m = m0 + mm, k = kb + kk;
+            float v = 0.f;
+            if (m < m1 && k < k1) v = g.trans_a ? g.A[k * g.lda + m] : g.A[m * g.lda + k];
+            As[kk][mm] = v;
+        }
+        for (int e = tid; e < GBK * GBN; e += 256) {
+            const int kk = e / GBN, nn = e % GBN;
+            const int64_t k = kb + kk, n = n0 + nn;
+            float v = 0.f;
+            if (k < k1 && n < g.N) {
+                int64_t br = k;
+                if (g.trans_a && g.b_rows) {
+                    br = g.b_rows[k];
+                    if (br < 0 || br >= g.n_b_rows) { record_error(g.err, MOM_DEVERR_ROW_INDEX, k); br = -1; }
+                }
+                if (br >= 0) v = to_f(Bg[br * g.ldb + n]);
+            }
+            Bs[kk][nn] = v;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < GBK; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t m = m0 + ty * 4 + i;
+        if (m >= m1) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t n = n0 + tx * 4 + j;
+            if (n >= g.N) continue;
+            float* c = Cg + m * g.ldc + n;
+            *c = g.accumulate ? *c + acc[i][j] : acc[i][j];
+        }
+    }
+}
+
+unsigned grid_rows(int64_t rows, int per_block) {
+    const int64_t want = cdiv(rows > 0 ? rows : 1, per_block);
+    return (unsigned)(want < 148 * 16 ? want : 148 * 16);
+}
+
+}  // namespace
+
+cudaError_t launch_combine_bwd(const void* dout, const void* o_p, const int32_t* row_of, const float* gate,
+                               int64_t n_tok, int K, int HD, int64_t n_rows, int dt, void* do_p, float* dgate,
+                               void* err, cudaStream_t st) {
+    if (n_tok == 0) return cudaSuccess;
+    if (dt == MOM_BF16)
+        combine_bwd_kernel<bf16><<<grid_rows(n_tok, 8), 256, 0, st>>>((const bf16*)dout, (const bf16*)o_p, row_of, gate,
+                                                                     n_tok, K, HD, n_rows, (bf16*)do_p, dgate, err);
+    else
+        combine_bwd_kernel<float><<<grid_rows(n_tok, 8), 256, 0, st>>>((const float*)dout, (const float*)o_p, row_of,
+                                                                      gate, n_tok, K, HD, n_rows, (float*)do_p, dgate,
+                                                                      err);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_bwd(const int32_t* idx, const float* gate, const float* dgate, int64_t n_tok, int K, int M,
+                              float* dlogits, void* err, cudaStream_t st) {
+    if (n_tok == 0) return cudaSuccess;
+    router_bwd_kernel<<<grid_rows(n_tok, 256), 256, 0, st>>>(idx, gate, dgate, n_tok, K, M, dlogits, err);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rows_sum(const float* src, int64_t n_src, const int32_t* row_of, int K, const float* base,
+                            int64_t n_tok, int W, float* dst, void* err, cudaStream_t st) {
+    if (n_tok == 0) return cudaSuccess;
+    rows_sum_kernel<<<grid_rows(n_tok, 8), 256, 0, st>>>(src, n_src, row_of, K, base, n_tok, W, dst, err);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_l2norm_bwd(const void* y, const float* dy, const float* nrm, int64_t rows, int H, int d, int dt,
+                              float* dz, int64_t ldz, int64_t col0, cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    if (dt == MOM_BF16)
+        l2norm_bwd_kernel<bf16><<<grid_rows(rows * H, 8), 256, 0, st>>>((const bf16*)y, dy, nrm, rows, H, d, dz, ldz, col0);
+    else
+        l2norm_bwd_kernel<float><<<grid_rows(rows * H, 8), 256, 0, st>>>((const float*)y, dy, nrm, rows, H, d, dz, ldz,
+                                                                        col0);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gates_bwd(const float* beta, const float* la, const float* dbeta, const float* dla, const float* A,
+                             int64_t n, int H, float* dz, int64_t ldz, int64_t col_b, int64_t col_a, float* dala,
+                             cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    gates_bwd_kernel<<<grid_rows(n * H, 256), 256, 0, st>>>(beta, la, dbeta, dla, A, n, H, dz, ldz, col_b, col_a, dala);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_col_sums(const float* a, int64_t rows, int64_t lda, int64_t C, float* out, cudaStream_t st) {
+    if (C == 0) return cudaSuccess;
+    col_sums_kernel<<<grid_rows(C, 8), 256, 0, st>>>(a, rows, lda, C, out);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_grouped(int trans_a, const float* A, int64_t lda, const void* B, int64_t ldb, int dt,
+                                const int32_t* b_rows, int64_t n_b_rows, float* C, int64_t ldc, int64_t M, int64_t N,
+                                int64_t K, int64_t total_rows, const int32_t* goff, const int32_t* gmem, int n_groups,
+                                int64_t b_group_stride, int64_t c_group_stride, int accumulate, void* err,
+                                cudaStream_t st) {
+    if (n_groups == 0 || N == 0) return cudaSuccess;
+    GemmArgs g{trans_a, A, lda, B, ldb, b_rows, C, ldc, M, N, K, goff, gmem, n_groups, b_group_stride,
+               c_group_stride, accumulate, n_b_rows, err};
+    dim3 grid;
+    if (!trans_a) grid = dim3((unsigned)cdiv(N, GBN), (unsigned)(cdiv(total_rows, GBM) + n_groups), 1);
+    else grid = dim3((unsigned)cdiv(N, GBN), (unsigned)cdiv(M, GBM), (unsigned)n_groups);
+    if (dt == MOM_BF16) gemm_grouped_kernel<bf16><<<grid, 256, 0, st>>>(g);
+    else gemm_grouped_kernel<float><<<grid, 256, 0, st>>>(g);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace mom

@@ -35,6 +35,7 @@ proj_simt_kernel(ProjArgs a, int64_t sh_tiles) {
     const T* W;
     T* out;
     bool norm;
+    float* nout;
     if (bid < sh_tiles) {
         const int nb = 3 * H;
         cb = (int)(bid % nb);
@@ -44,6 +45,7 @@ proj_simt_kernel(ProjArgs a, int64_t sh_tiles) {
         W = reinterpret_cast<const T*>(a.w_shared) + (size_t)cb * DH * D;
         out = reinterpret_cast<T*>(part == 0 ? a.q : part == 1 ? a.k_sh : a.v_sh);
         norm = part < 2;
+        nout = part == 0 ? a.q_norm : part == 1 ? a.k_sh_norm : nullptr;
     } else {
         const int nb = 2 * H;
         int64_t local = bid - sh_tiles;
@@ -66,6 +68,7 @@ proj_simt_kernel(ProjArgs a, int64_t sh_tiles) {
         W = reinterpret_cast<const T*>(a.w_kv) + ((size_t)m * 2 * H * DH + (size_t)cb * DH) * D;
         out = reinterpret_cast<T*>(part == 0 ? a.k_p : a.v_p);
         norm = part == 0;
+        nout = part == 0 ? a.k_p_norm : nullptr;
     }
     const int h = cb % H;
 
@@ -128,6 +131,7 @@ proj_simt_kernel(ProjArgs a, int64_t sh_tiles) {
             for (int j = 0; j < NJ; ++j) ss = fmaf(acc[i][j], acc[i][j], ss);
             ss = warp_sum(ss);
             sc = rsqrtf(ss + 1e-6f);
+            if (nout && lane == 0 && r < r_end) nout[r * H + h] = sqrtf(ss + 1e-6f);
         }
         if (r < r_end) {
             T* o = out + (r * H + h) * DH;

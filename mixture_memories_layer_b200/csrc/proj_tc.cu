@@ -52,6 +52,7 @@ struct TcParams {
     bf16 *q, *k_sh, *v_sh, *k_p, *v_p;
     int64_t n_tok, n_routed;
     int D, H, d, M, K, n_groups;
+    float *q_norm, *k_sh_norm, *k_p_norm;     // optional per-(row, head) lengths
     int sh_ct, rt_ct;       // column tiles per row tile (shared / routed)
     int64_t sh_tiles;       // shared tiles
     int64_t n_tiles;        // shared + an upper bound of routed tiles
@@ -235,12 +236,15 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
             const int part_i = col0 / Hd, cc0 = col0 % Hd;
             bf16* base;
             bool norm;
+            float* nout;
             if (T.m < 0) {
                 base = part_i == 0 ? p.q : part_i == 1 ? p.k_sh : p.v_sh;
                 norm = part_i < 2;
+                nout = part_i == 0 ? p.q_norm : part_i == 1 ? p.k_sh_norm : nullptr;
             } else {
                 base = part_i == 0 ? p.k_p : p.v_p;
                 norm = part_i == 0;
+                nout = part_i == 0 ? p.k_p_norm : nullptr;
             }
             const CUtensorMap* omap = T.m < 0 ? (part_i == 0 ? &om.q : part_i == 1 ? &om.k_sh : &om.v_sh)
                                               : (part_i == 0 ? &om.k_p : &om.v_p);
@@ -263,6 +267,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
                     for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
                 }
                 sc_full = rsqrtf(ss + 1e-6f);
+                if (nout && live && hf == 0) nout[row * p.H + cc0 / p.d] = sqrtf(ss + 1e-6f);
             }
             float scg[HALF / 64 * 2];                        // per 32-column block scale
 #pragma unroll
@@ -278,6 +283,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
                         for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
                     }
                     const float sc = rsqrtf(ss + 1e-6f);
+                    if (nout && live) nout[row * p.H + (cc0 + hf * HALF + g) / p.d] = sqrtf(ss + 1e-6f);
 #pragma unroll
                     for (int j = 0; j < HALF / 32; ++j)
                         if (j * 32 >= g && j * 32 < g + gw) scg[j] = sc;
@@ -403,6 +409,9 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     p.perm = a.perm_token;
     p.mem_offset = a.mem_offset;
     p.group_mem = a.group_mem;
+    p.q_norm = a.q_norm;
+    p.k_sh_norm = a.k_sh_norm;
+    p.k_p_norm = a.k_p_norm;
     p.q = reinterpret_cast<bf16*>(a.q);
     p.k_sh = reinterpret_cast<bf16*>(a.k_sh);
     p.v_sh = reinterpret_cast<bf16*>(a.v_sh);

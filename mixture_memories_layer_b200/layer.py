@@ -242,6 +242,102 @@ class MoMLayer:
                     errs[key[1]] = (code, info)
         return errs
 
+    # ------------------------------------------------------------- backward
+    def backward(self, x: torch.Tensor, cu_seqlens: torch.Tensor, dout: torch.Tensor, dh_shared=None, dh_mem=None,
+                 h0_shared=None, h0_mem=None, stream=None) -> Dict[str, torch.Tensor]:
+        """Gradients of <dout, out> + <dh_shared, h_shared> + <dh_mem, h_mem>
+        for the forward just run on the same x and cu_seqlens (its buffers
+        are read): dx, dw_r, db_r, dw_shared [3Hd, D] (W_q | W_k_sh | W_v_sh),
+        dw_gate [2H, D] (W_beta | W_a), dA, db_a, dw_kv [M, 2Hd, D], dh0_shared
+        [S, H, d, d], dh0_mem [M, S, H, d, d]; all float32.  The routing is
+        held fixed; gradients flow through the renormalised gates.  Every step
+        runs in the CUDA library (the recurrences' reverse passes, then the
+        combine, router, norm and gate adjoints and the projections' GEMMs)."""
+        if self.mem_gates:
+            raise NotImplementedError("the backward of per-memory gates is not provided")
+        n_tok, D = x.shape
+        n_seq = cu_seqlens.numel() - 1
+        H, d, K, M, dt = self.H, self.d, self.top_k, self.n_mem, self.dtype
+        Hd, R = H * d, n_tok * K
+        w, b = self.w, self.buffers(n_tok, n_seq)
+        dev, f32 = self.device, torch.float32
+        st = stream if stream is not None else torch.cuda.current_stream()
+        g = lambda name, shape, dtype=f32: self._buf("bwd_" + name, shape, dtype)
+        ws = self._ws("bwd", B.MOM_WS_HEADER_BYTES)
+        # the lengths the norms' backward needs (the projections again, with their norm outputs)
+        qn, kshn, kpn = g("qn", (n_tok, H)), g("kshn", (n_tok, H)), g("kpn", (R, H))
+        B.mom_proj_shared(x, w["w_shared"], H, d, g("q2", (n_tok, H, d), dt), g("k2", (n_tok, H, d), dt),
+                          g("v2", (n_tok, H, d), dt), ws, stream=st, q_norm=qn, k_sh_norm=kshn)
+        mem_index = self._buf("mem_index", (M,), torch.int32)
+        mem_index.copy_(torch.arange(M, dtype=torch.int32, device=dev))
+        B.mom_kv_proj_groups(x, b["perm"], b["mem_offset"], mem_index, w["w_kv"], H, d, g("kp2", (R, H, d), dt),
+                             g("vp2", (R, H, d), dt), ws, stream=st, k_norm=kpn)
+        # combine and router
+        do_p, dgate = g("do_p", (R, H, d), dt), g("dgate", (n_tok, K))
+        B.mom_combine_bwd(dout, b["o_p"], b["row_of"], b["gate"], do_p, dgate, ws, stream=st)
+        dlogits = g("dlogits", (n_tok, M))
+        B.mom_router_bwd(b["idx"], b["gate"], dgate, dlogits, ws, stream=st)
+        # the recurrences' reverse passes
+        dq_sh, dk_sh, dv_sh = (g(n, (n_tok, H, d)) for n in ("dq_sh", "dk_sh", "dv_sh"))
+        db_sh, dla_sh = g("db_sh", (n_tok, H)), g("dla_sh", (n_tok, H))
+        dq_p, dk_p, dv_p = (g(n, (R, H, d)) for n in ("dq_p", "dk_p", "dv_p"))
+        db_p, dla_p = g("db_p", (R, H)), g("dla_p", (R, H))
+        dh0_sh, dh0_m = g("dh0_sh", (n_seq, H, d, d)), g("dh0_m", (M, n_seq, H, d, d))
+        ws_sh = self._ws("bwd_sh", B.mom_memory_chunk_bwd_workspace_size(n_tok, n_seq, H, d))
+        ws_p = self._ws("bwd_p", B.mom_memory_chunk_bwd_workspace_size(R, M * n_seq, H, d))
+        B.mom_memory_chunk_bwd(b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens, self.scale,
+                               self.rule, h0_shared, dout, dh_shared, dq_sh, dk_sh, dv_sh, db_sh, dla_sh, dh0_sh, ws_sh,
+                               stream=st)
+        dhm = None if dh_mem is None else dh_mem.reshape(M * n_seq, H, d, d)
+        h0m = None if h0_mem is None else h0_mem.reshape(M * n_seq, H, d, d)
+        B.mom_memory_chunk_bwd(b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
+                               self.scale, self.rule, h0m, do_p, dhm, dq_p, dk_p, dv_p, db_p, dla_p,
+                               dh0_m.view(M * n_seq, H, d, d), ws_p, stream=st)
+        # per token: the shared memory's gradients plus those of its routed rows
+        dq, dbeta, dla = g("dq", (n_tok, H, d)), g("dbeta", (n_tok, H)), g("dla", (n_tok, H))
+        B.mom_rows_sum(dq_p.view(R, Hd), b["row_of"], K, dq_sh.view(n_tok, Hd), dq.view(n_tok, Hd), ws, stream=st)
+        B.mom_rows_sum(db_p, b["row_of"], K, db_sh, dbeta, ws, stream=st)
+        B.mom_rows_sum(dla_p, b["row_of"], K, dla_sh, dla, ws, stream=st)
+        # pre-activation gradients: shared [N, 3Hd + 2H] (q | k_sh | v_sh | beta | a), routed [N*K, 2Hd] (k | v)
+        ldz = (3 * Hd + 2 * H + 3) // 4 * 4        # rows 16-byte aligned for the row copies
+        dz = g("dz", (n_tok, ldz))
+        B.mom_l2norm_bwd(b["q"], dq, qn, dz, 0, stream=st)
+        B.mom_l2norm_bwd(b["k_sh"], dk_sh, kshn, dz, Hd, stream=st)
+        B.mom_copy_rows(dv_sh.view(n_tok, Hd), None, dz, Hd * 4, src_off=0, dst_off=2 * Hd * 4, ws=ws, stream=st)
+        dala = g("dala", (n_tok, H))
+        B.mom_gates_bwd(b["beta"], b["log_alpha"], dbeta, dla, w["A"], dz, 3 * Hd, 3 * Hd + H, dala, stream=st)
+        dzr = g("dzr", (R, 2 * Hd))
+        rows = int(R)
+        B.mom_l2norm_bwd(b["k_p"], dk_p, kpn, dzr, 0, stream=st)
+        B.mom_copy_rows(dv_p.view(R, Hd), None, dzr, Hd * 4, src_off=0, dst_off=Hd * 4, ws=ws, stream=st)
+        # input gradient: shared, gates, router, then the routed rows summed per token
+        one = self._buf("one_group", (2,), torch.int32)
+        one.copy_(torch.tensor([0, n_tok], dtype=torch.int32, device=dev))
+        dx = g("dx", (n_tok, D))
+        B.mom_gemm_grouped(0, dz, w["w_shared"], dx, 0, D, 3 * Hd, one, None, 1, ws, total_rows=n_tok, stream=st)
+        B.mom_gemm_grouped(0, dz, w["w_gate"], dx, 0, D, 2 * H, one, None, 1, ws, a_col=3 * Hd, total_rows=n_tok,
+                           accumulate=True, stream=st)
+        B.mom_gemm_grouped(0, dlogits, w["w_r"], dx, 0, D, M, one, None, 1, ws, total_rows=n_tok, accumulate=True,
+                           stream=st)
+        dx_rows = g("dx_rows", (R, D))
+        B.mom_gemm_grouped(0, dzr, w["w_kv"], dx_rows, 0, D, 2 * Hd, b["mem_offset"], None, M, ws, total_rows=rows,
+                           b_group_stride=2 * Hd * D, stream=st)
+        B.mom_rows_sum(dx_rows, b["row_of"], K, dx, dx, ws, stream=st)
+        # weight gradients
+        dw_shared, dw_gate, dw_r = g("dw_shared", (3 * Hd, D)), g("dw_gate", (2 * H, D)), g("dw_r", (M, D))
+        dw_kv = g("dw_kv", (M, 2 * Hd, D))
+        B.mom_gemm_grouped(1, dz, x, dw_shared, 3 * Hd, D, 0, one, None, 1, ws, stream=st)
+        B.mom_gemm_grouped(1, dz, x, dw_gate, 2 * H, D, 0, one, None, 1, ws, a_col=3 * Hd, stream=st)
+        B.mom_gemm_grouped(1, dlogits, x, dw_r, M, D, 0, one, None, 1, ws, stream=st)
+        B.mom_gemm_grouped(1, dzr, x, dw_kv.view(M * 2 * Hd, D), 2 * Hd, D, 0, b["mem_offset"], None, M, ws,
+                           b_rows=b["perm"], c_group_stride=2 * Hd * D, stream=st)
+        db_r, dA, db_a = g("db_r", (M,)), g("dA", (H,)), g("db_a", (H,))
+        B.mom_col_sums(dlogits, db_r, stream=st)
+        B.mom_col_sums(dala, dA, stream=st)
+        B.mom_col_sums(dz, db_a, col0=3 * Hd + H, stream=st)
+        return dict(dx=dx, dw_r=dw_r, db_r=db_r, dw_shared=dw_shared, dw_gate=dw_gate, dA=dA, db_a=db_a, dw_kv=dw_kv,
+                    dh0_shared=dh0_sh, dh0_mem=dh0_m)
+
     # --------------------------------------------------------------- decode
     def decode_step(self, x: torch.Tensor, state: torch.Tensor, stream=None):
         """x [B, d_model]; state [B, M+1, H, d, d] float32, updated in place.

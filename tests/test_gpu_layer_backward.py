@@ -1,0 +1,79 @@
+"""GPU parity of the whole layer's backward (MoMLayer.backward: the
+recurrences' reverse passes, the combine, router, norm and gate adjoints and
+the projections' gradient GEMMs) against the oracle's layer backward, itself
+pinned by finite differences of the forward ("MoM: Linear Sequence Modeling
+with Mixture-of-Memories", Key points: training; explainer, Router
+mechanics: the gradients flow through the renormalised gates, the top-k
+choice held fixed).  The oracle runs with the GPU's routing.  float32 layers
+within 1e-5 (measured ~1e-6), bf16 layers (operands rounded to bf16 in the
+forward) within 2e-2 (measured 2e-4 .. 1.3e-2), per gradient tensor,
+max |gpu - ref| / max |ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_memories_layer_b200 import synth
+from oracle import mom_oracle_bwd as obwd
+from tests.gpu_helpers import max_abs_rel
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True):
+    from mixture_memories_layer_b200 import layer as L
+    w = synth.Workload("bwd", 0, 0, D, H, d, M, K, dtype, seed=seed)
+    rng = np.random.default_rng(seed)
+    p = synth.make_weights(w, rng)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    x = synth.make_tokens(w, rng, int(cu[-1]))
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    lay = L.MoMLayer(L.pack_weights(p, dt), H, d, K)
+    xt = torch.as_tensor(x).to("cuda", dt)
+    cut = torch.as_tensor(cu).cuda()
+    b = lay.forward(xt, cut)
+    n, S = xt.shape[0], len(cu) - 1
+    dout = synth._act(rng.standard_normal((n, H, d)).astype(np.float32), dtype)
+    dh_sh = rng.standard_normal((S, H, d, d)).astype(np.float32) * 0.1 if with_states else None
+    dh_m = rng.standard_normal((M, S, H, d, d)).astype(np.float32) * 0.1 if with_states else None
+    t = lambda a, ty=torch.float32: None if a is None else torch.as_tensor(a).to("cuda", ty)
+    g = lay.backward(xt, cut, t(dout, dt), dh_shared=t(dh_sh), dh_mem=t(dh_m))
+    torch.cuda.synchronize()
+    assert lay.device_errors() == {}
+    got = {k: v.cpu().numpy().astype(np.float64) for k, v in g.items()}
+    idx = b["idx"].cpu().numpy()
+    ref = obwd.mom_backward(x, p, cu, K, H, d, dout, forced_idx=idx, dh_shared=dh_sh, dh_mem=dh_m)
+    Hd = H * d
+    pairs = {
+        "dx": (got["dx"], ref["dx"]), "dw_r": (got["dw_r"], ref["dw_r"]), "db_r": (got["db_r"], ref["db_r"]),
+        "dw_q": (got["dw_shared"][:Hd], ref["dw_q"]), "dw_k_sh": (got["dw_shared"][Hd:2 * Hd], ref["dw_k_sh"]),
+        "dw_v_sh": (got["dw_shared"][2 * Hd:], ref["dw_v_sh"]), "dw_beta": (got["dw_gate"][:H], ref["dw_beta"]),
+        "dw_a": (got["dw_gate"][H:], ref["dw_a"]), "dA": (got["dA"], ref["dA"]), "db_a": (got["db_a"], ref["db_a"]),
+        "dw_k": (got["dw_kv"][:, :Hd], ref["dw_k"]), "dw_v": (got["dw_kv"][:, Hd:], ref["dw_v"]),
+        "dh0_shared": (got["dh0_shared"], ref["dh0_shared"]), "dh0_mem": (got["dh0_mem"], ref["dh0_mem"]),
+    }
+    return {k: max_abs_rel(a, r) for k, (a, r) in pairs.items()}
+
+
+@pytest.mark.parametrize("lens", [(130, 64, 65, 2), (77, 0, 200)])
+def test_layer_backward_fp32(lens):
+    errs = _run("f32", 64, lens)
+    bad = {k: e for k, e in errs.items() if not e < 1e-5}
+    assert not bad, bad
+
+
+def test_layer_backward_bf16_tensor_core_forward():
+    errs = _run("bf16", 128, (150, 61, 1), seed=82)
+    bad = {k: e for k, e in errs.items() if not e < 2e-2}
+    assert not bad, (bad, errs)
+
+
+def test_layer_backward_without_state_gradients():
+    errs = _run("f32", 64, (90, 33), M=5, K=3, seed=83, with_states=False)
+    bad = {k: e for k, e in errs.items() if not e < 1e-5}
+    assert not bad, bad
