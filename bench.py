@@ -407,6 +407,7 @@ def gpu_arm(args):
         configs = {extra_key(name, rule, mg): config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule, mg)
                    for name, rule, mg in EXTRA}
         configs["recurrence_backward"] = backward_bench(lay, w, x, cu, flush)
+        configs["layer_backward"] = layer_backward_bench(lay, w, x, cu, flush)
     clocks.__exit__(None, None, None)
     layer_roof["near_tie_tokens"] = near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)
     return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,
@@ -534,6 +535,35 @@ def backward_bench(lay, w, x, cu, flush, steps=3):
     out["value"] = w.n_tokens / (total / 1e3)
     out["unit"] = UNIT
     return out
+
+
+def layer_backward_bench(lay, w, x, cu, flush, steps=3):
+    """MoMLayer.backward after a forward on the same tokens (dout ~ N(0,1)):
+    every weight's and the tokens' gradients.  First path: the recurrences'
+    reverse passes token-serial and the gradient GEMMs on CUDA cores, float32."""
+    import torch
+    g = torch.Generator(device=x.device).manual_seed(2)
+    dout = torch.randn((w.n_tokens, w.heads, w.d_head), device=x.device, generator=g).to(x.dtype)
+    lay.forward(x, cu)
+    lay.backward(x, cu, dout)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        lay.forward(x, cu)
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lay.backward(x, cu, dout)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    errs = lay.device_errors()
+    if errs:
+        raise SystemExit("device error records in the layer backward: %s" % errs)
+    t = sum(ms) / steps
+    return {"workload": "backward of the %s layer (all weight and token gradients), dout ~ N(0,1)" % w.name,
+            "path": "recurrence reverse passes token-serial float32; gradient GEMMs float32 on CUDA cores",
+            "ms": t, "value": w.n_tokens / (t / 1e3), "unit": UNIT}
 
 
 def decode_bench(args, dev, world, rank, max_over_ranks, barrier):
