@@ -135,7 +135,11 @@ col_sums_kernel(const float* __restrict__ a, int64_t rows, int64_t lda, int64_t 
 }
 
 // ------------------------------------------------------------ grouped GEMM
-constexpr int GBM = 64, GBN = 64, GBK = 16;
+// 128 x 128 output tiles, 8-deep k steps double-buffered in shared memory,
+// 256 threads with 8 x 8 outputs each (two 4 x 4 blocks 64 apart in each
+// direction, so that a warp's shared-memory reads are broadcasts or
+// consecutive 16-byte chunks).
+constexpr int GBM = 128, GBN = 128, GBK = 8;
 
 struct GemmArgs {
     int trans_a;
@@ -154,23 +158,23 @@ struct GemmArgs {
     int accumulate;
     int64_t n_b_rows;          // rows of B (bounds of b_rows)
     void* err;
+    int splits;                // TRANS: the reduction of a group split over this many CTAs (atomic sums)
 };
 
-// trans_a = 0: the CTA's 64-row tile of a group (tiles listed over all groups)
+// trans_a = 0: the CTA's 128-row tile of a group (tiles listed over all groups)
 // trans_a = 1: blockIdx.z is the group, the tile of C_g is (blockIdx.y, blockIdx.x)
 template <typename TB>
 __global__ void __launch_bounds__(256)
 gemm_grouped_kernel(GemmArgs g) {
-    __shared__ float As[GBK][GBM + 4];
-    __shared__ float Bs[GBK][GBN + 4];
+    __shared__ __align__(16) float As[2][GBK][GBM];
+    __shared__ __align__(16) float Bs[2][GBK][GBN];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const TB* B = reinterpret_cast<const TB*>(g.B);
     const int64_t n0 = (int64_t)blockIdx.x * GBN;
-    int64_t m0, m1, k0, k1;
+    int64_t m0 = 0, m1 = 0, k0 = 0, k1 = 0;
     const TB* Bg = B;
     float* Cg = g.C;
     if (!g.trans_a) {
-        // find this tile's group: tiles are numbered group by group
         int64_t t = blockIdx.y;
         int grp = -1;
         for (int q = 0; q < g.n_groups; ++q) {
@@ -186,72 +190,105 @@ gemm_grouped_kernel(GemmArgs g) {
         k0 = 0;
         k1 = g.K;
     } else {
-        const int grp = blockIdx.z;
+        const int grp = blockIdx.z / g.splits, sp = blockIdx.z % g.splits;
         m0 = (int64_t)blockIdx.y * GBM;
         m1 = m0 + GBM < g.M ? m0 + GBM : g.M;
         if (m0 >= g.M) return;
-        k0 = g.goff[grp];
-        k1 = g.goff[grp + 1];
-        if (k0 < 0 || k1 < k0) { if (tid == 0 && blockIdx.x == 0) record_error(g.err, MOM_DEVERR_SEGMENT, grp); return; }
+        const int64_t lo = g.goff[grp], hi = g.goff[grp + 1];
+        if (lo < 0 || hi < lo) { if (tid == 0 && blockIdx.x == 0) record_error(g.err, MOM_DEVERR_SEGMENT, grp); return; }
+        // this CTA's share of the reduction, in whole k steps
+        const int64_t steps = (hi - lo + GBK - 1) / GBK, per = (steps + g.splits - 1) / g.splits;
+        k0 = lo + sp * per * GBK;
+        k1 = k0 + per * GBK < hi ? k0 + per * GBK : hi;
+        if (k0 >= k1) return;
         const int64_t w = g.gmem ? g.gmem[grp] : grp;
         Cg = g.C + w * g.c_group_stride;
     }
-    float acc[4][4];
+    // loader: 4 A values and 4 B values per thread per k step
+    float ra[4], rb[4];
+    auto load = [&](int64_t kb) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    for (int64_t kb = k0; kb < k1; kb += GBK) {
-        // A tile (GBK x GBM) and B tile (GBK x GBN), zero past the ends
-        for (int e = tid; e < GBK * GBM; e += 256) {
+        for (int e = 0; e < 4; ++e) {
             int kk, mm;
-            if (!g.trans_a) { mm = e / GBK; kk = e % GBK; } else { kk = e / GBM; mm = e % GBM; }
+            if (!g.trans_a) { mm = tid >> 1; kk = (tid & 1) * 4 + e; } else { kk = tid >> 5; mm = (tid & 31) * 4 + e; }
             const int64_t m = m0 + mm, k = kb + kk;
-            float v = 0.f;
-            if (m < m1 && k < k1) v = g.trans_a ? g.A[k * g.lda + m] : g.A[m * g.lda + k];
-            As[kk][mm] = v;
+            ra[e] = (m < m1 && k < k1) ? (g.trans_a ? g.A[k * g.lda + m] : g.A[m * g.lda + k]) : 0.f;
         }
-        for (int e = tid; e < GBK * GBN; e += 256) {
-            const int kk = e / GBN, nn = e % GBN;
-            const int64_t k = kb + kk, n = n0 + nn;
-            float v = 0.f;
-            if (k < k1 && n < g.N) {
-                int64_t br = k;
-                if (g.trans_a && g.b_rows) {
-                    br = g.b_rows[k];
-                    if (br < 0 || br >= g.n_b_rows) { record_error(g.err, MOM_DEVERR_ROW_INDEX, k); br = -1; }
-                }
-                if (br >= 0) v = to_f(Bg[br * g.ldb + n]);
-            }
-            Bs[kk][nn] = v;
+        const int kk = tid >> 5;
+        const int64_t k = kb + kk;
+        int64_t br = k;
+        if (k < k1 && g.trans_a && g.b_rows) {
+            br = g.b_rows[k];
+            if (br < 0 || br >= g.n_b_rows) { record_error(g.err, MOM_DEVERR_ROW_INDEX, k); br = -1; }
         }
-        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int64_t n = n0 + (tid & 31) * 4 + e;
+            rb[e] = (k < k1 && br >= 0 && n < g.N) ? to_f(Bg[br * g.ldb + n]) : 0.f;
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (!g.trans_a) As[buf][(tid & 1) * 4 + e][tid >> 1] = ra[e];
+            else As[buf][tid >> 5][(tid & 31) * 4 + e] = ra[e];
+        }
+        *reinterpret_cast<float4*>(&Bs[buf][tid >> 5][(tid & 31) * 4]) = make_float4(rb[0], rb[1], rb[2], rb[3]);
+    };
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    int buf = 0;
+    if (k0 < k1) {
+        load(k0);
+        store(0);
+    }
+    __syncthreads();
+    for (int64_t kb = k0; kb < k1; kb += GBK) {
+        const bool more = kb + GBK < k1;
+        if (more) load(kb + GBK);
 #pragma unroll
         for (int kk = 0; kk < GBK; ++kk) {
-            float a[4], b[4];
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
         }
+        if (more) store(buf ^ 1);
         __syncthreads();
+        buf ^= 1;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t m = m0 + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int64_t m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
         if (m >= m1) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t n = n0 + tx * 4 + j;
+        for (int j = 0; j < 8; ++j) {
+            const int64_t n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
             if (n >= g.N) continue;
             float* c = Cg + m * g.ldc + n;
-            *c = g.accumulate ? *c + acc[i][j] : acc[i][j];
+            if (g.trans_a) atomicAdd(c, acc[i][j]);          // split partial sums; C zeroed first unless accumulating
+            else *c = g.accumulate ? *c + acc[i][j] : acc[i][j];
         }
     }
+}
+
+// C_g = 0 for every group (the reduction form's partial sums are added into it)
+__global__ void __launch_bounds__(256)
+zero_groups_kernel(float* C, int64_t ldc, int64_t M, int64_t N, const int32_t* gmem, int64_t c_group_stride) {
+    const int grp = blockIdx.y;
+    const int64_t w = gmem ? gmem[grp] : grp;
+    float* Cg = C + w * c_group_stride;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < M * N; i += (int64_t)gridDim.x * blockDim.x)
+        Cg[(i / N) * ldc + i % N] = 0.f;
 }
 
 unsigned grid_rows(int64_t rows, int per_block) {
@@ -327,10 +364,22 @@ cudaError_t launch_gemm_grouped(int trans_a, const float* A, int64_t lda, const 
                                 cudaStream_t st) {
     if (n_groups == 0 || N == 0) return cudaSuccess;
     GemmArgs g{trans_a, A, lda, B, ldb, b_rows, C, ldc, M, N, K, goff, gmem, n_groups, b_group_stride,
-               c_group_stride, accumulate, n_b_rows, err};
+               c_group_stride, accumulate, n_b_rows, err, 1};
     dim3 grid;
-    if (!trans_a) grid = dim3((unsigned)cdiv(N, GBN), (unsigned)(cdiv(total_rows, GBM) + n_groups), 1);
-    else grid = dim3((unsigned)cdiv(N, GBN), (unsigned)cdiv(M, GBM), (unsigned)n_groups);
+    if (!trans_a) {
+        grid = dim3((unsigned)cdiv(N, GBN), (unsigned)(cdiv(total_rows, GBM) + n_groups), 1);
+    } else {
+        // split each group's reduction until there are ~4 CTAs per SM
+        const int64_t tiles = cdiv(N, GBN) * cdiv(M, GBM) * n_groups;
+        int64_t sp = cdiv(148 * 4, tiles);
+        g.splits = (int)(sp < 1 ? 1 : sp > 64 ? 64 : sp);
+        grid = dim3((unsigned)cdiv(N, GBN), (unsigned)cdiv(M, GBM), (unsigned)(n_groups * g.splits));
+        if (!accumulate) {
+            zero_groups_kernel<<<dim3((unsigned)grid_rows(M * N, 256), (unsigned)n_groups), 256, 0, st>>>(
+                C, ldc, M, N, gmem, c_group_stride);
+            count_launches(1);
+        }
+    }
     if (dt == MOM_BF16) gemm_grouped_kernel<bf16><<<grid, 256, 0, st>>>(g);
     else gemm_grouped_kernel<float><<<grid, 256, 0, st>>>(g);
     count_launches(1);
