@@ -17,7 +17,13 @@ shared memory, memory-count scaling to 16):
 * varlen workloads draw sequence lengths U{512..2048} until the packed batch
   reaches the token budget, the last length clipped to the remainder;
 * with per-memory gates, each routed memory's W_beta, W_a ~ N(0, 1/d_model),
-  A ~ U(0, 2.7), b_a ~ U(-4, 0), from a stream of their own.
+  A ~ U(0, 2.7), b_a ~ U(-4, 0), from a stream of their own;
+* with the Gated DeltaNet block around the memories, from a stream of their
+  own: the output gate W_g ~ N(0, 1/d_model), the output projection W_o ~
+  N(0, 1/(H d)), the short convolutions' weights (width 4, one filter per
+  channel of q, k, v, shared and per memory) ~ U(-1/2, 1/2) (the default
+  initialisation of a depthwise convolution of width 4: bound 1/sqrt(4)),
+  float32, and the norm weight ~ U(0.5, 1.5) per head channel, float32.
 
 Storage layout of every projection weight is [out_features, in_features]
 (y = x @ W.T).  In bf16 workloads every array that the kernels read as bf16
@@ -51,6 +57,8 @@ class Workload:
     decode_steps: int = 0       # >0: recurrent decode workload
     prefill_len: int = 0
     mem_gates: bool = False     # every routed memory has its own W_beta, W_a, A, b_a
+    block: bool = False         # the Gated DeltaNet block around the memories (conv, norm, gate, W_o)
+    conv_width: int = 4         # taps of the block's short convolutions
 
     @property
     def n_tokens(self) -> int:
@@ -70,6 +78,9 @@ WORKLOADS: Dict[str, Workload] = {
     "mom380m_skew_varlen": Workload("mom380m_skew_varlen", 0, 0, 1024, 4, 256, 4, 2,
                                     "bf16", seed=2, router_bias0=2.0,
                                     varlen_total=16384),
+    # the 380M-shape layer inside its Gated DeltaNet block (the same tokens and
+    # memory weights as mom380m, the block's weights from a stream of their own)
+    "mom380m_block": Workload("mom380m_block", 8, 2048, 1024, 4, 256, 4, 2, "bf16", seed=1, block=True),
     # 1.3B-shape memory-scaling forward: 16 memories, top-4
     "mom1p3b_m16": Workload("mom1p3b_m16", 4, 4096, 2048, 8, 256, 16, 4, "bf16", seed=3),
     # recurrent decode: 256 sequences, 8 memories top-2, one token per step
@@ -142,6 +153,18 @@ def make_weights(w: Workload, rng: np.random.Generator,
         p["w_a_mem"] = _act(g.standard_normal((w.n_mem, w.heads, D), dtype=np.float32) * std, w.dtype)
         p["A_mem"] = g.uniform(0.0, 2.7, size=(w.n_mem, w.heads)).astype(np.float32)
         p["b_a_mem"] = g.uniform(-4.0, 0.0, size=(w.n_mem, w.heads)).astype(np.float32)
+    if w.block:
+        g = np.random.default_rng((w.seed, 2))
+        W = w.conv_width
+        conv = lambda *shape: g.uniform(-0.5, 0.5, size=shape + (W,)).astype(np.float32)
+        p["w_g"] = _act(g.standard_normal((Hd, D), dtype=np.float32) * std, w.dtype)
+        p["w_o"] = _act(g.standard_normal((D, Hd), dtype=np.float32) / np.sqrt(Hd), w.dtype)
+        p["conv_q"] = conv(Hd)
+        p["conv_k_sh"] = conv(Hd)
+        p["conv_v_sh"] = conv(Hd)
+        p["conv_k"] = conv(w.n_mem, Hd)
+        p["conv_v"] = conv(w.n_mem, Hd)
+        p["w_norm"] = g.uniform(0.5, 1.5, size=w.d_head).astype(np.float32)
     return p
 
 
