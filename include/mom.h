@@ -547,6 +547,92 @@ mom_status mom_decode_step_rule(const void* x, const mom_weights* w, const mom_m
                                 float* state, void* out, int32_t* topk_idx,
                                 void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The Gated DeltaNet block around the memories.  The pages name Gated
+ * DeltaNet as each memory's token mixer (the authors' MoM blog post,
+ * experiments section) and print nothing of the block that holds it; the
+ * calls below are the plain Gated DeltaNet block's steps, in bf16:
+ *
+ *   q^, k^_sh, v^_sh, g = x [W_q | W_k_sh | W_v_sh | W_g]^T     (unnormalised)
+ *   k^_p, v^_p          = x_perm [W_k^m | W_v^m]^T              (mom_block_proj)
+ *   q = l2norm(SiLU(conv(q^))), k likewise, v = SiLU(conv(v^))  (mom_short_conv)
+ *   the recurrences and the combine as in the layer, then per head
+ *   o~ = o / sqrt(mean(o^2) + eps) * w_norm * SiLU(g)           (mom_combine_norm_gate)
+ *   y  = o~ W_o^T                                               (mom_linear)
+ *
+ * conv is a causal depthwise convolution along the rows a recurrence sees
+ * (a sequence for the shared q, k, v; a (memory, sequence) segment of the
+ * reordered rows for memory m's k, v, with memory m's own filters).
+ * ---------------------------------------------------------------------- */
+
+/* mom_block_proj -- the layer's projection GEMM in the block's form: every
+ * output unnormalised (the norm follows the convolution) and the output gate
+ * as a fourth shared part.  w_shared4 [4*H*d, d_model] (rows W_q | W_k_sh |
+ * W_v_sh | W_g); w_kv, perm_token, mem_offset and the routed outputs as in
+ * mom_kv_proj_grouped; q, k_sh, v_sh, g [n_tok, H*d]; k_p, v_p [n_tok*top_k,
+ * H*d].  bf16 only (MOM_ERR_UNSUPPORTED otherwise), H*d a multiple of 256,
+ * d_model of 64; every pointer 16-byte aligned.  ws: MOM_WS_HEADER_BYTES. */
+mom_status mom_block_proj(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
+                          const void* w_shared4, const void* w_kv, mom_dtype dt,
+                          int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k,
+                          void* q, void* k_sh, void* v_sh, void* g, void* k_p, void* v_p,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* mom_short_conv -- out[r, c] = SiLU(sum_{j<width} w[grp, width-1-j, c] *
+ * z[r-j, c]) over the taps with r-j >= the start of r's segment, then, when
+ * l2norm is 1, each head of head_dim channels divided by sqrt(|.|^2 +
+ * 1e-6).  Segment s covers rows seg_cu[s] .. seg_cu[s+1]-1 (device int32
+ * [n_seg+1], non-decreasing, seg_cu[n_seg] <= n_rows); its filters are group
+ * grp = s / seg_per_group (< n_groups).  Rows outside every segment are not
+ * written.  z, out [n_rows, channels] bf16, distinct buffers, 16-byte
+ * aligned; w [n_groups, width, channels] float32, tap-major (w[grp, j, c];
+ * tap width-1 multiplies the current row), 16-byte aligned.  channels a multiple of 8; width 1..4; with l2norm, head_dim
+ * a power of two in 8..256 dividing channels.  Corrupt segment bounds are
+ * recorded in ws (MOM_DEVERR_SEGMENT).  ws: MOM_WS_HEADER_BYTES. */
+mom_status mom_short_conv(const void* z, int64_t n_rows, int channels, const int32_t* seg_cu, int n_seg,
+                          int seg_per_group, int n_groups, const float* w, int width, int head_dim,
+                          int l2norm, mom_dtype dt, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* One convolution of a batch (fields as the arguments of mom_short_conv). */
+typedef struct mom_conv_problem {
+    const void*    z;
+    void*          out;
+    int64_t        n_rows;
+    const int32_t* seg_cu;
+    int            n_seg;
+    int            seg_per_group;
+    int            n_groups;
+    const float*   w;
+    int            l2norm;
+} mom_conv_problem;
+
+/* mom_short_conv_batch -- 1..8 convolutions of the same channel count, width
+ * and head_dim in one launch (the block's five: q, k_sh, v_sh over the
+ * sequences, k_p, v_p over the memory segments).  `problems` is a HOST
+ * array read during the call only; each problem is validated as in
+ * mom_short_conv. */
+mom_status mom_short_conv_batch(const mom_conv_problem* problems, int n_problems, int channels, int width,
+                                int head_dim, mom_dtype dt, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_combine_norm_gate -- the combine of mom_combine_unpermute followed,
+ * per head of d channels, by the block's gated RMS norm:
+ *   o = o_sh[t] + sum_j topk_gate[t,j] o_p[row_of[t*top_k+j]],
+ *   out[t] = o / sqrt(mean(o^2) + eps) * w_norm * SiLU(g[t]).
+ * o_sh, g, out [n_tok, H*d], o_p [n_tok*top_k, H*d] bf16; w_norm [d]
+ * float32; d a power of two in 8..256; every array 16-byte aligned.  Row
+ * errors as in the combine. */
+mom_status mom_combine_norm_gate(const void* o_sh, const void* o_p, const int32_t* row_of,
+                                 const float* topk_gate, const void* g, const float* w_norm, float eps,
+                                 int64_t n_tok, int top_k, int H, int d, mom_dtype dt, void* out,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* mom_linear -- y = x w^T on the tensor cores (the block's output
+ * projection): x [n_rows, k_in], w [n_out, k_in], y [n_rows, n_out], bf16,
+ * fp32 accumulation; k_in a multiple of 64, n_out of 256; 16-byte aligned.
+ * ws: MOM_WS_HEADER_BYTES. */
+mom_status mom_linear(const void* x, const void* w, mom_dtype dt, int64_t n_rows, int k_in, int n_out, void* y,
+                      void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -74,6 +74,12 @@ SIGNATURES = {
                               _I, _I64, _I64, _I, _VP, _SZ, _VP]),
     "mom_memory_chunk_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I, _I,
                                   _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mom_block_proj": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP,
+                            _VP, _SZ, _VP]),
+    "mom_short_conv": (_I, [_VP, _I64, _I, _VP, _I, _I, _I, _VP, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
+    "mom_short_conv_batch": (_I, [_VP, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
+    "mom_combine_norm_gate": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _F, _I64, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
+    "mom_linear": (_I, [_VP, _VP, _I, _I64, _I, _I, _VP, _VP, _SZ, _VP]),
 }
 
 
@@ -81,6 +87,12 @@ class MomWeights(ctypes.Structure):
     """Mirror of ``struct mom_weights`` (device pointers)."""
     _fields_ = [("w_r", c_void_p), ("b_r", c_void_p), ("w_shared", c_void_p), ("w_gate", c_void_p),
                 ("A", c_void_p), ("b_a", c_void_p), ("w_kv", c_void_p)]
+
+
+class MomConvProblem(ctypes.Structure):
+    """Mirror of ``struct mom_conv_problem``."""
+    _fields_ = [("z", c_void_p), ("out", c_void_p), ("n_rows", c_int64), ("seg_cu", c_void_p), ("n_seg", c_int),
+                ("seg_per_group", c_int), ("n_groups", c_int), ("w", c_void_p), ("l2norm", c_int)]
 
 
 class MomMemoryGates(ctypes.Structure):
@@ -397,6 +409,63 @@ def mom_combine_unpermute(o_sh, o_p, row_of, topk_gate, out, ws, stream=None):
     _check(lib.mom_combine_unpermute(_p(o_sh), _p(o_p), _p(row_of), _p(topk_gate), n_tok, top_k, H, d,
                                      dtype_code(o_sh.dtype), _p(out), _p(ws), ws.numel(), _s(stream)),
            "mom_combine_unpermute")
+
+
+# -------------------------------------------------- the Gated DeltaNet block
+
+def mom_block_proj(x, perm, mem_offset, w_shared4, w_kv, H, d, top_k, q, k_sh, v_sh, g, k_p, v_p, ws, stream=None):
+    """Unnormalised q, k_sh, v_sh, the output gate g (x W_shared4^T) and the
+    routed rows' unnormalised k_p, v_p."""
+    n_tok, d_model = x.shape
+    _check(lib.mom_block_proj(_p(x), _p(perm), _p(mem_offset), _p(w_shared4), _p(w_kv), dtype_code(x.dtype), n_tok,
+                              d_model, H, d, w_kv.shape[0], top_k, _p(q), _p(k_sh), _p(v_sh), _p(g), _p(k_p), _p(v_p),
+                              _p(ws), ws.numel(), _s(stream)), "mom_block_proj")
+
+
+def mom_short_conv(z, seg_cu, w, out, ws, seg_per_group=None, head_dim=0, l2norm=False, stream=None, n_rows=None):
+    """out = SiLU(causal depthwise conv of z along the segments of seg_cu)
+    (then the per-head L2 norm when l2norm); w [n_groups, width, C] float32
+    (tap-major), segment s using group s // seg_per_group (default: one
+    group)."""
+    n = z.shape[0] if n_rows is None else n_rows
+    C = z.numel() // max(z.shape[0], 1)
+    n_seg = seg_cu.numel() - 1
+    n_groups, width, _ = w.shape
+    spg = n_seg if seg_per_group is None else seg_per_group
+    _check(lib.mom_short_conv(_p(z), n, C, _p(seg_cu), n_seg, spg, n_groups, _p(w), width, head_dim, int(l2norm),
+                              dtype_code(z.dtype), _p(out), _p(ws), ws.numel(), _s(stream)), "mom_short_conv")
+
+
+def mom_short_conv_batch(problems, head_dim, ws, stream=None):
+    """problems: a list of dicts with z, out, seg_cu, w and optionally
+    seg_per_group (default: one group), l2norm; the same channel count and
+    width for all."""
+    arr = (MomConvProblem * len(problems))()
+    C = width = None
+    for i, q in enumerate(problems):
+        z, seg_cu, w = q["z"], q["seg_cu"], q["w"]
+        n_seg = seg_cu.numel() - 1
+        C = z.numel() // max(z.shape[0], 1)
+        width = w.shape[1]
+        arr[i] = MomConvProblem(_p(z).value, _p(q["out"]).value, z.shape[0], _p(seg_cu).value, n_seg,
+                                q.get("seg_per_group") or n_seg, w.shape[0], _p(w).value, int(q.get("l2norm", False)))
+    _check(lib.mom_short_conv_batch(arr, len(problems), C, width, head_dim, dtype_code(problems[0]["z"].dtype),
+                                    _p(ws), ws.numel(), _s(stream)), "mom_short_conv_batch")
+
+
+def mom_combine_norm_gate(o_sh, o_p, row_of, topk_gate, g, w_norm, eps, out, ws, stream=None):
+    n_tok, H, d = o_sh.shape
+    top_k = topk_gate.shape[1]
+    _check(lib.mom_combine_norm_gate(_p(o_sh), _p(o_p), _p(row_of), _p(topk_gate), _p(g), _p(w_norm), eps, n_tok,
+                                     top_k, H, d, dtype_code(o_sh.dtype), _p(out), _p(ws), ws.numel(), _s(stream)),
+           "mom_combine_norm_gate")
+
+
+def mom_linear(x, w, y, ws, stream=None):
+    """y = x w^T (x [n, k_in], w [n_out, k_in])."""
+    n, k_in = x.shape
+    _check(lib.mom_linear(_p(x), _p(w), dtype_code(x.dtype), n, k_in, w.shape[0], _p(y), _p(ws), ws.numel(),
+                          _s(stream)), "mom_linear")
 
 
 def mom_decode_workspace_size(B, d_model, H, d, n_mem, top_k):

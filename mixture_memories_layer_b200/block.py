@@ -1,0 +1,128 @@
+"""The MoM layer inside its Gated DeltaNet block, on the GPU.
+
+The pages name Gated DeltaNet as every memory's token mixer (the authors'
+MoM blog post, experiments section) and print nothing of the block around
+it; the plain Gated DeltaNet block is taken:
+
+    router -> permute -> projections (unnormalised, plus the output gate g)
+           -> short causal convolutions + SiLU (+ L2 norm of q, k)
+           -> GDN prep / walks (shared | routed) -> combine + gated RMS norm
+           -> output projection W_o
+
+Every step runs in the CUDA library (mom_block_proj, mom_short_conv, the
+recurrences, mom_combine_norm_gate, mom_linear); this module packs weights,
+holds buffers and passes pointers.  bf16 only.
+"""
+from __future__ import annotations
+
+from typing import Dict
+
+import numpy as np
+import torch
+
+from . import binding as B
+from .layer import MoMLayer, pack_weights
+
+RMS_EPS = 1e-5
+
+
+def pack_block_weights(p: Dict[str, np.ndarray], dtype: torch.dtype, device="cuda") -> Dict[str, torch.Tensor]:
+    """pack_weights plus the block's: w_shared4 = [W_q; W_k_sh; W_v_sh; W_g],
+    w_o [d_model, H d], the convolution filters tap-major as float32 [groups,
+    width, H d] (conv_q, conv_k_sh, conv_v_sh: one group; conv_k, conv_v: one
+    group per memory) and w_norm [d]."""
+    w = pack_weights(p, dtype, device)
+    t = lambda a, dt=dtype: torch.as_tensor(np.ascontiguousarray(a)).to(device=device, dtype=dt)
+    f32 = torch.float32
+    w["w_shared4"] = t(np.concatenate([p["w_q"], p["w_k_sh"], p["w_v_sh"], p["w_g"]], axis=0))
+    w["w_o"] = t(p["w_o"])
+    for name in ("conv_q", "conv_k_sh", "conv_v_sh"):
+        w[name] = t(np.swapaxes(p[name][None], 1, 2), f32)
+    w["conv_k"] = t(np.swapaxes(p["conv_k"], 1, 2), f32)
+    w["conv_v"] = t(np.swapaxes(p["conv_v"], 1, 2), f32)
+    w["w_norm"] = t(p["w_norm"], f32)
+    return w
+
+
+class MoMBlock(MoMLayer):
+    """The layer with its block: forward(x, cu_seqlens)["y"] [N, d_model]."""
+
+    def __init__(self, weights: Dict[str, torch.Tensor], heads: int, d_head: int, top_k: int, scale: float = 1.0,
+                 gdn_schedule: str = "streams", rule: str = "gated_delta", eps: float = RMS_EPS):
+        super().__init__(weights, heads, d_head, top_k, scale, gdn_schedule, rule)
+        if self.dtype != torch.bfloat16:
+            raise ValueError("the block runs in bf16")
+        self.eps = eps
+
+    def block_buffers(self, n_tok: int, n_seq: int):
+        b = self.buffers(n_tok, n_seq)
+        H, d, K, dt = self.H, self.d, self.top_k, self.dtype
+        for name, rows in (("q_raw", n_tok), ("k_sh_raw", n_tok), ("v_sh_raw", n_tok), ("g", n_tok),
+                           ("k_p_raw", n_tok * K), ("v_p_raw", n_tok * K), ("o_tilde", n_tok)):
+            b[name] = self._buf(name, (rows, H, d), dt)
+        b["y"] = self._buf("y", (n_tok, self.d_model), dt)
+        b["ws_conv"] = self._ws("conv", B.MOM_WS_HEADER_BYTES)
+        b["ws_lin"] = self._ws("lin", B.MOM_WS_HEADER_BYTES)
+        return b
+
+    def forward(self, x: torch.Tensor, cu_seqlens: torch.Tensor, h0_shared=None, h0_mem=None,
+                want_states: bool = True, stream=None, marks=None) -> Dict[str, torch.Tensor]:
+        """x [N, d_model] bf16, cu_seqlens [S+1] int32 (device).  Returns the
+        buffers dict: ``y`` the block output, ``o_tilde`` the normalised and
+        gated memories' output, ``h_shared`` / ``h_mem`` the final states.
+        ``marks``: optional 7 CUDA events, recorded before the first call and
+        after each of router, permute, projections + convolutions, GDN,
+        combine + norm, output projection."""
+        n_tok = x.shape[0]
+        n_seq = cu_seqlens.numel() - 1
+        w, b = self.w, self.block_buffers(n_tok, n_seq)
+        st = stream if stream is not None else torch.cuda.current_stream()
+        mark = (lambda i: marks[i].record(st)) if marks is not None else (lambda i: None)
+        side = self._side_stream()
+        mark(0)
+        start = torch.cuda.Event()
+        start.record(st)
+        side.wait_event(start)
+        B.mom_gate_proj(x, w["w_gate"], w["A"], w["b_a"], b["beta"], b["log_alpha"], b["ws_gate"], stream=side)
+        gates_done = torch.cuda.Event()
+        gates_done.record(side)
+        B.mom_router_topk(x, w["w_r"], w["b_r"], self.top_k, b["idx"], b["gate"], stream=st)
+        mark(1)
+        B.mom_permute(b["idx"], self.n_mem, cu_seqlens, b["perm"], b["row_of"], b["mem_offset"], b["seg_cu"],
+                      b["ws_perm"], stream=st)
+        if self.mem_gates:
+            permuted = torch.cuda.Event()
+            permuted.record(st)
+            side.wait_event(permuted)
+            B.mom_mem_gate_proj(x, b["perm"], b["mem_offset"], w["w_gate_mem"], w["A_mem"], w["b_a_mem"],
+                                self.top_k, b["beta_p"], b["log_alpha_p"], b["ws_mem_gate"], stream=side)
+            gates_done.record(side)
+        mark(2)
+        B.mom_block_proj(x, b["perm"], b["mem_offset"], w["w_shared4"], w["w_kv"], self.H, self.d, self.top_k,
+                         b["q_raw"], b["k_sh_raw"], b["v_sh_raw"], b["g"], b["k_p_raw"], b["v_p_raw"], b["ws_proj"],
+                         stream=st)
+        # one launch for the five convolutions; memory m's rows of sequence s
+        # are segment m * S + s of seg_cu
+        B.mom_short_conv_batch([
+            dict(z=b["q_raw"], out=b["q"], seg_cu=cu_seqlens, w=w["conv_q"], l2norm=True),
+            dict(z=b["k_sh_raw"], out=b["k_sh"], seg_cu=cu_seqlens, w=w["conv_k_sh"], l2norm=True),
+            dict(z=b["v_sh_raw"], out=b["v_sh"], seg_cu=cu_seqlens, w=w["conv_v_sh"]),
+            dict(z=b["k_p_raw"], out=b["k_p"], seg_cu=b["seg_cu"], w=w["conv_k"], seg_per_group=n_seq, l2norm=True),
+            dict(z=b["v_p_raw"], out=b["v_p"], seg_cu=b["seg_cu"], w=w["conv_v"], seg_per_group=n_seq),
+        ], self.d, b["ws_conv"], stream=st)
+        st.wait_event(gates_done)
+        mark(3)
+        self._gdn_calls(b, cu_seqlens, h0_shared, h0_mem, want_states, st, side)
+        mark(4)
+        B.mom_combine_norm_gate(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["g"], w["w_norm"], self.eps,
+                                b["o_tilde"], b["ws_comb"], stream=st)
+        mark(5)
+        B.mom_linear(b["o_tilde"].view(n_tok, -1), w["w_o"], b["y"], b["ws_lin"], stream=st)
+        mark(6)
+        return b
+
+    def decode_step(self, *a, **k):
+        raise NotImplementedError("the block's decode (convolution states per sequence and memory) is not provided")
+
+    def backward(self, *a, **k):
+        raise NotImplementedError("the block's backward is not provided (MoMLayer.backward is the layer's)")

@@ -420,6 +420,99 @@ mom_status mom_gemm_grouped(int trans_a, const float* A, int64_t lda, const void
                                            accumulate, ws, as_stream(stream)));
 }
 
+// ------------------------------------------------------------------- block
+mom_status mom_block_proj(const void* x, const int32_t* perm_token, const int32_t* mem_offset,
+                          const void* w_shared4, const void* w_kv, mom_dtype dt,
+                          int64_t n_tok, int d_model, int H, int d, int n_mem, int top_k,
+                          void* q, void* k_sh, void* v_sh, void* g, void* k_p, void* v_p,
+                          void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || d_model <= 0 || d_model % 64 != 0) return MOM_ERR_ARG;
+    if (H < 1 || H > MOM_MAX_HEADS || top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM) return MOM_ERR_ARG;
+    if (!head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (n_tok * top_k >= ((int64_t)1 << 31)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {x, perm_token, mem_offset, w_shared4, w_kv, q, k_sh, v_sh, g, k_p, v_p};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    ProjArgs a{x, perm_token, mem_offset, w_shared4, w_kv, n_tok, d_model, H, d, n_mem, top_k,
+               q, k_sh, v_sh, k_p, v_p, ws};
+    a.raw = 1;
+    a.g = g;
+    if (!proj_tc_supported(a, dt)) return MOM_ERR_UNSUPPORTED;
+    return cuda_status(launch_proj_tc(a, as_stream(stream)));
+}
+
+namespace {
+mom_status conv_check(const mom_conv_problem& q, int channels, int head_dim) {
+    if (q.n_rows < 0 || q.n_seg < 1 || q.seg_per_group < 1 || q.n_groups < 1) return MOM_ERR_ARG;
+    if (q.l2norm != 0 && q.l2norm != 1) return MOM_ERR_ARG;
+    if (q.l2norm && (head_dim < 8 || head_dim > 256 || (head_dim & (head_dim - 1)) != 0 || channels % head_dim != 0))
+        return MOM_ERR_ARG;
+    if (q.n_rows > 0 && (!q.z || !q.out || !q.seg_cu || !q.w || !al16(q.z) || !al16(q.out) || !al16(q.w) ||
+                         q.z == q.out))
+        return MOM_ERR_ARG;
+    return MOM_OK;
+}
+}  // namespace
+
+mom_status mom_short_conv_batch(const mom_conv_problem* problems, int n_problems, int channels, int width,
+                                int head_dim, mom_dtype dt, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || !problems || n_problems < 1 || channels < 8 || channels % 8 != 0 || width < 1)
+        return MOM_ERR_ARG;
+    if (dt != MOM_BF16 || width > 4 || n_problems > 8) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    ConvProblem pr[8];
+    int n = 0;
+    for (int i = 0; i < n_problems; ++i) {
+        const mom_conv_problem& q = problems[i];
+        const mom_status e = conv_check(q, channels, head_dim);
+        if (e != MOM_OK) return e;
+        if (q.n_rows > 0)
+            pr[n++] = ConvProblem{q.z, q.out, q.n_rows, q.seg_cu, q.n_seg, q.seg_per_group, q.n_groups, q.w, q.l2norm};
+    }
+    if (n == 0) return MOM_OK;
+    return cuda_status(launch_short_conv(pr, n, channels, width, head_dim, ws, as_stream(stream)));
+}
+
+mom_status mom_short_conv(const void* z, int64_t n_rows, int channels, const int32_t* seg_cu, int n_seg,
+                          int seg_per_group, int n_groups, const float* w, int width, int head_dim,
+                          int l2norm, mom_dtype dt, void* out, void* ws, size_t ws_bytes, void* stream) {
+    const mom_conv_problem q{z, out, n_rows, seg_cu, n_seg, seg_per_group, n_groups, w, l2norm};
+    return mom_short_conv_batch(&q, 1, channels, width, head_dim, dt, ws, ws_bytes, stream);
+}
+
+mom_status mom_combine_norm_gate(const void* o_sh, const void* o_p, const int32_t* row_of,
+                                 const float* topk_gate, const void* g, const float* w_norm, float eps,
+                                 int64_t n_tok, int top_k, int H, int d, mom_dtype dt, void* out,
+                                 void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || top_k < 1 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (d < 8 || d > 256 || (d & (d - 1)) != 0 || !(eps >= 0.f)) return MOM_ERR_ARG;
+    if (dt != MOM_BF16) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_tok == 0) return MOM_OK;
+    const void* ptrs[] = {o_sh, o_p, row_of, topk_gate, g, w_norm, out};
+    for (const void* p : ptrs)
+        if (!p) return MOM_ERR_ARG;
+    if (!al16(o_sh) || !al16(o_p) || !al16(g) || !al16(out) || !al16(w_norm)) return MOM_ERR_ARG;
+    return cuda_status(launch_combine_norm_gate(o_sh, o_p, row_of, topk_gate, g, w_norm, eps, n_tok, top_k, H, d,
+                                                out, ws, as_stream(stream)));
+}
+
+mom_status mom_linear(const void* x, const void* w, mom_dtype dt, int64_t n_rows, int k_in, int n_out, void* y,
+                      void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_rows < 0 || k_in <= 0 || n_out <= 0) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_rows == 0) return MOM_OK;
+    if (!x || !w || !y || !al16(x) || !al16(w) || !al16(y)) return MOM_ERR_ARG;
+    ProjArgs a{x, nullptr, nullptr, w, nullptr, n_rows, k_in, 1, n_out, 1, 1,
+               y, nullptr, nullptr, nullptr, nullptr, ws};
+    a.parts = PROJ_SHARED;
+    a.plain_n = n_out;
+    if (!proj_tc_supported(a, dt)) return MOM_ERR_UNSUPPORTED;
+    return cuda_status(launch_proj_tc(a, as_stream(stream)));
+}
+
 // ----------------------------------------------------------------- combine
 mom_status mom_combine_unpermute(const void* o_sh, const void* o_p, const int32_t* row_of,
                                  const float* topk_gate, int64_t n_tok, int top_k, int H, int d,

@@ -84,6 +84,14 @@ struct ProjArgs {
     float* q_norm = nullptr;
     float* k_sh_norm = nullptr;
     float* k_p_norm = nullptr;
+    // the Gated DeltaNet block's form: raw = 1 leaves q, k_sh and k_p
+    // unnormalised (the norm follows the short convolution); g non-null adds
+    // the output gate x W_g^T as a fourth shared part (w_shared holds
+    // [W_q | W_k_sh | W_v_sh | W_g]); plain_n > 0 makes the shared problem
+    // one plain product y = x w_shared^T of plain_n columns, written to q
+    int raw = 0;
+    void* g = nullptr;
+    int plain_n = 0;
     __host__ __device__ int groups() const { return n_groups > 0 ? n_groups : M; }
     __host__ __device__ int64_t routed_rows() const { return n_routed >= 0 ? n_routed : n_tok * K; }
 };
@@ -202,5 +210,22 @@ struct DecodeArgs {
     const float *beta_p = nullptr, *log_alpha_p = nullptr;
 };
 cudaError_t launch_decode_state(const DecodeArgs& a, int dt, cudaStream_t st);
+
+// conv.cu: the block's short causal convolutions (SiLU, optional per-head L2
+// norm), up to 8 problems of the same channel count per launch
+struct ConvProblem {
+    const void* z;
+    void* out;
+    int64_t n_rows;
+    const int32_t* seg_cu;
+    int n_seg, seg_per_group, n_groups;
+    const float* w;               // [n_groups, W, C] (tap-major)
+    int l2;
+};
+cudaError_t launch_short_conv(const ConvProblem* problems, int n, int C, int W, int d, void* err, cudaStream_t st);
+// combine.cu: the combine with the block's gated per-head RMS norm
+cudaError_t launch_combine_norm_gate(const void* o_sh, const void* o_p, const int32_t* row_of, const float* gate,
+                                     const void* g, const float* w_norm, float eps, int64_t n_tok, int K, int H,
+                                     int d, void* out, void* ws, cudaStream_t st);
 
 }  // namespace mom

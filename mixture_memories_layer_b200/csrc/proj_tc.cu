@@ -8,7 +8,11 @@
 //             perm_token[r]) x [W_k^m | W_v^m]^T           -> k_p, v_p
 // Output tiles are 128 rows x 256 columns; a tile never straddles two
 // memories or two projections, and holds whole heads, so the per-head L2
-// norm of q and k is applied in the epilogue straight from TMEM.
+// norm of q and k is applied in the epilogue straight from TMEM.  In the
+// Gated DeltaNet block's form the outputs stay unnormalised (the short
+// convolution comes first) and the shared problem has a fourth part, the
+// output gate x W_g^T; the same kernel also runs one plain product
+// y = x W^T (the block's output projection).
 //
 // Roles (416 threads, one CTA per SM, persistent over tiles):
 //   warps 0-3  producers: A rows gathered with 16-byte cp.async into the
@@ -49,8 +53,10 @@ struct TcParams {
     const int32_t* perm;
     const int32_t* mem_offset;       // routed group offsets [n_groups + 1]
     const int32_t* group_mem;        // memory of each group (null: group g = memory g)
-    bf16 *q, *k_sh, *v_sh, *k_p, *v_p;
+    bf16 *q, *k_sh, *v_sh, *k_p, *v_p, *g;
     int64_t n_tok, n_routed;
+    int sh_parts, part_w;   // shared problem: parts (q, k_sh, v_sh[, g]) of part_w columns each
+    int raw;                // 1: no L2 norm in the epilogue
     int D, H, d, M, K, n_groups;
     float *q_norm, *k_sh_norm, *k_p_norm;     // optional per-(row, head) lengths
     int sh_ct, rt_ct;       // column tiles per row tile (shared / routed)
@@ -97,7 +103,7 @@ __device__ __forceinline__ bool tile_at(const TcParams& p, int64_t t, Tile& T) {
 }
 
 struct OutMaps {
-    CUtensorMap q, k_sh, v_sh, k_p, v_p;   // [rows, H*d] bf16, boxes of 32 rows x 64 columns
+    CUtensorMap q, k_sh, v_sh, k_p, v_p, g;   // [rows, columns] bf16, boxes of 32 rows x 64 columns
 };
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -233,24 +239,26 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
             const int64_t row = T.r0 + row_local;
             const bool live = row < T.r1;
             const int col0 = T.ct * BN;
-            const int part_i = col0 / Hd, cc0 = col0 % Hd;
+            const int pw = T.m < 0 ? p.part_w : Hd;          // columns of the tile's output part
+            const int part_i = col0 / pw, cc0 = col0 % pw;
             bf16* base;
             bool norm;
             float* nout;
             if (T.m < 0) {
-                base = part_i == 0 ? p.q : part_i == 1 ? p.k_sh : p.v_sh;
-                norm = part_i < 2;
-                nout = part_i == 0 ? p.q_norm : part_i == 1 ? p.k_sh_norm : nullptr;
+                base = part_i == 0 ? p.q : part_i == 1 ? p.k_sh : part_i == 2 ? p.v_sh : p.g;
+                norm = !p.raw && p.sh_parts >= 3 && part_i < 2;
+                nout = !norm ? nullptr : part_i == 0 ? p.q_norm : p.k_sh_norm;
             } else {
                 base = part_i == 0 ? p.k_p : p.v_p;
-                norm = part_i == 0;
-                nout = part_i == 0 ? p.k_p_norm : nullptr;
+                norm = !p.raw && part_i == 0;
+                nout = norm ? p.k_p_norm : nullptr;
             }
-            const CUtensorMap* omap = T.m < 0 ? (part_i == 0 ? &om.q : part_i == 1 ? &om.k_sh : &om.v_sh)
-                                              : (part_i == 0 ? &om.k_p : &om.v_p);
+            const CUtensorMap* omap =
+                T.m < 0 ? (part_i == 0 ? &om.q : part_i == 1 ? &om.k_sh : part_i == 2 ? &om.v_sh : &om.g)
+                        : (part_i == 0 ? &om.k_p : &om.v_p);
             // a piece goes out by TMA only when all 32 of its rows belong to this tile
             const bool full_piece = T.r0 + 32 * qd + 32 <= T.r1;
-            bf16* orow = base + (live ? row : 0) * (int64_t)Hd + cc0 + hf * HALF;
+            bf16* orow = base + (live ? row : 0) * (int64_t)pw + cc0 + hf * HALF;
             const uint32_t taddr = tmem_base + ((uint32_t)(32 * qd) << 16) + acc * BN + hf * HALF;
             const uint32_t piece = smem_u32(sOut + e * STAGE_PIECE);
             const int gw = p.d < HALF ? p.d : HALF;          // head-group width inside this half
@@ -380,30 +388,37 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_sh, const __grid_constant_
 
 bool proj_tc_supported(const ProjArgs& a, int dt) {
     if (dt != MOM_BF16 || a.n_tok <= 0) return false;
-    if ((a.H * a.d) % BN != 0 || a.D % BK != 0) return false;
+    if (a.plain_n > 0 ? a.plain_n % BN != 0 : (a.H * a.d) % BN != 0) return false;
+    if (a.D % BK != 0) return false;
     return device_is_sm100() && tma_available();
 }
 
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     const int Hd = a.H * a.d;
-    const bool sh = a.parts & PROJ_SHARED, rt = (a.parts & PROJ_ROUTED) && a.routed_rows() > 0;
+    const bool plain = a.plain_n > 0;
+    const bool sh = a.parts & PROJ_SHARED, rt = !plain && (a.parts & PROJ_ROUTED) && a.routed_rows() > 0;
     if (!sh && !rt) return cudaSuccess;
+    const int sh_parts = plain ? 1 : a.g ? 4 : 3, part_w = plain ? a.plain_n : Hd;
     // maps of a problem that does not run are copies of one that does (never used)
     CUtensorMap tm_sh, tm_kv;
-    if (sh && !make_tma_2d_bf16(&tm_sh, a.w_shared, (uint64_t)3 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
+    if (sh && !make_tma_2d_bf16(&tm_sh, a.w_shared, (uint64_t)sh_parts * part_w, a.D, a.D, 64, BN))
+        return cudaErrorInvalidValue;
     if (rt && !make_tma_2d_bf16(&tm_kv, a.w_kv, (uint64_t)a.M * 2 * Hd, a.D, a.D, 64, BN)) return cudaErrorInvalidValue;
     if (!sh) tm_sh = tm_kv;
     if (!rt) tm_kv = tm_sh;
     OutMaps om;
     const uint64_t nrp = (uint64_t)a.routed_rows();
-    if (sh && (!make_tma_2d_bf16(&om.q, a.q, a.n_tok, Hd, Hd, 64, 32) ||
-               !make_tma_2d_bf16(&om.k_sh, a.k_sh, a.n_tok, Hd, Hd, 64, 32) ||
-               !make_tma_2d_bf16(&om.v_sh, a.v_sh, a.n_tok, Hd, Hd, 64, 32)))
+    if (sh && !make_tma_2d_bf16(&om.q, a.q, a.n_tok, part_w, part_w, 64, 32)) return cudaErrorInvalidValue;
+    if (sh && !plain && (!make_tma_2d_bf16(&om.k_sh, a.k_sh, a.n_tok, Hd, Hd, 64, 32) ||
+                         !make_tma_2d_bf16(&om.v_sh, a.v_sh, a.n_tok, Hd, Hd, 64, 32)))
         return cudaErrorInvalidValue;
+    if (sh && a.g && !plain && !make_tma_2d_bf16(&om.g, a.g, a.n_tok, Hd, Hd, 64, 32)) return cudaErrorInvalidValue;
+    if (sh && plain) om.k_sh = om.v_sh = om.q;
     if (rt && (!make_tma_2d_bf16(&om.k_p, a.k_p, nrp, Hd, Hd, 64, 32) || !make_tma_2d_bf16(&om.v_p, a.v_p, nrp, Hd, Hd, 64, 32)))
         return cudaErrorInvalidValue;
     if (!sh) om.q = om.k_sh = om.v_sh = om.k_p;
     if (!rt) om.k_p = om.v_p = om.q;
+    if (!(sh && a.g && !plain)) om.g = om.q;
     TcParams p;
     p.x = reinterpret_cast<const bf16*>(a.x);
     p.perm = a.perm_token;
@@ -417,11 +432,15 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t st) {
     p.v_sh = reinterpret_cast<bf16*>(a.v_sh);
     p.k_p = reinterpret_cast<bf16*>(a.k_p);
     p.v_p = reinterpret_cast<bf16*>(a.v_p);
+    p.g = reinterpret_cast<bf16*>(a.g);
+    p.sh_parts = sh_parts;
+    p.part_w = part_w;
+    p.raw = a.raw || plain;
     p.n_tok = a.n_tok;
     p.n_routed = nrp;
     p.n_groups = a.groups();
     p.D = a.D; p.H = a.H; p.d = a.d; p.M = a.M; p.K = a.K;
-    p.sh_ct = 3 * Hd / BN;
+    p.sh_ct = sh_parts * part_w / BN;
     p.rt_ct = 2 * Hd / BN;
     p.sh_tiles = sh ? cdiv(a.n_tok, BM) * p.sh_ct : 0;
     p.n_tiles = p.sh_tiles + (rt ? (cdiv((int64_t)nrp, BM) + p.n_groups) * p.rt_ct : 0);

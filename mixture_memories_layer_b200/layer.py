@@ -167,6 +167,15 @@ class MoMLayer:
                               None, b["k_p"], b["v_p"], b["ws_proj"], stream=st)
         st.wait_event(gates_done)
         mark(3)
+        self._gdn_calls(b, cu_seqlens, h0_shared, h0_mem, want_states, st, side)
+        mark(4)
+        B.mom_combine_unpermute(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["out"], b["ws_comb"], stream=st)
+        mark(5)
+        return b
+
+    def _gdn_calls(self, b, cu_seqlens, h0_shared, h0_mem, want_states, st, side):
+        """The shared and routed recurrences (b: the buffers, q, k and v
+        filled); on return st waits for both."""
         hs = b["h_shared"] if want_states else None
         hm = b["h_mem"] if want_states else None
         gdn_sh = (b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens,
@@ -210,10 +219,6 @@ class MoMLayer:
         join = torch.cuda.Event()
         join.record(side)
         st.wait_event(join)
-        mark(4)
-        B.mom_combine_unpermute(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["out"], b["ws_comb"], stream=st)
-        mark(5)
-        return b
 
     def _side_stream(self):
         """Side stream: the gate projections beside the router and the

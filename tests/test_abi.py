@@ -90,3 +90,27 @@ def test_binding_refuses_host_tensors(lib):
     with pytest.raises(ValueError, match="CUDA tensors"):
         lib._p(torch.zeros(4))
     assert lib._p(None) is None
+
+
+def test_block_calls_validate_on_the_host(lib):
+    """The Gated DeltaNet block's calls refuse bad shapes before any launch."""
+    L, B = lib.lib, lib
+    fake, other = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
+    conv = lambda z, out, C, width, hd, l2, dt=B.MOM_BF16, spg=1, ng=1: L.mom_short_conv(
+        z, 10, C, fake, 2, spg, ng, fake, width, hd, l2, dt, out, fake, 4096, None)
+    assert conv(fake, other, 256, 5, 64, 1) == B.MOM_ERR_UNSUPPORTED          # width > 4
+    assert conv(fake, other, 256, 4, 64, 1, dt=B.MOM_F32) == B.MOM_ERR_UNSUPPORTED
+    assert conv(fake, other, 256, 4, 96, 1) == B.MOM_ERR_ARG                  # head_dim not a power of two
+    assert conv(fake, other, 252, 4, 64, 0) == B.MOM_ERR_ARG                  # channels % 8
+    assert conv(fake, fake, 256, 4, 64, 1) == B.MOM_ERR_ARG                   # in place
+    assert conv(fake, other, 256, 4, 64, 1, spg=0) == B.MOM_ERR_ARG           # no segments per group
+    s = L.mom_combine_norm_gate(*([fake] * 6), 1e-5, 10, 2, 2, 96, B.MOM_BF16, fake, fake, 4096, None)
+    assert s == B.MOM_ERR_ARG                                                 # d = 96
+    s = L.mom_combine_norm_gate(*([fake] * 6), -1.0, 10, 2, 2, 64, B.MOM_BF16, fake, fake, 4096, None)
+    assert s == B.MOM_ERR_ARG                                                 # eps < 0
+    s = L.mom_combine_norm_gate(*([fake] * 6), 1e-5, 10, 2, 2, 64, B.MOM_F32, fake, fake, 4096, None)
+    assert s == B.MOM_ERR_UNSUPPORTED
+    s = L.mom_linear(fake, fake, B.MOM_BF16, 10, 100, 256, fake, fake, 8, None)
+    assert s == B.MOM_ERR_ARG                                                 # workspace too small
+    s = L.mom_block_proj(*([fake] * 5), B.MOM_BF16, 10, 256, 2, 96, 4, 2, *([fake] * 6), fake, 4096, None)
+    assert s == B.MOM_ERR_UNSUPPORTED                                         # d = 96
