@@ -120,6 +120,52 @@ def layer_roofline(w, peaks, n_seq=None):
     return flops, bytes_, t
 
 
+def block_roofline(w, peaks, n_seq=None):
+    """(FLOPs, bytes, roofline seconds) of one forward of the layer inside its
+    Gated DeltaNet block: the layer's, plus the output gate's and the output
+    projection's products, the short convolutions (W taps per channel of q,
+    k, v and the routed k, v) and the gated norm; bytes: x, every weight
+    (the block's included), the output y, the final states and the routing."""
+    N, D, H, d, M, K, W = w.n_tokens, w.d_model, w.heads, w.d_head, w.n_mem, w.top_k, w.conv_width
+    S = w.batch if n_seq is None else n_seq
+    Hd = H * d
+    lf, _, _ = layer_roofline(w, peaks, n_seq)
+    flops = lf + 2 * N * D * Hd + 2 * N * Hd * D + 2 * W * (3 + 2 * K) * N * Hd + 8 * N * Hd
+    weights = (M * D + 4 * Hd * D + 2 * H * D + M * 2 * Hd * D + D * Hd) * 2 + ((3 + 2 * M) * Hd * W + d) * 4
+    bytes_ = N * D * 2 + weights + N * D * 2 + (S + M * S) * H * d * d * 4 + N * K * 8
+    t = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    return flops, bytes_, t
+
+
+def block_bench(dev, steps, warmup, peaks, flush, name="mom380m_block"):
+    """The 380M-shape layer inside its Gated DeltaNet block (short
+    convolutions, gated norm, output projection), timed like the headline
+    forward."""
+    import torch
+    from mixture_memories_layer_b200 import block as BL
+    from mixture_memories_layer_b200 import synth
+    w = synth.WORKLOADS[name]
+    p = synth.make_problem(w)
+    blk = BL.MoMBlock(BL.pack_block_weights(p, torch.bfloat16, dev), w.heads, w.d_head, w.top_k)
+    x = torch.as_tensor(p["x"]).to(dev, torch.bfloat16)
+    cu = torch.as_tensor(p["cu_seqlens"]).to(dev)
+    for _ in range(warmup):
+        blk.forward(x, cu)
+    torch.cuda.synchronize()
+    errs = blk.device_errors()
+    if errs:
+        raise SystemExit("device error records in %s: %s" % (name, errs))
+    step_ms, per_call = time_forward(blk, x, cu, steps, flush)
+    ms = sum(step_ms) / steps
+    S = int(cu.numel()) - 1
+    bf, bb, bt = block_roofline(w, peaks, n_seq=S)
+    return {"workload": workload_desc(w) + "; inside its Gated DeltaNet block (short convolutions of width %d, "
+                                          "gated RMS norm, output projection)" % w.conv_width,
+            "tokens": w.n_tokens, "sequences": S, "ms_per_step": ms, "value": w.n_tokens / (ms / 1e3), "unit": UNIT,
+            "per_call_ms": per_call,
+            "block_roofline": {"flops": bf, "bytes": bb, "roofline_ms": bt * 1e3, "frac": bt * 1e3 / ms}}
+
+
 def kernel_source_sha(name):
     path = os.path.join(ROOT, "mixture_memories_layer_b200", "csrc", name)
     if not os.path.exists(path):
@@ -270,8 +316,8 @@ def time_forward(lay, x, cu, steps, flush):
     """`steps` layer forwards, L2 flushed before each outside its events.
     Returns (per-step ms list, mean ms per call of MoMLayer.STEPS)."""
     import torch
-    from mixture_memories_layer_b200 import layer as L
-    n_calls = len(L.MoMLayer.STEPS)
+    names = type(lay).STEPS
+    n_calls = len(names)
     marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_calls + 1)] for _ in range(steps)]
     torch.cuda.synchronize()
     for s in range(steps):
@@ -280,7 +326,7 @@ def time_forward(lay, x, cu, steps, flush):
     torch.cuda.synchronize()
     step_ms = [marks[s][0].elapsed_time(marks[s][n_calls]) for s in range(steps)]
     per_call = {name: sum(marks[s][i].elapsed_time(marks[s][i + 1]) for s in range(steps)) / steps
-                for i, name in enumerate(L.MoMLayer.STEPS)}
+                for i, name in enumerate(names)}
     return step_ms, per_call
 
 
@@ -406,6 +452,7 @@ def gpu_arm(args):
     if not args.no_configs and world == 1:
         configs = {extra_key(name, rule, mg): config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule, mg)
                    for name, rule, mg in EXTRA}
+        configs["block"] = block_bench(dev, args.steps, args.warmup, peaks, flush)
         configs["recurrence_backward"] = backward_bench(lay, w, x, cu, flush)
         configs["layer_backward"] = layer_backward_bench(lay, w, x, cu, flush)
     clocks.__exit__(None, None, None)

@@ -47,6 +47,8 @@ def pack_block_weights(p: Dict[str, np.ndarray], dtype: torch.dtype, device="cud
 class MoMBlock(MoMLayer):
     """The layer with its block: forward(x, cu_seqlens)["y"] [N, d_model]."""
 
+    STEPS = ("router", "permute", "proj_conv", "gdn", "combine_norm", "o_proj")
+
     def __init__(self, weights: Dict[str, torch.Tensor], heads: int, d_head: int, top_k: int, scale: float = 1.0,
                  gdn_schedule: str = "streams", rule: str = "gated_delta", eps: float = RMS_EPS):
         super().__init__(weights, heads, d_head, top_k, scale, gdn_schedule, rule)

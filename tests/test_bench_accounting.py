@@ -109,3 +109,17 @@ def test_load_peaks_measured_partial_and_fallback(tmp_path, monkeypatch):
     assert p["source"].startswith("measured (hbm_gbs)")
     (tmp_path / "MEASURED_PEAKS.json").write_text("not json")
     assert bench.load_peaks()["source"] == "fallback"
+
+
+def test_380m_block_roofline():
+    """The block adds the output gate's and the output projection's products
+    (2 N D Hd each), the convolutions (2 W (3 + 2k) N Hd) and the gated norm
+    (8 N Hd) to the layer; its bytes replace the layer's output [N, Hd] by y
+    [N, D] and add W_g, W_o and the filters."""
+    w = synth.WORKLOADS["mom380m_block"]
+    flops, bytes_, t = bench.block_roofline(w, PEAKS)
+    N, D, Hd = 16384, 1024, 1024
+    assert _close(flops, 318.3e9 + 4 * N * D * Hd + 2 * 4 * 7 * N * Hd + 8 * N * Hd, 1e-3)
+    assert _close(flops, 388.1e9, 1e-3)
+    assert _close(bytes_, 136.8e6, 2e-3)
+    assert _close(t, 388.1e9 / 1631.7e12, 1e-3)        # tensor-bound
