@@ -461,23 +461,31 @@ def gpu_arm(args):
                   configs)
 
 
+SETS = 2          # e2e buffer sets
+E2E_STEPS = 64    # e2e steps at least
+
+
 def e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks):
     """The same metric through the user-facing calls with host buffers:
     every step uploads its tokens from pinned host memory, runs the layer
     and reads its output back to pinned host memory.  Steps are pipelined
-    the way a serving loop streams batches: two buffer sets (two layer
-    objects over the same weights), the upload of step i+1 and the download
-    of step i-1 on their own streams beside step i's compute.  No L2 flush:
-    a step touches ~0.6 GB, several times L2."""
+    the way a serving loop streams batches: SETS buffer sets (layer objects
+    over the same weights), the upload of a later step and the download of
+    an earlier one on their own streams beside a step's compute, so that the
+    PCIe link (both directions at once) is the bound.  At least E2E_STEPS
+    steps, so the pipeline's fill and drain (one upload, one download) are
+    a small part of the timed region.  No L2 flush: a step touches ~0.6 GB,
+    several times L2."""
     import torch
     from mixture_memories_layer_b200 import layer as L
-    n = max(3, args.steps)
-    lays = [lay, L.MoMLayer(lay.w, w.heads, w.d_head, w.top_k)]
-    xs = [x, torch.empty_like(x)]
+    n = max(E2E_STEPS, args.steps)
+    lays = [lay] + [L.MoMLayer(lay.w, w.heads, w.d_head, w.top_k) for _ in range(SETS - 1)]
+    xs = [x] + [torch.empty_like(x) for _ in range(SETS - 1)]
     x_host = torch.empty(x.shape, dtype=dt, pin_memory=True)
     x_host.copy_(x.cpu())
-    outs_host = [torch.empty((w.n_tokens, w.heads, w.d_head), dtype=dt, pin_memory=True) for _ in range(2)]
-    lays[1].forward(xs[0], cu)                 # the second buffer set, warm
+    outs_host = [torch.empty((w.n_tokens, w.heads, w.d_head), dtype=dt, pin_memory=True) for _ in range(SETS)]
+    for j in range(1, SETS):
+        lays[j].forward(xs[0], cu)             # the other buffer sets, warm
     torch.cuda.synchronize()
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(n)]
@@ -486,15 +494,15 @@ def e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(h2d)
     for i in range(n):
-        j = i % 2
-        if i >= 2:
-            h2d.wait_event(ev_fwd[i - 2])      # forward i-2 has read xs[j]
+        j = i % SETS
+        if i >= SETS:
+            h2d.wait_event(ev_fwd[i - SETS])   # the forward SETS steps back has read xs[j]
         with torch.cuda.stream(h2d):
             xs[j].copy_(x_host, non_blocking=True)
         ev_in[i].record(h2d)
         stream.wait_event(ev_in[i])
-        if i >= 2:
-            stream.wait_event(ev_out[i - 2])   # output i-2 has left lays[j]'s buffer
+        if i >= SETS:
+            stream.wait_event(ev_out[i - SETS])   # that step's output has left lays[j]'s buffer
         b = lays[j].forward(xs[j], cu, stream=stream)
         ev_fwd[i].record(stream)
         d2h.wait_event(ev_fwd[i])
@@ -508,8 +516,8 @@ def e2e_bench(args, w, lay, x, cu, flush, stream, dt, world, max_over_ranks):
     return {"value": w.n_tokens * world * n / (e2e_ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": x.numel() * x.element_size(),
             "d2h_bytes_per_step": outs_host[0].numel() * outs_host[0].element_size(),
-            "steps": n, "pipelined": "upload of step i+1 and download of step i-1 beside step i's compute "
-                                      "(two buffer sets, three streams); no L2 flush (each step touches ~0.6 GB)"}
+            "steps": n, "pipelined": "uploads of later steps and downloads of earlier ones beside each step's compute "
+                                      "(%d buffer sets, three streams); no L2 flush (each step touches ~0.6 GB)" % SETS}
 
 
 def finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,
