@@ -32,9 +32,11 @@ Gated DeltaNet block, each choice a reading listed in the design notes:
 The gates beta, log alpha, the router and the recurrences are those of
 mom_oracle.  Parity pins: tests/test_oracle_block.py (numpy's convolution,
 torch's RMS norm and SiLU, causality and segment locality of the
-convolution, the routed-subsequence convolution, and the reduction of the
+convolution, the routed-subsequence convolution, the reduction of the
 block to mom_oracle.mom_forward when the convolution is the identity and
-the activation is dropped).
+the activation is dropped, and the decode step continuing a prefill: the
+forward over T tokens, its states and windows, then block_decode_step,
+equals the forward over T + 1 tokens).
 """
 from __future__ import annotations
 
@@ -156,3 +158,90 @@ def block_forward(x, p, cu_seqlens, top_k: int, H: int, d: int, scale: float = 1
     return dict(y=y, o_tilde=o_tilde, out=out, g=g, q=q, k_sh=k_sh, v_sh=v_sh, k_mem=k_mem, v_mem=v_mem,
                 o_shared=o_shared, o_mem=o_mem, idx=idx, gate=gate, logits=logits, near_tie=near_tie,
                 h_shared=h_shared, h_mem=h_mem, beta=beta, log_alpha=log_alpha)
+
+
+def conv_window_step(window, z, w, act):
+    """One row of the causal convolution from the W-1 rows before it:
+    window [W-1, C] (oldest first; zeros before the segment's start), z [C]
+    the current row, w [C, W].  Returns (act(out) [C], the next window)."""
+    rows = np.concatenate([np.asarray(window, F64), np.asarray(z, F64)[None]], axis=0)   # [W, C], oldest first
+    out = np.einsum("wc,cw->c", rows, np.asarray(w, F64))
+    return act(out), rows[1:]
+
+
+def block_decode_step(x, p, state, conv_sh, conv_mem, top_k: int, H: int, d: int, scale: float = 1.0,
+                      forced_idx=None, rule: str = "gated_delta", act=silu):
+    """One new token per sequence through the block.  x [B, d_model]; state
+    [B, M+1, H, d, d] (slot M = the shared memory), conv_sh [B, 3, W-1, Hd]
+    (the raw q, k_sh, v_sh of the sequence's last W-1 tokens, oldest first,
+    zero before its start) and conv_mem [B, M, 2, W-1, Hd] (the raw k, v of
+    the last W-1 tokens routed to each memory); none is modified.  Each
+    sequence updates only its k routed memories' states and windows and the
+    shared ones.  Returns (y [B, d_model], new state, new conv_sh, new
+    conv_mem, idx)."""
+    x = np.asarray(x, F64)
+    Bn = x.shape[0]
+    M = np.shape(p["w_r"])[0]
+    lin = lambda a, w_: a @ np.asarray(w_, F64).T
+    idx, gate, logits, _ = orc.router_topk(x, p["w_r"], p.get("b_r"), top_k)
+    if forced_idx is not None:
+        idx = np.asarray(forced_idx, np.int32)
+        gate = orc.gates_for(logits, idx)
+    _, _, _, beta, log_alpha = orc.shared_projections(x, p, H, d)
+    raw_sh = [lin(x, p["w_q"]), lin(x, p["w_k_sh"]), lin(x, p["w_v_sh"])]
+    filt_sh = [p["conv_q"], p["conv_k_sh"], p["conv_v_sh"]]
+    g = lin(x, p["w_g"]).reshape(Bn, H, d)
+    new = np.array(state, F64, copy=True)
+    csh = np.array(conv_sh, F64, copy=True)
+    cmem = np.array(conv_mem, F64, copy=True)
+    out = np.zeros((Bn, H, d), F64)
+    for b in range(Bn):
+        qkv = []
+        for i in range(3):
+            c, csh[b, i] = conv_window_step(csh[b, i], raw_sh[i][b], filt_sh[i], act)
+            qkv.append(c.reshape(H, d))
+        q, k_sh, v_sh = orc.l2norm(qkv[0]), orc.l2norm(qkv[1]), qkv[2]
+        out[b], new[b, M] = orc.RULES[rule](new[b, M], q, k_sh, v_sh, beta[b], log_alpha[b], scale)
+        for j in range(top_k):
+            m = int(idx[b, j])
+            ck, cmem[b, m, 0] = conv_window_step(cmem[b, m, 0], lin(x[b], p["w_k"][m]), p["conv_k"][m], act)
+            cv, cmem[b, m, 1] = conv_window_step(cmem[b, m, 1], lin(x[b], p["w_v"][m]), p["conv_v"][m], act)
+            if orc.has_memory_gates(p):
+                b_m, la_m = orc.memory_gates(x[b:b + 1], p, m)
+                b_m, la_m = b_m[0], la_m[0]
+            else:
+                b_m, la_m = beta[b], log_alpha[b]
+            o_m, new[b, m] = orc.RULES[rule](new[b, m], q, orc.l2norm(ck.reshape(H, d)), cv.reshape(H, d), b_m, la_m,
+                                             scale)
+            out[b] += gate[b, j] * o_m
+    y = lin(rms_norm_gated(out, p["w_norm"], g).reshape(Bn, H * d), p["w_o"])
+    return y, new, csh, cmem, idx
+
+
+def block_conv_state(x, p, cu_seqlens, idx, W: int):
+    """The convolution windows after a block forward over whole sequences:
+    conv_sh [S, 3, W-1, Hd] (raw q, k_sh, v_sh of each sequence's last W-1
+    tokens, oldest first, zero before its start) and conv_mem [S, M, 2, W-1,
+    Hd] (raw k, v of the last W-1 tokens of each sequence routed to each
+    memory).  idx [N, k] the routing the forward used."""
+    x = np.asarray(x, F64)
+    cu = np.asarray(cu_seqlens, np.int64)
+    S = len(cu) - 1
+    M = np.shape(p["w_r"])[0]
+    Hd = np.shape(p["w_q"])[0]
+    lin = lambda a, w_: a @ np.asarray(w_, F64).T
+    csh = np.zeros((S, 3, W - 1, Hd), F64)
+    cmem = np.zeros((S, M, 2, W - 1, Hd), F64)
+    for s in range(S):
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        last = np.arange(max(t0, t1 - (W - 1)), t1)
+        for i, name in enumerate(("w_q", "w_k_sh", "w_v_sh")):
+            if len(last):
+                csh[s, i, W - 1 - len(last):] = lin(x[last], p[name])
+        for m in range(M):
+            rows = t0 + np.nonzero((idx[t0:t1] == m).any(axis=1))[0]
+            rows = rows[max(0, len(rows) - (W - 1)):]
+            if len(rows):
+                cmem[s, m, 0, W - 1 - len(rows):] = lin(x[rows], p["w_k"][m])
+                cmem[s, m, 1, W - 1 - len(rows):] = lin(x[rows], p["w_v"][m])
+    return csh, cmem

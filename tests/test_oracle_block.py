@@ -15,6 +15,9 @@ print none of it).
   gated norm of its output (pure-Python dot products).
 * Planted mistakes in the convolution (a flipped filter, a window crossing
   the segment start) and in the norm (the mean over all heads) fail their pins.
+* Decode (constant-cost inference through the block): the one-row window
+  step reproduces the convolution, and a decode step after a prefill equals
+  the forward over one more token.
 """
 import numpy as np
 import pytest
@@ -163,3 +166,40 @@ def test_planted_mistakes_fail_their_pins():
     ref = (ref * torch.nn.functional.silu(torch.from_numpy(g))).numpy()
     assert np.abs(whole - ref).max() > 1e-3
     assert np.abs(blk.rms_norm_gated(o, w, g) - ref).max() < 1e-12
+
+
+def test_block_decode_continues_a_prefill():
+    """Constant-cost inference through the block: the forward over T tokens,
+    its final states and convolution windows, then one decode step per
+    sequence, equals the forward over T + 1 tokens (the last token's y, every
+    final state) -- the decode's window arithmetic is written apart from the
+    forward's convolution."""
+    w, p, _, _ = _block_problem(seed=7, cu=(0, 2))
+    rng = np.random.default_rng(70)
+    lens = (9, 1, 6)
+    H, d, K = w.heads, w.d_head, w.top_k
+    xs = [synth.make_tokens(w, rng, n + 1) for n in lens]
+    pre = [blk.block_forward(xi[:-1], p, np.array([0, len(xi) - 1]), K, H, d) for xi in xs]
+    full = [blk.block_forward(xi, p, np.array([0, len(xi)]), K, H, d) for xi in xs]
+    state = np.stack([orc.decode_state_from_prefill(r["h_shared"], r["h_mem"])[0] for r in pre])
+    conv = [blk.block_conv_state(xi[:-1], p, np.array([0, len(xi) - 1]), r["idx"], 4) for xi, r in zip(xs, pre)]
+    conv_sh = np.stack([c[0][0] for c in conv])
+    conv_mem = np.stack([c[1][0] for c in conv])
+    x_new = np.stack([xi[-1] for xi in xs])
+    forced = np.stack([f["idx"][-1] for f in full])
+    y, new, _, _, _ = blk.block_decode_step(x_new, p, state, conv_sh, conv_mem, K, H, d, forced_idx=forced)
+    for b, f in enumerate(full):
+        np.testing.assert_allclose(y[b], f["y"][-1], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(new[b, w.n_mem], f["h_shared"][0], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(new[b, :w.n_mem], f["h_mem"][:, 0], rtol=1e-10, atol=1e-12)
+
+
+def test_conv_window_step_is_the_convolution():
+    """The decode's one-row window step, run row by row from a zero window,
+    reproduces the forward's convolution (numpy-pinned above)."""
+    z, w, _ = _conv_case(seed=8)
+    win = np.zeros((w.shape[1] - 1, z.shape[1]))
+    ref = blk.short_conv(z, w, [(0, len(z))])
+    for t in range(len(z)):
+        out, win = blk.conv_window_step(win, z[t], w, blk.identity)
+        np.testing.assert_allclose(out, ref[t], rtol=0, atol=1e-13)
