@@ -620,7 +620,8 @@ mom_status mom_short_conv_batch(const mom_conv_problem* problems, int n_problems
  *   out[t] = o / sqrt(mean(o^2) + eps) * w_norm * SiLU(g[t]).
  * o_sh, g, out [n_tok, H*d], o_p [n_tok*top_k, H*d] bf16; w_norm [d]
  * float32; d a power of two in 8..256; every array 16-byte aligned.  Row
- * errors as in the combine. */
+ * errors as in the combine.  top_k = 0: o = o_sh (o_p, row_of and
+ * topk_gate unused): the norm and gate of an output combined elsewhere. */
 mom_status mom_combine_norm_gate(const void* o_sh, const void* o_p, const int32_t* row_of,
                                  const float* topk_gate, const void* g, const float* w_norm, float eps,
                                  int64_t n_tok, int top_k, int H, int d, mom_dtype dt, void* out,
@@ -632,6 +633,58 @@ mom_status mom_combine_norm_gate(const void* o_sh, const void* o_p, const int32_
  * ws: MOM_WS_HEADER_BYTES. */
 mom_status mom_linear(const void* x, const void* w, mom_dtype dt, int64_t n_rows, int k_in, int n_out, void* y,
                       void* ws, size_t ws_bytes, void* stream);
+
+/* The block's weights for its decode step (device pointers). */
+typedef struct mom_block_weights {
+    const void*  w_shared4;   /* [4*H*d, d_model]: W_q | W_k_sh | W_v_sh | W_g */
+    const void*  w_o;         /* [d_model, H*d] */
+    const float* conv_q;      /* [width, H*d] tap-major (tap width-1: the current row) */
+    const float* conv_k_sh;   /* [width, H*d] */
+    const float* conv_v_sh;   /* [width, H*d] */
+    const float* conv_k;      /* [n_mem, width, H*d] */
+    const float* conv_v;      /* [n_mem, width, H*d] */
+    const float* w_norm;      /* [d] */
+} mom_block_weights;
+
+/* mom_block_decode_step -- one new token per sequence through the block
+ * (constant-cost inference: the blog post's introduction, "推理效率"; the
+ * paper card, Summary): router, reordering and gates as mom_decode_step; the
+ * block's raw projections and output gate; one row of each short
+ * convolution from the sequence's window (the shared q, k, v) or from the
+ * (sequence, memory) window of each routed memory (its k, v); the k+1
+ * recurrence steps and the combine; the gated per-head RMS norm (eps); W_o.
+ *   state     [B, n_mem+1, H, d, d] float32, as mom_decode_step, in place;
+ *   conv_sh   [B, 3, width-1, H*d] (dt): the raw q, k_sh, v_sh of each
+ *             sequence's last width-1 tokens, oldest first, zero before its
+ *             start; updated in place;
+ *   conv_mem  [B, n_mem, 2, width-1, H*d] (dt): the raw k, v of the last
+ *             width-1 tokens of each sequence routed to each memory; the
+ *             windows of the memories a token is not routed to are kept;
+ *   y         [B, d_model] (dt); topk_idx [B, top_k] or NULL; mg as in
+ *             mom_decode_step_rule (a HOST pointer) or NULL.
+ * bf16 only, width 2..4 (MOM_ERR_UNSUPPORTED otherwise); H*d a multiple of
+ * 256, d_model of 256; ws: mom_block_decode_workspace_size(). */
+size_t mom_block_decode_workspace_size(int B, int d_model, int H, int d, int n_mem, int top_k);
+mom_status mom_block_decode_step(const void* x, const mom_weights* w, const mom_block_weights* bw,
+                                 const mom_memory_gates* mg, int width, float eps, int B, int d_model, int H, int d,
+                                 int n_mem, int top_k, float scale, mom_dtype dt, mom_rule rule, float* state,
+                                 void* conv_sh, void* conv_mem, void* y, int32_t* topk_idx, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* mom_block_conv_state -- the convolution windows a block forward over
+ * whole sequences leaves, for mom_block_decode_step: conv_sh[s, i, j] = raw
+ * row cu_seqlens[s+1] - (width-1) + j of q, k_sh, v_sh (i = 0, 1, 2), zero
+ * when it falls before the sequence's start; conv_mem[s, m, i, j] the same
+ * over memory m's segment seg_cu[m*n_seq + s] .. of k_p, v_p (i = 0, 1).
+ * q_raw, k_sh_raw, v_sh_raw [n_tok, channels], k_p_raw, v_p_raw
+ * [n_tok*top_k, channels] (dt): the forward's unnormalised projections
+ * (mom_block_proj); cu_seqlens [n_seq+1], seg_cu [n_mem*n_seq+1] device
+ * int32 (corrupt bounds are recorded in ws and give zero windows).  bf16
+ * only, width 2..4. */
+mom_status mom_block_conv_state(const void* q_raw, const void* k_sh_raw, const void* v_sh_raw, const void* k_p_raw,
+                                const void* v_p_raw, int64_t n_tok, int top_k, const int32_t* cu_seqlens,
+                                const int32_t* seg_cu, int n_seq, int n_mem, int channels, int width, mom_dtype dt,
+                                void* conv_sh, void* conv_mem, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -80,6 +80,11 @@ SIGNATURES = {
     "mom_short_conv_batch": (_I, [_VP, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "mom_combine_norm_gate": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _F, _I64, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
     "mom_linear": (_I, [_VP, _VP, _I, _I64, _I, _I, _VP, _VP, _SZ, _VP]),
+    "mom_block_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "mom_block_decode_step": (_I, [_VP, _VP, _VP, _VP, _I, _F, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP, _VP,
+                                   _VP, _VP, _SZ, _VP]),
+    "mom_block_conv_state": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _I, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ,
+                                  _VP]),
 }
 
 
@@ -93,6 +98,12 @@ class MomConvProblem(ctypes.Structure):
     """Mirror of ``struct mom_conv_problem``."""
     _fields_ = [("z", c_void_p), ("out", c_void_p), ("n_rows", c_int64), ("seg_cu", c_void_p), ("n_seg", c_int),
                 ("seg_per_group", c_int), ("n_groups", c_int), ("w", c_void_p), ("l2norm", c_int)]
+
+
+class MomBlockWeights(ctypes.Structure):
+    """Mirror of ``struct mom_block_weights`` (device pointers)."""
+    _fields_ = [("w_shared4", c_void_p), ("w_o", c_void_p), ("conv_q", c_void_p), ("conv_k_sh", c_void_p),
+                ("conv_v_sh", c_void_p), ("conv_k", c_void_p), ("conv_v", c_void_p), ("w_norm", c_void_p)]
 
 
 class MomMemoryGates(ctypes.Structure):
@@ -466,6 +477,33 @@ def mom_linear(x, w, y, ws, stream=None):
     n, k_in = x.shape
     _check(lib.mom_linear(_p(x), _p(w), dtype_code(x.dtype), n, k_in, w.shape[0], _p(y), _p(ws), ws.numel(),
                           _s(stream)), "mom_linear")
+
+
+def mom_block_decode_workspace_size(B, d_model, H, d, n_mem, top_k):
+    return lib.mom_block_decode_workspace_size(B, d_model, H, d, n_mem, top_k)
+
+
+def mom_block_decode_step(x, weights, block_weights, width, eps, H, d, n_mem, top_k, scale, rule, state, conv_sh,
+                          conv_mem, y, topk_idx, ws, stream=None, mem_gates=None):
+    """One token per sequence through the block; state, conv_sh, conv_mem
+    updated in place.  weights / block_weights / mem_gates: MomWeights,
+    MomBlockWeights, MomMemoryGates (or None)."""
+    B, d_model = x.shape
+    _check(lib.mom_block_decode_step(_p(x), ctypes.byref(weights), ctypes.byref(block_weights),
+                                     None if mem_gates is None else ctypes.byref(mem_gates), width, eps, B, d_model, H,
+                                     d, n_mem, top_k, scale, dtype_code(x.dtype), rule, _p(state), _p(conv_sh),
+                                     _p(conv_mem), _p(y), _p(topk_idx), _p(ws), ws.numel(), _s(stream)),
+           "mom_block_decode_step")
+
+
+def mom_block_conv_state(q_raw, k_sh_raw, v_sh_raw, k_p_raw, v_p_raw, cu_seqlens, seg_cu, n_mem, top_k, width,
+                         conv_sh, conv_mem, ws, stream=None):
+    n_tok = q_raw.shape[0]
+    C = q_raw.numel() // max(n_tok, 1)
+    _check(lib.mom_block_conv_state(_p(q_raw), _p(k_sh_raw), _p(v_sh_raw), _p(k_p_raw), _p(v_p_raw), n_tok, top_k,
+                                    _p(cu_seqlens), _p(seg_cu), cu_seqlens.numel() - 1, n_mem, C, width,
+                                    dtype_code(q_raw.dtype), _p(conv_sh), _p(conv_mem), _p(ws), ws.numel(),
+                                    _s(stream)), "mom_block_conv_state")
 
 
 def mom_decode_workspace_size(B, d_model, H, d, n_mem, top_k):

@@ -123,8 +123,49 @@ class MoMBlock(MoMLayer):
         mark(6)
         return b
 
-    def decode_step(self, *a, **k):
-        raise NotImplementedError("the block's decode (convolution states per sequence and memory) is not provided")
+    # ------------------------------------------------------------ decode
+    @property
+    def width(self) -> int:
+        return self.w["conv_q"].shape[1]
+
+    def _c_block(self):
+        cb = getattr(self, "_cb", None)
+        if cb is None:
+            from .layer import ctypes_ptr
+            cb = self._cb = B.MomBlockWeights(*[ctypes_ptr(self.w[k]) for k in
+                                                ("w_shared4", "w_o", "conv_q", "conv_k_sh", "conv_v_sh", "conv_k",
+                                                 "conv_v", "w_norm")])
+        return cb
+
+    def new_conv_state(self, n_seq: int):
+        """Zero windows: conv_sh [S, 3, W-1, H, d], conv_mem [S, M, 2, W-1, H, d]."""
+        Wm = self.width - 1
+        z = lambda *shape: torch.zeros(shape, dtype=self.dtype, device=self.device)
+        return z(n_seq, 3, Wm, self.H, self.d), z(n_seq, self.n_mem, 2, Wm, self.H, self.d)
+
+    def conv_state(self, b, cu_seqlens, stream=None):
+        """The windows the forward that returned buffers ``b`` leaves (for
+        decode_step): (conv_sh, conv_mem)."""
+        n_seq = cu_seqlens.numel() - 1
+        conv_sh, conv_mem = self.new_conv_state(n_seq)
+        B.mom_block_conv_state(b["q_raw"], b["k_sh_raw"], b["v_sh_raw"], b["k_p_raw"], b["v_p_raw"], cu_seqlens,
+                               b["seg_cu"], self.n_mem, self.top_k, self.width, conv_sh, conv_mem, b["ws_conv"],
+                               stream=stream)
+        return conv_sh, conv_mem
+
+    def decode_step(self, x: torch.Tensor, state: torch.Tensor, conv_sh: torch.Tensor, conv_mem: torch.Tensor,
+                    stream=None):
+        """x [B, d_model]; state [B, M+1, H, d, d] float32 and the windows,
+        all updated in place.  Returns (y [B, d_model], topk_idx [B, k])."""
+        Bn = x.shape[0]
+        y = self._buf("bdec_y", (Bn, self.d_model), self.dtype)
+        idx = self._buf("bdec_idx", (Bn, self.top_k), torch.int32)
+        ws = self._ws("bdecode", B.mom_block_decode_workspace_size(Bn, self.d_model, self.H, self.d, self.n_mem,
+                                                                   self.top_k))
+        B.mom_block_decode_step(x, self._c_weights, self._c_block(), self.width, self.eps, self.H, self.d, self.n_mem,
+                                self.top_k, self.scale, self.rule, state, conv_sh, conv_mem, y, idx, ws,
+                                stream=stream, mem_gates=self._c_mem_gates)
+        return y, idx
 
     def backward(self, *a, **k):
         raise NotImplementedError("the block's backward is not provided (MoMLayer.backward is the layer's)")

@@ -486,15 +486,16 @@ mom_status mom_combine_norm_gate(const void* o_sh, const void* o_p, const int32_
                                  const float* topk_gate, const void* g, const float* w_norm, float eps,
                                  int64_t n_tok, int top_k, int H, int d, mom_dtype dt, void* out,
                                  void* ws, size_t ws_bytes, void* stream) {
-    if (!dt_ok(dt) || n_tok < 0 || top_k < 1 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (!dt_ok(dt) || n_tok < 0 || top_k < 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
     if (d < 8 || d > 256 || (d & (d - 1)) != 0 || !(eps >= 0.f)) return MOM_ERR_ARG;
     if (dt != MOM_BF16) return MOM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
     if (n_tok == 0) return MOM_OK;
-    const void* ptrs[] = {o_sh, o_p, row_of, topk_gate, g, w_norm, out};
+    const void* ptrs[] = {o_sh, g, w_norm, out};
     for (const void* p : ptrs)
         if (!p) return MOM_ERR_ARG;
-    if (!al16(o_sh) || !al16(o_p) || !al16(g) || !al16(out) || !al16(w_norm)) return MOM_ERR_ARG;
+    if (top_k > 0 && (!o_p || !row_of || !topk_gate || !al16(o_p))) return MOM_ERR_ARG;
+    if (!al16(o_sh) || !al16(g) || !al16(out) || !al16(w_norm)) return MOM_ERR_ARG;
     return cuda_status(launch_combine_norm_gate(o_sh, o_p, row_of, topk_gate, g, w_norm, eps, n_tok, top_k, H, d,
                                                 out, ws, as_stream(stream)));
 }
@@ -626,6 +627,154 @@ mom_status mom_decode_step_rule(const void* x, const mom_weights* w, const mom_m
         da.log_alpha_p = la_p;
     }
     return cuda_status(launch_decode_state(da, dt, st));
+}
+
+// ------------------------------------------------------------ block decode
+namespace {
+struct BlockDecodeLayout {
+    DecodeLayout base;
+    size_t q_raw, k_sh_raw, v_sh_raw, g, k_p_raw, v_p_raw, comb, o_tilde, total;
+};
+BlockDecodeLayout block_decode_layout(int B, int H, int d, int M, int K) {
+    BlockDecodeLayout L;
+    L.base = decode_layout(B, H, d, M, K, MOM_F32);
+    size_t off = L.base.total;
+    auto take = [&](size_t bytes) { size_t o = off; off += up256(bytes); return o; };
+    const size_t row = (size_t)H * d * 2, BK = (size_t)B * K;
+    L.q_raw = take(B * row);
+    L.k_sh_raw = take(B * row);
+    L.v_sh_raw = take(B * row);
+    L.g = take(B * row);
+    L.k_p_raw = take(BK * row);
+    L.v_p_raw = take(BK * row);
+    L.comb = take(B * row);
+    L.o_tilde = take(B * row);
+    L.total = off;
+    return L;
+}
+}  // namespace
+
+size_t mom_block_decode_workspace_size(int B, int d_model, int H, int d, int n_mem, int top_k) {
+    (void)d_model;
+    if (B < 0 || H < 1 || d < 1 || n_mem < 1 || top_k < 1) return 0;
+    return block_decode_layout(B, H, d, n_mem, top_k).total;
+}
+
+mom_status mom_block_decode_step(const void* x, const mom_weights* w, const mom_block_weights* bw,
+                                 const mom_memory_gates* mg, int width, float eps, int B, int d_model, int H, int d,
+                                 int n_mem, int top_k, float scale, mom_dtype dt, mom_rule rule, float* state,
+                                 void* conv_sh, void* conv_mem, void* y, int32_t* topk_idx, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || B < 0 || d_model <= 0 || d_model % 64 != 0 || H < 1 || H > MOM_MAX_HEADS) return MOM_ERR_ARG;
+    if (rule != MOM_RULE_GATED_DELTA && rule != MOM_RULE_GATED_LINEAR) return MOM_ERR_ARG;
+    if (top_k < 1 || n_mem < top_k || n_mem > MOM_MAX_MEM || !w || !bw || !(eps >= 0.f)) return MOM_ERR_ARG;
+    if (width < 2 || width > 4 || dt != MOM_BF16 || !head_dim_ok(d)) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < mom_block_decode_workspace_size(B, d_model, H, d, n_mem, top_k)) return MOM_ERR_ARG;
+    if (B == 0) return MOM_OK;
+    const void* ptrs[] = {x, w->w_r, w->w_gate, w->A, w->b_a, w->w_kv, bw->w_shared4, bw->w_o, bw->conv_q,
+                          bw->conv_k_sh, bw->conv_v_sh, bw->conv_k, bw->conv_v, bw->w_norm, state, conv_sh,
+                          conv_mem, y};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    if (mg && (!mg->w_gate_mem || !al16(mg->w_gate_mem) || !mg->A_mem || !mg->b_a_mem)) return MOM_ERR_ARG;
+    const int Hd = H * d;
+    cudaStream_t st = as_stream(stream);
+    const BlockDecodeLayout BL = block_decode_layout(B, H, d, n_mem, top_k);
+    const DecodeLayout& L = BL.base;
+    char* base = reinterpret_cast<char*>(ws);
+    int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(base + L.idx);
+    float* gate = reinterpret_cast<float*>(base + L.gate);
+    int32_t* perm = reinterpret_cast<int32_t*>(base + L.perm);
+    int32_t* row_of = reinterpret_cast<int32_t*>(base + L.row_of);
+    int32_t* mem_off = reinterpret_cast<int32_t*>(base + L.mem_off);
+    int32_t* seg_cu = reinterpret_cast<int32_t*>(base + L.seg_cu);
+    float* beta = reinterpret_cast<float*>(base + L.beta);
+    float* la = reinterpret_cast<float*>(base + L.la);
+
+    cudaError_t e = launch_router(x, w->w_r, w->b_r, dt, B, d_model, n_mem, top_k, idx, gate, nullptr, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    e = launch_permute(idx, B, top_k, n_mem, nullptr, 1, perm, row_of, mem_off, seg_cu, ws, base + L.perm_scratch, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    e = launch_gate_proj(x, w->w_gate, w->A, w->b_a, dt, B, d_model, H, beta, la, ws, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    // the raw projections and the output gate
+    ProjArgs pa{x, perm, mem_off, bw->w_shared4, w->w_kv, B, d_model, H, d, n_mem, top_k,
+                base + BL.q_raw, base + BL.k_sh_raw, base + BL.v_sh_raw, base + BL.k_p_raw, base + BL.v_p_raw, ws};
+    pa.raw = 1;
+    pa.g = base + BL.g;
+    if (!proj_tc_supported(pa, dt)) return MOM_ERR_UNSUPPORTED;
+    e = launch_proj_tc(pa, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    // one row of every convolution, the windows shifted
+    ConvStepArgs ca;
+    const char* raws[5] = {base + BL.q_raw, base + BL.k_sh_raw, base + BL.v_sh_raw, base + BL.k_p_raw,
+                           base + BL.v_p_raw};
+    char* outs[5] = {base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p};
+    const float* filts[5] = {bw->conv_q, bw->conv_k_sh, bw->conv_v_sh, bw->conv_k, bw->conv_v};
+    for (int i = 0; i < 5; ++i) {
+        ca.z[i] = reinterpret_cast<const bf16*>(raws[i]);
+        ca.out[i] = reinterpret_cast<bf16*>(outs[i]);
+        ca.w[i] = filts[i];
+    }
+    ca.st_sh = reinterpret_cast<bf16*>(conv_sh);
+    ca.st_mem = reinterpret_cast<bf16*>(conv_mem);
+    ca.perm = perm;
+    ca.mem_offset = mem_off;
+    ca.B = B; ca.K = top_k; ca.M = n_mem; ca.C = Hd; ca.d = d;
+    ca.err = ws;
+    e = launch_conv_step(ca, width, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    // the recurrences' step and the combine
+    DecodeArgs da{base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, beta, la, gate,
+                  idx, row_of, B, H, d, n_mem, top_k, scale, state, base + BL.comb, ws};
+    da.rule = rule;
+    if (mg) {
+        float* beta_p = reinterpret_cast<float*>(base + L.beta_p);
+        float* la_p = reinterpret_cast<float*>(base + L.la_p);
+        e = launch_mem_gate_proj(x, perm, mem_off, mg->w_gate_mem, mg->A_mem, mg->b_a_mem, dt, B, (int64_t)B * top_k,
+                                 d_model, H, n_mem, beta_p, la_p, ws, st);
+        if (e != cudaSuccess) return MOM_ERR_CUDA;
+        da.beta_p = beta_p;
+        da.log_alpha_p = la_p;
+    }
+    e = launch_decode_state(da, dt, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    // the gated norm, then W_o
+    e = launch_combine_norm_gate(base + BL.comb, nullptr, nullptr, nullptr, base + BL.g, bw->w_norm, eps, B, 0, H, d,
+                                 base + BL.o_tilde, ws, st);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    ProjArgs lo{base + BL.o_tilde, nullptr, nullptr, bw->w_o, nullptr, B, Hd, 1, d_model, 1, 1,
+                y, nullptr, nullptr, nullptr, nullptr, ws};
+    lo.parts = PROJ_SHARED;
+    lo.plain_n = d_model;
+    if (!proj_tc_supported(lo, dt)) return MOM_ERR_UNSUPPORTED;
+    return cuda_status(launch_proj_tc(lo, st));
+}
+
+mom_status mom_block_conv_state(const void* q_raw, const void* k_sh_raw, const void* v_sh_raw, const void* k_p_raw,
+                                const void* v_p_raw, int64_t n_tok, int top_k, const int32_t* cu_seqlens,
+                                const int32_t* seg_cu, int n_seq, int n_mem, int channels, int width, mom_dtype dt,
+                                void* conv_sh, void* conv_mem, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || top_k < 1 || n_seq < 1 || n_mem < 1 || n_mem > MOM_MAX_MEM) return MOM_ERR_ARG;
+    if (channels < 8 || channels % 8 != 0) return MOM_ERR_ARG;
+    if (width < 2 || width > 4 || dt != MOM_BF16) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    const void* ptrs[] = {q_raw, k_sh_raw, v_sh_raw, k_p_raw, v_p_raw, conv_sh, conv_mem};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    if (!cu_seqlens || !seg_cu) return MOM_ERR_ARG;
+    ConvStateArgs a;
+    const void* raws[5] = {q_raw, k_sh_raw, v_sh_raw, k_p_raw, v_p_raw};
+    for (int i = 0; i < 5; ++i) a.z[i] = reinterpret_cast<const bf16*>(raws[i]);
+    a.st_sh = reinterpret_cast<bf16*>(conv_sh);
+    a.st_mem = reinterpret_cast<bf16*>(conv_mem);
+    a.cu = cu_seqlens;
+    a.seg_cu = seg_cu;
+    a.S = n_seq; a.M = n_mem; a.C = channels; a.W = width;
+    a.n_tok = n_tok;
+    a.n_rows = n_tok * top_k;
+    a.err = ws;
+    return cuda_status(launch_conv_state(a, as_stream(stream)));
 }
 
 }  // extern "C"

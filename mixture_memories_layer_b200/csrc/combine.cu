@@ -108,6 +108,8 @@ combine_kernel(const T* __restrict__ o_sh, const T* __restrict__ o_p, const int3
 // channels of token t, with o the combined output above,
 //   out = o / sqrt(mean(o^2) + eps) * w_norm * SiLU(g[t])
 // A head is d/8 consecutive lanes of one 256-column piece (d divides 256).
+// With K = 0 (o_p, row_of and gate unused) o is o_sh: the norm and gate of
+// an output combined elsewhere (the decode step's).
 template <int KMAX, int CH>
 __global__ void __launch_bounds__(256, 2)
 combine_norm_gate_kernel(const bf16* __restrict__ o_sh, const bf16* __restrict__ o_p,
@@ -168,6 +170,12 @@ combine_norm_gate_kernel(const bf16* __restrict__ o_sh, const bf16* __restrict__
                     }
                 }
                 first = false;
+            }
+            if (first) {                                  // top_k = 0: o = o_sh
+#pragma unroll
+                for (int q = 0; q < CH; ++q)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[q][e] = sh[q].at(e);
             }
 #pragma unroll
             for (int q = 0; q < CH; ++q) {

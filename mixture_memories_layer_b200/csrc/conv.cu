@@ -255,4 +255,172 @@ cudaError_t launch_short_conv(const ConvProblem* problems, int n, int C, int W, 
     return cudaErrorInvalidValue;
 }
 
+
+// ---------------------------------------------------------------- decode --
+// One new row per sequence: each convolution reads its window of the W-1 raw
+// rows before (bf16, oldest first, zero before the sequence's -- or for a
+// memory, its routed tokens' -- start), writes act(conv) (+ the L2 norm)
+// and shifts the new raw row into the window.  The shared q, k, v windows
+// are per sequence; memory m's k, v windows per (sequence, memory), found
+// through the routed row's token (perm) and its memory (the mem_offset range
+// holding the row).  A sequence routes each memory at most once, so no two
+// warps touch one window.
+namespace {
+
+template <int W>
+__global__ void __launch_bounds__(256) conv_step_kernel(const __grid_constant__ ConvStepArgs a) {
+    static_assert(W >= 2, "a window needs at least one row");
+    const int lane = threadIdx.x & 31;
+    const int nblk = (a.C + 255) / 256;
+    const int64_t n_sh = 3LL * a.B * nblk, n_rt = 2LL * a.B * a.K * nblk;
+    const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t it = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); it < n_sh + n_rt; it += nw) {
+        int pi, l2, m = 0;
+        int64_t row, b;
+        const float* filt;
+        bf16* win;
+        int blk;
+        if (it < n_sh) {
+            pi = (int)(it / ((int64_t)a.B * nblk));
+            const int64_t rem = it % ((int64_t)a.B * nblk);
+            row = rem / nblk;
+            blk = (int)(rem % nblk);
+            b = row;
+            win = a.st_sh + ((b * 3 + pi) * (W - 1)) * (int64_t)a.C;
+            filt = a.w[pi];
+            l2 = pi < 2;
+        } else {
+            const int64_t it2 = it - n_sh;
+            const int64_t per = (int64_t)a.B * a.K * nblk;
+            pi = 3 + (int)(it2 / per);
+            const int64_t rem = it2 % per;
+            row = rem / nblk;
+            blk = (int)(rem % nblk);
+            b = __ldg(a.perm + row);
+            const int32_t v = lane <= a.M ? __ldg(a.mem_offset + lane) : 0x7fffffff;
+            m = __popc(__ballot_sync(0xffffffffu, v <= row)) - 1;
+            if (b < 0 || b >= a.B || m < 0 || m >= a.M) {
+                if (lane == 0) record_error(a.err, MOM_DEVERR_ROW_INDEX, row);
+                continue;                                 // uniform over the warp
+            }
+            win = a.st_mem + (((b * a.M + m) * 2 + (pi - 3)) * (W - 1)) * (int64_t)a.C;
+            filt = a.w[pi] + (int64_t)m * W * a.C;
+            l2 = pi == 3;
+        }
+        const int c = blk * 256 + 8 * lane;
+        const bool on = c < a.C;
+        uint4 z = make_uint4(0u, 0u, 0u, 0u), wr[W - 1];
+        float wv[8][W];
+        if (on) {
+            z = __ldg(reinterpret_cast<const uint4*>(a.z[pi] + row * a.C + c));
+#pragma unroll
+            for (int t = 0; t < W - 1; ++t) wr[t] = *reinterpret_cast<const uint4*>(win + (int64_t)t * a.C + c);
+            load_filters<W>(filt, a.C, 0, c, wv);
+        } else {
+#pragma unroll
+            for (int t = 0; t < W - 1; ++t) wr[t] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+#pragma unroll
+                for (int t = 0; t < W; ++t) wv[e][t] = 0.f;
+        }
+        float acc[8], ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float s = wv[e][W - 1] * bf_at(z, e);
+#pragma unroll
+            for (int t = 0; t < W - 1; ++t) s = fmaf(wv[e][t], bf_at(wr[t], e), s);
+            acc[e] = silu_tanh(s);
+            ss = fmaf(acc[e], acc[e], ss);
+        }
+        if (l2) {                                         // uniform over the warp
+            for (int o = a.d >> 4; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float sc = rsqrtf(ss + 1e-6f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] *= sc;
+        }
+        if (on) {
+            store_vec<8>(a.out[pi] + row * a.C + c, acc);
+#pragma unroll
+            for (int t = 0; t < W - 2; ++t) *reinterpret_cast<uint4*>(win + (int64_t)t * a.C + c) = wr[t + 1];
+            *reinterpret_cast<uint4*>(win + (int64_t)(W - 2) * a.C + c) = z;
+        }
+    }
+}
+
+// The windows a forward leaves: the raw rows of each sequence's (and each
+// (memory, sequence) segment's) last W-1 rows, zero where the segment is
+// shorter.
+__global__ void __launch_bounds__(256) conv_state_kernel(const __grid_constant__ ConvStateArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int nblk = (a.C + 255) / 256;
+    const int Wm = a.W - 1;
+    const int64_t n_sh = 3LL * a.S * Wm * nblk, n_rt = 2LL * a.M * a.S * Wm * nblk;
+    const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t it = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); it < n_sh + n_rt; it += nw) {
+        const bool sh = it < n_sh;
+        int64_t r = sh ? it : it - n_sh;
+        const int blk = (int)(r % nblk);
+        r /= nblk;
+        const int j = (int)(r % Wm);
+        r /= Wm;
+        const int pi = (int)(r % (sh ? 3 : 2));
+        r /= sh ? 3 : 2;
+        int64_t lo, hi, lim;
+        bf16* dst;
+        const bf16* src;
+        if (sh) {
+            const int s = (int)r;
+            lo = a.cu[s];
+            hi = a.cu[s + 1];
+            lim = a.n_tok;
+            dst = a.st_sh + (((int64_t)s * 3 + pi) * Wm + j) * a.C;
+            src = a.z[pi];
+        } else {
+            const int s = (int)(r % a.S), m = (int)(r / a.S);
+            lo = a.seg_cu[m * a.S + s];
+            hi = a.seg_cu[m * a.S + s + 1];
+            lim = a.n_rows;
+            dst = a.st_mem + ((((int64_t)s * a.M + m) * 2 + pi) * Wm + j) * a.C;
+            src = a.z[3 + pi];
+        }
+        const bool bad = lo < 0 || hi < lo || hi > lim;
+        if (bad && lane == 0 && blk == 0 && j == 0) record_error(a.err, MOM_DEVERR_SEGMENT, it);
+        const int64_t row = hi - Wm + j;
+        const int c = blk * 256 + 8 * lane;
+        if (c < a.C) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (!bad && row >= lo) v = __ldg(reinterpret_cast<const uint4*>(src + row * a.C + c));
+            *reinterpret_cast<uint4*>(dst + c) = v;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_conv_step(const ConvStepArgs& a, int W, cudaStream_t st) {
+    const int64_t items = (3LL * a.B + 2LL * a.B * a.K) * ((a.C + 255) / 256);
+    if (items == 0) return cudaSuccess;
+    int64_t grid = cdiv(items, 8);
+    if (grid > 148 * 8) grid = 148 * 8;
+    switch (W) {
+        case 2: conv_step_kernel<2><<<(unsigned)grid, 256, 0, st>>>(a); break;
+        case 3: conv_step_kernel<3><<<(unsigned)grid, 256, 0, st>>>(a); break;
+        case 4: conv_step_kernel<4><<<(unsigned)grid, 256, 0, st>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_conv_state(const ConvStateArgs& a, cudaStream_t st) {
+    const int64_t items = (3LL * a.S + 2LL * a.M * a.S) * (a.W - 1) * ((a.C + 255) / 256);
+    if (items == 0) return cudaSuccess;
+    int64_t grid = cdiv(items, 8);
+    if (grid > 148 * 8) grid = 148 * 8;
+    conv_state_kernel<<<(unsigned)grid, 256, 0, st>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 }  // namespace mom

@@ -223,6 +223,31 @@ struct ConvProblem {
     int l2;
 };
 cudaError_t launch_short_conv(const ConvProblem* problems, int n, int C, int W, int d, void* err, cudaStream_t st);
+// one decode row per sequence through the five convolutions, windows updated in place
+struct ConvStepArgs {
+    const bf16* z[5];             // raw rows: q, k_sh, v_sh [B, C]; k_p, v_p [B*K, C]
+    bf16* out[5];
+    const float* w[5];            // tap-major filters: [W, C] (shared), [M, W, C] (memories)
+    bf16* st_sh;                  // [B][3][W-1][C]
+    bf16* st_mem;                 // [B][M][2][W-1][C]
+    const int32_t* perm;          // routed row -> sequence
+    const int32_t* mem_offset;    // [M + 1]
+    int B, K, M, C, d;
+    void* err;
+};
+cudaError_t launch_conv_step(const ConvStepArgs& a, int W, cudaStream_t st);
+// the windows a forward leaves
+struct ConvStateArgs {
+    const bf16* z[5];             // raw forward rows: q, k_sh, v_sh [n_tok, C]; k_p, v_p [n_rows, C]
+    bf16* st_sh;
+    bf16* st_mem;
+    const int32_t* cu;            // [S + 1]
+    const int32_t* seg_cu;        // [M * S + 1]
+    int S, M, C, W;
+    int64_t n_tok, n_rows;
+    void* err;
+};
+cudaError_t launch_conv_state(const ConvStateArgs& a, cudaStream_t st);
 // combine.cu: the combine with the block's gated per-head RMS norm
 cudaError_t launch_combine_norm_gate(const void* o_sh, const void* o_p, const int32_t* row_of, const float* gate,
                                      const void* g, const float* w_norm, float eps, int64_t n_tok, int K, int H,

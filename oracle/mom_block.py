@@ -178,7 +178,8 @@ def block_decode_step(x, p, state, conv_sh, conv_mem, top_k: int, H: int, d: int
     the last W-1 tokens routed to each memory); none is modified.  Each
     sequence updates only its k routed memories' states and windows and the
     shared ones.  Returns (y [B, d_model], new state, new conv_sh, new
-    conv_mem, idx)."""
+    conv_mem, idx, parts) with parts = {"out": the combined output [B, H, d]
+    before the gated norm, "g": the output gate's pre-activation}."""
     x = np.asarray(x, F64)
     Bn = x.shape[0]
     M = np.shape(p["w_r"])[0]
@@ -215,7 +216,7 @@ def block_decode_step(x, p, state, conv_sh, conv_mem, top_k: int, H: int, d: int
                                              scale)
             out[b] += gate[b, j] * o_m
     y = lin(rms_norm_gated(out, p["w_norm"], g).reshape(Bn, H * d), p["w_o"])
-    return y, new, csh, cmem, idx
+    return y, new, csh, cmem, idx, {"out": out, "g": g}
 
 
 def block_conv_state(x, p, cu_seqlens, idx, W: int):

@@ -187,7 +187,7 @@ def test_block_decode_continues_a_prefill():
     conv_mem = np.stack([c[1][0] for c in conv])
     x_new = np.stack([xi[-1] for xi in xs])
     forced = np.stack([f["idx"][-1] for f in full])
-    y, new, _, _, _ = blk.block_decode_step(x_new, p, state, conv_sh, conv_mem, K, H, d, forced_idx=forced)
+    y, new, _, _, _, _ = blk.block_decode_step(x_new, p, state, conv_sh, conv_mem, K, H, d, forced_idx=forced)
     for b, f in enumerate(full):
         np.testing.assert_allclose(y[b], f["y"][-1], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(new[b, w.n_mem], f["h_shared"][0], rtol=1e-10, atol=1e-12)
