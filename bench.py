@@ -453,6 +453,7 @@ def gpu_arm(args):
         configs = {extra_key(name, rule, mg): config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule, mg)
                    for name, rule, mg in EXTRA}
         configs["block"] = block_bench(dev, args.steps, args.warmup, peaks, flush)
+        configs["block_decode"] = block_decode_bench(dev, args.warmup)
         configs["recurrence_backward"] = backward_bench(lay, w, x, cu, flush)
         configs["layer_backward"] = layer_backward_bench(lay, w, x, cu, flush)
     clocks.__exit__(None, None, None)
@@ -661,6 +662,48 @@ def decode_bench(args, dev, world, rank, max_over_ranks, barrier):
             "state_bytes_per_step": state_bytes,
             "state_gbs": state_bytes / (per_step / 1e3) / 1e9,
             "frac_hbm": state_bytes / (per_step / 1e3) / 1e9 / hbm}
+
+
+def block_decode_bench(dev, warmup, steps=128):
+    """Decode through the Gated DeltaNet block: the decode workload's shape
+    (256 sequences, 8 memories top-2 + shared) with the block, after a
+    prefill through MoMBlock.forward and the windows it leaves."""
+    import dataclasses
+
+    import torch
+    from mixture_memories_layer_b200 import block as BL
+    from mixture_memories_layer_b200 import synth
+    w = dataclasses.replace(synth.WORKLOADS[DEC], block=True)
+    p = synth.make_decode_problem(w, steps=steps + warmup)
+    blk = BL.MoMBlock(BL.pack_block_weights(p, torch.bfloat16, dev), w.heads, w.d_head, w.top_k)
+    cu = torch.as_tensor(p["cu_prefill"]).to(dev)
+    b = blk.forward(torch.as_tensor(p["x_prefill"]).to(dev, torch.bfloat16), cu)
+    conv0 = blk.conv_state(b, cu)
+    state0 = torch.empty((w.batch, w.n_mem + 1, w.heads, w.d_head, w.d_head), dtype=torch.float32, device=dev)
+    state0[:, :w.n_mem] = b["h_mem"].permute(1, 0, 2, 3, 4)
+    state0[:, w.n_mem] = b["h_shared"]
+    xs = torch.as_tensor(p["x_steps"]).to(dev, torch.bfloat16)
+    state, conv_sh, conv_mem = state0.clone(), conv0[0].clone(), conv0[1].clone()
+    for s in range(warmup):
+        blk.decode_step(xs[steps + s], state, conv_sh, conv_mem)
+    state.copy_(state0)
+    conv_sh.copy_(conv0[0])
+    conv_mem.copy_(conv0[1])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(steps):
+        blk.decode_step(xs[s], state, conv_sh, conv_mem)
+    e1.record()
+    torch.cuda.synchronize()
+    errs = blk.device_errors()
+    if errs:
+        raise SystemExit("device error records in the block decode: %s" % errs)
+    ms = e0.elapsed_time(e1)
+    return {"workload": "decode through the Gated DeltaNet block: B=%d sequences, d_model=%d, H=%d, d=%d, M=%d top-%d "
+                        "+ shared, %d steps after a %d-token prefill" % (w.batch, w.d_model, w.heads, w.d_head,
+                                                                         w.n_mem, w.top_k, steps, w.prefill_len),
+            "value": w.batch * steps / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms / steps}
 
 
 # --------------------------------------------------------- CPU oracle timing
