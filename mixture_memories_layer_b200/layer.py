@@ -273,8 +273,9 @@ class MoMLayer:
         qn, kshn, kpn = g("qn", (n_tok, H)), g("kshn", (n_tok, H)), g("kpn", (R, H))
         B.mom_proj_shared(x, w["w_shared"], H, d, g("q2", (n_tok, H, d), dt), g("k2", (n_tok, H, d), dt),
                           g("v2", (n_tok, H, d), dt), ws, stream=st, q_norm=qn, k_sh_norm=kshn)
-        mem_index = self._buf("mem_index", (M,), torch.int32)
-        mem_index.copy_(torch.arange(M, dtype=torch.int32, device=dev))
+        mem_index = getattr(self, "_mem_index", None)       # group g = memory g (set up once)
+        if mem_index is None:
+            mem_index = self._mem_index = torch.arange(M, dtype=torch.int32, device=dev)
         B.mom_kv_proj_groups(x, b["perm"], b["mem_offset"], mem_index, w["w_kv"], H, d, g("kp2", (R, H, d), dt),
                              g("vp2", (R, H, d), dt), ws, stream=st, k_norm=kpn)
         # combine and router
