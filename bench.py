@@ -32,6 +32,10 @@ import statistics
 import sys
 import time
 
+# NCCL writes its version / debug lines to stdout when NCCL_DEBUG asks for
+# them; the result line must be the only line on stdout, so they go to stderr
+os.environ.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -835,8 +839,10 @@ def memory_parallel_arm(args):
                    "data": "synthetic: seeded, same generator as the data-parallel arm",
                    "config": {"workload": workload_desc(w), "tokens_per_gpu": w.n_tokens,
                               "global_tokens": w.n_tokens * world,
-                              "parallelism": "mp%d (memories sharded, routed rows to their owners and back by "
-                                             "NCCL all-to-all)" % world,
+                              "parallelism": ("mp%d (memories sharded, routed rows to their owners and back by "
+                                              "NCCL all-to-all)" % world) if world > 1 else
+                                             "mp1 (every memory on the one rank: the row exchanges are the "
+                                             "identity; the metadata still goes through the process group)",
                               "l2": "flushed before every timed step (256 MiB write, untimed)"},
                    "layer_roofline": {"flops": lf, "bytes": lb, "roofline_ms": lt * 1e3,
                                       "frac": lt * 1e3 / (total_ms / args.steps)},

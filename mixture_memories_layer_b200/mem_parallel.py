@@ -387,9 +387,16 @@ class MemoryParallelMoM:
         own = self.part.hi(self.rank) - self.part.lo(self.rank)
         seg_from = self.comm.exchange_ints(st.seg_out, [own * n_seq_of[r] for r in range(G)])
         tables = receive_tables(seg_from, n_seq_of, self.part, self.rank)
-        recv = torch.empty((tables.n_rows, st.send.shape[1]), dtype=torch.uint8, device=dev)
-        self.comm.all_to_all(recv, st.send, tables.rows, st.send_rows)
+        if G == 1:
+            # one rank owns every memory: both exchanges are the identity
+            recv = st.send
+        else:
+            recv = torch.empty((tables.n_rows, st.send.shape[1]), dtype=torch.uint8, device=dev)
+            self.comm.all_to_all(recv, st.send, tables.rows, st.send_rows)
         o_r, h_r = self.owner_phase(recv, tables, x.dtype, stream)
-        o_back = torch.empty((st.send.shape[0], self.H, self.d), dtype=x.dtype, device=dev)
-        self.comm.all_to_all(o_back, o_r, st.send_rows, tables.rows)
+        if G == 1:
+            o_back = o_r
+        else:
+            o_back = torch.empty((st.send.shape[0], self.H, self.d), dtype=x.dtype, device=dev)
+            self.comm.all_to_all(o_back, o_r, st.send_rows, tables.rows)
         return self.finish_phase(st, o_back, stream), st.h_shared, h_r, tables
