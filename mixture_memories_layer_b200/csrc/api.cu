@@ -3,6 +3,9 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
+
+#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -32,6 +35,78 @@ inline size_t esize(int dt) { return dt == MOM_BF16 ? 2 : 4; }
 inline bool dt_ok(int dt) { return dt == MOM_F32 || dt == MOM_BF16; }
 inline bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
 inline mom_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOM_OK : MOM_ERR_CUDA; }
+
+// A side stream of the library for work inside one call that does not
+// depend on the rest of it (the decode step's gate projection beside its
+// router and reordering): forked from the caller's stream by an event and
+// joined back by another before anything reads its results, so the call as
+// a whole stays ordered on the caller's stream.  One per (device, context):
+// a stream belongs to the context it was made in.
+struct Side {
+    CUcontext ctx = nullptr;
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kSideDevices = 64;
+std::mutex g_side_mutex;
+Side g_side[kSideDevices];
+
+PFN_cuCtxGetCurrent_v4000 current_ctx_fn() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+    });
+    return fn;
+}
+
+// The side stream of the current device and context (created on first use),
+// or nullptr when none can be had: the caller then runs everything on its
+// own stream.
+const Side* side_stream() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSideDevices) return nullptr;
+    auto get_ctx = current_ctx_fn();
+    CUcontext ctx = nullptr;
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
+    std::lock_guard<std::mutex> lock(g_side_mutex);
+    Side& sd = g_side[dev];
+    if (sd.s != nullptr && sd.ctx == ctx) return &sd;
+    Side fresh;
+    fresh.ctx = ctx;
+    if (cudaStreamCreateWithFlags(&fresh.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&fresh.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&fresh.join, cudaEventDisableTiming) != cudaSuccess) {
+        cudaStreamDestroy(fresh.s);
+        return nullptr;
+    }
+    sd = fresh;        // a stream of a context no longer current is left to that context
+    return &sd;
+}
+
+// The side stream forked from `st` (work queued there starts after what is
+// already queued on `st`), or `st` itself when there is none.  Every fork is
+// closed by join_side(st, side) before anything on `st` reads the side's
+// results.
+cudaStream_t fork_side(cudaStream_t st) {
+    const Side* sd = side_stream();
+    if (sd == nullptr) return st;
+    if (cudaEventRecord(sd->fork, st) != cudaSuccess || cudaStreamWaitEvent(sd->s, sd->fork, 0) != cudaSuccess)
+        return st;
+    return sd->s;
+}
+
+cudaError_t join_side(cudaStream_t st, cudaStream_t side) {
+    if (side == st) return cudaSuccess;
+    const Side* sd = side_stream();
+    if (sd == nullptr || sd->s != side) return cudaErrorInvalidValue;
+    cudaError_t e = cudaEventRecord(sd->join, side);
+    return e == cudaSuccess ? cudaStreamWaitEvent(st, sd->join, 0) : e;
+}
 
 }  // namespace
 
@@ -603,15 +678,18 @@ mom_status mom_decode_step_rule(const void* x, const mom_weights* w, const mom_m
     float* beta = reinterpret_cast<float*>(base + L.beta);
     float* la = reinterpret_cast<float*>(base + L.la);
 
-    cudaError_t e = launch_router(x, w->w_r, w->b_r, dt, B, d_model, n_mem, top_k, idx, gate, nullptr, st);
+    // the gates need no routing: on the side stream beside the router and the reordering
+    const cudaStream_t ss = fork_side(st);
+    cudaError_t e = launch_gate_proj(x, w->w_gate, w->A, w->b_a, dt, B, d_model, H, beta, la, ws, ss);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    e = launch_router(x, w->w_r, w->b_r, dt, B, d_model, n_mem, top_k, idx, gate, nullptr, st);
     if (e != cudaSuccess) return MOM_ERR_CUDA;
     e = launch_permute(idx, B, top_k, n_mem, nullptr, 1, perm, row_of, mem_off, seg_cu, ws,
                        base + L.perm_scratch, st);
     if (e != cudaSuccess) return MOM_ERR_CUDA;
+    if (join_side(st, ss) != cudaSuccess) return MOM_ERR_CUDA;
     ProjArgs pa{x, perm, mem_off, w->w_shared, w->w_kv, B, d_model, H, d, n_mem, top_k,
                 base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, ws};
-    e = launch_gate_proj(x, w->w_gate, w->A, w->b_a, dt, B, d_model, H, beta, la, ws, st);
-    if (e != cudaSuccess) return MOM_ERR_CUDA;
     e = proj_tc_supported(pa, dt) ? launch_proj_tc(pa, st) : launch_proj_simt(pa, dt, st);
     if (e != cudaSuccess) return MOM_ERR_CUDA;
     DecodeArgs da{base + L.q, base + L.k_sh, base + L.v_sh, base + L.k_p, base + L.v_p, beta, la, gate,
@@ -691,12 +769,14 @@ mom_status mom_block_decode_step(const void* x, const mom_weights* w, const mom_
     float* beta = reinterpret_cast<float*>(base + L.beta);
     float* la = reinterpret_cast<float*>(base + L.la);
 
-    cudaError_t e = launch_router(x, w->w_r, w->b_r, dt, B, d_model, n_mem, top_k, idx, gate, nullptr, st);
+    const cudaStream_t ss = fork_side(st);
+    cudaError_t e = launch_gate_proj(x, w->w_gate, w->A, w->b_a, dt, B, d_model, H, beta, la, ws, ss);
+    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    e = launch_router(x, w->w_r, w->b_r, dt, B, d_model, n_mem, top_k, idx, gate, nullptr, st);
     if (e != cudaSuccess) return MOM_ERR_CUDA;
     e = launch_permute(idx, B, top_k, n_mem, nullptr, 1, perm, row_of, mem_off, seg_cu, ws, base + L.perm_scratch, st);
     if (e != cudaSuccess) return MOM_ERR_CUDA;
-    e = launch_gate_proj(x, w->w_gate, w->A, w->b_a, dt, B, d_model, H, beta, la, ws, st);
-    if (e != cudaSuccess) return MOM_ERR_CUDA;
+    if (join_side(st, ss) != cudaSuccess) return MOM_ERR_CUDA;
     // the raw projections and the output gate
     ProjArgs pa{x, perm, mem_off, bw->w_shared4, w->w_kv, B, d_model, H, d, n_mem, top_k,
                 base + BL.q_raw, base + BL.k_sh_raw, base + BL.v_sh_raw, base + BL.k_p_raw, base + BL.v_p_raw, ws};
