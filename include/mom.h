@@ -473,7 +473,9 @@ mom_status mom_col_sums(const float* a, int64_t rows, int64_t lda, int64_t cols,
  *     group_index[g] * c_group_stride, [M, N] (the weight gradient dZ^T X).
  * group_index NULL: g.  total_rows: group_offset[n_groups] (trans_a = 0).
  * accumulate: 0 overwrite, 1 add.  A bad row index is recorded in ws and
- * reads as zero. */
+ * reads as zero.  With B in bf16 the products run on the tensor cores in
+ * tf32 (B exact, A rounded to a 10-bit mantissa, fp32 accumulation); with B
+ * in float32, on CUDA cores in fp32. */
 mom_status mom_gemm_grouped(int trans_a, const float* A, int64_t lda, const void* B, int64_t ldb, mom_dtype dt,
                             const int32_t* b_rows, int64_t n_b_rows, float* C, int64_t ldc, int64_t M, int64_t N,
                             int64_t K, int64_t total_rows, const int32_t* group_offset, const int32_t* group_index,

@@ -281,6 +281,167 @@ gemm_grouped_kernel(GemmArgs g) {
     }
 }
 
+// The same products on the tensor cores when B is bf16: tf32 operands (B
+// exactly, A rounded to a 10-bit mantissa), fp32 accumulation, m16n8k8
+// MMAs.  Tiles of 128 x 128 over k steps of 16 held in padded shared memory
+// (stride 136 floats: the fragment reads of a warp hit 32 banks), the next
+// step's operands loaded into registers while the current one is multiplied;
+// 8 warps, each a 64 x 32 piece (4 x 4 MMAs per k8 step).
+constexpr int TBK = 16, TPAD = GBM + 8, TVAL = TBK * GBM / 256;   // values per thread per operand and step
+constexpr int TPR = GBM / TVAL;                                      // threads per k row of an operand tile
+static_assert(TBK / TVAL == 2, "two threads per row of a row-major A tile");
+constexpr size_t TF32_SMEM = 2ull * 2 * TBK * TPAD * 4;
+
+__device__ __forceinline__ uint32_t tf32_bits(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__global__ void __launch_bounds__(256, 2)
+gemm_grouped_tf32_kernel(GemmArgs g) {
+    extern __shared__ __align__(16) uint32_t tf32_smem[];
+    auto As = reinterpret_cast<uint32_t (*)[TBK][TPAD]>(tf32_smem);
+    auto Bs = reinterpret_cast<uint32_t (*)[TBK][TPAD]>(tf32_smem + 2 * TBK * TPAD);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bf16* B = reinterpret_cast<const bf16*>(g.B);
+    const int64_t n0 = (int64_t)blockIdx.x * GBN;
+    int64_t m0 = 0, m1 = 0, k0 = 0, k1 = 0;
+    const bf16* Bg = B;
+    float* Cg = g.C;
+    if (!g.trans_a) {
+        int64_t t = blockIdx.y;
+        int grp = -1;
+        for (int q = 0; q < g.n_groups; ++q) {
+            const int64_t lo = g.goff[q], hi = g.goff[q + 1];
+            if (lo < 0 || hi < lo) { if (tid == 0 && blockIdx.x == 0) record_error(g.err, MOM_DEVERR_SEGMENT, q); return; }
+            const int64_t nt = (hi - lo + GBM - 1) / GBM;
+            if (t < nt) { grp = q; m0 = lo + t * GBM; m1 = m0 + GBM < hi ? m0 + GBM : hi; break; }
+            t -= nt;
+        }
+        if (grp < 0) return;
+        const int64_t w = g.gmem ? g.gmem[grp] : grp;
+        Bg = B + w * g.b_group_stride;
+        k0 = 0;
+        k1 = g.K;
+    } else {
+        const int grp = blockIdx.z / g.splits, sp = blockIdx.z % g.splits;
+        m0 = (int64_t)blockIdx.y * GBM;
+        m1 = m0 + GBM < g.M ? m0 + GBM : g.M;
+        if (m0 >= g.M) return;
+        const int64_t lo = g.goff[grp], hi = g.goff[grp + 1];
+        if (lo < 0 || hi < lo) { if (tid == 0 && blockIdx.x == 0) record_error(g.err, MOM_DEVERR_SEGMENT, grp); return; }
+        const int64_t steps = (hi - lo + TBK - 1) / TBK, per = (steps + g.splits - 1) / g.splits;
+        k0 = lo + sp * per * TBK;
+        k1 = k0 + per * TBK < hi ? k0 + per * TBK : hi;
+        if (k0 >= k1) return;
+        const int64_t w = g.gmem ? g.gmem[grp] : grp;
+        Cg = g.C + w * g.c_group_stride;
+    }
+    // loader: TVAL A and B values per thread per k step.  A: row m = tid / 2,
+    // k = (tid % 2) TVAL + e (trans_a = 0) or k = tid / TPR, m = (tid % TPR)
+    // TVAL + e (trans_a = 1); B: k = tid / TPR, n = (tid % TPR) TVAL + e
+    float ra[TVAL], rb[TVAL];
+    auto load = [&](int64_t kb) {
+#pragma unroll
+        for (int e = 0; e < TVAL; ++e) {
+            int kk, mm;
+            if (!g.trans_a) { mm = tid >> 1; kk = (tid & 1) * TVAL + e; } else { kk = tid / TPR; mm = (tid % TPR) * TVAL + e; }
+            const int64_t m = m0 + mm, k = kb + kk;
+            ra[e] = (m < m1 && k < k1) ? (g.trans_a ? g.A[k * g.lda + m] : g.A[m * g.lda + k]) : 0.f;
+        }
+        const int kk = tid / TPR;
+        const int64_t k = kb + kk;
+        int64_t br = k;
+        if (k < k1 && g.trans_a && g.b_rows) {
+            br = g.b_rows[k];
+            if (br < 0 || br >= g.n_b_rows) { record_error(g.err, MOM_DEVERR_ROW_INDEX, k); br = -1; }
+        }
+#pragma unroll
+        for (int e = 0; e < TVAL; ++e) {
+            const int64_t n = n0 + (tid % TPR) * TVAL + e;
+            rb[e] = (k < k1 && br >= 0 && n < g.N) ? __bfloat162float(Bg[br * g.ldb + n]) : 0.f;
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int e = 0; e < TVAL; ++e) {
+            if (!g.trans_a) As[buf][(tid & 1) * TVAL + e][tid >> 1] = tf32_bits(ra[e]);
+            else As[buf][tid / TPR][(tid % TPR) * TVAL + e] = tf32_bits(ra[e]);
+            Bs[buf][tid / TPR][(tid % TPR) * TVAL + e] = tf32_bits(rb[e]);
+        }
+    };
+    const int wm = warp >> 2, wn = warp & 3;          // 2 x 4 warps of 64 x 32
+    const int gr = lane >> 2, gc = lane & 3;
+    float acc[4][4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+    int buf = 0;
+    if (k0 < k1) {
+        load(k0);
+        store(0);
+    }
+    __syncthreads();
+    for (int64_t kb = k0; kb < k1; kb += TBK) {
+        const bool more = kb + TBK < k1;
+        if (more) load(kb + TBK);
+#pragma unroll
+        for (int ks = 0; ks < TBK; ks += 8) {
+            uint32_t af[4][4], bfr[4][2];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int mb = wm * 64 + 16 * i + gr;
+                af[i][0] = As[buf][ks + gc][mb];
+                af[i][1] = As[buf][ks + gc][mb + 8];
+                af[i][2] = As[buf][ks + gc + 4][mb];
+                af[i][3] = As[buf][ks + gc + 4][mb + 8];
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int nb = wn * 32 + 8 * j + gr;
+                bfr[j][0] = Bs[buf][ks + gc][nb];
+                bfr[j][1] = Bs[buf][ks + gc + 4][nb];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) mma_16x8x8_tf32(acc[i][j], af[i], bfr[j]);
+        }
+        if (more) store(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t m = m0 + wm * 64 + 16 * i + gr + 8 * h;
+            if (m >= m1) continue;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int64_t n = n0 + wn * 32 + 8 * j + 2 * gc + e;
+                    if (n >= g.N) continue;
+                    const float v = acc[i][j][2 * h + e];
+                    float* c = Cg + m * g.ldc + n;
+                    if (g.trans_a) atomicAdd(c, v);
+                    else *c = g.accumulate ? *c + v : v;
+                }
+        }
+}
+
 // C_g = 0 for every group (the reduction form's partial sums are added into it)
 __global__ void __launch_bounds__(256)
 zero_groups_kernel(float* C, int64_t ldc, int64_t M, int64_t N, const int32_t* gmem, int64_t c_group_stride) {
@@ -380,8 +541,14 @@ cudaError_t launch_gemm_grouped(int trans_a, const float* A, int64_t lda, const 
             count_launches(1);
         }
     }
-    if (dt == MOM_BF16) gemm_grouped_kernel<bf16><<<grid, 256, 0, st>>>(g);
-    else gemm_grouped_kernel<float><<<grid, 256, 0, st>>>(g);
+    if (dt == MOM_BF16) {
+        static unsigned long long optin_done = 0;
+        cudaError_t e = smem_optin((const void*)gemm_grouped_tf32_kernel, (int)TF32_SMEM, &optin_done);
+        if (e != cudaSuccess) return e;
+        gemm_grouped_tf32_kernel<<<grid, 256, TF32_SMEM, st>>>(g);
+    } else {
+        gemm_grouped_kernel<float><<<grid, 256, 0, st>>>(g);
+    }
     count_launches(1);
     return cudaGetLastError();
 }
