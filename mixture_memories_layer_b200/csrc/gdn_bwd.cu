@@ -14,8 +14,9 @@
 //   G_i  <- a G_i - c a b (G_i . k) k
 // (sums over the rows i; dlog_alpha = a dalpha).
 //
-// One CTA owns 64 state rows of one (segment, head): 16 warps of 4 rows, a
-// lane holding d/32 columns of each, as in the token-serial forward.  The
+// One CTA owns 32 state rows of one (segment, head): 8 warps of 4 rows, a
+// lane holding d/32 columns of each, as in the token-serial forward; two
+// CTAs share an SM, so two token-serial chains interleave there.  The
 // reverse pass needs S(t-1) at every token: a forward sweep stores the rows
 // every 64 tokens; the chunks are then walked backwards, each recomputed from
 // its stored state with a copy kept every 4 tokens, and the state before a
@@ -24,7 +25,7 @@
 // by the whole CTA into shared memory, so the replayed steps never wait on
 // L2.  The sums over
 // rows are reduced inside the CTA per token and written as one partial per
-// 64-row tile, which a second kernel adds up (deterministic, no atomics).
+// 32-row tile, which a second kernel adds up (deterministic, no atomics).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,7 +33,7 @@ namespace mom {
 namespace {
 
 constexpr int BR = 4;               // state rows per warp
-constexpr int BW = 16;              // warps per CTA
+constexpr int BW = 8;               // warps per CTA (two CTAs fit an SM: two chains interleave)
 constexpr int ROWS = BR * BW;       // state rows per CTA
 constexpr int CK = 64;              // tokens between stored states
 constexpr int SUB = 4;              // tokens between the copies kept inside a chunk
@@ -75,7 +76,7 @@ struct BwdSmem {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(BW * 32)
+__global__ void __launch_bounds__(BW * 32, 2)
 gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
     using SM = BwdSmem<D>;
     constexpr int E = D / 32;
