@@ -562,7 +562,8 @@ def backward_bench(lay, w, x, cu, flush, steps=3):
     probs = {"shared": (b["q"], None, b["k_sh"], b["v_sh"], cu), "routed": (b["q"], b["perm"], b["k_p"], b["v_p"],
                                                                           b["seg_cu"])}
     out = {"workload": "reverse pass of the %s layer's recurrences (shared + routed), dout ~ N(0,1)" % w.name,
-           "path": "token-serial float32 on CUDA cores, states kept every 64 tokens and re-walked every 8"}
+           "path": "token-serial float32 on CUDA cores (32 state rows per CTA, two CTAs per SM), states kept every 64 "
+                   "tokens, chunks re-walked keeping a copy every 4"}
     total = 0.0
     g = torch.Generator(device=x.device).manual_seed(1)
     for name, (q, qidx, k, v, seg) in probs.items():
@@ -622,7 +623,8 @@ def layer_backward_bench(lay, w, x, cu, flush, steps=3):
         raise SystemExit("device error records in the layer backward: %s" % errs)
     t = sum(ms) / steps
     return {"workload": "backward of the %s layer (all weight and token gradients), dout ~ N(0,1)" % w.name,
-            "path": "recurrence reverse passes token-serial float32; gradient GEMMs float32 on CUDA cores",
+            "path": "recurrence reverse passes token-serial float32; gradient GEMMs on the tf32 tensor cores "
+                    "(fp32 accumulation)",
             "ms": t, "value": w.n_tokens / (t / 1e3), "unit": UNIT}
 
 
