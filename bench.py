@@ -163,11 +163,43 @@ def block_bench(dev, steps, warmup, peaks, flush, name="mom380m_block"):
     ms = sum(step_ms) / steps
     S = int(cu.numel()) - 1
     bf, bb, bt = block_roofline(w, peaks, n_seq=S)
-    return {"workload": workload_desc(w) + "; inside its Gated DeltaNet block (short convolutions of width %d, "
-                                          "gated RMS norm, output projection)" % w.conv_width,
-            "tokens": w.n_tokens, "sequences": S, "ms_per_step": ms, "value": w.n_tokens / (ms / 1e3), "unit": UNIT,
-            "per_call_ms": per_call,
-            "block_roofline": {"flops": bf, "bytes": bb, "roofline_ms": bt * 1e3, "frac": bt * 1e3 / ms}}
+    res = {"workload": workload_desc(w) + "; inside its Gated DeltaNet block (short convolutions of width %d, "
+                                         "gated RMS norm, output projection)" % w.conv_width,
+           "tokens": w.n_tokens, "sequences": S, "ms_per_step": ms, "value": w.n_tokens / (ms / 1e3), "unit": UNIT,
+           "per_call_ms": per_call,
+           "block_roofline": {"flops": bf, "bytes": bb, "roofline_ms": bt * 1e3, "frac": bt * 1e3 / ms}}
+    return res, (blk, w, x, cu)
+
+
+def block_backward_bench(blk, w, x, cu, flush, steps=3):
+    """MoMBlock.backward after a forward on the same tokens (dy ~ N(0,1)):
+    the output projection's and the gated norm's adjoints, the layer's
+    reverse pass, the convolutions' adjoints and every weight's and the
+    tokens' gradients."""
+    import torch
+    g = torch.Generator(device=x.device).manual_seed(3)
+    dy = torch.randn((w.n_tokens, w.d_model), device=x.device, generator=g).to(x.dtype)
+    blk.forward(x, cu)
+    blk.backward(x, cu, dy)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        blk.forward(x, cu)
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        blk.backward(x, cu, dy)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    errs = blk.device_errors()
+    if errs:
+        raise SystemExit("device error records in the block backward: %s" % errs)
+    t = sum(ms) / steps
+    return {"workload": "backward of the %s block (all weight and token gradients), dy ~ N(0,1)" % w.name,
+            "path": "output projection's adjoint on the tcgen05 tensor cores; gated norm and convolution adjoints "
+                    "HBM-streamed; the layer's reverse pass as in layer_backward",
+            "ms": t, "value": w.n_tokens / (t / 1e3), "unit": UNIT}
 
 
 def kernel_source_sha(name):
@@ -454,12 +486,23 @@ def gpu_arm(args):
     decode = None if args.no_decode else decode_bench(args, dev, world, rank, max_over_ranks, barrier)
     configs = None
     if not args.no_configs and world == 1:
+        want = None if args.configs is None else set(args.configs.split(","))
+        on = lambda key: want is None or key in want
         configs = {extra_key(name, rule, mg): config_bench(name, dev, args.steps, args.warmup, peaks, flush, rule, mg)
-                   for name, rule, mg in EXTRA}
-        configs["block"] = block_bench(dev, args.steps, args.warmup, peaks, flush)
-        configs["block_decode"] = block_decode_bench(dev, args.warmup)
-        configs["recurrence_backward"] = backward_bench(lay, w, x, cu, flush)
-        configs["layer_backward"] = layer_backward_bench(lay, w, x, cu, flush)
+                   for name, rule, mg in EXTRA if on(extra_key(name, rule, mg))}
+        if on("block") or on("block_backward"):
+            res, blk_run = block_bench(dev, args.steps, args.warmup, peaks, flush)
+            if on("block"):
+                configs["block"] = res
+            if on("block_backward"):
+                configs["block_backward"] = block_backward_bench(*blk_run, flush)
+            del blk_run
+        if on("block_decode"):
+            configs["block_decode"] = block_decode_bench(dev, args.warmup)
+        if on("recurrence_backward"):
+            configs["recurrence_backward"] = backward_bench(lay, w, x, cu, flush)
+        if on("layer_backward"):
+            configs["layer_backward"] = layer_backward_bench(lay, w, x, cu, flush)
     clocks.__exit__(None, None, None)
     layer_roof["near_tie_tokens"] = near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)
     return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,
@@ -901,6 +944,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode timing")
     ap.add_argument("--no-configs", action="store_true", help="skip the other forward workloads")
+    ap.add_argument("--configs", default=None,
+                    help="comma-separated subset of the other workloads to run (names as in the JSON line's "
+                         "configs; default: all)")
     ap.add_argument("--parallel", default="data", choices=["data", "memory"],
                     help="data: every rank runs the whole layer on its own sequences; memory: the routed "
                          "memories are sharded over the ranks")

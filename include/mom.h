@@ -688,6 +688,55 @@ mom_status mom_block_conv_state(const void* q_raw, const void* k_sh_raw, const v
                                 const int32_t* seg_cu, int n_seq, int n_mem, int channels, int width, mom_dtype dt,
                                 void* conv_sh, void* conv_mem, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The block's reverse pass (training is the pages' main workload: the paper
+ * card, Key points).  With the forward of the calls above:
+ * ---------------------------------------------------------------------- */
+
+/* mom_norm_gate_bwd -- the adjoint of mom_combine_norm_gate: per head of the
+ * combined output o (recomputed from o_sh and the routed rows), r =
+ * 1/sqrt(mean(o^2) + eps), n = o r, s = SiLU(g), dn = d_y w_norm s:
+ *   d_o = r (dn - n mean(dn n))                 [n_tok, H*d] (dt)
+ *   dg[t*ldg + c] = d_y n w_norm SiLU'(g)        float32
+ *   dw_norm = sum over tokens and heads of d_y n s   [d] float32 (overwritten)
+ * The other arguments as mom_combine_norm_gate (d_y is the adjoint of its
+ * output).  bf16 only. */
+mom_status mom_norm_gate_bwd(const void* o_sh, const void* o_p, const int32_t* row_of, const float* topk_gate,
+                             const void* g, const float* w_norm, float eps, const void* d_y, int64_t n_tok,
+                             int top_k, int H, int d, mom_dtype dt, void* d_o, float* dg, int64_t ldg,
+                             float* dw_norm, void* ws, size_t ws_bytes, void* stream);
+
+/* One convolution's adjoint (the forward: one problem of mom_short_conv_batch):
+ * out = [l2norm] SiLU(a), a = conv(z). */
+typedef struct mom_conv_bwd_problem {
+    const void*    z;         /* the forward's raw rows [n_rows, channels] (dt) */
+    const float*   dout;      /* adjoint of out [n_rows, channels] */
+    float*         da;        /* scratch [n_rows, channels] */
+    float*         dz;        /* adjoint of z: dz[r*ldz + col0 + c], overwritten for rows in a segment */
+    int64_t        ldz;
+    int64_t        col0;
+    int64_t        n_rows;
+    const int32_t* seg_cu;    /* as the forward */
+    int            n_seg;
+    int            seg_per_group;
+    int            n_groups;
+    const float*   w;         /* the forward's filters [n_groups, width, channels] */
+    float*         dw;        /* their adjoint, same layout (overwritten) */
+    int            l2norm;
+} mom_conv_bwd_problem;
+
+/* mom_short_conv_bwd -- for 1..8 problems of the same channel count, width
+ * and head_dim: da = the adjoint of a (a recomputed from z, the L2 norm's
+ * adjoint per head when l2norm, then SiLU's); dz[t] = sum_j w[W-1-j] da[t+j]
+ * over the rows t+j in t's segment; dw[grp][W-1-j] = sum_t da[t] z[t-j].
+ * `problems` is a HOST array read during the call.  bf16 z only. */
+mom_status mom_short_conv_bwd(const mom_conv_bwd_problem* problems, int n_problems, int channels, int width,
+                              int head_dim, mom_dtype dt, void* ws, size_t ws_bytes, void* stream);
+
+/* mom_convert -- dst[i] = src[i] converted between float32 and bf16 (round
+ * to nearest even), i < n. */
+mom_status mom_convert(const void* src, mom_dtype src_dt, void* dst, mom_dtype dst_dt, int64_t n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -80,6 +80,10 @@ SIGNATURES = {
     "mom_short_conv_batch": (_I, [_VP, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "mom_combine_norm_gate": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _F, _I64, _I, _I, _I, _I, _VP, _VP, _SZ, _VP]),
     "mom_linear": (_I, [_VP, _VP, _I, _I64, _I, _I, _VP, _VP, _SZ, _VP]),
+    "mom_norm_gate_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _F, _VP, _I64, _I, _I, _I, _I, _VP, _VP, _I64, _VP, _VP,
+                               _SZ, _VP]),
+    "mom_short_conv_bwd": (_I, [_VP, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
+    "mom_convert": (_I, [_VP, _I, _VP, _I, _I64, _VP]),
     "mom_block_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "mom_block_decode_step": (_I, [_VP, _VP, _VP, _VP, _I, _F, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP, _VP,
                                    _VP, _VP, _SZ, _VP]),
@@ -104,6 +108,13 @@ class MomBlockWeights(ctypes.Structure):
     """Mirror of ``struct mom_block_weights`` (device pointers)."""
     _fields_ = [("w_shared4", c_void_p), ("w_o", c_void_p), ("conv_q", c_void_p), ("conv_k_sh", c_void_p),
                 ("conv_v_sh", c_void_p), ("conv_k", c_void_p), ("conv_v", c_void_p), ("w_norm", c_void_p)]
+
+
+class MomConvBwdProblem(ctypes.Structure):
+    """Mirror of ``struct mom_conv_bwd_problem``."""
+    _fields_ = [("z", c_void_p), ("dout", c_void_p), ("da", c_void_p), ("dz", c_void_p), ("ldz", c_int64),
+                ("col0", c_int64), ("n_rows", c_int64), ("seg_cu", c_void_p), ("n_seg", c_int),
+                ("seg_per_group", c_int), ("n_groups", c_int), ("w", c_void_p), ("dw", c_void_p), ("l2norm", c_int)]
 
 
 class MomMemoryGates(ctypes.Structure):
@@ -477,6 +488,48 @@ def mom_linear(x, w, y, ws, stream=None):
     n, k_in = x.shape
     _check(lib.mom_linear(_p(x), _p(w), dtype_code(x.dtype), n, k_in, w.shape[0], _p(y), _p(ws), ws.numel(),
                           _s(stream)), "mom_linear")
+
+
+def mom_norm_gate_bwd(o_sh, o_p, row_of, topk_gate, g, w_norm, eps, d_y, d_o, dg, dw_norm, ws, stream=None,
+                      ldg=None):
+    """d_o [N, H, d] (dt), dg [N, ldg] float32 (columns 0 .. H*d of each row),
+    dw_norm [d] float32."""
+    n_tok, H, d = o_sh.shape
+    top_k = 0 if topk_gate is None else topk_gate.shape[1]
+    ldg = dg.stride(0) if ldg is None else ldg
+    _check(lib.mom_norm_gate_bwd(_p(o_sh), _p(o_p), _p(row_of), _p(topk_gate), _p(g), _p(w_norm), eps, _p(d_y), n_tok,
+                                 top_k, H, d, dtype_code(o_sh.dtype), _p(d_o), ctypes.c_void_p(dg.data_ptr()), ldg,
+                                 _p(dw_norm), _p(ws), ws.numel(), _s(stream)), "mom_norm_gate_bwd")
+
+
+def mom_short_conv_bwd(problems, head_dim, ws, stream=None):
+    """problems: dicts with z, dout, da, dz (a 2-D float32 tensor, possibly a
+    column slice: its row stride and offset are passed), seg_cu, w, dw and
+    optionally seg_per_group, l2norm."""
+    arr = (MomConvBwdProblem * len(problems))()
+    C = width = None
+    for i, q in enumerate(problems):
+        z, w, dz = q["z"], q["w"], q["dz"]
+        n_seg = q["seg_cu"].numel() - 1
+        C = 1
+        for n in z.shape[1:]:
+            C *= n
+        width = w.shape[1]
+        if not dz.is_cuda or dz.dtype != torch.float32 or dz.dim() != 2 or dz.stride(1) != 1:
+            raise ValueError("MoM: dz must be a 2-D float32 CUDA tensor of unit column stride")
+        ldz = dz.stride(0)
+        col0 = dz.storage_offset() % ldz if ldz else 0
+        arr[i] = MomConvBwdProblem(_p(z).value, _p(q["dout"]).value, _p(q["da"]).value,
+                                   dz.data_ptr() - col0 * dz.element_size(), ldz, col0, z.shape[0],
+                                   _p(q["seg_cu"]).value, n_seg, q.get("seg_per_group") or n_seg, w.shape[0],
+                                   _p(w).value, _p(q["dw"]).value, int(q.get("l2norm", False)))
+    _check(lib.mom_short_conv_bwd(arr, len(problems), C, width, head_dim, dtype_code(problems[0]["z"].dtype), _p(ws),
+                                  ws.numel(), _s(stream)), "mom_short_conv_bwd")
+
+
+def mom_convert(src, dst, stream=None):
+    _check(lib.mom_convert(_p(src), dtype_code(src.dtype), _p(dst), dtype_code(dst.dtype), src.numel(), _s(stream)),
+           "mom_convert")
 
 
 def mom_block_decode_workspace_size(B, d_model, H, d, n_mem, top_k):

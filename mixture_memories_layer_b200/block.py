@@ -28,14 +28,15 @@ RMS_EPS = 1e-5
 
 def pack_block_weights(p: Dict[str, np.ndarray], dtype: torch.dtype, device="cuda") -> Dict[str, torch.Tensor]:
     """pack_weights plus the block's: w_shared4 = [W_q; W_k_sh; W_v_sh; W_g],
-    w_o [d_model, H d], the convolution filters tap-major as float32 [groups,
-    width, H d] (conv_q, conv_k_sh, conv_v_sh: one group; conv_k, conv_v: one
-    group per memory) and w_norm [d]."""
+    w_o [d_model, H d] and its transpose w_o_t, the convolution filters
+    tap-major as float32 [groups, width, H d] (conv_q, conv_k_sh, conv_v_sh:
+    one group; conv_k, conv_v: one group per memory) and w_norm [d]."""
     w = pack_weights(p, dtype, device)
     t = lambda a, dt=dtype: torch.as_tensor(np.ascontiguousarray(a)).to(device=device, dtype=dt)
     f32 = torch.float32
     w["w_shared4"] = t(np.concatenate([p["w_q"], p["w_k_sh"], p["w_v_sh"], p["w_g"]], axis=0))
     w["w_o"] = t(p["w_o"])
+    w["w_o_t"] = t(np.transpose(p["w_o"]))                # [H d, d_model]: the reverse pass's dy W_o
     for name in ("conv_q", "conv_k_sh", "conv_v_sh"):
         w[name] = t(np.swapaxes(p[name][None], 1, 2), f32)
     w["conv_k"] = t(np.swapaxes(p["conv_k"], 1, 2), f32)
@@ -167,5 +168,73 @@ class MoMBlock(MoMLayer):
                                 stream=stream, mem_gates=self._c_mem_gates)
         return y, idx
 
-    def backward(self, *a, **k):
-        raise NotImplementedError("the block's backward is not provided (MoMLayer.backward is the layer's)")
+    # ----------------------------------------------------------- backward
+    def backward(self, x: torch.Tensor, cu_seqlens: torch.Tensor, dy: torch.Tensor, dh_shared=None, dh_mem=None,
+                 h0_shared=None, h0_mem=None, stream=None) -> Dict[str, torch.Tensor]:
+        """Gradients of <dy, y> + <dh_shared, h_shared> + <dh_mem, h_mem> for
+        the forward just run on the same x and cu_seqlens (its buffers are
+        read; dy [N, d_model] bf16).  Returns float32: dx; dw_o [d_model, Hd];
+        dw_norm [d]; dw_shared4 [4Hd, D] (W_q | W_k_sh | W_v_sh | W_g);
+        dw_gate [2H, D]; dA, db_a; dw_r, db_r; dw_kv [M, 2Hd, D]; the filters'
+        dconv_q, dconv_k_sh, dconv_v_sh [1, W, Hd] and dconv_k, dconv_v [M, W,
+        Hd] (tap-major, as packed); dh0_shared, dh0_mem.  The routing is held
+        fixed.  Every step runs in the CUDA library: the output projection's
+        two GEMMs, the gated norm's adjoint (which also gives the output
+        gate's), the layer's reverse pass, the five convolutions' adjoints in
+        one launch pair, the gates' adjoint and the projections' GEMMs."""
+        if self.mem_gates:
+            raise NotImplementedError("the backward of per-memory gates is not provided")
+        n_tok, D = x.shape
+        n_seq = cu_seqlens.numel() - 1
+        H, d, K, M, dt = self.H, self.d, self.top_k, self.n_mem, self.dtype
+        Hd, R = H * d, n_tok * K
+        w, b = self.w, self.block_buffers(n_tok, n_seq)
+        st = stream if stream is not None else torch.cuda.current_stream()
+        g = self._bwd_buf
+        ws = self._ws("bwd", B.MOM_WS_HEADER_BYTES)
+        # y = o~ W_o^T: do~ = dy W_o (tensor cores, bf16 out), dW_o = dy^T o~
+        dot = g("do_tilde", (n_tok, H, d), dt)
+        B.mom_linear(dy, w["w_o_t"], dot.view(n_tok, Hd), b["ws_lin"], stream=st)
+        dy32 = g("dy32", (n_tok, D))
+        B.mom_convert(dy, dy32, stream=st)
+        dw_o = g("dw_o", (D, Hd))
+        one = self._buf("one_group", (2,), torch.int32)
+        if getattr(self, "_one_n", None) != n_tok:
+            one.copy_(torch.tensor([0, n_tok], dtype=torch.int32))
+            self._one_n = n_tok
+        B.mom_gemm_grouped(1, dy32, b["o_tilde"].view(n_tok, Hd), dw_o, D, Hd, 0, one, None, 1, ws, stream=st)
+        # o~ = rmsnorm(o) w_norm SiLU(g): do (bf16), dg into the pre-activation
+        # gradients' g columns, dw_norm.  dz [N, 4Hd + 2H]: q | k_sh | v_sh | g | beta | a
+        ldz = (4 * Hd + 2 * H + 3) // 4 * 4
+        dz = g("dz4", (n_tok, ldz))
+        do = g("do", (n_tok, H, d), dt)
+        dw_norm = g("dw_norm", (d,))
+        B.mom_norm_gate_bwd(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["g"], w["w_norm"], self.eps, dot, do,
+                            dz[:, 3 * Hd:], dw_norm, ws, stream=st)
+        c = self._core_bwd(b, cu_seqlens, do, dh_shared, dh_mem, h0_shared, h0_mem, st, ws)
+        # the convolutions (+ SiLU, + L2 norm of q and k) backwards, in place
+        # on the recurrences' input gradients, into the raw projections' columns
+        dzr = g("dzr", (R, 2 * Hd))
+        f = lambda t: t.view(t.shape[0], Hd)
+        dconv = {n: g("d" + n, tuple(w[n].shape)) for n in ("conv_q", "conv_k_sh", "conv_v_sh", "conv_k", "conv_v")}
+        B.mom_short_conv_bwd([
+            dict(z=b["q_raw"], dout=f(c["dq"]), da=f(c["dq"]), dz=dz[:, 0:Hd], seg_cu=cu_seqlens, w=w["conv_q"],
+                 dw=dconv["conv_q"], l2norm=True),
+            dict(z=b["k_sh_raw"], dout=f(c["dk_sh"]), da=f(c["dk_sh"]), dz=dz[:, Hd:2 * Hd], seg_cu=cu_seqlens,
+                 w=w["conv_k_sh"], dw=dconv["conv_k_sh"], l2norm=True),
+            dict(z=b["v_sh_raw"], dout=f(c["dv_sh"]), da=f(c["dv_sh"]), dz=dz[:, 2 * Hd:3 * Hd], seg_cu=cu_seqlens,
+                 w=w["conv_v_sh"], dw=dconv["conv_v_sh"]),
+            dict(z=b["k_p_raw"], dout=f(c["dk_p"]), da=f(c["dk_p"]), dz=dzr[:, 0:Hd], seg_cu=b["seg_cu"],
+                 seg_per_group=n_seq, w=w["conv_k"], dw=dconv["conv_k"], l2norm=True),
+            dict(z=b["v_p_raw"], dout=f(c["dv_p"]), da=f(c["dv_p"]), dz=dzr[:, Hd:], seg_cu=b["seg_cu"],
+                 seg_per_group=n_seq, w=w["conv_v"], dw=dconv["conv_v"]),
+        ], d, ws, stream=st)
+        dala = g("dala", (n_tok, H))
+        B.mom_gates_bwd(b["beta"], b["log_alpha"], c["dbeta"], c["dla"], w["A"], dz, 4 * Hd, 4 * Hd + H, dala,
+                        stream=st)
+        r = self._proj_bwd(x, b, dz, 4 * Hd, w["w_shared4"], dzr, c["dlogits"], dala, st, ws)
+        out = dict(dx=r["dx"], dw_o=dw_o, dw_norm=dw_norm, dw_shared4=r["dw_sh"], dw_gate=r["dw_gate"], dA=r["dA"],
+                   db_a=r["db_a"], dw_r=r["dw_r"], db_r=r["db_r"], dw_kv=r["dw_kv"], dh0_shared=c["dh0_shared"],
+                   dh0_mem=c["dh0_mem"])
+        out.update({"d" + n: t for n, t in dconv.items()})
+        return out

@@ -857,4 +857,51 @@ mom_status mom_block_conv_state(const void* q_raw, const void* k_sh_raw, const v
     return cuda_status(launch_conv_state(a, as_stream(stream)));
 }
 
+// ----------------------------------------------------------- block bwd
+mom_status mom_norm_gate_bwd(const void* o_sh, const void* o_p, const int32_t* row_of, const float* topk_gate,
+                             const void* g, const float* w_norm, float eps, const void* d_y, int64_t n_tok,
+                             int top_k, int H, int d, mom_dtype dt, void* d_o, float* dg, int64_t ldg,
+                             float* dw_norm, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_tok < 0 || top_k < 0 || H < 1 || H > MOM_MAX_HEADS || !(eps >= 0.f)) return MOM_ERR_ARG;
+    if (d < 8 || d > 256 || (d & (d - 1)) != 0 || ldg < (int64_t)H * d) return MOM_ERR_ARG;
+    if (dt != MOM_BF16) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES || !dw_norm || !al16(w_norm)) return MOM_ERR_ARG;
+    const void* ptrs[] = {o_sh, g, d_y, d_o, dg};
+    for (const void* p : ptrs)
+        if (!p || !al16(p)) return MOM_ERR_ARG;
+    if (ldg % 4 != 0) return MOM_ERR_ARG;
+    if (top_k > 0 && (!o_p || !row_of || !topk_gate || !al16(o_p))) return MOM_ERR_ARG;
+    return cuda_status(launch_norm_gate_bwd(o_sh, o_p, row_of, topk_gate, g, w_norm, eps, d_y, n_tok, top_k, H, d,
+                                            d_o, dg, ldg, dw_norm, ws, as_stream(stream)));
+}
+
+mom_status mom_short_conv_bwd(const mom_conv_bwd_problem* problems, int n_problems, int channels, int width,
+                              int head_dim, mom_dtype dt, void* ws, size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || !problems || n_problems < 1 || channels < 8 || channels % 8 != 0 || width < 1) return MOM_ERR_ARG;
+    if (dt != MOM_BF16 || width > 4 || n_problems > 8) return MOM_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    ConvBwdArgs pr[8];
+    for (int i = 0; i < n_problems; ++i) {
+        const mom_conv_bwd_problem& q = problems[i];
+        if (q.n_rows < 0 || q.n_seg < 1 || q.seg_per_group < 1 || q.n_groups < 1) return MOM_ERR_ARG;
+        if (q.l2norm != 0 && q.l2norm != 1) return MOM_ERR_ARG;
+        if (q.l2norm && (head_dim < 8 || head_dim > 256 || (head_dim & (head_dim - 1)) != 0 || channels % head_dim))
+            return MOM_ERR_ARG;
+        if (q.ldz < q.col0 + channels || q.col0 < 0 || q.ldz % 4 || q.col0 % 4) return MOM_ERR_ARG;
+        const void* ptrs[] = {q.z, q.dout, q.da, q.dz, q.seg_cu, q.w, q.dw};
+        for (const void* p : ptrs)
+            if (!p || !al16(p)) return MOM_ERR_ARG;
+        pr[i] = ConvBwdArgs{q.z, q.dout, q.da, q.dz, q.ldz, q.col0, q.n_rows, q.seg_cu, q.n_seg, q.seg_per_group,
+                            q.n_groups, q.w, q.dw, q.l2norm};
+    }
+    return cuda_status(launch_conv_bwd(pr, n_problems, channels, width, head_dim, ws, as_stream(stream)));
+}
+
+mom_status mom_convert(const void* src, mom_dtype src_dt, void* dst, mom_dtype dst_dt, int64_t n, void* stream) {
+    if (!dt_ok(src_dt) || !dt_ok(dst_dt) || n < 0) return MOM_ERR_ARG;
+    if (n == 0) return MOM_OK;
+    if (!src || !dst) return MOM_ERR_ARG;
+    return cuda_status(launch_convert(src, src_dt, dst, dst_dt, n, as_stream(stream)));
+}
+
 }  // extern "C"

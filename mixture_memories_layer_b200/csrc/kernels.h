@@ -253,4 +253,24 @@ cudaError_t launch_combine_norm_gate(const void* o_sh, const void* o_p, const in
                                      const void* g, const float* w_norm, float eps, int64_t n_tok, int K, int H,
                                      int d, void* out, void* ws, cudaStream_t st);
 
+// block_bwd.cu: the block's reverse pass
+cudaError_t launch_norm_gate_bwd(const void* o_sh, const void* o_p, const int32_t* row_of, const float* gate,
+                                 const void* g, const float* w_norm, float eps, const void* dy, int64_t n_tok, int K,
+                                 int H, int d, void* d_o, float* dg, int64_t ldg, float* dw_norm, void* ws,
+                                 cudaStream_t st);
+struct ConvBwdArgs {
+    const void* z;                // raw rows [n_rows, C] (bf16)
+    const float* dout;            // adjoint of the convolution's (normalised) output [n_rows, C]
+    float* da;                    // scratch [n_rows, C]
+    float* dz;                    // adjoint of the raw rows: dz[r * ldz + col0 + c]
+    int64_t ldz, col0, n_rows;
+    const int32_t* seg_cu;
+    int n_seg, seg_per_group, n_groups;
+    const float* w;               // [n_groups, W, C] tap-major
+    float* dw;                    // [n_groups, W, C] (zeroed, then summed into)
+    int l2;
+};
+cudaError_t launch_conv_bwd(const ConvBwdArgs* problems, int n, int C, int W, int d, void* err, cudaStream_t st);
+cudaError_t launch_convert(const void* src, int src_dt, void* dst, int dst_dt, int64_t n, cudaStream_t st);
+
 }  // namespace mom

@@ -262,28 +262,61 @@ class MoMLayer:
             raise NotImplementedError("the backward of per-memory gates is not provided")
         n_tok, D = x.shape
         n_seq = cu_seqlens.numel() - 1
-        H, d, K, M, dt = self.H, self.d, self.top_k, self.n_mem, self.dtype
+        H, d, K, dt = self.H, self.d, self.top_k, self.dtype
         Hd, R = H * d, n_tok * K
         w, b = self.w, self.buffers(n_tok, n_seq)
-        dev, f32 = self.device, torch.float32
         st = stream if stream is not None else torch.cuda.current_stream()
-        g = lambda name, shape, dtype=f32: self._buf("bwd_" + name, shape, dtype)
+        g = self._bwd_buf
         ws = self._ws("bwd", B.MOM_WS_HEADER_BYTES)
         # the lengths the norms' backward needs (the projections again, with their norm outputs)
         qn, kshn, kpn = g("qn", (n_tok, H)), g("kshn", (n_tok, H)), g("kpn", (R, H))
         B.mom_proj_shared(x, w["w_shared"], H, d, g("q2", (n_tok, H, d), dt), g("k2", (n_tok, H, d), dt),
                           g("v2", (n_tok, H, d), dt), ws, stream=st, q_norm=qn, k_sh_norm=kshn)
-        mem_index = getattr(self, "_mem_index", None)       # group g = memory g (set up once)
+        B.mom_kv_proj_groups(x, b["perm"], b["mem_offset"], self._mem_groups(), w["w_kv"], H, d,
+                             g("kp2", (R, H, d), dt), g("vp2", (R, H, d), dt), ws, stream=st, k_norm=kpn)
+        c = self._core_bwd(b, cu_seqlens, dout, dh_shared, dh_mem, h0_shared, h0_mem, st, ws)
+        # pre-activation gradients: shared [N, 3Hd + 2H] (q | k_sh | v_sh | beta | a), routed [N*K, 2Hd] (k | v)
+        ldz = (3 * Hd + 2 * H + 3) // 4 * 4        # rows 16-byte aligned for the row copies
+        dz = g("dz", (n_tok, ldz))
+        B.mom_l2norm_bwd(b["q"], c["dq"], qn, dz, 0, stream=st)
+        B.mom_l2norm_bwd(b["k_sh"], c["dk_sh"], kshn, dz, Hd, stream=st)
+        B.mom_copy_rows(c["dv_sh"].view(n_tok, Hd), None, dz, Hd * 4, src_off=0, dst_off=2 * Hd * 4, ws=ws,
+                        stream=st)
+        dala = g("dala", (n_tok, H))
+        B.mom_gates_bwd(b["beta"], b["log_alpha"], c["dbeta"], c["dla"], w["A"], dz, 3 * Hd, 3 * Hd + H, dala,
+                        stream=st)
+        dzr = g("dzr", (R, 2 * Hd))
+        B.mom_l2norm_bwd(b["k_p"], c["dk_p"], kpn, dzr, 0, stream=st)
+        B.mom_copy_rows(c["dv_p"].view(R, Hd), None, dzr, Hd * 4, src_off=0, dst_off=Hd * 4, ws=ws, stream=st)
+        r = self._proj_bwd(x, b, dz, 3 * Hd, w["w_shared"], dzr, c["dlogits"], dala, st, ws)
+        return dict(dx=r["dx"], dw_r=r["dw_r"], db_r=r["db_r"], dw_shared=r["dw_sh"], dw_gate=r["dw_gate"],
+                    dA=r["dA"], db_a=r["db_a"], dw_kv=r["dw_kv"], dh0_shared=c["dh0_shared"], dh0_mem=c["dh0_mem"])
+
+    def _bwd_buf(self, name, shape, dtype=torch.float32):
+        return self._buf("bwd_" + name, shape, dtype)
+
+    def _mem_groups(self):
+        """[0, 1, .., M-1] int32 on the device: group g of the routed rows is memory g."""
+        mem_index = getattr(self, "_mem_index", None)
         if mem_index is None:
-            mem_index = self._mem_index = torch.arange(M, dtype=torch.int32, device=dev)
-        B.mom_kv_proj_groups(x, b["perm"], b["mem_offset"], mem_index, w["w_kv"], H, d, g("kp2", (R, H, d), dt),
-                             g("vp2", (R, H, d), dt), ws, stream=st, k_norm=kpn)
-        # combine and router
-        do_p, dgate = g("do_p", (R, H, d), dt), g("dgate", (n_tok, K))
+            mem_index = self._mem_index = torch.arange(self.n_mem, dtype=torch.int32, device=self.device)
+        return mem_index
+
+    def _core_bwd(self, b, cu_seqlens, dout, dh_shared, dh_mem, h0_shared, h0_mem, st, ws):
+        """The reverse pass from the adjoint of the combined output (dout [N, H,
+        d], the model dtype) to the recurrences' inputs: the combine's and the
+        router's adjoints, both recurrences' reverse passes, and each token's
+        routed rows summed into its own.  Returns float32 dq, dk_sh, dv_sh
+        [N, H, d], dk_p, dv_p [N*K, H, d], dbeta, dla [N, H], dlogits [N, M],
+        dh0_shared, dh0_mem."""
+        n_tok, n_seq = b["idx"].shape[0], cu_seqlens.numel() - 1
+        H, d, K, M = self.H, self.d, self.top_k, self.n_mem
+        Hd, R = H * d, n_tok * K
+        g = self._bwd_buf
+        do_p, dgate = g("do_p", (R, H, d), self.dtype), g("dgate", (n_tok, K))
         B.mom_combine_bwd(dout, b["o_p"], b["row_of"], b["gate"], do_p, dgate, ws, stream=st)
         dlogits = g("dlogits", (n_tok, M))
         B.mom_router_bwd(b["idx"], b["gate"], dgate, dlogits, ws, stream=st)
-        # the recurrences' reverse passes
         dq_sh, dk_sh, dv_sh = (g(n, (n_tok, H, d)) for n in ("dq_sh", "dk_sh", "dv_sh"))
         db_sh, dla_sh = g("db_sh", (n_tok, H)), g("dla_sh", (n_tok, H))
         dq_p, dk_p, dv_p = (g(n, (R, H, d)) for n in ("dq_p", "dk_p", "dv_p"))
@@ -304,45 +337,45 @@ class MoMLayer:
         B.mom_rows_sum(dq_p.view(R, Hd), b["row_of"], K, dq_sh.view(n_tok, Hd), dq.view(n_tok, Hd), ws, stream=st)
         B.mom_rows_sum(db_p, b["row_of"], K, db_sh, dbeta, ws, stream=st)
         B.mom_rows_sum(dla_p, b["row_of"], K, dla_sh, dla, ws, stream=st)
-        # pre-activation gradients: shared [N, 3Hd + 2H] (q | k_sh | v_sh | beta | a), routed [N*K, 2Hd] (k | v)
-        ldz = (3 * Hd + 2 * H + 3) // 4 * 4        # rows 16-byte aligned for the row copies
-        dz = g("dz", (n_tok, ldz))
-        B.mom_l2norm_bwd(b["q"], dq, qn, dz, 0, stream=st)
-        B.mom_l2norm_bwd(b["k_sh"], dk_sh, kshn, dz, Hd, stream=st)
-        B.mom_copy_rows(dv_sh.view(n_tok, Hd), None, dz, Hd * 4, src_off=0, dst_off=2 * Hd * 4, ws=ws, stream=st)
-        dala = g("dala", (n_tok, H))
-        B.mom_gates_bwd(b["beta"], b["log_alpha"], dbeta, dla, w["A"], dz, 3 * Hd, 3 * Hd + H, dala, stream=st)
-        dzr = g("dzr", (R, 2 * Hd))
-        rows = int(R)
-        B.mom_l2norm_bwd(b["k_p"], dk_p, kpn, dzr, 0, stream=st)
-        B.mom_copy_rows(dv_p.view(R, Hd), None, dzr, Hd * 4, src_off=0, dst_off=Hd * 4, ws=ws, stream=st)
-        # input gradient: shared, gates, router, then the routed rows summed per token
-        one = self._buf("one_group", (2,), torch.int32)
-        one.copy_(torch.tensor([0, n_tok], dtype=torch.int32, device=dev))
+        return dict(dq=dq, dk_sh=dk_sh, dv_sh=dv_sh, dk_p=dk_p, dv_p=dv_p, dbeta=dbeta, dla=dla, dlogits=dlogits,
+                    dh0_shared=dh0_sh, dh0_mem=dh0_m)
+
+    def _proj_bwd(self, x, b, dz, n_sh, w_sh, dzr, dlogits, dala, st, ws):
+        """The projections' input and weight gradients from the pre-activation
+        gradients: dz [N, ldz] float32 holds n_sh columns against w_sh [n_sh,
+        D] then beta | a (2H) against w_gate; dzr [N*K, 2Hd] the routed rows'
+        against w_kv; dlogits [N, M] against w_r.  Returns dx, dw_sh, dw_gate,
+        dw_r, dw_kv, db_r, dA, db_a (float32)."""
+        n_tok, D = x.shape
+        H, Hd, K, M = self.H, self.H * self.d, self.top_k, self.n_mem
+        R = n_tok * K
+        w, g = self.w, self._bwd_buf
+        one = self._buf("one_group", (2,), torch.int32)     # one group of all n_tok rows
+        if getattr(self, "_one_n", None) != n_tok:
+            one.copy_(torch.tensor([0, n_tok], dtype=torch.int32))
+            self._one_n = n_tok
         dx = g("dx", (n_tok, D))
-        B.mom_gemm_grouped(0, dz, w["w_shared"], dx, 0, D, 3 * Hd, one, None, 1, ws, total_rows=n_tok, stream=st)
-        B.mom_gemm_grouped(0, dz, w["w_gate"], dx, 0, D, 2 * H, one, None, 1, ws, a_col=3 * Hd, total_rows=n_tok,
+        B.mom_gemm_grouped(0, dz, w_sh, dx, 0, D, n_sh, one, None, 1, ws, total_rows=n_tok, stream=st)
+        B.mom_gemm_grouped(0, dz, w["w_gate"], dx, 0, D, 2 * H, one, None, 1, ws, a_col=n_sh, total_rows=n_tok,
                            accumulate=True, stream=st)
         B.mom_gemm_grouped(0, dlogits, w["w_r"], dx, 0, D, M, one, None, 1, ws, total_rows=n_tok, accumulate=True,
                            stream=st)
         dx_rows = g("dx_rows", (R, D))
-        B.mom_gemm_grouped(0, dzr, w["w_kv"], dx_rows, 0, D, 2 * Hd, b["mem_offset"], None, M, ws, total_rows=rows,
+        B.mom_gemm_grouped(0, dzr, w["w_kv"], dx_rows, 0, D, 2 * Hd, b["mem_offset"], None, M, ws, total_rows=R,
                            b_group_stride=2 * Hd * D, stream=st)
         B.mom_rows_sum(dx_rows, b["row_of"], K, dx, dx, ws, stream=st)
-        # weight gradients
-        dw_shared, dw_gate, dw_r = g("dw_shared", (3 * Hd, D)), g("dw_gate", (2 * H, D)), g("dw_r", (M, D))
+        dw_sh, dw_gate, dw_r = g("dw_sh", (n_sh, D)), g("dw_gate", (2 * H, D)), g("dw_r", (M, D))
         dw_kv = g("dw_kv", (M, 2 * Hd, D))
-        B.mom_gemm_grouped(1, dz, x, dw_shared, 3 * Hd, D, 0, one, None, 1, ws, stream=st)
-        B.mom_gemm_grouped(1, dz, x, dw_gate, 2 * H, D, 0, one, None, 1, ws, a_col=3 * Hd, stream=st)
+        B.mom_gemm_grouped(1, dz, x, dw_sh, n_sh, D, 0, one, None, 1, ws, stream=st)
+        B.mom_gemm_grouped(1, dz, x, dw_gate, 2 * H, D, 0, one, None, 1, ws, a_col=n_sh, stream=st)
         B.mom_gemm_grouped(1, dlogits, x, dw_r, M, D, 0, one, None, 1, ws, stream=st)
         B.mom_gemm_grouped(1, dzr, x, dw_kv.view(M * 2 * Hd, D), 2 * Hd, D, 0, b["mem_offset"], None, M, ws,
                            b_rows=b["perm"], c_group_stride=2 * Hd * D, stream=st)
         db_r, dA, db_a = g("db_r", (M,)), g("dA", (H,)), g("db_a", (H,))
         B.mom_col_sums(dlogits, db_r, stream=st)
         B.mom_col_sums(dala, dA, stream=st)
-        B.mom_col_sums(dz, db_a, col0=3 * Hd + H, stream=st)
-        return dict(dx=dx, dw_r=dw_r, db_r=db_r, dw_shared=dw_shared, dw_gate=dw_gate, dA=dA, db_a=db_a, dw_kv=dw_kv,
-                    dh0_shared=dh0_sh, dh0_mem=dh0_m)
+        B.mom_col_sums(dz, db_a, col0=n_sh + H, stream=st)
+        return dict(dx=dx, dw_sh=dw_sh, dw_gate=dw_gate, dw_r=dw_r, dw_kv=dw_kv, db_r=db_r, dA=dA, db_a=db_a)
 
     # --------------------------------------------------------------- decode
     def decode_step(self, x: torch.Tensor, state: torch.Tensor, stream=None):
