@@ -349,13 +349,29 @@ gemm_grouped_tf32_kernel(GemmArgs g) {
     // k = (tid % 2) TVAL + e (trans_a = 0) or k = tid / TPR, m = (tid % TPR)
     // TVAL + e (trans_a = 1); B: k = tid / TPR, n = (tid % TPR) TVAL + e
     float ra[TVAL], rb[TVAL];
+    // each thread's TVAL values of an operand are contiguous in memory (A's
+    // k run or m run, B's n run): two 16-byte loads of A, one of B where the
+    // run is whole and aligned, element loads at the ragged edges
+    const bool a_vec = ((reinterpret_cast<uintptr_t>(g.A) & 15) == 0) && (g.lda % 4 == 0) &&
+                       (g.trans_a || (k0 & 3) == 0);
+    const bool b_vec = ((reinterpret_cast<uintptr_t>(Bg) & 15) == 0) && (g.ldb % 8 == 0);
     auto load = [&](int64_t kb) {
+        int64_t am, ak;                                   // the first of the thread's A values
+        if (!g.trans_a) { am = m0 + (tid >> 1); ak = kb + (tid & 1) * TVAL; } else { ak = kb + tid / TPR; am = m0 + (tid % TPR) * TVAL; }
+        const bool a_whole = g.trans_a ? (ak < k1 && am + TVAL <= m1) : (am < m1 && ak + TVAL <= k1);
+        if (a_vec && a_whole) {
+            const float4* src = reinterpret_cast<const float4*>(g.A + (g.trans_a ? ak * g.lda + am : am * g.lda + ak));
 #pragma unroll
-        for (int e = 0; e < TVAL; ++e) {
-            int kk, mm;
-            if (!g.trans_a) { mm = tid >> 1; kk = (tid & 1) * TVAL + e; } else { kk = tid / TPR; mm = (tid % TPR) * TVAL + e; }
-            const int64_t m = m0 + mm, k = kb + kk;
-            ra[e] = (m < m1 && k < k1) ? (g.trans_a ? g.A[k * g.lda + m] : g.A[m * g.lda + k]) : 0.f;
+            for (int v = 0; v < TVAL / 4; ++v) {
+                const float4 q = __ldg(src + v);
+                ra[4 * v] = q.x; ra[4 * v + 1] = q.y; ra[4 * v + 2] = q.z; ra[4 * v + 3] = q.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < TVAL; ++e) {
+                const int64_t m = g.trans_a ? am + e : am, k = g.trans_a ? ak : ak + e;
+                ra[e] = (m < m1 && k < k1) ? (g.trans_a ? g.A[k * g.lda + m] : g.A[m * g.lda + k]) : 0.f;
+            }
         }
         const int kk = tid / TPR;
         const int64_t k = kb + kk;
@@ -364,10 +380,26 @@ gemm_grouped_tf32_kernel(GemmArgs g) {
             br = g.b_rows[k];
             if (br < 0 || br >= g.n_b_rows) { record_error(g.err, MOM_DEVERR_ROW_INDEX, k); br = -1; }
         }
+        const int64_t nb = n0 + (tid % TPR) * TVAL;
+        if (b_vec && k < k1 && br >= 0 && nb + TVAL <= g.N) {
+            static_assert(TVAL % 8 == 0, "whole 16-byte runs of B");
+            const uint4* src = reinterpret_cast<const uint4*>(Bg + br * g.ldb + nb);
 #pragma unroll
-        for (int e = 0; e < TVAL; ++e) {
-            const int64_t n = n0 + (tid % TPR) * TVAL + e;
-            rb[e] = (k < k1 && br >= 0 && n < g.N) ? __bfloat162float(Bg[br * g.ldb + n]) : 0.f;
+            for (int v = 0; v < TVAL / 8; ++v) {
+                const uint4 q = __ldg(src + v);
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    rb[8 * v + 2 * e] = __uint_as_float(w4[e] << 16);
+                    rb[8 * v + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < TVAL; ++e) {
+                const int64_t n = nb + e;
+                rb[e] = (k < k1 && br >= 0 && n < g.N) ? __bfloat162float(Bg[br * g.ldb + n]) : 0.f;
+            }
         }
     };
     auto store = [&](int buf) {

@@ -77,3 +77,57 @@ def test_layer_backward_without_state_gradients():
     errs = _run("f32", 64, (90, 33), M=5, K=3, seed=83, with_states=False)
     bad = {k: e for k, e in errs.items() if not e < 1e-5}
     assert not bad, bad
+
+
+# ------------------------------------------------- the grouped GEMM alone --
+def _gemm_case(trans_a, a_col, lda_pad, seed):
+    """mom_gemm_grouped with bf16 B (the tf32 tensor-core kernel) against
+    numpy in fp64: groups of ragged sizes (one empty), a ragged N, A read
+    from column a_col of a wider matrix (a_col and the row pitch decide
+    whether the 16-byte loads or the element loads run), the routed form's
+    gathered B rows and per-group C, and accumulation into C."""
+    from mixture_memories_layer_b200 import binding as B
+    rng = np.random.default_rng(seed)
+    sizes = [130, 0, 77, 256, 5]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    rows, G = int(off[-1]), len(sizes)
+    ws = B.new_workspace(B.MOM_WS_HEADER_BYTES)
+    bf = lambda a: torch.as_tensor(a, dtype=torch.float32).to("cuda", torch.bfloat16)
+    if not trans_a:
+        K, N = 96, 200
+        A = rng.standard_normal((rows, K + lda_pad)).astype(np.float32)
+        Bw = bf(rng.standard_normal((G, K, N)))
+        gidx = rng.permutation(G).astype(np.int32)
+        C0 = rng.standard_normal((rows, N)).astype(np.float32)
+        C = torch.as_tensor(C0).cuda()
+        B.mom_gemm_grouped(0, torch.as_tensor(A).cuda(), Bw, C, 0, N, K, torch.as_tensor(off).cuda(),
+                           torch.as_tensor(gidx).cuda(), G, ws, a_col=a_col, total_rows=rows, b_group_stride=K * N,
+                           accumulate=True)
+        Bn = Bw.float().cpu().numpy().astype(np.float64)
+        ref = C0.astype(np.float64).copy()
+        for q in range(G):
+            ref[off[q]:off[q + 1]] += A[off[q]:off[q + 1], a_col:a_col + K].astype(np.float64) @ Bn[gidx[q]]
+    else:
+        M, N, n_b = 72, 136, 700
+        A = rng.standard_normal((rows, M + lda_pad)).astype(np.float32)
+        Bx = bf(rng.standard_normal((n_b, N)))
+        b_rows = rng.integers(0, n_b, rows).astype(np.int32)
+        C = torch.zeros((G * M, N), device="cuda")
+        B.mom_gemm_grouped(1, torch.as_tensor(A).cuda(), Bx, C, M, N, 0, torch.as_tensor(off).cuda(), None, G, ws,
+                           a_col=a_col, b_rows=torch.as_tensor(b_rows).cuda(), c_group_stride=M * N)
+        Bn = Bx.float().cpu().numpy().astype(np.float64)
+        ref = np.zeros((G * M, N))
+        for q in range(G):
+            r = slice(off[q], off[q + 1])
+            ref[q * M:(q + 1) * M] = A[r, a_col:a_col + M].astype(np.float64).T @ Bn[b_rows[r]]
+    torch.cuda.synchronize()
+    assert B.mom_get_error(ws)[0] == 0
+    return max_abs_rel(C.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("trans_a", [0, 1])
+@pytest.mark.parametrize("a_col,lda_pad", [(0, 0), (4, 8), (1, 3)])
+def test_gemm_grouped_tf32(trans_a, a_col, lda_pad):
+    """tf32 products (A rounded to a 10-bit mantissa, B exact, fp32 sums):
+    within 2e-3 of the fp64 product per tensor."""
+    assert _gemm_case(trans_a, a_col, lda_pad, seed=10 * trans_a + a_col) < 2e-3
