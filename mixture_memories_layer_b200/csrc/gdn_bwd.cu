@@ -18,9 +18,15 @@
 // lane holding d/32 columns of each, as in the token-serial forward; two
 // CTAs share an SM, so two token-serial chains interleave there.  The
 // reverse pass needs S(t-1) at every token: a forward sweep stores the rows
-// every 64 tokens; the chunks are then walked backwards, each recomputed from
-// its stored state with a copy kept every 4 tokens, and the state before a
-// token is rebuilt from the nearest copy (at most 3 steps).  The operands of
+// every 16 tokens; the chunks are then walked backwards, each recomputed from
+// its stored state with a copy kept every 2 tokens, and the state before a
+// token is rebuilt from the nearest copy (at most 1 step).  The copies of
+// the chunks in flight stay in L2 (8 per CTA: 256 KB; with 64-token chunks
+// the ~300 resident CTAs' copies overflowed it and every rebuild waited on
+// HBM).  The kernel is
+// bound by instruction issue, the warp shuffles of the per-row dot products
+// first: the 4 rows of a warp are summed together by a reduce-scatter and
+// gather (9 shuffles, not 20).  The operands of
 // each 16-token block (k, q, the CTA's v and d_o, the gates) are loaded once
 // by the whole CTA into shared memory, so the replayed steps never wait on
 // L2.  The sums over
@@ -33,12 +39,14 @@ namespace mom {
 namespace {
 
 constexpr int BR = 4;               // state rows per warp
+static_assert(BR == 4, "warp_allreduce4 sums the 4 rows of a warp");
 constexpr int BW = 8;               // warps per CTA (two CTAs fit an SM: two chains interleave)
 constexpr int ROWS = BR * BW;       // state rows per CTA
-constexpr int CK = 64;              // tokens between stored states
-constexpr int SUB = 4;              // tokens between the copies kept inside a chunk
+constexpr int CK = 16;              // tokens between stored states (a chunk: one operand block)
+constexpr int SUB = 2;              // tokens between the copies kept inside a chunk
 constexpr int NSUB = CK / SUB;
 constexpr int CACHE = 16;           // tokens whose operands one fill brings into shared memory
+static_assert(CK % CACHE == 0 && CACHE % SUB == 0, "stored states and copies on operand-block bounds");
 
 struct BwdTables {
     int32_t* chunk_cu;   // [n_seg + 1] first stored state of each segment
@@ -46,6 +54,29 @@ struct BwdTables {
     float* sub;          // [n_seg * tiles * H][NSUB][ROWS][D]
     float* part;         // [tiles][n_rows][H][2D + 2]: dq | dk | dlog_alpha | dbeta
 };
+
+// The sums over a warp of 4 values per lane, in every lane: a reduce-scatter
+// (each lane pair halves its set of values, twice), the last value summed
+// over the remaining 8 lanes, then the 4 totals gathered back -- 9 shuffles
+// where four independent butterflies take 20.
+__device__ __forceinline__ void warp_allreduce4(float* v) {
+    const int lane = threadIdx.x & 31;
+    const bool hi = lane & 16, hb = lane & 8;
+    const float r0 = __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[2], 16);
+    const float r1 = __shfl_xor_sync(0xffffffffu, hi ? v[1] : v[3], 16);
+    const float k0 = (hi ? v[2] : v[0]) + r0, k1 = (hi ? v[3] : v[1]) + r1;   // values base, base+1
+    float x = (hb ? k1 : k0) + __shfl_xor_sync(0xffffffffu, hb ? k0 : k1, 8); // value base + hb
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    const float o = __shfl_xor_sync(0xffffffffu, x, 8);
+    const float t0 = hb ? o : x, t1 = hb ? x : o;                            // totals base, base+1
+    const float u0 = __shfl_xor_sync(0xffffffffu, t0, 16), u1 = __shfl_xor_sync(0xffffffffu, t1, 16);
+    v[0] = hi ? u0 : t0;
+    v[1] = hi ? u1 : t1;
+    v[2] = hi ? t0 : u0;
+    v[3] = hi ? t1 : u1;
+}
 
 __global__ void bwd_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_seg, int64_t n_rows,
                                     int32_t* __restrict__ chunk_cu, void* err) {
@@ -63,8 +94,8 @@ __global__ void bwd_schedule_kernel(const int32_t* __restrict__ seg_cu, int n_se
 template <int D>
 struct BwdSmem {
     static constexpr int PW = 2 * D + 2;                      // partial width: dq | dk | dlog_alpha | dbeta
-    static constexpr int RED = 0;                             // [BW][PW] per-warp sums over rows
-    static constexpr int KC = RED + BW * PW;                  // [CACHE][D] k of the cached tokens
+    static constexpr int RED = 0;                             // [2][BW][PW] per-warp sums over rows (two tokens)
+    static constexpr int KC = RED + 2 * BW * PW;              // [CACHE][D] k of the cached tokens
     static constexpr int QC = KC + CACHE * D;                 // [CACHE][D] q
     static constexpr int VC = QC + CACHE * D;                 // [CACHE][ROWS] v of this CTA's rows
     static constexpr int DC = VC + CACHE * ROWS;              // [CACHE][ROWS] d_o
@@ -114,29 +145,47 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
     // the whole CTA (every replay and reverse step then reads them from there)
     auto fill = [&](int64_t ts, int n, bool want_do) {
         __syncthreads();                                      // the previous block's readers are done
-        for (int i = threadIdx.x; i < n; i += NT) {
-            const int64_t r = ts + i;
+        if (threadIdx.x < n) {
+            const int64_t r = ts + threadIdx.x;
             const int64_t qr = a.qidx ? (int64_t)a.qidx[r] : r;
             const bool ok = qr >= 0 && qr < a.n_q_rows;
             if (!ok && tile == 0) record_error(a.ws, MOM_DEVERR_ROW_INDEX, r);
             const int64_t gr = a.gates_by_row ? r : qr;
-            okc[i] = ok ? 1.f : 0.f;
-            bc[i] = ok ? a.beta[gr * H + h] : 0.f;
-            ac[i] = ok ? expf(a.log_alpha[gr * H + h]) : 1.f;
+            okc[threadIdx.x] = ok ? 1.f : 0.f;
+            bc[threadIdx.x] = ok ? a.beta[gr * H + h] : 0.f;
+            ac[threadIdx.x] = ok ? expf(a.log_alpha[gr * H + h]) : 1.f;
         }
-        for (int i = threadIdx.x; i < n * D; i += NT) {
-            const int j = i / D, c = i - j * D;
-            const int64_t r = ts + j;
-            const int64_t qr = a.qidx ? (int64_t)a.qidx[r] : r;
-            const bool ok = qr >= 0 && qr < a.n_q_rows;
-            kc[j * D + c] = to_f(k[(r * H + h) * D + c]);
-            qc[j * D + c] = ok ? to_f(q[(qr * H + h) * D + c]) : 0.f;
+        // k and q rows in pieces of 8 values (one 16-byte load of bf16):
+        // a thread's k and q pieces loaded together, then stored (the state
+        // and its adjoint stay in registers meanwhile, so one pair at a time)
+        constexpr int PR = D / 8;                             // pieces per row
+        constexpr int ITK = (CACHE * PR + NT - 1) / NT;
+#pragma unroll
+        for (int it = 0; it < ITK; ++it) {
+            const int i = threadIdx.x + it * NT, j = i / PR, c = (i % PR) * 8;
+            if (j < n) {
+                const int64_t r = ts + j;
+                const int64_t qr = a.qidx ? (int64_t)a.qidx[r] : r;
+                float kv[8], qv[8];
+                load_vec<8>(k + (r * H + h) * D + c, kv);
+                if (qr >= 0 && qr < a.n_q_rows) load_vec<8>(q + (qr * H + h) * D + c, qv);
+                else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) qv[e] = 0.f;
+                }
+                store_vec<8>(kc + j * D + c, kv);
+                store_vec<8>(qc + j * D + c, qv);
+            }
         }
-        for (int i = threadIdx.x; i < n * ROWS; i += NT) {
-            const int j = i / ROWS, c = i - j * ROWS;
+        // this CTA's rows of v (and d_o): threads 0 .. VP-1 and VP .. 2 VP-1
+        constexpr int VP = CACHE * ROWS / 8;
+        static_assert(2 * VP <= NT, "one piece of v or d_o per thread");
+        const int which = threadIdx.x / VP, i = threadIdx.x % VP, j = i / (ROWS / 8), c = (i % (ROWS / 8)) * 8;
+        if (which < 2 && j < n && (which == 0 || want_do)) {
             const int64_t off = ((ts + j) * H + h) * D + tile * ROWS + c;
-            vc[j * ROWS + c] = to_f(v[off]);
-            dc[j * ROWS + c] = want_do ? to_f(dout[off]) : 0.f;
+            float vv[8];
+            load_vec<8>((which == 0 ? v : dout) + off, vv);
+            store_vec<8>((which == 0 ? vc : dc) + j * ROWS + c, vv);
         }
         __syncthreads();
     };
@@ -156,7 +205,7 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
             for (int e = 0; e < E; ++e) acc = fmaf(S[i][e], kk[e], acc);
             y[i] = acc;
         }
-        warp_sum_n<BR>(y);
+        warp_allreduce4(y);
         const float dl = delta ? al : 0.f;
 #pragma unroll
         for (int i = 0; i < BR; ++i) {
@@ -196,14 +245,20 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
             for (int e = 0; e < E; ++e) G[i][e] = 0.f;
         }
     }
-    float* w = red + warp * PW;
+    // the per-warp sums of consecutive tokens alternate between two buffers:
+    // a buffer is written again two tokens later, after every thread that
+    // read it has passed the next token's barrier, so one barrier per token
+    // suffices
+    int par = 0;
     for (int64_t jc = nck - 1; jc >= 0; --jc) {
         const int64_t t0 = r0 + jc * CK, t1 = t0 + CK < r1 ? t0 + CK : r1;
 #pragma unroll
         for (int i = 0; i < BR; ++i) load_vec<E>(ck + (size_t)jc * ck_stride + (size_t)i * D, S[i]);
+        // a chunk of one operand block: the re-walk's fill (with d_o) serves the reverse too
+        const int ncb = (int)((t1 - t0 + CACHE - 1) / CACHE);
         for (int64_t tc = t0; tc < t1; tc += CACHE) {
             const int n = (int)(t1 - tc < CACHE ? t1 - tc : CACHE);
-            fill(tc, n, false);
+            fill(tc, n, ncb == 1);
             for (int j = 0; j < n; ++j) {
                 if (j % SUB == 0) {
 #pragma unroll
@@ -213,11 +268,10 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
                 step(j);
             }
         }
-        const int ncb = (int)((t1 - t0 + CACHE - 1) / CACHE);
         for (int cb = ncb - 1; cb >= 0; --cb) {
             const int64_t tc = t0 + (int64_t)cb * CACHE;
             const int n = (int)(t1 - tc < CACHE ? t1 - tc : CACHE);
-            fill(tc, n, true);
+            if (ncb > 1) fill(tc, n, true);
             for (int jt = n - 1; jt >= 0; --jt) {
                 const int64_t t = tc + jt;
                 // S(t-1): the nearest kept copy, then forward to t
@@ -227,6 +281,7 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
                     load_vec<E>(sub + (size_t)((tc + js - t0) / SUB) * ROWS * D + (size_t)i * D, S[i]);
                 for (int j = js; j < jt; ++j) step(j);
                 // the token's own reverse step
+                float* w = red + (par * BW + warp) * PW;
                 if (okc[jt] != 0.f) {
                     float kk[E], qq[E];
                     load_vec<E>(kc + jt * D + lane * E, kk);
@@ -242,11 +297,11 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
                         for (int e = 0; e < E; ++e) acc = fmaf(S[i][e], kk[e], acc);
                         y[i] = acc;
                     }
-                    warp_sum_n<BR>(y);
+                    warp_allreduce4(y);
                     float u[BR], dq[E], dk[E];
 #pragma unroll
                     for (int e = 0; e < E; ++e) { dq[e] = 0.f; dk[e] = 0.f; }
-                    float red2[2 * BR];                   // G.k, G.S(t-1) per row
+                    float gkv[BR], gsum = 0.f;            // G.k per row; G.S(t-1) summed over the rows
 #pragma unroll
                     for (int i = 0; i < BR; ++i) {
                         u[i] = b * (vv[i] - dl * y[i]);
@@ -260,16 +315,17 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
                             gk = fmaf(G[i][e], kk[e], gk);
                             gs = fmaf(G[i][e], S[i][e], gs);
                         }
-                        red2[2 * i] = gk;
-                        red2[2 * i + 1] = gs;
+                        gkv[i] = gk;
+                        gsum += gs;
                     }
-                    warp_sum_n<2 * BR>(red2);
-                    float dalpha = 0.f, dbeta = 0.f;
+                    warp_allreduce4(gkv);
+                    warp_sum_n<1>(&gsum);
+                    float dalpha = gsum, dbeta = 0.f;
 #pragma unroll
                     for (int i = 0; i < BR; ++i) {
-                        const float gk = red2[2 * i], gs = red2[2 * i + 1];
+                        const float gk = gkv[i];
                         dbeta += (vv[i] - dl * y[i]) * gk;
-                        dalpha += gs - (delta ? b * y[i] * gk : 0.f);
+                        dalpha -= delta ? b * y[i] * gk : 0.f;
                         if (lane == i) a.dv[(t * H + h) * D + row0 + i] = b * gk;
 #pragma unroll
                         for (int e = 0; e < E; ++e) {
@@ -285,13 +341,14 @@ gdn_bwd_kernel(GdnBwdArgs a, BwdTables tb) {
                 }
                 __syncthreads();
                 float* pout = tb.part + (((size_t)tile * a.n_rows + t) * H + h) * PW;
+                const float* rb = red + par * BW * PW;
                 for (int c = threadIdx.x; c < PW; c += NT) {
                     float acc = 0.f;
 #pragma unroll
-                    for (int ww = 0; ww < BW; ++ww) acc += red[ww * PW + c];
+                    for (int ww = 0; ww < BW; ++ww) acc += rb[ww * PW + c];
                     pout[c] = acc;
                 }
-                __syncthreads();
+                par ^= 1;
             }
         }
     }
