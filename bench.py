@@ -141,6 +141,16 @@ def block_roofline(w, peaks, n_seq=None):
     return flops, bytes_, t
 
 
+def backward_roofline(fwd_flops, peaks, ms):
+    """The usual estimate of a backward's algorithmic work, twice its
+    forward's FLOPs (an input and a weight gradient per product, the
+    recurrence's reverse pass about twice its forward), against the bf16
+    peak: {"flops", "roofline_ms", "frac"}."""
+    flops = 2 * fwd_flops
+    t_ms = flops / (peaks["bf16_tflops"] * 1e12) * 1e3
+    return {"flops": flops, "roofline_ms": t_ms, "frac": t_ms / ms, "estimate": "2 x the forward's FLOPs"}
+
+
 def block_bench(dev, steps, warmup, peaks, flush, name="mom380m_block"):
     """The 380M-shape layer inside its Gated DeltaNet block (short
     convolutions, gated norm, output projection), timed like the headline
@@ -171,7 +181,7 @@ def block_bench(dev, steps, warmup, peaks, flush, name="mom380m_block"):
     return res, (blk, w, x, cu)
 
 
-def block_backward_bench(blk, w, x, cu, flush, steps=3):
+def block_backward_bench(blk, w, x, cu, flush, peaks, steps=3):
     """MoMBlock.backward after a forward on the same tokens (dy ~ N(0,1)):
     the output projection's and the gated norm's adjoints, the layer's
     reverse pass, the convolutions' adjoints and every weight's and the
@@ -199,7 +209,8 @@ def block_backward_bench(blk, w, x, cu, flush, steps=3):
     return {"workload": "backward of the %s block (all weight and token gradients), dy ~ N(0,1)" % w.name,
             "path": "output projection's adjoint on the tcgen05 tensor cores; gated norm and convolution adjoints "
                     "HBM-streamed; the layer's reverse pass as in layer_backward",
-            "ms": t, "value": w.n_tokens / (t / 1e3), "unit": UNIT}
+            "ms": t, "value": w.n_tokens / (t / 1e3), "unit": UNIT,
+            "roofline": backward_roofline(block_roofline(w, peaks, int(cu.numel()) - 1)[0], peaks, t)}
 
 
 def kernel_source_sha(name):
@@ -495,14 +506,14 @@ def gpu_arm(args):
             if on("block"):
                 configs["block"] = res
             if on("block_backward"):
-                configs["block_backward"] = block_backward_bench(*blk_run, flush)
+                configs["block_backward"] = block_backward_bench(*blk_run, flush, peaks)
             del blk_run
         if on("block_decode"):
             configs["block_decode"] = block_decode_bench(dev, args.warmup)
         if on("recurrence_backward"):
             configs["recurrence_backward"] = backward_bench(lay, w, x, cu, flush)
         if on("layer_backward"):
-            configs["layer_backward"] = layer_backward_bench(lay, w, x, cu, flush)
+            configs["layer_backward"] = layer_backward_bench(lay, w, x, cu, flush, peaks)
     clocks.__exit__(None, None, None)
     layer_roof["near_tie_tokens"] = near_tie_tokens(x, lay.w["w_r"], lay.w["b_r"], w.top_k)
     return finish(args, w, world, rank, value, ms_per_step, roof, layer_roof, per_call, e2e, launches, clocks, decode,
@@ -605,8 +616,8 @@ def backward_bench(lay, w, x, cu, flush, steps=3):
     probs = {"shared": (b["q"], None, b["k_sh"], b["v_sh"], cu), "routed": (b["q"], b["perm"], b["k_p"], b["v_p"],
                                                                           b["seg_cu"])}
     out = {"workload": "reverse pass of the %s layer's recurrences (shared + routed), dout ~ N(0,1)" % w.name,
-           "path": "token-serial float32 on CUDA cores (32 state rows per CTA, two CTAs per SM), states kept every 64 "
-                   "tokens, chunks re-walked keeping a copy every 4"}
+           "path": "token-serial float32 on CUDA cores (32 state rows per CTA, two CTAs per SM), states kept every 16 "
+                   "tokens, chunks re-walked keeping a copy every 2"}
     total = 0.0
     g = torch.Generator(device=x.device).manual_seed(1)
     for name, (q, qidx, k, v, seg) in probs.items():
@@ -641,7 +652,7 @@ def backward_bench(lay, w, x, cu, flush, steps=3):
     return out
 
 
-def layer_backward_bench(lay, w, x, cu, flush, steps=3):
+def layer_backward_bench(lay, w, x, cu, flush, peaks, steps=3):
     """MoMLayer.backward after a forward on the same tokens (dout ~ N(0,1)):
     every weight's and the tokens' gradients.  First path: the recurrences'
     reverse passes token-serial and the gradient GEMMs on CUDA cores, float32."""
@@ -668,7 +679,8 @@ def layer_backward_bench(lay, w, x, cu, flush, steps=3):
     return {"workload": "backward of the %s layer (all weight and token gradients), dout ~ N(0,1)" % w.name,
             "path": "recurrence reverse passes token-serial float32; gradient GEMMs on the tf32 tensor cores "
                     "(fp32 accumulation)",
-            "ms": t, "value": w.n_tokens / (t / 1e3), "unit": UNIT}
+            "ms": t, "value": w.n_tokens / (t / 1e3), "unit": UNIT,
+            "roofline": backward_roofline(layer_roofline(w, peaks, int(cu.numel()) - 1)[0], peaks, t)}
 
 
 def decode_bench(args, dev, world, rank, max_over_ranks, barrier):
