@@ -10,8 +10,10 @@ it; the plain Gated DeltaNet block is taken:
            -> output projection W_o
 
 Every step runs in the CUDA library (mom_block_proj, mom_short_conv, the
-recurrences, mom_combine_norm_gate, mom_linear); this module packs weights,
-holds buffers and passes pointers.  bf16 only.
+recurrences, mom_combine_norm_gate, mom_linear; the reverse pass adds
+mom_norm_gate_bwd, mom_short_conv_bwd, mom_convert and the layer's backward
+calls); this module packs weights, holds buffers and passes pointers.
+bf16 only.
 """
 from __future__ import annotations
 
