@@ -324,14 +324,26 @@ class MoMLayer:
         dh0_sh, dh0_m = g("dh0_sh", (n_seq, H, d, d)), g("dh0_m", (M, n_seq, H, d, d))
         ws_sh = self._ws("bwd_sh", B.mom_memory_chunk_bwd_workspace_size(n_tok, n_seq, H, d))
         ws_p = self._ws("bwd_p", B.mom_memory_chunk_bwd_workspace_size(R, M * n_seq, H, d))
+        # the two reverse passes side by side: the shared memory's (whole
+        # sequences, the longest chains) on the high-priority stream, so that
+        # its CTAs are dispatched first, the routed memories' filling the rest
+        hi, side = self._hi_stream(), self._side_stream()
+        fork = torch.cuda.Event()
+        fork.record(st)
+        hi.wait_event(fork)
+        side.wait_event(fork)
         B.mom_memory_chunk_bwd(b["q"], None, b["k_sh"], b["v_sh"], b["beta"], b["log_alpha"], cu_seqlens, self.scale,
                                self.rule, h0_shared, dout, dh_shared, dq_sh, dk_sh, dv_sh, db_sh, dla_sh, dh0_sh, ws_sh,
-                               stream=st)
+                               stream=hi)
         dhm = None if dh_mem is None else dh_mem.reshape(M * n_seq, H, d, d)
         h0m = None if h0_mem is None else h0_mem.reshape(M * n_seq, H, d, d)
         B.mom_memory_chunk_bwd(b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
                                self.scale, self.rule, h0m, do_p, dhm, dq_p, dk_p, dv_p, db_p, dla_p,
-                               dh0_m.view(M * n_seq, H, d, d), ws_p, stream=st)
+                               dh0_m.view(M * n_seq, H, d, d), ws_p, stream=side)
+        for s_ in (hi, side):
+            done = torch.cuda.Event()
+            done.record(s_)
+            st.wait_event(done)
         # per token: the shared memory's gradients plus those of its routed rows
         dq, dbeta, dla = g("dq", (n_tok, H, d)), g("dbeta", (n_tok, H)), g("dla", (n_tok, H))
         B.mom_rows_sum(dq_p.view(R, Hd), b["row_of"], K, dq_sh.view(n_tok, Hd), dq.view(n_tok, Hd), ws, stream=st)
@@ -354,6 +366,13 @@ class MoMLayer:
         if getattr(self, "_one_n", None) != n_tok:
             one.copy_(torch.tensor([0, n_tok], dtype=torch.int32))
             self._one_n = n_tok
+        # the weight gradients on the side stream beside the input gradient
+        # (both only read dz, dzr, dlogits, dala): their last waves fill each
+        # other's idle SMs
+        side = self._side_stream()
+        fork = torch.cuda.Event()
+        fork.record(st)
+        side.wait_event(fork)
         dx = g("dx", (n_tok, D))
         B.mom_gemm_grouped(0, dz, w_sh, dx, 0, D, n_sh, one, None, 1, ws, total_rows=n_tok, stream=st)
         B.mom_gemm_grouped(0, dz, w["w_gate"], dx, 0, D, 2 * H, one, None, 1, ws, a_col=n_sh, total_rows=n_tok,
@@ -366,15 +385,19 @@ class MoMLayer:
         B.mom_rows_sum(dx_rows, b["row_of"], K, dx, dx, ws, stream=st)
         dw_sh, dw_gate, dw_r = g("dw_sh", (n_sh, D)), g("dw_gate", (2 * H, D)), g("dw_r", (M, D))
         dw_kv = g("dw_kv", (M, 2 * Hd, D))
-        B.mom_gemm_grouped(1, dz, x, dw_sh, n_sh, D, 0, one, None, 1, ws, stream=st)
-        B.mom_gemm_grouped(1, dz, x, dw_gate, 2 * H, D, 0, one, None, 1, ws, a_col=n_sh, stream=st)
-        B.mom_gemm_grouped(1, dlogits, x, dw_r, M, D, 0, one, None, 1, ws, stream=st)
-        B.mom_gemm_grouped(1, dzr, x, dw_kv.view(M * 2 * Hd, D), 2 * Hd, D, 0, b["mem_offset"], None, M, ws,
-                           b_rows=b["perm"], c_group_stride=2 * Hd * D, stream=st)
+        ws_w = self._ws("bwd_w", B.MOM_WS_HEADER_BYTES)
+        B.mom_gemm_grouped(1, dz, x, dw_sh, n_sh, D, 0, one, None, 1, ws_w, stream=side)
+        B.mom_gemm_grouped(1, dz, x, dw_gate, 2 * H, D, 0, one, None, 1, ws_w, a_col=n_sh, stream=side)
+        B.mom_gemm_grouped(1, dlogits, x, dw_r, M, D, 0, one, None, 1, ws_w, stream=side)
+        B.mom_gemm_grouped(1, dzr, x, dw_kv.view(M * 2 * Hd, D), 2 * Hd, D, 0, b["mem_offset"], None, M, ws_w,
+                           b_rows=b["perm"], c_group_stride=2 * Hd * D, stream=side)
         db_r, dA, db_a = g("db_r", (M,)), g("dA", (H,)), g("db_a", (H,))
-        B.mom_col_sums(dlogits, db_r, stream=st)
-        B.mom_col_sums(dala, dA, stream=st)
-        B.mom_col_sums(dz, db_a, col0=n_sh + H, stream=st)
+        B.mom_col_sums(dlogits, db_r, stream=side)
+        B.mom_col_sums(dala, dA, stream=side)
+        B.mom_col_sums(dz, db_a, col0=n_sh + H, stream=side)
+        done = torch.cuda.Event()
+        done.record(side)
+        st.wait_event(done)
         return dict(dx=dx, dw_sh=dw_sh, dw_gate=dw_gate, dw_r=dw_r, dw_kv=dw_kv, db_r=db_r, dA=dA, db_a=db_a)
 
     # --------------------------------------------------------------- decode
