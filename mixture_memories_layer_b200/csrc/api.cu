@@ -865,7 +865,7 @@ mom_status mom_norm_gate_bwd(const void* o_sh, const void* o_p, const int32_t* r
     if (!dt_ok(dt) || n_tok < 0 || top_k < 0 || H < 1 || H > MOM_MAX_HEADS || !(eps >= 0.f)) return MOM_ERR_ARG;
     if (d < 8 || d > 256 || (d & (d - 1)) != 0 || ldg < (int64_t)H * d) return MOM_ERR_ARG;
     if (dt != MOM_BF16) return MOM_ERR_UNSUPPORTED;
-    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES || !dw_norm || !al16(w_norm)) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES || !dw_norm || !w_norm || !al16(w_norm)) return MOM_ERR_ARG;
     const void* ptrs[] = {o_sh, g, d_y, d_o, dg};
     for (const void* p : ptrs)
         if (!p || !al16(p)) return MOM_ERR_ARG;

@@ -114,3 +114,47 @@ def test_block_calls_validate_on_the_host(lib):
     assert s == B.MOM_ERR_ARG                                                 # workspace too small
     s = L.mom_block_proj(*([fake] * 5), B.MOM_BF16, 10, 256, 2, 96, 4, 2, *([fake] * 6), fake, 4096, None)
     assert s == B.MOM_ERR_UNSUPPORTED                                         # d = 96
+
+
+def test_block_backward_calls_validate_on_the_host(lib):
+    """The block's reverse-pass calls refuse bad shapes and pointers before
+    any launch."""
+    L, B = lib.lib, lib
+    fake, odd = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10004)
+    ng = lambda o_p=fake, w_norm=fake, eps=1e-5, top_k=2, d=64, dt=B.MOM_BF16, dg=fake, ldg=128, ws_bytes=4096: \
+        L.mom_norm_gate_bwd(fake, o_p, fake, fake, fake, w_norm, eps, fake, 10, top_k, 2, d, dt, fake, dg, ldg,
+                            fake, fake, ws_bytes, None)
+    assert ng(d=96) == B.MOM_ERR_ARG                                          # d not a power of two
+    assert ng(eps=-1.0) == B.MOM_ERR_ARG
+    assert ng(ldg=100) == B.MOM_ERR_ARG                                       # ldg < H d
+    assert ng(ldg=130) == B.MOM_ERR_ARG                                       # rows not 16-byte aligned
+    assert ng(dt=B.MOM_F32) == B.MOM_ERR_UNSUPPORTED
+    assert ng(w_norm=None) == B.MOM_ERR_ARG
+    assert ng(dg=odd) == B.MOM_ERR_ARG
+    assert ng(o_p=None) == B.MOM_ERR_ARG                                      # routed rows missing, top_k 2
+    assert ng(ws_bytes=8) == B.MOM_ERR_ARG
+
+    def conv(**kw):
+        q = dict(z=fake.value, dout=fake.value, da=fake.value, dz=fake.value, ldz=256, col0=0, n_rows=10,
+                 seg_cu=fake.value, n_seg=2, seg_per_group=1, n_groups=2, w=fake.value, dw=fake.value, l2norm=1)
+        channels = kw.pop("channels", 256)
+        width = kw.pop("width", 4)
+        head_dim = kw.pop("head_dim", 64)
+        n = kw.pop("n", 1)
+        q.update(kw)
+        arr = (B.MomConvBwdProblem * 9)(*[B.MomConvBwdProblem(**q)] * 9)
+        return L.mom_short_conv_bwd(arr, n, channels, width, head_dim, B.MOM_BF16, fake, 4096, None)
+    assert conv(width=5) == B.MOM_ERR_UNSUPPORTED
+    assert conv(n=9) == B.MOM_ERR_UNSUPPORTED                                 # more than 8 problems
+    assert conv(n=0) == B.MOM_ERR_ARG
+    assert conv(channels=252) == B.MOM_ERR_ARG                                # channels % 8
+    assert conv(head_dim=96) == B.MOM_ERR_ARG                                 # with the L2 norm
+    assert conv(ldz=200) == B.MOM_ERR_ARG                                     # ldz < col0 + channels
+    assert conv(col0=2, ldz=260) == B.MOM_ERR_ARG                             # col0 not 16-byte aligned
+    assert conv(seg_per_group=0) == B.MOM_ERR_ARG
+    assert conv(l2norm=2) == B.MOM_ERR_ARG
+    assert conv(dz=0) == B.MOM_ERR_ARG
+    assert conv(w=odd.value) == B.MOM_ERR_ARG
+    assert L.mom_convert(fake, B.MOM_F32, fake, B.MOM_BF16, -1, None) == B.MOM_ERR_ARG
+    assert L.mom_convert(fake, B.MOM_F32, fake, B.MOM_BF16, 0, None) == B.MOM_OK  # nothing to do
+    assert L.mom_convert(None, B.MOM_F32, fake, B.MOM_BF16, 5, None) == B.MOM_ERR_ARG
