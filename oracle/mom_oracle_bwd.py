@@ -236,7 +236,11 @@ def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: floa
 
     Returns a dict: dx, dw_r, db_r, dw_q, dw_k_sh, dw_v_sh, dw_beta, dw_a,
     dA, db_a, dw_k [M,..], dw_v [M,..], dh0_shared [S,..], dh0_mem [M,S,..],
-    and the forward's own results under "fwd".
+    and the forward's own results under "fwd".  With per-memory gates
+    (mom_oracle.memory_gates: each memory's routed rows take that memory's
+    beta and alpha) also dw_beta_mem, dw_a_mem [M,H,d_model], dA_mem,
+    db_a_mem [M,H]; the shared gates then carry the shared memory's
+    adjoints alone.
     """
     x = np.asarray(x, F64)
     dout = np.asarray(dout, F64)
@@ -249,6 +253,10 @@ def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: floa
     f = fwd.mom_forward(x, p, cu, top_k, H, d, scale, forced_idx=forced_idx,
                         h0_shared=h0_shared, h0_mem=h0_mem)
     idx, gate = f["idx"], f["gate"]
+    mem_gates = fwd.has_memory_gates(p)
+    if mem_gates:
+        WM = {name: np.asarray(p[name], F64) for name in ("w_beta_mem", "w_a_mem", "A_mem", "b_a_mem")}
+        gm = {"d" + name: np.zeros_like(arr) for name, arr in WM.items()}
 
     # combine: out = o_shared + sum_j gate_j o_mem[:, j]
     dgate = np.einsum("nhd,njhd->nj", dout, f["o_mem"])
@@ -293,11 +301,27 @@ def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: floa
             k_m = fwd.l2norm(z_k)
             v_m = (x[rows] @ W["w_v"][m].T).reshape(len(rows), H, d)
             h0 = None if h0_mem is None else h0_mem[m, s]
-            r = gdn_recurrence_bwd(f["q"][rows], k_m, v_m, f["beta"][rows], f["log_alpha"][rows],
-                                   g[:, None, None] * dout[rows], h0, dhf, scale)
+            if mem_gates:
+                b_m, la_m = fwd.memory_gates(x[rows], p, m)
+            else:
+                b_m, la_m = f["beta"][rows], f["log_alpha"][rows]
+            r = gdn_recurrence_bwd(f["q"][rows], k_m, v_m, b_m, la_m, g[:, None, None] * dout[rows], h0, dhf,
+                                   scale)
             dq[rows] += r["dq"]
-            dbeta[rows] += r["dbeta"]
-            dlog_alpha[rows] += r["dlog_alpha"]
+            if mem_gates:
+                # memory m's own gates: beta = sigmoid(x W_beta^m^T), log alpha =
+                # -exp(A^m) softplus(x W_a^m^T + b_a^m)
+                dzb = r["dbeta"] * b_m * (1.0 - b_m)
+                za = x[rows] @ WM["w_a_mem"][m].T + WM["b_a_mem"][m]
+                dza = r["dlog_alpha"] * (-np.exp(WM["A_mem"][m])) * fwd.sigmoid(za)
+                gm["dw_beta_mem"][m] += dzb.T @ x[rows]
+                gm["dw_a_mem"][m] += dza.T @ x[rows]
+                gm["dA_mem"][m] += np.sum(r["dlog_alpha"] * la_m, axis=0)
+                gm["db_a_mem"][m] += dza.sum(axis=0)
+                dx[rows] += dzb @ WM["w_beta_mem"][m] + dza @ WM["w_a_mem"][m]
+            else:
+                dbeta[rows] += r["dbeta"]
+                dlog_alpha[rows] += r["dlog_alpha"]
             dh0_mem[m, s] = r["dh0"]
             # memory m's projections of its rows
             dz_k = l2norm_bwd(z_k, r["dk"]).reshape(len(rows), H * d)
@@ -326,6 +350,9 @@ def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: floa
     dA = np.sum(dlog_alpha * f["log_alpha"], axis=0)
     db_a = dz_a.sum(axis=0)
     dx += dz_q @ W["w_q"] + dz_k @ W["w_k_sh"] + dz_v @ W["w_v_sh"] + dz_beta @ W["w_beta"] + dz_a @ W["w_a"]
-    return dict(dx=dx, dw_r=dw_r, db_r=db_r, dw_q=dz_q.T @ x, dw_k_sh=dz_k.T @ x, dw_v_sh=dz_v.T @ x,
-                dw_beta=dz_beta.T @ x, dw_a=dz_a.T @ x, dA=dA, db_a=db_a, dw_k=dw_k, dw_v=dw_v,
-                dh0_shared=dh0_shared, dh0_mem=dh0_mem, fwd=f)
+    out = dict(dx=dx, dw_r=dw_r, db_r=db_r, dw_q=dz_q.T @ x, dw_k_sh=dz_k.T @ x, dw_v_sh=dz_v.T @ x,
+               dw_beta=dz_beta.T @ x, dw_a=dz_a.T @ x, dA=dA, db_a=db_a, dw_k=dw_k, dw_v=dw_v,
+               dh0_shared=dh0_shared, dh0_mem=dh0_mem, fwd=f)
+    if mem_gates:
+        out.update(gm)
+    return out

@@ -94,8 +94,8 @@ def test_gdn_chunked_bwd_equals_token_loop(chunk, with_states):
         assert _rel(got[key], ref[key]) < 1e-12, (key, chunk)
 
 
-def _layer_case(lens=(4, 0, 3), D=5, H=2, d=3, M=3, k=2, seed=1):
-    w = synth.Workload("bwd_tiny", 0, 0, D, H, d, M, k, "f32", seed=seed)
+def _layer_case(lens=(4, 0, 3), D=5, H=2, d=3, M=3, k=2, seed=1, mem_gates=False):
+    w = synth.Workload("bwd_tiny", 0, 0, D, H, d, M, k, "f32", seed=seed, mem_gates=mem_gates)
     rng = np.random.default_rng(seed)
     p = {key: np.array(val, np.float64) for key, val in synth.make_weights(w, rng).items()}
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
@@ -125,6 +125,29 @@ def test_mom_backward_matches_finite_differences():
     checks = [("dx", x)] + [("d" + name, p[name]) for name in
                             ("w_r", "b_r", "w_q", "w_k_sh", "w_v_sh", "w_beta", "w_a", "A", "b_a", "w_k", "w_v")]
     checks += [("dh0_shared", h0s), ("dh0_mem", h0m)]
+    for key, arr in checks:
+        e = _rel(g[key], _fd(loss, arr))
+        assert e < 1e-6, (key, e)
+
+
+def test_mom_backward_with_per_memory_gates_matches_finite_differences():
+    """Per-memory gates ("MoM", Summary: each memory its own parameters; the
+    gates' placement is a reading): every gradient, the memories' own gate
+    weights included, against central differences of the forward."""
+    w, p, cu, x, adj, h0s, h0m = _layer_case(seed=4, mem_gates=True)
+    H, d, K = w.heads, w.d_head, w.top_k
+    idx = fwd.router_topk(x, p["w_r"], p["b_r"], K)[0]
+
+    def loss():
+        f = fwd.mom_forward(x, p, cu, K, H, d, 1.0, forced_idx=idx, h0_shared=h0s, h0_mem=h0m)
+        return float(np.sum(adj["dout"] * f["out"]) + np.sum(adj["dhs"] * f["h_shared"])
+                     + np.sum(adj["dhm"] * f["h_mem"]))
+
+    g = bwd.mom_backward(x, p, cu, K, H, d, adj["dout"], 1.0, forced_idx=idx, h0_shared=h0s, h0_mem=h0m,
+                         dh_shared=adj["dhs"], dh_mem=adj["dhm"])
+    checks = [("dx", x)] + [("d" + name, p[name]) for name in
+                            ("w_beta", "w_a", "A", "b_a", "w_k", "w_v", "w_q", "w_beta_mem", "w_a_mem", "A_mem",
+                             "b_a_mem")]
     for key, arr in checks:
         e = _rel(g[key], _fd(loss, arr))
         assert e < 1e-6, (key, e)
