@@ -462,6 +462,21 @@ mom_status mom_gates_bwd(const float* beta, const float* log_alpha, const float*
 /* mom_col_sums -- out[c] = sum_r a[r*lda + c], c < cols (float32). */
 mom_status mom_col_sums(const float* a, int64_t rows, int64_t lda, int64_t cols, float* out, void* stream);
 
+/* mom_gates_bwd_by_group -- mom_gates_bwd for rows in groups with their own
+ * A: group g covers rows group_offset[g] .. group_offset[g+1]-1 (device
+ * array, n_groups + 1 entries, non-decreasing, covering 0 .. n) and its rows
+ * take A[g*H + h] (the per-memory gates' A_mem [M, H] over the reordered
+ * rows, group g = memory g). */
+mom_status mom_gates_bwd_by_group(const float* beta, const float* log_alpha, const float* dbeta, const float* dlog_alpha,
+                                  const float* A, const int32_t* group_offset, int n_groups, int64_t n, int H, float* dz,
+                                  int64_t ldz, int64_t col_b, int64_t col_a, float* dala, void* stream);
+
+/* mom_col_sums_grouped -- out[g*cols + c] = sum over the rows r of group g
+ * (group_offset as above, clipped to 0 .. rows) of a[r*lda + c] (float32):
+ * the per-memory gates' dA and db_a. */
+mom_status mom_col_sums_grouped(const float* a, int64_t rows, int64_t lda, int64_t cols, const int32_t* group_offset,
+                                int n_groups, float* out, void* stream);
+
 /* mom_gemm_grouped -- float32 C (+)= op(A) B over groups of rows, for the
  * projections' input and weight gradients.  A float32, B (dt), C float32,
  * row-major with leading dimensions lda, ldb, ldc (elements):

@@ -70,6 +70,8 @@ SIGNATURES = {
     "mom_l2norm_bwd": (_I, [_VP, _VP, _VP, _I64, _I, _I, _I, _VP, _I64, _I64, _VP]),
     "mom_gates_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _I, _VP, _I64, _I64, _I64, _VP, _VP]),
     "mom_col_sums": (_I, [_VP, _I64, _I64, _I64, _VP, _VP]),
+    "mom_gates_bwd_by_group": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _VP, _I64, _I64, _I64, _VP, _VP]),
+    "mom_col_sums_grouped": (_I, [_VP, _I64, _I64, _I64, _VP, _I, _VP, _VP]),
     "mom_gemm_grouped": (_I, [_I, _VP, _I64, _VP, _I64, _I, _VP, _I64, _VP, _I64, _I64, _I64, _I64, _I64, _VP, _VP,
                               _I, _I64, _I64, _I, _VP, _SZ, _VP]),
     "mom_memory_chunk_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I64, _I, _I, _F, _I, _I, _I,
@@ -405,6 +407,23 @@ def mom_gates_bwd(beta, log_alpha, dbeta, dlog_alpha, A, dz, col_b, col_a, dala,
     n, H = beta.shape
     _check(lib.mom_gates_bwd(_p(beta), _p(log_alpha), _p(dbeta), _p(dlog_alpha), _p(A), n, H, _p(dz), dz.shape[1],
                              col_b, col_a, _p(dala), _s(stream)), "mom_gates_bwd")
+
+
+def mom_gates_bwd_by_group(beta, log_alpha, dbeta, dlog_alpha, A, group_offset, dz, col_b, col_a, dala,
+                           stream=None):
+    """mom_gates_bwd with A [n_groups, H] taken per row group."""
+    n, H = beta.shape
+    _check(lib.mom_gates_bwd_by_group(_p(beta), _p(log_alpha), _p(dbeta), _p(dlog_alpha), _p(A), _p(group_offset),
+                                      group_offset.numel() - 1, n, H, _p(dz), dz.shape[1], col_b, col_a, _p(dala),
+                                      _s(stream)), "mom_gates_bwd_by_group")
+
+
+def mom_col_sums_grouped(a, group_offset, out, col0=0, cols=None, stream=None):
+    """out [n_groups, cols]: per row group, the sums of a's columns col0 ..."""
+    rows, lda = a.shape
+    cols = out.shape[-1] if cols is None else cols
+    _check(lib.mom_col_sums_grouped(_pa(a, col0), rows, lda, cols, _p(group_offset), group_offset.numel() - 1,
+                                    _p(out), _s(stream)), "mom_col_sums_grouped")
 
 
 def mom_col_sums(a, out, col0=0, stream=None):

@@ -468,15 +468,36 @@ mom_status mom_gates_bwd(const float* beta, const float* log_alpha, const float*
     const void* ptrs[] = {beta, log_alpha, dbeta, dlog_alpha, A, dz, dala};
     for (const void* p : ptrs)
         if (!p) return MOM_ERR_ARG;
-    return cuda_status(launch_gates_bwd(beta, log_alpha, dbeta, dlog_alpha, A, n, H, dz, ldz, col_b, col_a, dala,
-                                        as_stream(stream)));
+    return cuda_status(launch_gates_bwd(beta, log_alpha, dbeta, dlog_alpha, A, nullptr, 1, n, H, dz, ldz, col_b,
+                                        col_a, dala, as_stream(stream)));
+}
+
+mom_status mom_gates_bwd_by_group(const float* beta, const float* log_alpha, const float* dbeta, const float* dlog_alpha,
+                                  const float* A, const int32_t* group_offset, int n_groups, int64_t n, int H, float* dz,
+                                  int64_t ldz, int64_t col_b, int64_t col_a, float* dala, void* stream) {
+    if (n < 0 || H < 1 || n_groups < 1 || col_b < 0 || col_a < 0 || ldz < col_b + H || ldz < col_a + H)
+        return MOM_ERR_ARG;
+    if (n == 0) return MOM_OK;
+    const void* ptrs[] = {beta, log_alpha, dbeta, dlog_alpha, A, group_offset, dz, dala};
+    for (const void* p : ptrs)
+        if (!p) return MOM_ERR_ARG;
+    return cuda_status(launch_gates_bwd(beta, log_alpha, dbeta, dlog_alpha, A, group_offset, n_groups, n, H, dz, ldz,
+                                        col_b, col_a, dala, as_stream(stream)));
 }
 
 mom_status mom_col_sums(const float* a, int64_t rows, int64_t lda, int64_t cols, float* out, void* stream) {
     if (rows < 0 || cols < 0 || lda < cols) return MOM_ERR_ARG;
     if (cols == 0) return MOM_OK;
     if (!out || (rows > 0 && !a)) return MOM_ERR_ARG;
-    return cuda_status(launch_col_sums(a, rows, lda, cols, out, as_stream(stream)));
+    return cuda_status(launch_col_sums(a, rows, lda, cols, nullptr, 1, out, as_stream(stream)));
+}
+
+mom_status mom_col_sums_grouped(const float* a, int64_t rows, int64_t lda, int64_t cols, const int32_t* group_offset,
+                                int n_groups, float* out, void* stream) {
+    if (rows < 0 || cols < 0 || lda < cols || n_groups < 1) return MOM_ERR_ARG;
+    if (cols == 0) return MOM_OK;
+    if (!out || !group_offset || (rows > 0 && !a)) return MOM_ERR_ARG;
+    return cuda_status(launch_col_sums(a, rows, lda, cols, group_offset, n_groups, out, as_stream(stream)));
 }
 
 mom_status mom_gemm_grouped(int trans_a, const float* A, int64_t lda, const void* B, int64_t ldb, mom_dtype dt,

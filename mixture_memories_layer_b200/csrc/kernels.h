@@ -171,9 +171,10 @@ cudaError_t launch_rows_sum(const float* src, int64_t n_src, const int32_t* row_
 cudaError_t launch_l2norm_bwd(const void* y, const float* dy, const float* nrm, int64_t rows, int H, int d, int dt,
                               float* dz, int64_t ldz, int64_t col0, cudaStream_t st);
 cudaError_t launch_gates_bwd(const float* beta, const float* la, const float* dbeta, const float* dla, const float* A,
-                             int64_t n, int H, float* dz, int64_t ldz, int64_t col_b, int64_t col_a, float* dala,
-                             cudaStream_t st);
-cudaError_t launch_col_sums(const float* a, int64_t rows, int64_t lda, int64_t C, float* out, cudaStream_t st);
+                             const int32_t* goff, int n_groups, int64_t n, int H, float* dz, int64_t ldz,
+                             int64_t col_b, int64_t col_a, float* dala, cudaStream_t st);
+cudaError_t launch_col_sums(const float* a, int64_t rows, int64_t lda, int64_t C, const int32_t* goff, int n_groups,
+                            float* out, cudaStream_t st);
 cudaError_t launch_gemm_grouped(int trans_a, const float* A, int64_t lda, const void* B, int64_t ldb, int dt,
                                 const int32_t* b_rows, int64_t n_b_rows, float* C, int64_t ldc, int64_t M, int64_t N,
                                 int64_t K, int64_t total_rows, const int32_t* goff, const int32_t* gmem, int n_groups,

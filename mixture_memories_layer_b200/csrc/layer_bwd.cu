@@ -104,15 +104,28 @@ l2norm_bwd_kernel(const T* __restrict__ y, const float* __restrict__ dy, const f
 // beta = sigmoid(z_b): dz_b = dbeta beta (1 - beta).
 // log alpha = -e^A softplus(z_a): dz_a = dla (-e^A) sigmoid(z_a), with
 // sigmoid(z_a) = 1 - e^(-softplus(z_a)) and softplus(z_a) = -log alpha e^-A;
-// dala = dla log alpha (summed over tokens: dA).
+// dala = dla log alpha (summed over tokens: dA).  With a group table (goff,
+// n_groups: the rows of group g are goff[g] .. goff[g+1]-1) row r takes the
+// A of its group, A[g * H + h] (per-memory gates of the reordered rows).
+__device__ __forceinline__ int group_of(const int32_t* goff, int n_groups, int64_t r) {
+    int lo = 0, hi = n_groups;                       // the last g with goff[g] <= r
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(goff + mid) <= r) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
 __global__ void __launch_bounds__(256)
 gates_bwd_kernel(const float* __restrict__ beta, const float* __restrict__ la, const float* __restrict__ dbeta,
-                 const float* __restrict__ dla, const float* __restrict__ A, int64_t n, int H, float* __restrict__ dz,
-                 int64_t ldz, int64_t col_b, int64_t col_a, float* __restrict__ dala) {
+                 const float* __restrict__ dla, const float* __restrict__ A, const int32_t* __restrict__ goff,
+                 int n_groups, int64_t n, int H, float* __restrict__ dz, int64_t ldz, int64_t col_b, int64_t col_a,
+                 float* __restrict__ dala) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n * H; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = i / H;
         const int h = (int)(i - r * H);
-        const float b = beta[i], l = la[i], eA = expf(A[h]);
+        const int g = goff ? group_of(goff, n_groups, r) : 0;
+        const float b = beta[i], l = la[i], eA = expf(A[(int64_t)g * H + h]);
         dz[r * ldz + col_b + h] = dbeta[i] * b * (1.f - b);
         const float sp = -l / eA;
         const float sg = -expm1f(-sp);                  // 1 - e^-sp
@@ -121,16 +134,28 @@ gates_bwd_kernel(const float* __restrict__ beta, const float* __restrict__ la, c
     }
 }
 
-// out[c] = sum_r a[r * lda + c], c < C: one warp per column, lanes over rows.
+// out[g * C + c] = sum over the rows r of group g of a[r * lda + c], c < C:
+// one warp per (group, column), lanes over rows.  No group table: one group
+// of rows 0 .. rows-1.
 __global__ void __launch_bounds__(256)
-col_sums_kernel(const float* __restrict__ a, int64_t rows, int64_t lda, int64_t C, float* __restrict__ out) {
+col_sums_kernel(const float* __restrict__ a, int64_t rows, int64_t lda, int64_t C, const int32_t* __restrict__ goff,
+                int n_groups, float* __restrict__ out) {
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t c = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); c < C; c += warps) {
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < (int64_t)n_groups * C;
+         w += warps) {
+        const int64_t g = w / C, c = w - g * C;
+        int64_t lo = 0, hi = rows;
+        if (goff) {
+            lo = __ldg(goff + g);
+            hi = __ldg(goff + g + 1);
+            if (lo < 0) lo = 0;
+            if (hi > rows) hi = rows;
+        }
         float acc = 0.f;
-        for (int64_t r = lane; r < rows; r += 32) acc += a[r * lda + c];
+        for (int64_t r = lo + lane; r < hi; r += 32) acc += a[r * lda + c];
         acc = warp_sum(acc);
-        if (lane == 0) out[c] = acc;
+        if (lane == 0) out[w] = acc;
     }
 }
 
@@ -535,17 +560,19 @@ cudaError_t launch_l2norm_bwd(const void* y, const float* dy, const float* nrm, 
 }
 
 cudaError_t launch_gates_bwd(const float* beta, const float* la, const float* dbeta, const float* dla, const float* A,
-                             int64_t n, int H, float* dz, int64_t ldz, int64_t col_b, int64_t col_a, float* dala,
-                             cudaStream_t st) {
+                             const int32_t* goff, int n_groups, int64_t n, int H, float* dz, int64_t ldz,
+                             int64_t col_b, int64_t col_a, float* dala, cudaStream_t st) {
     if (n == 0) return cudaSuccess;
-    gates_bwd_kernel<<<grid_rows(n * H, 256), 256, 0, st>>>(beta, la, dbeta, dla, A, n, H, dz, ldz, col_b, col_a, dala);
+    gates_bwd_kernel<<<grid_rows(n * H, 256), 256, 0, st>>>(beta, la, dbeta, dla, A, goff, n_groups, n, H, dz, ldz,
+                                                            col_b, col_a, dala);
     count_launches(1);
     return cudaGetLastError();
 }
 
-cudaError_t launch_col_sums(const float* a, int64_t rows, int64_t lda, int64_t C, float* out, cudaStream_t st) {
-    if (C == 0) return cudaSuccess;
-    col_sums_kernel<<<grid_rows(C, 8), 256, 0, st>>>(a, rows, lda, C, out);
+cudaError_t launch_col_sums(const float* a, int64_t rows, int64_t lda, int64_t C, const int32_t* goff, int n_groups,
+                            float* out, cudaStream_t st) {
+    if (C == 0 || n_groups == 0) return cudaSuccess;
+    col_sums_kernel<<<grid_rows((int64_t)n_groups * C, 8), 256, 0, st>>>(a, rows, lda, C, goff, n_groups, out);
     count_launches(1);
     return cudaGetLastError();
 }

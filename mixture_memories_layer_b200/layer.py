@@ -255,11 +255,12 @@ class MoMLayer:
         are read): dx, dw_r, db_r, dw_shared [3Hd, D] (W_q | W_k_sh | W_v_sh),
         dw_gate [2H, D] (W_beta | W_a), dA, db_a, dw_kv [M, 2Hd, D], dh0_shared
         [S, H, d, d], dh0_mem [M, S, H, d, d]; all float32.  The routing is
-        held fixed; gradients flow through the renormalised gates.  Every step
-        runs in the CUDA library (the recurrences' reverse passes, then the
-        combine, router, norm and gate adjoints and the projections' GEMMs)."""
-        if self.mem_gates:
-            raise NotImplementedError("the backward of per-memory gates is not provided")
+        held fixed; gradients flow through the renormalised gates.  With
+        per-memory gates also dw_gate_mem [M, 2H, D] (W_beta^m | W_a^m),
+        dA_mem, db_a_mem [M, H], and dw_gate, dA, db_a carry the shared
+        memory's adjoints alone.  Every step runs in the CUDA library (the
+        recurrences' reverse passes, then the combine, router, norm and gate
+        adjoints and the projections' GEMMs)."""
         n_tok, D = x.shape
         n_seq = cu_seqlens.numel() - 1
         H, d, K, dt = self.H, self.d, self.top_k, self.dtype
@@ -288,9 +289,24 @@ class MoMLayer:
         dzr = g("dzr", (R, 2 * Hd))
         B.mom_l2norm_bwd(b["k_p"], c["dk_p"], kpn, dzr, 0, stream=st)
         B.mom_copy_rows(c["dv_p"].view(R, Hd), None, dzr, Hd * 4, src_off=0, dst_off=Hd * 4, ws=ws, stream=st)
-        r = self._proj_bwd(x, b, dz, 3 * Hd, w["w_shared"], dzr, c["dlogits"], dala, st, ws)
-        return dict(dx=r["dx"], dw_r=r["dw_r"], db_r=r["db_r"], dw_shared=r["dw_sh"], dw_gate=r["dw_gate"],
-                    dA=r["dA"], db_a=r["db_a"], dw_kv=r["dw_kv"], dh0_shared=c["dh0_shared"], dh0_mem=c["dh0_mem"])
+        mg = self._mem_gates_bwd(b, c, st)
+        r = self._proj_bwd(x, b, dz, 3 * Hd, w["w_shared"], dzr, c["dlogits"], dala, st, ws, mg)
+        out = dict(dx=r["dx"], dw_r=r["dw_r"], db_r=r["db_r"], dw_shared=r["dw_sh"], dw_gate=r["dw_gate"],
+                   dA=r["dA"], db_a=r["db_a"], dw_kv=r["dw_kv"], dh0_shared=c["dh0_shared"], dh0_mem=c["dh0_mem"])
+        out.update({k_: r[k_] for k_ in ("dw_gate_mem", "dA_mem", "db_a_mem") if k_ in r})
+        return out
+
+    def _mem_gates_bwd(self, b, c, st):
+        """With per-memory gates: the routed rows' gate adjoints under their
+        memory's A (pre-activation gradients [N*K, 2H]: beta | a) and
+        dla * log alpha per row; None without them."""
+        if not self.mem_gates:
+            return None
+        R, H = c["db_p"].shape
+        dzg, dala_p = self._bwd_buf("dzg", (R, 2 * H)), self._bwd_buf("dala_p", (R, H))
+        B.mom_gates_bwd_by_group(b["beta_p"], b["log_alpha_p"], c["db_p"], c["dla_p"], self.w["A_mem"],
+                                 b["mem_offset"], dzg, 0, H, dala_p, stream=st)
+        return dict(dzg=dzg, dala_p=dala_p)
 
     def _bwd_buf(self, name, shape, dtype=torch.float32):
         return self._buf("bwd_" + name, shape, dtype)
@@ -337,27 +353,38 @@ class MoMLayer:
                                stream=hi)
         dhm = None if dh_mem is None else dh_mem.reshape(M * n_seq, H, d, d)
         h0m = None if h0_mem is None else h0_mem.reshape(M * n_seq, H, d, d)
-        B.mom_memory_chunk_bwd(b["q"], b["perm"], b["k_p"], b["v_p"], b["beta"], b["log_alpha"], b["seg_cu"],
+        if self.mem_gates:
+            gates_p = (b["beta_p"], b["log_alpha_p"], B.MOM_GATES_BY_ROW)
+        else:
+            gates_p = (b["beta"], b["log_alpha"], B.MOM_GATES_BY_TOKEN)
+        B.mom_memory_chunk_bwd(b["q"], b["perm"], b["k_p"], b["v_p"], gates_p[0], gates_p[1], b["seg_cu"],
                                self.scale, self.rule, h0m, do_p, dhm, dq_p, dk_p, dv_p, db_p, dla_p,
-                               dh0_m.view(M * n_seq, H, d, d), ws_p, stream=side)
+                               dh0_m.view(M * n_seq, H, d, d), ws_p, stream=side, gates=gates_p[2])
         for s_ in (hi, side):
             done = torch.cuda.Event()
             done.record(s_)
             st.wait_event(done)
         # per token: the shared memory's gradients plus those of its routed rows
-        dq, dbeta, dla = g("dq", (n_tok, H, d)), g("dbeta", (n_tok, H)), g("dla", (n_tok, H))
+        # (with per-memory gates the routed rows' gate adjoints stay per row)
+        dq = g("dq", (n_tok, H, d))
         B.mom_rows_sum(dq_p.view(R, Hd), b["row_of"], K, dq_sh.view(n_tok, Hd), dq.view(n_tok, Hd), ws, stream=st)
-        B.mom_rows_sum(db_p, b["row_of"], K, db_sh, dbeta, ws, stream=st)
-        B.mom_rows_sum(dla_p, b["row_of"], K, dla_sh, dla, ws, stream=st)
+        if self.mem_gates:
+            dbeta, dla = db_sh, dla_sh
+        else:
+            dbeta, dla = g("dbeta", (n_tok, H)), g("dla", (n_tok, H))
+            B.mom_rows_sum(db_p, b["row_of"], K, db_sh, dbeta, ws, stream=st)
+            B.mom_rows_sum(dla_p, b["row_of"], K, dla_sh, dla, ws, stream=st)
         return dict(dq=dq, dk_sh=dk_sh, dv_sh=dv_sh, dk_p=dk_p, dv_p=dv_p, dbeta=dbeta, dla=dla, dlogits=dlogits,
-                    dh0_shared=dh0_sh, dh0_mem=dh0_m)
+                    dh0_shared=dh0_sh, dh0_mem=dh0_m, db_p=db_p, dla_p=dla_p)
 
-    def _proj_bwd(self, x, b, dz, n_sh, w_sh, dzr, dlogits, dala, st, ws):
+    def _proj_bwd(self, x, b, dz, n_sh, w_sh, dzr, dlogits, dala, st, ws, mg=None):
         """The projections' input and weight gradients from the pre-activation
         gradients: dz [N, ldz] float32 holds n_sh columns against w_sh [n_sh,
         D] then beta | a (2H) against w_gate; dzr [N*K, 2Hd] the routed rows'
-        against w_kv; dlogits [N, M] against w_r.  Returns dx, dw_sh, dw_gate,
-        dw_r, dw_kv, db_r, dA, db_a (float32)."""
+        against w_kv; dlogits [N, M] against w_r; with per-memory gates (mg:
+        _mem_gates_bwd's) the routed rows' gate gradients against w_gate_mem.
+        Returns dx, dw_sh, dw_gate, dw_r, dw_kv, db_r, dA, db_a (float32), and
+        dw_gate_mem, dA_mem, db_a_mem with mg."""
         n_tok, D = x.shape
         H, Hd, K, M = self.H, self.H * self.d, self.top_k, self.n_mem
         R = n_tok * K
@@ -382,6 +409,9 @@ class MoMLayer:
         dx_rows = g("dx_rows", (R, D))
         B.mom_gemm_grouped(0, dzr, w["w_kv"], dx_rows, 0, D, 2 * Hd, b["mem_offset"], None, M, ws, total_rows=R,
                            b_group_stride=2 * Hd * D, stream=st)
+        if mg is not None:
+            B.mom_gemm_grouped(0, mg["dzg"], w["w_gate_mem"], dx_rows, 0, D, 2 * H, b["mem_offset"], None, M, ws,
+                               total_rows=R, b_group_stride=2 * H * D, accumulate=True, stream=st)
         B.mom_rows_sum(dx_rows, b["row_of"], K, dx, dx, ws, stream=st)
         dw_sh, dw_gate, dw_r = g("dw_sh", (n_sh, D)), g("dw_gate", (2 * H, D)), g("dw_r", (M, D))
         dw_kv = g("dw_kv", (M, 2 * Hd, D))
@@ -395,10 +425,18 @@ class MoMLayer:
         B.mom_col_sums(dlogits, db_r, stream=side)
         B.mom_col_sums(dala, dA, stream=side)
         B.mom_col_sums(dz, db_a, col0=n_sh + H, stream=side)
+        out = dict(dx=dx, dw_sh=dw_sh, dw_gate=dw_gate, dw_r=dw_r, dw_kv=dw_kv, db_r=db_r, dA=dA, db_a=db_a)
+        if mg is not None:
+            dw_gm, dA_m, db_am = g("dw_gate_mem", (M, 2 * H, D)), g("dA_mem", (M, H)), g("db_a_mem", (M, H))
+            B.mom_gemm_grouped(1, mg["dzg"], x, dw_gm.view(M * 2 * H, D), 2 * H, D, 0, b["mem_offset"], None, M, ws_w,
+                               b_rows=b["perm"], c_group_stride=2 * H * D, stream=side)
+            B.mom_col_sums_grouped(mg["dala_p"], b["mem_offset"], dA_m, stream=side)
+            B.mom_col_sums_grouped(mg["dzg"], b["mem_offset"], db_am, col0=H, cols=H, stream=side)
+            out.update(dw_gate_mem=dw_gm, dA_mem=dA_m, db_a_mem=db_am)
         done = torch.cuda.Event()
         done.record(side)
         st.wait_event(done)
-        return dict(dx=dx, dw_sh=dw_sh, dw_gate=dw_gate, dw_r=dw_r, dw_kv=dw_kv, db_r=db_r, dA=dA, db_a=db_a)
+        return out
 
     # --------------------------------------------------------------- decode
     def decode_step(self, x: torch.Tensor, state: torch.Tensor, stream=None):

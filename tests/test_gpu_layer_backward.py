@@ -25,9 +25,9 @@ def _need_cuda():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
 
 
-def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True):
+def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True, mem_gates=False):
     from mixture_memories_layer_b200 import layer as L
-    w = synth.Workload("bwd", 0, 0, D, H, d, M, K, dtype, seed=seed)
+    w = synth.Workload("bwd", 0, 0, D, H, d, M, K, dtype, seed=seed, mem_gates=mem_gates)
     rng = np.random.default_rng(seed)
     p = synth.make_weights(w, rng)
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
@@ -57,6 +57,10 @@ def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True):
         "dw_k": (got["dw_kv"][:, :Hd], ref["dw_k"]), "dw_v": (got["dw_kv"][:, Hd:], ref["dw_v"]),
         "dh0_shared": (got["dh0_shared"], ref["dh0_shared"]), "dh0_mem": (got["dh0_mem"], ref["dh0_mem"]),
     }
+    if mem_gates:
+        pairs.update({"dw_beta_mem": (got["dw_gate_mem"][:, :H], ref["dw_beta_mem"]),
+                      "dw_a_mem": (got["dw_gate_mem"][:, H:], ref["dw_a_mem"]),
+                      "dA_mem": (got["dA_mem"], ref["dA_mem"]), "db_a_mem": (got["db_a_mem"], ref["db_a_mem"])})
     return {k: max_abs_rel(a, r) for k, (a, r) in pairs.items()}
 
 
@@ -131,3 +135,13 @@ def test_gemm_grouped_tf32(trans_a, a_col, lda_pad):
     """tf32 products (A rounded to a 10-bit mantissa, B exact, fp32 sums):
     within 2e-3 of the fp64 product per tensor."""
     assert _gemm_case(trans_a, a_col, lda_pad, seed=10 * trans_a + a_col) < 2e-3
+
+
+@pytest.mark.parametrize("dtype,tol", [("f32", 1e-5), ("bf16", 2e-2)])
+def test_layer_backward_per_memory_gates(dtype, tol):
+    """Each memory's own gates (MOM_GATES_BY_ROW): the routed reverse pass on
+    the rows' gates, their adjoints through mom_gates_bwd_by_group into the
+    memories' gate weights, A_mem and b_a_mem."""
+    errs = _run(dtype, 64, (120, 0, 77), M=4, K=2, seed=84, mem_gates=True)
+    bad = {k: e for k, e in errs.items() if not e < tol}
+    assert not bad, (bad, errs)
