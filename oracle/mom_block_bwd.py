@@ -103,9 +103,10 @@ def block_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dy, scale: floa
     Returns a dict: dx; dw_r, db_r; dw_q, dw_k_sh, dw_v_sh, dw_g; dconv_q,
     dconv_k_sh, dconv_v_sh [Hd, W], dconv_k, dconv_v [M, Hd, W]; dw_norm;
     dw_o; dw_beta, dw_a, dA, db_a; dw_k, dw_v [M, Hd, D]; dh0_shared,
-    dh0_mem; and the forward's results under "fwd"."""
-    if fwd.has_memory_gates(p):
-        raise NotImplementedError("the backward of per-memory gates is not written")
+    dh0_mem; and the forward's results under "fwd".  With per-memory gates
+    (each memory's routed rows on its own beta and alpha, as in the forward)
+    also dw_beta_mem, dw_a_mem [M, H, D], dA_mem, db_a_mem [M, H]."""
+    mem_gates = fwd.has_memory_gates(p)
     x = np.asarray(x, F64)
     dy = np.asarray(dy, F64)
     cu = np.asarray(cu_seqlens, np.int64)
@@ -138,6 +139,9 @@ def block_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dy, scale: floa
         out[name] = np.zeros_like(P[name[1:]])
     out["dconv_k"] = np.zeros_like(P["conv_k"])
     out["dconv_v"] = np.zeros_like(P["conv_v"])
+    if mem_gates:
+        for name in ("w_beta_mem", "w_a_mem", "A_mem", "b_a_mem"):
+            out["d" + name] = np.zeros_like(P[name])
     for s in range(S):
         t0, t1 = int(cu[s]), int(cu[s + 1])
         dhf = None if dh_shared is None else dh_shared[s]
@@ -164,11 +168,26 @@ def block_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dy, scale: floa
             k_m = f["k_mem"][rows, slot]
             v_m = f["v_mem"][rows, slot]
             h0 = None if h0_mem is None else h0_mem[m, s]
-            r = lbwd.gdn_recurrence_bwd(f["q"][rows], k_m, v_m, f["beta"][rows], f["log_alpha"][rows],
-                                        g_m[:, None, None] * do[rows], h0, dhf, scale, rule)
+            if mem_gates:
+                b_m, la_m = fwd.memory_gates(x[rows], p, m)
+            else:
+                b_m, la_m = f["beta"][rows], f["log_alpha"][rows]
+            r = lbwd.gdn_recurrence_bwd(f["q"][rows], k_m, v_m, b_m, la_m, g_m[:, None, None] * do[rows], h0, dhf,
+                                        scale, rule)
             dq[rows] += r["dq"]
-            dbeta[rows] += r["dbeta"]
-            dla[rows] += r["dlog_alpha"]
+            if mem_gates:
+                # memory m's own gates (mom_oracle.memory_gates)
+                dzb = r["dbeta"] * b_m * (1.0 - b_m)
+                za = x[rows] @ P["w_a_mem"][m].T + P["b_a_mem"][m]
+                dza = r["dlog_alpha"] * (-np.exp(P["A_mem"][m])) * fwd.sigmoid(za)
+                out["dw_beta_mem"][m] += dzb.T @ x[rows]
+                out["dw_a_mem"][m] += dza.T @ x[rows]
+                out["dA_mem"][m] += np.sum(r["dlog_alpha"] * la_m, axis=0)
+                out["db_a_mem"][m] += dza.sum(axis=0)
+                dx[rows] += dzb @ P["w_beta_mem"][m] + dza @ P["w_a_mem"][m]
+            else:
+                dbeta[rows] += r["dbeta"]
+                dla[rows] += r["dlog_alpha"]
             dh0_mem[m, s] = r["dh0"]
             seg = [(0, len(rows))]
             dxk, dwk, dck = _mixer_bwd(x[rows], P["w_k"][m], P["conv_k"][m], seg, r["dk"], H, d, True)

@@ -78,8 +78,8 @@ def test_planted_mistake_in_the_convolution_adjoint_fails():
     assert _rel(causal_adjoint(z, w, [(0, 7)], dc), ref) > 1e-2
 
 
-def _case(lens=(4, 0, 3), D=5, H=2, d=3, M=3, k=2, seed=2):
-    w = synth.Workload("bwd_tiny_block", 0, 0, D, H, d, M, k, "f32", seed=seed, block=True)
+def _case(lens=(4, 0, 3), D=5, H=2, d=3, M=3, k=2, seed=2, mem_gates=False):
+    w = synth.Workload("bwd_tiny_block", 0, 0, D, H, d, M, k, "f32", seed=seed, block=True, mem_gates=mem_gates)
     rng = np.random.default_rng(seed)
     p = {key: np.array(val, np.float64) for key, val in synth.make_weights(w, rng).items()}
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
@@ -110,3 +110,22 @@ def test_block_backward_matches_finite_differences(rule):
     for key, arr in checks:
         e = _rel(g[key], _fd(loss, arr))
         assert e < 1e-6, (rule, key, e)
+
+
+def test_block_backward_with_per_memory_gates_matches_finite_differences():
+    """Per-memory gates inside the block: the memories' own gate weights and
+    everything upstream of them against central differences."""
+    w, p, cu, x, adj, h0s, h0m = _case(seed=6, mem_gates=True)
+    H, d, K = w.heads, w.d_head, w.top_k
+    idx = fwd.router_topk(x, p["w_r"], p["b_r"], K)[0]
+
+    def loss():
+        f = blk.block_forward(x, p, cu, K, H, d, 1.0, forced_idx=idx, h0_shared=h0s, h0_mem=h0m)
+        return float(np.sum(adj["dy"] * f["y"]) + np.sum(adj["dhs"] * f["h_shared"]) + np.sum(adj["dhm"] * f["h_mem"]))
+
+    g = bb.block_backward(x, p, cu, K, H, d, adj["dy"], 1.0, forced_idx=idx, h0_shared=h0s, h0_mem=h0m,
+                          dh_shared=adj["dhs"], dh_mem=adj["dhm"])
+    names = ("w_beta", "w_a", "A", "b_a", "w_k", "w_q", "conv_k", "w_beta_mem", "w_a_mem", "A_mem", "b_a_mem")
+    for key, arr in [("dx", x)] + [("d" + n, p[n]) for n in names]:
+        e = _rel(g[key], _fd(loss, arr))
+        assert e < 1e-6, (key, e)
