@@ -183,9 +183,9 @@ class MoMBlock(MoMLayer):
         fixed.  Every step runs in the CUDA library: the output projection's
         two GEMMs, the gated norm's adjoint (which also gives the output
         gate's), the layer's reverse pass, the five convolutions' adjoints in
-        one launch pair, the gates' adjoint and the projections' GEMMs."""
-        if self.mem_gates:
-            raise NotImplementedError("the backward of per-memory gates is not provided")
+        one launch pair, the gates' adjoint and the projections' GEMMs.  With
+        per-memory gates also dw_gate_mem [M, 2H, D], dA_mem, db_a_mem [M, H]
+        (as MoMLayer.backward)."""
         n_tok, D = x.shape
         n_seq = cu_seqlens.numel() - 1
         H, d, K, M, dt = self.H, self.d, self.top_k, self.n_mem, self.dtype
@@ -234,9 +234,11 @@ class MoMBlock(MoMLayer):
         dala = g("dala", (n_tok, H))
         B.mom_gates_bwd(b["beta"], b["log_alpha"], c["dbeta"], c["dla"], w["A"], dz, 4 * Hd, 4 * Hd + H, dala,
                         stream=st)
-        r = self._proj_bwd(x, b, dz, 4 * Hd, w["w_shared4"], dzr, c["dlogits"], dala, st, ws)
+        mg = self._mem_gates_bwd(b, c, st)
+        r = self._proj_bwd(x, b, dz, 4 * Hd, w["w_shared4"], dzr, c["dlogits"], dala, st, ws, mg)
         out = dict(dx=r["dx"], dw_o=dw_o, dw_norm=dw_norm, dw_shared4=r["dw_sh"], dw_gate=r["dw_gate"], dA=r["dA"],
                    db_a=r["db_a"], dw_r=r["dw_r"], db_r=r["db_r"], dw_kv=r["dw_kv"], dh0_shared=c["dh0_shared"],
                    dh0_mem=c["dh0_mem"])
         out.update({"d" + n: t for n, t in dconv.items()})
+        out.update({k_: r[k_] for k_ in ("dw_gate_mem", "dA_mem", "db_a_mem") if k_ in r})
         return out

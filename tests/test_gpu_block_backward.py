@@ -212,7 +212,10 @@ def _pairs(got, ref, H, d):
         "dconv_k": (np.swapaxes(got["dconv_k"], 1, 2), ref["dconv_k"]),
         "dconv_v": (np.swapaxes(got["dconv_v"], 1, 2), ref["dconv_v"]),
         "dh0_shared": (got["dh0_shared"], ref["dh0_shared"]), "dh0_mem": (got["dh0_mem"], ref["dh0_mem"]),
-    }
+    } | ({"dw_beta_mem": (got["dw_gate_mem"][:, :H], ref["dw_beta_mem"]),
+          "dw_a_mem": (got["dw_gate_mem"][:, H:], ref["dw_a_mem"]),
+          "dA_mem": (got["dA_mem"], ref["dA_mem"]), "db_a_mem": (got["db_a_mem"], ref["db_a_mem"])}
+         if "dw_gate_mem" in got else {})
 
 
 def _run_block_bwd(w, p, rule="gated_delta", with_states=True, dy_rows=None, seqs=None):
@@ -275,6 +278,9 @@ def _tolerances(oracle, x, ref, H, d, seed):
 def _as_gpu_layout(r):
     """The oracle's gradients laid out as MoMBlock.backward returns them."""
     out = {k: r[k] for k in ("dx", "dw_o", "dw_norm", "dA", "db_a", "dw_r", "db_r", "dh0_shared", "dh0_mem")}
+    if "dw_beta_mem" in r:
+        out.update(dw_gate_mem=np.concatenate([r["dw_beta_mem"], r["dw_a_mem"]], axis=1), dA_mem=r["dA_mem"],
+                   db_a_mem=r["db_a_mem"])
     out.update(dw_shared4=np.concatenate([r["dw_q"], r["dw_k_sh"], r["dw_v_sh"], r["dw_g"]]),
                dw_gate=np.concatenate([r["dw_beta"], r["dw_a"]]),
                dw_kv=np.concatenate([r["dw_k"], r["dw_v"]], axis=1),
@@ -298,6 +304,16 @@ def test_block_backward_small_ragged(d, H, lens):
 def test_block_backward_other_rule_and_no_state_adjoints(rule, with_states):
     w, p = _problem(128, (120, 1, 70), 2, M=3, k=1, seed=12)
     _assert_within(_run_block_bwd(w, p, rule=rule, with_states=with_states))
+
+
+def test_block_backward_per_memory_gates():
+    """The block around memories with their own gates."""
+    import dataclasses
+    w, p = _problem(128, (150, 1, 60), 2, M=4, k=2, seed=14)
+    w = dataclasses.replace(w, mem_gates=True)
+    rng = np.random.default_rng(14)
+    p.update({k: v for k, v in synth.make_weights(w, rng).items() if k.endswith("_mem")})
+    _assert_within(_run_block_bwd(w, p))
 
 
 def test_block_backward_380m_shape_one_sequence():
