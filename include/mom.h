@@ -302,6 +302,20 @@ mom_status mom_mem_gate_proj(const void* x, const int32_t* perm_token, const int
                              int64_t n_tok, int d_model, int H, int n_mem, int top_k,
                              float* beta_p, float* log_alpha_p, void* ws, size_t ws_bytes, void* stream);
 
+/* mom_mem_gate_proj_groups -- mom_mem_gate_proj over groups of rows that
+ * name their memory: rows group_offset[g] .. group_offset[g+1]-1 (device,
+ * n_groups + 1 entries, n_groups <= MOM_MAX_MEM) take memory group_mem[g]'s
+ * gates (W^m, A^m, b_a^m of the n_mem in w_gate_mem, A_mem, b_a_mem), and
+ * row r reads x row perm_token[r] (NULL: row r).  For the rows a
+ * memory-parallel owner receives (groups: (source rank, memory)).  A group
+ * whose memory is out of range is recorded (MOM_DEVERR_ROW_INDEX) and its
+ * rows get beta = log_alpha = 0. */
+mom_status mom_mem_gate_proj_groups(const void* x, int64_t n_x, const int32_t* perm_token, int64_t n_rows,
+                                    const int32_t* group_offset, const int32_t* group_mem, int n_groups,
+                                    const void* w_gate_mem, const float* A_mem, const float* b_a_mem, int n_mem,
+                                    mom_dtype dt, int d_model, int H, float* beta_p, float* log_alpha_p, void* ws,
+                                    size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * mom_gdn_chunk_fwd -- the Gated DeltaNet recurrence of one memory over
  * each segment (blog post, experiments section: every memory uses Gated

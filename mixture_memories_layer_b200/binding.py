@@ -70,6 +70,8 @@ SIGNATURES = {
     "mom_l2norm_bwd": (_I, [_VP, _VP, _VP, _I64, _I, _I, _I, _VP, _I64, _I64, _VP]),
     "mom_gates_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _I, _VP, _I64, _I64, _I64, _VP, _VP]),
     "mom_col_sums": (_I, [_VP, _I64, _I64, _I64, _VP, _VP]),
+    "mom_mem_gate_proj_groups": (_I, [_VP, _I64, _VP, _I64, _VP, _VP, _I, _VP, _VP, _VP, _I, _I, _I, _I, _VP, _VP,
+                                      _VP, _SZ, _VP]),
     "mom_gates_bwd_by_group": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _VP, _I64, _I64, _I64, _VP, _VP]),
     "mom_col_sums_grouped": (_I, [_VP, _I64, _I64, _I64, _VP, _I, _VP, _VP]),
     "mom_gemm_grouped": (_I, [_I, _VP, _I64, _VP, _I64, _I, _VP, _I64, _VP, _I64, _I64, _I64, _I64, _I64, _VP, _VP,
@@ -424,6 +426,17 @@ def mom_col_sums_grouped(a, group_offset, out, col0=0, cols=None, stream=None):
     cols = out.shape[-1] if cols is None else cols
     _check(lib.mom_col_sums_grouped(_pa(a, col0), rows, lda, cols, _p(group_offset), group_offset.numel() - 1,
                                     _p(out), _s(stream)), "mom_col_sums_grouped")
+
+
+def mom_mem_gate_proj_groups(x, group_offset, group_mem, w_gate_mem, A_mem, b_a_mem, beta_p, log_alpha_p, ws,
+                             perm_token=None, stream=None):
+    """Per-memory gates of rows grouped by (group_offset, group_mem); row r
+    reads x row perm_token[r] (None: row r)."""
+    n_rows, H = beta_p.shape
+    _check(lib.mom_mem_gate_proj_groups(_p(x), x.shape[0], _p(perm_token), n_rows, _p(group_offset), _p(group_mem),
+                                        group_mem.numel(), _p(w_gate_mem), _p(A_mem), _p(b_a_mem), w_gate_mem.shape[0],
+                                        dtype_code(x.dtype), x.shape[1], H, _p(beta_p), _p(log_alpha_p), _p(ws),
+                                        ws.numel(), _s(stream)), "mom_mem_gate_proj_groups")
 
 
 def mom_col_sums(a, out, col0=0, stream=None):

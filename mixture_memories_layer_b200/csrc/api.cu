@@ -309,6 +309,26 @@ mom_status mom_mem_gate_proj(const void* x, const int32_t* perm_token, const int
                                             as_stream(stream)));
 }
 
+mom_status mom_mem_gate_proj_groups(const void* x, int64_t n_x, const int32_t* perm_token, int64_t n_rows,
+                                    const int32_t* group_offset, const int32_t* group_mem, int n_groups,
+                                    const void* w_gate_mem, const float* A_mem, const float* b_a_mem, int n_mem,
+                                    mom_dtype dt, int d_model, int H, float* beta_p, float* log_alpha_p, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    if (!dt_ok(dt) || n_x < 0 || n_rows < 0 || d_model <= 0 || d_model % 8 != 0 || H < 1 || H > MOM_MAX_HEADS)
+        return MOM_ERR_ARG;
+    if (n_groups < 1 || n_groups > MOM_MAX_MEM || n_mem < 1) return MOM_ERR_ARG;
+    if (!ws || ws_bytes < MOM_WS_HEADER_BYTES) return MOM_ERR_ARG;
+    if (n_rows == 0) return MOM_OK;
+    const void* ptrs[] = {x, group_offset, group_mem, w_gate_mem, A_mem, b_a_mem, beta_p, log_alpha_p};
+    for (const void* p : ptrs)
+        if (!p) return MOM_ERR_ARG;
+    if (!perm_token && n_x < n_rows) return MOM_ERR_ARG;
+    if (!al16(x) || !al16(w_gate_mem)) return MOM_ERR_ARG;
+    return cuda_status(launch_mem_gate_proj(x, perm_token, group_offset, w_gate_mem, A_mem, b_a_mem, dt, n_x, n_rows,
+                                            d_model, H, n_groups, beta_p, log_alpha_p, ws, as_stream(stream),
+                                            group_mem, n_mem));
+}
+
 // --------------------------------------------------------- chunked GDN
 size_t mom_gdn_workspace_size(int64_t n_rows, int n_seg, int H, int d, mom_dtype dt) {
     size_t extra = (dt == MOM_BF16 && head_dim_ok(d)) ? gdn_tc_ws_bytes(n_rows, n_seg, H, d) : 0;

@@ -37,7 +37,8 @@ cudaError_t launch_router(const void* x, const void* w_r, const float* b_r, int 
 // mem_gates.cu: per-memory gates of the routed rows (beta_p, log_alpha_p [n_rows, H])
 cudaError_t launch_mem_gate_proj(const void* x, const int32_t* perm, const int32_t* mem_offset, const void* w_gate_mem,
                                  const float* A_mem, const float* b_a_mem, int dt, int64_t n_tok, int64_t n_rows, int D,
-                                 int H, int M, float* beta, float* log_alpha, void* err, cudaStream_t st);
+                                 int H, int M, float* beta, float* log_alpha, void* err, cudaStream_t st,
+                                 const int32_t* group_mem = nullptr, int n_w = 0);
 cudaError_t launch_gate_proj(const void* x, const void* w_gate, const float* A, const float* b_a, int dt,
                              int64_t n_tok, int D, int H, float* beta, float* log_alpha, void* err, cudaStream_t st);
 

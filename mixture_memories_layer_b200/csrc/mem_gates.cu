@@ -32,17 +32,29 @@ constexpr int MG_WARPS = 8;    // warps (tiles) per CTA
 
 struct MemGateArgs {
     const void* x;              // [n_tok, D]
-    const int32_t* perm;        // [n_rows] token of each routed row
-    const int32_t* mem_offset;  // [M + 1] first row of each memory
-    const void* w;              // [M, 2H, D]: rows W_beta^m | W_a^m
-    const float* A;             // [M, H]
-    const float* b_a;           // [M, H]
+    const int32_t* perm;        // [n_rows] token of each routed row (null: row r reads x row r)
+    const int32_t* mem_offset;  // [M + 1] first row of each group (a memory, or a (source, memory) group)
+    const void* w;              // [n_w, 2H, D]: rows W_beta^m | W_a^m
+    const float* A;             // [n_w, H]
+    const float* b_a;           // [n_w, H]
     int64_t n_tok, n_rows;
     int D, H, M;
     float* beta;                // [n_rows, H]
     float* la;                  // [n_rows, H]
     void* err;
+    const int32_t* gmem;        // [M] weights of each group (null: group m = memory m)
+    int n_w;                    // memories in w, A, b_a
 };
+
+// the group table and each group's memory (-1: out of range) into shared memory
+__device__ __forceinline__ void load_tables(const MemGateArgs& a, int* off, int* wix) {
+    for (int i = threadIdx.x; i <= a.M; i += blockDim.x) off[i] = a.mem_offset[i];
+    for (int i = threadIdx.x; i < a.M; i += blockDim.x) {
+        const int m = a.gmem ? a.gmem[i] : i;
+        wix[i] = (m >= 0 && m < a.n_w) ? m : -1;
+    }
+    __syncthreads();
+}
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
@@ -100,9 +112,8 @@ __device__ __forceinline__ void write_gates(const MemGateArgs& a, int64_t r, int
 template <int NT>
 __global__ void __launch_bounds__(MG_WARPS * 32)
 mem_gate_mma_kernel(MemGateArgs a) {
-    __shared__ int off[MOM_MAX_MEM + 1];
-    for (int i = threadIdx.x; i <= a.M; i += blockDim.x) off[i] = a.mem_offset[i];
-    __syncthreads();
+    __shared__ int off[MOM_MAX_MEM + 1], wix[MOM_MAX_MEM];
+    load_tables(a, off, wix);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     const int64_t tile = (int64_t)blockIdx.x * MG_WARPS + warp;
     const int64_t r0 = tile * MG_TOK;
@@ -122,8 +133,8 @@ mem_gate_mma_kernel(MemGateArgs a) {
         mem[e] = -1;
         if (r < a.n_rows) {
             const int m = memory_of(off, a.M, r);
-            const int64_t t = a.perm[r];
-            if (m >= 0 && t >= 0 && t < a.n_tok) {
+            const int64_t t = a.perm ? a.perm[r] : r;
+            if (m >= 0 && wix[m] >= 0 && t >= 0 && t < a.n_tok) {
                 tok[e] = t;
                 mem[e] = m;
                 mlo = min(mlo, m);
@@ -142,8 +153,8 @@ mem_gate_mma_kernel(MemGateArgs a) {
     const bf16* x0 = x + (tok[0] >= 0 ? tok[0] : 0) * D + 8 * c;
     const bf16* x1 = x + (tok[1] >= 0 ? tok[1] : 0) * D + 8 * c;
     for (int m = mlo; m <= mhi; ++m) {
-        if (off[m] == off[m + 1]) continue;
-        const bf16* wm = w + (size_t)m * ncol * D + 8 * c;
+        if (off[m] == off[m + 1] || wix[m] < 0) continue;
+        const bf16* wm = w + (size_t)wix[m] * ncol * D + 8 * c;
         // two accumulator sets (the two 32-feature halves of each 64-feature
         // block) halve the dependent MMA chain
         float acc[2][NT][4];
@@ -188,7 +199,7 @@ mem_gate_mma_kernel(MemGateArgs a) {
             for (int e = 0; e < 4; ++e) {
                 const int half = e >> 1;
                 if (mem[half] != m) continue;
-                write_gates(a, r0 + g + 8 * half, m, n * 8 + 2 * c + (e & 1), acc[0][n][e] + acc[1][n][e]);
+                write_gates(a, r0 + g + 8 * half, wix[m], n * 8 + 2 * c + (e & 1), acc[0][n][e] + acc[1][n][e]);
             }
     }
 }
@@ -197,16 +208,16 @@ mem_gate_mma_kernel(MemGateArgs a) {
 template <typename T>
 __global__ void __launch_bounds__(256)
 mem_gate_simt_kernel(MemGateArgs a) {
-    __shared__ int off[MOM_MAX_MEM + 1];
-    for (int i = threadIdx.x; i <= a.M; i += blockDim.x) off[i] = a.mem_offset[i];
-    __syncthreads();
+    __shared__ int off[MOM_MAX_MEM + 1], wix[MOM_MAX_MEM];
+    load_tables(a, off, wix);
     const int lane = threadIdx.x & 31, warps = blockDim.x >> 5;
     const T* x = reinterpret_cast<const T*>(a.x);
     const T* w = reinterpret_cast<const T*>(a.w);
     const int D = a.D, ncol = 2 * a.H;
     for (int64_t r = (int64_t)blockIdx.x * warps + (threadIdx.x >> 5); r < a.n_rows; r += (int64_t)gridDim.x * warps) {
-        const int m = memory_of(off, a.M, r);
-        const int64_t t = a.perm[r];
+        const int m0 = memory_of(off, a.M, r);
+        const int m = m0 >= 0 ? wix[m0] : -1;
+        const int64_t t = a.perm ? a.perm[r] : r;
         if (m < 0 || t < 0 || t >= a.n_tok) {
             if (lane == 0) record_error(a.err, MOM_DEVERR_ROW_INDEX, r);
             for (int h = lane; h < a.H; h += 32) { a.beta[r * a.H + h] = 0.f; a.la[r * a.H + h] = 0.f; }
@@ -236,9 +247,11 @@ mem_gate_simt_kernel(MemGateArgs a) {
 
 cudaError_t launch_mem_gate_proj(const void* x, const int32_t* perm, const int32_t* mem_offset, const void* w_gate_mem,
                                  const float* A_mem, const float* b_a_mem, int dt, int64_t n_tok, int64_t n_rows, int D,
-                                 int H, int M, float* beta, float* log_alpha, void* err, cudaStream_t st) {
+                                 int H, int M, float* beta, float* log_alpha, void* err, cudaStream_t st,
+                                 const int32_t* group_mem, int n_w) {
     if (n_rows == 0) return cudaSuccess;
-    MemGateArgs a{x, perm, mem_offset, w_gate_mem, A_mem, b_a_mem, n_tok, n_rows, D, H, M, beta, log_alpha, err};
+    MemGateArgs a{x, perm, mem_offset, w_gate_mem, A_mem, b_a_mem, n_tok, n_rows, D, H, M, beta, log_alpha, err,
+                  group_mem, group_mem ? n_w : M};
     if (dt == MOM_BF16 && D % 64 == 0 && 2 * H <= 32) {
         const unsigned grid = (unsigned)cdiv(cdiv(n_rows, MG_TOK), MG_WARPS);
         if (2 * H <= 8) mem_gate_mma_kernel<1><<<grid, MG_WARPS * 32, 0, st>>>(a);

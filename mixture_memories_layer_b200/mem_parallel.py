@@ -34,6 +34,9 @@ import numpy as np
 import torch
 
 
+MAX_GATE_GROUPS = 32        # mom_mem_gate_proj_groups' group limit (MOM_MAX_MEM)
+
+
 # ----------------------------------------------------------------- planning
 class Partition:
     """Memories [lo(g), hi(g)) of rank g: contiguous blocks whose sizes
@@ -185,6 +188,10 @@ class CudaKernels:
     def gates(self, x, w_gate, A, b_a, beta, log_alpha, ws, stream):
         self.B.mom_gate_proj(x, w_gate, A, b_a, beta, log_alpha, ws, stream=stream)
 
+    def mem_gates_groups(self, x, group_offset, group_mem, w_gate_mem, A_mem, b_a_mem, beta, log_alpha, ws, stream):
+        self.B.mom_mem_gate_proj_groups(x, group_offset, group_mem, w_gate_mem, A_mem, b_a_mem, beta, log_alpha, ws,
+                                        stream=stream)
+
     def copy_rows(self, src, idx, dst, row_bytes, src_off, dst_off, ws, stream):
         self.B.mom_copy_rows(src, idx, dst, row_bytes, src_off=src_off, dst_off=dst_off, ws=ws, stream=stream)
 
@@ -226,7 +233,10 @@ class MemoryParallelMoM:
 
     weights: the replicated parameters (w_r, b_r, w_shared, w_gate, A, b_a
     as pack_weights lays them out) and, under "w_kv", this rank's memories
-    only: [hi - lo, 2*H*d, d_model] for its block of the Partition."""
+    only: [hi - lo, 2*H*d, d_model] for its block of the Partition; with
+    per-memory gates also this rank's w_gate_mem [hi - lo, 2*H, d_model],
+    A_mem and b_a_mem [hi - lo, H]: the owner computes the gates of the rows
+    it receives with them."""
 
     def __init__(self, weights, heads: int, d_head: int, top_k: int, n_mem: int, comm, scale: float = 1.0,
                  rule: str = "gated_delta", kernels=None):
@@ -240,8 +250,12 @@ class MemoryParallelMoM:
         own = self.part.hi(self.rank) - self.part.lo(self.rank)
         if weights["w_kv"].shape[0] != own:
             raise ValueError("w_kv holds %d memories; rank %d owns %d" % (weights["w_kv"].shape[0], self.rank, own))
-        if any(k.endswith("_mem") for k in weights):
-            raise ValueError("per-memory gates are not provided by the memory-parallel layer")
+        self.mem_gates = "w_gate_mem" in weights
+        if self.mem_gates:
+            for name in ("w_gate_mem", "A_mem", "b_a_mem"):
+                if weights[name].shape[0] != own:
+                    raise ValueError("%s holds %d memories; rank %d owns %d" % (name, weights[name].shape[0],
+                                                                                self.rank, own))
 
     def _workspace(self, name, nbytes, device):
         """A workspace kept across calls (zeroed once, grown when needed)."""
@@ -354,10 +368,17 @@ class MemoryParallelMoM:
         k.copy_rows(recv, None, q_r.view(torch.uint8).view(n, qb), qb, xb, 0, ws, stream)
         beta = torch.empty((n, H), dtype=torch.float32, device=dev)
         log_alpha = torch.empty_like(beta)
-        k.gates(x_r, w["w_gate"], w["A"], w["b_a"], beta, log_alpha, ws, stream)
         lo = self.part.lo(self.rank)
         go = self._to_device(tables.group_offset, dev)
-        gm = self._to_device(tables.group_mem - lo, dev)             # index into this rank's w_kv block
+        gm = self._to_device(tables.group_mem - lo, dev)             # index into this rank's weight blocks
+        if self.mem_gates:
+            # each (source, memory) group on its memory's own gates
+            if len(tables.group_mem) > MAX_GATE_GROUPS:
+                raise ValueError("per-memory gates take at most %d (source, memory) groups per owner, not %d"
+                                 % (MAX_GATE_GROUPS, len(tables.group_mem)))
+            k.mem_gates_groups(x_r, go, gm, w["w_gate_mem"], w["A_mem"], w["b_a_mem"], beta, log_alpha, ws, stream)
+        else:
+            k.gates(x_r, w["w_gate"], w["A"], w["b_a"], beta, log_alpha, ws, stream)
         seg = self._to_device(tables.seg_cu, dev)
         k_p = torch.empty((n, H, d), dtype=dt, device=dev)
         v_p = torch.empty_like(k_p)

@@ -31,8 +31,9 @@ def _need_cuda():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
 
 
-def _problem(D=256, H=2, d=128, M=4, K=2, lens=(300, 77, 1, 130), seed=71, bias0=0.0, dtype="bf16"):
-    w = synth.Workload("mp", 0, 0, D, H, d, M, K, dtype, seed=seed, router_bias0=bias0)
+def _problem(D=256, H=2, d=128, M=4, K=2, lens=(300, 77, 1, 130), seed=71, bias0=0.0, dtype="bf16",
+             mem_gates=False):
+    w = synth.Workload("mp", 0, 0, D, H, d, M, K, dtype, seed=seed, router_bias0=bias0, mem_gates=mem_gates)
     rng = np.random.default_rng(seed)
     p = synth.make_weights(w, rng)
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
@@ -46,8 +47,13 @@ def _layer(w, p, dt):
 
 
 def _local_weights(weights, part, g):
-    lw = {k: v for k, v in weights.items() if k != "w_kv"}
-    lw["w_kv"] = weights["w_kv"][part.lo(g):part.hi(g)].contiguous()
+    """The replicated weights plus rank g's memories' own (w_kv and, with
+    per-memory gates, w_gate_mem, A_mem, b_a_mem)."""
+    own = ("w_kv", "w_gate_mem", "A_mem", "b_a_mem")
+    lw = {k: v for k, v in weights.items() if k not in own}
+    for k in own:
+        if k in weights:
+            lw[k] = weights[k][part.lo(g):part.hi(g)].contiguous()
     return lw
 
 
@@ -183,9 +189,13 @@ def _emulated_ranks(w, p, x, cu, world, split):
     return lay, res, owner_out
 
 
-@pytest.mark.parametrize("case", ["mom380m_short", "skewed_ragged"])
+@pytest.mark.parametrize("case", ["mom380m_short", "skewed_ragged", "per_memory_gates"])
 def test_two_emulated_ranks_equal_the_layer(case):
-    if case == "mom380m_short":
+    if case == "per_memory_gates":
+        # each owner computes its memories' gates for the rows it receives
+        w, p, x, cu = _problem(M=5, lens=(300, 0, 77, 1, 130, 64), seed=74, mem_gates=True)
+        split = (0, 3, 6)
+    elif case == "mom380m_short":
         w0 = synth.WORKLOADS["mom380m"]
         w, p, x, cu = _problem(D=w0.d_model, H=w0.heads, d=w0.d_head, M=w0.n_mem, K=w0.top_k,
                                lens=(512,) * 8, seed=72)

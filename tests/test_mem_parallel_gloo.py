@@ -104,6 +104,19 @@ class OracleKernels:
         beta.copy_(torch.as_tensor(b.astype(np.float32)))
         log_alpha.copy_(torch.as_tensor(la.astype(np.float32)))
 
+    def mem_gates_groups(self, x, group_offset, group_mem, w_gate_mem, A_mem, b_a_mem, beta, log_alpha, ws, stream):
+        H = beta.shape[1]
+        xx = np.asarray(x.numpy(), np.float64)
+        go, gm = group_offset.numpy(), group_mem.numpy()
+        for g in range(len(gm)):
+            a, b = int(go[g]), int(go[g + 1])
+            m = int(gm[g])
+            p = {"w_beta_mem": w_gate_mem.numpy()[:, :H], "w_a_mem": w_gate_mem.numpy()[:, H:],
+                 "A_mem": A_mem.numpy(), "b_a_mem": b_a_mem.numpy()}
+            bb, la = orc.memory_gates(xx[a:b], p, m)
+            beta[a:b] = torch.as_tensor(bb.astype(np.float32))
+            log_alpha[a:b] = torch.as_tensor(la.astype(np.float32))
+
     def copy_rows(self, src, idx, dst, row_bytes, src_off, dst_off, ws, stream):
         s = src.contiguous().view(torch.uint8).reshape(src.shape[0], -1).numpy()
         d = dst.view(torch.uint8).reshape(dst.shape[0], -1).numpy()
@@ -149,8 +162,8 @@ class OracleKernels:
         return rule
 
 
-def _problem(seed=61, M=5, K=2, H=2, d=8, D=32, lens=((9, 0, 13), (7, 11), (5,))):
-    w = synth.Workload("mp", 0, 0, D, H, d, M, K, "f32", seed=seed)
+def _problem(seed=61, M=5, K=2, H=2, d=8, D=32, lens=((9, 0, 13), (7, 11), (5,)), mem_gates=False):
+    w = synth.Workload("mp", 0, 0, D, H, d, M, K, "f32", seed=seed, mem_gates=mem_gates)
     rng = np.random.default_rng(seed)
     p = synth.make_weights(w, rng)
     xs = [synth.make_tokens(w, rng, int(sum(l))) for l in lens]
@@ -165,15 +178,18 @@ def _pack(p, part, g):
                 w_shared=t(np.concatenate([p["w_q"], p["w_k_sh"], p["w_v_sh"]])),
                 w_gate=t(np.concatenate([p["w_beta"], p["w_a"]])), A=t(p["A"]), b_a=t(p["b_a"]),
                 w_kv=t(np.stack([np.concatenate([p["w_k"][m], p["w_v"][m]]) for m in range(lo, hi)])
-                       if hi > lo else np.zeros((0, 2 * Hd, p["w_q"].shape[1]))))
+                       if hi > lo else np.zeros((0, 2 * Hd, p["w_q"].shape[1]))),
+                **({} if "w_beta_mem" not in p else dict(
+                    w_gate_mem=t(np.concatenate([p["w_beta_mem"][lo:hi], p["w_a_mem"][lo:hi]], axis=1)),
+                    A_mem=t(p["A_mem"][lo:hi]), b_a_mem=t(p["b_a_mem"][lo:hi]))))
 
 
-def _rank_main(rank, world, port, seed, M, rule, q):
+def _rank_main(rank, world, port, seed, M, rule, q, mem_gates=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        w, p, xs, lens = _problem(seed=seed, M=M, lens=((9, 0, 13), (7, 11), (5,))[:world])
+        w, p, xs, lens = _problem(seed=seed, M=M, lens=((9, 0, 13), (7, 11), (5,))[:world], mem_gates=mem_gates)
         part = Partition(M, world)
         layer = MemoryParallelMoM(_pack(p, part, rank), w.heads, w.d_head, w.top_k, M, TorchComm(), rule=rule,
                                   kernels=OracleKernels(w.heads, w.d_head))
@@ -202,11 +218,16 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("world,M,rule", [(2, 5, "gated_delta"), (2, 4, "gated_linear"), (3, 2, "gated_delta")])
-def test_memory_parallel_forward_on_gloo_ranks(world, M, rule):
+@pytest.mark.parametrize("world,M,rule,mem_gates", [(2, 5, "gated_delta", False), (2, 4, "gated_linear", False),
+                                                   (3, 2, "gated_delta", False), (2, 5, "gated_delta", True),
+                                                   (3, 2, "gated_linear", True)])
+def test_memory_parallel_forward_on_gloo_ranks(world, M, rule, mem_gates):
+    """The data flow over 2 and 3 gloo ranks against the oracle, with the
+    shared gates and with per-memory gates (computed by each owner for the
+    rows it receives)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    mp.start_processes(_rank_main, args=(world, _free_port(), 61, M, rule, q), nprocs=world, join=True,
+    mp.start_processes(_rank_main, args=(world, _free_port(), 61, M, rule, q, mem_gates), nprocs=world, join=True,
                        start_method="spawn")
     res = sorted(q.get() for _ in range(world))
     part = Partition(M, world)
