@@ -229,7 +229,8 @@ def router_gates_bwd(logits, idx, dgate):
 
 
 def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: float = 1.0,
-                 forced_idx=None, h0_shared=None, h0_mem=None, dh_shared=None, dh_mem=None):
+                 forced_idx=None, h0_shared=None, h0_mem=None, dh_shared=None, dh_mem=None,
+                 rule: str = "gated_delta"):
     """Gradients of L (module docstring) for one layer forward over a packed
     batch; arguments as ``mom_oracle.mom_forward`` plus the adjoints dout
     [N,H,d], dh_shared [S,H,d,d] and dh_mem [M,S,H,d,d] (None: zero).
@@ -251,7 +252,7 @@ def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: floa
     W = {name: np.asarray(p[name], F64) for name in
          ("w_r", "w_q", "w_k_sh", "w_v_sh", "w_beta", "w_a", "A", "b_a", "w_k", "w_v")}
     f = fwd.mom_forward(x, p, cu, top_k, H, d, scale, forced_idx=forced_idx,
-                        h0_shared=h0_shared, h0_mem=h0_mem)
+                        h0_shared=h0_shared, h0_mem=h0_mem, rule=rule)
     idx, gate = f["idx"], f["gate"]
     mem_gates = fwd.has_memory_gates(p)
     if mem_gates:
@@ -279,7 +280,7 @@ def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: floa
         dhf = None if dh_shared is None else dh_shared[s]
         if t1 > t0:
             r = gdn_recurrence_bwd(f["q"][t0:t1], f["k_sh"][t0:t1], f["v_sh"][t0:t1], f["beta"][t0:t1],
-                                   f["log_alpha"][t0:t1], do_shared[t0:t1], h0, dhf, scale)
+                                   f["log_alpha"][t0:t1], do_shared[t0:t1], h0, dhf, scale, rule)
             dq[t0:t1] += r["dq"]
             dk_sh[t0:t1] += r["dk"]
             dv_sh[t0:t1] += r["dv"]
@@ -306,7 +307,7 @@ def mom_backward(x, p, cu_seqlens, top_k: int, H: int, d: int, dout, scale: floa
             else:
                 b_m, la_m = f["beta"][rows], f["log_alpha"][rows]
             r = gdn_recurrence_bwd(f["q"][rows], k_m, v_m, b_m, la_m, g[:, None, None] * dout[rows], h0, dhf,
-                                   scale)
+                                   scale, rule)
             dq[rows] += r["dq"]
             if mem_gates:
                 # memory m's own gates: beta = sigmoid(x W_beta^m^T), log alpha =

@@ -109,19 +109,20 @@ def _layer_case(lens=(4, 0, 3), D=5, H=2, d=3, M=3, k=2, seed=1, mem_gates=False
     return w, p, cu, x, adj, h0s, h0m
 
 
-def test_mom_backward_matches_finite_differences():
+@pytest.mark.parametrize("rule", ["gated_delta", "gated_linear"])
+def test_mom_backward_matches_finite_differences(rule):
     w, p, cu, x, adj, h0s, h0m = _layer_case()
     H, d, K = w.heads, w.d_head, w.top_k
     idx = fwd.router_topk(x, p["w_r"], p["b_r"], K)[0]       # routing held fixed
     scale = 0.8
 
     def loss():
-        f = fwd.mom_forward(x, p, cu, K, H, d, scale, forced_idx=idx, h0_shared=h0s, h0_mem=h0m)
+        f = fwd.mom_forward(x, p, cu, K, H, d, scale, forced_idx=idx, h0_shared=h0s, h0_mem=h0m, rule=rule)
         return float(np.sum(adj["dout"] * f["out"]) + np.sum(adj["dhs"] * f["h_shared"])
                      + np.sum(adj["dhm"] * f["h_mem"]))
 
     g = bwd.mom_backward(x, p, cu, K, H, d, adj["dout"], scale, forced_idx=idx, h0_shared=h0s, h0_mem=h0m,
-                         dh_shared=adj["dhs"], dh_mem=adj["dhm"])
+                         dh_shared=adj["dhs"], dh_mem=adj["dhm"], rule=rule)
     checks = [("dx", x)] + [("d" + name, p[name]) for name in
                             ("w_r", "b_r", "w_q", "w_k_sh", "w_v_sh", "w_beta", "w_a", "A", "b_a", "w_k", "w_v")]
     checks += [("dh0_shared", h0s), ("dh0_mem", h0m)]
