@@ -740,7 +740,7 @@ mom_status mom_norm_gate_bwd(const void* o_sh, const void* o_p, const int32_t* r
 typedef struct mom_conv_bwd_problem {
     const void*    z;         /* the forward's raw rows [n_rows, channels] (dt) */
     const float*   dout;      /* adjoint of out [n_rows, channels] */
-    float*         da;        /* scratch [n_rows, channels] */
+    float*         da;        /* reserved: not read or written (may be NULL) */
     float*         dz;        /* adjoint of z: dz[r*ldz + col0 + c], overwritten for rows in a segment */
     int64_t        ldz;
     int64_t        col0;
@@ -756,9 +756,10 @@ typedef struct mom_conv_bwd_problem {
 
 /* mom_short_conv_bwd -- for 1..8 problems of the same channel count, width
  * and head_dim: da = the adjoint of a (a recomputed from z, the L2 norm's
- * adjoint per head when l2norm, then SiLU's); dz[t] = sum_j w[W-1-j] da[t+j]
- * over the rows t+j in t's segment; dw[grp][W-1-j] = sum_t da[t] z[t-j].
- * `problems` is a HOST array read during the call.  bf16 z only. */
+ * adjoint per head when l2norm, then SiLU's, kept on chip); dz[t] = sum_j
+ * w[W-1-j] da[t+j] over the rows t+j in t's segment; dw[grp][W-1-j] =
+ * sum_t da[t] z[t-j].  `problems` is a HOST array read during the call.
+ * bf16 z only.  dout may alias nothing that the call writes. */
 mom_status mom_short_conv_bwd(const mom_conv_bwd_problem* problems, int n_problems, int channels, int width,
                               int head_dim, mom_dtype dt, void* ws, size_t ws_bytes, void* stream);
 

@@ -535,9 +535,9 @@ def mom_norm_gate_bwd(o_sh, o_p, row_of, topk_gate, g, w_norm, eps, d_y, d_o, dg
 
 
 def mom_short_conv_bwd(problems, head_dim, ws, stream=None):
-    """problems: dicts with z, dout, da, dz (a 2-D float32 tensor, possibly a
+    """problems: dicts with z, dout, dz (a 2-D float32 tensor, possibly a
     column slice: its row stride and offset are passed), seg_cu, w, dw and
-    optionally seg_per_group, l2norm."""
+    optionally seg_per_group, l2norm (da: reserved, ignored)."""
     arr = (MomConvBwdProblem * len(problems))()
     C = width = None
     for i, q in enumerate(problems):
@@ -551,7 +551,8 @@ def mom_short_conv_bwd(problems, head_dim, ws, stream=None):
             raise ValueError("MoM: dz must be a 2-D float32 CUDA tensor of unit column stride")
         ldz = dz.stride(0)
         col0 = dz.storage_offset() % ldz if ldz else 0
-        arr[i] = MomConvBwdProblem(_p(z).value, _p(q["dout"]).value, _p(q["da"]).value,
+        da = q.get("da")
+        arr[i] = MomConvBwdProblem(_p(z).value, _p(q["dout"]).value, None if da is None else _p(da).value,
                                    dz.data_ptr() - col0 * dz.element_size(), ldz, col0, z.shape[0],
                                    _p(q["seg_cu"]).value, n_seg, q.get("seg_per_group") or n_seg, w.shape[0],
                                    _p(w).value, _p(q["dw"]).value, int(q.get("l2norm", False)))

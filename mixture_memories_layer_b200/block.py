@@ -214,21 +214,21 @@ class MoMBlock(MoMLayer):
         B.mom_norm_gate_bwd(b["o_sh"], b["o_p"], b["row_of"], b["gate"], b["g"], w["w_norm"], self.eps, dot, do,
                             dz[:, 3 * Hd:], dw_norm, ws, stream=st)
         c = self._core_bwd(b, cu_seqlens, do, dh_shared, dh_mem, h0_shared, h0_mem, st, ws)
-        # the convolutions (+ SiLU, + L2 norm of q and k) backwards, in place
-        # on the recurrences' input gradients, into the raw projections' columns
+        # the convolutions (+ SiLU, + L2 norm of q and k) backwards, from the
+        # recurrences' input gradients into the raw projections' columns
         dzr = g("dzr", (R, 2 * Hd))
         f = lambda t: t.view(t.shape[0], Hd)
         dconv = {n: g("d" + n, tuple(w[n].shape)) for n in ("conv_q", "conv_k_sh", "conv_v_sh", "conv_k", "conv_v")}
         B.mom_short_conv_bwd([
-            dict(z=b["q_raw"], dout=f(c["dq"]), da=f(c["dq"]), dz=dz[:, 0:Hd], seg_cu=cu_seqlens, w=w["conv_q"],
+            dict(z=b["q_raw"], dout=f(c["dq"]), dz=dz[:, 0:Hd], seg_cu=cu_seqlens, w=w["conv_q"],
                  dw=dconv["conv_q"], l2norm=True),
-            dict(z=b["k_sh_raw"], dout=f(c["dk_sh"]), da=f(c["dk_sh"]), dz=dz[:, Hd:2 * Hd], seg_cu=cu_seqlens,
+            dict(z=b["k_sh_raw"], dout=f(c["dk_sh"]), dz=dz[:, Hd:2 * Hd], seg_cu=cu_seqlens,
                  w=w["conv_k_sh"], dw=dconv["conv_k_sh"], l2norm=True),
-            dict(z=b["v_sh_raw"], dout=f(c["dv_sh"]), da=f(c["dv_sh"]), dz=dz[:, 2 * Hd:3 * Hd], seg_cu=cu_seqlens,
+            dict(z=b["v_sh_raw"], dout=f(c["dv_sh"]), dz=dz[:, 2 * Hd:3 * Hd], seg_cu=cu_seqlens,
                  w=w["conv_v_sh"], dw=dconv["conv_v_sh"]),
-            dict(z=b["k_p_raw"], dout=f(c["dk_p"]), da=f(c["dk_p"]), dz=dzr[:, 0:Hd], seg_cu=b["seg_cu"],
+            dict(z=b["k_p_raw"], dout=f(c["dk_p"]), dz=dzr[:, 0:Hd], seg_cu=b["seg_cu"],
                  seg_per_group=n_seq, w=w["conv_k"], dw=dconv["conv_k"], l2norm=True),
-            dict(z=b["v_p_raw"], dout=f(c["dv_p"]), da=f(c["dv_p"]), dz=dzr[:, Hd:], seg_cu=b["seg_cu"],
+            dict(z=b["v_p_raw"], dout=f(c["dv_p"]), dz=dzr[:, Hd:], seg_cu=b["seg_cu"],
                  seg_per_group=n_seq, w=w["conv_v"], dw=dconv["conv_v"]),
         ], d, ws, stream=st)
         dala = g("dala", (n_tok, H))

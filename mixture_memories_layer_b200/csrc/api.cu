@@ -929,7 +929,7 @@ mom_status mom_short_conv_bwd(const mom_conv_bwd_problem* problems, int n_proble
         if (q.l2norm && (head_dim < 8 || head_dim > 256 || (head_dim & (head_dim - 1)) != 0 || channels % head_dim))
             return MOM_ERR_ARG;
         if (q.ldz < q.col0 + channels || q.col0 < 0 || q.ldz % 4 || q.col0 % 4) return MOM_ERR_ARG;
-        const void* ptrs[] = {q.z, q.dout, q.da, q.dz, q.seg_cu, q.w, q.dw};
+        const void* ptrs[] = {q.z, q.dout, q.dz, q.seg_cu, q.w, q.dw};
         for (const void* p : ptrs)
             if (!p || !al16(p)) return MOM_ERR_ARG;
         pr[i] = ConvBwdArgs{q.z, q.dout, q.da, q.dz, q.ldz, q.col0, q.n_rows, q.seg_cu, q.n_seg, q.seg_per_group,

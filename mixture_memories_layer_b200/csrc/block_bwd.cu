@@ -9,13 +9,12 @@
 //                   n = o r, s = SiLU(g), dn = dy w_norm s:
 //                     do = r (dn - n mean(dn n)),  dg = dy n w_norm SiLU'(g),
 //                     dw_norm += dy n s  (summed over tokens and heads)
-//   conv_bwd_act  : for out = [l2norm] SiLU(a), a = conv(z): da from d out
+//   conv_bwd_fused: for out = [l2norm] SiLU(a), a = conv(z): da from d out
 //                   (a recomputed from the raw rows, the norm's adjoint per
-//                   head, then SiLU's)
-//   conv_bwd_taps : dz[t] = sum_j w[W-1-j] da[t+j] over the rows t+j of t's
-//                   segment (the convolution run backwards in time), and
-//                   dw[g][W-1-j] += da[t] z[t-j]
-// HBM-bound elementwise work, one warp per (row, 256 channels) or per
+//                   head, then SiLU's), then dz[t] = sum_j w[W-1-j] da[t+j]
+//                   over the rows t+j of t's segment (the convolution run
+//                   backwards in time) and dw[g][W-1-j] += da[t] z[t-j]
+// Streaming elementwise work, one warp per (row, 256 channels) or per
 // (32 rows, 256 channels); the filter gradients are summed per warp task in
 // registers and added atomically.
 #include "common.cuh"
@@ -137,8 +136,7 @@ norm_gate_bwd_kernel(const bf16* __restrict__ o_sh, const bf16* __restrict__ o_p
 constexpr int MAXP = 8, RANGE = 32;
 struct ConvBwdBatch {
     ConvBwdArgs pr[MAXP];
-    int64_t base_row[MAXP + 1];   // items of the row pass (one per row x 256 channels)
-    int64_t base_rng[MAXP + 1];   // items of the tap pass (one per 32 rows x 256 channels)
+    int64_t base_rng[MAXP + 1];   // work items before each problem (one per 32 rows x 256 channels)
     int n, C, d;
     void* err;
 };
@@ -153,85 +151,14 @@ __device__ __forceinline__ int seg_of(const int32_t* seg_cu, int n_seg, int64_t 
     return lo;
 }
 
+// The convolution's adjoint: a warp's 32-row range (x 256 channels)
+// recomputes da for its rows and the W-1 rows after them (a ring in
+// registers), so da never goes to memory: per element z (2 B) and d out
+// (4 B) in, dz (4 B) out.  (As a row pass writing da and a tap pass reading
+// it back, twice the bytes, the two took 1.04 ms on the 380M block's five
+// convolutions against 0.86 ms fused.)
 template <int W>
-__global__ void __launch_bounds__(256) conv_bwd_act_kernel(const __grid_constant__ ConvBwdBatch B) {
-    const int lane = threadIdx.x & 31;
-    const int nblk = (B.C + 255) / 256;
-    const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
-    int pi = 0;
-    for (int64_t it = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); it < B.base_row[B.n]; it += nw) {
-        while (it >= B.base_row[pi + 1]) ++pi;
-        const ConvBwdArgs& a = B.pr[pi];
-        const int64_t r_beg = __ldg(a.seg_cu), r_end = __ldg(a.seg_cu + a.n_seg);
-        if (r_beg < 0 || r_end < r_beg || r_end > a.n_rows) {
-            if (lane == 0 && it == B.base_row[pi]) record_error(B.err, MOM_DEVERR_SEGMENT, pi);
-            continue;
-        }
-        const int64_t local = it - B.base_row[pi];
-        const int64_t r = r_beg + local / nblk;
-        if (r >= r_end) continue;
-        const int c = (int)(local % nblk) * 256 + 8 * lane;
-        const bool on = c < B.C;
-        const int s = seg_of(a.seg_cu, a.n_seg, r);
-        const int64_t s_beg = __ldg(a.seg_cu + s);
-        const int grp = s / a.seg_per_group;
-        const bool okg = grp < a.n_groups;
-        if (!okg && lane == 0) record_error(B.err, MOM_DEVERR_SEGMENT, s);
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        if (on && okg) {
-#pragma unroll
-            for (int j = 0; j < W; ++j) {
-                if (r - j >= s_beg) {
-                    const uint4 v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(a.z) + (r - j) * B.C + c));
-                    const float* wp = a.w + ((int64_t)grp * W + (W - 1 - j)) * B.C + c;
-                    const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
-                    const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp) + 1);
-                    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[e] = fmaf(wv[e], bfv(v, e), acc[e]);
-                }
-            }
-        }
-        float cv[8], dy[8], ss = 0.f, cdy = 0.f;
-        if (on) load_vec<8>(a.dout + r * B.C + c, dy);
-        else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dy[e] = 0.f;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            cv[e] = acc[e] * sigmoidf_(acc[e]);
-            ss = fmaf(cv[e], cv[e], ss);
-            cdy = fmaf(cv[e], dy[e], cdy);
-        }
-        float dc[8];
-        if (a.l2) {                                       // uniform over the warp
-            for (int sh = B.d >> 4; sh >= 1; sh >>= 1) {
-                ss += __shfl_xor_sync(0xffffffffu, ss, sh);
-                cdy += __shfl_xor_sync(0xffffffffu, cdy, sh);
-            }
-            const float nrm = sqrtf(ss + 1e-6f);
-            // y = c / n: dc = dy / n - c (c . dy) / n^3
-            const float inv = 1.f / nrm, k3 = cdy * inv * inv * inv;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dc[e] = dy[e] * inv - cv[e] * k3;
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dc[e] = dy[e];
-        }
-        if (on) {
-            float da[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) da[e] = okg ? dc[e] * silu_grad(acc[e]) : 0.f;
-            store_vec<8>(a.da + r * B.C + c, da);
-        }
-    }
-}
-
-template <int W>
-__global__ void __launch_bounds__(256) conv_bwd_taps_kernel(const __grid_constant__ ConvBwdBatch B) {
+__global__ void __launch_bounds__(256, 2) conv_bwd_fused_kernel(const __grid_constant__ ConvBwdBatch B) {
     const int lane = threadIdx.x & 31;
     const int nblk = (B.C + 255) / 256;
     const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -240,34 +167,26 @@ __global__ void __launch_bounds__(256) conv_bwd_taps_kernel(const __grid_constan
         while (it >= B.base_rng[pi + 1]) ++pi;
         const ConvBwdArgs& a = B.pr[pi];
         const int64_t r_beg = __ldg(a.seg_cu), r_end = __ldg(a.seg_cu + a.n_seg);
-        if (r_beg < 0 || r_end < r_beg || r_end > a.n_rows) continue;   // recorded by the row pass
+        if (r_beg < 0 || r_end < r_beg || r_end > a.n_rows) {
+            if (lane == 0 && it == B.base_rng[pi]) record_error(B.err, MOM_DEVERR_SEGMENT, pi);
+            continue;
+        }
         const int64_t local = it - B.base_rng[pi];
         const int64_t ra = r_beg + (local / nblk) * RANGE;
         if (ra >= r_end) continue;
         const int64_t rb = ra + RANGE < r_end ? ra + RANGE : r_end;
         const int c = (int)(local % nblk) * 256 + 8 * lane;
         const bool on = c < B.C;
-        int s = seg_of(a.seg_cu, a.n_seg, ra);
-        int64_t s_beg = __ldg(a.seg_cu + s), s_end = __ldg(a.seg_cu + s + 1);
-        int grp = s / a.seg_per_group;
+        const bf16* z = reinterpret_cast<const bf16*>(a.z);
         float wv[W][8], dwa[W][8];
-        auto load_w = [&]() {
 #pragma unroll
-            for (int t = 0; t < W; ++t) {
-                if (on && grp < a.n_groups) {
-                    const float* wp = a.w + ((int64_t)grp * W + t) * B.C + c;
-                    const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
-                    const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp) + 1);
-                    wv[t][0] = w0.x; wv[t][1] = w0.y; wv[t][2] = w0.z; wv[t][3] = w0.w;
-                    wv[t][4] = w1.x; wv[t][5] = w1.y; wv[t][6] = w1.z; wv[t][7] = w1.w;
-                } else {
+        for (int t = 0; t < W; ++t)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) wv[t][e] = 0.f;
-                }
-            }
-        };
+            for (int e = 0; e < 8; ++e) dwa[t][e] = 0.f;
+        int grp = -1;
+        bool okg = false;
         auto flush = [&]() {
-            if (on && grp < a.n_groups) {
+            if (on && okg) {
 #pragma unroll
                 for (int t = 0; t < W; ++t)
 #pragma unroll
@@ -279,52 +198,98 @@ __global__ void __launch_bounds__(256) conv_bwd_taps_kernel(const __grid_constan
 #pragma unroll
                 for (int e = 0; e < 8; ++e) dwa[t][e] = 0.f;
         };
-        load_w();
+        // da of row r of the segment [s_beg, s_end) (0 past its end); warp-uniform r
+        auto da_row = [&](int64_t r, int64_t s_beg, int64_t s_end, float (&out)[8]) {
+            const bool in = r < s_end;
+            float acc[8], dy[8];
 #pragma unroll
-        for (int t = 0; t < W; ++t)
+            for (int e = 0; e < 8; ++e) { acc[e] = 0.f; dy[e] = 0.f; }
+            if (in && on) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dwa[t][e] = 0.f;
-        for (int64_t r = ra; r < rb; ++r) {
-            if (r >= s_end) {                             // the next (non-empty) segment starts here
-                while (s + 1 < a.n_seg && r >= __ldg(a.seg_cu + s + 1)) ++s;
-                s_beg = __ldg(a.seg_cu + s);
-                s_end = __ldg(a.seg_cu + s + 1);
-                const int g2 = s / a.seg_per_group;
-                if (g2 != grp) {
-                    flush();
-                    grp = g2;
-                    load_w();
-                }
-            }
-            if (!on) continue;
-            float dz[8], dar[8];
+                for (int j = 0; j < W; ++j) {
+                    if (r - j >= s_beg) {
+                        const uint4 v = __ldg(reinterpret_cast<const uint4*>(z + (r - j) * B.C + c));
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dz[e] = 0.f;
-            load_vec<8>(a.da + r * B.C + c, dar);
-#pragma unroll
-            for (int j = 0; j < W; ++j) {
-                // output row r + j takes raw row r through tap W-1-j
-                if (r + j < s_end) {
-                    float dn[8];
-                    if (j == 0) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) dn[e] = dar[e];
-                    } else {
-                        load_vec<8>(a.da + (r + j) * B.C + c, dn);
+                        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wv[W - 1 - j][e], bfv(v, e), acc[e]);
                     }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) dz[e] = fmaf(wv[W - 1 - j][e], dn[e], dz[e]);
                 }
-                // this output row r took raw row r - j through tap W-1-j
-                if (r - j >= s_beg) {
-                    const uint4 v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(a.z) + (r - j) * B.C + c));
+                load_vec<8>(a.dout + r * B.C + c, dy);
+            }
+            float cv[8], ss = 0.f, cdy = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) dwa[W - 1 - j][e] = fmaf(dar[e], bfv(v, e), dwa[W - 1 - j][e]);
+            for (int e = 0; e < 8; ++e) {
+                cv[e] = acc[e] * sigmoidf_(acc[e]);
+                ss = fmaf(cv[e], cv[e], ss);
+                cdy = fmaf(cv[e], dy[e], cdy);
+            }
+            if (a.l2) {                                   // uniform over the warp
+                for (int sh = B.d >> 4; sh >= 1; sh >>= 1) {
+                    ss += __shfl_xor_sync(0xffffffffu, ss, sh);
+                    cdy += __shfl_xor_sync(0xffffffffu, cdy, sh);
+                }
+                const float inv = 1.f / sqrtf(ss + 1e-6f), k3 = cdy * inv * inv * inv;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) out[e] = (in && okg) ? (dy[e] * inv - cv[e] * k3) * silu_grad(acc[e]) : 0.f;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) out[e] = (in && okg) ? dy[e] * silu_grad(acc[e]) : 0.f;
+            }
+        };
+        int64_t t = ra;
+        while (t < rb) {
+            const int s = seg_of(a.seg_cu, a.n_seg, t);
+            const int64_t s_beg = __ldg(a.seg_cu + s), s_end = __ldg(a.seg_cu + s + 1);
+            const int g2 = s / a.seg_per_group;
+            if (g2 != grp) {
+                flush();
+                grp = g2;
+                okg = grp < a.n_groups;
+                if (!okg && lane == 0) record_error(B.err, MOM_DEVERR_SEGMENT, s);
+#pragma unroll
+                for (int tp = 0; tp < W; ++tp) {
+                    if (on && okg) {
+                        const float* wp = a.w + ((int64_t)grp * W + tp) * B.C + c;
+                        const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
+                        const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp) + 1);
+                        wv[tp][0] = w0.x; wv[tp][1] = w0.y; wv[tp][2] = w0.z; wv[tp][3] = w0.w;
+                        wv[tp][4] = w1.x; wv[tp][5] = w1.y; wv[tp][6] = w1.z; wv[tp][7] = w1.w;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) wv[tp][e] = 0.f;
+                    }
                 }
             }
-            float* dst = a.dz + r * a.ldz + a.col0 + c;
+            const int64_t t_stop = rb < s_end ? rb : s_end;
+            float ring[W][8];                             // da of rows t .. t+W-1
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dst[e] = dz[e];
+            for (int j = 0; j + 1 < W; ++j) da_row(t + j, s_beg, s_end, ring[j]);
+            for (; t < t_stop; ++t) {
+                da_row(t + W - 1, s_beg, s_end, ring[W - 1]);
+                if (on) {
+                    float dz[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dz[e] = 0.f;
+#pragma unroll
+                    for (int j = 0; j < W; ++j)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dz[e] = fmaf(wv[W - 1 - j][e], ring[j][e], dz[e]);
+#pragma unroll
+                    for (int j = 0; j < W; ++j) {
+                        if (t - j >= s_beg) {
+                            const uint4 v = __ldg(reinterpret_cast<const uint4*>(z + (t - j) * B.C + c));
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) dwa[W - 1 - j][e] = fmaf(ring[0][e], bfv(v, e), dwa[W - 1 - j][e]);
+                        }
+                    }
+                    float* dst = a.dz + t * a.ldz + a.col0 + c;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dst[e] = dz[e];
+                }
+#pragma unroll
+                for (int j = 0; j + 1 < W; ++j)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ring[j][e] = ring[j + 1][e];
+            }
         }
         flush();
     }
@@ -370,32 +335,27 @@ cudaError_t launch_conv_bwd(const ConvBwdArgs* problems, int n, int C, int W, in
     b.d = d;
     b.err = err;
     const int nblk = (C + 255) / 256;
-    b.base_row[0] = b.base_rng[0] = 0;
+    b.base_rng[0] = 0;
     for (int i = 0; i < n; ++i) {
         const ConvBwdArgs& q = problems[i];
         b.pr[i] = q;
-        b.base_row[i + 1] = b.base_row[i] + q.n_rows * nblk;
         b.base_rng[i + 1] = b.base_rng[i] + cdiv(q.n_rows, RANGE) * nblk;
         cudaError_t e = cudaMemsetAsync(q.dw, 0, (size_t)q.n_groups * W * C * 4, st);
         if (e != cudaSuccess) return e;
     }
-    if (b.base_row[n] == 0) return cudaSuccess;
+    if (b.base_rng[n] == 0) return cudaSuccess;
     auto grid_of = [](int64_t items) {
         int64_t g = cdiv(items, 8);
         return (unsigned)(g > 148 * 16 ? 148 * 16 : g < 1 ? 1 : g);
     };
     switch (W) {
-        case 1: conv_bwd_act_kernel<1><<<grid_of(b.base_row[n]), 256, 0, st>>>(b);
-                conv_bwd_taps_kernel<1><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
-        case 2: conv_bwd_act_kernel<2><<<grid_of(b.base_row[n]), 256, 0, st>>>(b);
-                conv_bwd_taps_kernel<2><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
-        case 3: conv_bwd_act_kernel<3><<<grid_of(b.base_row[n]), 256, 0, st>>>(b);
-                conv_bwd_taps_kernel<3><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
-        case 4: conv_bwd_act_kernel<4><<<grid_of(b.base_row[n]), 256, 0, st>>>(b);
-                conv_bwd_taps_kernel<4><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
+        case 1: conv_bwd_fused_kernel<1><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
+        case 2: conv_bwd_fused_kernel<2><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
+        case 3: conv_bwd_fused_kernel<3><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
+        case 4: conv_bwd_fused_kernel<4><<<grid_of(b.base_rng[n]), 256, 0, st>>>(b); break;
         default: return cudaErrorInvalidValue;
     }
-    count_launches(2);
+    count_launches(1);
     return cudaGetLastError();
 }
 

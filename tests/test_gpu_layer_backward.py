@@ -25,7 +25,7 @@ def _need_cuda():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
 
 
-def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True, mem_gates=False):
+def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True, mem_gates=False, rule="gated_delta"):
     from mixture_memories_layer_b200 import layer as L
     w = synth.Workload("bwd", 0, 0, D, H, d, M, K, dtype, seed=seed, mem_gates=mem_gates)
     rng = np.random.default_rng(seed)
@@ -33,7 +33,7 @@ def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True, mem_ga
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     x = synth.make_tokens(w, rng, int(cu[-1]))
     dt = torch.bfloat16 if dtype == "bf16" else torch.float32
-    lay = L.MoMLayer(L.pack_weights(p, dt), H, d, K)
+    lay = L.MoMLayer(L.pack_weights(p, dt), H, d, K, rule=rule)
     xt = torch.as_tensor(x).to("cuda", dt)
     cut = torch.as_tensor(cu).cuda()
     b = lay.forward(xt, cut)
@@ -47,7 +47,7 @@ def _run(dtype, d, lens, M=4, K=2, H=2, D=256, seed=81, with_states=True, mem_ga
     assert lay.device_errors() == {}
     got = {k: v.cpu().numpy().astype(np.float64) for k, v in g.items()}
     idx = b["idx"].cpu().numpy()
-    ref = obwd.mom_backward(x, p, cu, K, H, d, dout, forced_idx=idx, dh_shared=dh_sh, dh_mem=dh_m)
+    ref = obwd.mom_backward(x, p, cu, K, H, d, dout, forced_idx=idx, dh_shared=dh_sh, dh_mem=dh_m, rule=rule)
     Hd = H * d
     pairs = {
         "dx": (got["dx"], ref["dx"]), "dw_r": (got["dw_r"], ref["dw_r"]), "db_r": (got["db_r"], ref["db_r"]),
@@ -143,5 +143,13 @@ def test_layer_backward_per_memory_gates(dtype, tol):
     the rows' gates, their adjoints through mom_gates_bwd_by_group into the
     memories' gate weights, A_mem and b_a_mem."""
     errs = _run(dtype, 64, (120, 0, 77), M=4, K=2, seed=84, mem_gates=True)
+    bad = {k: e for k, e in errs.items() if not e < tol}
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("dtype,tol", [("f32", 1e-5), ("bf16", 2e-2)])
+def test_layer_backward_scalar_gated_linear_rule(dtype, tol):
+    """The layer backward with the scalar-gated linear memories (MOM_RULE_GATED_LINEAR)."""
+    errs = _run(dtype, 64, (100, 3, 60), seed=85, rule="gated_linear")
     bad = {k: e for k, e in errs.items() if not e < tol}
     assert not bad, (bad, errs)
