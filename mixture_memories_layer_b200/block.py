@@ -202,7 +202,8 @@ class MoMBlock(MoMLayer):
         dw_o = g("dw_o", (D, Hd))
         one = self._buf("one_group", (2,), torch.int32)
         if getattr(self, "_one_n", None) != n_tok:
-            one.copy_(torch.tensor([0, n_tok], dtype=torch.int32))
+            with torch.cuda.stream(st):                      # ordered before the GEMMs that read it
+                one.copy_(torch.tensor([0, n_tok], dtype=torch.int32))
             self._one_n = n_tok
         B.mom_gemm_grouped(1, dy32, b["o_tilde"].view(n_tok, Hd), dw_o, D, Hd, 0, one, None, 1, ws, stream=st)
         # o~ = rmsnorm(o) w_norm SiLU(g): do (bf16), dg into the pre-activation

@@ -391,7 +391,8 @@ class MoMLayer:
         w, g = self.w, self._bwd_buf
         one = self._buf("one_group", (2,), torch.int32)     # one group of all n_tok rows
         if getattr(self, "_one_n", None) != n_tok:
-            one.copy_(torch.tensor([0, n_tok], dtype=torch.int32))
+            with torch.cuda.stream(st):                      # ordered before the GEMMs that read it
+                one.copy_(torch.tensor([0, n_tok], dtype=torch.int32))
             self._one_n = n_tok
         # the weight gradients on the side stream beside the input gradient
         # (both only read dz, dzr, dlogits, dala): their last waves fill each
