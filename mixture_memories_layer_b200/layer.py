@@ -273,7 +273,7 @@ class MoMLayer:
         qn, kshn, kpn = g("qn", (n_tok, H)), g("kshn", (n_tok, H)), g("kpn", (R, H))
         B.mom_proj_shared(x, w["w_shared"], H, d, g("q2", (n_tok, H, d), dt), g("k2", (n_tok, H, d), dt),
                           g("v2", (n_tok, H, d), dt), ws, stream=st, q_norm=qn, k_sh_norm=kshn)
-        B.mom_kv_proj_groups(x, b["perm"], b["mem_offset"], self._mem_groups(), w["w_kv"], H, d,
+        B.mom_kv_proj_groups(x, b["perm"], b["mem_offset"], self._mem_groups(st), w["w_kv"], H, d,
                              g("kp2", (R, H, d), dt), g("vp2", (R, H, d), dt), ws, stream=st, k_norm=kpn)
         c = self._core_bwd(b, cu_seqlens, dout, dh_shared, dh_mem, h0_shared, h0_mem, st, ws)
         # pre-activation gradients: shared [N, 3Hd + 2H] (q | k_sh | v_sh | beta | a), routed [N*K, 2Hd] (k | v)
@@ -311,11 +311,13 @@ class MoMLayer:
     def _bwd_buf(self, name, shape, dtype=torch.float32):
         return self._buf("bwd_" + name, shape, dtype)
 
-    def _mem_groups(self):
-        """[0, 1, .., M-1] int32 on the device: group g of the routed rows is memory g."""
+    def _mem_groups(self, st):
+        """[0, 1, .., M-1] int32 on the device (made on the launching stream
+        st): group g of the routed rows is memory g."""
         mem_index = getattr(self, "_mem_index", None)
         if mem_index is None:
-            mem_index = self._mem_index = torch.arange(self.n_mem, dtype=torch.int32, device=self.device)
+            with torch.cuda.stream(st):
+                mem_index = self._mem_index = torch.arange(self.n_mem, dtype=torch.int32, device=self.device)
         return mem_index
 
     def _core_bwd(self, b, cu_seqlens, dout, dh_shared, dh_mem, h0_shared, h0_mem, st, ws):
