@@ -153,3 +153,30 @@ def test_layer_backward_scalar_gated_linear_rule(dtype, tol):
     errs = _run(dtype, 64, (100, 3, 60), seed=85, rule="gated_linear")
     bad = {k: e for k, e in errs.items() if not e < tol}
     assert not bad, (bad, errs)
+
+
+def test_layer_backward_on_a_caller_stream():
+    """Forward and backward launched on the caller's own stream (not torch's
+    current one) give the gradients of the default-stream run: every table
+    the calls read is made on the launching stream."""
+    from mixture_memories_layer_b200 import layer as L
+    w = synth.Workload("bwd", 0, 0, 256, 2, 64, 4, 2, "bf16", seed=86)
+    rng = np.random.default_rng(86)
+    p = synth.make_weights(w, rng)
+    cu = torch.as_tensor(np.array([0, 90, 91, 200], np.int32)).cuda()
+    x = torch.as_tensor(synth.make_tokens(w, rng, 200)).to("cuda", torch.bfloat16)
+    dout = torch.as_tensor(rng.standard_normal((200, 2, 64)).astype(np.float32)).to("cuda", torch.bfloat16)
+    grads = []
+    for use_stream in (False, True):
+        lay = L.MoMLayer(L.pack_weights(p, torch.bfloat16), 2, 64, 2)      # fresh tables each time
+        s = torch.cuda.Stream() if use_stream else None
+        if s is not None:
+            s.wait_stream(torch.cuda.current_stream())
+        lay.forward(x, cu, stream=s)
+        g = lay.backward(x, cu, dout, stream=s)
+        torch.cuda.synchronize()
+        assert lay.device_errors() == {}
+        grads.append({k: v.clone() for k, v in g.items()})
+    for k in grads[0]:
+        e = max_abs_rel(grads[1][k].cpu().numpy(), grads[0][k].cpu().numpy())
+        assert e < 1e-5, (k, e)
