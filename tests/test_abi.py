@@ -158,3 +158,30 @@ def test_block_backward_calls_validate_on_the_host(lib):
     assert L.mom_convert(fake, B.MOM_F32, fake, B.MOM_BF16, -1, None) == B.MOM_ERR_ARG
     assert L.mom_convert(fake, B.MOM_F32, fake, B.MOM_BF16, 0, None) == B.MOM_OK  # nothing to do
     assert L.mom_convert(None, B.MOM_F32, fake, B.MOM_BF16, 5, None) == B.MOM_ERR_ARG
+
+
+def test_grouped_gate_calls_validate_on_the_host(lib):
+    """The per-memory gates' grouped calls (backward and memory-parallel
+    owner) refuse bad shapes and pointers before any launch."""
+    L, B = lib.lib, lib
+    fake = ctypes.c_void_p(0x10000)
+    gb = lambda n_groups=2, ldz=4, col_b=0, col_a=2, A=fake: L.mom_gates_bwd_by_group(
+        fake, fake, fake, fake, A, fake, n_groups, 10, 2, fake, ldz, col_b, col_a, fake, None)
+    assert gb(n_groups=0) == B.MOM_ERR_ARG
+    assert gb(ldz=3) == B.MOM_ERR_ARG                                         # col_a + H > ldz
+    assert gb(col_b=-1) == B.MOM_ERR_ARG
+    assert gb(A=None) == B.MOM_ERR_ARG
+    cs = lambda n_groups=2, lda=4, cols=2, goff=fake: L.mom_col_sums_grouped(fake, 10, lda, cols, goff, n_groups,
+                                                                             fake, None)
+    assert cs(n_groups=0) == B.MOM_ERR_ARG
+    assert cs(lda=1) == B.MOM_ERR_ARG                                         # lda < cols
+    assert cs(goff=None) == B.MOM_ERR_ARG
+    assert cs(cols=0) == B.MOM_OK                                             # nothing to sum
+    mg = lambda n_x=10, perm=None, n_groups=2, d_model=64, ws_bytes=4096: L.mom_mem_gate_proj_groups(
+        fake, n_x, perm, 10, fake, fake, n_groups, fake, fake, fake, 4, B.MOM_BF16, d_model, 2, fake, fake, fake,
+        ws_bytes, None)
+    assert mg(n_groups=33) == B.MOM_ERR_ARG                                   # more groups than MOM_MAX_MEM
+    assert mg(n_groups=0) == B.MOM_ERR_ARG
+    assert mg(d_model=60) == B.MOM_ERR_ARG                                    # d_model % 8
+    assert mg(n_x=5) == B.MOM_ERR_ARG                                         # row r reads x row r: n_x < n_rows
+    assert mg(ws_bytes=8) == B.MOM_ERR_ARG
