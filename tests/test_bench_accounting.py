@@ -123,3 +123,17 @@ def test_380m_block_roofline():
     assert _close(flops, 388.1e9, 1e-3)
     assert _close(bytes_, 136.8e6, 2e-3)
     assert _close(t, 388.1e9 / 1631.7e12, 1e-3)        # tensor-bound
+
+
+def test_backward_roofline_is_twice_the_forward_at_the_bf16_peak():
+    """The backward's estimate: 2 x the forward's FLOPs (an input and a
+    weight gradient per product) against the bf16 peak; for the 380M layer
+    636.6 GFLOP, 0.390 ms at 1631.7 TFLOP/s, so 32 ms is 1.2 %."""
+    w = synth.WORKLOADS["mom380m"]
+    lf = bench.layer_roofline(w, PEAKS)[0]
+    r = bench.backward_roofline(lf, PEAKS, 32.0)
+    assert r["flops"] == 2 * lf
+    assert _close(r["flops"], 636.6e9, 1e-3)
+    assert _close(r["roofline_ms"], 636.6e9 / 1631.7e12 * 1e3, 1e-3)
+    assert _close(r["frac"], r["roofline_ms"] / 32.0)
+    assert 0.011 < r["frac"] < 0.013
