@@ -324,9 +324,11 @@ class MoMLayer:
         """The reverse pass from the adjoint of the combined output (dout [N, H,
         d], the model dtype) to the recurrences' inputs: the combine's and the
         router's adjoints, both recurrences' reverse passes, and each token's
-        routed rows summed into its own.  Returns float32 dq, dk_sh, dv_sh
-        [N, H, d], dk_p, dv_p [N*K, H, d], dbeta, dla [N, H], dlogits [N, M],
-        dh0_shared, dh0_mem."""
+        routed rows summed into its own (with per-memory gates the routed rows'
+        beta and alpha adjoints stay per row: dbeta, dla are then the shared
+        memory's).  Returns float32 dq, dk_sh, dv_sh [N, H, d], dk_p, dv_p
+        [N*K, H, d], dbeta, dla [N, H], dlogits [N, M], dh0_shared, dh0_mem,
+        and the routed rows' db_p, dla_p [N*K, H]."""
         n_tok, n_seq = b["idx"].shape[0], cu_seqlens.numel() - 1
         H, d, K, M = self.H, self.d, self.top_k, self.n_mem
         Hd, R = H * d, n_tok * K
