@@ -194,3 +194,23 @@ def test_gdn_recurrence_bwd_rules_differ_and_linear_rule_planted_mistake_fails()
 
     # the delta rule's adjoints are the linear rule's with the delta terms kept: they must fail here
     assert _rel(gd["dk"], _fd(loss, c["k"])) > 1e-3
+
+
+def test_per_memory_gate_pin_catches_the_shared_gates_mistake():
+    """The pin above fails a backward that runs the routed rows' reverse pass
+    on the shared gates (the per-memory gates dropped): planted by handing
+    the backward the weights without the memories' own gates."""
+    w, p, cu, x, adj, h0s, h0m = _layer_case(seed=4, mem_gates=True)
+    H, d, K = w.heads, w.d_head, w.top_k
+    idx = fwd.router_topk(x, p["w_r"], p["b_r"], K)[0]
+
+    def loss():
+        f = fwd.mom_forward(x, p, cu, K, H, d, 1.0, forced_idx=idx, h0_shared=h0s, h0_mem=h0m)
+        return float(np.sum(adj["dout"] * f["out"]) + np.sum(adj["dhs"] * f["h_shared"])
+                     + np.sum(adj["dhm"] * f["h_mem"]))
+
+    p_wrong = {k: v for k, v in p.items() if not k.endswith("_mem")}
+    g = bwd.mom_backward(x, p_wrong, cu, K, H, d, adj["dout"], 1.0, forced_idx=idx, h0_shared=h0s, h0_mem=h0m,
+                         dh_shared=adj["dhs"], dh_mem=adj["dhm"])
+    assert _rel(g["dx"], _fd(loss, x)) > 1e-3
+    assert _rel(g["dw_k"], _fd(loss, p["w_k"])) > 1e-3
