@@ -222,7 +222,7 @@ def _block_refs(w, p, res, seqs, rule="gated_delta"):
 
 
 def _check_block(w, p, res, seqs=None, rule="gated_delta"):
-    """Whole-tensor errors (the benchmark spec's measure: max-abs-rel per output
+    """Whole-tensor errors (the acceptance measure: max-abs-rel per output
     tensor) over the chosen sequences."""
     tol = TOL["bf16"]
     seqs = range(len(p["cu_seqlens"]) - 1) if seqs is None else seqs
